@@ -1,0 +1,365 @@
+"""Throughput of the DeepSeekMoE layer step on B200s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config v3_bf16] [--impl ours|reference]
+
+A step is one pass of the whole layer over one batch of synthetic tokens:
+route, permute, routed and shared SwiGLU expert FFNs, combine with the
+residual, and the per-step bias update (for N > 1 after an all-reduce of the
+per-expert load).  Inputs are resident in HBM before the timed region; the
+22.6 GB of V3-shaped expert weights stream through HBM every step (far larger
+than the 126 MB L2), so no flush is needed between steps.  Timing is CUDA
+events on the launching stream, bracketed by a barrier and a device
+synchronize, max over ranks.  Rank 0 prints one JSON line.
+
+--impl reference times the CPU oracle (oracle/) on the host cores over a
+bounded token sample per step; it is the only other use of oracle/ here.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+import torch.distributed as dist
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mixture_experts_layer_60_b200.configs import CONFIGS  # noqa: E402
+
+METRIC = "MoE-layer tokens/sec on 1 B200 + % of roofline (TFLOP/s, HBM GB/s)"
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm_gbs": j["hbm_gbs"], "bf16": j["bf16_tflops"],
+                "bf16_sustained": j.get("bf16_tflops_sustained", j["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.path = tempfile.mktemp(suffix=".csv")
+        self.proc = None
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", uuid, f"--query-gpu={self.FIELDS}", "--format=csv,noheader",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        self.proc.wait()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                sm.append(float(parts[2].split()[0]))
+                mx.append(float(parts[3].split()[0]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[6:10]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- helpers
+
+def dist_setup(n_gpus):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return ws, rank, local
+
+
+def gpu_launches_per_step(cfg):
+    # route: logits GEMM + top-K; permute: 4; routed FFN: 2; shared FFN: 2 each;
+    # combine: 1; bias update: 1; FP8: + activation quantiser
+    n = 2 + 4 + 2 + 2 * cfg.N_s + 1 + 1
+    if cfg.dtype == "e4m3":
+        n += 1
+    if cfg.dtype == "f32" or cfg.N_r % 64:
+        pass
+    return n
+
+
+def roofline_layer(cfg, p):
+    flops = cfg.flops()
+    tensor_peak = p["bf16"] * (2 if cfg.dtype == "e4m3" else 1) * 1e12
+    bytes_ = cfg.weight_bytes() + cfg.N_r * cfg.d * 2 + 2 * cfg.T * cfg.d * 2
+    t = max(flops / tensor_peak, bytes_ / (p["hbm_gbs"] * 1e9))
+    return cfg.T / t, flops, bytes_
+
+
+def cpu_oracle_sample(cfg, w, n_tokens, seed=0):
+    """Times the CPU oracle on the full route of `n_tokens` tokens and their
+    whole layer (expert-major, weights read from the device expert by expert)."""
+    import numpy as np
+    from oracle import moe_oracle as O
+
+    class Lazy:
+        def __init__(self, gu, dn):
+            self.gu, self.dn, self.I = gu, dn, gu.shape[1] // 2
+
+        def __len__(self):
+            return self.gu.shape[0]
+
+        def __getitem__(self, e):
+            gu = self.gu[e].to("cpu", torch.float64).numpy()
+            return gu[:self.I], gu[self.I:], self.dn[e].to("cpu", torch.float64).numpy()
+
+    rows = np.sort(np.random.default_rng(seed).choice(w["u"].shape[0], n_tokens, replace=False))
+    u = w["u"][torch.from_numpy(rows).to(w["u"].device)].to("cpu", torch.float64).numpy()
+    E = w["E"].to("cpu", torch.float64).numpy()
+    b = w["b"].cpu().numpy()
+    t0 = time.perf_counter()
+    r = O.route(u, E, b, cfg.K)
+    routed, shared = Lazy(w["W_gate_up"], w["W_down"]), Lazy(w["Ws_gate_up"], w["Ws_down"])
+    if cfg.dtype == "e4m3":
+        class Q:
+            def __init__(self, ex):
+                self.ex = ex
+
+            def __len__(self):
+                return len(self.ex)
+
+            def __getitem__(self, e):
+                g, u_, d_ = self.ex[e]
+                return O.quantise_expert(g.astype(np.float32), u_.astype(np.float32),
+                                         d_.astype(np.float32))
+        O.layer_forward_fp8(u, r["idx"], r["gate"], Q(routed), Q(shared))
+    else:
+        O.layer_forward(u, r["idx"], r["gate"], routed, shared)
+    return time.perf_counter() - t0
+
+
+def cpu_cores():
+    try:
+        import numpy as np  # noqa: F401
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------------- arms
+
+def run_reference(args, cfg, ws, rank):
+    if ws > 1 and rank != 0:
+        return
+    from mixture_experts_layer_60_b200.synth import make_layer_inputs
+    torch.cuda.set_device(0)
+    w = make_layer_inputs(cfg, "cuda")
+    n_tok = args.ref_tokens
+    for _ in range(args.warmup):
+        cpu_oracle_sample(cfg, w, n_tok, seed=1)
+    times = [cpu_oracle_sample(cfg, w, n_tok, seed=2 + i) for i in range(args.steps)]
+    tot = sum(times)
+    value = n_tok * args.steps / tot
+    cores = cpu_cores()
+    sample = (f"{n_tok} tokens per step drawn from the {cfg.T}-token batch: full route and "
+              f"whole layer (every selected and shared expert) in float64 on the host")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": tot / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "N_r": cfg.N_r, "K": cfg.K,
+                       "N_s": cfg.N_s, "I": cfg.I, "tokens_per_step": n_tok},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, cfg, ws, rank, local):
+    from mixture_experts_layer_60_b200 import moe_device_status
+    from mixture_experts_layer_60_b200.layer import MoELayer
+    from mixture_experts_layer_60_b200.synth import make_layer_inputs
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    p = peaks()
+    w = make_layer_inputs(cfg, dev)
+    layer = MoELayer(cfg, w, device=dev)
+    u = w["u"]
+    stream = torch.cuda.current_stream(dev)
+    group = dist.group.WORLD if ws > 1 else None
+    T_total = cfg.T * ws
+
+    def step(ev=None, u_in=u):
+        h = layer.forward(u_in, gate_up_events=ev)
+        if group is not None:
+            from mixture_experts_layer_60_b200.parallel_load import allreduce_load
+            counts, tt = allreduce_load(layer.counts, cfg.T, group, T_total=T_total)
+            layer.bias_update(counts, tt)
+        else:
+            layer.bias_update()
+        return h
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if moe_device_status() != 0:
+        raise RuntimeError("a kernel reported a bounded-wait timeout during warm-up")
+
+    # ---- device-resident timed region
+    gu_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    if group is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for i in range(args.steps):
+        step(gu_ev[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if group is not None:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = t0.elapsed_time(t1)
+    gu_ms = sum(a.elapsed_time(b) for a, b in gu_ev) / args.steps
+    if group is not None:
+        tt = torch.tensor([ms, gu_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms, gu_ms = float(tt[0]), float(tt[1])
+    ms_step = ms / args.steps
+    value = cfg.T * ws / (ms_step / 1e3)
+
+    # ---- end to end through the API with host buffers
+    u_host = u.to("cpu").pin_memory()
+    h_host = torch.empty(cfg.T, cfg.d, dtype=u.dtype).pin_memory()
+    u_dev = torch.empty_like(u)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(3, args.steps // 4)
+    for _ in range(2):
+        u_dev.copy_(u_host, non_blocking=True)
+        h_host.copy_(step(u_in=u_dev), non_blocking=True)
+    if group is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        u_dev.copy_(u_host, non_blocking=True)
+        h_host.copy_(step(u_in=u_dev), non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if group is not None:
+        tt = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt[0])
+    status = moe_device_status()
+
+    # ---- CPU oracle baseline (rank 0, N = 1 only)
+    cpu = None
+    if ws == 1 and not args.no_cpu_baseline:
+        n_tok = args.cpu_tokens
+        secs = cpu_oracle_sample(cfg, w, n_tok)
+        cpu = {"value": n_tok / secs, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
+               "sample": f"{n_tok} tokens of the {cfg.T}-token batch, full route + whole layer "
+                         f"in float64 ({secs:.1f} s)"}
+
+    if rank != 0:
+        return
+    roof_tps, flops, bytes_ = roofline_layer(cfg, p)
+    # dominant kernel: the routed gate/up grouped GEMM
+    gu_flops = 2.0 * cfg.T * cfg.K * cfg.d * 2 * cfg.I
+    timed_s = ms / 1e3
+    sustained = timed_s >= 1.0
+    pk = p["bf16_sustained"] if sustained else p["bf16"]
+    if cfg.dtype == "e4m3":
+        pk *= 2
+    achieved = gu_flops / (gu_ms / 1e3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": {"f32": "f32", "bf16": "bf16", "e4m3": "e4m3"}[cfg.dtype],
+        "data": "synthetic (seeded, random-init weights of the named shape)",
+        "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "N_r": cfg.N_r, "K": cfg.K,
+                   "N_s": cfg.N_s, "I": cfg.I, "tokens_per_rank": cfg.T,
+                   "parallelism": f"dp{ws} (replicas; per-expert load all-reduced)" if ws > 1
+                   else "single GPU",
+                   "l2": "inputs larger than L2: all expert weights (%.1f GB) stream from HBM "
+                         "every step" % (cfg.weight_bytes() / 1e9)},
+        "roofline": {"bound": "tensor", "kernel": "routed gate/up grouped GEMM (tcgen05, fused SwiGLU)",
+                     "achieved": achieved, "peak": pk, "unit": "TFLOP/s", "frac": achieved / pk,
+                     "peak_kind": ("sustained" if sustained else "burst") + " bf16 of " +
+                                  p["source"] + (" x2 (FP8 nominal ratio)" if cfg.dtype == "e4m3" else ""),
+                     "kernel_ms": gu_ms, "flops_per_launch": gu_flops, "traffic": None},
+        "layer_roofline": {"tokens_per_s": roof_tps, "frac": value / ws / roof_tps,
+                           "flops_per_step": flops, "bytes_per_step": bytes_},
+        "clocks": clk,
+        "e2e": {"value": cfg.T * ws / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": u.numel() * u.element_size(),
+                "d2h_bytes_per_step": u.numel() * u.element_size()},
+        "gpu_launches": gpu_launches_per_step(cfg) * args.steps,
+        "device_status": status,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=60)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="v3_bf16", choices=sorted(CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-tokens", type=int, default=16)
+    ap.add_argument("--ref-tokens", type=int, default=4)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    cfg = CONFIGS[args.config]
+    ws, rank, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            run_reference(args, cfg, ws, rank)
+        else:
+            run_ours(args, cfg, ws, rank, local)
+    finally:
+        if ws > 1 and dist.is_initialized():
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

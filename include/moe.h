@@ -1,0 +1,214 @@
+/*
+ * moe.h - C ABI of the B200 DeepSeekMoE layer library (libmoe.so).
+ *
+ * The layer is the one defined in "DeepSeek-V3 技術報告" (xyznot.com summary
+ * of arXiv 2412.19437), section 方法 / 2 "具備無輔助損失平衡機制的 DeepSeekMoE":
+ *
+ *   s_{i,t} = Sigmoid(u_t^T e_i)                               (affinity)
+ *   g'_{i,t} = s_{i,t} if s_{i,t} + b_i in Topk({s_{j,t} + b_j}, K), else 0
+ *   g_{i,t}  = g'_{i,t} / sum_j g'_{j,t}                        (normalised)
+ *   h'_t = u_t + sum_{j<N_s} FFN^(s)_j(u_t) + sum_i g_{i,t} FFN^(r)_i(u_t)
+ *   b_i <- b_i - gamma if expert i is overloaded, + gamma if underloaded
+ *
+ * with FFN(x) = W_down (SiLU(W_gate x) * (W_up x)), and, optionally, the FP8
+ * recipe of the same page's section 核心概念 (E4M3, 1x128 activation tiles,
+ * 128x128 weight blocks, FP32 promotion every 128 K-elements).
+ *
+ * Conventions shared by every call
+ *   - Pointers named as device buffers are CUDA device pointers on the current
+ *     device; the caller owns every buffer.  Scratch space, where a call needs
+ *     any, is the caller's `workspace`, sized by the matching *_workspace_size().
+ *   - Arrays are row-major and contiguous.  bf16 is IEEE bfloat16, e4m3 is the
+ *     OCP FP8 E4M3 ("fn") byte format.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call
+ *     only enqueues work on it and returns; none synchronises the host, except
+ *     moe_device_status().
+ *   - Arguments are checked before anything is launched; a bad argument
+ *     returns a status and launches nothing.  No call aborts, traps or prints.
+ *     moe_last_error() describes the last failure on the calling thread.
+ *   - Kernels run on sm_100a (B200) only; other devices get MOE_ERR_UNSUPPORTED.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum moe_status {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,   /* null pointer, non-positive or inconsistent size */
+  MOE_ERR_UNSUPPORTED = 2,   /* dtype/shape combination or device not supported */
+  MOE_ERR_WORKSPACE = 3,     /* workspace smaller than *_workspace_size() */
+  MOE_ERR_CUDA = 4,          /* a CUDA runtime call or a launch failed */
+  MOE_ERR_TIMEOUT = 5        /* a kernel gave up a bounded wait (see moe_device_status) */
+} moe_status;
+
+typedef enum moe_dtype {
+  MOE_F32 = 0,
+  MOE_BF16 = 1,
+  MOE_E4M3 = 2
+} moe_dtype;
+
+/* Version of this ABI (increments on any signature change). */
+int moe_abi_version(void);
+
+/* Text of the last error on the calling thread ("" if none).  Static storage
+ * owned by the library; valid until the next failing call on this thread. */
+const char* moe_last_error(void);
+
+/* Name of a status code. */
+const char* moe_status_string(moe_status status);
+
+/* ------------------------------------------------------------------------
+ * moe_route - affinity, biased top-K, gate normalisation and load histogram
+ * (affinity line and g'-equation of section 2).
+ *
+ *   u        [T, d]    device, dt (MOE_F32 or MOE_BF16): token states u_t
+ *   E        [N_r, d]  device, dt: expert centroids e_i
+ *   b        [N_r]     device, float32: routing bias (steers selection only)
+ *   topk_idx [T, K]    device, int32 out: selected experts, largest s+b first,
+ *                      lower index first on equal keys
+ *   topk_gate[T, K]    device, float32 out: g = s / (sum of the selected s),
+ *                      from the unbiased s
+ *   counts   [N_r]     device, int32 out: number of tokens routed to each
+ *                      expert (overwritten, not accumulated)
+ *   workspace          device, >= moe_route_workspace_size(T, N_r) bytes
+ * Logits are accumulated in float32 from the stored values; sigmoid, keys and
+ * gates are float32.  Requires 1 <= K <= N_r <= 1024 and d % 64 == 0.
+ * ------------------------------------------------------------------------ */
+size_t moe_route_workspace_size(int T, int N_r);
+moe_status moe_route(const void* u, const void* E, moe_dtype dt, const float* b,
+                     int T, int d, int N_r, int K,
+                     int32_t* topk_idx, float* topk_gate, int32_t* counts,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * moe_permute - group the T*K (token, slot) pairs by expert and copy the
+ * token rows into that order (the dispatch step that feeds FFN^(r)_i in the
+ * h'-equation).  Inside an expert's group tokens keep ascending order.
+ *
+ *   u        [T, d]      device, dt (MOE_F32, MOE_BF16 or MOE_E4M3)
+ *   u_scale  [T, d/128]  device, float32: only for MOE_E4M3 (tile scales of u), else NULL
+ *   topk_idx [T, K]      device, int32: from moe_route
+ *   x_perm   [T*K, d]    device, dt out: x_perm[p] = u[perm_src[p]]
+ *   x_scale  [T*K, d/128] device, float32 out (MOE_E4M3 only, else NULL)
+ *   offsets  [N_r+1]     device, int32 out: group g is rows [offsets[g], offsets[g+1])
+ *   perm_src [T*K]       device, int32 out: grouped row -> token
+ *   inv_row  [T, K]      device, int32 out: (token, slot) -> grouped row
+ *   workspace            device, >= moe_permute_workspace_size(T, N_r) bytes
+ * Requires d * sizeof(dt) % 16 == 0 and 1 <= K <= N_r <= 1024.
+ * ------------------------------------------------------------------------ */
+size_t moe_permute_workspace_size(int T, int N_r);
+moe_status moe_permute(const void* u, const float* u_scale, moe_dtype dt,
+                       const int32_t* topk_idx, int T, int d, int N_r, int K,
+                       void* x_perm, float* x_scale,
+                       int32_t* offsets, int32_t* perm_src, int32_t* inv_row,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * moe_expert_ffn - grouped SwiGLU expert FFN: for every group g and every row
+ * r in [offsets[g], offsets[g+1]):
+ *     y[r] = W_down[g] (SiLU(W_gate[g] x[r]) * (W_up[g] x[r]))
+ * (FFN_i of the h'-equation; the SwiGLU form is this library's reading).
+ *
+ *   x          [rows, d]        device, dt
+ *   x_scale    [rows, d/128]    device, float32 (MOE_E4M3 only, else NULL)
+ *   offsets    [n_groups+1]     device, int32, non-decreasing, offsets[0] = 0,
+ *                               offsets[n_groups] <= rows
+ *   W_gate_up  [n_groups, 2I, d] device, dt: rows [0,I) are W_gate, [I,2I) W_up
+ *   w_scale_gate_up [n_groups, 2I/128, d/128] float32 (MOE_E4M3 only, else NULL)
+ *   W_down     [n_groups, d, I] device, dt
+ *   w_scale_down    [n_groups, d/128, I/128]  float32 (MOE_E4M3 only, else NULL)
+ *   y          [rows, d]        device out: float32 for MOE_F32, bf16 otherwise.
+ *                               Rows outside every group are not written.
+ *   workspace                   device, >= moe_expert_ffn_workspace_size(dt, rows, I)
+ * Arithmetic: MOE_F32 - float32 FMA; MOE_BF16 - tcgen05 tensor cores, float32
+ * accumulation in TMEM, SwiGLU in float32, the intermediate rounded to bf16;
+ * MOE_E4M3 - each 128-wide K block's partial sum is promoted to float32 with
+ * its activation and weight scales, the intermediate is re-quantised 1x128.
+ * Requires d % 128 == 0 and I % 128 == 0.
+ * ------------------------------------------------------------------------ */
+size_t moe_expert_ffn_workspace_size(moe_dtype dt, int rows, int I);
+moe_status moe_expert_ffn(const void* x, const float* x_scale, const int32_t* offsets,
+                          int n_groups, int rows, int d, int I, moe_dtype dt,
+                          const void* W_gate_up, const float* w_scale_gate_up,
+                          const void* W_down, const float* w_scale_down,
+                          void* y, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * moe_expert_gate_up / moe_expert_down - the two halves of moe_expert_ffn,
+ * for callers that schedule or time them apart (same layouts and rules):
+ *   gate_up: h[r] = SiLU(W_gate[g] x[r]) * (W_up[g] x[r])
+ *            h [rows, I]: float32 (MOE_F32), bf16 (MOE_BF16) or e4m3 with
+ *            h_scale [rows, I/128] float32 (MOE_E4M3; h_scale NULL otherwise)
+ *   down:    y[r] = W_down[g] h[r]
+ * moe_expert_ffn(...) is gate_up into its workspace followed by down.
+ * ------------------------------------------------------------------------ */
+moe_status moe_expert_gate_up(const void* x, const float* x_scale, const int32_t* offsets,
+                              int n_groups, int rows, int d, int I, moe_dtype dt,
+                              const void* W_gate_up, const float* w_scale_gate_up,
+                              void* h, float* h_scale, void* stream);
+moe_status moe_expert_down(const void* h, const float* h_scale, const int32_t* offsets,
+                           int n_groups, int rows, int d, int I, moe_dtype dt,
+                           const void* W_down, const float* w_scale_down, void* y, void* stream);
+
+/* ------------------------------------------------------------------------
+ * moe_combine - the h'-equation with the residual:
+ *   h_out[t] = u[t] + sum_{j<N_s} y_shared[j][t] + sum_k topk_gate[t,k] y_perm[inv_row[t,k]]
+ * summed in float32, rounded once to dt.
+ *
+ *   u         [T, d]       device, dt (MOE_F32 or MOE_BF16)
+ *   y_shared  [N_s, T, d]  device, dt (may be NULL when N_s == 0)
+ *   y_perm    [T*K, d]     device, dt: routed expert outputs in grouped order
+ *   inv_row   [T, K]       device, int32: from moe_permute
+ *   topk_gate [T, K]       device, float32: from moe_route
+ *   h_out     [T, d]       device, dt out (must not alias the inputs)
+ * Requires d * sizeof(dt) % 16 == 0.
+ * ------------------------------------------------------------------------ */
+moe_status moe_combine(const void* u, const void* y_shared, int N_s,
+                       const void* y_perm, const int32_t* inv_row, const float* topk_gate,
+                       moe_dtype dt, int T, int d, int K, void* h_out, void* stream);
+
+/* ------------------------------------------------------------------------
+ * moe_bias_update - the bias rule of section 2: with the mean load T*K/N_r,
+ *   b_i <- b_i - gamma  if counts_i * N_r > T * K   (overloaded)
+ *   b_i <- b_i + gamma  if counts_i * N_r < T * K   (underloaded)
+ *   b_i unchanged       if equal                    (gamma = 0.001 on the page)
+ * float32 arithmetic, in place.  counts from moe_route (or their sum over
+ * data-parallel replicas, with T the replicas' total token count).
+ * ------------------------------------------------------------------------ */
+moe_status moe_bias_update(float* b, const int32_t* counts, int N_r, int T, int K,
+                           float gamma, void* stream);
+
+/* ------------------------------------------------------------------------
+ * FP8 quantisers (recipe of section 核心概念, FP8 bullet).  scale = amax/448
+ * in float32 (1 for an all-zero tile); q = E4M3_rne_satfinite(x / scale) with
+ * an IEEE float32 division.
+ *
+ * moe_quantize_1x128: x [rows, cols] bf16 -> q [rows, cols] e4m3,
+ *                     scale [rows, cols/128] float32.  cols % 128 == 0.
+ * moe_quantize_128x128: w [groups, rows, cols] bf16 -> q e4m3,
+ *                     scale [groups, rows/128, cols/128] float32.
+ *                     rows % 128 == 0, cols % 128 == 0.
+ * ------------------------------------------------------------------------ */
+moe_status moe_quantize_1x128(const void* x, int rows, int cols,
+                              uint8_t* q, float* scale, void* stream);
+moe_status moe_quantize_128x128(const void* w, int groups, int rows, int cols,
+                                uint8_t* q, float* scale, void* stream);
+
+/* ------------------------------------------------------------------------
+ * moe_device_status - synchronises the current device, then returns (and
+ * clears) the library's device-side error word: 0 if no kernel gave up a
+ * bounded wait since the last call, else a bit set naming the kernel.
+ * ------------------------------------------------------------------------ */
+moe_status moe_device_status(int* flags);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -1,0 +1,197 @@
+"""Python binding of libmoe.so, the B200 DeepSeekMoE layer library.
+
+Argument marshalling only: every function here takes torch tensors that
+already live on the GPU, passes their device pointers and sizes to the C ABI
+of include/moe.h, and raises MoeError on a non-zero status.  All arithmetic
+runs in the library's CUDA kernels.  There is no CPU path: importing works
+without a GPU, but every call needs the built library and a B200.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "MoeError", "lib", "LIB_PATH", "SYMBOLS",
+    "moe_route", "moe_permute", "moe_expert_ffn", "moe_expert_gate_up", "moe_expert_down", "moe_combine", "moe_bias_update",
+    "moe_quantize_1x128", "moe_quantize_128x128", "moe_device_status",
+    "moe_route_workspace_size", "moe_permute_workspace_size", "moe_expert_ffn_workspace_size",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
+
+MOE_F32, MOE_BF16, MOE_E4M3 = 0, 1, 2
+STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
+          4: "MOE_ERR_CUDA", 5: "MOE_ERR_TIMEOUT"}
+
+_vp, _i, _sz, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+
+# name -> (restype, argtypes); mirrors include/moe.h
+SYMBOLS = {
+    "moe_abi_version": (_i, []),
+    "moe_last_error": (ctypes.c_char_p, []),
+    "moe_status_string": (ctypes.c_char_p, [_i]),
+    "moe_route_workspace_size": (_sz, [_i, _i]),
+    "moe_route": (_i, [_vp, _vp, _i, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_permute_workspace_size": (_sz, [_i, _i]),
+    "moe_permute": (_i, [_vp, _vp, _i, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_expert_ffn_workspace_size": (_sz, [_i, _i, _i]),
+    "moe_expert_ffn": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
+                            _vp]),
+    "moe_expert_gate_up": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp]),
+    "moe_expert_down": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
+    "moe_combine": (_i, [_vp, _vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp]),
+    "moe_bias_update": (_i, [_vp, _vp, _i, _i, _i, _f, _vp]),
+    "moe_quantize_1x128": (_i, [_vp, _i, _i, _vp, _vp, _vp]),
+    "moe_quantize_128x128": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp]),
+    "moe_device_status": (_i, [ctypes.POINTER(_i)]),
+}
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+_LIB = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libmoe.so; raises if it has not been built."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m mixture_experts_layer_60_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SYMBOLS.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = L
+    return _LIB
+
+
+def _check(status: int):
+    if status != 0:
+        raise MoeError(status, lib().moe_last_error().decode(errors="replace"))
+
+
+def _p(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libmoe takes device tensors only")
+    if not t.is_contiguous():
+        raise ValueError("libmoe takes contiguous tensors only")
+    return t.data_ptr()
+
+
+def _s(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dt(t):
+    if t.dtype == torch.float32:
+        return MOE_F32
+    if t.dtype == torch.bfloat16:
+        return MOE_BF16
+    if t.dtype in (torch.uint8, torch.float8_e4m3fn):
+        return MOE_E4M3
+    raise ValueError(f"unsupported dtype {t.dtype}")
+
+
+def _nbytes(t):
+    return 0 if t is None else t.numel() * t.element_size()
+
+
+# ------------------------------------------------------------------ sizes
+
+def moe_route_workspace_size(T: int, N_r: int) -> int:
+    return lib().moe_route_workspace_size(T, N_r)
+
+
+def moe_permute_workspace_size(T: int, N_r: int) -> int:
+    return lib().moe_permute_workspace_size(T, N_r)
+
+
+def moe_expert_ffn_workspace_size(dt: int, rows: int, I: int) -> int:
+    return lib().moe_expert_ffn_workspace_size(dt, rows, I)
+
+
+# ------------------------------------------------------------------ calls
+
+def moe_route(u, E, b, K, topk_idx, topk_gate, counts, workspace, stream=None):
+    T, d = u.shape
+    _check(lib().moe_route(_p(u), _p(E), _dt(u), _p(b), T, d, E.shape[0], K, _p(topk_idx),
+                           _p(topk_gate), _p(counts), _p(workspace), _nbytes(workspace),
+                           _s(stream)))
+
+
+def moe_permute(u, topk_idx, N_r, x_perm, offsets, perm_src, inv_row, workspace,
+                u_scale=None, x_scale=None, stream=None):
+    T, d = u.shape
+    K = topk_idx.shape[1]
+    _check(lib().moe_permute(_p(u), _p(u_scale), _dt(u), _p(topk_idx), T, d, N_r, K, _p(x_perm),
+                             _p(x_scale), _p(offsets), _p(perm_src), _p(inv_row), _p(workspace),
+                             _nbytes(workspace), _s(stream)))
+
+
+def moe_expert_ffn(x, offsets, W_gate_up, W_down, y, workspace, x_scale=None,
+                   w_scale_gate_up=None, w_scale_down=None, stream=None):
+    rows, d = x.shape
+    n_groups, two_i, _ = W_gate_up.shape
+    _check(lib().moe_expert_ffn(_p(x), _p(x_scale), _p(offsets), n_groups, rows, d, two_i // 2,
+                                _dt(x), _p(W_gate_up), _p(w_scale_gate_up), _p(W_down),
+                                _p(w_scale_down), _p(y), _p(workspace), _nbytes(workspace),
+                                _s(stream)))
+
+
+def moe_expert_gate_up(x, offsets, W_gate_up, h, x_scale=None, w_scale_gate_up=None,
+                       h_scale=None, stream=None):
+    rows, d = x.shape
+    n_groups, two_i, _ = W_gate_up.shape
+    _check(lib().moe_expert_gate_up(_p(x), _p(x_scale), _p(offsets), n_groups, rows, d,
+                                    two_i // 2, _dt(x), _p(W_gate_up), _p(w_scale_gate_up), _p(h),
+                                    _p(h_scale), _s(stream)))
+
+
+def moe_expert_down(h, offsets, W_down, y, h_scale=None, w_scale_down=None, stream=None):
+    rows, I = h.shape
+    n_groups, d, _ = W_down.shape
+    _check(lib().moe_expert_down(_p(h), _p(h_scale), _p(offsets), n_groups, rows, d, I, _dt(h),
+                                 _p(W_down), _p(w_scale_down), _p(y), _s(stream)))
+
+
+def moe_combine(u, y_shared, y_perm, inv_row, topk_gate, h_out, stream=None):
+    T, d = u.shape
+    N_s = 0 if y_shared is None else y_shared.shape[0]
+    _check(lib().moe_combine(_p(u), _p(y_shared), N_s, _p(y_perm), _p(inv_row), _p(topk_gate),
+                             _dt(u), T, d, inv_row.shape[1], _p(h_out), _s(stream)))
+
+
+def moe_bias_update(b, counts, T, K, gamma=0.001, stream=None):
+    _check(lib().moe_bias_update(_p(b), _p(counts), b.shape[0], T, K, gamma, _s(stream)))
+
+
+def moe_quantize_1x128(x, q, scale, stream=None):
+    rows, cols = x.shape
+    _check(lib().moe_quantize_1x128(_p(x), rows, cols, _p(q), _p(scale), _s(stream)))
+
+
+def moe_quantize_128x128(w, q, scale, stream=None):
+    groups, rows, cols = w.shape
+    _check(lib().moe_quantize_128x128(_p(w), groups, rows, cols, _p(q), _p(scale), _s(stream)))
+
+
+def moe_device_status() -> int:
+    flags = ctypes.c_int(0)
+    st = lib().moe_device_status(ctypes.byref(flags))
+    if st not in (0, 5):
+        _check(st)
+    return flags.value

@@ -1,0 +1,349 @@
+// extern "C" entry points of libmoe.so (declared in include/moe.h).  Each
+// validates its arguments on the host, then enqueues kernels on `stream`.
+#include "launch.h"
+
+namespace moe {
+const char* last_error_text();
+void clear_last_error();
+}  // namespace moe
+
+using namespace moe;
+
+namespace {
+
+constexpr int kAbiVersion = 1;
+
+inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+int dtype_bytes(moe_dtype dt) {
+  switch (dt) {
+    case MOE_F32: return 4;
+    case MOE_BF16: return 2;
+    case MOE_E4M3: return 1;
+  }
+  return 0;
+}
+
+moe_status check_device() {
+  if (!device_is_sm100())
+    return fail(MOE_ERR_UNSUPPORTED, "libmoe kernels need an sm_100 (B200) device");
+  return MOE_OK;
+}
+
+#define MOE_REQUIRE(cond, status, ...) \
+  do {                                 \
+    if (!(cond)) return fail(status, __VA_ARGS__); \
+  } while (0)
+
+#define MOE_TRY(expr)                 \
+  do {                                \
+    moe_status _st = (expr);          \
+    if (_st != MOE_OK) return _st;    \
+  } while (0)
+
+size_t route_ws(int T, int N_r) {
+  if (T <= 0 || N_r <= 0) return 0;
+  return align_up((size_t)T * N_r * sizeof(float), 256);
+}
+
+size_t ffn_ws(moe_dtype dt, int rows, int I) {
+  if (rows <= 0 || I <= 0) return 0;
+  switch (dt) {
+    case MOE_F32: return align_up((size_t)rows * I * 4, 256);
+    case MOE_BF16: return align_up((size_t)rows * I * 2, 256);
+    case MOE_E4M3:
+      return align_up((size_t)rows * I, 256) + align_up((size_t)rows * (I / 128) * 4, 256);
+  }
+  return 0;
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_abi_version(void) { return kAbiVersion; }
+
+const char* moe_last_error(void) { return last_error_text(); }
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+  }
+  return "MOE_STATUS_UNKNOWN";
+}
+
+size_t moe_route_workspace_size(int T, int N_r) { return route_ws(T, N_r); }
+
+moe_status moe_route(const void* u, const void* E, moe_dtype dt, const float* b, int T, int d,
+                     int N_r, int K, int32_t* topk_idx, float* topk_gate, int32_t* counts,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+  clear_last_error();
+  MOE_REQUIRE(dt == MOE_F32 || dt == MOE_BF16, MOE_ERR_UNSUPPORTED,
+              "moe_route: dtype must be MOE_F32 or MOE_BF16");
+  MOE_REQUIRE(T >= 0 && d > 0 && N_r > 0 && K > 0, MOE_ERR_INVALID_ARG,
+              "moe_route: bad sizes T=%d d=%d N_r=%d K=%d", T, d, N_r, K);
+  MOE_REQUIRE(N_r <= 1024 && K <= N_r, MOE_ERR_UNSUPPORTED,
+              "moe_route: need 1 <= K <= N_r <= 1024 (K=%d N_r=%d)", K, N_r);
+  MOE_REQUIRE(d % 64 == 0, MOE_ERR_UNSUPPORTED, "moe_route: d=%d must be a multiple of 64", d);
+  MOE_REQUIRE(E && b && counts, MOE_ERR_INVALID_ARG, "moe_route: null pointer");
+  MOE_REQUIRE(T == 0 || (u && topk_idx && topk_gate && workspace), MOE_ERR_INVALID_ARG,
+              "moe_route: null pointer");
+  MOE_REQUIRE(workspace_bytes >= route_ws(T, N_r), MOE_ERR_WORKSPACE,
+              "moe_route: workspace %zu < %zu bytes", workspace_bytes, route_ws(T, N_r));
+  MOE_REQUIRE(T == 0 || reinterpret_cast<uintptr_t>(workspace) % 256 == 0, MOE_ERR_INVALID_ARG,
+              "moe_route: workspace must be 256-byte aligned");
+  MOE_TRY(check_device());
+  cudaStream_t s = as_stream(stream);
+  MOE_TRY(cuda_check(cudaMemsetAsync(counts, 0, (size_t)N_r * sizeof(int32_t), s), "zero counts"));
+  if (T == 0) return MOE_OK;
+  float* logits = static_cast<float*>(workspace);
+  if (dt == MOE_BF16 && N_r % 64 == 0) {
+    MOE_TRY(launch_tc_gemm(u, E, N_r, nullptr, 1, T, N_r, d, TC_EPI_STORE_F32, logits, s));
+  } else {
+    MOE_TRY(launch_logits_simt(u, E, dt, T, d, N_r, logits, s));
+  }
+  return launch_topk(logits, b, T, N_r, K, topk_idx, topk_gate, counts, s);
+}
+
+size_t moe_permute_workspace_size(int T, int N_r) {
+  if (T <= 0 || N_r <= 0) return 0;
+  return permute_ws_bytes(T, N_r);
+}
+
+moe_status moe_permute(const void* u, const float* u_scale, moe_dtype dt, const int32_t* topk_idx,
+                       int T, int d, int N_r, int K, void* x_perm, float* x_scale,
+                       int32_t* offsets, int32_t* perm_src, int32_t* inv_row, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  clear_last_error();
+  const int eb = dtype_bytes(dt);
+  MOE_REQUIRE(eb > 0, MOE_ERR_UNSUPPORTED, "moe_permute: unknown dtype %d", (int)dt);
+  MOE_REQUIRE(T >= 0 && d > 0 && N_r > 0 && K > 0, MOE_ERR_INVALID_ARG,
+              "moe_permute: bad sizes T=%d d=%d N_r=%d K=%d", T, d, N_r, K);
+  MOE_REQUIRE(N_r <= 1024 && K <= N_r, MOE_ERR_UNSUPPORTED,
+              "moe_permute: need 1 <= K <= N_r <= 1024");
+  MOE_REQUIRE(((size_t)d * eb) % 16 == 0, MOE_ERR_UNSUPPORTED,
+              "moe_permute: a row (%d x %d bytes) must be a multiple of 16 bytes", d, eb);
+  MOE_REQUIRE((8LL * N_r + 256LL * K) * 4 <= 200 * 1024, MOE_ERR_UNSUPPORTED,
+              "moe_permute: K=%d with N_r=%d exceeds the rank kernel's shared memory", K, N_r);
+  MOE_REQUIRE(offsets, MOE_ERR_INVALID_ARG, "moe_permute: null offsets");
+  MOE_REQUIRE(T == 0 || (u && topk_idx && x_perm && perm_src && inv_row && workspace),
+              MOE_ERR_INVALID_ARG, "moe_permute: null pointer");
+  if (dt == MOE_E4M3) {
+    MOE_REQUIRE(d % 128 == 0, MOE_ERR_UNSUPPORTED, "moe_permute: e4m3 needs d %% 128 == 0");
+    MOE_REQUIRE(T == 0 || (u_scale && x_scale), MOE_ERR_INVALID_ARG,
+                "moe_permute: e4m3 needs u_scale and x_scale");
+  } else {
+    MOE_REQUIRE(!u_scale && !x_scale, MOE_ERR_INVALID_ARG,
+                "moe_permute: scales are only for MOE_E4M3");
+  }
+  MOE_REQUIRE(workspace_bytes >= moe_permute_workspace_size(T, N_r), MOE_ERR_WORKSPACE,
+              "moe_permute: workspace %zu < %zu bytes", workspace_bytes,
+              moe_permute_workspace_size(T, N_r));
+  MOE_REQUIRE(reinterpret_cast<uintptr_t>(u) % 16 == 0 &&
+                  reinterpret_cast<uintptr_t>(x_perm) % 16 == 0,
+              MOE_ERR_INVALID_ARG, "moe_permute: u and x_perm must be 16-byte aligned");
+  MOE_TRY(check_device());
+  cudaStream_t s = as_stream(stream);
+  if (T == 0)
+    return cuda_check(cudaMemsetAsync(offsets, 0, (size_t)(N_r + 1) * sizeof(int32_t), s),
+                      "zero offsets");
+  return launch_permute(u, dt == MOE_E4M3 ? u_scale : nullptr, eb, topk_idx, T, d, N_r, K, x_perm,
+                        dt == MOE_E4M3 ? x_scale : nullptr, offsets, perm_src, inv_row, workspace,
+                        s);
+}
+
+size_t moe_expert_ffn_workspace_size(moe_dtype dt, int rows, int I) { return ffn_ws(dt, rows, I); }
+
+namespace {
+
+moe_status check_ffn_common(const char* who, const void* x, const int32_t* offsets, int n_groups,
+                            int rows, int d, int I, moe_dtype dt, const void* W) {
+  MOE_REQUIRE(dtype_bytes(dt) > 0, MOE_ERR_UNSUPPORTED, "%s: unknown dtype", who);
+  MOE_REQUIRE(rows >= 0 && d > 0 && I > 0 && n_groups > 0, MOE_ERR_INVALID_ARG,
+              "%s: bad sizes rows=%d d=%d I=%d n_groups=%d", who, rows, d, I, n_groups);
+  MOE_REQUIRE(n_groups <= 1024, MOE_ERR_UNSUPPORTED, "%s: at most 1024 groups", who);
+  MOE_REQUIRE(d % 128 == 0 && I % 128 == 0, MOE_ERR_UNSUPPORTED,
+              "%s: d=%d and I=%d must be multiples of 128", who, d, I);
+  MOE_REQUIRE(offsets && W, MOE_ERR_INVALID_ARG, "%s: null pointer", who);
+  MOE_REQUIRE(rows == 0 || x, MOE_ERR_INVALID_ARG, "%s: null pointer", who);
+  return MOE_OK;
+}
+
+moe_status run_gate_up(const void* x, const float* x_scale, const int32_t* offsets, int n_groups,
+                       int rows, int d, int I, moe_dtype dt, const void* W_gate_up,
+                       const float* w_scale_gate_up, void* h, float* h_scale, cudaStream_t s) {
+  if (dt == MOE_F32)
+    return launch_simt_gemm(x, W_gate_up, 2LL * I * d, offsets, n_groups, rows, I, d, true,
+                            MOE_F32, h, MOE_F32, s);
+  if (dt == MOE_BF16)
+    return launch_tc_gemm(x, W_gate_up, 2 * I, offsets, n_groups, rows, I, d, TC_EPI_SWIGLU_BF16,
+                          h, s);
+  return launch_fp8_gemm(x, x_scale, W_gate_up, w_scale_gate_up, 2 * I, offsets, n_groups, rows,
+                         I, d, true, h, h_scale, s);
+}
+
+moe_status run_down(const void* h, const float* h_scale, const int32_t* offsets, int n_groups,
+                    int rows, int d, int I, moe_dtype dt, const void* W_down,
+                    const float* w_scale_down, void* y, cudaStream_t s) {
+  if (dt == MOE_F32)
+    return launch_simt_gemm(h, W_down, (long long)d * I, offsets, n_groups, rows, d, I, false,
+                            MOE_F32, y, MOE_F32, s);
+  if (dt == MOE_BF16)
+    return launch_tc_gemm(h, W_down, d, offsets, n_groups, rows, d, I, TC_EPI_STORE_BF16, y, s);
+  return launch_fp8_gemm(h, h_scale, W_down, w_scale_down, d, offsets, n_groups, rows, d, I,
+                         false, y, nullptr, s);
+}
+
+moe_status check_scales(const char* who, moe_dtype dt, const void* a, const void* b) {
+  if (dt == MOE_E4M3)
+    MOE_REQUIRE(a && b, MOE_ERR_INVALID_ARG, "%s: e4m3 needs activation and weight scales", who);
+  else
+    MOE_REQUIRE(!a && !b, MOE_ERR_INVALID_ARG, "%s: scales are only for MOE_E4M3", who);
+  return MOE_OK;
+}
+
+}  // namespace
+
+moe_status moe_expert_ffn(const void* x, const float* x_scale, const int32_t* offsets,
+                          int n_groups, int rows, int d, int I, moe_dtype dt,
+                          const void* W_gate_up, const float* w_scale_gate_up,
+                          const void* W_down, const float* w_scale_down, void* y,
+                          void* workspace, size_t workspace_bytes, void* stream) {
+  clear_last_error();
+  MOE_TRY(check_ffn_common("moe_expert_ffn", x, offsets, n_groups, rows, d, I, dt, W_gate_up));
+  MOE_REQUIRE(W_down, MOE_ERR_INVALID_ARG, "moe_expert_ffn: null pointer");
+  if (rows == 0) return MOE_OK;
+  MOE_REQUIRE(y && workspace, MOE_ERR_INVALID_ARG, "moe_expert_ffn: null pointer");
+  MOE_TRY(check_scales("moe_expert_ffn", dt, x_scale, w_scale_gate_up));
+  MOE_TRY(check_scales("moe_expert_ffn", dt, x_scale, w_scale_down));
+  MOE_REQUIRE(workspace_bytes >= ffn_ws(dt, rows, I), MOE_ERR_WORKSPACE,
+              "moe_expert_ffn: workspace %zu < %zu bytes", workspace_bytes, ffn_ws(dt, rows, I));
+  MOE_REQUIRE(reinterpret_cast<uintptr_t>(workspace) % 256 == 0 &&
+                  reinterpret_cast<uintptr_t>(y) % 16 == 0,
+              MOE_ERR_INVALID_ARG, "moe_expert_ffn: workspace 256-byte and y 16-byte alignment");
+  MOE_TRY(check_device());
+  cudaStream_t s = as_stream(stream);
+  void* h = workspace;
+  float* hs = dt == MOE_E4M3
+                  ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                             align_up((size_t)rows * I, 256))
+                  : nullptr;
+  MOE_TRY(run_gate_up(x, x_scale, offsets, n_groups, rows, d, I, dt, W_gate_up, w_scale_gate_up, h,
+                      hs, s));
+  return run_down(h, hs, offsets, n_groups, rows, d, I, dt, W_down, w_scale_down, y, s);
+}
+
+moe_status moe_expert_gate_up(const void* x, const float* x_scale, const int32_t* offsets,
+                              int n_groups, int rows, int d, int I, moe_dtype dt,
+                              const void* W_gate_up, const float* w_scale_gate_up, void* h,
+                              float* h_scale, void* stream) {
+  clear_last_error();
+  MOE_TRY(check_ffn_common("moe_expert_gate_up", x, offsets, n_groups, rows, d, I, dt, W_gate_up));
+  if (rows == 0) return MOE_OK;
+  MOE_REQUIRE(h, MOE_ERR_INVALID_ARG, "moe_expert_gate_up: null h");
+  MOE_TRY(check_scales("moe_expert_gate_up", dt, x_scale, w_scale_gate_up));
+  MOE_REQUIRE(dt != MOE_E4M3 || h_scale, MOE_ERR_INVALID_ARG, "moe_expert_gate_up: null h_scale");
+  MOE_REQUIRE(dt == MOE_E4M3 || !h_scale, MOE_ERR_INVALID_ARG,
+              "moe_expert_gate_up: h_scale is only for MOE_E4M3");
+  MOE_REQUIRE(reinterpret_cast<uintptr_t>(h) % 16 == 0, MOE_ERR_INVALID_ARG,
+              "moe_expert_gate_up: h must be 16-byte aligned");
+  MOE_TRY(check_device());
+  return run_gate_up(x, x_scale, offsets, n_groups, rows, d, I, dt, W_gate_up, w_scale_gate_up, h,
+                     h_scale, as_stream(stream));
+}
+
+moe_status moe_expert_down(const void* h, const float* h_scale, const int32_t* offsets,
+                           int n_groups, int rows, int d, int I, moe_dtype dt, const void* W_down,
+                           const float* w_scale_down, void* y, void* stream) {
+  clear_last_error();
+  MOE_TRY(check_ffn_common("moe_expert_down", h, offsets, n_groups, rows, d, I, dt, W_down));
+  if (rows == 0) return MOE_OK;
+  MOE_REQUIRE(y, MOE_ERR_INVALID_ARG, "moe_expert_down: null y");
+  MOE_TRY(check_scales("moe_expert_down", dt, h_scale, w_scale_down));
+  MOE_REQUIRE(reinterpret_cast<uintptr_t>(y) % 16 == 0 &&
+                  reinterpret_cast<uintptr_t>(h) % 16 == 0,
+              MOE_ERR_INVALID_ARG, "moe_expert_down: h and y must be 16-byte aligned");
+  MOE_TRY(check_device());
+  return run_down(h, h_scale, offsets, n_groups, rows, d, I, dt, W_down, w_scale_down, y,
+                  as_stream(stream));
+}
+
+moe_status moe_combine(const void* u, const void* y_shared, int N_s, const void* y_perm,
+                       const int32_t* inv_row, const float* topk_gate, moe_dtype dt, int T, int d,
+                       int K, void* h_out, void* stream) {
+  clear_last_error();
+  MOE_REQUIRE(dt == MOE_F32 || dt == MOE_BF16, MOE_ERR_UNSUPPORTED,
+              "moe_combine: dtype must be MOE_F32 or MOE_BF16");
+  MOE_REQUIRE(T >= 0 && d > 0 && K > 0 && N_s >= 0, MOE_ERR_INVALID_ARG,
+              "moe_combine: bad sizes T=%d d=%d K=%d N_s=%d", T, d, K, N_s);
+  MOE_REQUIRE(((size_t)d * dtype_bytes(dt)) % 16 == 0, MOE_ERR_UNSUPPORTED,
+              "moe_combine: a row must be a multiple of 16 bytes");
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE(u && y_perm && inv_row && topk_gate && h_out && (N_s == 0 || y_shared),
+              MOE_ERR_INVALID_ARG, "moe_combine: null pointer");
+  MOE_REQUIRE(reinterpret_cast<uintptr_t>(u) % 16 == 0 &&
+                  reinterpret_cast<uintptr_t>(y_perm) % 16 == 0 &&
+                  reinterpret_cast<uintptr_t>(h_out) % 16 == 0 &&
+                  reinterpret_cast<uintptr_t>(y_shared) % 16 == 0,
+              MOE_ERR_INVALID_ARG, "moe_combine: rows must be 16-byte aligned");
+  MOE_TRY(check_device());
+  return launch_combine(u, y_shared, N_s, y_perm, inv_row, topk_gate, dt, T, d, K, h_out,
+                        as_stream(stream));
+}
+
+moe_status moe_bias_update(float* b, const int32_t* counts, int N_r, int T, int K, float gamma,
+                           void* stream) {
+  clear_last_error();
+  MOE_REQUIRE(b && counts, MOE_ERR_INVALID_ARG, "moe_bias_update: null pointer");
+  MOE_REQUIRE(N_r > 0 && T >= 0 && K > 0, MOE_ERR_INVALID_ARG,
+              "moe_bias_update: bad sizes N_r=%d T=%d K=%d", N_r, T, K);
+  MOE_TRY(check_device());
+  return launch_bias_update(b, counts, N_r, T, K, gamma, as_stream(stream));
+}
+
+moe_status moe_quantize_1x128(const void* x, int rows, int cols, uint8_t* q, float* scale,
+                              void* stream) {
+  clear_last_error();
+  MOE_REQUIRE(rows >= 0 && cols > 0 && cols % 128 == 0, MOE_ERR_UNSUPPORTED,
+              "moe_quantize_1x128: cols=%d must be a positive multiple of 128", cols);
+  if (rows == 0) return MOE_OK;
+  MOE_REQUIRE(x && q && scale, MOE_ERR_INVALID_ARG, "moe_quantize_1x128: null pointer");
+  MOE_REQUIRE(reinterpret_cast<uintptr_t>(x) % 16 == 0 && reinterpret_cast<uintptr_t>(q) % 16 == 0,
+              MOE_ERR_INVALID_ARG, "moe_quantize_1x128: x and q must be 16-byte aligned");
+  MOE_TRY(check_device());
+  return launch_quant_1x128(x, rows, cols, q, scale, as_stream(stream));
+}
+
+moe_status moe_quantize_128x128(const void* w, int groups, int rows, int cols, uint8_t* q,
+                                float* scale, void* stream) {
+  clear_last_error();
+  MOE_REQUIRE(groups >= 0 && rows > 0 && cols > 0 && rows % 128 == 0 && cols % 128 == 0,
+              MOE_ERR_UNSUPPORTED, "moe_quantize_128x128: rows=%d cols=%d must be multiples of 128",
+              rows, cols);
+  if (groups == 0) return MOE_OK;
+  MOE_REQUIRE(w && q && scale, MOE_ERR_INVALID_ARG, "moe_quantize_128x128: null pointer");
+  MOE_REQUIRE(reinterpret_cast<uintptr_t>(w) % 16 == 0 && reinterpret_cast<uintptr_t>(q) % 16 == 0,
+              MOE_ERR_INVALID_ARG, "moe_quantize_128x128: w and q must be 16-byte aligned");
+  MOE_TRY(check_device());
+  return launch_quant_128x128(w, groups, rows, cols, q, scale, as_stream(stream));
+}
+
+moe_status moe_device_status(int* flags) {
+  clear_last_error();
+  MOE_REQUIRE(flags, MOE_ERR_INVALID_ARG, "moe_device_status: null pointer");
+  *flags = 0;
+  MOE_TRY(cuda_check(cudaDeviceSynchronize(), "moe_device_status synchronize"));
+  int* word = device_error_word();
+  MOE_REQUIRE(word, MOE_ERR_CUDA, "moe_device_status: error word unavailable");
+  MOE_TRY(cuda_check(cudaMemcpy(flags, word, sizeof(int), cudaMemcpyDeviceToHost), "read error word"));
+  MOE_TRY(cuda_check(cudaMemset(word, 0, sizeof(int)), "clear error word"));
+  return *flags ? fail(MOE_ERR_TIMEOUT, "a kernel gave up a bounded wait (flags 0x%x)", *flags)
+                : MOE_OK;
+}
+
+}  // extern "C"

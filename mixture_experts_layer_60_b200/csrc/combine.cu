@@ -1,0 +1,165 @@
+// Combine with the residual, the h'-equation of "DeepSeek-V3 技術報告"
+// (section 方法 / 2):
+//   h'_t = u_t + sum_j FFN^(s)_j(u_t) + sum_k g_{t,k} FFN^(r)_{idx(t,k)}(u_t),
+// and the per-step bias rule of the same section.
+#include "launch.h"
+
+namespace moe {
+
+// 8 bf16 or 4 f32 lanes per 16-byte vector.
+template <typename T> struct Vec;
+template <> struct Vec<float> {
+  static constexpr int N = 4;
+  static __device__ __forceinline__ void load(const uint4& v, float* f) {
+    f[0] = __uint_as_float(v.x); f[1] = __uint_as_float(v.y);
+    f[2] = __uint_as_float(v.z); f[3] = __uint_as_float(v.w);
+  }
+  static __device__ __forceinline__ uint4 store(const float* f) {
+    return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                      __float_as_uint(f[3]));
+  }
+};
+template <> struct Vec<__nv_bfloat16> {
+  static constexpr int N = 8;
+  static __device__ __forceinline__ void load(const uint4& v, float* f) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      f[2 * i] = __uint_as_float(w[i] << 16);
+      f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  }
+  static __device__ __forceinline__ uint4 store(const float* f) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __nv_bfloat162 p = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+      w[i] = *reinterpret_cast<uint32_t*>(&p);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+  }
+};
+
+// One warp per token; each lane walks the row in 16-byte vectors.  Every
+// input row is read exactly once; sums are float32 in the order
+// u, shared experts (j ascending), routed experts (slot k ascending).
+template <typename E, int KMAX>
+__global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ u,
+                                                      const uint4* __restrict__ ys, int N_s,
+                                                      const uint4* __restrict__ yp,
+                                                      const int32_t* __restrict__ inv_row,
+                                                      const float* __restrict__ gate, int T,
+                                                      int nvec, int K, uint4* __restrict__ out) {
+  constexpr int N = Vec<E>::N;
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  int rows[KMAX];
+  float g[KMAX];
+#pragma unroll
+  for (int k = 0; k < KMAX; ++k) {
+    if (k < K) {
+      rows[k] = inv_row[(size_t)t * K + k];
+      g[k] = gate[(size_t)t * K + k];
+    }
+  }
+  for (int c = lane; c < nvec; c += 32) {
+    float acc[N], tmp[N];
+    Vec<E>::load(u[(size_t)t * nvec + c], acc);
+    for (int j = 0; j < N_s; ++j) {
+      Vec<E>::load(ys[((size_t)j * T + t) * nvec + c], tmp);
+#pragma unroll
+      for (int i = 0; i < N; ++i) acc[i] += tmp[i];
+    }
+    uint4 raw[KMAX];
+#pragma unroll
+    for (int k = 0; k < KMAX; ++k)
+      if (k < K) raw[k] = yp[(size_t)rows[k] * nvec + c];
+#pragma unroll
+    for (int k = 0; k < KMAX; ++k) {
+      if (k < K) {
+        Vec<E>::load(raw[k], tmp);
+#pragma unroll
+        for (int i = 0; i < N; ++i) acc[i] = fmaf(g[k], tmp[i], acc[i]);
+      }
+    }
+    out[(size_t)t * nvec + c] = Vec<E>::store(acc);
+  }
+}
+
+// Generic K (> 16): slots read one after another.
+template <typename E>
+__global__ void __launch_bounds__(256) combine_kernel_anyk(const uint4* __restrict__ u,
+                                                           const uint4* __restrict__ ys, int N_s,
+                                                           const uint4* __restrict__ yp,
+                                                           const int32_t* __restrict__ inv_row,
+                                                           const float* __restrict__ gate, int T,
+                                                           int nvec, int K,
+                                                           uint4* __restrict__ out) {
+  constexpr int N = Vec<E>::N;
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  for (int c = lane; c < nvec; c += 32) {
+    float acc[N], tmp[N];
+    Vec<E>::load(u[(size_t)t * nvec + c], acc);
+    for (int j = 0; j < N_s; ++j) {
+      Vec<E>::load(ys[((size_t)j * T + t) * nvec + c], tmp);
+      for (int i = 0; i < N; ++i) acc[i] += tmp[i];
+    }
+    for (int k = 0; k < K; ++k) {
+      const float gk = gate[(size_t)t * K + k];
+      Vec<E>::load(yp[(size_t)inv_row[(size_t)t * K + k] * nvec + c], tmp);
+      for (int i = 0; i < N; ++i) acc[i] = fmaf(gk, tmp[i], acc[i]);
+    }
+    out[(size_t)t * nvec + c] = Vec<E>::store(acc);
+  }
+}
+
+template <typename E>
+static void combine_dispatch(const void* u, const void* ys, int N_s, const void* yp,
+                             const int32_t* inv_row, const float* gate, int T, int d, int K,
+                             void* out, cudaStream_t s) {
+  const int nvec = d / Vec<E>::N;
+  const int wpb = 8;
+  dim3 grid((T + wpb - 1) / wpb), block(wpb * 32);
+  auto U = static_cast<const uint4*>(u);
+  auto YS = static_cast<const uint4*>(ys);
+  auto YP = static_cast<const uint4*>(yp);
+  auto O = static_cast<uint4*>(out);
+  if (K <= 8)
+    combine_kernel<E, 8><<<grid, block, 0, s>>>(U, YS, N_s, YP, inv_row, gate, T, nvec, K, O);
+  else if (K <= 16)
+    combine_kernel<E, 16><<<grid, block, 0, s>>>(U, YS, N_s, YP, inv_row, gate, T, nvec, K, O);
+  else
+    combine_kernel_anyk<E><<<grid, block, 0, s>>>(U, YS, N_s, YP, inv_row, gate, T, nvec, K, O);
+}
+
+moe_status launch_combine(const void* u, const void* y_shared, int N_s, const void* y_perm,
+                          const int32_t* inv_row, const float* gate, moe_dtype dt, int T,
+                          int d, int K, void* h_out, cudaStream_t s) {
+  if (dt == MOE_F32)
+    combine_dispatch<float>(u, y_shared, N_s, y_perm, inv_row, gate, T, d, K, h_out, s);
+  else
+    combine_dispatch<__nv_bfloat16>(u, y_shared, N_s, y_perm, inv_row, gate, T, d, K, h_out, s);
+  return cuda_check(cudaGetLastError(), "combine launch");
+}
+
+// Bias rule: compare the load with the mean T*K/N_r in integers
+// (counts*N_r vs T*K) so that the mean need not be representable.
+__global__ void bias_update_kernel(float* __restrict__ b, const int32_t* __restrict__ counts,
+                                   int N_r, long long TK, float gamma) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= N_r) return;
+  const long long load = (long long)counts[i] * N_r;
+  if (load > TK) b[i] = b[i] - gamma;
+  else if (load < TK) b[i] = b[i] + gamma;
+}
+
+moe_status launch_bias_update(float* b, const int32_t* counts, int N_r, int T, int K,
+                              float gamma, cudaStream_t s) {
+  bias_update_kernel<<<(N_r + 255) / 256, 256, 0, s>>>(b, counts, N_r, (long long)T * K, gamma);
+  return cuda_check(cudaGetLastError(), "bias_update launch");
+}
+
+}  // namespace moe

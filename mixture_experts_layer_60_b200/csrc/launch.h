@@ -1,0 +1,57 @@
+// Internal launchers behind the C ABI (include/moe.h).  Every launcher
+// assumes its arguments were validated by the entry point in api.cu.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+// router.cu ------------------------------------------------------------------
+// logits[t, i] = sum_k u[t,k] E[i,k] on CUDA cores (float32 accumulation).
+moe_status launch_logits_simt(const void* u, const void* E, moe_dtype dt, int T, int d,
+                              int N_r, float* logits, cudaStream_t s);
+// sigmoid, biased top-K, gates, histogram (counts must be zeroed beforehand).
+moe_status launch_topk(const float* logits, const float* b, int T, int N_r, int K,
+                       int32_t* idx, float* gate, int32_t* counts, cudaStream_t s);
+
+// permute.cu -----------------------------------------------------------------
+size_t permute_ws_bytes(int T, int N_r);
+moe_status launch_permute(const void* u, const float* u_scale, int elem_bytes, const int32_t* idx,
+                          int T, int d, int N_r, int K, void* x_perm, float* x_scale,
+                          int32_t* offsets, int32_t* perm_src, int32_t* inv_row,
+                          void* ws, cudaStream_t s);
+
+// ffn_simt.cu ----------------------------------------------------------------
+// Grouped C[r, :] = epilogue(A[r, :] . B[g]^T) on CUDA cores.  swiglu: B has
+// 2N rows (gate rows [0,N), up rows [N,2N)); C = SiLU(gate) * up.
+// offsets == nullptr means one group covering all rows.
+moe_status launch_simt_gemm(const void* A, const void* B, long long b_group_stride,
+                            const int32_t* offsets, int n_groups, int rows, int N, int K,
+                            bool swiglu, moe_dtype in_dt, void* C, moe_dtype out_dt,
+                            cudaStream_t s);
+
+// gemm_tc.cu -----------------------------------------------------------------
+// Grouped bf16 GEMM on tcgen05 tensor cores (TMA -> smem -> tcgen05.mma -> TMEM).
+enum TcEpilogue { TC_EPI_STORE_BF16 = 0, TC_EPI_STORE_F32 = 1, TC_EPI_SWIGLU_BF16 = 2 };
+moe_status launch_tc_gemm(const void* A, const void* B, int b_rows_per_group,
+                          const int32_t* offsets, int n_groups, int rows, int N, int K,
+                          TcEpilogue epi, void* C, cudaStream_t s);
+
+// gemm_fp8.cu ----------------------------------------------------------------
+moe_status launch_fp8_gemm(const void* A, const float* a_scale, const void* B,
+                           const float* b_scale, int b_rows_per_group,
+                           const int32_t* offsets, int n_groups, int rows, int N, int K,
+                           bool swiglu, void* C, float* c_scale, cudaStream_t s);
+moe_status launch_quant_1x128(const void* x, int rows, int cols, uint8_t* q, float* scale,
+                              cudaStream_t s);
+moe_status launch_quant_128x128(const void* w, int groups, int rows, int cols, uint8_t* q,
+                                float* scale, cudaStream_t s);
+
+// combine.cu -----------------------------------------------------------------
+moe_status launch_combine(const void* u, const void* y_shared, int N_s, const void* y_perm,
+                          const int32_t* inv_row, const float* gate, moe_dtype dt, int T,
+                          int d, int K, void* h_out, cudaStream_t s);
+moe_status launch_bias_update(float* b, const int32_t* counts, int N_r, int T, int K,
+                              float gamma, cudaStream_t s);
+
+}  // namespace moe

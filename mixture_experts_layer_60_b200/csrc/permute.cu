@@ -1,0 +1,192 @@
+// Dispatch permutation: groups the T*K (token, slot) pairs by expert, tokens
+// ascending inside each group, and copies the token rows into that order.
+// This is the dispatch step that hands every token to the routed experts
+// FFN_i of the h'-equation ("DeepSeek-V3 技術報告", section 方法 / 2).
+//
+// Four launches:
+//   1. chunk_hist   per 256-token chunk, how many pairs go to each expert
+//   2. chunk_scan   offsets (exclusive scan of the load) and, per chunk and
+//                   expert, the first grouped row the chunk writes
+//   3. chunk_rank   stable rank of each pair inside its chunk -> perm_src, inv_row
+//   4. scatter_rows one warp per token: read the row once, store it K times
+//                   with 16-byte vectors (and the FP8 tile scales, if any)
+#include "launch.h"
+
+namespace moe {
+
+static constexpr int kChunk = 256;  // tokens per chunk = threads per block of steps 1 and 3
+
+static inline int n_chunks(int T) { return (T + kChunk - 1) / kChunk; }
+
+size_t permute_ws_bytes(int T, int N_r) {
+  // chunk_hist and chunk_base, [n_chunks, N_r] int32 each
+  return 2 * align_up((size_t)n_chunks(T) * N_r * sizeof(int32_t), 256);
+}
+
+__global__ void __launch_bounds__(kChunk) chunk_hist_kernel(const int32_t* __restrict__ idx, int T,
+                                                            int N_r, int K,
+                                                            int32_t* __restrict__ chunk_hist) {
+  extern __shared__ int h[];
+  for (int i = threadIdx.x; i < N_r; i += blockDim.x) h[i] = 0;
+  __syncthreads();
+  const int c = blockIdx.x;
+  const int t = c * kChunk + threadIdx.x;
+  if (t < T)
+    for (int k = 0; k < K; ++k) atomicAdd(&h[idx[(size_t)t * K + k]], 1);
+  __syncthreads();
+  for (int i = threadIdx.x; i < N_r; i += blockDim.x) chunk_hist[(size_t)c * N_r + i] = h[i];
+}
+
+// One block of >= N_r threads (<= 1024).  Thread e owns expert e.
+__global__ void __launch_bounds__(1024) chunk_scan_kernel(const int32_t* __restrict__ chunk_hist,
+                                                          int nch, int N_r,
+                                                          int32_t* __restrict__ chunk_base,
+                                                          int32_t* __restrict__ offsets) {
+  __shared__ int warp_sums[32];
+  const int e = threadIdx.x;
+  const int lane = e & 31, warp = e >> 5;
+  int total = 0;
+  if (e < N_r)
+    for (int c = 0; c < nch; ++c) total += chunk_hist[(size_t)c * N_r + e];
+  // block-wide exclusive scan of `total`
+  int incl = total;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = (blockDim.x + 31) >> 5;
+    int w = lane < nw ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, w, off);
+      if (lane >= off) w += v;
+    }
+    if (lane < nw) warp_sums[lane] = w;  // inclusive over warps
+  }
+  __syncthreads();
+  const int excl = incl - total + (warp > 0 ? warp_sums[warp - 1] : 0);
+  if (e < N_r) {
+    offsets[e] = excl;
+    if (e == N_r - 1) offsets[N_r] = excl + total;
+    int run = excl;
+    for (int c = 0; c < nch; ++c) {
+      chunk_base[(size_t)c * N_r + e] = run;
+      run += chunk_hist[(size_t)c * N_r + e];
+    }
+  }
+}
+
+// Stable rank: pair (t, k) with expert e lands on
+//   chunk_base[c][e] + #(earlier warps of the chunk routed to e)
+//                    + #(earlier lanes of this warp routed to e).
+// A token never holds the same expert twice, so ordering by token is total.
+__global__ void __launch_bounds__(kChunk) chunk_rank_kernel(const int32_t* __restrict__ idx, int T,
+                                                            int N_r, int K,
+                                                            const int32_t* __restrict__ chunk_base,
+                                                            int32_t* __restrict__ perm_src,
+                                                            int32_t* __restrict__ inv_row) {
+  extern __shared__ int sm[];
+  int* whist = sm;                          // [kChunk/32][N_r]
+  int* ids = sm + (kChunk / 32) * N_r;      // [kChunk][K]
+  const int c = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int t = c * kChunk + threadIdx.x;
+  for (int i = threadIdx.x; i < (kChunk / 32) * N_r; i += blockDim.x) whist[i] = 0;
+  for (int k = 0; k < K; ++k) ids[threadIdx.x * K + k] = t < T ? idx[(size_t)t * K + k] : -1;
+  __syncthreads();
+  if (t < T)
+    for (int k = 0; k < K; ++k) atomicAdd(&whist[warp * N_r + ids[threadIdx.x * K + k]], 1);
+  __syncthreads();
+  if (t < T) {
+    for (int k = 0; k < K; ++k) {
+      const int e = ids[threadIdx.x * K + k];
+      int r = chunk_base[(size_t)c * N_r + e];
+      for (int w = 0; w < warp; ++w) r += whist[w * N_r + e];
+      const int* base = ids + (warp * 32) * K;
+      for (int l = 0; l < lane; ++l)
+        for (int kk = 0; kk < K; ++kk) r += (base[l * K + kk] == e);
+      perm_src[r] = t;
+      inv_row[(size_t)t * K + k] = r;
+    }
+  }
+}
+
+// One warp per token: each 16-byte vector of the row is loaded once and
+// stored to the token's K grouped rows.
+__global__ void __launch_bounds__(256) scatter_rows_kernel(const uint4* __restrict__ u,
+                                                           const float* __restrict__ u_scale,
+                                                           const int32_t* __restrict__ inv_row,
+                                                           int T, int nvec, int nscale, int K,
+                                                           uint4* __restrict__ x_perm,
+                                                           float* __restrict__ x_scale) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  int rows[16];  // K <= 16 on this path; larger K takes the generic loop below
+  const int Kc = K < 16 ? K : 16;
+#pragma unroll
+  for (int k = 0; k < 16; ++k)
+    if (k < Kc) rows[k] = inv_row[(size_t)t * K + k];
+  const uint4* src = u + (size_t)t * nvec;
+  int c = lane;
+  for (; c + 96 < nvec; c += 128) {
+    const uint4 v0 = src[c], v1 = src[c + 32], v2 = src[c + 64], v3 = src[c + 96];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      if (k < Kc) {
+        uint4* dst = x_perm + (size_t)rows[k] * nvec;
+        dst[c] = v0; dst[c + 32] = v1; dst[c + 64] = v2; dst[c + 96] = v3;
+      }
+    }
+  }
+  for (; c < nvec; c += 32) {
+    const uint4 v = src[c];
+#pragma unroll
+    for (int k = 0; k < 16; ++k)
+      if (k < Kc) x_perm[(size_t)rows[k] * nvec + c] = v;
+  }
+  for (int k = 16; k < K; ++k) {
+    const int r = inv_row[(size_t)t * K + k];
+    for (int cc = lane; cc < nvec; cc += 32) x_perm[(size_t)r * nvec + cc] = src[cc];
+  }
+  if (u_scale) {
+    for (int k = 0; k < K; ++k) {
+      const int r = inv_row[(size_t)t * K + k];
+      for (int j = lane; j < nscale; j += 32)
+        x_scale[(size_t)r * nscale + j] = u_scale[(size_t)t * nscale + j];
+    }
+  }
+}
+
+moe_status launch_permute(const void* u, const float* u_scale, int elem_bytes, const int32_t* idx,
+                          int T, int d, int N_r, int K, void* x_perm, float* x_scale,
+                          int32_t* offsets, int32_t* perm_src, int32_t* inv_row, void* ws,
+                          cudaStream_t s) {
+  const int nch = n_chunks(T);
+  int32_t* chunk_hist = static_cast<int32_t*>(ws);
+  int32_t* chunk_base =
+      chunk_hist + align_up((size_t)nch * N_r * sizeof(int32_t), 256) / sizeof(int32_t);
+  chunk_hist_kernel<<<nch, kChunk, N_r * sizeof(int), s>>>(idx, T, N_r, K, chunk_hist);
+  const int scan_threads = (N_r + 31) / 32 * 32;
+  chunk_scan_kernel<<<1, scan_threads, 0, s>>>(chunk_hist, nch, N_r, chunk_base, offsets);
+  const size_t rank_smem = ((size_t)(kChunk / 32) * N_r + (size_t)kChunk * K) * sizeof(int);
+  if (rank_smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(chunk_rank_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)rank_smem);
+    if (e != cudaSuccess) return cuda_check(e, "chunk_rank_kernel smem attribute");
+  }
+  chunk_rank_kernel<<<nch, kChunk, rank_smem, s>>>(idx, T, N_r, K, chunk_base, perm_src, inv_row);
+  const int nvec = (int)((size_t)d * elem_bytes / 16);
+  const int wpb = 8;
+  scatter_rows_kernel<<<(T + wpb - 1) / wpb, wpb * 32, 0, s>>>(
+      static_cast<const uint4*>(u), u_scale, inv_row, T, nvec, u_scale ? d / 128 : 0, K,
+      static_cast<uint4*>(x_perm), x_scale);
+  return cuda_check(cudaGetLastError(), "permute launches");
+}
+
+}  // namespace moe

@@ -1,0 +1,121 @@
+// FP8 quantisers of the fine-grained recipe in "DeepSeek-V3 技術報告",
+// section 核心概念 (FP8 bullet): E4M3 values with one float32 scale per 1x128
+// activation tile or per 128x128 weight block.
+//   scale = amax / 448 (1 for an all-zero tile)
+//   q     = E4M3 round-to-nearest-even, saturated to +-448, of x / scale
+// x / scale is an IEEE float32 division so the code of every element is a
+// function of the stored inputs alone.
+#include "launch.h"
+
+namespace moe {
+
+namespace {
+
+__device__ __forceinline__ float tile_scale(float amax) {
+  return amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
+}
+
+__device__ __forceinline__ uint8_t to_e4m3(float v) {
+  return static_cast<uint8_t>(__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3));
+}
+
+// One warp per (row, 128-column tile); lane j holds columns 4j..4j+3.
+__global__ void __launch_bounds__(256) quant_1x128_kernel(const __nv_bfloat16* __restrict__ x,
+                                                          int rows, int cols,
+                                                          uint8_t* __restrict__ q,
+                                                          float* __restrict__ scale) {
+  const int lane = threadIdx.x & 31;
+  const int tiles_per_row = cols / 128;
+  const long long tile = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (tile >= (long long)rows * tiles_per_row) return;
+  const long long r = tile / tiles_per_row;
+  const int tb = (int)(tile % tiles_per_row);
+  const size_t base = (size_t)r * cols + tb * 128 + lane * 4;
+  const uint2 raw = *reinterpret_cast<const uint2*>(x + base);
+  float v[4];
+  v[0] = __uint_as_float(raw.x << 16);
+  v[1] = __uint_as_float(raw.x & 0xffff0000u);
+  v[2] = __uint_as_float(raw.y << 16);
+  v[3] = __uint_as_float(raw.y & 0xffff0000u);
+  float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  const float sc = tile_scale(amax);
+  uint32_t packed = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) packed |= (uint32_t)to_e4m3(__fdiv_rn(v[i], sc)) << (8 * i);
+  *reinterpret_cast<uint32_t*>(q + base) = packed;
+  if (lane == 0) scale[(size_t)r * tiles_per_row + tb] = sc;
+}
+
+// One 256-thread block per 128x128 block of one group.
+__global__ void __launch_bounds__(256) quant_128x128_kernel(const __nv_bfloat16* __restrict__ w,
+                                                            int rows, int cols,
+                                                            uint8_t* __restrict__ q,
+                                                            float* __restrict__ scale) {
+  __shared__ float red[8];
+  const int cb = blockIdx.x, rb = blockIdx.y, g = blockIdx.z;
+  const int nrb = rows / 128, ncb = cols / 128;
+  const __nv_bfloat16* src = w + ((size_t)g * rows + (size_t)rb * 128) * cols + (size_t)cb * 128;
+  uint8_t* dst = q + ((size_t)g * rows + (size_t)rb * 128) * cols + (size_t)cb * 128;
+  // thread -> (row = tid/16 + 16*i, 8 columns at (tid%16)*8), i = 0..7
+  const int c8 = (threadIdx.x & 15) * 8;
+  const int r0 = threadIdx.x >> 4;
+  float v[8][8];
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint4 raw = *reinterpret_cast<const uint4*>(src + (size_t)(r0 + 16 * i) * cols + c8);
+    const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[i][2 * j] = __uint_as_float(wv[j] << 16);
+      v[i][2 * j + 1] = __uint_as_float(wv[j] & 0xffff0000u);
+      amax = fmaxf(amax, fmaxf(fabsf(v[i][2 * j]), fabsf(v[i][2 * j + 1])));
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  amax = red[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) amax = fmaxf(amax, red[i]);
+  const float sc = tile_scale(amax);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    uint32_t lo = 0, hi = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      lo |= (uint32_t)to_e4m3(__fdiv_rn(v[i][j], sc)) << (8 * j);
+      hi |= (uint32_t)to_e4m3(__fdiv_rn(v[i][4 + j], sc)) << (8 * j);
+    }
+    *reinterpret_cast<uint2*>(dst + (size_t)(r0 + 16 * i) * cols + c8) = make_uint2(lo, hi);
+  }
+  if (threadIdx.x == 0) scale[((size_t)g * nrb + rb) * ncb + cb] = sc;
+}
+
+}  // namespace
+
+moe_status launch_quant_1x128(const void* x, int rows, int cols, uint8_t* q, float* scale,
+                              cudaStream_t s) {
+  const long long tiles = (long long)rows * (cols / 128);
+  const int wpb = 8;
+  const long long blocks = (tiles + wpb - 1) / wpb;
+  if (blocks > 0x7fffffffLL) return fail(MOE_ERR_UNSUPPORTED, "quantize_1x128: too many tiles");
+  quant_1x128_kernel<<<(unsigned)blocks, wpb * 32, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(x), rows, cols, q, scale);
+  return cuda_check(cudaGetLastError(), "quant_1x128 launch");
+}
+
+moe_status launch_quant_128x128(const void* w, int groups, int rows, int cols, uint8_t* q,
+                                float* scale, cudaStream_t s) {
+  if (groups > 65535 || rows / 128 > 65535)
+    return fail(MOE_ERR_UNSUPPORTED, "quantize_128x128: grid too large");
+  dim3 grid(cols / 128, rows / 128, groups);
+  quant_128x128_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(w), rows, cols, q,
+                                            scale);
+  return cuda_check(cudaGetLastError(), "quant_128x128 launch");
+}
+
+}  // namespace moe

@@ -1,0 +1,139 @@
+"""The DeepSeekMoE layer step built from the C-ABI calls.
+
+MoELayer owns the layer's device state (centroids, bias, expert weights,
+FP8 copies of them) and the per-step buffers, and runs one step as
+    moe_route -> [moe_quantize_1x128] -> moe_permute -> moe_expert_ffn (routed)
+    -> moe_expert_ffn (each shared expert) -> moe_combine [-> moe_bias_update]
+on one CUDA stream.  Every step of the layer runs in libmoe's kernels; this
+module only allocates buffers and sequences calls.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import (MOE_BF16, MOE_E4M3, MOE_F32, moe_bias_update, moe_combine, moe_expert_down,
+               moe_expert_ffn, moe_expert_ffn_workspace_size, moe_expert_gate_up, moe_permute, moe_permute_workspace_size,
+               moe_quantize_128x128, moe_quantize_1x128, moe_route, moe_route_workspace_size)
+from .configs import LayerConfig
+
+GAMMA = 0.001
+
+
+def _ws(nbytes, device):
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+class MoELayer:
+    def __init__(self, cfg: LayerConfig, weights: dict, T_max: int | None = None, device="cuda"):
+        self.cfg = cfg
+        self.device = torch.device(device)
+        self.T_max = cfg.T if T_max is None else T_max
+        self.E = weights["E"]
+        self.b = weights["b"].clone()
+        self.fp8 = cfg.dtype == "e4m3"
+        if self.fp8:
+            self.W = {k: self._quantise(weights[k]) for k in
+                      ("W_gate_up", "W_down", "Ws_gate_up", "Ws_down")}
+        else:
+            self.W = {k: (weights[k], None) for k in ("W_gate_up", "W_down", "Ws_gate_up", "Ws_down")}
+        self._alloc(self.T_max)
+
+    # -- setup ---------------------------------------------------------------
+    def _quantise(self, w):
+        G, R, C = w.shape
+        q = torch.empty(G, R, C, dtype=torch.uint8, device=self.device)
+        s = torch.empty(G, R // 128, C // 128, dtype=torch.float32, device=self.device)
+        moe_quantize_128x128(w, q, s)
+        return q, s
+
+    def _alloc(self, T):
+        c, dev = self.cfg, self.device
+        d, K, N_r, N_s = c.d, c.K, c.N_r, c.N_s
+        R = T * K
+        act = torch.float32 if c.dtype == "f32" else torch.bfloat16
+        xdt = torch.uint8 if self.fp8 else act
+        ffn_dt = {"f32": MOE_F32, "bf16": MOE_BF16, "e4m3": MOE_E4M3}[c.dtype]
+        self.topk_idx = torch.empty(T, K, dtype=torch.int32, device=dev)
+        self.topk_gate = torch.empty(T, K, dtype=torch.float32, device=dev)
+        self.counts = torch.zeros(N_r, dtype=torch.int32, device=dev)
+        self.route_ws = _ws(moe_route_workspace_size(T, N_r), dev)
+        self.perm_ws = _ws(moe_permute_workspace_size(T, N_r), dev)
+        self.x_perm = torch.empty(R, d, dtype=xdt, device=dev)
+        self.offsets = torch.zeros(N_r + 1, dtype=torch.int32, device=dev)
+        self.perm_src = torch.empty(R, dtype=torch.int32, device=dev)
+        self.inv_row = torch.empty(T, K, dtype=torch.int32, device=dev)
+        self.y_perm = torch.empty(R, d, dtype=act, device=dev)
+        self.y_shared = torch.empty(N_s, T, d, dtype=act, device=dev)
+        self.ffn_ws = _ws(moe_expert_ffn_workspace_size(ffn_dt, T, c.I), dev)
+        hdt = torch.uint8 if self.fp8 else act
+        self.h_mid = torch.empty(R, c.I, dtype=hdt, device=dev)
+        self.h_scale = torch.empty(R, c.I // 128, dtype=torch.float32, device=dev) if self.fp8 \
+            else None
+        self.h_out = torch.empty(T, d, dtype=act, device=dev)
+        self.shared_offsets = torch.tensor([0, T], dtype=torch.int32, device=dev)
+        if self.fp8:
+            self.u_q = torch.empty(T, d, dtype=torch.uint8, device=dev)
+            self.u_s = torch.empty(T, d // 128, dtype=torch.float32, device=dev)
+            self.x_scale = torch.empty(R, d // 128, dtype=torch.float32, device=dev)
+        self.T_alloc = T
+
+    # -- one step ------------------------------------------------------------
+    def forward(self, u: torch.Tensor, stream=None, gate_up_events=None) -> torch.Tensor:
+        """h' for the T tokens of u; returns h_out (overwritten by the next call).
+        gate_up_events=(start, end) records CUDA events around the routed
+        gate/up GEMM launch on the same stream."""
+        c = self.cfg
+        T = u.shape[0]
+        if T != self.T_alloc:
+            self._alloc(T)
+        moe_route(u, self.E, self.b, c.K, self.topk_idx, self.topk_gate, self.counts,
+                  self.route_ws, stream)
+        if self.fp8:
+            moe_quantize_1x128(u, self.u_q, self.u_s, stream)
+            moe_permute(self.u_q, self.topk_idx, c.N_r, self.x_perm, self.offsets, self.perm_src,
+                        self.inv_row, self.perm_ws, u_scale=self.u_s, x_scale=self.x_scale,
+                        stream=stream)
+            x_sh, xs_sh = self.u_q, self.u_s
+        else:
+            moe_permute(u, self.topk_idx, c.N_r, self.x_perm, self.offsets, self.perm_src,
+                        self.inv_row, self.perm_ws, stream=stream)
+            x_sh, xs_sh = u, None
+        (wgu, sgu), (wdn, sdn) = self.W["W_gate_up"], self.W["W_down"]
+        st = torch.cuda.current_stream() if stream is None else stream
+        if gate_up_events:
+            gate_up_events[0].record(st)
+        moe_expert_gate_up(self.x_perm, self.offsets, wgu, self.h_mid,
+                           x_scale=self.x_scale if self.fp8 else None, w_scale_gate_up=sgu,
+                           h_scale=self.h_scale, stream=stream)
+        if gate_up_events:
+            gate_up_events[1].record(st)
+        moe_expert_down(self.h_mid, self.offsets, wdn, self.y_perm, h_scale=self.h_scale,
+                        w_scale_down=sdn, stream=stream)
+        (wsgu, ssgu), (wsdn, ssdn) = self.W["Ws_gate_up"], self.W["Ws_down"]
+        for j in range(c.N_s):
+            moe_expert_ffn(x_sh, self.shared_offsets, wsgu[j:j + 1], wsdn[j:j + 1],
+                           self.y_shared[j], self.ffn_ws, x_scale=xs_sh,
+                           w_scale_gate_up=None if ssgu is None else ssgu[j:j + 1],
+                           w_scale_down=None if ssdn is None else ssdn[j:j + 1], stream=stream)
+        u_res = u
+        moe_combine(u_res, self.y_shared if c.N_s else None, self.y_perm, self.inv_row,
+                    self.topk_gate, self.h_out, stream)
+        return self.h_out
+
+    def bias_update(self, counts=None, T_total=None, stream=None):
+        """b <- b -/+ gamma from the load of the last step (or from the given
+        global counts / token total of data-parallel replicas)."""
+        counts = self.counts if counts is None else counts
+        T_total = self.T_alloc if T_total is None else T_total
+        moe_bias_update(self.b, counts, T_total, self.cfg.K, GAMMA, stream)
+
+    def step(self, u, stream=None, process_group=None):
+        """One training-style step: forward, global load, bias update."""
+        h = self.forward(u, stream)
+        if process_group is not None:
+            from .parallel_load import allreduce_load
+            counts, T_total = allreduce_load(self.counts, u.shape[0], process_group)
+            self.bias_update(counts, T_total, stream)
+        else:
+            self.bias_update(stream=stream)
+        return h

@@ -1,0 +1,127 @@
+"""The C-ABI library builds, loads and exports every entry point of
+include/moe.h; argument checks answer with a status before any CUDA work.
+No GPU is needed: only calls that fail validation are made."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import mixture_experts_layer_60_b200 as moe
+from mixture_experts_layer_60_b200 import build as moe_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    moe_build.build()
+    return moe.lib()
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_\w+)\s*\(", text)))
+
+
+def test_header_symbols_exported(L):
+    names = header_functions()
+    assert len(names) >= 14
+    raw = ctypes.CDLL(moe.LIB_PATH)
+    for n in names:
+        assert hasattr(raw, n), f"{n} declared in moe.h but not exported"
+        assert n in moe.SYMBOLS, f"{n} has no binding"
+
+
+def test_binding_names_match_header():
+    assert set(moe.SYMBOLS) == set(header_functions())
+
+
+def test_abi_version_and_status_strings(L):
+    assert L.moe_abi_version() == 1
+    assert L.moe_status_string(0) == b"MOE_OK"
+    assert L.moe_status_string(3) == b"MOE_ERR_WORKSPACE"
+
+
+def test_workspace_sizes(L):
+    assert L.moe_route_workspace_size(8192, 256) == 8192 * 256 * 4
+    assert L.moe_route_workspace_size(0, 256) == 0
+    assert L.moe_permute_workspace_size(8192, 256) >= 2 * 32 * 256 * 4
+    assert L.moe_expert_ffn_workspace_size(1, 65536, 2048) == 65536 * 2048 * 2
+    assert L.moe_expert_ffn_workspace_size(0, 100, 128) >= 100 * 128 * 4
+    fp8 = L.moe_expert_ffn_workspace_size(2, 1000, 256)
+    assert fp8 >= 1000 * 256 + 1000 * 2 * 4
+
+
+def _last(L):
+    return L.moe_last_error().decode()
+
+
+def test_route_argument_errors(L):
+    dummy = ctypes.c_void_p(256)  # never dereferenced: validation fails first
+    assert L.moe_route(dummy, dummy, 2, dummy, 8, 64, 16, 4, dummy, dummy, dummy, dummy, 4096,
+                       None) == 2
+    assert "dtype" in _last(L)
+    assert L.moe_route(dummy, dummy, 1, dummy, 8, 64, 16, 17, dummy, dummy, dummy, dummy, 4096,
+                       None) == 2
+    assert L.moe_route(dummy, dummy, 1, dummy, 8, 64, 2000, 4, dummy, dummy, dummy, dummy, 1 << 20,
+                       None) == 2
+    assert L.moe_route(dummy, dummy, 1, dummy, 8, 96, 16, 4, dummy, dummy, dummy, dummy, 4096,
+                       None) == 2
+    assert L.moe_route(dummy, None, 1, dummy, 8, 64, 16, 4, dummy, dummy, dummy, dummy, 4096,
+                       None) == 1
+    assert L.moe_route(dummy, dummy, 1, dummy, -1, 64, 16, 4, dummy, dummy, dummy, dummy, 4096,
+                       None) == 1
+    assert L.moe_route(dummy, dummy, 1, dummy, 8, 64, 16, 4, dummy, dummy, dummy, dummy, 16,
+                       None) == 3
+    assert "workspace" in _last(L)
+
+
+def test_permute_argument_errors(L):
+    d = ctypes.c_void_p(256)
+    assert L.moe_permute(d, None, 7, d, 8, 64, 16, 4, d, None, d, d, d, d, 1 << 20, None) == 2
+    assert L.moe_permute(d, None, 2, d, 8, 64, 16, 4, d, None, d, d, d, d, 1 << 20, None) == 2
+    assert L.moe_permute(d, None, 1, d, 8, 64, 16, 4, d, None, None, d, d, d, 1 << 20, None) == 1
+    assert L.moe_permute(d, d, 1, d, 8, 64, 16, 4, d, None, d, d, d, d, 1 << 20, None) == 1
+    assert L.moe_permute(d, None, 1, d, 8, 64, 16, 4, d, None, d, d, d, d, 8, None) == 3
+    assert L.moe_permute(d, None, 1, d, 8, 4, 16, 4, d, None, d, d, d, d, 1 << 20, None) == 2
+
+
+def test_expert_ffn_argument_errors(L):
+    d = ctypes.c_void_p(256)
+    assert L.moe_expert_ffn(d, None, d, 4, 100, 192, 128, 1, d, None, d, None, d, d, 1 << 30,
+                            None) == 2
+    assert L.moe_expert_ffn(d, None, d, 4, 100, 256, 100, 1, d, None, d, None, d, d, 1 << 30,
+                            None) == 2
+    assert L.moe_expert_ffn(d, None, d, 2000, 100, 256, 128, 1, d, None, d, None, d, d, 1 << 30,
+                            None) == 2
+    assert L.moe_expert_ffn(d, None, d, 4, 100, 256, 128, 2, d, None, d, None, d, d, 1 << 30,
+                            None) == 1
+    assert L.moe_expert_ffn(d, d, d, 4, 100, 256, 128, 1, d, None, d, None, d, d, 1 << 30,
+                            None) == 1
+    assert L.moe_expert_ffn(d, None, d, 4, 100, 256, 128, 1, d, None, d, None, d, d, 64,
+                            None) == 3
+    assert L.moe_expert_ffn(d, None, None, 4, 100, 256, 128, 1, d, None, d, None, d, d, 1 << 30,
+                            None) == 1
+
+
+def test_combine_bias_quant_argument_errors(L):
+    d = ctypes.c_void_p(256)
+    assert L.moe_combine(d, d, 1, d, d, d, 2, 8, 64, 4, d, None) == 2
+    assert L.moe_combine(d, None, 1, d, d, d, 1, 8, 64, 4, d, None) == 1
+    assert L.moe_combine(d, d, 1, d, d, d, 1, 8, 4, 4, d, None) == 2
+    assert L.moe_bias_update(None, d, 16, 8, 4, ctypes.c_float(0.001), None) == 1
+    assert L.moe_bias_update(d, d, 0, 8, 4, ctypes.c_float(0.001), None) == 1
+    assert L.moe_quantize_1x128(d, 4, 100, d, d, None) == 2
+    assert L.moe_quantize_1x128(None, 4, 128, d, d, None) == 1
+    assert L.moe_quantize_128x128(d, 1, 100, 128, d, d, None) == 2
+    assert L.moe_device_status(None) == 1
+
+
+def test_product_path_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(moe, "_LIB", None)
+    monkeypatch.setattr(moe, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        moe.lib()

@@ -1,0 +1,264 @@
+"""Per-call parity of libmoe's kernels against the CPU oracle, through the
+C ABI, at sizes that span several tiles with ragged tails, plus edge cases.
+Integer and index outputs must match bit for bit; floating-point outputs
+within the tolerances of tests/harness.py."""
+import numpy as np
+import pytest
+import torch
+
+import mixture_experts_layer_60_b200 as moe
+from oracle import moe_oracle as O
+from tests.harness import TOL, LazyExperts, assert_close, check_routing, f64
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _gen(seed):
+    g = torch.Generator(device=DEV)
+    g.manual_seed(seed)
+    return g
+
+
+def _randn(shape, g, std=1.0, dtype=torch.bfloat16):
+    return (torch.randn(*shape, generator=g, device=DEV) * std).to(dtype)
+
+
+def _ws(n):
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=DEV)
+
+
+def _route(u, E, b, K):
+    T, N_r = u.shape[0], E.shape[0]
+    idx = torch.empty(T, K, dtype=torch.int32, device=DEV)
+    gate = torch.empty(T, K, dtype=torch.float32, device=DEV)
+    counts = torch.full((N_r,), -7, dtype=torch.int32, device=DEV)
+    moe.moe_route(u, E, b, K, idx, gate, counts, _ws(moe.moe_route_workspace_size(T, N_r)))
+    torch.cuda.synchronize()
+    return idx, gate, counts
+
+
+# ------------------------------------------------------------------ router
+
+@pytest.mark.parametrize("T,d,N_r,K,dt", [
+    (1000, 512, 64, 6, torch.bfloat16),     # tensor-core logits, BN = 64
+    (517, 1024, 256, 8, torch.bfloat16),    # BN = 256, ragged last tile
+    (300, 256, 128, 8, torch.bfloat16),     # BN = 128
+    (333, 256, 16, 4, torch.float32),       # CUDA-core logits
+    (257, 192, 32, 3, torch.float32),
+    (200, 128, 16, 4, torch.bfloat16),      # N_r not a multiple of 64 -> CUDA-core logits
+    (64, 128, 64, 1, torch.bfloat16),       # K = 1
+    (50, 128, 64, 64, torch.bfloat16),      # K = N_r
+    (1, 128, 64, 6, torch.bfloat16),        # one token
+])
+def test_route_matches_oracle(T, d, N_r, K, dt):
+    g = _gen(T * 31 + d)
+    u = _randn((T, d), g, 1.0, dt)
+    E = _randn((N_r, d), g, d ** -0.5, dt)
+    b = ((torch.rand(N_r, generator=g, device=DEV) * 2 - 1) * 0.01).float()
+    idx, gate, counts = _route(u, E, b, K)
+    ref = O.route(f64(u), f64(E), b.cpu().numpy(), K)
+    check_routing(idx.cpu().numpy(), gate.cpu().numpy(), counts.cpu().numpy(), ref, K)
+    np.testing.assert_allclose(gate.double().sum(1).cpu().numpy(), 1.0, atol=4e-7)
+
+
+def test_route_zero_centroids_gates_are_uniform():
+    """E = 0: s = 1/2 everywhere, selection follows b, gates are exactly 1/K."""
+    T, d, N_r, K = 100, 256, 64, 4
+    u = _randn((T, d), _gen(1))
+    E = torch.zeros(N_r, d, dtype=torch.bfloat16, device=DEV)
+    b = torch.linspace(-0.01, 0.01, N_r, device=DEV).flip(0).contiguous()
+    idx, gate, counts = _route(u, E, b, K)
+    assert (idx.cpu() == torch.arange(K, dtype=torch.int32)).all()
+    assert (gate.cpu() == 0.25).all()
+    assert counts[:K].tolist() == [T] * K and int(counts[K:].sum()) == 0
+
+
+def test_route_empty_batch():
+    N_r = 64
+    E = _randn((N_r, 128), _gen(2))
+    b = torch.zeros(N_r, device=DEV)
+    u = torch.empty(0, 128, dtype=torch.bfloat16, device=DEV)
+    idx, gate, counts = _route(u, E, b, 4)
+    assert int(counts.abs().sum()) == 0
+
+
+# ------------------------------------------------------------------ permute
+
+def _rand_idx(T, N_r, K, seed, skew=False):
+    rng = np.random.default_rng(seed)
+    p = None
+    if skew:
+        p = 1.0 / np.arange(1, N_r + 1) ** 1.2
+        p[N_r // 2: N_r // 2 + 3] = 0           # a few experts never chosen
+        p /= p.sum()
+    return np.stack([rng.choice(N_r, K, replace=False, p=p) for _ in range(T)]).astype(np.int32)
+
+
+@pytest.mark.parametrize("T,d,N_r,K,dtype", [
+    (1000, 256, 64, 6, torch.bfloat16),
+    (777, 512, 256, 8, torch.bfloat16),
+    (300, 128, 16, 4, torch.float32),
+    (513, 256, 32, 2, torch.uint8),           # FP8 rows + tile scales
+    (40, 128, 64, 17, torch.bfloat16),        # K > 16 path
+])
+def test_permute_bit_exact(T, d, N_r, K, dtype):
+    idx_np = _rand_idx(T, N_r, K, T + K, skew=True)
+    g = _gen(T)
+    if dtype == torch.uint8:
+        u = torch.randint(0, 255, (T, d), generator=g, device=DEV, dtype=torch.uint8)
+        u_scale = torch.rand(T, d // 128, generator=g, device=DEV)
+        x_scale = torch.empty(T * K, d // 128, device=DEV)
+    else:
+        u = _randn((T, d), g, 1.0, dtype)
+        u_scale = x_scale = None
+    idx = torch.from_numpy(idx_np).to(DEV)
+    x_perm = torch.empty(T * K, d, dtype=dtype, device=DEV)
+    offsets = torch.empty(N_r + 1, dtype=torch.int32, device=DEV)
+    perm_src = torch.empty(T * K, dtype=torch.int32, device=DEV)
+    inv_row = torch.empty(T, K, dtype=torch.int32, device=DEV)
+    ws = _ws(moe.moe_permute_workspace_size(T, N_r))
+    moe.moe_permute(u, idx, N_r, x_perm, offsets, perm_src, inv_row, ws, u_scale=u_scale,
+                    x_scale=x_scale)
+    torch.cuda.synchronize()
+    r_off, r_src, r_inv = O.permute_indices(idx_np, N_r)
+    np.testing.assert_array_equal(offsets.cpu().numpy(), r_off)
+    np.testing.assert_array_equal(perm_src.cpu().numpy(), r_src)
+    np.testing.assert_array_equal(inv_row.cpu().numpy(), r_inv)
+    src = torch.from_numpy(r_src.astype(np.int64)).to(DEV)
+    assert torch.equal(x_perm, u[src])
+    if x_scale is not None:
+        assert torch.equal(x_scale, u_scale[src])
+
+
+def test_permute_empty_batch():
+    N_r = 32
+    offsets = torch.full((N_r + 1,), 5, dtype=torch.int32, device=DEV)
+    z = torch.empty(0, 8, dtype=torch.int32, device=DEV)
+    u = torch.empty(0, 128, dtype=torch.bfloat16, device=DEV)
+    moe.moe_permute(u, z, N_r, torch.empty(0, 128, dtype=torch.bfloat16, device=DEV), offsets,
+                    torch.empty(0, dtype=torch.int32, device=DEV), z.clone(), _ws(256))
+    torch.cuda.synchronize()
+    assert int(offsets.abs().sum()) == 0
+
+
+# ------------------------------------------------------------------ expert FFN
+
+def _groups(sizes):
+    off = np.zeros(len(sizes) + 1, np.int32)
+    off[1:] = np.cumsum(sizes)
+    return off
+
+
+def _ffn_case(sizes, d, I, dtype, seed, extra_rows=0):
+    g = _gen(seed)
+    G = len(sizes)
+    off = _groups(sizes)
+    rows = int(off[-1]) + extra_rows
+    x = _randn((rows, d), g, 1.0, dtype)
+    wgu = _randn((G, 2 * I, d), g, d ** -0.5, dtype)
+    wdn = _randn((G, d, I), g, I ** -0.5, dtype)
+    y = torch.full((rows, d), float("nan"), dtype=dtype, device=DEV)
+    dt = moe.MOE_F32 if dtype == torch.float32 else moe.MOE_BF16
+    ws = _ws(moe.moe_expert_ffn_workspace_size(dt, rows, I))
+    offsets = torch.from_numpy(off).to(DEV)
+    moe.moe_expert_ffn(x, offsets, wgu, wdn, y, ws)
+    torch.cuda.synchronize()
+    ex = LazyExperts(wgu, wdn)
+    xs = f64(x)
+    ref = np.zeros((int(off[-1]), d))
+    for e in range(G):
+        a, b_ = int(off[e]), int(off[e + 1])
+        if b_ > a:
+            ref[a:b_] = O.swiglu_ffn(xs[a:b_], *ex[e])
+    got = f64(y)
+    return got, ref, int(off[-1])
+
+
+@pytest.mark.parametrize("sizes,d,I", [
+    ([0, 1, 127, 128, 129, 300, 0, 5], 256, 256),   # ragged groups, empty groups
+    ([64, 200, 333], 512, 384),                     # I not a multiple of 256
+    ([1000, 700, 1300, 60], 1024, 512),             # many tiles per CTA, stage wrap-around
+    ([5000], 768, 256),                             # one large group (the shared-expert shape)
+])
+def test_expert_ffn_bf16(sizes, d, I):
+    got, ref, n = _ffn_case(sizes, d, I, torch.bfloat16, sum(sizes) + d, extra_rows=3)
+    assert_close(got[:n], ref, TOL["bf16"], "y")
+    assert np.isnan(got[n:]).all(), "rows outside every group were written"
+    assert moe.moe_device_status() == 0
+
+
+@pytest.mark.parametrize("sizes,d,I", [([3, 0, 64, 65, 130], 256, 128), ([200], 128, 256)])
+def test_expert_ffn_f32(sizes, d, I):
+    got, ref, n = _ffn_case(sizes, d, I, torch.float32, 7 + d)
+    assert_close(got[:n], ref, TOL["f32"], "y")
+
+
+# ------------------------------------------------------------------ combine, bias
+
+@pytest.mark.parametrize("T,d,K,N_s,dtype", [
+    (1000, 512, 6, 2, torch.bfloat16), (333, 256, 8, 1, torch.bfloat16),
+    (200, 128, 4, 0, torch.float32), (64, 256, 17, 1, torch.bfloat16),
+])
+def test_combine(T, d, K, N_s, dtype):
+    g = _gen(T + K)
+    u = _randn((T, d), g, 1.0, dtype)
+    ys = _randn((N_s, T, d), g, 0.5, dtype) if N_s else None
+    yp = _randn((T * K, d), g, 0.5, dtype)
+    perm = torch.randperm(T * K, generator=torch.Generator().manual_seed(T))
+    inv = perm.view(T, K).to(torch.int32).to(DEV)
+    gate = torch.rand(T, K, generator=g, device=DEV)
+    gate = (gate / gate.sum(1, keepdim=True)).contiguous()
+    out = torch.empty(T, d, dtype=dtype, device=DEV)
+    moe.moe_combine(u, ys, yp, inv, gate, out)
+    torch.cuda.synchronize()
+    ref = f64(u) + (f64(ys).sum(0) if N_s else 0)
+    ref = ref + np.einsum("tk,tkd->td", f64(gate), f64(yp)[inv.long().cpu().numpy()])
+    tol = TOL["f32"] if dtype == torch.float32 else 2 ** -8
+    assert_close(f64(out), ref, tol, "h'")
+
+
+def test_bias_update_bit_exact():
+    N_r, T, K = 256, 8192, 8            # mean load 256
+    rng = np.random.default_rng(3)
+    counts = rng.integers(200, 313, N_r).astype(np.int32)
+    counts[:10] = 256                   # equal to the mean: unchanged
+    b = rng.uniform(-0.05, 0.05, N_r).astype(np.float32)
+    bd = torch.from_numpy(b).to(DEV)
+    moe.moe_bias_update(bd, torch.from_numpy(counts).to(DEV), T, K, 0.001)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(bd.cpu().numpy(), O.bias_update(b, counts, T, K))
+
+
+# ------------------------------------------------------------------ FP8 quantisers
+
+def _e4m3_values(q_u8):
+    return q_u8.cpu().view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def test_quantize_1x128_bit_exact():
+    g = _gen(5)
+    x = _randn((300, 7 * 128), g, 1.0)
+    mask = torch.rand(300, 7 * 128, generator=g, device=DEV) < 0.001
+    x = torch.where(mask, x * 50, x).to(torch.bfloat16)
+    x[7, 128:256] = 0
+    q = torch.empty(300, 896, dtype=torch.uint8, device=DEV)
+    s = torch.empty(300, 7, device=DEV)
+    moe.moe_quantize_1x128(x, q, s)
+    torch.cuda.synchronize()
+    rq, rs = O.quant_1x128(f64(x).astype(np.float32))
+    np.testing.assert_array_equal(s.cpu().numpy(), rs)
+    np.testing.assert_array_equal(_e4m3_values(q), rq)
+
+
+def test_quantize_128x128_bit_exact():
+    g = _gen(6)
+    w = _randn((3, 256, 384), g, 0.02)
+    q = torch.empty(3, 256, 384, dtype=torch.uint8, device=DEV)
+    s = torch.empty(3, 2, 3, device=DEV)
+    moe.moe_quantize_128x128(w, q, s)
+    torch.cuda.synchronize()
+    for e in range(3):
+        rq, rs = O.quant_128x128(f64(w[e]).astype(np.float32))
+        np.testing.assert_array_equal(s[e].cpu().numpy(), rs)
+        np.testing.assert_array_equal(_e4m3_values(q[e]), rq)

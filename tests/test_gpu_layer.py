@@ -1,0 +1,129 @@
+"""Whole-layer parity on the five synthetic configurations: the GPU layer
+(route -> permute -> routed and shared FFNs -> combine -> bias update, all
+through the C ABI) against the CPU oracle.  Routing is compared for every
+token; h' in full for the small shapes and on a seeded token sample for the
+V3 shapes, in the launch configuration the benchmark times."""
+import numpy as np
+import pytest
+import torch
+
+from mixture_experts_layer_60_b200.configs import CONFIGS
+from mixture_experts_layer_60_b200.layer import MoELayer
+from mixture_experts_layer_60_b200.synth import make_layer_inputs, step_u
+from oracle import moe_oracle as O
+from tests.harness import TOL, LazyExperts, assert_close, check_routing, f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _oracle_layer(cfg, w, u_rows, idx, gate):
+    routed = LazyExperts(w["W_gate_up"], w["W_down"])
+    shared = LazyExperts(w["Ws_gate_up"], w["Ws_down"])
+    if cfg.dtype == "e4m3":
+        rq = _QuantExperts(routed)
+        sq = _QuantExperts(shared)
+        return O.layer_forward_fp8(u_rows, idx, gate, rq, sq)
+    return O.layer_forward(u_rows, idx, gate, routed, shared)
+
+
+class _QuantExperts:
+    def __init__(self, ex):
+        self.ex = ex
+
+    def __len__(self):
+        return len(self.ex)
+
+    def __getitem__(self, e):
+        g, u, d = self.ex[e]
+        return O.quantise_expert(g.astype(np.float32), u.astype(np.float32), d.astype(np.float32))
+
+
+def _run(cfg, T=None, sample=None, seed_sample=0):
+    w = make_layer_inputs(cfg, "cuda", T=T)
+    u = w["u"]
+    layer = MoELayer(cfg, w, T_max=u.shape[0])
+    h = layer.forward(u)
+    torch.cuda.synchronize()
+    ref = O.route(f64(u), f64(w["E"]), w["b"].cpu().numpy(), cfg.K)
+    exempt, idx, gate = check_routing(layer.topk_idx.cpu().numpy(), layer.topk_gate.cpu().numpy(),
+                                      layer.counts.cpu().numpy(), ref, cfg.K)
+    Tn = u.shape[0]
+    rows = np.arange(Tn) if sample is None else \
+        np.sort(np.random.default_rng(seed_sample).choice(Tn, sample, replace=False))
+    want = _oracle_layer(cfg, w, f64(u)[rows], idx[rows], gate[rows])
+    got = f64(h)[rows]
+    err = assert_close(got, want, TOL[cfg.dtype], f"h' {cfg.name}")
+    return layer, w, err, exempt
+
+
+def test_layer_tiny_f32():
+    _run(CONFIGS["tiny_f32"])
+
+
+def test_layer_small_bf16():
+    _run(CONFIGS["small_bf16"])
+
+
+def test_layer_v3_bf16_sampled():
+    _run(CONFIGS["v3_bf16"], sample=48)
+
+
+def test_layer_v3_bf16_ragged_T():
+    """T not a multiple of the 128-row tile, V3 shape."""
+    _run(CONFIGS["v3_bf16"], T=1000, sample=24, seed_sample=1)
+
+
+def test_layer_all_tokens_one_expert():
+    """K = 1 and a dominant bias: one group holds every token, the others are empty."""
+    cfg = CONFIGS["small_bf16"]
+    w = make_layer_inputs(cfg, "cuda", T=600)
+    w["b"] = torch.zeros_like(w["b"])
+    w["b"][5] = 10.0
+    from dataclasses import replace
+    cfg1 = replace(cfg, K=1)
+    layer = MoELayer(cfg1, w)
+    h = layer.forward(w["u"])
+    torch.cuda.synchronize()
+    assert (layer.topk_idx.cpu() == 5).all()
+    assert (layer.topk_gate.cpu() == 1.0).all()
+    assert layer.offsets.cpu().tolist() == [0] * 6 + [600] * 59
+    idx = np.full((600, 1), 5, np.int32)
+    gate = np.ones((600, 1), np.float32)
+    want = _oracle_layer(cfg1, w, f64(w["u"]), idx, gate)
+    assert_close(f64(h), want, TOL["bf16"], "h'")
+
+
+def test_bias_update_steps_and_resume():
+    """Steps of forward + bias update: b follows the oracle's rule bit for bit
+    from the GPU's load, and a run split in two with b saved and reloaded in
+    between equals the uninterrupted run."""
+    cfg = CONFIGS["small_bf16"]
+    from dataclasses import replace
+    cfg = replace(cfg, T=512)
+    w = make_layer_inputs(cfg, "cuda", T=512)
+    a = MoELayer(cfg, w)
+    b_hist = []
+    for s in range(6):
+        u = step_u(cfg, s, "cuda", T=512)
+        b_before = a.b.cpu().numpy().copy()
+        a.step(u)
+        torch.cuda.synchronize()
+        want = O.bias_update(b_before, a.counts.cpu().numpy(), 512, cfg.K)
+        np.testing.assert_array_equal(a.b.cpu().numpy(), want)
+        b_hist.append(a.b.clone())
+    # resume: 3 steps, save b, fresh layer, 3 more
+    b1 = MoELayer(cfg, w)
+    for s in range(3):
+        b1.step(step_u(cfg, s, "cuda", T=512))
+    saved = b1.b.cpu().clone()
+    w2 = dict(w)
+    w2["b"] = saved.to("cuda")
+    b2 = MoELayer(cfg, w2)
+    for s in range(3, 6):
+        h2 = b2.step(step_u(cfg, s, "cuda", T=512))
+    torch.cuda.synchronize()
+    assert torch.equal(b2.b, b_hist[-1])
+    a_last = MoELayer(cfg, dict(w, b=b_hist[-2]))
+    h_re = a_last.forward(step_u(cfg, 5, "cuda", T=512))
+    torch.cuda.synchronize()
+    assert torch.equal(h2, h_re)
