@@ -346,10 +346,19 @@ def main():
     ap.add_argument("--cpu-tokens", type=int, default=16)
     ap.add_argument("--ref-tokens", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="scaled-down variant: tokens per rank (default: the config's T)")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="scaled-down variant: routed experts (default: the config's N_r)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     cfg = CONFIGS[args.config]
+    if args.tokens or args.experts:
+        from dataclasses import replace
+        T = args.tokens or cfg.T
+        N_r = args.experts or cfg.N_r
+        cfg = replace(cfg, name=f"{cfg.name}[T={T},N_r={N_r}]", T=T, N_r=N_r)
     ws, rank, local = dist_setup(args.gpus)
     try:
         if args.impl == "reference":

@@ -1,12 +1,428 @@
-// FP8 grouped GEMM with per-128-K promotion (placeholder until the tcgen05
-// kind::f8f6f4 kernel lands).
+// FP8 grouped GEMM with fine-grained scales and FP32 promotion every 128
+// K-elements: the FP8 recipe of "DeepSeek-V3 技術報告", section 核心概念
+// (E4M3 operands, 1x128 activation-tile scales, 128x128 weight-block scales,
+// N_c = 128), applied to the expert FFNs of the h'-equation (section 方法 / 2).
+//
+//   acc[r, n] = sum_kb  P_kb[r, n] * sa[r, kb] * sw[g, n / 128, kb]
+//   P_kb[r, n] = sum_{k in kb} qa[r, k] qw[g*b_rows + n, k]      (tensor cores)
+//
+// Each 128-wide K block is one shared-memory stage (128 bytes per row, the
+// 128-byte swizzle width).  The MMA warp writes P_kb into one of two TMEM
+// partial buffers (4 x tcgen05.mma kind::f8f6f4, K = 32 each); two epilogue
+// warpgroups read it back with tcgen05.ld, multiply by the two scales and add
+// into float32 registers, then release the buffer.  After the last block:
+//   SWIGLU   h = SiLU(acc_gate) * acc_up (float32), quantised 1x128 to E4M3
+//            with scale amax/448 (the 128 columns of a row span both
+//            warpgroups: their amax meet in shared memory)
+//   STORE    y = bf16(acc)
+// Warp roles: 0 TMA producer, 1 TMEM allocator + MMA issuer, 2-9 epilogue
+// (warpgroup 0 = warps 2-5, warpgroup 1 = warps 6-9).  Waits are bounded.
+#include <math.h>
+
 #include "launch.h"
+#include "sm100.cuh"
 
 namespace moe {
 
-moe_status launch_fp8_gemm(const void*, const float*, const void*, const float*, int,
-                           const int32_t*, int, int, int, int, bool, void*, float*, cudaStream_t) {
-  return fail(MOE_ERR_UNSUPPORTED, "moe_expert_ffn: the e4m3 path is not built yet");
+moe_status make_tmap_2d(CUtensorMap* tm, const void* base, CUtensorMapDataType dtype,
+                        int elem_bytes, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                        uint32_t box_outer);
+
+namespace {
+
+using namespace sm100;
+
+constexpr int BM = 128;
+constexpr int BN = 256;               // MMA N: SWIGLU = 128 gate + 128 up columns
+constexpr int BK = 128;               // e4m3 bytes per row = one promotion block
+constexpr int STAGES = 4;
+constexpr int kThreads = 320;
+constexpr int kMaxGroups = 1024;
+constexpr uint64_t kWaitNs = 1000000000ull;
+constexpr uint32_t TMEM_COLS = 512;   // two partial buffers of BN columns
+
+constexpr int A_BYTES = BM * BK;
+constexpr int B_BYTES = BN * BK;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int OFF_B = STAGES * A_BYTES;
+constexpr int OFF_BAR = OFF_B + STAGES * B_BYTES;
+constexpr int N_BARS = 2 * STAGES + 7;
+constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
+constexpr int OFF_AMAX = OFF_MISC + 16;                 // [2 slots][2 warpgroups][BM] float
+constexpr int OFF_TAB = OFF_AMAX + 2 * 2 * BM * 4;
+constexpr int SMEM_BYTES = OFF_TAB + 2 * (kMaxGroups + 1) * 4;
+constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
+
+struct Fp8Params {
+  const int32_t* offsets;
+  int n_groups;
+  int rows;
+  int N;                // output columns
+  int K;
+  int b_rows_per_group;
+  int half_b;           // SWIGLU: I
+  const float* a_scale; // [rows, K/128]
+  const float* b_scale; // [G, b_rows/128, K/128]
+  void* C;              // SWIGLU: e4m3 [rows, N]; STORE: bf16 [rows, N]
+  float* c_scale;       // SWIGLU: [rows, N/128]
+  int* err;
+};
+
+__device__ __forceinline__ void decode_tile(int t, const int* prefix, const int* roff, int G,
+                                            int& g, int& nt, int& row0, int& m_valid) {
+  int lo = 0, hi = G - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (prefix[mid] <= t) lo = mid; else hi = mid - 1;
+  }
+  g = lo;
+  const int m = roff[g + 1] - roff[g];
+  const int mtc = (m + BM - 1) / BM;
+  const int local = t - prefix[g];
+  nt = local / mtc;
+  const int mt = local - nt * mtc;
+  row0 = roff[g] + mt * BM;
+  m_valid = min(BM, m - mt * BM);
+}
+
+__device__ __forceinline__ void raise_abort(volatile int* abort, int* err) {
+  *abort = 1;
+  atomicOr(err, ERR_GEMM_FP8_TIMEOUT);
+}
+
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
+  return (uint32_t)__nv_cvt_float_to_fp8(a, __NV_SATFINITE, __NV_E4M3) |
+         ((uint32_t)__nv_cvt_float_to_fp8(b, __NV_SATFINITE, __NV_E4M3) << 8) |
+         ((uint32_t)__nv_cvt_float_to_fp8(c, __NV_SATFINITE, __NV_E4M3) << 16) |
+         ((uint32_t)__nv_cvt_float_to_fp8(d, __NV_SATFINITE, __NV_E4M3) << 24);
+}
+
+template <bool SWIGLU>
+__global__ void __launch_bounds__(kThreads, 1)
+    fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                    const __grid_constant__ CUtensorMap tmB, const Fp8Params p) {
+  constexpr int BN_OUT = SWIGLU ? BN / 2 : BN;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + OFF_B;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* empty = full + STAGES;
+  uint64_t* pfull = empty + STAGES;   // [2] partial ready
+  uint64_t* pempty = pfull + 2;       // [2] partial consumed (256 arrivals)
+  uint64_t* mma_done = pempty + 2;
+  uint64_t* xbar = mma_done + 1;      // [2] amax exchange between the warpgroups (256 arrivals)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
+  float* amax_x = reinterpret_cast<float*>(smem + OFF_AMAX);
+  int* prefix = reinterpret_cast<int*>(smem + OFF_TAB);
+  int* roff = prefix + kMaxGroups + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = p.offsets ? p.n_groups : 1;
+  const int n_tiles_n = p.N / BN_OUT;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&pfull[a], 1); mbar_init(&pempty[a], 256); }
+    mbar_init(mma_done, 1);
+    mbar_init(&xbar[0], 256);
+    mbar_init(&xbar[1], 256);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 2) {
+    const int per = (G + 31) / 32;
+    const int g0 = lane * per;
+    int local = 0;
+    for (int i = 0; i < per; ++i) {
+      const int g = g0 + i;
+      if (g < G) {
+        const int a = p.offsets ? p.offsets[g] : 0;
+        const int b = p.offsets ? p.offsets[g + 1] : p.rows;
+        roff[g] = a;
+        if (g == G - 1) roff[G] = b;
+        local += ((b - a + BM - 1) / BM) * n_tiles_n;
+      }
+    }
+    int incl = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    __syncwarp();
+    int run = incl - local;
+    for (int i = 0; i < per; ++i) {
+      const int g = g0 + i;
+      if (g < G) {
+        prefix[g] = run;
+        run += ((roff[g + 1] - roff[g] + BM - 1) / BM) * n_tiles_n;
+      }
+    }
+    if (lane == 31) prefix[G] = incl;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = prefix[G];
+  const int nk = p.K / BK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        int g, nt, row0, mv;
+        decode_tile(t, prefix, roff, G, g, nt, row0, mv);
+        const int brow = g * p.b_rows_per_group + nt * BN_OUT;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, kWaitNs)) {
+            raise_abort(abort_flag, p.err);
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+          tma_load_2d(sA + stage * A_BYTES, &tmA, kb * BK, row0, &full[stage]);
+          if (SWIGLU) {
+            tma_load_2d(sB + stage * B_BYTES, &tmB, kb * BK, brow, &full[stage]);
+            tma_load_2d(sB + stage * B_BYTES + B_BYTES / 2, &tmB, kb * BK, brow + p.half_b,
+                        &full[stage]);
+          } else {
+            tma_load_2d(sB + stage * B_BYTES, &tmB, kb * BK, brow, &full[stage]);
+          }
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+      for (int s = 0; s < STAGES; ++s)
+        mbar_wait_bounded(&full[s], ((s < stage) ? phase : phase ^ 1), nullptr, kWaitNs);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_e4m3_f32(BM, BN);
+      int stage = 0, pb = 0;
+      uint32_t phase = 0, pphase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait_bounded(&pempty[pb], pphase ^ 1, abort_flag, kWaitNs) ||
+              !mbar_wait_bounded(&full[stage], phase, abort_flag, kWaitNs)) {
+            raise_abort(abort_flag, p.err);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * A_BYTES);
+          const uint32_t b0 = smem_u32(sB + stage * B_BYTES);
+          const uint32_t d_tmem = tmem_base + pb * BN;
+#pragma unroll
+          for (int k = 0; k < BK / 32; ++k)
+            mma_f8_ss(d_tmem, smem_desc_k_sw128(a0 + k * 32), smem_desc_k_sw128(b0 + k * 32),
+                      idesc, k != 0);
+          mma_commit(&empty[stage]);
+          mma_commit(&pfull[pb]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          if (++pb == 2) { pb = 0; pphase ^= 1; }
+        }
+      }
+      mma_commit(mma_done);
+      mbar_wait_bounded(mma_done, 0, nullptr, kWaitNs);
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int ew = warp - 2;            // 0..7
+    const int wg = ew >> 2;             // warpgroup 0 or 1
+    const int sub = warp & 3;           // TMEM lane quarter of this warp
+    const int rit = sub * 32 + lane;    // row inside the tile
+    const int nkb_a = p.K / BK;
+    int pb = 0;
+    uint32_t pphase = 0;
+    bool ok = true;
+    int it = 0;  // tiles done by this CTA (amax exchange slot and phase)
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
+      int g, nt, row0, mv;
+      decode_tile(t, prefix, roff, G, g, nt, row0, mv);
+      const bool valid = rit < mv;
+      const int arow = valid ? row0 + rit : row0;   // clamp scale reads for padding rows
+      const float* sa_row = p.a_scale + (size_t)arow * nkb_a;
+      const int nbw = p.b_rows_per_group / 128;     // weight row blocks per group
+      const float* sw_g = p.b_scale + (size_t)g * nbw * nkb_a;
+      // weight row block of this thread's two column halves
+      int blk0, blk1;
+      if (SWIGLU) {
+        blk0 = nt;                                   // gate rows nt*128 ..
+        blk1 = (p.half_b / 128) + nt;                // up rows I + nt*128 ..
+      } else {
+        blk0 = blk1 = 2 * nt + wg;                   // 128 output columns per warpgroup
+      }
+      float acc[128];
+#pragma unroll
+      for (int i = 0; i < 128; ++i) acc[i] = 0.f;
+      float sa = sa_row[0];
+      for (int kb = 0; kb < nk; ++kb) {
+        const float sa_next = (kb + 1 < nk) ? sa_row[kb + 1] : 0.f;
+        const float s0 = sa * sw_g[(size_t)blk0 * nkb_a + kb];
+        const float s1 = sa * sw_g[(size_t)blk1 * nkb_a + kb];
+        const bool got = mbar_wait_bounded(&pfull[pb], pphase, abort_flag, kWaitNs);
+        if (!__all_sync(0xffffffffu, got)) {
+          raise_abort(abort_flag, p.err);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t tb = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + pb * BN;
+        // SWIGLU: gate columns [wg*64, +64) then up columns 128 + [wg*64, +64);
+        // STORE: columns [wg*128, +128).
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint32_t col = SWIGLU ? (c < 2 ? wg * 64 + c * 32 : 128 + wg * 64 + (c - 2) * 32)
+                                      : wg * 128 + c * 32;
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tb + col, r);
+          tmem_wait_ld();
+          if (c == 3) {
+            tc_fence_before();
+            mbar_arrive(&pempty[pb]);   // partial fully read: the MMA may overwrite it
+          }
+          const float sc = (SWIGLU && c >= 2) ? s1 : s0;
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            acc[c * 32 + j] = fmaf(__uint_as_float(r[j]), sc, acc[c * 32 + j]);
+        }
+        if (++pb == 2) { pb = 0; pphase ^= 1; }
+        sa = sa_next;
+      }
+      if (!ok) break;
+      if (SWIGLU) {
+        float amax = 0.f;
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          const float gt = acc[j];
+          acc[j] = (gt / (1.0f + __expf(-gt))) * acc[64 + j];
+          amax = fmaxf(amax, fabsf(acc[j]));
+        }
+        // The row's 128 h columns live in both warpgroups: exchange amax.
+        const int sl = it & 1;
+        float* slot = amax_x + sl * 2 * BM;
+        slot[wg * BM + rit] = amax;
+        mbar_arrive(&xbar[sl]);
+        const bool xok = mbar_wait_bounded(&xbar[sl], (it >> 1) & 1, abort_flag, kWaitNs);
+        if (!xok) {
+          raise_abort(abort_flag, p.err);
+          break;
+        }
+        amax = fmaxf(amax, slot[(wg ^ 1) * BM + rit]);
+        const float sc = amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
+        if (valid) {
+          uint8_t* dst = static_cast<uint8_t*>(p.C) + (size_t)(row0 + rit) * p.N + nt * 128 + wg * 64;
+          uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t w[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int j = q * 16 + i * 4;
+              w[i] = e4m3x4(__fdiv_rn(acc[j], sc), __fdiv_rn(acc[j + 1], sc),
+                            __fdiv_rn(acc[j + 2], sc), __fdiv_rn(acc[j + 3], sc));
+            }
+            d4[q] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+          if (wg == 0) p.c_scale[(size_t)(row0 + rit) * (p.N / 128) + nt] = sc;
+        }
+      } else if (valid) {
+        __nv_bfloat16* dst =
+            static_cast<__nv_bfloat16*>(p.C) + (size_t)(row0 + rit) * p.N + nt * BN + wg * 128;
+        uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          uint32_t w[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            __nv_bfloat162 pr = __floats2bfloat162_rn(acc[q * 8 + 2 * i], acc[q * 8 + 2 * i + 1]);
+            w[i] = *reinterpret_cast<uint32_t*>(&pr);
+          }
+          d4[q] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+template <bool SWIGLU>
+moe_status fp8_launch(const void* A, const float* a_scale, const void* B, const float* b_scale,
+                      int b_rows_per_group, const int32_t* offsets, int n_groups, int rows, int N,
+                      int K, void* C, float* c_scale, cudaStream_t s) {
+  constexpr int BN_OUT = SWIGLU ? BN / 2 : BN;
+  CUtensorMap tmA, tmB;
+  moe_status st = make_tmap_2d(&tmA, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, rows, BK, BM);
+  if (st != MOE_OK) return st;
+  const int G = offsets ? n_groups : 1;
+  st = make_tmap_2d(&tmB, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, (uint64_t)G * b_rows_per_group,
+                    BK, SWIGLU ? 128 : BN);
+  if (st != MOE_OK) return st;
+  auto kern = fp8_gemm_kernel<SWIGLU>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
+    if (e != cudaSuccess) return cuda_check(e, "fp8_gemm smem attribute");
+    attr_set = true;
+  }
+  Fp8Params p;
+  p.offsets = offsets;
+  p.n_groups = n_groups;
+  p.rows = rows;
+  p.N = N;
+  p.K = K;
+  p.b_rows_per_group = b_rows_per_group;
+  p.half_b = SWIGLU ? b_rows_per_group / 2 : 0;
+  p.a_scale = a_scale;
+  p.b_scale = b_scale;
+  p.C = C;
+  p.c_scale = c_scale;
+  p.err = device_error_word();
+  if (!p.err) return fail(MOE_ERR_CUDA, "device error word unavailable");
+  const long long max_tiles = ((long long)(rows + BM - 1) / BM + (offsets ? G : 0)) * (N / BN_OUT);
+  int grid = sm_count();
+  if (max_tiles < grid) grid = (int)(max_tiles > 0 ? max_tiles : 1);
+  kern<<<grid, kThreads, SMEM_ALLOC, s>>>(tmA, tmB, p);
+  return cuda_check(cudaGetLastError(), "fp8_gemm launch");
+}
+
+}  // namespace
+
+moe_status launch_fp8_gemm(const void* A, const float* a_scale, const void* B,
+                           const float* b_scale, int b_rows_per_group, const int32_t* offsets,
+                           int n_groups, int rows, int N, int K, bool swiglu, void* C,
+                           float* c_scale, cudaStream_t s) {
+  if (rows <= 0) return MOE_OK;
+  if (K % BK) return fail(MOE_ERR_UNSUPPORTED, "fp8 gemm: K=%d not a multiple of 128", K);
+  if (offsets && n_groups > kMaxGroups)
+    return fail(MOE_ERR_UNSUPPORTED, "fp8 gemm: at most %d groups", kMaxGroups);
+  if (swiglu) {
+    if (N % 128) return fail(MOE_ERR_UNSUPPORTED, "fp8 gemm swiglu: N=%d %% 128", N);
+    return fp8_launch<true>(A, a_scale, B, b_scale, b_rows_per_group, offsets, n_groups, rows, N,
+                            K, C, c_scale, s);
+  }
+  if (N % 256) return fail(MOE_ERR_UNSUPPORTED, "fp8 gemm down: d=%d must be a multiple of 256", N);
+  return fp8_launch<false>(A, a_scale, B, b_scale, b_rows_per_group, offsets, n_groups, rows, N, K,
+                           C, c_scale, s);
 }
 
 }  // namespace moe

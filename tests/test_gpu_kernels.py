@@ -262,3 +262,88 @@ def test_quantize_128x128_bit_exact():
         rq, rs = O.quant_128x128(f64(w[e]).astype(np.float32))
         np.testing.assert_array_equal(s[e].cpu().numpy(), rs)
         np.testing.assert_array_equal(_e4m3_values(q[e]), rq)
+
+
+# ------------------------------------------------------------------ FP8 expert FFN
+
+def _fp8_ffn_case(sizes, d, I, seed, outliers=False):
+    g = _gen(seed)
+    G = len(sizes)
+    off = _groups(sizes)
+    rows = int(off[-1])
+    x = _randn((rows, d), g, 1.0)
+    if outliers:
+        mask = torch.rand(rows, d, generator=g, device=DEV) < 0.001
+        x = torch.where(mask, x.float() * 50, x.float()).to(torch.bfloat16)
+    wgu = _randn((G, 2 * I, d), g, d ** -0.5)
+    wdn = _randn((G, d, I), g, I ** -0.5)
+    xq = torch.empty(rows, d, dtype=torch.uint8, device=DEV)
+    xs = torch.empty(rows, d // 128, device=DEV)
+    moe.moe_quantize_1x128(x, xq, xs)
+    qgu = torch.empty(G, 2 * I, d, dtype=torch.uint8, device=DEV)
+    sgu = torch.empty(G, 2 * I // 128, d // 128, device=DEV)
+    qdn = torch.empty(G, d, I, dtype=torch.uint8, device=DEV)
+    sdn = torch.empty(G, d // 128, I // 128, device=DEV)
+    moe.moe_quantize_128x128(wgu, qgu, sgu)
+    moe.moe_quantize_128x128(wdn, qdn, sdn)
+    y = torch.full((rows, d), float("nan"), dtype=torch.bfloat16, device=DEV)
+    ws = _ws(moe.moe_expert_ffn_workspace_size(moe.MOE_E4M3, rows, I))
+    offsets = torch.from_numpy(off).to(DEV)
+    moe.moe_expert_ffn(xq, offsets, qgu, qdn, y, ws, x_scale=xs, w_scale_gate_up=sgu,
+                       w_scale_down=sdn)
+    torch.cuda.synchronize()
+    assert moe.moe_device_status() == 0
+    # the oracle quantises from the bf16 originals itself
+    ex = LazyExperts(wgu, wdn)
+    xs64 = f64(x)
+    ref = np.zeros((rows, d))
+    for e in range(G):
+        a, b_ = int(off[e]), int(off[e + 1])
+        if b_ > a:
+            wg_, wu_, wd_ = ex[e]
+            Wq = O.quantise_expert(wg_.astype(np.float32), wu_.astype(np.float32),
+                                   wd_.astype(np.float32))
+            ref[a:b_] = O.fp8_swiglu_ffn(xs64[a:b_].astype(np.float32), Wq)
+    return f64(y), ref
+
+
+@pytest.mark.parametrize("sizes,d,I,outliers", [
+    ([0, 1, 127, 128, 129, 300, 0, 5], 256, 256, False),
+    ([64, 200, 333], 512, 384, True),
+    ([1000, 700, 1300, 60], 1024, 512, False),
+])
+def test_expert_ffn_fp8(sizes, d, I, outliers):
+    got, ref = _fp8_ffn_case(sizes, d, I, sum(sizes) + 3 * d, outliers)
+    assert_close(got, ref, TOL["e4m3"], "y fp8")
+
+
+def test_expert_gate_up_fp8_codes_close():
+    """The FP8 gate/up half alone: its E4M3 codes and 1x128 scales against the
+    oracle's h quantisation (ties of the float32 h may round differently, so
+    codes agree for nearly all elements and scales closely)."""
+    g = _gen(77)
+    rows, d, I = 384, 512, 256
+    x = _randn((rows, d), g, 1.0)
+    wgu = _randn((1, 2 * I, d), g, d ** -0.5)
+    xq = torch.empty(rows, d, dtype=torch.uint8, device=DEV)
+    xs = torch.empty(rows, d // 128, device=DEV)
+    moe.moe_quantize_1x128(x, xq, xs)
+    qgu = torch.empty(1, 2 * I, d, dtype=torch.uint8, device=DEV)
+    sgu = torch.empty(1, 2 * I // 128, d // 128, device=DEV)
+    moe.moe_quantize_128x128(wgu, qgu, sgu)
+    h = torch.empty(rows, I, dtype=torch.uint8, device=DEV)
+    hs = torch.empty(rows, I // 128, device=DEV)
+    offsets = torch.tensor([0, rows], dtype=torch.int32, device=DEV)
+    moe.moe_expert_gate_up(xq, offsets, qgu, h, x_scale=xs, w_scale_gate_up=sgu, h_scale=hs)
+    torch.cuda.synchronize()
+    gu = f64(wgu[0]).astype(np.float32)
+    qx, sx = O.quant_1x128(f64(x).astype(np.float32))
+    qg, sg = O.quant_128x128(gu[:I])
+    qu, su = O.quant_128x128(gu[I:])
+    hg = O.fp8_promoted_gemm(qx, sx, qg, sg)
+    hu = O.fp8_promoted_gemm(qx, sx, qu, su)
+    href = (O.silu(hg) * hu).astype(np.float32)
+    rq, rs = O.quant_1x128(href)
+    np.testing.assert_allclose(hs.cpu().numpy(), rs, rtol=1e-5)
+    codes_equal = (_e4m3_values(h) == rq).mean()
+    assert codes_equal > 0.999, codes_equal

@@ -73,6 +73,18 @@ def test_layer_v3_bf16_ragged_T():
     _run(CONFIGS["v3_bf16"], T=1000, sample=24, seed_sample=1)
 
 
+def test_layer_v3_fp8_sampled():
+    """FP8 V3 shape (T = 16384, 0.1 % outliers x50) against the FP8-emulating oracle."""
+    _run(CONFIGS["v3_fp8"], sample=12, seed_sample=2)
+
+
+def test_layer_fp8_small_full():
+    """FP8 layer on a small shape, every token compared."""
+    from dataclasses import replace
+    cfg = replace(CONFIGS["v3_fp8"], name="fp8_small", T=1024, d=512, N_r=32, K=4, N_s=1, I=256)
+    _run(cfg)
+
+
 def test_layer_all_tokens_one_expert():
     """K = 1 and a dominant bias: one group holds every token, the others are empty."""
     cfg = CONFIGS["small_bf16"]
