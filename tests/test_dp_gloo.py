@@ -89,6 +89,8 @@ def _leaver(rank, world, port, q):
     allreduce_load(c, 10, T_total=20)          # one good step on every rank
     if rank == 1:
         q.put((rank, "left"))
+        q.close()
+        q.join_thread()                          # flush the message before leaving
         os._exit(0)                              # leaves between steps, nothing in flight
     try:
         allreduce_load(c, 10, T_total=20)
@@ -104,8 +106,10 @@ def test_rank_leaving_between_steps_is_an_error_not_a_hang():
     procs = [ctx.Process(target=_leaver, args=(r, 2, port, q)) for r in range(2)]
     for p in procs:
         p.start()
-    res = dict(q.get(timeout=120) for _ in range(2))
+    res = dict(q.get(timeout=90) for _ in range(2))
     for p in procs:
         p.join(timeout=60)
+        if p.is_alive():
+            p.kill()
     assert res[1] == "left"
     assert res[0].startswith("error:"), res[0]
