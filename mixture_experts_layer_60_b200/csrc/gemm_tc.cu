@@ -436,17 +436,23 @@ moe_status launch_tc_gemm(const void* A, const void* B, int b_rows_per_group,
         return tc_launch<128, TC_EPI_STORE_BF16, 6>(A, B, b_rows_per_group, offsets, n_groups,
                                                      rows, N, K, C, s);
       return fail(MOE_ERR_UNSUPPORTED, "tc gemm store: N=%d %% 128", N);
-    case TC_EPI_STORE_F32:
-      if (N % 256 == 0)
+    case TC_EPI_STORE_F32: {
+      // Router logits: one group of `rows` tokens.  Take narrower N tiles
+      // while the wide ones would leave a quarter of the SMs idle.
+      const long long m_tiles = (rows + BM - 1) / BM;
+      const long long busy = (3LL * sm_count()) / 4;
+      int bn = (N % 256 == 0) ? 256 : (N % 128 == 0) ? 128 : 64;
+      while (bn > 64 && N % (bn / 2) == 0 && m_tiles * (N / bn) < busy) bn /= 2;
+      if (N % bn) return fail(MOE_ERR_UNSUPPORTED, "tc gemm f32: N=%d %% 64", N);
+      if (bn == 256)
         return tc_launch<256, TC_EPI_STORE_F32, 4>(A, B, b_rows_per_group, offsets, n_groups,
                                                     rows, N, K, C, s);
-      if (N % 128 == 0)
+      if (bn == 128)
         return tc_launch<128, TC_EPI_STORE_F32, 6>(A, B, b_rows_per_group, offsets, n_groups,
                                                     rows, N, K, C, s);
-      if (N % 64 == 0)
-        return tc_launch<64, TC_EPI_STORE_F32, 8>(A, B, b_rows_per_group, offsets, n_groups,
-                                                   rows, N, K, C, s);
-      return fail(MOE_ERR_UNSUPPORTED, "tc gemm f32: N=%d %% 64", N);
+      return tc_launch<64, TC_EPI_STORE_F32, 8>(A, B, b_rows_per_group, offsets, n_groups, rows,
+                                                 N, K, C, s);
+    }
   }
   return fail(MOE_ERR_INVALID_ARG, "tc gemm: bad epilogue");
 }

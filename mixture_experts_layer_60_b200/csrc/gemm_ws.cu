@@ -1,0 +1,392 @@
+// Weights-stationary grouped bf16 GEMM on tcgen05 for the expert FFNs
+// (FFN_i of the h'-equation, "DeepSeek-V3 技術報告", section 方法 / 2).
+//
+// The MMA's M side is the weight matrix and its N side the expert's tokens:
+//   D[n, j] = sum_k W[g*b_rows + w0 + n, k] * X[tok0 + j, k]
+// A tile is 256 weight rows x up to 256 token rows.  Each 64-wide K step
+// issues two M=128 MMAs per 16-element slice (SWIGLU: the 128 gate rows and
+// the 128 matching up rows of one h-column block; STORE: output columns
+// [0,128) and [128,256) of a 256-column block), both with N = the tile's token
+// count rounded up to 16.  An expert with M tokens is cut into
+// ceil(M/256) token tiles of equal size (multiples of 16), so ragged expert
+// loads cost at most 15 padding rows per tile instead of a 128-row tail.
+//
+// Epilogue (4 warps; warp w owns TMEM lanes 32*(w%4).. = weight rows):
+//   SWIGLU  h[tok0+j, nt*128 + n] = bf16(SiLU(D_gate[n,j]) * D_up[n,j])
+//   STORE   y[tok0+j, nt*256 + n] = bf16(D0[n,j]), y[.., nt*256+128+n] = bf16(D1[n,j])
+// Values are transposed through a 2 KB shared-memory patch per warp so that
+// global stores are 16-byte vectors along token rows.
+//
+// Roles: warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer, warps 2-5
+// epilogue.  3 shared-memory stages of 64 KB; one TMEM accumulator pair
+// (512 columns).  Every wait is bounded (1 s) and reported through the
+// device error word.
+#include <math.h>
+
+#include "launch.h"
+#include "sm100.cuh"
+
+namespace moe {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int WROWS = 256;          // weight rows per tile (two M=128 MMAs)
+constexpr int TMAX = 256;           // max token rows per tile (MMA N)
+constexpr int BK = 64;              // bf16 elements per 128-byte swizzle row
+constexpr int XBOX = 32;            // token rows per TMA box
+constexpr int STAGES = 3;
+constexpr int kThreads = 192;
+constexpr int kMaxGroups = 1024;
+constexpr uint64_t kWaitNs = 1000000000ull;
+constexpr uint32_t TMEM_COLS = 512;
+
+constexpr int W_BYTES = WROWS * BK * 2;       // 32 KB
+constexpr int X_BYTES = TMAX * BK * 2;        // 32 KB
+constexpr int XBOX_BYTES = XBOX * BK * 2;     // 4 KB
+constexpr int OFF_X = STAGES * W_BYTES;
+constexpr int OFF_STAGE_OUT = OFF_X + STAGES * X_BYTES;   // 4 warps x 2 KB transpose patches
+constexpr int OFF_BAR = OFF_STAGE_OUT + 4 * 2048;
+constexpr int N_BARS = 2 * STAGES + 3;
+constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
+constexpr int OFF_TAB = OFF_MISC + 16;
+constexpr int SMEM_BYTES = OFF_TAB + 2 * (kMaxGroups + 1) * 4;
+constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
+
+struct WsParams {
+  const int32_t* offsets;   // [n_groups+1] or nullptr (one group of `rows`)
+  int n_groups;
+  int rows;
+  int N;                    // output columns (SWIGLU: I; STORE: d)
+  int K;
+  int b_rows_per_group;
+  int half_b;               // SWIGLU: I
+  __nv_bfloat16* C;
+  int* err;
+};
+
+template <bool SWIGLU>
+struct TileMath {
+  static constexpr int OUT_COLS = SWIGLU ? 128 : 256;   // output columns per weight tile
+};
+
+// Token tiling of a group of m rows: tiles of `step` rows (a multiple of 16,
+// at most 256, about m / ceil(m/256)); n_t = ceil(m / step) tiles, each with
+// at least one row, the last one possibly shorter.
+__device__ __forceinline__ void token_tiling(int m, int& n_t, int& step) {
+  if (m <= 0) { n_t = 0; step = 16; return; }
+  const int n0 = (m + TMAX - 1) / TMAX;
+  step = ((m + n0 - 1) / n0 + 15) / 16 * 16;
+  n_t = (m + step - 1) / step;
+}
+
+__device__ __forceinline__ void decode_tile(int t, const int* prefix, const int* roff,
+                                            int G, int& g, int& nt,
+                                            int& tok0, int& count) {
+  int lo = 0, hi = G - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (prefix[mid] <= t) lo = mid; else hi = mid - 1;
+  }
+  g = lo;
+  const int m = roff[g + 1] - roff[g];
+  int n_t, step;
+  token_tiling(m, n_t, step);
+  const int local = t - prefix[g];
+  nt = local / n_t;
+  const int ti = local - nt * n_t;
+  tok0 = roff[g] + ti * step;
+  count = min(step, m - ti * step);
+}
+
+__device__ __forceinline__ void raise_abort(volatile int* abort, int* err) {
+  *abort = 1;
+  atomicOr(err, ERR_GEMM_TIMEOUT);
+}
+
+__device__ __forceinline__ float silu_f(float x) { return x / (1.0f + __expf(-x)); }
+
+template <bool SWIGLU>
+__global__ void __launch_bounds__(kThreads, 1)
+    ws_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                   const WsParams p) {
+  constexpr int OUT_COLS = TileMath<SWIGLU>::OUT_COLS;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sW = smem;
+  uint8_t* sX = smem + OFF_X;
+  uint8_t* sOut = smem + OFF_STAGE_OUT;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 1;
+  uint64_t* mma_done = tempty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
+  int* prefix = reinterpret_cast<int*>(smem + OFF_TAB);
+  int* roff = prefix + kMaxGroups + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = p.offsets ? p.n_groups : 1;
+  const int n_wt = p.N / OUT_COLS;   // weight tiles per group
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    mbar_init(tfull, 1);
+    mbar_init(tempty, 128);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmW);
+    tma_prefetch_desc(&tmX);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 2) {
+    // Tile table: prefix[g] = first tile of group g; tiles of a group are
+    // ordered weight-tile major, token-tile fastest.
+    const int per = (G + 31) / 32;
+    const int g0 = lane * per;
+    int local = 0;
+    for (int i = 0; i < per; ++i) {
+      const int g = g0 + i;
+      if (g < G) {
+        const int a = p.offsets ? p.offsets[g] : 0;
+        const int b = p.offsets ? p.offsets[g + 1] : p.rows;
+        int n_t, step;
+        token_tiling(b - a, n_t, step);
+        roff[g] = a;
+        if (g == G - 1) roff[G] = b;
+        local += n_t * n_wt;
+      }
+    }
+    int incl = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    __syncwarp();
+    int run = incl - local;
+    for (int i = 0; i < per; ++i) {
+      const int g = g0 + i;
+      if (g < G) {
+        prefix[g] = run;
+        int n_t, step;
+        token_tiling(roff[g + 1] - roff[g], n_t, step);
+        run += n_t * n_wt;
+      }
+    }
+    if (lane == 31) prefix[G] = incl;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = prefix[G];
+  const int nk = p.K / BK;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        int g, nt, tok0, count;
+        decode_tile(t, prefix, roff, G, g, nt, tok0, count);
+        const int nbox = (count + XBOX - 1) / XBOX;
+        const uint32_t bytes = W_BYTES + nbox * XBOX_BYTES;
+        const int wrow = g * p.b_rows_per_group + nt * (SWIGLU ? 128 : 256);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, kWaitNs)) {
+            raise_abort(abort_flag, p.err);
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], bytes);
+          uint8_t* w_dst = sW + stage * W_BYTES;
+          tma_load_2d(w_dst, &tmW, kb * BK, wrow, &full[stage]);
+          tma_load_2d(w_dst + W_BYTES / 2, &tmW, kb * BK, wrow + (SWIGLU ? p.half_b : 128),
+                      &full[stage]);
+          uint8_t* x_dst = sX + stage * X_BYTES;
+          for (int b = 0; b < nbox; ++b)
+            tma_load_2d(x_dst + b * XBOX_BYTES, &tmX, kb * BK, tok0 + b * XBOX, &full[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+      for (int s = 0; s < STAGES; ++s)
+        mbar_wait_bounded(&full[s], ((s < stage) ? phase : phase ^ 1), nullptr, kWaitNs);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, tphase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        int g, nt, tok0, count;
+        decode_tile(t, prefix, roff, G, g, nt, tok0, count);
+        const int n_mma = (count + 15) / 16 * 16;
+        const uint32_t idesc = idesc_bf16_f32(128, n_mma);
+        if (!mbar_wait_bounded(tempty, tphase ^ 1, abort_flag, kWaitNs)) {
+          raise_abort(abort_flag, p.err);
+          break;
+        }
+        tc_fence_after();
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait_bounded(&full[stage], phase, abort_flag, kWaitNs)) {
+            raise_abort(abort_flag, p.err);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t w0 = smem_u32(sW + stage * W_BYTES);
+          const uint32_t x0 = smem_u32(sX + stage * X_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t xd = smem_desc_k_sw128(x0 + k * 32);
+            const uint32_t acc = (kb | k) != 0;
+            mma_f16_ss(tmem_base, smem_desc_k_sw128(w0 + k * 32), xd, idesc, acc);
+            mma_f16_ss(tmem_base + 256, smem_desc_k_sw128(w0 + W_BYTES / 2 + k * 32), xd, idesc,
+                       acc);
+          }
+          mma_commit(&empty[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+        mma_commit(tfull);
+        tphase ^= 1;
+      }
+      mma_commit(mma_done);
+      mbar_wait_bounded(mma_done, 0, nullptr, kWaitNs);
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int q = warp & 3;                       // TMEM lane quarter
+    const int n = q * 32 + lane;                  // weight row inside each 128-row half
+    uint16_t* patch = reinterpret_cast<uint16_t*>(sOut + (warp - 2) * 2048);   // [32 tok][32 col]
+    uint32_t tphase = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      int g, nt, tok0, count;
+      decode_tile(t, prefix, roff, G, g, nt, tok0, count);
+      const bool got = mbar_wait_bounded(tfull, tphase, abort_flag, kWaitNs);
+      if (!__all_sync(0xffffffffu, got)) {
+        raise_abort(abort_flag, p.err);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tl = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+      const int nch = (count + 31) / 32;
+      for (int c = 0; c < nch; ++c) {
+        uint32_t r0[32], r1[32];
+        tmem_ld_32x32b_x32(tl + c * 32, r0);
+        tmem_ld_32x32b_x32(tl + 256 + c * 32, r1);
+        tmem_wait_ld();
+        const int half_n = SWIGLU ? 1 : 2;
+#pragma unroll
+        for (int hh = 0; hh < half_n; ++hh) {
+          // patch[j][lane] = value of token (c*32 + j), column (q*32 + lane)
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            float v;
+            if (SWIGLU) v = silu_f(__uint_as_float(r0[j])) * __uint_as_float(r1[j]);
+            else v = __uint_as_float(hh == 0 ? r0[j] : r1[j]);
+            patch[j * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+          }
+          __syncwarp();
+          // 32 token rows x 64 bytes: lane -> (row lane/4 + 8*it, 16-byte chunk lane%4)
+          const int col0 = nt * OUT_COLS + hh * 128 + q * 32;
+#pragma unroll
+          for (int it = 0; it < 4; ++it) {
+            const int j = it * 8 + (lane >> 2);
+            const int tok = c * 32 + j;
+            const uint4 v = *reinterpret_cast<const uint4*>(patch + j * 32 + (lane & 3) * 8);
+            if (tok < count) {
+              __nv_bfloat16* dst = p.C + (size_t)(tok0 + tok) * p.N + col0 + (lane & 3) * 8;
+              *reinterpret_cast<uint4*>(dst) = v;
+            }
+          }
+          __syncwarp();
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(tempty);
+      tphase ^= 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace
+
+moe_status make_tmap_2d(CUtensorMap* tm, const void* base, CUtensorMapDataType dtype,
+                        int elem_bytes, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                        uint32_t box_outer);
+
+namespace {
+
+template <bool SWIGLU>
+moe_status ws_launch(const void* X, const void* W, int b_rows_per_group, const int32_t* offsets,
+                     int n_groups, int rows, int N, int K, void* C, cudaStream_t s) {
+  constexpr int OUT_COLS = TileMath<SWIGLU>::OUT_COLS;
+  CUtensorMap tmW, tmX;
+  const int G = offsets ? n_groups : 1;
+  moe_status st = make_tmap_2d(&tmW, W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K,
+                               (uint64_t)G * b_rows_per_group, BK, 128);
+  if (st != MOE_OK) return st;
+  st = make_tmap_2d(&tmX, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, rows, BK, XBOX);
+  if (st != MOE_OK) return st;
+  auto kern = ws_gemm_kernel<SWIGLU>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
+    if (e != cudaSuccess) return cuda_check(e, "ws_gemm smem attribute");
+    attr_set = true;
+  }
+  WsParams p;
+  p.offsets = offsets;
+  p.n_groups = n_groups;
+  p.rows = rows;
+  p.N = N;
+  p.K = K;
+  p.b_rows_per_group = b_rows_per_group;
+  p.half_b = SWIGLU ? b_rows_per_group / 2 : 0;
+  p.C = static_cast<__nv_bfloat16*>(C);
+  p.err = device_error_word();
+  if (!p.err) return fail(MOE_ERR_CUDA, "device error word unavailable");
+  const long long max_tiles = ((long long)(rows + TMAX - 1) / TMAX + (offsets ? G : 0)) * (N / OUT_COLS);
+  int grid = sm_count();
+  if (max_tiles < grid) grid = (int)(max_tiles > 0 ? max_tiles : 1);
+  kern<<<grid, kThreads, SMEM_ALLOC, s>>>(tmW, tmX, p);
+  return cuda_check(cudaGetLastError(), "ws_gemm launch");
+}
+
+}  // namespace
+
+moe_status launch_ws_gemm(const void* X, const void* W, int b_rows_per_group,
+                          const int32_t* offsets, int n_groups, int rows, int N, int K,
+                          bool swiglu, void* C, cudaStream_t s) {
+  if (rows <= 0) return MOE_OK;
+  if (K % BK) return fail(MOE_ERR_UNSUPPORTED, "ws gemm: K=%d not a multiple of %d", K, BK);
+  if (offsets && n_groups > kMaxGroups)
+    return fail(MOE_ERR_UNSUPPORTED, "ws gemm: at most %d groups", kMaxGroups);
+  if (swiglu) {
+    if (N % 128) return fail(MOE_ERR_UNSUPPORTED, "ws gemm swiglu: N=%d %% 128", N);
+    return ws_launch<true>(X, W, b_rows_per_group, offsets, n_groups, rows, N, K, C, s);
+  }
+  if (N % 256) return fail(MOE_ERR_UNSUPPORTED, "ws gemm store: N=%d %% 256", N);
+  return ws_launch<false>(X, W, b_rows_per_group, offsets, n_groups, rows, N, K, C, s);
+}
+
+}  // namespace moe

@@ -37,6 +37,14 @@ moe_status launch_tc_gemm(const void* A, const void* B, int b_rows_per_group,
                           const int32_t* offsets, int n_groups, int rows, int N, int K,
                           TcEpilogue epi, void* C, cudaStream_t s);
 
+// gemm_ws.cu -----------------------------------------------------------------
+// Weights-stationary grouped bf16 GEMM (expert FFNs): weights on the MMA's M
+// side, each expert's tokens on N (tiles of <= 256 tokens, 16-row granularity).
+// swiglu: B holds W_gate rows [0, I) and W_up rows [I, 2I) of a group.
+moe_status launch_ws_gemm(const void* X, const void* W, int b_rows_per_group,
+                          const int32_t* offsets, int n_groups, int rows, int N, int K,
+                          bool swiglu, void* C, cudaStream_t s);
+
 // gemm_fp8.cu ----------------------------------------------------------------
 moe_status launch_fp8_gemm(const void* A, const float* a_scale, const void* B,
                            const float* b_scale, int b_rows_per_group,

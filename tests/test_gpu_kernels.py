@@ -180,6 +180,8 @@ def _ffn_case(sizes, d, I, dtype, seed, extra_rows=0):
     ([64, 200, 333], 512, 384),                     # I not a multiple of 256
     ([1000, 700, 1300, 60], 1024, 512),             # many tiles per CTA, stage wrap-around
     ([5000], 768, 256),                             # one large group (the shared-expert shape)
+    ([64, 200, 333], 384, 256),                     # d not a multiple of 256 (128-column down tiles)
+    ([255, 256, 257, 511, 513, 17, 16, 15], 256, 128),  # token tiling around 256-row boundaries
 ])
 def test_expert_ffn_bf16(sizes, d, I):
     got, ref, n = _ffn_case(sizes, d, I, torch.bfloat16, sum(sizes) + d, extra_rows=3)
