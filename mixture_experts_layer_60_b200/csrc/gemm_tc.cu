@@ -38,7 +38,6 @@ constexpr int BM = 128;            // tile rows (TMEM lanes)
 constexpr int BK = 64;             // bf16 elements per 128-byte swizzle row
 constexpr int kThreads = 192;
 constexpr int kMaxGroups = 1024;
-constexpr int kPrefetch = 8;       // K-steps of L2 prefetch ahead of the loads
 constexpr uint64_t kWaitNs = 1000000000ull;
 
 struct TcParams {
@@ -180,34 +179,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
-    // Shared-memory ring of STAGES K-steps; L2 prefetches run kPrefetch
-    // K-steps ahead of the loads (into the next tile near a tile's end).
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      auto prefetch = [&](int g, int nt, int row0, int kb) {
-        const int brow = g * p.b_rows_per_group + nt * BN_OUT;
-        tma_prefetch_l2_2d(&tmA, kb * BK, row0);
-        tma_prefetch_l2_2d(&tmB, kb * BK, brow);
-        if (EPI == TC_EPI_SWIGLU_BF16) tma_prefetch_l2_2d(&tmB, kb * BK, brow + p.half_b);
-      };
-      if (blockIdx.x < total) {
-        int g, nt, row0, mv;
-        decode_tile(blockIdx.x, prefix, roff, G, g, nt, row0, mv);
-        for (int kb = 0; kb < kPrefetch && kb < nk; ++kb) prefetch(g, nt, row0, kb);
-      }
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
         int g, nt, row0, mv;
         decode_tile(t, prefix, roff, G, g, nt, row0, mv);
-        int g2 = 0, nt2 = 0, row2 = 0, mv2 = 0;
-        const bool has_next = t + (int)gridDim.x < total;
-        if (has_next) decode_tile(t + gridDim.x, prefix, roff, G, g2, nt2, row2, mv2);
         const int brow = g * p.b_rows_per_group + nt * BN_OUT;
         for (int kb = 0; kb < nk; ++kb) {
-          const int pk = kb + kPrefetch;
-          if (pk < nk) prefetch(g, nt, row0, pk);
-          else if (has_next && pk - nk < nk) prefetch(g2, nt2, row2, pk - nk);
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, kWaitNs)) {
             raise_abort(abort_flag, p.err, ERR_GEMM_TIMEOUT);
             ok = false;

@@ -37,7 +37,6 @@ constexpr int TMAX = 256;           // max token rows per tile (MMA N)
 constexpr int BK = 64;              // bf16 elements per 128-byte swizzle row
 constexpr int XBOX = 32;            // token rows per TMA box
 constexpr int STAGES = 3;
-constexpr int kPrefetch = 6;        // K-steps of L2 prefetch ahead of the loads
 constexpr int kThreads = 192;
 constexpr int kMaxGroups = 1024;
 constexpr uint64_t kWaitNs = 1000000000ull;
@@ -193,37 +192,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
-    // Loads run through a 3-stage shared-memory ring; L2 prefetches run
-    // kPrefetch K-steps ahead of them (into the next tile near a tile's end)
-    // so that the weight stream from HBM is requested well before it is needed.
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      auto prefetch = [&](int g, int nt, int tok0, int count, int kb) {
-        const int wrow = g * p.b_rows_per_group + nt * (SWIGLU ? 128 : 256);
-        tma_prefetch_l2_2d(&tmW, kb * BK, wrow);
-        tma_prefetch_l2_2d(&tmW, kb * BK, wrow + (SWIGLU ? p.half_b : 128));
-        for (int b = 0; b < count; b += XBOX) tma_prefetch_l2_2d(&tmX, kb * BK, tok0 + b);
-      };
-      if (blockIdx.x < total) {
-        int g, nt, tok0, count;
-        decode_tile(blockIdx.x, prefix, roff, G, g, nt, tok0, count);
-        for (int kb = 0; kb < kPrefetch && kb < nk; ++kb) prefetch(g, nt, tok0, count, kb);
-      }
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
         int g, nt, tok0, count;
         decode_tile(t, prefix, roff, G, g, nt, tok0, count);
-        int g2 = 0, nt2 = 0, tok2 = 0, count2 = 0;
-        const bool has_next = t + (int)gridDim.x < total;
-        if (has_next) decode_tile(t + gridDim.x, prefix, roff, G, g2, nt2, tok2, count2);
         const int nbox = (count + XBOX - 1) / XBOX;
         const uint32_t bytes = W_BYTES + nbox * XBOX_BYTES;
         const int wrow = g * p.b_rows_per_group + nt * (SWIGLU ? 128 : 256);
         for (int kb = 0; kb < nk; ++kb) {
-          const int pk = kb + kPrefetch;
-          if (pk < nk) prefetch(g, nt, tok0, count, pk);
-          else if (has_next && pk - nk < nk) prefetch(g2, nt2, tok2, count2, pk - nk);
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, kWaitNs)) {
             raise_abort(abort_flag, p.err);
             ok = false;
@@ -288,6 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ---------------------------------------------------------------- epilogue
     const int q = warp & 3;                       // TMEM lane quarter
+    const int n = q * 32 + lane;                  // weight row inside each 128-row half
     uint16_t* patch = reinterpret_cast<uint16_t*>(sOut + (warp - 2) * 2048);   // [32 tok][32 col]
     uint32_t tphase = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
