@@ -10,13 +10,14 @@
 // 128-byte swizzle width).  The MMA warp writes P_kb into one of two TMEM
 // partial buffers (4 x tcgen05.mma kind::f8f6f4, K = 32 each); two epilogue
 // warpgroups read it back with tcgen05.ld, multiply by the two scales and add
-// into float32 registers, then release the buffer.  After the last block:
+// into float32 registers (4 warpgroups, 64 columns each), then release the
+// buffer.  After the last block:
 //   SWIGLU   h = SiLU(acc_gate) * acc_up (float32), quantised 1x128 to E4M3
-//            with scale amax/448 (the 128 columns of a row span both
+//            with scale amax/448 (the 128 columns of a row span the four
 //            warpgroups: their amax meet in shared memory)
 //   STORE    y = bf16(acc)
-// Warp roles: 0 TMA producer, 1 TMEM allocator + MMA issuer, 2-9 epilogue
-// (warpgroup 0 = warps 2-5, warpgroup 1 = warps 6-9).  Waits are bounded.
+// Warp roles: 0 TMA producer, 1 TMEM allocator + MMA issuer, 2-17 epilogue
+// (warpgroup w = warps 2+4w .. 5+4w).  Waits are bounded.
 #include <math.h>
 
 #include "launch.h"
@@ -36,7 +37,8 @@ constexpr int BM = 128;
 constexpr int BN = 256;               // MMA N: SWIGLU = 128 gate + 128 up columns
 constexpr int BK = 128;               // e4m3 bytes per row = one promotion block
 constexpr int STAGES = 4;
-constexpr int kThreads = 320;
+constexpr int kEpiWG = 4;             // epilogue warpgroups; each owns BN / kEpiWG columns
+constexpr int kThreads = 64 + 128 * kEpiWG;
 constexpr int kMaxGroups = 1024;
 constexpr uint64_t kWaitNs = 1000000000ull;
 constexpr uint32_t TMEM_COLS = 512;   // two partial buffers of BN columns
@@ -48,8 +50,8 @@ constexpr int OFF_B = STAGES * A_BYTES;
 constexpr int OFF_BAR = OFF_B + STAGES * B_BYTES;
 constexpr int N_BARS = 2 * STAGES + 7;
 constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
-constexpr int OFF_AMAX = OFF_MISC + 16;                 // [2 slots][2 warpgroups][BM] float
-constexpr int OFF_TAB = OFF_AMAX + 2 * 2 * BM * 4;
+constexpr int OFF_AMAX = OFF_MISC + 16;                 // [2 slots][kEpiWG][BM] float
+constexpr int OFF_TAB = OFF_AMAX + 2 * kEpiWG * BM * 4;
 constexpr int SMEM_BYTES = OFF_TAB + 2 * (kMaxGroups + 1) * 4;
 constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
 
@@ -125,10 +127,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int a = 0; a < 2; ++a) { mbar_init(&pfull[a], 1); mbar_init(&pempty[a], 256); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&pfull[a], 1); mbar_init(&pempty[a], 128 * kEpiWG); }
     mbar_init(mma_done, 1);
-    mbar_init(&xbar[0], 256);
-    mbar_init(&xbar[1], 256);
+    mbar_init(&xbar[0], 128 * kEpiWG);
+    mbar_init(&xbar[1], 128 * kEpiWG);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
@@ -239,8 +241,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------------------------------------------------------- epilogue
-    const int ew = warp - 2;            // 0..7
-    const int wg = ew >> 2;             // warpgroup 0 or 1
+    // kEpiWG warpgroups; warpgroup wg owns, for every row of the tile,
+    //   SWIGLU: gate columns [wg*32, +32) and the matching up columns 128 + [wg*32, +32)
+    //   STORE:  output columns [wg*64, +64)
+    constexpr int CW = BN / kEpiWG;     // 64 accumulator columns per thread
+    const int wg = (warp - 2) >> 2;
     const int sub = warp & 3;           // TMEM lane quarter of this warp
     const int rit = sub * 32 + lane;    // row inside the tile
     const int nkb_a = p.K / BK;
@@ -256,17 +261,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float* sa_row = p.a_scale + (size_t)arow * nkb_a;
       const int nbw = p.b_rows_per_group / 128;     // weight row blocks per group
       const float* sw_g = p.b_scale + (size_t)g * nbw * nkb_a;
-      // weight row block of this thread's two column halves
+      // weight row blocks of this thread's two 32-column chunks
       int blk0, blk1;
+      uint32_t col0, col1;
       if (SWIGLU) {
         blk0 = nt;                                   // gate rows nt*128 ..
         blk1 = (p.half_b / 128) + nt;                // up rows I + nt*128 ..
+        col0 = wg * 32;
+        col1 = 128 + wg * 32;
       } else {
-        blk0 = blk1 = 2 * nt + wg;                   // 128 output columns per warpgroup
+        blk0 = blk1 = 2 * nt + (wg * CW) / 128;      // output columns nt*256 + wg*64 ..
+        col0 = wg * CW;
+        col1 = wg * CW + 32;
       }
-      float acc[128];
+      float acc[CW];
 #pragma unroll
-      for (int i = 0; i < 128; ++i) acc[i] = 0.f;
+      for (int i = 0; i < CW; ++i) acc[i] = 0.f;
       float sa = sa_row[0];
       for (int kb = 0; kb < nk; ++kb) {
         const float sa_next = (kb + 1 < nk) ? sa_row[kb + 1] : 0.f;
@@ -280,23 +290,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t tb = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + pb * BN;
-        // SWIGLU: gate columns [wg*64, +64) then up columns 128 + [wg*64, +64);
-        // STORE: columns [wg*128, +128).
+        // Four 16-column pieces; many warps per sub-partition hide the load latency.
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          const uint32_t col = SWIGLU ? (c < 2 ? wg * 64 + c * 32 : 128 + wg * 64 + (c - 2) * 32)
-                                      : wg * 128 + c * 32;
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(tb + col, r);
+          uint32_t r[16];
+          tmem_ld_32x32b_x16(tb + (c < 2 ? col0 : col1) + (c & 1) * 16, r);
           tmem_wait_ld();
           if (c == 3) {
             tc_fence_before();
-            mbar_arrive(&pempty[pb]);   // partial fully read: the MMA may overwrite it
+            mbar_arrive(&pempty[pb]);   // partial read: the MMA may overwrite it
           }
-          const float sc = (SWIGLU && c >= 2) ? s1 : s0;
+          const float sc = c < 2 ? s0 : s1;
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            acc[c * 32 + j] = fmaf(__uint_as_float(r[j]), sc, acc[c * 32 + j]);
+          for (int j = 0; j < 16; ++j) acc[c * 16 + j] = fmaf(__uint_as_float(r[j]), sc, acc[c * 16 + j]);
         }
         if (++pb == 2) { pb = 0; pphase ^= 1; }
         sa = sa_next;
@@ -305,14 +311,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (SWIGLU) {
         float amax = 0.f;
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
+        for (int j = 0; j < 32; ++j) {
           const float gt = acc[j];
-          acc[j] = (gt / (1.0f + __expf(-gt))) * acc[64 + j];
+          acc[j] = __fdividef(gt, 1.0f + __expf(-gt)) * acc[32 + j];
           amax = fmaxf(amax, fabsf(acc[j]));
         }
-        // The row's 128 h columns live in both warpgroups: exchange amax.
+        // The row's 128 h columns are spread over the warpgroups: exchange amax.
         const int sl = it & 1;
-        float* slot = amax_x + sl * 2 * BM;
+        float* slot = amax_x + sl * kEpiWG * BM;
         slot[wg * BM + rit] = amax;
         mbar_arrive(&xbar[sl]);
         const bool xok = mbar_wait_bounded(&xbar[sl], (it >> 1) & 1, abort_flag, kWaitNs);
@@ -320,13 +326,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           raise_abort(abort_flag, p.err);
           break;
         }
-        amax = fmaxf(amax, slot[(wg ^ 1) * BM + rit]);
+#pragma unroll
+        for (int o = 0; o < kEpiWG; ++o) amax = fmaxf(amax, slot[o * BM + rit]);
         const float sc = amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
         if (valid) {
-          uint8_t* dst = static_cast<uint8_t*>(p.C) + (size_t)(row0 + rit) * p.N + nt * 128 + wg * 64;
+          uint8_t* dst = static_cast<uint8_t*>(p.C) + (size_t)(row0 + rit) * p.N + nt * 128 + wg * 32;
           uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
+          for (int q = 0; q < 2; ++q) {
             uint32_t w[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -340,10 +347,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else if (valid) {
         __nv_bfloat16* dst =
-            static_cast<__nv_bfloat16*>(p.C) + (size_t)(row0 + rit) * p.N + nt * BN + wg * 128;
+            static_cast<__nv_bfloat16*>(p.C) + (size_t)(row0 + rit) * p.N + nt * BN + wg * CW;
         uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
+        for (int q = 0; q < CW / 8; ++q) {
           uint32_t w[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {

@@ -11,13 +11,14 @@
 // ceil(M/256) token tiles of equal size (multiples of 16), so ragged expert
 // loads cost at most 15 padding rows per tile instead of a 128-row tail.
 //
-// Epilogue (4 warps; warp w owns TMEM lanes 32*(w%4).. = weight rows):
+// Epilogue (8 warps; warp w owns TMEM lanes 32*(w%4).. = weight rows, and
+// every other 32-token chunk):
 //   SWIGLU  h[tok0+j, nt*128 + n] = bf16(SiLU(D_gate[n,j]) * D_up[n,j])
 //   STORE   y[tok0+j, nt*256 + n] = bf16(D0[n,j]), y[.., nt*256+128+n] = bf16(D1[n,j])
 // Values are transposed through a 2 KB shared-memory patch per warp so that
 // global stores are 16-byte vectors along token rows.
 //
-// Roles: warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer, warps 2-5
+// Roles: warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer, warps 2-9
 // epilogue.  3 shared-memory stages of 64 KB; one TMEM accumulator pair
 // (512 columns).  Every wait is bounded (1 s) and reported through the
 // device error word.
@@ -37,7 +38,8 @@ constexpr int TMAX = 256;           // max token rows per tile (MMA N)
 constexpr int BK = 64;              // bf16 elements per 128-byte swizzle row
 constexpr int XBOX = 32;            // token rows per TMA box
 constexpr int STAGES = 3;
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;        // two warps per TMEM lane quarter, alternating token chunks
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kMaxGroups = 1024;
 constexpr uint64_t kWaitNs = 1000000000ull;
 constexpr uint32_t TMEM_COLS = 512;
@@ -46,8 +48,8 @@ constexpr int W_BYTES = WROWS * BK * 2;       // 32 KB
 constexpr int X_BYTES = TMAX * BK * 2;        // 32 KB
 constexpr int XBOX_BYTES = XBOX * BK * 2;     // 4 KB
 constexpr int OFF_X = STAGES * W_BYTES;
-constexpr int OFF_STAGE_OUT = OFF_X + STAGES * X_BYTES;   // 4 warps x 2 KB transpose patches
-constexpr int OFF_BAR = OFF_STAGE_OUT + 4 * 2048;
+constexpr int OFF_STAGE_OUT = OFF_X + STAGES * X_BYTES;   // one 2 KB transpose patch per epilogue warp
+constexpr int OFF_BAR = OFF_STAGE_OUT + kEpiWarps * 2048;
 constexpr int N_BARS = 2 * STAGES + 3;
 constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
 constexpr int OFF_TAB = OFF_MISC + 16;
@@ -105,7 +107,8 @@ __device__ __forceinline__ void raise_abort(volatile int* abort, int* err) {
   atomicOr(err, ERR_GEMM_TIMEOUT);
 }
 
-__device__ __forceinline__ float silu_f(float x) { return x / (1.0f + __expf(-x)); }
+// SiLU for a bf16 result: fast exponential and division are well inside bf16 rounding.
+__device__ __forceinline__ float silu_f(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
 
 template <bool SWIGLU>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -135,7 +138,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     mbar_init(tfull, 1);
-    mbar_init(tempty, 128);
+    mbar_init(tempty, 32 * kEpiWarps);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -267,7 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ---------------------------------------------------------------- epilogue
     const int q = warp & 3;                       // TMEM lane quarter
-    const int n = q * 32 + lane;                  // weight row inside each 128-row half
+    const int ch = (warp - 2) >> 2;               // which alternate 32-token chunks this warp takes
     uint16_t* patch = reinterpret_cast<uint16_t*>(sOut + (warp - 2) * 2048);   // [32 tok][32 col]
     uint32_t tphase = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
@@ -281,7 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t tl = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
       const int nch = (count + 31) / 32;
-      for (int c = 0; c < nch; ++c) {
+      for (int c = ch; c < nch; c += 2) {
         uint32_t r0[32], r1[32];
         tmem_ld_32x32b_x32(tl + c * 32, r0);
         tmem_ld_32x32b_x32(tl + 256 + c * 32, r1);
