@@ -201,6 +201,28 @@ moe_status moe_quantize_128x128(const void* w, int groups, int rows, int cols,
                                 uint8_t* q, float* scale, void* stream);
 
 /* ------------------------------------------------------------------------
+ * moe_permute_noalloc - moe_permute for callers that cannot allocate device
+ * memory.  The DeepSeek-V3 pages have no counterpart; it exists for callers
+ * that run inside a host framework which owns every device allocation (a
+ * caching allocator or fixed arena it does not expose) or in loops that must
+ * not allocate once started, and so cannot pass a workspace.
+ *
+ * Same arguments, layouts and results as moe_permute, without the workspace.
+ * Its scratch is a static 1 MiB device array inside the library (held by
+ * every GPU that loads libmoe.so until the process exits), so it accepts
+ * only 2 * ceil(T/256) * N_r * 4 bytes <= 1 MiB (T <= 131072 at N_r = 256);
+ * larger problems get MOE_ERR_UNSUPPORTED and launch nothing.  The first
+ * call on a device looks up the array's device address (make it before any
+ * stream capture).  Every call uses the same array: calls whose work
+ * overlaps on the GPU (other streams or host threads) race on it.
+ * ------------------------------------------------------------------------ */
+moe_status moe_permute_noalloc(const void* u, const float* u_scale, moe_dtype dt,
+                               const int32_t* topk_idx, int T, int d, int N_r, int K,
+                               void* x_perm, float* x_scale,
+                               int32_t* offsets, int32_t* perm_src, int32_t* inv_row,
+                               void* stream);
+
+/* ------------------------------------------------------------------------
  * moe_device_status - synchronises the current device, then returns (and
  * clears) the library's device-side error word: 0 if no kernel gave up a
  * bounded wait since the last call, else a bit set naming the kernel.

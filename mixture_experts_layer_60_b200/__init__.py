@@ -15,7 +15,7 @@ import torch
 
 __all__ = [
     "MoeError", "lib", "LIB_PATH", "SYMBOLS",
-    "moe_route", "moe_permute", "moe_expert_ffn", "moe_expert_gate_up", "moe_expert_down", "moe_combine", "moe_bias_update",
+    "moe_route", "moe_permute", "moe_permute_noalloc", "moe_expert_ffn", "moe_expert_gate_up", "moe_expert_down", "moe_combine", "moe_bias_update",
     "moe_quantize_1x128", "moe_quantize_128x128", "moe_device_status",
     "moe_route_workspace_size", "moe_permute_workspace_size", "moe_expert_ffn_workspace_size",
 ]
@@ -47,6 +47,7 @@ SYMBOLS = {
     "moe_quantize_1x128": (_i, [_vp, _i, _i, _vp, _vp, _vp]),
     "moe_quantize_128x128": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp]),
     "moe_device_status": (_i, [ctypes.POINTER(_i)]),
+    "moe_permute_noalloc": (_i, [_vp, _vp, _i, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
 }
 
 
@@ -140,6 +141,18 @@ def moe_permute(u, topk_idx, N_r, x_perm, offsets, perm_src, inv_row, workspace,
     _check(lib().moe_permute(_p(u), _p(u_scale), _dt(u), _p(topk_idx), T, d, N_r, K, _p(x_perm),
                              _p(x_scale), _p(offsets), _p(perm_src), _p(inv_row), _p(workspace),
                              _nbytes(workspace), _s(stream)))
+
+
+def moe_permute_noalloc(u, topk_idx, N_r, x_perm, offsets, perm_src, inv_row, u_scale=None,
+                        x_scale=None, stream=None):
+    """moe_permute without a workspace, for callers that cannot allocate device
+    memory: the library keeps a static 1 MiB scratch array per GPU (see
+    include/moe.h for the size limit and the rule that overlapping calls race)."""
+    T, d = u.shape
+    K = topk_idx.shape[1]
+    _check(lib().moe_permute_noalloc(_p(u), _p(u_scale), _dt(u), _p(topk_idx), T, d, N_r, K,
+                                     _p(x_perm), _p(x_scale), _p(offsets), _p(perm_src),
+                                     _p(inv_row), _s(stream)))
 
 
 def moe_expert_ffn(x, offsets, W_gate_up, W_down, y, workspace, x_scale=None,

@@ -190,3 +190,100 @@ moe_status launch_permute(const void* u, const float* u_scale, int elem_bytes, c
 }
 
 }  // namespace moe
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of moe_permute.
+//
+// Some callers cannot hand this library a workspace: code that runs inside a
+// host framework which owns every device allocation (a caching allocator or a
+// fixed arena it does not expose), or a loop that must not allocate device
+// memory once it has started.  For them, the permutation's scratch (the
+// per-chunk expert histograms and first rows, 2 * ceil(T/256) * N_r int32)
+// lives in a file-scope device array of kNoAllocScratchBytes that every GPU
+// loading this library holds until the process exits.
+//
+// In host code the array's name is only a host-side handle, so its device
+// address is looked up once per device (cudaGetSymbolAddress, with that
+// device current) on the first call there; make that first call before any
+// stream capture.  All calls share the array: two calls whose work overlaps
+// on the GPU (different streams, or different host threads) race on it.
+// Every word a call reads is first written by the same call, so nothing has
+// to be cleared between calls.
+namespace moe {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 1u << 20;   // 1 MiB: T up to 131072 at N_r = 256
+constexpr int kNoAllocMaxDevices = 64;
+
+__device__ __align__(256) unsigned char g_permute_scratch[kNoAllocScratchBytes];
+void* g_permute_scratch_addr[kNoAllocMaxDevices] = {nullptr};
+
+moe_status permute_scratch_address(void** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_check(e, "moe_permute_noalloc: cudaGetDevice");
+  if (dev < 0 || dev >= kNoAllocMaxDevices)
+    return fail(MOE_ERR_UNSUPPORTED, "moe_permute_noalloc: device %d out of range", dev);
+  if (!g_permute_scratch_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_permute_scratch);
+    if (e != cudaSuccess || !p)
+      return cuda_check(e != cudaSuccess ? e : cudaErrorInvalidSymbol,
+                        "moe_permute_noalloc: cudaGetSymbolAddress of the static scratch");
+    g_permute_scratch_addr[dev] = p;
+  }
+  *out = g_permute_scratch_addr[dev];
+  return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" moe_status moe_permute_noalloc(const void* u, const float* u_scale, moe_dtype dt,
+                                          const int32_t* topk_idx, int T, int d, int N_r, int K,
+                                          void* x_perm, float* x_scale, int32_t* offsets,
+                                          int32_t* perm_src, int32_t* inv_row, void* stream) {
+  using namespace moe;
+  const int eb = dt == MOE_F32 ? 4 : dt == MOE_BF16 ? 2 : dt == MOE_E4M3 ? 1 : 0;
+  if (eb == 0) return fail(MOE_ERR_UNSUPPORTED, "moe_permute_noalloc: unknown dtype %d", (int)dt);
+  if (T < 0 || d <= 0 || N_r <= 0 || K <= 0)
+    return fail(MOE_ERR_INVALID_ARG, "moe_permute_noalloc: bad sizes T=%d d=%d N_r=%d K=%d", T,
+                d, N_r, K);
+  if (N_r > 1024 || K > N_r)
+    return fail(MOE_ERR_UNSUPPORTED, "moe_permute_noalloc: need 1 <= K <= N_r <= 1024");
+  if ((8LL * N_r + 256LL * K) * 4 > 200 * 1024)
+    return fail(MOE_ERR_UNSUPPORTED,
+                "moe_permute_noalloc: K=%d with N_r=%d exceeds the rank kernel's shared memory", K,
+                N_r);
+  if (((size_t)d * eb) % 16 != 0)
+    return fail(MOE_ERR_UNSUPPORTED, "moe_permute_noalloc: a row must be a multiple of 16 bytes");
+  if (!offsets) return fail(MOE_ERR_INVALID_ARG, "moe_permute_noalloc: null offsets");
+  if (T > 0 && !(u && topk_idx && x_perm && perm_src && inv_row))
+    return fail(MOE_ERR_INVALID_ARG, "moe_permute_noalloc: null pointer");
+  if (dt == MOE_E4M3) {
+    if (d % 128) return fail(MOE_ERR_UNSUPPORTED, "moe_permute_noalloc: e4m3 needs d %% 128 == 0");
+    if (T > 0 && !(u_scale && x_scale))
+      return fail(MOE_ERR_INVALID_ARG, "moe_permute_noalloc: e4m3 needs u_scale and x_scale");
+  } else if (u_scale || x_scale) {
+    return fail(MOE_ERR_INVALID_ARG, "moe_permute_noalloc: scales are only for MOE_E4M3");
+  }
+  if (reinterpret_cast<uintptr_t>(u) % 16 || reinterpret_cast<uintptr_t>(x_perm) % 16)
+    return fail(MOE_ERR_INVALID_ARG, "moe_permute_noalloc: u and x_perm must be 16-byte aligned");
+  const size_t need = T > 0 ? permute_ws_bytes(T, N_r) : 0;
+  if (need > kNoAllocScratchBytes)
+    return fail(MOE_ERR_UNSUPPORTED,
+                "moe_permute_noalloc: T=%d, N_r=%d needs %zu bytes of scratch, more than the "
+                "%zu-byte static array; use moe_permute with a workspace",
+                T, N_r, need, kNoAllocScratchBytes);
+  if (!device_is_sm100())
+    return fail(MOE_ERR_UNSUPPORTED, "libmoe kernels need an sm_100 (B200) device");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (T == 0)
+    return cuda_check(cudaMemsetAsync(offsets, 0, (size_t)(N_r + 1) * sizeof(int32_t), s),
+                      "zero offsets");
+  void* scratch = nullptr;
+  moe_status st = permute_scratch_address(&scratch);
+  if (st != MOE_OK) return st;
+  return launch_permute(u, dt == MOE_E4M3 ? u_scale : nullptr, eb, topk_idx, T, d, N_r, K, x_perm,
+                        dt == MOE_E4M3 ? x_scale : nullptr, offsets, perm_src, inv_row, scratch, s);
+}
