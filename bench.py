@@ -124,6 +124,15 @@ def roofline_layer(cfg, p):
     return cfg.T / t, flops, bytes_
 
 
+def _load_balance(load_hist, cfg):
+    """max/mean expert load of every timed step (mean = T*K/N_r)."""
+    h = load_hist.float().cpu()
+    r = (h.max(dim=1).values / (cfg.T * cfg.K / cfg.N_r)).tolist()
+    return {"max_over_mean_per_step": [round(x, 3) for x in r], "first": round(r[0], 3),
+            "last": round(r[-1], 3), "steps": len(r),
+            "note": "fresh tokens every step; bias updated after every step (gamma 0.001)"}
+
+
 def cpu_oracle_sample(cfg, w, n_tokens, seed=0):
     """Times the CPU oracle on the full route of `n_tokens` tokens and their
     whole layer (expert-major, weights read from the device expert by expert)."""
@@ -238,6 +247,13 @@ def run_ours(args, cfg, ws, rank, local):
         raise RuntimeError("a kernel reported a bounded-wait timeout during warm-up")
 
     # ---- device-resident timed region
+    # Multi-step configurations draw fresh tokens every step (generated before
+    # the timed region) and record each step's per-expert load.
+    multi = cfg.steps > 1
+    if multi:
+        from mixture_experts_layer_60_b200.synth import step_u
+        u_steps = [step_u(cfg, i, dev) for i in range(args.steps)]
+        load_hist = torch.empty(args.steps, cfg.N_r, dtype=torch.int32, device=dev)
     gu_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
              for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -247,7 +263,11 @@ def run_ours(args, cfg, ws, rank, local):
     torch.cuda.synchronize()
     t0.record(stream)
     for i in range(args.steps):
-        step(gu_ev[i])
+        if multi:
+            step(gu_ev[i], u_in=u_steps[i])
+            load_hist[i].copy_(layer.counts)
+        else:
+            step(gu_ev[i])
     t1.record(stream)
     torch.cuda.synchronize()
     if group is not None:
@@ -330,6 +350,7 @@ def run_ours(args, cfg, ws, rank, local):
                 "h2d_bytes_per_step": u.numel() * u.element_size(),
                 "d2h_bytes_per_step": u.numel() * u.element_size()},
         "gpu_launches": gpu_launches_per_step(cfg) * args.steps,
+        "load_balance": _load_balance(load_hist, cfg) if multi else None,
         "device_status": status,
         "cpu_baseline": cpu,
     }

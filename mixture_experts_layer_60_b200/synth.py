@@ -40,6 +40,16 @@ def _normal(gen, shape, std, device, dtype):
     return x.to(dtype)
 
 
+def zipf_lambda_v3():
+    """Centroid norms of the skewed-load V3 recipe (fitted once, stored as data;
+    see data/zipf_lambda_v3.json for the target and achieved popularity)."""
+    import json
+    import os
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "data", "zipf_lambda_v3.json")
+    with open(path) as f:
+        return json.load(f)["lambda"]
+
+
 def make_layer_inputs(cfg: LayerConfig, device="cuda", T: int | None = None,
                       zipf_lambda=None) -> dict:
     """All tensors of one configuration, generated on `device`.
@@ -78,6 +88,8 @@ def make_layer_inputs(cfg: LayerConfig, device="cuda", T: int | None = None,
         mask = torch.rand(T, d, generator=gen, device=device) < cfg.outlier_frac
         u32 = torch.where(mask, u32 * cfg.outlier_scale, u32)
     out["u"] = u32.to(dt)
+    if zipf_lambda is None and cfg.zipf > 0:
+        zipf_lambda = zipf_lambda_v3()
     if zipf_lambda is not None:
         lam = torch.as_tensor(zipf_lambda, dtype=torch.float32, device=device)
         E = out["E"]

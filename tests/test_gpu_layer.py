@@ -139,3 +139,38 @@ def test_bias_update_steps_and_resume():
     h_re = a_last.forward(step_u(cfg, 5, "cuda", T=512))
     torch.cuda.synchronize()
     assert torch.equal(h2, h_re)
+
+
+def test_skewed_load_steps_route_and_balance():
+    """Skewed-popularity V3 shape: each step's routing equals the oracle's
+    (with the bias the GPU carries), the bias follows the oracle's rule bit for
+    bit from the GPU's load, the load is skewed at the start, and a run of
+    4 + 4 steps with the bias saved and reloaded equals 8 steps bit for bit."""
+    from dataclasses import replace
+    cfg = replace(CONFIGS["v3_zipf_bf16"], T=1024)
+    w = make_layer_inputs(cfg, "cuda")
+    a = MoELayer(cfg, w)
+    E = f64(w["E"])
+    first_ratio = None
+    for s in range(8):
+        u = step_u(cfg, s, "cuda")
+        b_before = a.b.cpu().numpy().copy()
+        a.step(u)
+        torch.cuda.synchronize()
+        ref = O.route(f64(u), E, b_before, cfg.K)
+        check_routing(a.topk_idx.cpu().numpy(), a.topk_gate.cpu().numpy(),
+                      a.counts.cpu().numpy(), ref, cfg.K)
+        np.testing.assert_array_equal(a.b.cpu().numpy(),
+                                      O.bias_update(b_before, a.counts.cpu().numpy(), cfg.T, cfg.K))
+        if s == 0:
+            first_ratio = a.counts.max().item() / (cfg.T * cfg.K / cfg.N_r)
+    assert first_ratio > 4.0, first_ratio          # the recipe does skew the load
+    b_half = MoELayer(cfg, w)
+    for s in range(4):
+        b_half.step(step_u(cfg, s, "cuda"))
+    w2 = dict(w, b=b_half.b.clone())
+    b2 = MoELayer(cfg, w2)
+    for s in range(4, 8):
+        b2.step(step_u(cfg, s, "cuda"))
+    torch.cuda.synchronize()
+    assert torch.equal(b2.b, a.b)
