@@ -105,6 +105,16 @@ def dist_setup(n_gpus):
     return ws, rank, local
 
 
+# DRAM bytes (read + write) of one routed gate/up launch, from one ncu capture
+# of a scaled-down case (32 experts, ~256 tokens each) multiplied by the units
+# processed (both weights and rows scale x8 to the full 256-expert launch).
+# Must be re-taken (or set to None) whenever that kernel changes.
+MEASURED_GATE_UP_TRAFFIC = {
+    "v3_bf16": (2.102503e9 + 0.03406464e9) * 8,   # profiles/ws_gemm_gateup_v3shape_32experts.md
+    "v3_fp8": (1.087124e9 + 0.044804864e9) * 8,   # profiles/fp8_gemm_gateup_v3shape_32experts.md
+}
+
+
 def gpu_launches_per_step(cfg):
     # route: logits GEMM + top-K; permute: 4; routed FFN: 2; shared FFN: 2 each;
     # combine: 1; bias update: 1; FP8: + activation quantiser
@@ -321,8 +331,11 @@ def run_ours(args, cfg, ws, rank, local):
     roof_tps, flops, bytes_ = roofline_layer(cfg, p)
     # dominant kernel: the routed gate/up grouped GEMM
     gu_flops = 2.0 * cfg.T * cfg.K * cfg.d * 2 * cfg.I
-    timed_s = ms / 1e3
-    sustained = timed_s >= 1.0
+    el = 1 if cfg.dtype == "e4m3" else 2
+    gu_bytes = (cfg.N_r * 2 * cfg.I * cfg.d + cfg.T * cfg.K * (cfg.d + cfg.I)) * el
+    # The kernel is timed inside a loop of whole layer steps at the power cap:
+    # the sustained bf16 figure is the matching denominator.
+    sustained = True
     pk = p["bf16_sustained"] if sustained else p["bf16"]
     if cfg.dtype == "e4m3":
         pk *= 2
@@ -342,7 +355,9 @@ def run_ours(args, cfg, ws, rank, local):
                      "achieved": achieved, "peak": pk, "unit": "TFLOP/s", "frac": achieved / pk,
                      "peak_kind": ("sustained" if sustained else "burst") + " bf16 of " +
                                   p["source"] + (" x2 (FP8 nominal ratio)" if cfg.dtype == "e4m3" else ""),
-                     "kernel_ms": gu_ms, "flops_per_launch": gu_flops, "traffic": None},
+                     "kernel_ms": gu_ms, "flops_per_launch": gu_flops,
+                     "traffic": MEASURED_GATE_UP_TRAFFIC.get(cfg.name),
+                     "algorithmic_bytes": gu_bytes},
         "layer_roofline": {"tokens_per_s": roof_tps, "frac": value / ws / roof_tps,
                            "flops_per_step": flops, "bytes_per_step": bytes_},
         "clocks": clk,
