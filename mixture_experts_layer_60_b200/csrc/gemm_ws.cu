@@ -36,7 +36,7 @@ using namespace sm100;
 constexpr int WROWS = 256;          // weight rows per tile (two M=128 MMAs)
 constexpr int TMAX = 256;           // max token rows per tile (MMA N)
 constexpr int BK = 64;              // bf16 elements per 128-byte swizzle row
-constexpr int XBOX = 32;            // token rows per TMA box
+constexpr int XBOX = 64;            // token rows per TMA box (fewer, larger TMA operations)
 constexpr int STAGES = 3;
 constexpr int kEpiWarps = 8;        // two warps per TMEM lane quarter, alternating token chunks
 constexpr int kThreads = 64 + 32 * kEpiWarps;
@@ -46,7 +46,7 @@ constexpr uint32_t TMEM_COLS = 512;
 
 constexpr int W_BYTES = WROWS * BK * 2;       // 32 KB
 constexpr int X_BYTES = TMAX * BK * 2;        // 32 KB
-constexpr int XBOX_BYTES = XBOX * BK * 2;     // 4 KB
+constexpr int XBOX_BYTES = XBOX * BK * 2;     // 8 KB
 constexpr int OFF_X = STAGES * W_BYTES;
 constexpr int OFF_STAGE_OUT = OFF_X + STAGES * X_BYTES;   // one 2 KB transpose patch per epilogue warp
 constexpr int OFF_BAR = OFF_STAGE_OUT + kEpiWarps * 2048;
