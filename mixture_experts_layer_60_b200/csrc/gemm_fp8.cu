@@ -92,6 +92,24 @@ __device__ __forceinline__ void raise_abort(volatile int* abort, int* err) {
   atomicOr(err, ERR_GEMM_FP8_TIMEOUT);
 }
 
+// Packed pair of float32 in one 64-bit register, and the sm_100 paired FMA
+// (two IEEE fused multiply-adds per instruction, each rounded like fmaf).
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+// c += (x0, x1) * s2, x0/x1 the raw bits of two float32 TMEM words
+__device__ __forceinline__ uint64_t fma2_bits(uint32_t x0, uint32_t x1, uint64_t s2, uint64_t c) {
+  asm("{\n\t.reg .b64 t;\n\tmov.b64 t, {%1, %2};\n\tfma.rn.f32x2 %0, t, %3, %0;\n\t}"
+      : "+l"(c)
+      : "r"(x0), "r"(x1), "l"(s2));
+  return c;
+}
+
 __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
   return (uint32_t)__nv_cvt_float_to_fp8(a, __NV_SATFINITE, __NV_E4M3) |
          ((uint32_t)__nv_cvt_float_to_fp8(b, __NV_SATFINITE, __NV_E4M3) << 8) |
@@ -274,9 +292,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         col0 = wg * CW;
         col1 = wg * CW + 32;
       }
-      float acc[CW];
+      uint64_t acc2[CW / 2];   // accumulator pairs: columns (2i, 2i+1) of this thread's chunks
 #pragma unroll
-      for (int i = 0; i < CW; ++i) acc[i] = 0.f;
+      for (int i = 0; i < CW / 2; ++i) acc2[i] = 0ull;
       float sa = sa_row[0];
       for (int kb = 0; kb < nk; ++kb) {
         const float sa_next = (kb + 1 < nk) ? sa_row[kb + 1] : 0.f;
@@ -300,14 +318,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             mbar_arrive(&pempty[pb]);   // partial read: the MMA may overwrite it
           }
-          const float sc = c < 2 ? s0 : s1;
+          const uint64_t sc2 = c < 2 ? f2_pack(s0, s0) : f2_pack(s1, s1);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) acc[c * 16 + j] = fmaf(__uint_as_float(r[j]), sc, acc[c * 16 + j]);
+          for (int i = 0; i < 8; ++i) acc2[c * 8 + i] = fma2_bits(r[2 * i], r[2 * i + 1], sc2, acc2[c * 8 + i]);
         }
         if (++pb == 2) { pb = 0; pphase ^= 1; }
         sa = sa_next;
       }
       if (!ok) break;
+      float acc[CW];
+#pragma unroll
+      for (int i = 0; i < CW / 2; ++i) f2_unpack(acc2[i], acc[2 * i], acc[2 * i + 1]);
       if (SWIGLU) {
         float amax = 0.f;
 #pragma unroll
