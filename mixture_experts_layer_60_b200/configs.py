@@ -51,6 +51,10 @@ CONFIGS = {
                            dtype="bf16", seed=2),
     "v3_zipf_bf16": LayerConfig("v3_zipf_bf16", T=8192, d=7168, N_r=256, K=8, N_s=1, I=2048,
                                 dtype="bf16", seed=2, zipf=1.2, steps=100),
+    # decode-shaped batch at the V3 shape: ~8 tokens per expert, so the expert
+    # GEMMs stream all weights for little arithmetic (HBM-bound)
+    "v3_decode_bf16": LayerConfig("v3_decode_bf16", T=256, d=7168, N_r=256, K=8, N_s=1, I=2048,
+                                  dtype="bf16", seed=5),
     "v3_fp8": LayerConfig("v3_fp8", T=16384, d=7168, N_r=256, K=8, N_s=1, I=2048,
                           dtype="e4m3", seed=4, outlier_frac=0.001, outlier_scale=50.0),
 }

@@ -86,6 +86,11 @@ def test_layer_fp8_small_full():
     _run(cfg)
 
 
+def test_layer_v3_decode_sampled():
+    """Decode-shaped batch (T = 256, ~8 tokens per expert): 16-row token tiles."""
+    _run(CONFIGS["v3_decode_bf16"], sample=16, seed_sample=3)
+
+
 def test_layer_all_tokens_one_expert():
     """K = 1 and a dominant bias: one group holds every token, the others are empty."""
     cfg = CONFIGS["small_bf16"]
