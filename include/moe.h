@@ -87,6 +87,23 @@ moe_status moe_route(const void* u, const void* E, moe_dtype dt, const float* b,
                      void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * moe_route_grouped - moe_route with a group limit: experts form n_groups
+ * groups of N_r/n_groups consecutive indices and each token may only select
+ * experts of its topk_groups best groups (the per-token node limit of
+ * "DeepSeek V3 & R1 論文研究", section Cross-Node All-to-All, which gives
+ * only the limit).  A group's score is its largest key s+b (this library's
+ * reading); ties keep the lower group index.  Same arguments, outputs and
+ * workspace as moe_route, plus
+ *   n_groups     1..32, dividing N_r
+ *   topk_groups  1..n_groups, with topk_groups * N_r/n_groups >= K
+ * moe_route is moe_route_grouped with n_groups = topk_groups = 1.
+ * ------------------------------------------------------------------------ */
+moe_status moe_route_grouped(const void* u, const void* E, moe_dtype dt, const float* b,
+                             int T, int d, int N_r, int K, int n_groups, int topk_groups,
+                             int32_t* topk_idx, float* topk_gate, int32_t* counts,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * moe_permute - group the T*K (token, slot) pairs by expert and copy the
  * token rows into that order (the dispatch step that feeds FFN^(r)_i in the
  * h'-equation).  Inside an expert's group tokens keep ascending order.

@@ -15,7 +15,7 @@ import torch
 
 __all__ = [
     "MoeError", "lib", "LIB_PATH", "SYMBOLS",
-    "moe_route", "moe_permute", "moe_permute_noalloc", "moe_expert_ffn", "moe_expert_gate_up", "moe_expert_down", "moe_combine", "moe_bias_update",
+    "moe_route", "moe_route_grouped", "moe_permute", "moe_permute_noalloc", "moe_expert_ffn", "moe_expert_gate_up", "moe_expert_down", "moe_combine", "moe_bias_update",
     "moe_quantize_1x128", "moe_quantize_128x128", "moe_device_status",
     "moe_route_workspace_size", "moe_permute_workspace_size", "moe_expert_ffn_workspace_size",
 ]
@@ -35,6 +35,8 @@ SYMBOLS = {
     "moe_status_string": (ctypes.c_char_p, [_i]),
     "moe_route_workspace_size": (_sz, [_i, _i]),
     "moe_route": (_i, [_vp, _vp, _i, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_route_grouped": (_i, [_vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _sz,
+                               _vp]),
     "moe_permute_workspace_size": (_sz, [_i, _i]),
     "moe_permute": (_i, [_vp, _vp, _i, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_expert_ffn_workspace_size": (_sz, [_i, _i, _i]),
@@ -132,6 +134,14 @@ def moe_route(u, E, b, K, topk_idx, topk_gate, counts, workspace, stream=None):
     _check(lib().moe_route(_p(u), _p(E), _dt(u), _p(b), T, d, E.shape[0], K, _p(topk_idx),
                            _p(topk_gate), _p(counts), _p(workspace), _nbytes(workspace),
                            _s(stream)))
+
+
+def moe_route_grouped(u, E, b, K, n_groups, topk_groups, topk_idx, topk_gate, counts, workspace,
+                      stream=None):
+    T, d = u.shape
+    _check(lib().moe_route_grouped(_p(u), _p(E), _dt(u), _p(b), T, d, E.shape[0], K, n_groups,
+                                   topk_groups, _p(topk_idx), _p(topk_gate), _p(counts),
+                                   _p(workspace), _nbytes(workspace), _s(stream)))
 
 
 def moe_permute(u, topk_idx, N_r, x_perm, offsets, perm_src, inv_row, workspace,

@@ -25,6 +25,8 @@ class LayerConfig:
     steps: int = 1        # forward + bias-update steps per run
     outlier_frac: float = 0.0
     outlier_scale: float = 1.0
+    n_groups: int = 1        # > 1: expert groups for the per-token group (node) limit
+    topk_groups: int = 1     # groups a token may use when n_groups > 1
 
     @property
     def R(self):
@@ -55,6 +57,9 @@ CONFIGS = {
     # GEMMs stream all weights for little arithmetic (HBM-bound)
     "v3_decode_bf16": LayerConfig("v3_decode_bf16", T=256, d=7168, N_r=256, K=8, N_s=1, I=2048,
                                   dtype="bf16", seed=5),
+    # V3 shape with the node limit: 8 groups of 32 experts, at most 4 per token
+    "v3_grouped_bf16": LayerConfig("v3_grouped_bf16", T=8192, d=7168, N_r=256, K=8, N_s=1,
+                                   I=2048, dtype="bf16", seed=6, n_groups=8, topk_groups=4),
     "v3_fp8": LayerConfig("v3_fp8", T=16384, d=7168, N_r=256, K=8, N_s=1, I=2048,
                           dtype="e4m3", seed=4, outlier_frac=0.001, outlier_scale=50.0),
 }

@@ -79,24 +79,35 @@ const char* moe_status_string(moe_status s) {
 
 size_t moe_route_workspace_size(int T, int N_r) { return route_ws(T, N_r); }
 
-moe_status moe_route(const void* u, const void* E, moe_dtype dt, const float* b, int T, int d,
-                     int N_r, int K, int32_t* topk_idx, float* topk_gate, int32_t* counts,
-                     void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+moe_status route_impl(const char* who, const void* u, const void* E, moe_dtype dt, const float* b,
+                      int T, int d, int N_r, int K, int n_groups, int topk_groups,
+                      int32_t* topk_idx, float* topk_gate, int32_t* counts, void* workspace,
+                      size_t workspace_bytes, void* stream) {
   clear_last_error();
   MOE_REQUIRE(dt == MOE_F32 || dt == MOE_BF16, MOE_ERR_UNSUPPORTED,
-              "moe_route: dtype must be MOE_F32 or MOE_BF16");
+              "%s: dtype must be MOE_F32 or MOE_BF16", who);
   MOE_REQUIRE(T >= 0 && d > 0 && N_r > 0 && K > 0, MOE_ERR_INVALID_ARG,
-              "moe_route: bad sizes T=%d d=%d N_r=%d K=%d", T, d, N_r, K);
+              "%s: bad sizes T=%d d=%d N_r=%d K=%d", who, T, d, N_r, K);
   MOE_REQUIRE(N_r <= 1024 && K <= N_r, MOE_ERR_UNSUPPORTED,
-              "moe_route: need 1 <= K <= N_r <= 1024 (K=%d N_r=%d)", K, N_r);
-  MOE_REQUIRE(d % 64 == 0, MOE_ERR_UNSUPPORTED, "moe_route: d=%d must be a multiple of 64", d);
-  MOE_REQUIRE(E && b && counts, MOE_ERR_INVALID_ARG, "moe_route: null pointer");
+              "%s: need 1 <= K <= N_r <= 1024 (K=%d N_r=%d)", who, K, N_r);
+  MOE_REQUIRE(n_groups >= 1 && n_groups <= 32 && N_r % n_groups == 0 && topk_groups >= 1 &&
+                  topk_groups <= n_groups,
+              MOE_ERR_INVALID_ARG,
+              "%s: need 1 <= topk_groups <= n_groups <= 32 with N_r %% n_groups == 0", who);
+  MOE_REQUIRE((long long)topk_groups * (N_r / n_groups) >= K, MOE_ERR_INVALID_ARG,
+              "%s: the kept groups hold fewer than K experts", who);
+  MOE_REQUIRE(d % 64 == 0, MOE_ERR_UNSUPPORTED, "%s: d=%d must be a multiple of 64", who, d);
+  MOE_REQUIRE(E && b && counts, MOE_ERR_INVALID_ARG, "%s: null pointer", who);
   MOE_REQUIRE(T == 0 || (u && topk_idx && topk_gate && workspace), MOE_ERR_INVALID_ARG,
-              "moe_route: null pointer");
+              "%s: null pointer", who);
   MOE_REQUIRE(workspace_bytes >= route_ws(T, N_r), MOE_ERR_WORKSPACE,
-              "moe_route: workspace %zu < %zu bytes", workspace_bytes, route_ws(T, N_r));
+              "%s: workspace %zu < %zu bytes", who, workspace_bytes, route_ws(T, N_r));
   MOE_REQUIRE(T == 0 || reinterpret_cast<uintptr_t>(workspace) % 256 == 0, MOE_ERR_INVALID_ARG,
-              "moe_route: workspace must be 256-byte aligned");
+              "%s: workspace must be 256-byte aligned", who);
   MOE_TRY(check_device());
   cudaStream_t s = as_stream(stream);
   MOE_TRY(cuda_check(cudaMemsetAsync(counts, 0, (size_t)N_r * sizeof(int32_t), s), "zero counts"));
@@ -107,7 +118,26 @@ moe_status moe_route(const void* u, const void* E, moe_dtype dt, const float* b,
   } else {
     MOE_TRY(launch_logits_simt(u, E, dt, T, d, N_r, logits, s));
   }
-  return launch_topk(logits, b, T, N_r, K, topk_idx, topk_gate, counts, s);
+  return launch_topk(logits, b, T, N_r, K, n_groups, topk_groups, topk_idx, topk_gate, counts, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_route(const void* u, const void* E, moe_dtype dt, const float* b, int T, int d,
+                     int N_r, int K, int32_t* topk_idx, float* topk_gate, int32_t* counts,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+  return route_impl("moe_route", u, E, dt, b, T, d, N_r, K, 1, 1, topk_idx, topk_gate, counts,
+                    workspace, workspace_bytes, stream);
+}
+
+moe_status moe_route_grouped(const void* u, const void* E, moe_dtype dt, const float* b, int T,
+                             int d, int N_r, int K, int n_groups, int topk_groups,
+                             int32_t* topk_idx, float* topk_gate, int32_t* counts,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+  return route_impl("moe_route_grouped", u, E, dt, b, T, d, N_r, K, n_groups, topk_groups,
+                    topk_idx, topk_gate, counts, workspace, workspace_bytes, stream);
 }
 
 size_t moe_permute_workspace_size(int T, int N_r) {

@@ -11,8 +11,10 @@ namespace moe {
 moe_status launch_logits_simt(const void* u, const void* E, moe_dtype dt, int T, int d,
                               int N_r, float* logits, cudaStream_t s);
 // sigmoid, biased top-K, gates, histogram (counts must be zeroed beforehand).
-moe_status launch_topk(const float* logits, const float* b, int T, int N_r, int K,
-                       int32_t* idx, float* gate, int32_t* counts, cudaStream_t s);
+// n_groups > 1 && topk_groups < n_groups restricts each token to its best groups.
+moe_status launch_topk(const float* logits, const float* b, int T, int N_r, int K, int n_groups,
+                       int topk_groups, int32_t* idx, float* gate, int32_t* counts,
+                       cudaStream_t s);
 
 // permute.cu -----------------------------------------------------------------
 size_t permute_ws_bytes(int T, int N_r);

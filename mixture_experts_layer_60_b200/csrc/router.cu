@@ -20,16 +20,26 @@ moe_status launch_logits_simt(const void* u, const void* E, moe_dtype dt, int T,
 // token's logits are read with coalesced loads.  K rounds of a warp-wide
 // arg-max with the order (key descending, index ascending) give the
 // selection in the documented output order.
+//
+// Group limit (n_groups > 1, topk_groups < n_groups): experts form n_groups
+// groups of N_r/n_groups consecutive indices; a group's score is its largest
+// key s+b; only the topk_groups best groups (ties to the lower group index)
+// stay eligible.  This is the per-token node limit of "DeepSeek V3 & R1
+// 論文研究", section Cross-Node All-to-All; the score rule is this library's
+// reading (the pages give only the limit).
 template <int V>
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits,
                                                    const float* __restrict__ bias, int T,
-                                                   int N_r, int K, int32_t* __restrict__ idx,
+                                                   int N_r, int K, int n_groups, int topk_groups,
+                                                   int32_t* __restrict__ idx,
                                                    float* __restrict__ gate,
                                                    int32_t* __restrict__ counts) {
   extern __shared__ int hist[];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int warps_per_block = blockDim.x >> 5;
+  const bool grouped = n_groups > 1 && topk_groups < n_groups;
+  float* wkeys = reinterpret_cast<float*>(hist + N_r) + warp * N_r;   // per-warp key staging
   for (int i = threadIdx.x; i < N_r; i += blockDim.x) hist[i] = 0;
   __syncthreads();
 
@@ -46,6 +56,36 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
       } else {
         sv[j] = 0.f;
         key[j] = -INFINITY;
+      }
+    }
+    if (grouped) {
+      const int gs = N_r / n_groups;
+#pragma unroll
+      for (int j = 0; j < V; ++j) {
+        const int e = j * 32 + lane;
+        if (e < N_r) wkeys[e] = key[j];
+      }
+      __syncwarp();
+      float gscore = -INFINITY;                       // lane g holds group g's score
+      if (lane < n_groups)
+        for (int i = 0; i < gs; ++i) gscore = fmaxf(gscore, wkeys[lane * gs + i]);
+      __syncwarp();
+      unsigned kept = 0;
+      for (int r = 0; r < topk_groups; ++r) {
+        float bk = (lane < n_groups && !((kept >> lane) & 1u)) ? gscore : -INFINITY;
+        int bg = lane < n_groups && !((kept >> lane) & 1u) ? lane : 0x7fffffff;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
+          const int og = __shfl_xor_sync(0xffffffffu, bg, off);
+          if (ok > bk || (ok == bk && og < bg)) { bk = ok; bg = og; }
+        }
+        kept |= 1u << bg;
+      }
+#pragma unroll
+      for (int j = 0; j < V; ++j) {
+        const int e = j * 32 + lane;
+        if (e < N_r && !((kept >> (e / gs)) & 1u)) key[j] = -INFINITY;
       }
     }
     float sum = 0.f;
@@ -93,18 +133,20 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
     if (hist[i]) atomicAdd(&counts[i], hist[i]);
 }
 
-moe_status launch_topk(const float* logits, const float* b, int T, int N_r, int K,
-                       int32_t* idx, float* gate, int32_t* counts, cudaStream_t s) {
+moe_status launch_topk(const float* logits, const float* b, int T, int N_r, int K, int n_groups,
+                       int topk_groups, int32_t* idx, float* gate, int32_t* counts,
+                       cudaStream_t s) {
   const int threads = 256;
   const int wpb = threads / 32;
   int blocks = (T + wpb - 1) / wpb;
   const int cap = 4 * sm_count();
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
-  const size_t smem = (size_t)N_r * sizeof(int);
+  const size_t smem = (size_t)N_r * sizeof(int) * (1 + threads / 32);   // histogram + key staging
   const int V = (N_r + 31) / 32;
 #define MOE_TOPK_CASE(v)                                                                    \
-  topk_kernel<v><<<blocks, threads, smem, s>>>(logits, b, T, N_r, K, idx, gate, counts); \
+  topk_kernel<v><<<blocks, threads, smem, s>>>(logits, b, T, N_r, K, n_groups, topk_groups, idx, \
+                                               gate, counts);                                  \
   break;
   switch (V <= 1 ? 1 : V <= 2 ? 2 : V <= 4 ? 4 : V <= 8 ? 8 : V <= 16 ? 16 : 32) {
     case 1: MOE_TOPK_CASE(1)

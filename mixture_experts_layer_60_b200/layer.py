@@ -11,7 +11,7 @@ from __future__ import annotations
 
 import torch
 
-from . import (MOE_BF16, MOE_E4M3, MOE_F32, moe_bias_update, moe_combine, moe_expert_down,
+from . import (MOE_BF16, MOE_E4M3, MOE_F32, moe_bias_update, moe_route_grouped, moe_combine, moe_expert_down,
                moe_expert_ffn, moe_expert_ffn_workspace_size, moe_expert_gate_up, moe_permute, moe_permute_workspace_size,
                moe_quantize_128x128, moe_quantize_1x128, moe_route, moe_route_workspace_size)
 from .configs import LayerConfig
@@ -86,8 +86,12 @@ class MoELayer:
         T = u.shape[0]
         if T != self.T_alloc:
             self._alloc(T)
-        moe_route(u, self.E, self.b, c.K, self.topk_idx, self.topk_gate, self.counts,
-                  self.route_ws, stream)
+        if c.n_groups > 1:
+            moe_route_grouped(u, self.E, self.b, c.K, c.n_groups, c.topk_groups, self.topk_idx,
+                              self.topk_gate, self.counts, self.route_ws, stream)
+        else:
+            moe_route(u, self.E, self.b, c.K, self.topk_idx, self.topk_gate, self.counts,
+                      self.route_ws, stream)
         if self.fp8:
             moe_quantize_1x128(u, self.u_q, self.u_s, stream)
             moe_permute(self.u_q, self.topk_idx, c.N_r, self.x_perm, self.offsets, self.perm_src,

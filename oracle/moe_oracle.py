@@ -29,6 +29,9 @@ Readings taken where the page is silent (each listed again in the design doc):
       T*K/N_r, in integers (counts*N_r vs T*K); equal load leaves b unchanged.
   R5  FFN_i is SwiGLU: W_down (SiLU(W_gate x) * (W_up x)), SiLU(z) = z / (1 + e^-z);
       shared experts have the same width I as routed ones and weight 1.
+  R11 group limit (optional): a group's score is its largest s+b; keep the
+      topk_groups best groups (ties to the lower group index), select top-K
+      inside them.  The pages give only the limit (at most 4 nodes per token).
   R6  FP8: E4M3 max 448, round-to-nearest-even, saturate to +-448; a tile's
       scale is amax/448 in float32 (1 for an all-zero tile); q = E4M3(x / scale)
       with x / scale an IEEE float32 division; weights quantised per 128x128
@@ -73,6 +76,35 @@ def biased_topk(s: np.ndarray, b: np.ndarray, K: int):
     key = (s + np.asarray(b, np.float32)[None, :]).astype(np.float32)
     order = np.argsort(-key, axis=1, kind="stable")
     return order[:, :K].astype(np.int32), key
+
+
+def grouped_topk(s, b, K, n_groups, topk_groups):
+    """Group-limited selection (the node limit of "DeepSeek V3 & R1 論文研究",
+    section Cross-Node All-to-All: a token reaches at most a few nodes).
+    Experts form n_groups groups of N_r/n_groups consecutive indices.  Reading
+    R11: a group's score is its largest biased key s+b; the topk_groups groups
+    with the largest scores are kept (ties to the lower group index), then the
+    K largest keys among the kept groups' experts are selected exactly as in
+    biased_topk.  Returns (idx [T, K] int32, key [T, N_r] float32)."""
+    s = np.asarray(s, np.float32)
+    key = (s + np.asarray(b, np.float32)[None, :]).astype(np.float32)
+    T, N_r = key.shape
+    gs = N_r // n_groups
+    gscore = key.reshape(T, n_groups, gs).max(axis=2)
+    gorder = np.argsort(-gscore, axis=1, kind="stable")[:, :topk_groups]
+    keep = np.zeros((T, n_groups), bool)
+    np.put_along_axis(keep, gorder, True, axis=1)
+    masked = np.where(np.repeat(keep, gs, axis=1), key, -np.inf).astype(np.float32)
+    order = np.argsort(-masked, axis=1, kind="stable")
+    return order[:, :K].astype(np.int32), key
+
+
+def route_grouped(u, E, b, K, n_groups, topk_groups):
+    """Router with the group limit: as route(), selection by grouped_topk."""
+    s = affinity(u, E)
+    idx, key = grouped_topk(s, b, K, n_groups, topk_groups)
+    return {"s": s, "key": key, "idx": idx, "gate": gates(s, idx),
+            "counts": load_counts(idx, E.shape[0])}
 
 
 def gates(s: np.ndarray, idx: np.ndarray) -> np.ndarray:

@@ -87,3 +87,28 @@ def check_routing(idx_gpu, gate_gpu, counts_gpu, ref, K, gate_tol=TOL["f32"]):
     merged_gate = ref["gate"].copy()
     merged_gate[sel_tie | ord_tie] = O.gates(ref["s"], idx_gpu)[sel_tie | ord_tie]
     return sel_tie | ord_tie, merged_idx, merged_gate
+
+
+def grouped_reference(ref, K, n_groups, topk_groups):
+    """Reference routing reshaped so that check_routing exempts grouped near-ties:
+    keys outside the oracle's kept groups become -inf, and tokens whose
+    topk_groups-th and next group scores are closer than TIE_GAP get a zero
+    margin (their kept groups may legitimately differ)."""
+    key = ref["key"]
+    T, N_r = key.shape
+    gs = N_r // n_groups
+    g = key.reshape(T, n_groups, gs).max(axis=2)
+    gsrt = -np.sort(-g, axis=1)
+    gtie = (gsrt[:, topk_groups - 1] - gsrt[:, topk_groups]) < TIE_GAP if topk_groups < n_groups \
+        else np.zeros(T, bool)
+    kept = np.zeros((T, n_groups), bool)
+    np.put_along_axis(kept, np.argsort(-g, axis=1, kind="stable")[:, :topk_groups], True, axis=1)
+    masked = np.where(np.repeat(kept, gs, axis=1), key, -np.inf).astype(np.float32)
+    # group-score near-tie: give the excluded experts the K-th key, so the gap
+    # between the K-th and (K+1)-th key is zero and the token is exempt
+    if gtie.any():
+        kth = -np.sort(-masked[gtie], axis=1)[:, K - 1:K]
+        masked[gtie] = np.where(np.isinf(masked[gtie]), kth, masked[gtie])
+    out = dict(ref)
+    out["key"] = masked
+    return out

@@ -8,7 +8,8 @@ import torch
 
 import mixture_experts_layer_60_b200 as moe
 from oracle import moe_oracle as O
-from tests.harness import GATE_TOL, TOL, LazyExperts, assert_close, check_routing, f64
+from tests.harness import (GATE_TOL, TOL, LazyExperts, assert_close, check_routing, f64,
+                           grouped_reference)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -61,6 +62,28 @@ def test_route_matches_oracle(T, d, N_r, K, dt):
     check_routing(idx.cpu().numpy(), gate.cpu().numpy(), counts.cpu().numpy(), ref, K,
                   gate_tol=GATE_TOL["f32" if dt == torch.float32 else "bf16"])
     np.testing.assert_allclose(gate.double().sum(1).cpu().numpy(), 1.0, atol=4e-7)
+
+
+@pytest.mark.parametrize("T,d,N_r,K,G,M", [
+    (1000, 512, 256, 8, 8, 4), (333, 256, 64, 6, 4, 2), (200, 128, 64, 4, 16, 1),
+    (300, 256, 128, 8, 8, 8),    # keeping every group: same as no limit
+])
+def test_route_grouped_matches_oracle(T, d, N_r, K, G, M):
+    g = _gen(T + G * 7)
+    u = _randn((T, d), g)
+    E = _randn((N_r, d), g, d ** -0.5)
+    b = ((torch.rand(N_r, generator=g, device=DEV) * 2 - 1) * 0.01).float()
+    idx = torch.empty(T, K, dtype=torch.int32, device=DEV)
+    gate = torch.empty(T, K, dtype=torch.float32, device=DEV)
+    counts = torch.empty(N_r, dtype=torch.int32, device=DEV)
+    moe.moe_route_grouped(u, E, b, K, G, M, idx, gate, counts,
+                          _ws(moe.moe_route_workspace_size(T, N_r)))
+    torch.cuda.synchronize()
+    ref = O.route_grouped(f64(u), f64(E), b.cpu().numpy(), K, G, M)
+    check_routing(idx.cpu().numpy(), gate.cpu().numpy(), counts.cpu().numpy(),
+                  grouped_reference(ref, K, G, M), K, gate_tol=GATE_TOL["bf16"])
+    gsz = N_r // G
+    assert max(len(set((r // gsz).tolist())) for r in idx.cpu().numpy()) <= M
 
 
 def test_route_zero_centroids_gates_are_uniform():

@@ -11,7 +11,8 @@ from mixture_experts_layer_60_b200.configs import CONFIGS
 from mixture_experts_layer_60_b200.layer import MoELayer
 from mixture_experts_layer_60_b200.synth import make_layer_inputs, step_u
 from oracle import moe_oracle as O
-from tests.harness import GATE_TOL, TOL, LazyExperts, assert_close, check_routing, f64
+from tests.harness import (GATE_TOL, TOL, LazyExperts, assert_close, check_routing, f64,
+                           grouped_reference)
 
 pytestmark = pytest.mark.gpu
 
@@ -44,10 +45,19 @@ def _run(cfg, T=None, sample=None, seed_sample=0):
     layer = MoELayer(cfg, w, T_max=u.shape[0])
     h = layer.forward(u)
     torch.cuda.synchronize()
-    ref = O.route(f64(u), f64(w["E"]), w["b"].cpu().numpy(), cfg.K)
+    if cfg.n_groups > 1:
+        ref = O.route_grouped(f64(u), f64(w["E"]), w["b"].cpu().numpy(), cfg.K, cfg.n_groups,
+                              cfg.topk_groups)
+        ref_chk = grouped_reference(ref, cfg.K, cfg.n_groups, cfg.topk_groups)
+    else:
+        ref = ref_chk = O.route(f64(u), f64(w["E"]), w["b"].cpu().numpy(), cfg.K)
     exempt, idx, gate = check_routing(layer.topk_idx.cpu().numpy(), layer.topk_gate.cpu().numpy(),
-                                      layer.counts.cpu().numpy(), ref, cfg.K,
+                                      layer.counts.cpu().numpy(), ref_chk, cfg.K,
                                       gate_tol=GATE_TOL[cfg.dtype])
+    if cfg.n_groups > 1:
+        gsz = cfg.N_r // cfg.n_groups
+        used = [len(set((r // gsz).tolist())) for r in layer.topk_idx.cpu().numpy()]
+        assert max(used) <= cfg.topk_groups
     Tn = u.shape[0]
     rows = np.arange(Tn) if sample is None else \
         np.sort(np.random.default_rng(seed_sample).choice(Tn, sample, replace=False))
@@ -89,6 +99,11 @@ def test_layer_fp8_small_full():
 def test_layer_v3_decode_sampled():
     """Decode-shaped batch (T = 256, ~8 tokens per expert): 16-row token tiles."""
     _run(CONFIGS["v3_decode_bf16"], sample=16, seed_sample=3)
+
+
+def test_layer_v3_grouped_sampled():
+    """Node-limited routing at V3 shape: 8 groups of 32 experts, at most 4 per token."""
+    _run(CONFIGS["v3_grouped_bf16"], sample=16, seed_sample=4)
 
 
 def test_layer_all_tokens_one_expert():

@@ -422,3 +422,46 @@ def test_fp8_ffn_close_to_exact():
     rms = np.sqrt(((got - want) ** 2).mean() / (want ** 2).mean())
     assert rms <= 0.09
     assert np.abs(got - want).max() <= 0.15 * np.abs(want).max()
+
+
+# --------------------------------------------------------------------------
+# group-limited routing
+# --------------------------------------------------------------------------
+
+def _brute_grouped(key_row, K, G, M):
+    """Enumerate every choice of M groups (score = best key, ties to lower
+    group index as a dominant set), then the best K keys inside them."""
+    n = len(key_row)
+    gs = n // G
+    gscore = [max(key_row[g * gs:(g + 1) * gs]) for g in range(G)]
+    best = None
+    for gsub in itertools.combinations(range(G), M):
+        rest = [g for g in range(G) if g not in gsub]
+        if all(gscore[a] > gscore[c] or (gscore[a] == gscore[c] and a < c)
+               for a in gsub for c in rest):
+            best = gsub
+    allowed = [i for i in range(n) if i // gs in best]
+    return sorted(allowed, key=lambda i: (-key_row[i], i))[:K]
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_grouped_topk_bruteforce(seed):
+    rng = np.random.default_rng(100 + seed)
+    N_r, G, M, K = [(16, 4, 2, 3), (12, 3, 1, 4), (16, 8, 3, 5), (8, 2, 2, 8)][seed]
+    s = (rng.integers(0, 6, size=(50, N_r)) / 8.0 + 0.2).astype(np.float32)
+    b = (rng.integers(-2, 3, size=N_r) / 16.0).astype(np.float32)
+    idx, key = O.grouped_topk(s, b, K, G, M)
+    for t in range(50):
+        assert idx[t].tolist() == _brute_grouped(key[t].tolist(), K, G, M)
+        assert len({int(e) // (N_r // G) for e in idx[t]}) <= M
+
+
+def test_grouped_topk_special_cases():
+    rng = np.random.default_rng(5)
+    s = rng.uniform(0, 1, (200, 32)).astype(np.float32)
+    b = rng.uniform(-0.05, 0.05, 32).astype(np.float32)
+    plain, _ = O.biased_topk(s, b, 6)
+    for G in (1, 2, 4, 8):                       # keeping every group is no limit
+        np.testing.assert_array_equal(O.grouped_topk(s, b, 6, G, G)[0], plain)
+    idx, key = O.grouped_topk(s, b, 6, 8, 2)
+    assert np.all(idx[:, 0] == np.argmax(key, axis=1))   # the best expert's group always survives
