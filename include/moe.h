@@ -78,7 +78,10 @@ const char* moe_status_string(moe_status status);
  *                      expert (overwritten, not accumulated)
  *   workspace          device, >= moe_route_workspace_size(T, N_r) bytes
  * Logits are accumulated in float32 from the stored values; sigmoid, keys and
- * gates are float32.  Requires 1 <= K <= N_r <= 1024 and d % 64 == 0.
+ * gates are float32.  Tokens whose selection (or output order) was decided by
+ * a key gap below 3e-5 are re-routed from float64 logits (sigmoid in float64,
+ * s rounded once to float32), so the float32 accumulation error cannot flip
+ * them.  Requires 1 <= K <= N_r <= 1024 and d % 64 == 0.
  * ------------------------------------------------------------------------ */
 size_t moe_route_workspace_size(int T, int N_r);
 moe_status moe_route(const void* u, const void* E, moe_dtype dt, const float* b,

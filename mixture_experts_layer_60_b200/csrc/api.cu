@@ -41,10 +41,15 @@ moe_status check_device() {
     if (_st != MOE_OK) return _st;    \
   } while (0)
 
+// Router workspace: float32 logits [T, N_r], then the tie-break list [1 + T] int32.
 size_t route_ws(int T, int N_r) {
   if (T <= 0 || N_r <= 0) return 0;
-  return align_up((size_t)T * N_r * sizeof(float), 256);
+  return align_up((size_t)T * N_r * sizeof(float), 256) + align_up((size_t)(T + 1) * 4, 256);
 }
+
+// Routing decided by a key gap below this is redone from float64 logits: the
+// float32 tensor-core logits over d <= 16384 products stay well within it.
+constexpr float kRefineGap = 3e-5f;
 
 size_t ffn_ws(moe_dtype dt, int rows, int I) {
   if (rows <= 0 || I <= 0) return 0;
@@ -118,7 +123,13 @@ moe_status route_impl(const char* who, const void* u, const void* E, moe_dtype d
   } else {
     MOE_TRY(launch_logits_simt(u, E, dt, T, d, N_r, logits, s));
   }
-  return launch_topk(logits, b, T, N_r, K, n_groups, topk_groups, topk_idx, topk_gate, counts, s);
+  int32_t* refine = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) +
+                                               align_up((size_t)T * N_r * sizeof(float), 256));
+  MOE_TRY(cuda_check(cudaMemsetAsync(refine, 0, sizeof(int32_t), s), "zero tie-break list"));
+  MOE_TRY(launch_topk(logits, b, T, N_r, K, n_groups, topk_groups, topk_idx, topk_gate, counts,
+                      refine, kRefineGap, s));
+  return launch_refine(u, E, dt, b, d, N_r, K, n_groups, topk_groups, refine, T, topk_idx,
+                       topk_gate, counts, s);
 }
 
 }  // namespace

@@ -12,9 +12,15 @@ moe_status launch_logits_simt(const void* u, const void* E, moe_dtype dt, int T,
                               int N_r, float* logits, cudaStream_t s);
 // sigmoid, biased top-K, gates, histogram (counts must be zeroed beforehand).
 // n_groups > 1 && topk_groups < n_groups restricts each token to its best groups.
+// Tokens whose routing was decided by a key gap < refine_gap are appended to
+// refine ([0] = count, zeroed beforehand; [1..T] = token ids).
 moe_status launch_topk(const float* logits, const float* b, int T, int N_r, int K, int n_groups,
                        int topk_groups, int32_t* idx, float* gate, int32_t* counts,
-                       cudaStream_t s);
+                       int32_t* refine, float refine_gap, cudaStream_t s);
+// Redoes the routing of the listed tokens from float64 logits.
+moe_status launch_refine(const void* u, const void* E, moe_dtype dt, const float* b, int d,
+                         int N_r, int K, int n_groups, int topk_groups, const int32_t* refine,
+                         int T, int32_t* idx, float* gate, int32_t* counts, cudaStream_t s);
 
 // permute.cu -----------------------------------------------------------------
 size_t permute_ws_bytes(int T, int N_r);

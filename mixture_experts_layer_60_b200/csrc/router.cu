@@ -33,7 +33,8 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
                                                    int N_r, int K, int n_groups, int topk_groups,
                                                    int32_t* __restrict__ idx,
                                                    float* __restrict__ gate,
-                                                   int32_t* __restrict__ counts) {
+                                                   int32_t* __restrict__ counts,
+                                                   int32_t* __restrict__ refine, float refine_gap) {
   extern __shared__ int hist[];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -58,6 +59,7 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
         key[j] = -INFINITY;
       }
     }
+    float margin = INFINITY;   // smallest key gap that decided this token's routing
     if (grouped) {
       const int gs = N_r / n_groups;
 #pragma unroll
@@ -71,7 +73,8 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
         for (int i = 0; i < gs; ++i) gscore = fmaxf(gscore, wkeys[lane * gs + i]);
       __syncwarp();
       unsigned kept = 0;
-      for (int r = 0; r < topk_groups; ++r) {
+      float last_kept = INFINITY;
+      for (int r = 0; r <= topk_groups; ++r) {    // one extra round: the best excluded group
         float bk = (lane < n_groups && !((kept >> lane) & 1u)) ? gscore : -INFINITY;
         int bg = lane < n_groups && !((kept >> lane) & 1u) ? lane : 0x7fffffff;
 #pragma unroll
@@ -80,7 +83,12 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
           const int og = __shfl_xor_sync(0xffffffffu, bg, off);
           if (ok > bk || (ok == bk && og < bg)) { bk = ok; bg = og; }
         }
-        kept |= 1u << bg;
+        if (r < topk_groups) {
+          kept |= 1u << bg;
+          last_kept = bk;
+        } else {
+          margin = fminf(margin, last_kept - bk);   // kept vs excluded group scores
+        }
       }
 #pragma unroll
       for (int j = 0; j < V; ++j) {
@@ -88,8 +96,8 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
         if (e < N_r && !((kept >> (e / gs)) & 1u)) key[j] = -INFINITY;
       }
     }
-    float sum = 0.f;
-    for (int k = 0; k < K; ++k) {
+    float sum = 0.f, prev = INFINITY;
+    for (int k = 0; k <= K; ++k) {             // round K only measures the next key
       // lane-local best
       float bk = -INFINITY;
       int be = 0x7fffffff;
@@ -107,6 +115,9 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
         const int oe = __shfl_xor_sync(0xffffffffu, be, off);
         if (ok > bk || (ok == bk && oe < be)) { bk = ok; be = oe; }
       }
+      margin = fminf(margin, prev - bk);        // adjacent selected keys, and K-th vs next
+      prev = bk;
+      if (k == K) break;
       // the owner removes the winner and broadcasts its unbiased s
       float s_win = 0.f;
       if ((be & 31) == lane) {
@@ -127,15 +138,128 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
       const size_t p = (size_t)t * K + k;
       gate[p] = gate[p] / sum;
     }
+    if (lane == 0 && margin < refine_gap) refine[1 + atomicAdd(&refine[0], 1)] = t;
   }
   __syncthreads();
   for (int i = threadIdx.x; i < N_r; i += blockDim.x)
     if (hist[i]) atomicAdd(&counts[i], hist[i]);
 }
 
+// Precise tie-break.  The tensor-core logits are float32 sums of d products,
+// which can move s by a few 1e-6 at V3 width; for every token whose routing
+// was decided by a key gap below refine_gap, the logits are recomputed in
+// float64 (s = Sigmoid in float64, rounded once to float32, as the affinity
+// line's exact value) and the selection, gates and load are redone from
+// them.  One block per listed token; the block's warps share the experts.
+template <typename Tin>
+__global__ void __launch_bounds__(256) refine_kernel(const Tin* __restrict__ u,
+                                                     const Tin* __restrict__ E,
+                                                     const float* __restrict__ bias, int d, int N_r,
+                                                     int K, int n_groups, int topk_groups,
+                                                     const int32_t* __restrict__ refine,
+                                                     int32_t* __restrict__ idx,
+                                                     float* __restrict__ gate,
+                                                     int32_t* __restrict__ counts) {
+  extern __shared__ float sm_r[];
+  float* sv = sm_r;            // [N_r] float32 affinity
+  float* kv = sm_r + N_r;      // [N_r] key s + b
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int n = refine[0];
+  for (int i = blockIdx.x; i < n; i += gridDim.x) {
+    const int t = refine[1 + i];
+    const Tin* ut = u + (size_t)t * d;
+    for (int e = warp; e < N_r; e += nw) {
+      const Tin* er = E + (size_t)e * d;
+      double acc = 0.0;
+      for (int k = lane; k < d; k += 32)
+        acc = fma((double)IO<Tin>::cvt(ut[k]), (double)IO<Tin>::cvt(er[k]), acc);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      if (lane == 0) {
+        const float sf = (float)(1.0 / (1.0 + exp(-acc)));
+        sv[e] = sf;
+        kv[e] = sf + bias[e];
+      }
+    }
+    __syncthreads();
+    if (warp == 0) {
+      if (n_groups > 1 && topk_groups < n_groups) {
+        const int gs = N_r / n_groups;
+        float gscore = -INFINITY;
+        if (lane < n_groups)
+          for (int j = 0; j < gs; ++j) gscore = fmaxf(gscore, kv[lane * gs + j]);
+        unsigned kept = 0;
+        for (int r = 0; r < topk_groups; ++r) {
+          float bk = (lane < n_groups && !((kept >> lane) & 1u)) ? gscore : -INFINITY;
+          int bg = (lane < n_groups && !((kept >> lane) & 1u)) ? lane : 0x7fffffff;
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) {
+            const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
+            const int og = __shfl_xor_sync(0xffffffffu, bg, off);
+            if (ok > bk || (ok == bk && og < bg)) { bk = ok; bg = og; }
+          }
+          kept |= 1u << bg;
+        }
+        __syncwarp();
+        for (int e = lane; e < N_r; e += 32)
+          if (!((kept >> (e / gs)) & 1u)) kv[e] = -INFINITY;
+        __syncwarp();
+      }
+      float sum = 0.f;
+      for (int k = 0; k < K; ++k) {
+        float bk = -INFINITY;
+        int be = 0x7fffffff;
+        for (int e = lane; e < N_r; e += 32)
+          if (kv[e] > bk || (kv[e] == bk && e < be)) { bk = kv[e]; be = e; }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
+          const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+          if (ok > bk || (ok == bk && oe < be)) { bk = ok; be = oe; }
+        }
+        const float s_win = sv[be];
+        sum += s_win;
+        __syncwarp();
+        if (lane == 0) {
+          const size_t p = (size_t)t * K + k;
+          atomicSub(&counts[idx[p]], 1);
+          atomicAdd(&counts[be], 1);
+          idx[p] = be;
+          gate[p] = s_win;
+          kv[be] = -INFINITY;
+        }
+        __syncwarp();
+      }
+      for (int k = lane; k < K; k += 32) {
+        const size_t p = (size_t)t * K + k;
+        gate[p] = gate[p] / sum;
+      }
+    }
+    __syncthreads();
+  }
+}
+
+moe_status launch_refine(const void* u, const void* E, moe_dtype dt, const float* b, int d,
+                         int N_r, int K, int n_groups, int topk_groups, const int32_t* refine,
+                         int T, int32_t* idx, float* gate, int32_t* counts, cudaStream_t s) {
+  int blocks = 2 * sm_count();
+  if (blocks > T) blocks = T > 0 ? T : 1;
+  const size_t smem = 2 * (size_t)N_r * sizeof(float);
+  if (dt == MOE_F32)
+    refine_kernel<float><<<blocks, 256, smem, s>>>(static_cast<const float*>(u),
+                                                  static_cast<const float*>(E), b, d, N_r, K,
+                                                  n_groups, topk_groups, refine, idx, gate,
+                                                  counts);
+  else
+    refine_kernel<__nv_bfloat16><<<blocks, 256, smem, s>>>(
+        static_cast<const __nv_bfloat16*>(u), static_cast<const __nv_bfloat16*>(E), b, d, N_r, K,
+        n_groups, topk_groups, refine, idx, gate, counts);
+  return cuda_check(cudaGetLastError(), "refine_kernel launch");
+}
+
 moe_status launch_topk(const float* logits, const float* b, int T, int N_r, int K, int n_groups,
                        int topk_groups, int32_t* idx, float* gate, int32_t* counts,
-                       cudaStream_t s) {
+                       int32_t* refine, float refine_gap, cudaStream_t s) {
   const int threads = 256;
   const int wpb = threads / 32;
   int blocks = (T + wpb - 1) / wpb;
@@ -146,7 +270,7 @@ moe_status launch_topk(const float* logits, const float* b, int T, int N_r, int 
   const int V = (N_r + 31) / 32;
 #define MOE_TOPK_CASE(v)                                                                    \
   topk_kernel<v><<<blocks, threads, smem, s>>>(logits, b, T, N_r, K, n_groups, topk_groups, idx, \
-                                               gate, counts);                                  \
+                                               gate, counts, refine, refine_gap);             \
   break;
   switch (V <= 1 ? 1 : V <= 2 ? 2 : V <= 4 ? 4 : V <= 8 ? 8 : V <= 16 ? 16 : 32) {
     case 1: MOE_TOPK_CASE(1)

@@ -46,7 +46,7 @@ def test_abi_version_and_status_strings(L):
 
 
 def test_workspace_sizes(L):
-    assert L.moe_route_workspace_size(8192, 256) == 8192 * 256 * 4
+    assert L.moe_route_workspace_size(8192, 256) >= 8192 * 256 * 4 + 8193 * 4
     assert L.moe_route_workspace_size(0, 256) == 0
     assert L.moe_permute_workspace_size(8192, 256) >= 2 * 32 * 256 * 4
     assert L.moe_expert_ffn_workspace_size(1, 65536, 2048) == 65536 * 2048 * 2
