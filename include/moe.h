@@ -79,7 +79,7 @@ const char* moe_status_string(moe_status status);
  *   workspace          device, >= moe_route_workspace_size(T, N_r) bytes
  * Logits are accumulated in float32 from the stored values; sigmoid, keys and
  * gates are float32.  Tokens whose selection (or output order) was decided by
- * a key gap below 3e-5 are re-routed from float64 logits (sigmoid in float64,
+ * a key gap below 2e-5 are re-routed from float64 logits (sigmoid in float64,
  * s rounded once to float32), so the float32 accumulation error cannot flip
  * them.  Requires 1 <= K <= N_r <= 1024 and d % 64 == 0.
  * ------------------------------------------------------------------------ */

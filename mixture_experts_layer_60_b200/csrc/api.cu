@@ -49,7 +49,7 @@ size_t route_ws(int T, int N_r) {
 
 // Routing decided by a key gap below this is redone from float64 logits: the
 // float32 tensor-core logits over d <= 16384 products stay well within it.
-constexpr float kRefineGap = 3e-5f;
+constexpr float kRefineGap = 2e-5f;
 
 size_t ffn_ws(moe_dtype dt, int rows, int I) {
   if (rows <= 0 || I <= 0) return 0;
@@ -128,7 +128,7 @@ moe_status route_impl(const char* who, const void* u, const void* E, moe_dtype d
   MOE_TRY(cuda_check(cudaMemsetAsync(refine, 0, sizeof(int32_t), s), "zero tie-break list"));
   MOE_TRY(launch_topk(logits, b, T, N_r, K, n_groups, topk_groups, topk_idx, topk_gate, counts,
                       refine, kRefineGap, s));
-  return launch_refine(u, E, dt, b, d, N_r, K, n_groups, topk_groups, refine, T, topk_idx,
+  return launch_refine(u, E, dt, logits, b, d, N_r, K, n_groups, topk_groups, refine, T, topk_idx,
                        topk_gate, counts, s);
 }
 

@@ -18,7 +18,8 @@ moe_status launch_topk(const float* logits, const float* b, int T, int N_r, int 
                        int topk_groups, int32_t* idx, float* gate, int32_t* counts,
                        int32_t* refine, float refine_gap, cudaStream_t s);
 // Redoes the routing of the listed tokens from float64 logits.
-moe_status launch_refine(const void* u, const void* E, moe_dtype dt, const float* b, int d,
+moe_status launch_refine(const void* u, const void* E, moe_dtype dt, const float* logits,
+                         const float* b, int d,
                          int N_r, int K, int n_groups, int topk_groups, const int32_t* refine,
                          int T, int32_t* idx, float* gate, int32_t* counts, cudaStream_t s);
 

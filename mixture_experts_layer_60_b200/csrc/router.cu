@@ -146,14 +146,98 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
 }
 
 // Precise tie-break.  The tensor-core logits are float32 sums of d products,
-// which can move s by a few 1e-6 at V3 width; for every token whose routing
-// was decided by a key gap below refine_gap, the logits are recomputed in
-// float64 (s = Sigmoid in float64, rounded once to float32, as the affinity
-// line's exact value) and the selection, gates and load are redone from
-// them.  One block per listed token; the block's warps share the experts.
+// which can move s by a few 1e-6 at V3 width.  For every token whose routing
+// was decided by a key gap below the refine gap, the experts whose float32
+// key lies within kNearBoundary of a decision boundary get float64 logits
+// (s = Sigmoid in float64, rounded once to float32: the affinity line's exact
+// value); the others keep their float32 keys, which are too far below every
+// boundary for the float32 error to matter.  Selection (with the group limit),
+// gates and load are then redone.  If the group choice changes, every expert
+// is recomputed.  One block per listed token; its warps share the float64
+// dot products.
+constexpr float kNearBoundary = 6e-5f;   // > 2 x the largest float32 key error
+
+template <typename Tin>
+__device__ __forceinline__ float exact_affinity(const Tin* __restrict__ ut,
+                                                const Tin* __restrict__ er, int d, int lane) {
+  double a0 = 0.0, a1 = 0.0;
+  const int nv = d / (16 / (int)sizeof(Tin));
+  const uint4* u4 = reinterpret_cast<const uint4*>(ut);
+  const uint4* e4 = reinterpret_cast<const uint4*>(er);
+  for (int v0 = lane; v0 < nv; v0 += 128) {
+    uint4 x[4], w[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {         // four independent 16-byte loads in flight
+      const int v = v0 + q * 32;
+      x[q] = v < nv ? u4[v] : make_uint4(0, 0, 0, 0);
+      w[q] = v < nv ? e4[v] : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t xs[4] = {x[q].x, x[q].y, x[q].z, x[q].w};
+      const uint32_t ws[4] = {w[q].x, w[q].y, w[q].z, w[q].w};
+      if (sizeof(Tin) == 2) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          a0 = fma((double)__uint_as_float(xs[i] << 16), (double)__uint_as_float(ws[i] << 16), a0);
+          a1 = fma((double)__uint_as_float(xs[i] & 0xffff0000u),
+                   (double)__uint_as_float(ws[i] & 0xffff0000u), a1);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          a0 = fma((double)__uint_as_float(xs[i]), (double)__uint_as_float(ws[i]), a0);
+      }
+    }
+  }
+  double acc = a0 + a1;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  return (float)(1.0 / (1.0 + exp(-acc)));
+}
+
+// Warp-wide arg-max of (key desc, index asc) over keys held lane-strided in kv[].
+__device__ __forceinline__ void warp_best(const float* kv, int N_r, int lane, float& bk, int& be) {
+  bk = -INFINITY;
+  be = 0x7fffffff;
+  for (int e = lane; e < N_r; e += 32)
+    if (kv[e] > bk || (kv[e] == bk && e < be)) { bk = kv[e]; be = e; }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
+    const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+    if (ok > bk || (ok == bk && oe < be)) { bk = ok; be = oe; }
+  }
+}
+
+// Group limit on keys kv[]: returns the kept-group mask (topk_groups best
+// group maxima, ties to the lower group index).
+__device__ __forceinline__ unsigned keep_groups(const float* kv, int N_r, int n_groups,
+                                                int topk_groups, int lane, float* next_score) {
+  const int gs = N_r / n_groups;
+  float gscore = -INFINITY;
+  if (lane < n_groups)
+    for (int j = 0; j < gs; ++j) gscore = fmaxf(gscore, kv[lane * gs + j]);
+  unsigned kept = 0;
+  for (int r = 0; r <= topk_groups && r < n_groups; ++r) {
+    float bk = (lane < n_groups && !((kept >> lane) & 1u)) ? gscore : -INFINITY;
+    int bg = (lane < n_groups && !((kept >> lane) & 1u)) ? lane : 0x7fffffff;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
+      const int og = __shfl_xor_sync(0xffffffffu, bg, off);
+      if (ok > bk || (ok == bk && og < bg)) { bk = ok; bg = og; }
+    }
+    if (r < topk_groups) kept |= 1u << bg;
+    else *next_score = bk;
+  }
+  return kept;
+}
+
 template <typename Tin>
 __global__ void __launch_bounds__(256) refine_kernel(const Tin* __restrict__ u,
                                                      const Tin* __restrict__ E,
+                                                     const float* __restrict__ logits,
                                                      const float* __restrict__ bias, int d, int N_r,
                                                      int K, int n_groups, int topk_groups,
                                                      const int32_t* __restrict__ refine,
@@ -161,62 +245,94 @@ __global__ void __launch_bounds__(256) refine_kernel(const Tin* __restrict__ u,
                                                      float* __restrict__ gate,
                                                      int32_t* __restrict__ counts) {
   extern __shared__ float sm_r[];
-  float* sv = sm_r;            // [N_r] float32 affinity
-  float* kv = sm_r + N_r;      // [N_r] key s + b
+  float* sv = sm_r;            // s [N_r]
+  float* kv = sv + N_r;        // key [N_r]
+  float* kw = kv + N_r;        // scratch keys [N_r]
+  int* cand = reinterpret_cast<int*>(kw + N_r);   // [N_r] experts to recompute, [N_r] = count
+  __shared__ int s_full;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const bool grouped = n_groups > 1 && topk_groups < n_groups;
+  const int gs = grouped ? N_r / n_groups : N_r;
   const int n = refine[0];
   for (int i = blockIdx.x; i < n; i += gridDim.x) {
     const int t = refine[1 + i];
     const Tin* ut = u + (size_t)t * d;
-    for (int e = warp; e < N_r; e += nw) {
-      const Tin* er = E + (size_t)e * d;
-      double acc = 0.0;
-      for (int k = lane; k < d; k += 32)
-        acc = fma((double)IO<Tin>::cvt(ut[k]), (double)IO<Tin>::cvt(er[k]), acc);
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    for (int e = threadIdx.x; e < N_r; e += blockDim.x) {
+      const float sf = 1.0f / (1.0f + expf(-logits[(size_t)t * N_r + e]));   // as the top-K kernel
+      sv[e] = sf;
+      kv[e] = sf + bias[e];
+      kw[e] = kv[e];
+    }
+    __syncthreads();
+    unsigned kept32 = 0xffffffffu;
+    if (warp == 0) {
+      // lowest key any decision can hinge on: the (K+1)-th key inside the kept
+      // groups and, with the group limit, the best excluded group's score
+      float floor_key = INFINITY;
+      if (grouped) {
+        float next_g = -INFINITY;
+        kept32 = keep_groups(kw, N_r, n_groups, topk_groups, lane, &next_g);
+        floor_key = next_g;
+        for (int e = lane; e < N_r; e += 32)
+          if (!((kept32 >> (e / gs)) & 1u)) kw[e] = -INFINITY;
+        __syncwarp();
+      }
+      for (int k = 0; k <= K; ++k) {
+        float bk;
+        int be;
+        warp_best(kw, N_r, lane, bk, be);
+        if (k == K || be >= N_r) { floor_key = fminf(floor_key, bk); break; }
+        __syncwarp();
+        if (lane == 0) kw[be] = -INFINITY;
+        __syncwarp();
+      }
       if (lane == 0) {
-        const float sf = (float)(1.0 / (1.0 + exp(-acc)));
-        sv[e] = sf;
-        kv[e] = sf + bias[e];
+        int c = 0;
+        for (int e = 0; e < N_r; ++e)
+          if (kv[e] >= floor_key - kNearBoundary) cand[c++] = e;
+        cand[N_r] = c;
       }
     }
     __syncthreads();
-    if (warp == 0) {
-      if (n_groups > 1 && topk_groups < n_groups) {
-        const int gs = N_r / n_groups;
-        float gscore = -INFINITY;
-        if (lane < n_groups)
-          for (int j = 0; j < gs; ++j) gscore = fmaxf(gscore, kv[lane * gs + j]);
-        unsigned kept = 0;
-        for (int r = 0; r < topk_groups; ++r) {
-          float bk = (lane < n_groups && !((kept >> lane) & 1u)) ? gscore : -INFINITY;
-          int bg = (lane < n_groups && !((kept >> lane) & 1u)) ? lane : 0x7fffffff;
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) {
-            const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
-            const int og = __shfl_xor_sync(0xffffffffu, bg, off);
-            if (ok > bk || (ok == bk && og < bg)) { bk = ok; bg = og; }
-          }
-          kept |= 1u << bg;
-        }
+    // float64 affinity of the candidates, one warp per candidate
+    for (int c = warp; c < cand[N_r]; c += nw) {
+      const int e = cand[c];
+      const float sf = exact_affinity(ut, E + (size_t)e * d, d, lane);
+      if (lane == 0) { sv[e] = sf; kv[e] = sf + bias[e]; }
+    }
+    __syncthreads();
+    if (grouped) {
+      if (warp == 0) {
+        for (int e = lane; e < N_r; e += 32) kw[e] = kv[e];
         __syncwarp();
+        float next_g = -INFINITY;
+        const unsigned kept = keep_groups(kw, N_r, n_groups, topk_groups, lane, &next_g);
+        if (lane == 0) s_full = kept != kept32;   // group choice moved: refine every expert
+      }
+      __syncthreads();
+      if (s_full) {
+        for (int e = warp; e < N_r; e += nw) {
+          const float sf = exact_affinity(ut, E + (size_t)e * d, d, lane);
+          if (lane == 0) { sv[e] = sf; kv[e] = sf + bias[e]; }
+        }
+      }
+      __syncthreads();
+    }
+    if (warp == 0) {
+      for (int e = lane; e < N_r; e += 32) kw[e] = kv[e];
+      __syncwarp();
+      if (grouped) {
+        float next_g = -INFINITY;
+        const unsigned kept = keep_groups(kw, N_r, n_groups, topk_groups, lane, &next_g);
         for (int e = lane; e < N_r; e += 32)
-          if (!((kept >> (e / gs)) & 1u)) kv[e] = -INFINITY;
+          if (!((kept >> (e / gs)) & 1u)) kw[e] = -INFINITY;
         __syncwarp();
       }
       float sum = 0.f;
       for (int k = 0; k < K; ++k) {
-        float bk = -INFINITY;
-        int be = 0x7fffffff;
-        for (int e = lane; e < N_r; e += 32)
-          if (kv[e] > bk || (kv[e] == bk && e < be)) { bk = kv[e]; be = e; }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-          const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
-          const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-          if (ok > bk || (ok == bk && oe < be)) { bk = ok; be = oe; }
-        }
+        float bk;
+        int be;
+        warp_best(kw, N_r, lane, bk, be);
         const float s_win = sv[be];
         sum += s_win;
         __syncwarp();
@@ -226,7 +342,7 @@ __global__ void __launch_bounds__(256) refine_kernel(const Tin* __restrict__ u,
           atomicAdd(&counts[be], 1);
           idx[p] = be;
           gate[p] = s_win;
-          kv[be] = -INFINITY;
+          kw[be] = -INFINITY;
         }
         __syncwarp();
       }
@@ -239,21 +355,30 @@ __global__ void __launch_bounds__(256) refine_kernel(const Tin* __restrict__ u,
   }
 }
 
-moe_status launch_refine(const void* u, const void* E, moe_dtype dt, const float* b, int d,
-                         int N_r, int K, int n_groups, int topk_groups, const int32_t* refine,
-                         int T, int32_t* idx, float* gate, int32_t* counts, cudaStream_t s) {
+moe_status launch_refine(const void* u, const void* E, moe_dtype dt, const float* logits,
+                         const float* b, int d, int N_r, int K, int n_groups, int topk_groups,
+                         const int32_t* refine, int T, int32_t* idx, float* gate, int32_t* counts,
+                         cudaStream_t s) {
+  const int threads = 256;
   int blocks = 2 * sm_count();
   if (blocks > T) blocks = T > 0 ? T : 1;
-  const size_t smem = 2 * (size_t)N_r * sizeof(float);
+  const size_t smem = (size_t)4 * N_r * sizeof(float) + sizeof(int);
+  if (smem > 48 * 1024) {
+    cudaError_t e = dt == MOE_F32
+        ? cudaFuncSetAttribute(refine_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)smem)
+        : cudaFuncSetAttribute(refine_kernel<__nv_bfloat16>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return cuda_check(e, "refine_kernel smem attribute");
+  }
   if (dt == MOE_F32)
-    refine_kernel<float><<<blocks, 256, smem, s>>>(static_cast<const float*>(u),
-                                                  static_cast<const float*>(E), b, d, N_r, K,
-                                                  n_groups, topk_groups, refine, idx, gate,
-                                                  counts);
-  else
-    refine_kernel<__nv_bfloat16><<<blocks, 256, smem, s>>>(
-        static_cast<const __nv_bfloat16*>(u), static_cast<const __nv_bfloat16*>(E), b, d, N_r, K,
+    refine_kernel<float><<<blocks, threads, smem, s>>>(
+        static_cast<const float*>(u), static_cast<const float*>(E), logits, b, d, N_r, K,
         n_groups, topk_groups, refine, idx, gate, counts);
+  else
+    refine_kernel<__nv_bfloat16><<<blocks, threads, smem, s>>>(
+        static_cast<const __nv_bfloat16*>(u), static_cast<const __nv_bfloat16*>(E), logits, b, d,
+        N_r, K, n_groups, topk_groups, refine, idx, gate, counts);
   return cuda_check(cudaGetLastError(), "refine_kernel launch");
 }
 
