@@ -221,11 +221,8 @@ moe_status run_gate_up(const void* x, const float* x_scale, const int32_t* offse
   if (dt == MOE_F32)
     return launch_simt_gemm(x, W_gate_up, 2LL * I * d, offsets, n_groups, rows, I, d, true,
                             MOE_F32, h, MOE_F32, s);
-  if (dt == MOE_BF16) {
-    if (ws2_supports(true, I))
-      return launch_ws2_gemm(x, W_gate_up, 2 * I, offsets, n_groups, rows, I, d, true, h, s);
+  if (dt == MOE_BF16)
     return launch_ws_gemm(x, W_gate_up, 2 * I, offsets, n_groups, rows, I, d, true, h, s);
-  }
   return launch_fp8_gemm(x, x_scale, W_gate_up, w_scale_gate_up, 2 * I, offsets, n_groups, rows,
                          I, d, true, h, h_scale, s);
 }
@@ -237,8 +234,6 @@ moe_status run_down(const void* h, const float* h_scale, const int32_t* offsets,
     return launch_simt_gemm(h, W_down, (long long)d * I, offsets, n_groups, rows, d, I, false,
                             MOE_F32, y, MOE_F32, s);
   if (dt == MOE_BF16) {
-    if (ws2_supports(false, d))
-      return launch_ws2_gemm(h, W_down, d, offsets, n_groups, rows, d, I, false, y, s);
     if (d % 256 == 0)
       return launch_ws_gemm(h, W_down, d, offsets, n_groups, rows, d, I, false, y, s);
     return launch_tc_gemm(h, W_down, d, offsets, n_groups, rows, d, I, TC_EPI_STORE_BF16, y, s);

@@ -54,14 +54,6 @@ moe_status launch_ws_gemm(const void* X, const void* W, int b_rows_per_group,
                           const int32_t* offsets, int n_groups, int rows, int N, int K,
                           bool swiglu, void* C, cudaStream_t s);
 
-// gemm_ws2.cu ----------------------------------------------------------------
-// The weights-stationary GEMM on CTA pairs (tcgen05 cta_group::2): 512 weight
-// rows per pair tile.  Needs N % 256 == 0 (swiglu, N = I) or N % 512 == 0.
-bool ws2_supports(bool swiglu, int N);
-moe_status launch_ws2_gemm(const void* X, const void* W, int b_rows_per_group,
-                           const int32_t* offsets, int n_groups, int rows, int N, int K,
-                           bool swiglu, void* C, cudaStream_t s);
-
 // gemm_fp8.cu ----------------------------------------------------------------
 moe_status launch_fp8_gemm(const void* A, const float* a_scale, const void* B,
                            const float* b_scale, int b_rows_per_group,
