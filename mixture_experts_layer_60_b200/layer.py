@@ -78,10 +78,12 @@ class MoELayer:
         self.T_alloc = T
 
     # -- one step ------------------------------------------------------------
-    def forward(self, u: torch.Tensor, stream=None, gate_up_events=None) -> torch.Tensor:
-        """h' for the T tokens of u; returns h_out (overwritten by the next call).
-        gate_up_events=(start, end) records CUDA events around the routed
-        gate/up GEMM launch on the same stream."""
+    def forward(self, u: torch.Tensor, stream=None, gate_up_events=None,
+                out: torch.Tensor | None = None) -> torch.Tensor:
+        """h' for the T tokens of u, written to `out` (default: the layer's own
+        h_out buffer, overwritten by the next call).  gate_up_events=(start,
+        end) records CUDA events around the routed gate/up GEMM launch on the
+        same stream."""
         c = self.cfg
         T = u.shape[0]
         if T != self.T_alloc:
@@ -120,9 +122,10 @@ class MoELayer:
                            w_scale_gate_up=None if ssgu is None else ssgu[j:j + 1],
                            w_scale_down=None if ssdn is None else ssdn[j:j + 1], stream=stream)
         u_res = u
+        h = self.h_out if out is None else out
         moe_combine(u_res, self.y_shared if c.N_s else None, self.y_perm, self.inv_row,
-                    self.topk_gate, self.h_out, stream)
-        return self.h_out
+                    self.topk_gate, h, stream)
+        return h
 
     def bias_update(self, counts=None, T_total=None, stream=None):
         """b <- b -/+ gamma from the load of the last step (or from the given

@@ -195,3 +195,33 @@ def test_skewed_load_steps_route_and_balance():
         b2.step(step_u(cfg, s, "cuda"))
     torch.cuda.synchronize()
     assert torch.equal(b2.b, a.b)
+
+
+def test_host_stepper_overlapped_equals_device_steps():
+    """Steps fed from pinned host memory with uploads and downloads overlapped
+    on copy streams give, step for step, the same h' (bit for bit) and the same
+    final bias as the same steps run on device-resident tokens."""
+    from dataclasses import replace
+    from mixture_experts_layer_60_b200.hostio import HostStepper
+    cfg = replace(CONFIGS["small_bf16"], T=768)
+    w = make_layer_inputs(cfg, "cuda", T=768)
+    n = 5
+    us = [step_u(cfg, s, "cuda", T=768) for s in range(n)]
+    ref = MoELayer(cfg, w)
+    want = []
+    for u in us:
+        want.append(ref.step(u).cpu().clone())
+    lay = MoELayer(cfg, w)
+    st = HostStepper(cfg.T, cfg.d, us[0].dtype, "cuda")
+    u_h = [u.cpu().pin_memory() for u in us]
+    h_h = [torch.empty_like(x).pin_memory() for x in u_h]
+
+    def fn(u_in, out):
+        lay.forward(u_in, out=out)
+        lay.bias_update()
+
+    st.run(u_h, h_h, fn)
+    torch.cuda.synchronize()
+    for s in range(n):
+        assert torch.equal(h_h[s], want[s]), s
+    assert torch.equal(lay.b, ref.b)
