@@ -242,6 +242,104 @@ moe_status moe_permute_noalloc(const void* u, const float* u_scale, moe_dtype dt
                                int32_t* offsets, int32_t* perm_src, int32_t* inv_row,
                                void* stream);
 
+/* ========================================================================
+ * Layer backward.  "DeepSeek V3 & R1 論文研究", section FP8 mixed precision,
+ * names the three GEMM passes of training (Fprop, Dgrad for activations,
+ * Wgrad for weights) and keeps the MoE gating module in its original
+ * precision; the pages print no backward formulas, so these calls apply the
+ * chain rule to the forward of section 方法 / 2 of "DeepSeek-V3 技術報告".
+ * The selection (top-K of s + b) is piecewise constant and is held fixed:
+ * gradients reach s only through g = s_sel / sum(s_sel); b gets none.
+ * Expert GEMMs run in bf16 with float32 accumulation (MOE_BF16 only);
+ * d % 256 == 0 and I % 256 == 0.  Order of a training step:
+ *   forward:  moe_route, moe_permute, moe_expert_gate_up_save (routed and
+ *             shared), moe_expert_down, moe_combine
+ *   backward: moe_combine_backward, moe_expert_ffn_backward (routed with
+ *             dy_perm, shared with dh_out), moe_unpermute_backward,
+ *             moe_router_weight_grad
+ * ======================================================================== */
+
+/* ------------------------------------------------------------------------
+ * moe_expert_gate_up_save - moe_expert_gate_up (MOE_BF16) that also keeps
+ * the pre-activations the backward needs:
+ *   a_gu[r, 0:I]  = W_gate[g] x[r],  a_gu[r, I:2I] = W_up[g] x[r]  (bf16)
+ *   h[r]          = SiLU(a_gu[r, 0:I]) * a_gu[r, I:2I], from the float32 values
+ *   x [rows, d], offsets, W_gate_up as for moe_expert_ffn; h [rows, I] and
+ *   a_gu [rows, 2I] device bf16 out, 16-byte aligned.
+ * ------------------------------------------------------------------------ */
+moe_status moe_expert_gate_up_save(const void* x, const int32_t* offsets, int n_groups,
+                                   int rows, int d, int I, moe_dtype dt,
+                                   const void* W_gate_up, void* h, void* a_gu, void* stream);
+
+/* ------------------------------------------------------------------------
+ * moe_combine_backward - gradient of the h'-equation through the routed
+ * term, the gate normalisation and the affinity, for upstream dh_out = dL/dh':
+ *   dy_perm[inv_row[t,k]]      = topk_gate[t,k] * dh_out[t]       (dt)
+ *   d_gate[t,k]                = <dh_out[t], y_perm[inv_row[t,k]]>  (float32)
+ *   s_k = Sigmoid(u[t] . E[topk_idx[t,k]]) recomputed in float32, S = sum_k s_k
+ *   d_logit[t,k]               = (d_gate[t,k] - sum_j topk_gate[t,j] d_gate[t,j]) / S
+ *                                * s_k (1 - s_k)                    (float32)
+ *   d_logit_perm[inv_row[t,k]] = d_logit[t,k]                      (float32)
+ *   dh_out, u [T, d]; E [N_r, d]; y_perm [T*K, d]: device, dt (MOE_F32 or
+ *   MOE_BF16); inv_row, topk_idx [T, K] int32 and topk_gate [T, K] float32
+ *   from the forward; dy_perm [T*K, d] dt out; d_gate, d_logit [T, K] and
+ *   d_logit_perm [T*K] float32 out.  K <= 16, d * sizeof(dt) % 16 == 0.
+ * The shared experts' upstream gradient is dh_out itself (weight 1).
+ * ------------------------------------------------------------------------ */
+moe_status moe_combine_backward(const void* dh_out, const void* u, const void* E,
+                                const void* y_perm, const int32_t* inv_row,
+                                const int32_t* topk_idx, const float* topk_gate, moe_dtype dt,
+                                int T, int d, int K, void* dy_perm, float* d_gate,
+                                float* d_logit, float* d_logit_perm, void* stream);
+
+/* ------------------------------------------------------------------------
+ * moe_expert_ffn_backward - Dgrad and Wgrad of the grouped SwiGLU FFN for
+ * upstream dy (MOE_BF16).  For group g and its rows r, with a, b the gate
+ * and up halves of a_gu and h = SiLU(a) * b from moe_expert_gate_up_save:
+ *   dh  = dy W_down[g]                               (float32, not stored)
+ *   dA  = [dh * b * SiLU'(a) | dh * SiLU(a)]          (bf16, in the workspace)
+ *   dx[r]          = dA[r] W_gate_up[g]               (Dgrad, bf16)
+ *   dW_down[g]     = sum_r dy[r]^T h[r]               (Wgrad, [d, I] bf16)
+ *   dW_gate_up[g]  = sum_r dA[r]^T x[r]               (Wgrad, [2I, d] bf16)
+ *   x [rows, d], dy [rows, d], h [rows, I], a_gu [rows, 2I]: device bf16 in;
+ *   offsets [n_groups+1] as for moe_expert_ffn; W_gate_up [n_groups, 2I, d]
+ *   and W_down [n_groups, d, I] bf16; dx [rows, d], dW_gate_up and dW_down
+ *   (same shapes as the weights) device bf16 out.  A group with no rows gets
+ *   zero weight gradients.  Workspace: moe_expert_ffn_backward_workspace_size
+ *   bytes, 256-byte aligned.  d % 256 == 0, I % 256 == 0.
+ * ------------------------------------------------------------------------ */
+size_t moe_expert_ffn_backward_workspace_size(moe_dtype dt, int rows, int I);
+moe_status moe_expert_ffn_backward(const void* x, const int32_t* offsets, int n_groups, int rows,
+                                   int d, int I, moe_dtype dt, const void* W_gate_up,
+                                   const void* W_down, const void* a_gu, const void* h,
+                                   const void* dy, void* dx, void* dW_gate_up, void* dW_down,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * moe_unpermute_backward - the input gradient:
+ *   du[t] = dh_out[t] + sum_{j<N_s} dx_shared[j][t] + sum_k dx_perm[inv_row[t,k]]
+ *           + sum_k d_logit[t,k] E[topk_idx[t,k]]
+ * summed in float32 in that order, rounded once to dt.  dh_out, du [T, d];
+ * dx_shared [N_s, T, d] (NULL when N_s == 0); dx_perm [T*K, d]; E [N_r, d]:
+ * device, dt (MOE_F32 or MOE_BF16).  K <= 16, d * sizeof(dt) % 16 == 0.
+ * ------------------------------------------------------------------------ */
+moe_status moe_unpermute_backward(const void* dh_out, const void* dx_shared, int N_s,
+                                  const void* dx_perm, const int32_t* inv_row,
+                                  const int32_t* topk_idx, const float* d_logit, const void* E,
+                                  moe_dtype dt, int T, int d, int K, void* du, void* stream);
+
+/* ------------------------------------------------------------------------
+ * moe_router_weight_grad - gradient of the expert centroids E:
+ *   dE[i] = sum over grouped rows r of expert i of d_logit_perm[r] x_perm[r]
+ * rows in ascending order, float32 accumulation.  x_perm [rows, d] device dt
+ * (MOE_F32 or MOE_BF16), d_logit_perm [rows] float32 and offsets [N_r+1] from
+ * moe_combine_backward / moe_permute; dE [N_r, d] device float32 out
+ * (original precision for the gating module).  d * sizeof(dt) % 16 == 0.
+ * ------------------------------------------------------------------------ */
+moe_status moe_router_weight_grad(const void* x_perm, const float* d_logit_perm,
+                                  const int32_t* offsets, moe_dtype dt, int N_r, int d, float* dE,
+                                  void* stream);
+
 /* ------------------------------------------------------------------------
  * moe_device_status - synchronises the current device, then returns (and
  * clears) the library's device-side error word: 0 if no kernel gave up a

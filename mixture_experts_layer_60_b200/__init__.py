@@ -18,6 +18,8 @@ __all__ = [
     "moe_route", "moe_route_grouped", "moe_permute", "moe_permute_noalloc", "moe_expert_ffn", "moe_expert_gate_up", "moe_expert_down", "moe_combine", "moe_bias_update",
     "moe_quantize_1x128", "moe_quantize_128x128", "moe_device_status",
     "moe_route_workspace_size", "moe_permute_workspace_size", "moe_expert_ffn_workspace_size",
+    "moe_expert_gate_up_save", "moe_combine_backward", "moe_expert_ffn_backward",
+    "moe_expert_ffn_backward_workspace_size", "moe_unpermute_backward", "moe_router_weight_grad",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
@@ -50,6 +52,15 @@ SYMBOLS = {
     "moe_quantize_128x128": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp]),
     "moe_device_status": (_i, [ctypes.POINTER(_i)]),
     "moe_permute_noalloc": (_i, [_vp, _vp, _i, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "moe_expert_gate_up_save": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
+    "moe_combine_backward": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp,
+                                  _vp, _vp]),
+    "moe_expert_ffn_backward_workspace_size": (_sz, [_i, _i, _i]),
+    "moe_expert_ffn_backward": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp,
+                                     _vp, _vp, _vp, _sz, _vp]),
+    "moe_unpermute_backward": (_i, [_vp, _vp, _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp,
+                                    _vp]),
+    "moe_router_weight_grad": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp, _vp]),
 }
 
 
@@ -218,3 +229,50 @@ def moe_device_status() -> int:
     if st not in (0, 5):
         _check(st)
     return flags.value
+
+
+# ------------------------------------------------------------------ backward
+
+def moe_expert_ffn_backward_workspace_size(dt: int, rows: int, I: int) -> int:
+    return lib().moe_expert_ffn_backward_workspace_size(dt, rows, I)
+
+
+def moe_expert_gate_up_save(x, offsets, W_gate_up, h, a_gu, stream=None):
+    rows, d = x.shape
+    n_groups, two_i, _ = W_gate_up.shape
+    _check(lib().moe_expert_gate_up_save(_p(x), _p(offsets), n_groups, rows, d, two_i // 2,
+                                         _dt(x), _p(W_gate_up), _p(h), _p(a_gu), _s(stream)))
+
+
+def moe_combine_backward(dh_out, u, E, y_perm, inv_row, topk_idx, topk_gate, dy_perm, d_gate,
+                         d_logit, d_logit_perm, stream=None):
+    T, d = u.shape
+    _check(lib().moe_combine_backward(_p(dh_out), _p(u), _p(E), _p(y_perm), _p(inv_row),
+                                      _p(topk_idx), _p(topk_gate), _dt(u), T, d,
+                                      inv_row.shape[1], _p(dy_perm), _p(d_gate), _p(d_logit),
+                                      _p(d_logit_perm), _s(stream)))
+
+
+def moe_expert_ffn_backward(x, offsets, W_gate_up, W_down, a_gu, h, dy, dx, dW_gate_up, dW_down,
+                            workspace, stream=None):
+    rows, d = x.shape
+    n_groups, two_i, _ = W_gate_up.shape
+    _check(lib().moe_expert_ffn_backward(_p(x), _p(offsets), n_groups, rows, d, two_i // 2,
+                                         _dt(x), _p(W_gate_up), _p(W_down), _p(a_gu), _p(h),
+                                         _p(dy), _p(dx), _p(dW_gate_up), _p(dW_down),
+                                         _p(workspace), _nbytes(workspace), _s(stream)))
+
+
+def moe_unpermute_backward(dh_out, dx_shared, dx_perm, inv_row, topk_idx, d_logit, E, du,
+                           stream=None):
+    T, d = dh_out.shape
+    N_s = 0 if dx_shared is None else dx_shared.shape[0]
+    _check(lib().moe_unpermute_backward(_p(dh_out), _p(dx_shared), N_s, _p(dx_perm), _p(inv_row),
+                                        _p(topk_idx), _p(d_logit), _p(E), _dt(dh_out), T, d,
+                                        inv_row.shape[1], _p(du), _s(stream)))
+
+
+def moe_router_weight_grad(x_perm, d_logit_perm, offsets, dE, stream=None):
+    N_r, d = dE.shape
+    _check(lib().moe_router_weight_grad(_p(x_perm), _p(d_logit_perm), _p(offsets), _dt(x_perm),
+                                        N_r, d, _p(dE), _s(stream)))

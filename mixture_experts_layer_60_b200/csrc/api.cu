@@ -376,6 +376,147 @@ moe_status moe_quantize_128x128(const void* w, int groups, int rows, int cols, u
   return launch_quant_128x128(w, groups, rows, cols, q, scale, as_stream(stream));
 }
 
+// ---------------------------------------------------------------- backward
+
+namespace {
+
+inline bool al16(const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0; }
+
+size_t ffn_bwd_ws(moe_dtype dt, int rows, int I) {
+  if (dt != MOE_BF16 || rows <= 0 || I <= 0) return 0;
+  return align_up((size_t)rows * 2 * I * 2, 256);
+}
+
+moe_status check_rowwise(const char* who, moe_dtype dt, int T, int d, int K) {
+  MOE_REQUIRE(dt == MOE_F32 || dt == MOE_BF16, MOE_ERR_UNSUPPORTED,
+              "%s: dtype must be MOE_F32 or MOE_BF16", who);
+  MOE_REQUIRE(T >= 0 && d > 0 && K > 0, MOE_ERR_INVALID_ARG, "%s: bad sizes T=%d d=%d K=%d", who,
+              T, d, K);
+  MOE_REQUIRE(K <= 16, MOE_ERR_UNSUPPORTED, "%s: K=%d > 16", who, K);
+  MOE_REQUIRE(((size_t)d * dtype_bytes(dt)) % 16 == 0, MOE_ERR_UNSUPPORTED,
+              "%s: a row must be a multiple of 16 bytes", who);
+  return MOE_OK;
+}
+
+}  // namespace
+
+moe_status moe_expert_gate_up_save(const void* x, const int32_t* offsets, int n_groups, int rows,
+                                   int d, int I, moe_dtype dt, const void* W_gate_up, void* h,
+                                   void* a_gu, void* stream) {
+  clear_last_error();
+  MOE_TRY(check_ffn_common("moe_expert_gate_up_save", x, offsets, n_groups, rows, d, I, dt,
+                           W_gate_up));
+  MOE_REQUIRE(dt == MOE_BF16, MOE_ERR_UNSUPPORTED, "moe_expert_gate_up_save: MOE_BF16 only");
+  if (rows == 0) return MOE_OK;
+  MOE_REQUIRE(h && a_gu, MOE_ERR_INVALID_ARG, "moe_expert_gate_up_save: null pointer");
+  MOE_REQUIRE(al16(h) && al16(a_gu) && al16(x), MOE_ERR_INVALID_ARG,
+              "moe_expert_gate_up_save: x, h and a_gu must be 16-byte aligned");
+  MOE_TRY(check_device());
+  return launch_ws_gemm_ex(x, W_gate_up, 2 * I, offsets, n_groups, rows, I, d, WS_SWIGLU_SAVE,
+                           false, h, I, a_gu, 2 * I, as_stream(stream));
+}
+
+moe_status moe_combine_backward(const void* dh_out, const void* u, const void* E,
+                                const void* y_perm, const int32_t* inv_row,
+                                const int32_t* topk_idx, const float* topk_gate, moe_dtype dt,
+                                int T, int d, int K, void* dy_perm, float* d_gate,
+                                float* d_logit, float* d_logit_perm, void* stream) {
+  clear_last_error();
+  MOE_TRY(check_rowwise("moe_combine_backward", dt, T, d, K));
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE(dh_out && u && E && y_perm && inv_row && topk_idx && topk_gate && dy_perm &&
+                  d_gate && d_logit && d_logit_perm,
+              MOE_ERR_INVALID_ARG, "moe_combine_backward: null pointer");
+  MOE_REQUIRE(al16(dh_out) && al16(u) && al16(E) && al16(y_perm) && al16(dy_perm),
+              MOE_ERR_INVALID_ARG, "moe_combine_backward: rows must be 16-byte aligned");
+  MOE_TRY(check_device());
+  return launch_combine_backward(dh_out, u, E, y_perm, inv_row, topk_idx, topk_gate, dt, T, d, K,
+                                 dy_perm, d_gate, d_logit, d_logit_perm, as_stream(stream));
+}
+
+size_t moe_expert_ffn_backward_workspace_size(moe_dtype dt, int rows, int I) {
+  return ffn_bwd_ws(dt, rows, I);
+}
+
+moe_status moe_expert_ffn_backward(const void* x, const int32_t* offsets, int n_groups, int rows,
+                                   int d, int I, moe_dtype dt, const void* W_gate_up,
+                                   const void* W_down, const void* a_gu, const void* h,
+                                   const void* dy, void* dx, void* dW_gate_up, void* dW_down,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+  clear_last_error();
+  const char* who = "moe_expert_ffn_backward";
+  MOE_TRY(check_ffn_common(who, x, offsets, n_groups, rows, d, I, dt, W_gate_up));
+  MOE_REQUIRE(dt == MOE_BF16, MOE_ERR_UNSUPPORTED, "%s: MOE_BF16 only", who);
+  MOE_REQUIRE(d % 256 == 0 && I % 256 == 0, MOE_ERR_UNSUPPORTED,
+              "%s: d=%d and I=%d must be multiples of 256", who, d, I);
+  MOE_REQUIRE(W_down && dW_gate_up && dW_down, MOE_ERR_INVALID_ARG, "%s: null pointer", who);
+  MOE_REQUIRE(al16(dW_gate_up) && al16(dW_down), MOE_ERR_INVALID_ARG,
+              "%s: weight gradients must be 16-byte aligned", who);
+  cudaStream_t s = as_stream(stream);
+  if (rows == 0) {
+    MOE_TRY(check_device());
+    const size_t per = (size_t)n_groups * 2 * I * d * 2;
+    MOE_TRY(cuda_check(cudaMemsetAsync(dW_gate_up, 0, per, s), "zero dW_gate_up"));
+    return cuda_check(cudaMemsetAsync(dW_down, 0, (size_t)n_groups * d * I * 2, s),
+                      "zero dW_down");
+  }
+  MOE_REQUIRE(a_gu && h && dy && dx && workspace, MOE_ERR_INVALID_ARG, "%s: null pointer", who);
+  MOE_REQUIRE(al16(x) && al16(a_gu) && al16(h) && al16(dy) && al16(dx), MOE_ERR_INVALID_ARG,
+              "%s: activations must be 16-byte aligned", who);
+  MOE_REQUIRE(reinterpret_cast<uintptr_t>(workspace) % 256 == 0, MOE_ERR_INVALID_ARG,
+              "%s: workspace must be 256-byte aligned", who);
+  MOE_REQUIRE(workspace_bytes >= ffn_bwd_ws(dt, rows, I), MOE_ERR_WORKSPACE,
+              "%s: workspace %zu < %zu bytes", who, workspace_bytes, ffn_bwd_ws(dt, rows, I));
+  MOE_TRY(check_device());
+  void* dA = workspace;
+  // Wgrad of the down projection needs only dy and h
+  MOE_TRY(launch_wgrad_gemm(dy, d, h, I, offsets, n_groups, rows, dW_down, s));
+  // Dgrad of the down projection fused with the SwiGLU backward -> dA
+  MOE_TRY(launch_ws_gemm_ex(dy, W_down, 0, offsets, n_groups, rows, I, d, WS_DSWIGLU, true, dA,
+                            2 * I, const_cast<void*>(a_gu), 2 * I, s));
+  // Dgrad of the gate/up projection
+  MOE_TRY(launch_ws_gemm_ex(dA, W_gate_up, 0, offsets, n_groups, rows, d, 2 * I, WS_STORE, true,
+                            dx, d, nullptr, 0, s));
+  // Wgrad of the gate/up projection
+  return launch_wgrad_gemm(dA, 2 * I, x, d, offsets, n_groups, rows, dW_gate_up, s);
+}
+
+moe_status moe_unpermute_backward(const void* dh_out, const void* dx_shared, int N_s,
+                                  const void* dx_perm, const int32_t* inv_row,
+                                  const int32_t* topk_idx, const float* d_logit, const void* E,
+                                  moe_dtype dt, int T, int d, int K, void* du, void* stream) {
+  clear_last_error();
+  MOE_TRY(check_rowwise("moe_unpermute_backward", dt, T, d, K));
+  MOE_REQUIRE(N_s >= 0, MOE_ERR_INVALID_ARG, "moe_unpermute_backward: N_s=%d", N_s);
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE(dh_out && dx_perm && inv_row && topk_idx && d_logit && E && du &&
+                  (N_s == 0 || dx_shared),
+              MOE_ERR_INVALID_ARG, "moe_unpermute_backward: null pointer");
+  MOE_REQUIRE(al16(dh_out) && al16(dx_perm) && al16(E) && al16(du) && al16(dx_shared),
+              MOE_ERR_INVALID_ARG, "moe_unpermute_backward: rows must be 16-byte aligned");
+  MOE_TRY(check_device());
+  return launch_unpermute_backward(dh_out, dx_shared, N_s, dx_perm, inv_row, topk_idx, d_logit, E,
+                                   dt, T, d, K, du, as_stream(stream));
+}
+
+moe_status moe_router_weight_grad(const void* x_perm, const float* d_logit_perm,
+                                  const int32_t* offsets, moe_dtype dt, int N_r, int d, float* dE,
+                                  void* stream) {
+  clear_last_error();
+  MOE_REQUIRE(dt == MOE_F32 || dt == MOE_BF16, MOE_ERR_UNSUPPORTED,
+              "moe_router_weight_grad: dtype must be MOE_F32 or MOE_BF16");
+  MOE_REQUIRE(N_r > 0 && d > 0, MOE_ERR_INVALID_ARG, "moe_router_weight_grad: bad sizes");
+  MOE_REQUIRE(((size_t)d * dtype_bytes(dt)) % 16 == 0, MOE_ERR_UNSUPPORTED,
+              "moe_router_weight_grad: a row must be a multiple of 16 bytes");
+  MOE_REQUIRE(x_perm && d_logit_perm && offsets && dE, MOE_ERR_INVALID_ARG,
+              "moe_router_weight_grad: null pointer");
+  MOE_REQUIRE(al16(x_perm) && al16(dE), MOE_ERR_INVALID_ARG,
+              "moe_router_weight_grad: x_perm and dE must be 16-byte aligned");
+  MOE_TRY(check_device());
+  return launch_router_weight_grad(x_perm, d_logit_perm, offsets, dt, N_r, d, dE,
+                                   as_stream(stream));
+}
+
 moe_status moe_device_status(int* flags) {
   clear_last_error();
   MOE_REQUIRE(flags, MOE_ERR_INVALID_ARG, "moe_device_status: null pointer");

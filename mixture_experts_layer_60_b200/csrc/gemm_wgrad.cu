@@ -1,0 +1,311 @@
+// Grouped weight-gradient GEMM on tcgen05 (the Wgrad pass that "DeepSeek V3 &
+// R1 論文研究", section FP8 mixed precision, names beside Fprop and Dgrad):
+// for every expert g with token rows [off_g, off_g+1),
+//   C_g[m, n] = sum over those rows r of A[r, m] * B[r, n]
+// A [rows, M] and B [rows, N] are row-major activations, so both MMA operands
+// are MN-major (the contraction runs over rows).  dW_down = dy^T h and
+// dW_gate_up = dA^T x are the two uses.
+//
+// Tile: 128 rows of C (one M=128 MMA) x 256 columns (N=256), 64 token rows per
+// K step, 4 shared-memory stages of 48 KB (A: two [64 tok][64 m] TMA boxes,
+// B: four [64 tok][64 n] boxes, 128-byte swizzle), two TMEM accumulators of
+// 256 columns so the epilogue of one tile overlaps the MMAs of the next.
+// The last K step of a group is ragged: its A rows past the group's end are
+// zeroed in shared memory (they hold the next expert's tokens) before the
+// MMAs read them, and only ceil(valid/16) MMAs are issued.  A group with no
+// tokens gets C_g = 0 from the epilogue without touching TMEM.
+//
+// Roles: warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer (the whole
+// warp zeroes ragged rows, one lane issues), warps 2-9 epilogue (warp w
+// reads TMEM lanes 32*(w%4).. = C rows and one 128-column half).  Every wait
+// is bounded (1 s) and reported through the device error word.
+#include "launch.h"
+#include "sm100.cuh"
+
+namespace moe {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;              // token rows per stage
+constexpr int STAGES = 4;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr uint64_t kWaitNs = 1000000000ull;
+constexpr uint32_t TMEM_COLS = 512;
+
+constexpr int BOX_BYTES = 64 * BK * 2;         // one [64 tok][64 mn] bf16 box: 8 KB
+constexpr int A_BYTES = 2 * BOX_BYTES;         // 16 KB
+constexpr int B_BYTES = 4 * BOX_BYTES;         // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int OFF_BAR = STAGES * STAGE_BYTES;
+constexpr int N_BARS = 2 * STAGES + 5;
+constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
+constexpr int SMEM_BYTES = OFF_MISC + 16;
+constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
+
+struct WgParams {
+  const int32_t* offsets;   // [n_groups+1] or nullptr (one group of `rows`)
+  int n_groups;
+  int rows;
+  int M, N;
+  __nv_bfloat16* C;         // [G, M, N]
+  int* err;
+};
+
+__device__ __forceinline__ void group_rows(const WgParams& p, int g, int& r0, int& cnt) {
+  if (p.offsets) {
+    r0 = p.offsets[g];
+    cnt = p.offsets[g + 1] - r0;
+  } else {
+    r0 = 0;
+    cnt = p.rows;
+  }
+}
+
+__device__ __forceinline__ void raise_abort(volatile int* abort, int* err) {
+  *abort = 1;
+  atomicOr(err, ERR_GEMM_TIMEOUT);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    wgrad_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                      const __grid_constant__ CUtensorMap tmB, const WgParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;      // [2]
+  uint64_t* tempty = tfull + 2;          // [2]
+  uint64_t* mma_done = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = p.offsets ? p.n_groups : 1;
+  const int n_m = p.M / BM, n_n = p.N / BN;
+  const int per_group = n_m * n_n;
+  const int total = G * per_group;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], 32 * kEpiWarps); }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const int g = t / per_group, loc = t - g * per_group;
+        const int mt = loc / n_n, nt = loc - mt * n_n;
+        int r0, cnt;
+        group_rows(p, g, r0, cnt);
+        const int nkb = (cnt + BK - 1) / BK;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, kWaitNs)) {
+            raise_abort(abort_flag, p.err);
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+          uint8_t* a_dst = smem + stage * STAGE_BYTES;
+          uint8_t* b_dst = a_dst + A_BYTES;
+          const int row = r0 + kb * BK;
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+            tma_load_2d(a_dst + j * BOX_BYTES, &tmA, mt * BM + 64 * j, row, &full[stage]);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            tma_load_2d(b_dst + j * BOX_BYTES, &tmB, nt * BN + 64 * j, row, &full[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+      for (int s = 0; s < STAGES; ++s)
+        mbar_wait_bounded(&full[s], ((s < stage) ? phase : phase ^ 1), nullptr, kWaitNs);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    int stage = 0, used = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    const uint32_t idesc = idesc_bf16_f32_major(BM, BN, true, true);
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      const int g = t / per_group;
+      int r0, cnt;
+      group_rows(p, g, r0, cnt);
+      if (cnt <= 0) continue;
+      const int ab = used & 1;
+      const uint32_t tpar = ((used >> 1) & 1) ^ 1;
+      ++used;
+      const bool got = mbar_wait_bounded(&tempty[ab], tpar, abort_flag, kWaitNs);
+      if (!__all_sync(0xffffffffu, got)) {
+        if (lane == 0) raise_abort(abort_flag, p.err);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + ab * BN;
+      const int nkb = (cnt + BK - 1) / BK;
+      for (int kb = 0; kb < nkb; ++kb) {
+        const bool f = mbar_wait_bounded(&full[stage], phase, abort_flag, kWaitNs);
+        if (!__all_sync(0xffffffffu, f)) {
+          if (lane == 0) raise_abort(abort_flag, p.err);
+          ok = false;
+          break;
+        }
+        uint8_t* a_st = smem + stage * STAGE_BYTES;
+        const int valid = min(BK, cnt - kb * BK);
+        const int nks = (valid + 15) / 16;
+        if (valid < nks * 16) {
+          // rows [valid, nks*16) of both A boxes belong to the next group: zero them
+          const int zrows = nks * 16 - valid;
+          const int chunks = zrows * 8;                   // 16-byte chunks per box
+          for (int i = lane; i < 2 * chunks; i += 32) {
+            const int box = i / chunks, rem = i - box * chunks;
+            uint8_t* dst = a_st + box * BOX_BYTES + (valid + (rem >> 3)) * 128 + (rem & 7) * 16;
+            *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+          }
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t a0 = smem_u32(a_st), b0 = a0 + A_BYTES;
+          for (int k = 0; k < nks; ++k)
+            mma_f16_ss(d_tmem, smem_desc_mn_sw128(a0 + k * 2048, BOX_BYTES),
+                       smem_desc_mn_sw128(b0 + k * 2048, BOX_BYTES), idesc, (kb | k) != 0);
+          mma_commit(&empty[stage]);
+        }
+        __syncwarp();
+        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+      }
+      if (lane == 0) mma_commit(&tfull[ab]);
+      __syncwarp();
+    }
+    if (lane == 0) {
+      mma_commit(mma_done);
+      mbar_wait_bounded(mma_done, 0, nullptr, kWaitNs);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int q = warp & 3;                       // TMEM lane quarter = C rows q*32..
+    const int half = (warp - 2) >> 2;             // 128-column half of the tile
+    int used = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      const int g = t / per_group, loc = t - g * per_group;
+      const int mt = loc / n_n, nt = loc - mt * n_n;
+      int r0, cnt;
+      group_rows(p, g, r0, cnt);
+      const int m = mt * BM + q * 32 + lane;
+      __nv_bfloat16* dst_row = p.C + ((size_t)g * p.M + m) * p.N + nt * BN + half * 128;
+      if (cnt <= 0) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          reinterpret_cast<uint4*>(dst_row)[i] = make_uint4(0u, 0u, 0u, 0u);
+        continue;
+      }
+      const int ab = used & 1;
+      const uint32_t tpar = (used >> 1) & 1;
+      ++used;
+      const bool got = mbar_wait_bounded(&tfull[ab], tpar, abort_flag, kWaitNs);
+      if (!__all_sync(0xffffffffu, got)) {
+        if (lane == 0) raise_abort(abort_flag, p.err);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tl = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ab * BN + half * 128;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tl + c * 32, r);
+        tmem_wait_ld();
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          __nv_bfloat162 pr = __floats2bfloat162_rn(__uint_as_float(r[2 * i]),
+                                                    __uint_as_float(r[2 * i + 1]));
+          w[i] = *reinterpret_cast<uint32_t*>(&pr);
+        }
+        uint4* d4 = reinterpret_cast<uint4*>(dst_row + c * 32);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[ab]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace
+
+moe_status make_tmap_2d(CUtensorMap* tm, const void* base, CUtensorMapDataType dtype,
+                        int elem_bytes, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                        uint32_t box_outer);
+
+moe_status launch_wgrad_gemm(const void* A, int M, const void* B, int N, const int32_t* offsets,
+                             int n_groups, int rows, void* C, cudaStream_t s) {
+  const int G = offsets ? n_groups : 1;
+  if (G <= 0) return MOE_OK;
+  if (M % BM || N % BN)
+    return fail(MOE_ERR_UNSUPPORTED, "wgrad gemm: M=%d must be a multiple of %d, N=%d of %d", M,
+                BM, N, BN);
+  if (rows <= 0) {
+    // every group is empty: C = 0
+    return cuda_check(cudaMemsetAsync(C, 0, (size_t)G * M * N * 2, s), "wgrad zero fill");
+  }
+  CUtensorMap tmA, tmB;
+  moe_status st = make_tmap_2d(&tmA, A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, rows, 64, BK);
+  if (st != MOE_OK) return st;
+  st = make_tmap_2d(&tmB, B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, rows, 64, BK);
+  if (st != MOE_OK) return st;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(wgrad_gemm_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
+    if (e != cudaSuccess) return cuda_check(e, "wgrad smem attribute");
+    attr_set = true;
+  }
+  WgParams p;
+  p.offsets = offsets;
+  p.n_groups = G;
+  p.rows = rows;
+  p.M = M;
+  p.N = N;
+  p.C = static_cast<__nv_bfloat16*>(C);
+  p.err = device_error_word();
+  if (!p.err) return fail(MOE_ERR_CUDA, "device error word unavailable");
+  const long long tiles = (long long)G * (M / BM) * (N / BN);
+  int grid = sm_count();
+  if (tiles < grid) grid = (int)tiles;
+  wgrad_gemm_kernel<<<grid, kThreads, SMEM_ALLOC, s>>>(tmA, tmB, p);
+  return cuda_check(cudaGetLastError(), "wgrad gemm launch");
+}
+
+}  // namespace moe

@@ -47,6 +47,7 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr int W_BYTES = WROWS * BK * 2;       // 32 KB
 constexpr int X_BYTES = TMAX * BK * 2;        // 32 KB
 constexpr int XBOX_BYTES = XBOX * BK * 2;     // 8 KB
+constexpr int WBOX_MN_BYTES = 64 * BK * 2;    // MN-major weights: one [64 K][64 N] box, 8 KB
 constexpr int OFF_X = STAGES * W_BYTES;
 constexpr int OFF_STAGE_OUT = OFF_X + STAGES * X_BYTES;   // one 2 KB transpose patch per epilogue warp
 constexpr int OFF_BAR = OFF_STAGE_OUT + kEpiWarps * 2048;
@@ -60,17 +61,21 @@ struct WsParams {
   const int32_t* offsets;   // [n_groups+1] or nullptr (one group of `rows`)
   int n_groups;
   int rows;
-  int N;                    // output columns (SWIGLU: I; STORE: d)
+  int N;                    // output columns (SWIGLU*: I; STORE: d; DSWIGLU: I)
   int K;
-  int b_rows_per_group;
-  int half_b;               // SWIGLU: I
+  int b_rows_per_group;     // K-major weights: rows of W per group
+  int half_b;               // SWIGLU*: I (row offset of W_up inside a group)
   __nv_bfloat16* C;
+  int ldc;                  // row stride of C in elements
+  __nv_bfloat16* S;         // SWIGLU_SAVE: pre-activations written; DSWIGLU: read
+  int lds;                  // row stride of S (2I)
   int* err;
 };
 
-template <bool SWIGLU>
+template <int EPI>
 struct TileMath {
-  static constexpr int OUT_COLS = SWIGLU ? 128 : 256;   // output columns per weight tile
+  static constexpr bool SW = EPI == WS_SWIGLU || EPI == WS_SWIGLU_SAVE;
+  static constexpr int OUT_COLS = SW ? 128 : 256;   // output columns per weight tile
 };
 
 // Token tiling of a group of m rows: tiles of `step` rows (a multiple of 16,
@@ -110,11 +115,12 @@ __device__ __forceinline__ void raise_abort(volatile int* abort, int* err) {
 // SiLU for a bf16 result: fast exponential and division are well inside bf16 rounding.
 __device__ __forceinline__ float silu_f(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
 
-template <bool SWIGLU>
+template <int EPI, bool WMN>
 __global__ void __launch_bounds__(kThreads, 1)
     ws_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                    const WsParams p) {
-  constexpr int OUT_COLS = TileMath<SWIGLU>::OUT_COLS;
+  constexpr int OUT_COLS = TileMath<EPI>::OUT_COLS;
+  constexpr bool SWIGLU = TileMath<EPI>::SW;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -213,9 +219,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mbar_arrive_expect_tx(&full[stage], bytes);
           uint8_t* w_dst = sW + stage * W_BYTES;
-          tma_load_2d(w_dst, &tmW, kb * BK, wrow, &full[stage]);
-          tma_load_2d(w_dst + W_BYTES / 2, &tmW, kb * BK, wrow + (SWIGLU ? p.half_b : 128),
-                      &full[stage]);
+          if (WMN) {
+            // weights stored [K rows][N cols]: four [64 K][64 N] boxes of columns nt*256 + 64j
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              tma_load_2d(w_dst + j * WBOX_MN_BYTES, &tmW, nt * 256 + 64 * j,
+                          g * p.K + kb * BK, &full[stage]);
+          } else {
+            tma_load_2d(w_dst, &tmW, kb * BK, wrow, &full[stage]);
+            tma_load_2d(w_dst + W_BYTES / 2, &tmW, kb * BK, wrow + (SWIGLU ? p.half_b : 128),
+                        &full[stage]);
+          }
           uint8_t* x_dst = sX + stage * X_BYTES;
           for (int b = 0; b < nbox; ++b)
             tma_load_2d(x_dst + b * XBOX_BYTES, &tmX, kb * BK, tok0 + b * XBOX, &full[stage]);
@@ -235,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int g, nt, tok0, count;
         decode_tile(t, prefix, roff, G, g, nt, tok0, count);
         const int n_mma = (count + 15) / 16 * 16;
-        const uint32_t idesc = idesc_bf16_f32(128, n_mma);
+        const uint32_t idesc = idesc_bf16_f32_major(128, n_mma, WMN, false);
         if (!mbar_wait_bounded(tempty, tphase ^ 1, abort_flag, kWaitNs)) {
           raise_abort(abort_flag, p.err);
           break;
@@ -254,9 +268,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int k = 0; k < BK / 16; ++k) {
             const uint64_t xd = smem_desc_k_sw128(x0 + k * 32);
             const uint32_t acc = (kb | k) != 0;
-            mma_f16_ss(tmem_base, smem_desc_k_sw128(w0 + k * 32), xd, idesc, acc);
-            mma_f16_ss(tmem_base + 256, smem_desc_k_sw128(w0 + W_BYTES / 2 + k * 32), xd, idesc,
-                       acc);
+            const uint64_t a0 = WMN ? smem_desc_mn_sw128(w0 + k * 2048, WBOX_MN_BYTES)
+                                    : smem_desc_k_sw128(w0 + k * 32);
+            const uint64_t a1 = WMN ? smem_desc_mn_sw128(w0 + W_BYTES / 2 + k * 2048,
+                                                         WBOX_MN_BYTES)
+                                    : smem_desc_k_sw128(w0 + W_BYTES / 2 + k * 32);
+            mma_f16_ss(tmem_base, a0, xd, idesc, acc);
+            mma_f16_ss(tmem_base + 256, a1, xd, idesc, acc);
           }
           mma_commit(&empty[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -284,32 +302,66 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t tl = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
       const int nch = (count + 31) / 32;
+      if (EPI == WS_DSWIGLU) {
+        // dh[tok, col] from TMEM; a = S[tok, col], b = S[tok, I + col]:
+        //   dA[tok, col] = dh * b * SiLU'(a),  dA[tok, I + col] = dh * SiLU(a).
+        // Lane = feature column, so each access of the warp covers 64 contiguous bytes.
+        for (int c = ch; c < nch; c += 2) {
+          uint32_t r0[32], r1[32];
+          tmem_ld_32x32b_x32(tl + c * 32, r0);
+          tmem_ld_32x32b_x32(tl + 256 + c * 32, r1);
+          tmem_wait_ld();
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int col = nt * 256 + hh * 128 + q * 32 + lane;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int tok = c * 32 + j;
+              if (tok < count) {
+                const size_t row = (size_t)(tok0 + tok);
+                const float dhv = __uint_as_float(hh == 0 ? r0[j] : r1[j]);
+                const float a = __bfloat162float(p.S[row * p.lds + col]);
+                const float b = __bfloat162float(p.S[row * p.lds + p.N + col]);
+                const float sg = __fdividef(1.0f, 1.0f + __expf(-a));
+                p.C[row * p.ldc + col] = __float2bfloat16_rn(dhv * b * (sg * (1.0f + a * (1.0f - sg))));
+                p.C[row * p.ldc + p.N + col] = __float2bfloat16_rn(dhv * a * sg);
+              }
+            }
+          }
+        }
+      } else
       for (int c = ch; c < nch; c += 2) {
         uint32_t r0[32], r1[32];
         tmem_ld_32x32b_x32(tl + c * 32, r0);
         tmem_ld_32x32b_x32(tl + 256 + c * 32, r1);
         tmem_wait_ld();
-        const int half_n = SWIGLU ? 1 : 2;
+        // outputs: SWIGLU h; SWIGLU_SAVE h, gate and up pre-activations; STORE two halves
+        constexpr int n_out = EPI == WS_SWIGLU_SAVE ? 3 : (SWIGLU ? 1 : 2);
 #pragma unroll
-        for (int hh = 0; hh < half_n; ++hh) {
+        for (int hh = 0; hh < n_out; ++hh) {
           // patch[j][lane] = value of token (c*32 + j), column (q*32 + lane)
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             float v;
-            if (SWIGLU) v = silu_f(__uint_as_float(r0[j])) * __uint_as_float(r1[j]);
+            if (SWIGLU && hh == 0) v = silu_f(__uint_as_float(r0[j])) * __uint_as_float(r1[j]);
+            else if (SWIGLU) v = __uint_as_float(hh == 1 ? r0[j] : r1[j]);
             else v = __uint_as_float(hh == 0 ? r0[j] : r1[j]);
             patch[j * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
           }
           __syncwarp();
           // 32 token rows x 64 bytes: lane -> (row lane/4 + 8*it, 16-byte chunk lane%4)
-          const int col0 = nt * OUT_COLS + hh * 128 + q * 32;
+          __nv_bfloat16* base;
+          int ld, col0;
+          if (!SWIGLU) { base = p.C; ld = p.ldc; col0 = nt * OUT_COLS + hh * 128 + q * 32; }
+          else if (hh == 0) { base = p.C; ld = p.ldc; col0 = nt * 128 + q * 32; }
+          else { base = p.S; ld = p.lds; col0 = (hh == 2 ? p.N : 0) + nt * 128 + q * 32; }
 #pragma unroll
           for (int it = 0; it < 4; ++it) {
             const int j = it * 8 + (lane >> 2);
             const int tok = c * 32 + j;
             const uint4 v = *reinterpret_cast<const uint4*>(patch + j * 32 + (lane & 3) * 8);
             if (tok < count) {
-              __nv_bfloat16* dst = p.C + (size_t)(tok0 + tok) * p.N + col0 + (lane & 3) * 8;
+              __nv_bfloat16* dst = base + (size_t)(tok0 + tok) * ld + col0 + (lane & 3) * 8;
               *reinterpret_cast<uint4*>(dst) = v;
             }
           }
@@ -338,18 +390,21 @@ moe_status make_tmap_2d(CUtensorMap* tm, const void* base, CUtensorMapDataType d
 
 namespace {
 
-template <bool SWIGLU>
+template <int EPI, bool WMN>
 moe_status ws_launch(const void* X, const void* W, int b_rows_per_group, const int32_t* offsets,
-                     int n_groups, int rows, int N, int K, void* C, cudaStream_t s) {
-  constexpr int OUT_COLS = TileMath<SWIGLU>::OUT_COLS;
+                     int n_groups, int rows, int N, int K, void* C, int ldc, void* S, int lds,
+                     cudaStream_t s) {
+  constexpr int OUT_COLS = TileMath<EPI>::OUT_COLS;
   CUtensorMap tmW, tmX;
   const int G = offsets ? n_groups : 1;
-  moe_status st = make_tmap_2d(&tmW, W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K,
-                               (uint64_t)G * b_rows_per_group, BK, 128);
+  moe_status st = WMN ? make_tmap_2d(&tmW, W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N,
+                                     (uint64_t)G * K, 64, BK)
+                      : make_tmap_2d(&tmW, W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K,
+                                     (uint64_t)G * b_rows_per_group, BK, 128);
   if (st != MOE_OK) return st;
   st = make_tmap_2d(&tmX, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, rows, BK, XBOX);
   if (st != MOE_OK) return st;
-  auto kern = ws_gemm_kernel<SWIGLU>;
+  auto kern = ws_gemm_kernel<EPI, WMN>;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e =
@@ -364,8 +419,11 @@ moe_status ws_launch(const void* X, const void* W, int b_rows_per_group, const i
   p.N = N;
   p.K = K;
   p.b_rows_per_group = b_rows_per_group;
-  p.half_b = SWIGLU ? b_rows_per_group / 2 : 0;
+  p.half_b = TileMath<EPI>::SW ? b_rows_per_group / 2 : 0;
   p.C = static_cast<__nv_bfloat16*>(C);
+  p.ldc = ldc;
+  p.S = static_cast<__nv_bfloat16*>(S);
+  p.lds = lds;
   p.err = device_error_word();
   if (!p.err) return fail(MOE_ERR_CUDA, "device error word unavailable");
   const long long max_tiles = ((long long)(rows + TMAX - 1) / TMAX + (offsets ? G : 0)) * (N / OUT_COLS);
@@ -380,16 +438,40 @@ moe_status ws_launch(const void* X, const void* W, int b_rows_per_group, const i
 moe_status launch_ws_gemm(const void* X, const void* W, int b_rows_per_group,
                           const int32_t* offsets, int n_groups, int rows, int N, int K,
                           bool swiglu, void* C, cudaStream_t s) {
+  return launch_ws_gemm_ex(X, W, b_rows_per_group, offsets, n_groups, rows, N, K,
+                           swiglu ? WS_SWIGLU : WS_STORE, false, C, N, nullptr, 0, s);
+}
+
+moe_status launch_ws_gemm_ex(const void* X, const void* W, int b_rows_per_group,
+                             const int32_t* offsets, int n_groups, int rows, int N, int K,
+                             WsEpi epi, bool w_mn, void* C, int ldc, void* S, int lds,
+                             cudaStream_t s) {
   if (rows <= 0) return MOE_OK;
   if (K % BK) return fail(MOE_ERR_UNSUPPORTED, "ws gemm: K=%d not a multiple of %d", K, BK);
   if (offsets && n_groups > kMaxGroups)
     return fail(MOE_ERR_UNSUPPORTED, "ws gemm: at most %d groups", kMaxGroups);
-  if (swiglu) {
-    if (N % 128) return fail(MOE_ERR_UNSUPPORTED, "ws gemm swiglu: N=%d %% 128", N);
-    return ws_launch<true>(X, W, b_rows_per_group, offsets, n_groups, rows, N, K, C, s);
+  const bool sw = epi == WS_SWIGLU || epi == WS_SWIGLU_SAVE;
+  if (sw && N % 128) return fail(MOE_ERR_UNSUPPORTED, "ws gemm swiglu: N=%d %% 128", N);
+  if (!sw && N % 256) return fail(MOE_ERR_UNSUPPORTED, "ws gemm: N=%d %% 256", N);
+  if (w_mn && sw) return fail(MOE_ERR_UNSUPPORTED, "ws gemm: MN-major weights with swiglu");
+  switch (epi) {
+    case WS_SWIGLU:
+      return ws_launch<WS_SWIGLU, false>(X, W, b_rows_per_group, offsets, n_groups, rows, N, K,
+                                         C, ldc, S, lds, s);
+    case WS_SWIGLU_SAVE:
+      return ws_launch<WS_SWIGLU_SAVE, false>(X, W, b_rows_per_group, offsets, n_groups, rows,
+                                              N, K, C, ldc, S, lds, s);
+    case WS_STORE:
+      return w_mn ? ws_launch<WS_STORE, true>(X, W, b_rows_per_group, offsets, n_groups, rows, N,
+                                              K, C, ldc, S, lds, s)
+                  : ws_launch<WS_STORE, false>(X, W, b_rows_per_group, offsets, n_groups, rows,
+                                               N, K, C, ldc, S, lds, s);
+    case WS_DSWIGLU:
+      if (!w_mn) return fail(MOE_ERR_UNSUPPORTED, "ws gemm dswiglu: needs MN-major weights");
+      return ws_launch<WS_DSWIGLU, true>(X, W, b_rows_per_group, offsets, n_groups, rows, N, K,
+                                         C, ldc, S, lds, s);
   }
-  if (N % 256) return fail(MOE_ERR_UNSUPPORTED, "ws gemm store: N=%d %% 256", N);
-  return ws_launch<false>(X, W, b_rows_per_group, offsets, n_groups, rows, N, K, C, s);
+  return fail(MOE_ERR_INVALID_ARG, "ws gemm: unknown epilogue %d", (int)epi);
 }
 
 }  // namespace moe

@@ -53,6 +53,22 @@ moe_status launch_tc_gemm(const void* A, const void* B, int b_rows_per_group,
 moe_status launch_ws_gemm(const void* X, const void* W, int b_rows_per_group,
                           const int32_t* offsets, int n_groups, int rows, int N, int K,
                           bool swiglu, void* C, cudaStream_t s);
+// Epilogues: SWIGLU  C = SiLU(gate) * up (N = I columns);
+//            SWIGLU_SAVE  the same, plus S[:, 0:I] = gate, S[:, I:2I] = up;
+//            STORE   C = the product (N columns);
+//            DSWIGLU dh = the product (N = I columns), a = S[:, 0:I], b = S[:, I:2I]:
+//                    C[:, 0:I] = dh * b * SiLU'(a), C[:, I:2I] = dh * SiLU(a).
+// w_mn: W is stored [G*K rows][N cols] (N contiguous) instead of [G*rows_per_group][K].
+enum WsEpi { WS_SWIGLU = 0, WS_STORE = 1, WS_SWIGLU_SAVE = 2, WS_DSWIGLU = 3 };
+moe_status launch_ws_gemm_ex(const void* X, const void* W, int b_rows_per_group,
+                             const int32_t* offsets, int n_groups, int rows, int N, int K,
+                             WsEpi epi, bool w_mn, void* C, int ldc, void* S, int lds,
+                             cudaStream_t s);
+
+// gemm_wgrad.cu --------------------------------------------------------------
+// C[g] [M, N] = sum over the rows r of group g of A[r, :]^T B[r, :] (bf16 in and out).
+moe_status launch_wgrad_gemm(const void* A, int M, const void* B, int N, const int32_t* offsets,
+                             int n_groups, int rows, void* C, cudaStream_t s);
 
 // gemm_fp8.cu ----------------------------------------------------------------
 moe_status launch_fp8_gemm(const void* A, const float* a_scale, const void* B,
@@ -70,5 +86,20 @@ moe_status launch_combine(const void* u, const void* y_shared, int N_s, const vo
                           int d, int K, void* h_out, cudaStream_t s);
 moe_status launch_bias_update(float* b, const int32_t* counts, int N_r, int T, int K,
                               float gamma, cudaStream_t s);
+
+// backward.cu ----------------------------------------------------------------
+moe_status launch_combine_backward(const void* dh, const void* u, const void* E,
+                                   const void* y_perm, const int32_t* inv_row,
+                                   const int32_t* idx, const float* gate, moe_dtype dt, int T,
+                                   int d, int K, void* dy_perm, float* d_gate, float* d_logit,
+                                   float* d_logit_perm, cudaStream_t s);
+moe_status launch_unpermute_backward(const void* dh, const void* dx_shared, int N_s,
+                                     const void* dx_perm, const int32_t* inv_row,
+                                     const int32_t* idx, const float* d_logit, const void* E,
+                                     moe_dtype dt, int T, int d, int K, void* du,
+                                     cudaStream_t s);
+moe_status launch_router_weight_grad(const void* x_perm, const float* d_logit_perm,
+                                     const int32_t* offsets, moe_dtype dt, int N_r, int d,
+                                     float* dE, cudaStream_t s);
 
 }  // namespace moe

@@ -97,6 +97,12 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
   return p;
 }
 
+// Orders this thread's generic-proxy writes to shared memory before later
+// async-proxy reads of it (tcgen05.mma operands, TMA stores).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ TMEM / tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -187,6 +193,22 @@ __device__ __forceinline__ uint64_t smem_desc_k_sw128(uint32_t saddr) {
   return d;
 }
 
+// Shared-memory matrix descriptor for an MN-major tile written by TMA with
+// 128-byte swizzle as boxes of [k rows][64 MN elements]: each box row holds
+// 64 consecutive MN elements (128 bytes), 8 K rows form one 1024-byte swizzle
+// atom (stride byte offset 1024 between 8-row K groups), and the next 64 MN
+// elements start `mn_stride` bytes further (leading byte offset).  A 16-row
+// K step is two atoms: +2048 bytes on the start address.
+__device__ __forceinline__ uint64_t smem_desc_mn_sw128(uint32_t saddr, uint32_t mn_stride) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+  d |= (uint64_t)((mn_stride >> 4) & 0x3FFF) << 16;   // leading byte offset: next 64 MN
+  d |= (uint64_t)(1024 >> 4) << 32;                    // stride byte offset: next 8 K rows
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
 // Instruction descriptor, kind::f16: f32 accumulator, bf16 A and B, both K-major.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4)                        // D format f32
@@ -194,6 +216,11 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          | (1u << 10)                     // B format bf16
          | ((uint32_t)(N >> 3) << 17)     // N / 8
          | ((uint32_t)(M >> 4) << 24);    // M / 16
+}
+
+// Same with the operands' major-ness: bit 15 set = A is MN-major, bit 16 = B.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_major(int M, int N, bool a_mn, bool b_mn) {
+  return idesc_bf16_f32(M, N) | (a_mn ? 1u << 15 : 0u) | (b_mn ? 1u << 16 : 0u);
 }
 
 // Instruction descriptor, kind::f8f6f4: f32 accumulator, e4m3 A and B, K-major.

@@ -4,16 +4,22 @@ MoELayer owns the layer's device state (centroids, bias, expert weights,
 FP8 copies of them) and the per-step buffers, and runs one step as
     moe_route -> [moe_quantize_1x128] -> moe_permute -> moe_expert_ffn (routed)
     -> moe_expert_ffn (each shared expert) -> moe_combine [-> moe_bias_update]
-on one CUDA stream.  Every step of the layer runs in libmoe's kernels; this
+on one CUDA stream.  For training (bf16), forward_train keeps the activations
+the backward needs and backward(dh) returns du and fills self.grad with the
+gradients of E and of every expert weight.  Every step of the layer runs in libmoe's kernels; this
 module only allocates buffers and sequences calls.
 """
 from __future__ import annotations
 
 import torch
 
-from . import (MOE_BF16, MOE_E4M3, MOE_F32, moe_bias_update, moe_route_grouped, moe_combine, moe_expert_down,
-               moe_expert_ffn, moe_expert_ffn_workspace_size, moe_expert_gate_up, moe_permute, moe_permute_workspace_size,
-               moe_quantize_128x128, moe_quantize_1x128, moe_route, moe_route_workspace_size)
+from . import (MOE_BF16, MOE_E4M3, MOE_F32, moe_bias_update, moe_combine, moe_combine_backward,
+               moe_expert_down, moe_expert_ffn, moe_expert_ffn_backward,
+               moe_expert_ffn_backward_workspace_size, moe_expert_ffn_workspace_size,
+               moe_expert_gate_up, moe_expert_gate_up_save, moe_permute,
+               moe_permute_workspace_size, moe_quantize_128x128, moe_quantize_1x128, moe_route,
+               moe_route_grouped, moe_route_workspace_size, moe_router_weight_grad,
+               moe_unpermute_backward)
 from .configs import LayerConfig
 
 GAMMA = 0.001
@@ -126,6 +132,83 @@ class MoELayer:
         moe_combine(u_res, self.y_shared if c.N_s else None, self.y_perm, self.inv_row,
                     self.topk_gate, h, stream)
         return h
+
+    # -- training (bf16): forward that keeps activations, then the backward ---
+    def _alloc_train(self, T):
+        c, dev = self.cfg, self.device
+        R, bf = T * c.K, torch.bfloat16
+        self.a_gu = torch.empty(R, 2 * c.I, dtype=bf, device=dev)
+        self.h_s = torch.empty(c.N_s, T, c.I, dtype=bf, device=dev)
+        self.a_s = torch.empty(c.N_s, T, 2 * c.I, dtype=bf, device=dev)
+        self.dy_perm = torch.empty(R, c.d, dtype=bf, device=dev)
+        self.d_gate = torch.empty(T, c.K, dtype=torch.float32, device=dev)
+        self.d_logit = torch.empty(T, c.K, dtype=torch.float32, device=dev)
+        self.d_logit_perm = torch.empty(R, dtype=torch.float32, device=dev)
+        self.dx_perm = torch.empty(R, c.d, dtype=bf, device=dev)
+        self.dx_s = torch.empty(c.N_s, T, c.d, dtype=bf, device=dev)
+        self.du = torch.empty(T, c.d, dtype=bf, device=dev)
+        self.bwd_ws = _ws(moe_expert_ffn_backward_workspace_size(MOE_BF16, max(R, T), c.I), dev)
+        if not hasattr(self, "grad"):
+            self.grad = {k: torch.empty_like(self.W[k][0]) for k in
+                         ("W_gate_up", "W_down", "Ws_gate_up", "Ws_down")}
+            self.grad["E"] = torch.empty(c.N_r, c.d, dtype=torch.float32, device=dev)
+        self.T_train = T
+
+    def forward_train(self, u: torch.Tensor, stream=None) -> torch.Tensor:
+        """forward() that also keeps the gate/up pre-activations and h of the
+        routed and shared experts for backward().  bf16 layers only."""
+        c = self.cfg
+        if c.dtype != "bf16":
+            raise ValueError("the backward is implemented for bf16 layers")
+        T = u.shape[0]
+        if T != self.T_alloc:
+            self._alloc(T)
+        if getattr(self, "T_train", None) != T:
+            self._alloc_train(T)
+        if c.n_groups > 1:
+            moe_route_grouped(u, self.E, self.b, c.K, c.n_groups, c.topk_groups, self.topk_idx,
+                              self.topk_gate, self.counts, self.route_ws, stream)
+        else:
+            moe_route(u, self.E, self.b, c.K, self.topk_idx, self.topk_gate, self.counts,
+                      self.route_ws, stream)
+        moe_permute(u, self.topk_idx, c.N_r, self.x_perm, self.offsets, self.perm_src,
+                    self.inv_row, self.perm_ws, stream=stream)
+        wgu, wdn = self.W["W_gate_up"][0], self.W["W_down"][0]
+        moe_expert_gate_up_save(self.x_perm, self.offsets, wgu, self.h_mid, self.a_gu, stream)
+        moe_expert_down(self.h_mid, self.offsets, wdn, self.y_perm, stream=stream)
+        wsgu, wsdn = self.W["Ws_gate_up"][0], self.W["Ws_down"][0]
+        for j in range(c.N_s):
+            moe_expert_gate_up_save(u, self.shared_offsets, wsgu[j:j + 1], self.h_s[j],
+                                    self.a_s[j], stream)
+            moe_expert_down(self.h_s[j], self.shared_offsets, wsdn[j:j + 1], self.y_shared[j],
+                            stream=stream)
+        moe_combine(u, self.y_shared if c.N_s else None, self.y_perm, self.inv_row,
+                    self.topk_gate, self.h_out, stream)
+        self._u = u
+        return self.h_out
+
+    def backward(self, dh: torch.Tensor, stream=None) -> torch.Tensor:
+        """Gradients for upstream dh = dL/dh' of the last forward_train:
+        returns du (overwritten by the next call) and fills self.grad
+        (E: float32; W_gate_up, W_down, Ws_gate_up, Ws_down: bf16)."""
+        c, g = self.cfg, self.grad
+        u = self._u
+        moe_combine_backward(dh, u, self.E, self.y_perm, self.inv_row, self.topk_idx,
+                             self.topk_gate, self.dy_perm, self.d_gate, self.d_logit,
+                             self.d_logit_perm, stream)
+        moe_expert_ffn_backward(self.x_perm, self.offsets, self.W["W_gate_up"][0],
+                                self.W["W_down"][0], self.a_gu, self.h_mid, self.dy_perm,
+                                self.dx_perm, g["W_gate_up"], g["W_down"], self.bwd_ws, stream)
+        wsgu, wsdn = self.W["Ws_gate_up"][0], self.W["Ws_down"][0]
+        for j in range(c.N_s):
+            moe_expert_ffn_backward(u, self.shared_offsets, wsgu[j:j + 1], wsdn[j:j + 1],
+                                    self.a_s[j], self.h_s[j], dh, self.dx_s[j],
+                                    g["Ws_gate_up"][j:j + 1], g["Ws_down"][j:j + 1], self.bwd_ws,
+                                    stream)
+        moe_unpermute_backward(dh, self.dx_s if c.N_s else None, self.dx_perm, self.inv_row,
+                               self.topk_idx, self.d_logit, self.E, self.du, stream)
+        moe_router_weight_grad(self.x_perm, self.d_logit_perm, self.offsets, g["E"], stream)
+        return self.du
 
     def bias_update(self, counts=None, T_total=None, stream=None):
         """b <- b -/+ gamma from the load of the last step (or from the given

@@ -105,3 +105,13 @@ def step_u(cfg: LayerConfig, step: int, device="cuda", T: int | None = None) -> 
     gen.manual_seed(1_000_000 * cfg.seed + step + 1)
     return torch.randn(T, cfg.d, generator=gen, device=device,
                        dtype=torch.float32).to(storage_dtype(cfg))
+
+
+def upstream_grad(cfg: LayerConfig, device="cuda", T: int | None = None,
+                  step: int = 0) -> torch.Tensor:
+    """Upstream gradient dL/dh' [T, d] for a backward: N(0, 1/d) from the seed
+    2_000_000 * seed + step + 1, rounded once to the storage dtype."""
+    T = cfg.T if T is None else T
+    gen = torch.Generator(device=device)
+    gen.manual_seed(2_000_000 * cfg.seed + step + 1)
+    return _normal(gen, (T, cfg.d), cfg.d ** -0.5, device, storage_dtype(cfg))
