@@ -8,7 +8,11 @@ the chain-rule formulas it checks:
   * closed forms: W_down = 0 leaves only the residual in du and gives dE = 0;
     identical experts with K = N_r make h' independent of s, so dE = 0;
   * the gate invariant: scaling every selected s by one factor leaves g
-    unchanged, so sum_k ds_k s_k = 0.
+    unchanged, so sum_k ds_k s_k = 0;
+  * FP8 backward: the Wgrad quantiser equals the pinned forward quantiser on
+    the transpose, its blocks follow the groups, promoted Wgrad/Dgrad with
+    unit scales are plain products, scales act per block row and column, and
+    the FP8 expert and layer backward stay within E4M3's error of the exact one.
 """
 import numpy as np
 import pytest
@@ -148,3 +152,99 @@ def test_silu_grad_is_derivative(z):
     eps = 1e-6
     fd = (O.silu(z + eps) - O.silu(z - eps)) / (2 * eps)
     assert abs(B.silu_grad(z) - fd) < 1e-8
+
+
+# ---------------------------------------------------------------- FP8 backward (reading B5)
+
+def test_quant_128x1_matches_transposed_1x128():
+    """One group of whole 128-row blocks: the Wgrad quantiser is the forward's
+    1x128 quantiser applied to the transpose (an independent, pinned routine)."""
+    rng = np.random.default_rng(21)
+    X = (rng.standard_normal((256, 384)) * rng.uniform(0.1, 10, 384)[None, :]).astype(np.float32)
+    X[:128, 5] = 0.0                                   # an all-zero column block -> scale 1
+    q, sc, blocks = B.quant_128x1_grouped(X, [0, 256])
+    qt, sct = O.quant_1x128(X.T)
+    np.testing.assert_array_equal(q, qt.T)
+    np.testing.assert_array_equal(sc, sct.T)
+    assert blocks == [(0, 0, 128), (0, 128, 256)]
+    assert sc[0, 5] == 1.0
+
+
+def test_quant_128x1_grouped_blocks_follow_groups():
+    """Blocks start at every group's first row, the last one of a group may be
+    short, empty groups have none; each scale is its block's column amax/448."""
+    rng = np.random.default_rng(22)
+    sizes = [0, 3, 128, 130, 0, 257]
+    off = np.concatenate([[0], np.cumsum(sizes)])
+    X = rng.standard_normal((off[-1], 128)).astype(np.float32)
+    q, sc, blocks = B.quant_128x1_grouped(X, off)
+    want = [(1, 0, 3), (2, 3, 131), (3, 131, 259), (3, 259, 261),
+            (5, 261, 389), (5, 389, 517), (5, 517, 518)]
+    assert blocks == want
+    for i, (g, r0, r1) in enumerate(blocks):
+        amax = np.abs(X[r0:r1]).max(axis=0)
+        np.testing.assert_array_equal(sc[i], (amax / np.float32(448)).astype(np.float32))
+        # the largest element of every column maps to +-448 exactly
+        col = np.argmax(np.abs(X[r0:r1]), axis=0)
+        np.testing.assert_array_equal(np.abs(q[r0:r1][col, np.arange(128)]), 448.0)
+
+
+def test_fp8_wgrad_and_dgrad_with_unit_scales_are_plain_products():
+    rng = np.random.default_rng(23)
+    qa = O.e4m3_round(rng.standard_normal((300, 128)) * 8)
+    qb = O.e4m3_round(rng.standard_normal((300, 256)) * 8)
+    blocks = [(0, 0, 100), (1, 100, 228), (1, 228, 300)]
+    ones_a, ones_b = np.ones((3, 128), np.float32), np.ones((3, 256), np.float32)
+    got = B.fp8_wgrad(qa, ones_a, qb, ones_b, blocks, 2)
+    np.testing.assert_array_equal(got[0], qa[:100].T @ qb[:100])
+    np.testing.assert_array_equal(got[1], qa[100:].T @ qb[100:])
+    qdy = O.e4m3_round(rng.standard_normal((7, 256)) * 8)
+    qW = O.e4m3_round(rng.standard_normal((256, 384)) * 8)
+    got = B.fp8_dgrad(qdy, np.ones((7, 2), np.float32), qW, np.ones((2, 3), np.float32))
+    np.testing.assert_array_equal(got, qdy @ qW)
+
+
+def test_fp8_wgrad_scales_apply_per_block_row_and_column():
+    rng = np.random.default_rng(24)
+    qa = O.e4m3_round(rng.standard_normal((200, 128)))
+    qb = O.e4m3_round(rng.standard_normal((200, 128)))
+    sa = rng.uniform(0.5, 2, (2, 128)).astype(np.float32)
+    sb = rng.uniform(0.5, 2, (2, 128)).astype(np.float32)
+    blocks = [(0, 0, 128), (0, 128, 200)]
+    got = B.fp8_wgrad(qa, sa, qb, sb, blocks, 1)[0]
+    want = ((qa[:128] * sa[0]).T @ (qb[:128] * sb[0])) + ((qa[128:] * sa[1]).T @ (qb[128:] * sb[1]))
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+
+
+def test_fp8_ffn_backward_close_to_exact():
+    """The FP8 backward of one expert stays within the error E4M3 quantisation
+    of every GEMM input implies (3-bit mantissa: relative step 2^-3..2^-4, so a
+    few percent per quantised operand, compounded over two chained GEMMs)."""
+    rng = np.random.default_rng(25)
+    R, d, I = 300, 256, 256
+    x = rng.standard_normal((R, d)).astype(np.float32)
+    Wg = (rng.standard_normal((I, d)) / np.sqrt(d)).astype(np.float32)
+    Wu = (rng.standard_normal((I, d)) / np.sqrt(d)).astype(np.float32)
+    Wd = (rng.standard_normal((d, I)) / np.sqrt(I)).astype(np.float32)
+    dy = (rng.standard_normal((R, d)) * 0.05).astype(np.float32)
+    got = B.fp8_swiglu_ffn_backward(x, O.quantise_expert(Wg, Wu, Wd), dy)
+    want = B.swiglu_ffn_backward(x, Wg, Wu, Wd, dy)
+    for name, a, b in zip(["dx", "dW_gate", "dW_up", "dW_down"], got, want[:4]):
+        rel = np.sqrt(np.mean((a - b) ** 2) / np.mean(b ** 2))
+        assert rel < 0.12, (name, rel)
+        assert rel > 1e-3, (name, rel)      # the quantisation really happened
+
+
+def test_fp8_layer_backward_close_to_exact():
+    u, E, routed, shared, idx, dh = _problem(T=40, d=256, N_r=4, K=2, N_s=1, I=128, seed=26)
+    rq = [O.quantise_expert(*ex) for ex in routed]
+    sq = [O.quantise_expert(*ex) for ex in shared]
+    got = B.layer_backward_fp8(u, E, idx, rq, sq, dh)
+    want = B.layer_backward(u, E, idx, routed, shared, dh)
+    for key in ("du", "dE", "d_gate"):
+        a, b = got[key], want[key]
+        rel = np.sqrt(np.mean((a - b) ** 2) / np.mean(b ** 2))
+        assert rel < 0.12, (key, rel)
+    for e in got["routed"]:
+        for a, b in zip(got["routed"][e], want["routed"][e]):
+            assert np.sqrt(np.mean((a - b) ** 2) / np.mean(b ** 2)) < 0.12
