@@ -224,6 +224,70 @@ def run_reference(args, cfg, ws, rank):
     print(json.dumps(line), flush=True)
 
 
+def train_flops(cfg):
+    """Algorithmic FLOPs of one training step (forward_train + backward): the
+    expert FFNs three times (Fprop, Dgrad, Wgrad), the router logits, and the
+    router backward's K-sparse products (d_gate, s, the du term, dE)."""
+    ffn = (cfg.K + cfg.N_s) * cfg.T * 6 * cfg.d * cfg.I
+    return 3 * ffn + 2 * cfg.T * cfg.d * cfg.N_r + 8 * cfg.T * cfg.K * cfg.d
+
+
+def measure_train(args, cfg, layer, u, dev, group, p, steps):
+    """Times `steps` training steps (forward_train + backward) after 3 warm-up
+    steps; the routed expert FFN backward (2 Dgrad + 2 Wgrad grouped GEMMs) is
+    timed on its own with events on the same stream."""
+    from mixture_experts_layer_60_b200.synth import upstream_grad
+    dh = upstream_grad(cfg, dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(3):
+        layer.forward_train(u)
+        layer.backward(dh)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    fb = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if group is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for i in range(steps):
+        layer.forward_train(u)
+        fb[i][0].record(stream)
+        layer.backward(dh, ffn_events=ev[i])
+        fb[i][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / steps
+    bwd_ms = sum(a.elapsed_time(b) for a, b in fb) / steps
+    ffn_ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+    if group is not None:
+        tt = torch.tensor([ms, bwd_ms, ffn_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms, bwd_ms, ffn_ms = (float(x) for x in tt)
+    ws = dist.get_world_size() if group is not None else 1
+    R = cfg.T * cfg.K
+    ffn_flops = 12.0 * R * cfg.d * cfg.I
+    fp8 = cfg.dtype == "e4m3"
+    pk = p["bf16_sustained"] * (2 if fp8 else 1)
+    ach = ffn_flops / (ffn_ms / 1e3) / 1e12
+    return {
+        "metric": "training-step tokens/s (forward keeping activations + backward)",
+        "value": cfg.T * ws / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
+        "backward_ms": bwd_ms, "steps": steps, "warmup": 3,
+        "flops_per_step": train_flops(cfg),
+        "tflops": train_flops(cfg) / (ms / 1e3) / 1e12,
+        "roofline": {"bound": "tensor", "achieved": ach, "peak": pk, "unit": "TFLOP/s",
+                     "frac": ach / pk,
+                     "kernel": "routed expert FFN backward (Dgrad down + SwiGLU backward, "
+                               "Dgrad gate/up, Wgrad down, Wgrad gate/up; tcgen05" +
+                               (", E4M3 operands" if fp8 else "") + ")",
+                     "peak_kind": "sustained bf16 of " + p["source"] +
+                                  (" x2 (FP8 nominal ratio)" if fp8 else ""),
+                     "kernel_ms": ffn_ms, "flops_per_launch": ffn_flops, "traffic": None},
+    }
+
+
 def run_ours(args, cfg, ws, rank, local):
     from mixture_experts_layer_60_b200 import moe_device_status
     from mixture_experts_layer_60_b200.layer import MoELayer
@@ -248,6 +312,18 @@ def run_ours(args, cfg, ws, rank, local):
         else:
             layer.bias_update()
         return h
+
+    if args.mode == "train":
+        tr = measure_train(args, cfg, layer, u, dev, group, p, args.steps)
+        if moe_device_status() != 0:
+            raise RuntimeError("a kernel reported a bounded-wait timeout")
+        if rank == 0:
+            print(json.dumps({**tr, "n_gpus": ws, "dtype": {"bf16": "bf16", "e4m3": "e4m3"}.get(
+                cfg.dtype, cfg.dtype), "data": "synthetic",
+                              "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d,
+                                         "N_r": cfg.N_r, "K": cfg.K, "N_s": cfg.N_s,
+                                         "I": cfg.I}}), flush=True)
+        return
 
     for _ in range(args.warmup):
         step()
@@ -323,6 +399,10 @@ def run_ours(args, cfg, ws, rank, local):
         tt = torch.tensor([e2e_ms], device=dev)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         e2e_ms = float(tt[0])
+    # ---- training step (bf16 layers): forward keeping activations + backward
+    train = None
+    if cfg.dtype in ("bf16", "e4m3") and not args.no_train:
+        train = measure_train(args, cfg, layer, u, dev, group, p, max(3, args.steps // 4))
     status = moe_device_status()
 
     # ---- CPU oracle baseline (rank 0, N = 1 only)
@@ -388,6 +468,7 @@ def run_ours(args, cfg, ws, rank, local):
         "load_balance": _load_balance(load_hist, cfg) if multi else None,
         "device_status": status,
         "cpu_baseline": cpu,
+        "train": train,
     }
     print(json.dumps(line), flush=True)
 
@@ -402,6 +483,10 @@ def main():
     ap.add_argument("--cpu-tokens", type=int, default=16)
     ap.add_argument("--ref-tokens", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-train", action="store_true",
+                    help="skip the training-step (forward + backward) measurement")
+    ap.add_argument("--mode", default="forward", choices=["forward", "train"],
+                    help="train: time only training steps and print their line")
     ap.add_argument("--tokens", type=int, default=None,
                     help="scaled-down variant: tokens per rank (default: the config's T)")
     ap.add_argument("--experts", type=int, default=None,

@@ -250,8 +250,9 @@ moe_status moe_permute_noalloc(const void* u, const float* u_scale, moe_dtype dt
  * chain rule to the forward of section 方法 / 2 of "DeepSeek-V3 技術報告".
  * The selection (top-K of s + b) is piecewise constant and is held fixed:
  * gradients reach s only through g = s_sel / sum(s_sel); b gets none.
- * Expert GEMMs run in bf16 with float32 accumulation (MOE_BF16 only);
- * d % 256 == 0 and I % 256 == 0.  Order of a training step:
+ * Expert GEMMs run in bf16 with float32 accumulation (MOE_BF16) or under the
+ * FP8 recipe (MOE_E4M3); d % 256 == 0 and I % 256 == 0.  Order of a training
+ * step:
  *   forward:  moe_route, moe_permute, moe_expert_gate_up_save (routed and
  *             shared), moe_expert_down, moe_combine
  *   backward: moe_combine_backward, moe_expert_ffn_backward (routed with
@@ -260,16 +261,18 @@ moe_status moe_permute_noalloc(const void* u, const float* u_scale, moe_dtype dt
  * ======================================================================== */
 
 /* ------------------------------------------------------------------------
- * moe_expert_gate_up_save - moe_expert_gate_up (MOE_BF16) that also keeps
- * the pre-activations the backward needs:
- *   a_gu[r, 0:I]  = W_gate[g] x[r],  a_gu[r, I:2I] = W_up[g] x[r]  (bf16)
- *   h[r]          = SiLU(a_gu[r, 0:I]) * a_gu[r, I:2I], from the float32 values
- *   x [rows, d], offsets, W_gate_up as for moe_expert_ffn; h [rows, I] and
+ * moe_expert_gate_up_save - moe_expert_gate_up (MOE_BF16 or MOE_E4M3, same
+ * arguments and outputs) that also keeps the pre-activations the backward
+ * needs, computed in float32 and stored bf16:
+ *   a_gu[r, 0:I]  = W_gate[g] x[r],  a_gu[r, I:2I] = W_up[g] x[r]
+ *   h[r]          = SiLU(gate) * up from the float32 values (bf16, or e4m3
+ *                   with h_scale for MOE_E4M3)
  *   a_gu [rows, 2I] device bf16 out, 16-byte aligned.
  * ------------------------------------------------------------------------ */
-moe_status moe_expert_gate_up_save(const void* x, const int32_t* offsets, int n_groups,
-                                   int rows, int d, int I, moe_dtype dt,
-                                   const void* W_gate_up, void* h, void* a_gu, void* stream);
+moe_status moe_expert_gate_up_save(const void* x, const float* x_scale, const int32_t* offsets,
+                                   int n_groups, int rows, int d, int I, moe_dtype dt,
+                                   const void* W_gate_up, const float* w_scale_gate_up, void* h,
+                                   float* h_scale, void* a_gu, void* stream);
 
 /* ------------------------------------------------------------------------
  * moe_combine_backward - gradient of the h'-equation through the routed
@@ -293,27 +296,61 @@ moe_status moe_combine_backward(const void* dh_out, const void* u, const void* E
                                 float* d_logit, float* d_logit_perm, void* stream);
 
 /* ------------------------------------------------------------------------
+ * moe_quantize_128x1_grouped - FP8 quantiser of a weight-gradient operand
+ * (reading of the 1x128 activation tile for a contraction over an expert's
+ * tokens): blocks of 128 consecutive rows start at every group's first row
+ * (the last block of a group may be shorter; empty groups have none), and
+ * each column of a block gets scale = amax/448 (1 if all zero);
+ * q = E4M3_rne_satfinite(x / scale) with an IEEE float32 division.
+ *   x            [rows, cols] device bf16, cols % 128 == 0
+ *   offsets      [n_groups+1] device int32 (NULL: one group of all rows)
+ *   q            [rows, cols] device e4m3 out
+ *   scale        [ceil(rows/128) + n_groups, cols] device float32 out; row
+ *                block_start[g] + i holds block i of group g
+ *   block_start  [n_groups+1] device int32 out: first block of each group,
+ *                block_start[n_groups] = number of blocks
+ * ------------------------------------------------------------------------ */
+moe_status moe_quantize_128x1_grouped(const void* x, int rows, int cols, const int32_t* offsets,
+                                      int n_groups, uint8_t* q, float* scale,
+                                      int32_t* block_start, void* stream);
+
+/* ------------------------------------------------------------------------
  * moe_expert_ffn_backward - Dgrad and Wgrad of the grouped SwiGLU FFN for
- * upstream dy (MOE_BF16).  For group g and its rows r, with a, b the gate
- * and up halves of a_gu and h = SiLU(a) * b from moe_expert_gate_up_save:
+ * upstream dy.  For group g and its rows r, with a, b the gate and up halves
+ * of a_gu and h = SiLU(a) * b from moe_expert_gate_up_save:
  *   dh  = dy W_down[g]                               (float32, not stored)
- *   dA  = [dh * b * SiLU'(a) | dh * SiLU(a)]          (bf16, in the workspace)
+ *   dA  = [dh * b * SiLU'(a) | dh * SiLU(a)]          (in the workspace)
  *   dx[r]          = dA[r] W_gate_up[g]               (Dgrad, bf16)
  *   dW_down[g]     = sum_r dy[r]^T h[r]               (Wgrad, [d, I] bf16)
  *   dW_gate_up[g]  = sum_r dA[r]^T x[r]               (Wgrad, [2I, d] bf16)
- *   x [rows, d], dy [rows, d], h [rows, I], a_gu [rows, 2I]: device bf16 in;
- *   offsets [n_groups+1] as for moe_expert_ffn; W_gate_up [n_groups, 2I, d]
- *   and W_down [n_groups, d, I] bf16; dx [rows, d], dW_gate_up and dW_down
+ * MOE_BF16: bf16 GEMMs with float32 accumulation; x [rows, d] and h
+ *   [rows, I] bf16, x_rows and the weight scales NULL.
+ * MOE_E4M3: every GEMM input E4M3 (the FP8 recipe applied to Dgrad and
+ *   Wgrad): dy and dA quantised per row and 128 columns for the two Dgrads;
+ *   for the Wgrads dy, h, dA and x quantised per column and 128 consecutive
+ *   rows of one group (blocks start at the group's first row); weights
+ *   W_gate_up / W_down e4m3 with their forward 128x128 block scales
+ *   (w_scale_gate_up [n_groups, 2I/128, d/128], w_scale_down
+ *   [n_groups, d/128, I/128]); each 128-deep partial sum promoted with its
+ *   two scales.  x is the bf16 layer input: row r is x[x_rows[r]] when
+ *   x_rows (device int32 [rows]) is given, else x[r]; h may be NULL (it is
+ *   recomputed from a_gu).
+ *   x [*, d], dy [rows, d], a_gu [rows, 2I]: device bf16 in; offsets
+ *   [n_groups+1] as for moe_expert_ffn; dx [rows, d], dW_gate_up and dW_down
  *   (same shapes as the weights) device bf16 out.  A group with no rows gets
  *   zero weight gradients.  Workspace: moe_expert_ffn_backward_workspace_size
- *   bytes, 256-byte aligned.  d % 256 == 0, I % 256 == 0.
+ *   bytes (it depends on n_groups for MOE_E4M3), 256-byte aligned.
+ *   d % 256 == 0, I % 256 == 0.
  * ------------------------------------------------------------------------ */
-size_t moe_expert_ffn_backward_workspace_size(moe_dtype dt, int rows, int I);
-moe_status moe_expert_ffn_backward(const void* x, const int32_t* offsets, int n_groups, int rows,
-                                   int d, int I, moe_dtype dt, const void* W_gate_up,
-                                   const void* W_down, const void* a_gu, const void* h,
-                                   const void* dy, void* dx, void* dW_gate_up, void* dW_down,
-                                   void* workspace, size_t workspace_bytes, void* stream);
+size_t moe_expert_ffn_backward_workspace_size(moe_dtype dt, int rows, int d, int I,
+                                              int n_groups);
+moe_status moe_expert_ffn_backward(const void* x, const int32_t* x_rows, const int32_t* offsets,
+                                   int n_groups, int rows, int d, int I, moe_dtype dt,
+                                   const void* W_gate_up, const float* w_scale_gate_up,
+                                   const void* W_down, const float* w_scale_down,
+                                   const void* a_gu, const void* h, const void* dy, void* dx,
+                                   void* dW_gate_up, void* dW_down, void* workspace,
+                                   size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
  * moe_unpermute_backward - the input gradient:
@@ -330,15 +367,17 @@ moe_status moe_unpermute_backward(const void* dh_out, const void* dx_shared, int
 
 /* ------------------------------------------------------------------------
  * moe_router_weight_grad - gradient of the expert centroids E:
- *   dE[i] = sum over grouped rows r of expert i of d_logit_perm[r] x_perm[r]
- * rows in ascending order, float32 accumulation.  x_perm [rows, d] device dt
- * (MOE_F32 or MOE_BF16), d_logit_perm [rows] float32 and offsets [N_r+1] from
- * moe_combine_backward / moe_permute; dE [N_r, d] device float32 out
- * (original precision for the gating module).  d * sizeof(dt) % 16 == 0.
+ *   dE[i] = sum over grouped rows r of expert i of d_logit_perm[r] x(r)
+ * with x(r) = x[x_rows[r]] when x_rows is given (e.g. u and perm_src from
+ * moe_permute), else x[r] (x_perm); rows in ascending order, float32
+ * accumulation.  x device dt (MOE_F32 or MOE_BF16), d_logit_perm [rows]
+ * float32 and offsets [N_r+1] from moe_combine_backward / moe_permute;
+ * dE [N_r, d] device float32 out (original precision for the gating
+ * module).  d * sizeof(dt) % 16 == 0.
  * ------------------------------------------------------------------------ */
-moe_status moe_router_weight_grad(const void* x_perm, const float* d_logit_perm,
-                                  const int32_t* offsets, moe_dtype dt, int N_r, int d, float* dE,
-                                  void* stream);
+moe_status moe_router_weight_grad(const void* x, const int32_t* x_rows,
+                                  const float* d_logit_perm, const int32_t* offsets,
+                                  moe_dtype dt, int N_r, int d, float* dE, void* stream);
 
 /* ------------------------------------------------------------------------
  * moe_device_status - synchronises the current device, then returns (and

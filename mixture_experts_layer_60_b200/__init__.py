@@ -20,6 +20,7 @@ __all__ = [
     "moe_route_workspace_size", "moe_permute_workspace_size", "moe_expert_ffn_workspace_size",
     "moe_expert_gate_up_save", "moe_combine_backward", "moe_expert_ffn_backward",
     "moe_expert_ffn_backward_workspace_size", "moe_unpermute_backward", "moe_router_weight_grad",
+    "moe_quantize_128x1_grouped",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
@@ -52,15 +53,17 @@ SYMBOLS = {
     "moe_quantize_128x128": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp]),
     "moe_device_status": (_i, [ctypes.POINTER(_i)]),
     "moe_permute_noalloc": (_i, [_vp, _vp, _i, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
-    "moe_expert_gate_up_save": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
+    "moe_expert_gate_up_save": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp,
+                                     _vp]),
     "moe_combine_backward": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp,
                                   _vp, _vp]),
-    "moe_expert_ffn_backward_workspace_size": (_sz, [_i, _i, _i]),
-    "moe_expert_ffn_backward": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp,
-                                     _vp, _vp, _vp, _sz, _vp]),
+    "moe_expert_ffn_backward_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
+    "moe_expert_ffn_backward": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp,
+                                     _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_unpermute_backward": (_i, [_vp, _vp, _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp,
                                     _vp]),
-    "moe_router_weight_grad": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp, _vp]),
+    "moe_router_weight_grad": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp]),
+    "moe_quantize_128x1_grouped": (_i, [_vp, _i, _i, _vp, _i, _vp, _vp, _vp, _vp]),
 }
 
 
@@ -233,15 +236,18 @@ def moe_device_status() -> int:
 
 # ------------------------------------------------------------------ backward
 
-def moe_expert_ffn_backward_workspace_size(dt: int, rows: int, I: int) -> int:
-    return lib().moe_expert_ffn_backward_workspace_size(dt, rows, I)
+def moe_expert_ffn_backward_workspace_size(dt: int, rows: int, d: int, I: int,
+                                           n_groups: int) -> int:
+    return lib().moe_expert_ffn_backward_workspace_size(dt, rows, d, I, n_groups)
 
 
-def moe_expert_gate_up_save(x, offsets, W_gate_up, h, a_gu, stream=None):
+def moe_expert_gate_up_save(x, offsets, W_gate_up, h, a_gu, x_scale=None, w_scale_gate_up=None,
+                            h_scale=None, stream=None):
     rows, d = x.shape
     n_groups, two_i, _ = W_gate_up.shape
-    _check(lib().moe_expert_gate_up_save(_p(x), _p(offsets), n_groups, rows, d, two_i // 2,
-                                         _dt(x), _p(W_gate_up), _p(h), _p(a_gu), _s(stream)))
+    _check(lib().moe_expert_gate_up_save(_p(x), _p(x_scale), _p(offsets), n_groups, rows, d,
+                                         two_i // 2, _dt(x), _p(W_gate_up), _p(w_scale_gate_up),
+                                         _p(h), _p(h_scale), _p(a_gu), _s(stream)))
 
 
 def moe_combine_backward(dh_out, u, E, y_perm, inv_row, topk_idx, topk_gate, dy_perm, d_gate,
@@ -254,13 +260,18 @@ def moe_combine_backward(dh_out, u, E, y_perm, inv_row, topk_idx, topk_gate, dy_
 
 
 def moe_expert_ffn_backward(x, offsets, W_gate_up, W_down, a_gu, h, dy, dx, dW_gate_up, dW_down,
-                            workspace, stream=None):
-    rows, d = x.shape
+                            workspace, x_rows=None, w_scale_gate_up=None, w_scale_down=None,
+                            stream=None):
+    """dt follows the weights: bf16 weights -> MOE_BF16, e4m3 weights (uint8
+    with their 128x128 scales) -> MOE_E4M3.  x is bf16 in both cases."""
+    rows, d = dy.shape
     n_groups, two_i, _ = W_gate_up.shape
-    _check(lib().moe_expert_ffn_backward(_p(x), _p(offsets), n_groups, rows, d, two_i // 2,
-                                         _dt(x), _p(W_gate_up), _p(W_down), _p(a_gu), _p(h),
-                                         _p(dy), _p(dx), _p(dW_gate_up), _p(dW_down),
-                                         _p(workspace), _nbytes(workspace), _s(stream)))
+    _check(lib().moe_expert_ffn_backward(_p(x), _p(x_rows), _p(offsets), n_groups, rows, d,
+                                         two_i // 2, _dt(W_gate_up), _p(W_gate_up),
+                                         _p(w_scale_gate_up), _p(W_down), _p(w_scale_down),
+                                         _p(a_gu), _p(h), _p(dy), _p(dx), _p(dW_gate_up),
+                                         _p(dW_down), _p(workspace), _nbytes(workspace),
+                                         _s(stream)))
 
 
 def moe_unpermute_backward(dh_out, dx_shared, dx_perm, inv_row, topk_idx, d_logit, E, du,
@@ -272,7 +283,14 @@ def moe_unpermute_backward(dh_out, dx_shared, dx_perm, inv_row, topk_idx, d_logi
                                         inv_row.shape[1], _p(du), _s(stream)))
 
 
-def moe_router_weight_grad(x_perm, d_logit_perm, offsets, dE, stream=None):
+def moe_router_weight_grad(x, d_logit_perm, offsets, dE, x_rows=None, stream=None):
     N_r, d = dE.shape
-    _check(lib().moe_router_weight_grad(_p(x_perm), _p(d_logit_perm), _p(offsets), _dt(x_perm),
+    _check(lib().moe_router_weight_grad(_p(x), _p(x_rows), _p(d_logit_perm), _p(offsets), _dt(x),
                                         N_r, d, _p(dE), _s(stream)))
+
+
+def moe_quantize_128x1_grouped(x, offsets, q, scale, block_start, stream=None):
+    rows, cols = x.shape
+    n_groups = 1 if offsets is None else offsets.shape[0] - 1
+    _check(lib().moe_quantize_128x1_grouped(_p(x), rows, cols, _p(offsets), n_groups, _p(q),
+                                            _p(scale), _p(block_start), _s(stream)))

@@ -382,9 +382,40 @@ namespace {
 
 inline bool al16(const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0; }
 
-size_t ffn_bwd_ws(moe_dtype dt, int rows, int I) {
-  if (dt != MOE_BF16 || rows <= 0 || I <= 0) return 0;
-  return align_up((size_t)rows * 2 * I * 2, 256);
+// Backward workspace.  bf16: dA [rows, 2I] bf16.  e4m3: the FP8 operands of
+// the two Dgrads and two Wgrads and their scales (see fp8_bwd_layout).
+struct Fp8BwdLayout {
+  size_t dy_q, dy_s, dA_q, dA_s, dA_bf, blk, dyT_q, dyT_s, hT_q, hT_s, dAT_q, dAT_s, xT_q, xT_s,
+      total;
+};
+Fp8BwdLayout fp8_bwd_layout(int rows, int d, int I, int G) {
+  Fp8BwdLayout L;
+  const size_t R = (size_t)rows, nb = (size_t)(rows + 127) / 128 + G;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { const size_t at = o; o = align_up(o + bytes, 256); return at; };
+  L.dy_q = take(R * d);
+  L.dy_s = take(R * (d / 128) * 4);
+  L.dA_q = take(R * 2 * I);
+  L.dA_s = take(R * (2 * I / 128) * 4);
+  L.dA_bf = take(R * 2 * I * 2);
+  L.blk = take((size_t)(G + 1) * 4);
+  L.dyT_q = take(R * d);
+  L.dyT_s = take(nb * d * 4);
+  L.hT_q = take(R * I);
+  L.hT_s = take(nb * I * 4);
+  L.dAT_q = take(R * 2 * I);
+  L.dAT_s = take(nb * 2 * I * 4);
+  L.xT_q = take(R * d);
+  L.xT_s = take(nb * d * 4);
+  L.total = o;
+  return L;
+}
+
+size_t ffn_bwd_ws(moe_dtype dt, int rows, int d, int I, int G) {
+  if (rows <= 0 || I <= 0 || d <= 0 || G <= 0) return 0;
+  if (dt == MOE_BF16) return align_up((size_t)rows * 2 * I * 2, 256);
+  if (dt == MOE_E4M3) return fp8_bwd_layout(rows, d, I, G).total;
+  return 0;
 }
 
 moe_status check_rowwise(const char* who, moe_dtype dt, int T, int d, int K) {
@@ -400,18 +431,27 @@ moe_status check_rowwise(const char* who, moe_dtype dt, int T, int d, int K) {
 
 }  // namespace
 
-moe_status moe_expert_gate_up_save(const void* x, const int32_t* offsets, int n_groups, int rows,
-                                   int d, int I, moe_dtype dt, const void* W_gate_up, void* h,
-                                   void* a_gu, void* stream) {
+moe_status moe_expert_gate_up_save(const void* x, const float* x_scale, const int32_t* offsets,
+                                   int n_groups, int rows, int d, int I, moe_dtype dt,
+                                   const void* W_gate_up, const float* w_scale_gate_up, void* h,
+                                   float* h_scale, void* a_gu, void* stream) {
   clear_last_error();
-  MOE_TRY(check_ffn_common("moe_expert_gate_up_save", x, offsets, n_groups, rows, d, I, dt,
-                           W_gate_up));
-  MOE_REQUIRE(dt == MOE_BF16, MOE_ERR_UNSUPPORTED, "moe_expert_gate_up_save: MOE_BF16 only");
+  const char* who = "moe_expert_gate_up_save";
+  MOE_TRY(check_ffn_common(who, x, offsets, n_groups, rows, d, I, dt, W_gate_up));
+  MOE_REQUIRE(dt == MOE_BF16 || dt == MOE_E4M3, MOE_ERR_UNSUPPORTED,
+              "%s: MOE_BF16 or MOE_E4M3 only", who);
   if (rows == 0) return MOE_OK;
-  MOE_REQUIRE(h && a_gu, MOE_ERR_INVALID_ARG, "moe_expert_gate_up_save: null pointer");
+  MOE_REQUIRE(h && a_gu, MOE_ERR_INVALID_ARG, "%s: null pointer", who);
+  MOE_TRY(check_scales(who, dt, x_scale, w_scale_gate_up));
+  MOE_REQUIRE((dt == MOE_E4M3) == (h_scale != nullptr), MOE_ERR_INVALID_ARG,
+              "%s: h_scale is required for MOE_E4M3 and only for it", who);
   MOE_REQUIRE(al16(h) && al16(a_gu) && al16(x), MOE_ERR_INVALID_ARG,
-              "moe_expert_gate_up_save: x, h and a_gu must be 16-byte aligned");
+              "%s: x, h and a_gu must be 16-byte aligned", who);
   MOE_TRY(check_device());
+  if (dt == MOE_E4M3)
+    return launch_fp8_gemm_ex(x, x_scale, W_gate_up, w_scale_gate_up, 2 * I, offsets, n_groups,
+                              rows, I, d, F8_SWIGLU_SAVE, false, h, h_scale, a_gu, 2 * I, nullptr,
+                              as_stream(stream));
   return launch_ws_gemm_ex(x, W_gate_up, 2 * I, offsets, n_groups, rows, I, d, WS_SWIGLU_SAVE,
                            false, h, I, a_gu, 2 * I, as_stream(stream));
 }
@@ -434,24 +474,51 @@ moe_status moe_combine_backward(const void* dh_out, const void* u, const void* E
                                  dy_perm, d_gate, d_logit, d_logit_perm, as_stream(stream));
 }
 
-size_t moe_expert_ffn_backward_workspace_size(moe_dtype dt, int rows, int I) {
-  return ffn_bwd_ws(dt, rows, I);
+moe_status moe_quantize_128x1_grouped(const void* x, int rows, int cols, const int32_t* offsets,
+                                      int n_groups, uint8_t* q, float* scale,
+                                      int32_t* block_start, void* stream) {
+  clear_last_error();
+  MOE_REQUIRE(rows >= 0 && cols > 0 && cols % 128 == 0, MOE_ERR_UNSUPPORTED,
+              "moe_quantize_128x1_grouped: cols=%d must be a positive multiple of 128", cols);
+  MOE_REQUIRE(n_groups > 0 && n_groups <= 1 << 20, MOE_ERR_INVALID_ARG,
+              "moe_quantize_128x1_grouped: n_groups=%d", n_groups);
+  MOE_REQUIRE(block_start, MOE_ERR_INVALID_ARG, "moe_quantize_128x1_grouped: null block_start");
+  MOE_REQUIRE(rows == 0 || (x && q && scale), MOE_ERR_INVALID_ARG,
+              "moe_quantize_128x1_grouped: null pointer");
+  MOE_REQUIRE(al16(x) && al16(q) && al16(scale), MOE_ERR_INVALID_ARG,
+              "moe_quantize_128x1_grouped: x, q and scale must be 16-byte aligned");
+  MOE_TRY(check_device());
+  cudaStream_t s = as_stream(stream);
+  MOE_TRY(launch_block_table(offsets, offsets ? n_groups : 1, rows, block_start, s));
+  return launch_quant_128x1(x, cols, nullptr, false, rows, cols, offsets, n_groups, block_start, q,
+                            scale, s);
 }
 
-moe_status moe_expert_ffn_backward(const void* x, const int32_t* offsets, int n_groups, int rows,
-                                   int d, int I, moe_dtype dt, const void* W_gate_up,
-                                   const void* W_down, const void* a_gu, const void* h,
-                                   const void* dy, void* dx, void* dW_gate_up, void* dW_down,
-                                   void* workspace, size_t workspace_bytes, void* stream) {
+size_t moe_expert_ffn_backward_workspace_size(moe_dtype dt, int rows, int d, int I,
+                                              int n_groups) {
+  return ffn_bwd_ws(dt, rows, d, I, n_groups);
+}
+
+moe_status moe_expert_ffn_backward(const void* x, const int32_t* x_rows, const int32_t* offsets,
+                                   int n_groups, int rows, int d, int I, moe_dtype dt,
+                                   const void* W_gate_up, const float* w_scale_gate_up,
+                                   const void* W_down, const float* w_scale_down,
+                                   const void* a_gu, const void* h, const void* dy, void* dx,
+                                   void* dW_gate_up, void* dW_down, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
   clear_last_error();
   const char* who = "moe_expert_ffn_backward";
   MOE_TRY(check_ffn_common(who, x, offsets, n_groups, rows, d, I, dt, W_gate_up));
-  MOE_REQUIRE(dt == MOE_BF16, MOE_ERR_UNSUPPORTED, "%s: MOE_BF16 only", who);
+  MOE_REQUIRE(dt == MOE_BF16 || dt == MOE_E4M3, MOE_ERR_UNSUPPORTED,
+              "%s: MOE_BF16 or MOE_E4M3 only", who);
   MOE_REQUIRE(d % 256 == 0 && I % 256 == 0, MOE_ERR_UNSUPPORTED,
               "%s: d=%d and I=%d must be multiples of 256", who, d, I);
   MOE_REQUIRE(W_down && dW_gate_up && dW_down, MOE_ERR_INVALID_ARG, "%s: null pointer", who);
   MOE_REQUIRE(al16(dW_gate_up) && al16(dW_down), MOE_ERR_INVALID_ARG,
               "%s: weight gradients must be 16-byte aligned", who);
+  MOE_TRY(check_scales(who, dt, w_scale_gate_up, w_scale_down));
+  MOE_REQUIRE(dt == MOE_E4M3 || !x_rows, MOE_ERR_INVALID_ARG,
+              "%s: x_rows is only for MOE_E4M3", who);
   cudaStream_t s = as_stream(stream);
   if (rows == 0) {
     MOE_TRY(check_device());
@@ -460,25 +527,59 @@ moe_status moe_expert_ffn_backward(const void* x, const int32_t* offsets, int n_
     return cuda_check(cudaMemsetAsync(dW_down, 0, (size_t)n_groups * d * I * 2, s),
                       "zero dW_down");
   }
-  MOE_REQUIRE(a_gu && h && dy && dx && workspace, MOE_ERR_INVALID_ARG, "%s: null pointer", who);
+  MOE_REQUIRE(a_gu && dy && dx && workspace && (dt == MOE_E4M3 || h), MOE_ERR_INVALID_ARG,
+              "%s: null pointer", who);
   MOE_REQUIRE(al16(x) && al16(a_gu) && al16(h) && al16(dy) && al16(dx), MOE_ERR_INVALID_ARG,
               "%s: activations must be 16-byte aligned", who);
   MOE_REQUIRE(reinterpret_cast<uintptr_t>(workspace) % 256 == 0, MOE_ERR_INVALID_ARG,
               "%s: workspace must be 256-byte aligned", who);
-  MOE_REQUIRE(workspace_bytes >= ffn_bwd_ws(dt, rows, I), MOE_ERR_WORKSPACE,
-              "%s: workspace %zu < %zu bytes", who, workspace_bytes, ffn_bwd_ws(dt, rows, I));
+  const size_t need = ffn_bwd_ws(dt, rows, d, I, n_groups);
+  MOE_REQUIRE(workspace_bytes >= need, MOE_ERR_WORKSPACE, "%s: workspace %zu < %zu bytes", who,
+              workspace_bytes, need);
   MOE_TRY(check_device());
-  void* dA = workspace;
-  // Wgrad of the down projection needs only dy and h
-  MOE_TRY(launch_wgrad_gemm(dy, d, h, I, offsets, n_groups, rows, dW_down, s));
-  // Dgrad of the down projection fused with the SwiGLU backward -> dA
-  MOE_TRY(launch_ws_gemm_ex(dy, W_down, 0, offsets, n_groups, rows, I, d, WS_DSWIGLU, true, dA,
-                            2 * I, const_cast<void*>(a_gu), 2 * I, s));
+  if (dt == MOE_BF16) {
+    void* dA = workspace;
+    // Wgrad of the down projection needs only dy and h
+    MOE_TRY(launch_wgrad_gemm(dy, d, h, I, offsets, n_groups, rows, dW_down, s));
+    // Dgrad of the down projection fused with the SwiGLU backward -> dA
+    MOE_TRY(launch_ws_gemm_ex(dy, W_down, 0, offsets, n_groups, rows, I, d, WS_DSWIGLU, true, dA,
+                              2 * I, const_cast<void*>(a_gu), 2 * I, s));
+    // Dgrad of the gate/up projection
+    MOE_TRY(launch_ws_gemm_ex(dA, W_gate_up, 0, offsets, n_groups, rows, d, 2 * I, WS_STORE, true,
+                              dx, d, nullptr, 0, s));
+    // Wgrad of the gate/up projection
+    return launch_wgrad_gemm(dA, 2 * I, x, d, offsets, n_groups, rows, dW_gate_up, s);
+  }
+  // ---- FP8 (E4M3) backward
+  const Fp8BwdLayout L = fp8_bwd_layout(rows, d, I, n_groups);
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  auto f32 = [&](size_t off) { return reinterpret_cast<float*>(w + off); };
+  int32_t* blk = reinterpret_cast<int32_t*>(w + L.blk);
+  const int G = offsets ? n_groups : 1;
+  // Dgrad of the down projection (dy quantised 1x128) fused with the SwiGLU
+  // backward: dA as bf16 and as E4M3 1x128
+  MOE_TRY(launch_quant_1x128(dy, rows, d, w + L.dy_q, f32(L.dy_s), s));
+  MOE_TRY(launch_fp8_gemm_ex(w + L.dy_q, f32(L.dy_s), W_down, w_scale_down, 0, offsets, n_groups,
+                             rows, I, d, F8_DSWIGLU, true, w + L.dA_q, f32(L.dA_s),
+                             const_cast<void*>(a_gu), 2 * I, w + L.dA_bf, s));
   // Dgrad of the gate/up projection
-  MOE_TRY(launch_ws_gemm_ex(dA, W_gate_up, 0, offsets, n_groups, rows, d, 2 * I, WS_STORE, true,
-                            dx, d, nullptr, 0, s));
-  // Wgrad of the gate/up projection
-  return launch_wgrad_gemm(dA, 2 * I, x, d, offsets, n_groups, rows, dW_gate_up, s);
+  MOE_TRY(launch_fp8_gemm_ex(w + L.dA_q, f32(L.dA_s), W_gate_up, w_scale_gate_up, 0, offsets,
+                             n_groups, rows, d, 2 * I, F8_STORE, true, dx, nullptr, nullptr, 0,
+                             nullptr, s));
+  // Wgrad operands: 128-row blocks of each group, one scale per column
+  MOE_TRY(launch_block_table(offsets, G, rows, blk, s));
+  MOE_TRY(launch_quant_128x1(dy, d, nullptr, false, rows, d, offsets, n_groups, blk, w + L.dyT_q,
+                             f32(L.dyT_s), s));
+  MOE_TRY(launch_quant_128x1(a_gu, 2 * I, nullptr, true, rows, I, offsets, n_groups, blk,
+                             w + L.hT_q, f32(L.hT_s), s));
+  MOE_TRY(launch_wgrad_fp8(w + L.dyT_q, f32(L.dyT_s), d, w + L.hT_q, f32(L.hT_s), I, offsets,
+                           n_groups, rows, blk, dW_down, s));
+  MOE_TRY(launch_quant_128x1(w + L.dA_bf, 2 * I, nullptr, false, rows, 2 * I, offsets, n_groups,
+                             blk, w + L.dAT_q, f32(L.dAT_s), s));
+  MOE_TRY(launch_quant_128x1(x, d, x_rows, false, rows, d, offsets, n_groups, blk, w + L.xT_q,
+                             f32(L.xT_s), s));
+  return launch_wgrad_fp8(w + L.dAT_q, f32(L.dAT_s), 2 * I, w + L.xT_q, f32(L.xT_s), d, offsets,
+                          n_groups, rows, blk, dW_gate_up, s);
 }
 
 moe_status moe_unpermute_backward(const void* dh_out, const void* dx_shared, int N_s,
@@ -499,9 +600,9 @@ moe_status moe_unpermute_backward(const void* dh_out, const void* dx_shared, int
                                    dt, T, d, K, du, as_stream(stream));
 }
 
-moe_status moe_router_weight_grad(const void* x_perm, const float* d_logit_perm,
-                                  const int32_t* offsets, moe_dtype dt, int N_r, int d, float* dE,
-                                  void* stream) {
+moe_status moe_router_weight_grad(const void* x_perm, const int32_t* x_rows,
+                                  const float* d_logit_perm, const int32_t* offsets,
+                                  moe_dtype dt, int N_r, int d, float* dE, void* stream) {
   clear_last_error();
   MOE_REQUIRE(dt == MOE_F32 || dt == MOE_BF16, MOE_ERR_UNSUPPORTED,
               "moe_router_weight_grad: dtype must be MOE_F32 or MOE_BF16");
@@ -513,7 +614,7 @@ moe_status moe_router_weight_grad(const void* x_perm, const float* d_logit_perm,
   MOE_REQUIRE(al16(x_perm) && al16(dE), MOE_ERR_INVALID_ARG,
               "moe_router_weight_grad: x_perm and dE must be 16-byte aligned");
   MOE_TRY(check_device());
-  return launch_router_weight_grad(x_perm, d_logit_perm, offsets, dt, N_r, d, dE,
+  return launch_router_weight_grad(x_perm, x_rows, d_logit_perm, offsets, dt, N_r, d, dE,
                                    as_stream(stream));
 }
 

@@ -9,7 +9,7 @@
 //   ds_{t,k}        = (dg_{t,k} - sum_j g_{t,j} dg_{t,j}) / sum_j s_{t,j}
 //   dlogit_{t,k}    = ds_{t,k} s_{t,k} (1 - s_{t,k}),   s = Sigmoid(u_t . e_idx)
 //   du_t = dh'_t + sum_j dxs_j[t] + sum_k dx_perm[r(t,k)] + sum_k dlogit_{t,k} e_idx(t,k)
-//   dE_i = sum over rows r of expert i of dlogit_perm[r] x_perm[r]
+//   dE_i = sum over rows r of expert i of dlogit_perm[r] x(r)   (x_perm, or u gathered)
 #include "launch.h"
 
 namespace moe {
@@ -150,8 +150,9 @@ __global__ void __launch_bounds__(256) unpermute_backward_kernel(
 // each thread owns one vector and walks the expert's rows in order.
 template <typename E>
 __global__ void __launch_bounds__(128) router_weight_grad_kernel(
-    const uint4* __restrict__ xp, const float* __restrict__ dlp,
-    const int32_t* __restrict__ offsets, int nvec, float* __restrict__ dE) {
+    const uint4* __restrict__ xp, const int32_t* __restrict__ x_rows,
+    const float* __restrict__ dlp, const int32_t* __restrict__ offsets, int nvec,
+    float* __restrict__ dE) {
   constexpr int N = Vec<E>::N;
   const int e = blockIdx.x;
   const int c = blockIdx.y * blockDim.x + threadIdx.x;
@@ -162,7 +163,8 @@ __global__ void __launch_bounds__(128) router_weight_grad_kernel(
   for (int i = 0; i < N; ++i) acc[i] = 0.f;
   for (int r = r0; r < r1; ++r) {
     const float w = dlp[r];
-    Vec<E>::load(xp[(size_t)r * nvec + c], tmp);
+    const size_t row = x_rows ? (size_t)x_rows[r] : (size_t)r;
+    Vec<E>::load(xp[row * nvec + c], tmp);
 #pragma unroll
     for (int i = 0; i < N; ++i) acc[i] = fmaf(w, tmp[i], acc[i]);
   }
@@ -239,18 +241,18 @@ moe_status launch_unpermute_backward(const void* dh, const void* dx_shared, int 
                                                d_logit, E, T, d, K, du, s);
 }
 
-moe_status launch_router_weight_grad(const void* x_perm, const float* d_logit_perm,
-                                     const int32_t* offsets, moe_dtype dt, int N_r, int d,
-                                     float* dE, cudaStream_t s) {
+moe_status launch_router_weight_grad(const void* x_perm, const int32_t* x_rows,
+                                     const float* d_logit_perm, const int32_t* offsets,
+                                     moe_dtype dt, int N_r, int d, float* dE, cudaStream_t s) {
   const int per = dt == MOE_F32 ? 4 : 8;
   const int nvec = d / per;
   dim3 grid(N_r, (nvec + 127) / 128), block(128);
   if (dt == MOE_F32)
     router_weight_grad_kernel<float><<<grid, block, 0, s>>>(
-        static_cast<const uint4*>(x_perm), d_logit_perm, offsets, nvec, dE);
+        static_cast<const uint4*>(x_perm), x_rows, d_logit_perm, offsets, nvec, dE);
   else
     router_weight_grad_kernel<__nv_bfloat16><<<grid, block, 0, s>>>(
-        static_cast<const uint4*>(x_perm), d_logit_perm, offsets, nvec, dE);
+        static_cast<const uint4*>(x_perm), x_rows, d_logit_perm, offsets, nvec, dE);
   return cuda_check(cudaGetLastError(), "router_weight_grad launch");
 }
 

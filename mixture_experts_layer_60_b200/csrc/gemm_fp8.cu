@@ -16,6 +16,16 @@
 //            with scale amax/448 (the 128 columns of a row span the four
 //            warpgroups: their amax meet in shared memory)
 //   STORE    y = bf16(acc)
+//   SWIGLU_SAVE  SWIGLU that also writes the float32 gate and up values as
+//            bf16 pre-activations S [rows, 2I] for the backward
+//   DSWIGLU  the Dgrad of the down projection fused with the SwiGLU backward:
+//            dh = acc; a, b = S[:, 0:I], S[:, I:2I] (bf16);
+//            dA = [dh * b * SiLU'(a) | dh * SiLU(a)] written as bf16 (C2) and
+//            quantised 1x128 to E4M3 (C, c_scale); a 128-column tile spans two
+//            warpgroups, whose amax meet in shared memory
+// B_MN: the weight is stored [K rows][N cols] (a Dgrad reads W_down [d, I]
+// and W_gate_up [2I, d] as they are); its 128x128 block scales are then
+// indexed [K/128][N/128], and the MMA reads B as an MN-major operand.
 // Warp roles: 0 TMA producer, 1 TMEM allocator + MMA issuer, 2-17 epilogue
 // (warpgroup w = warps 2+4w .. 5+4w).  Waits are bounded.
 #include <math.h>
@@ -28,6 +38,9 @@ namespace moe {
 moe_status make_tmap_2d(CUtensorMap* tm, const void* base, CUtensorMapDataType dtype,
                         int elem_bytes, uint64_t inner, uint64_t outer, uint32_t box_inner,
                         uint32_t box_outer);
+moe_status make_tmap_col_blocks(CUtensorMap* tm, const void* base, CUtensorMapDataType dtype,
+                                int elem_bytes, uint64_t cols, uint64_t rows, uint32_t bc,
+                                uint32_t box_rows, uint32_t box_blocks);
 
 namespace {
 
@@ -50,8 +63,8 @@ constexpr int OFF_B = STAGES * A_BYTES;
 constexpr int OFF_BAR = OFF_B + STAGES * B_BYTES;
 constexpr int N_BARS = 2 * STAGES + 7;
 constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
-constexpr int OFF_AMAX = OFF_MISC + 16;                 // [2 slots][kEpiWG][BM] float
-constexpr int OFF_TAB = OFF_AMAX + 2 * kEpiWG * BM * 4;
+constexpr int OFF_AMAX = OFF_MISC + 16;                 // [2 slots][2][kEpiWG][BM] float
+constexpr int OFF_TAB = OFF_AMAX + 2 * 2 * kEpiWG * BM * 4;
 constexpr int SMEM_BYTES = OFF_TAB + 2 * (kMaxGroups + 1) * 4;
 constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
 
@@ -64,10 +77,19 @@ struct Fp8Params {
   int b_rows_per_group;
   int half_b;           // SWIGLU: I
   const float* a_scale; // [rows, K/128]
-  const float* b_scale; // [G, b_rows/128, K/128]
-  void* C;              // SWIGLU: e4m3 [rows, N]; STORE: bf16 [rows, N]
-  float* c_scale;       // SWIGLU: [rows, N/128]
+  const float* b_scale; // [G, b_rows/128, K/128] (B_MN: [G, K/128, N/128])
+  void* C;              // SWIGLU: e4m3 [rows, N]; STORE: bf16 [rows, N]; DSWIGLU: e4m3 [rows, 2N]
+  float* c_scale;       // SWIGLU: [rows, N/128]; DSWIGLU: [rows, 2N/128]
+  __nv_bfloat16* S;     // SWIGLU_SAVE: pre-activations out; DSWIGLU: in ([rows, lds])
+  int lds;
+  __nv_bfloat16* C2;    // DSWIGLU: bf16 dA [rows, 2N]
   int* err;
+};
+
+template <int EPI>
+struct Fp8Tile {
+  static constexpr bool SW = EPI == F8_SWIGLU || EPI == F8_SWIGLU_SAVE;
+  static constexpr int BN_OUT = SW ? BN / 2 : BN;
 };
 
 __device__ __forceinline__ void decode_tile(int t, const int* prefix, const int* roff, int G,
@@ -117,11 +139,14 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
          ((uint32_t)__nv_cvt_float_to_fp8(d, __NV_SATFINITE, __NV_E4M3) << 24);
 }
 
-template <bool SWIGLU>
+__device__ __forceinline__ float silu_fast(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
+
+template <int EPI, bool B_MN>
 __global__ void __launch_bounds__(kThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmB, const Fp8Params p) {
-  constexpr int BN_OUT = SWIGLU ? BN / 2 : BN;
+  constexpr bool SWIGLU = Fp8Tile<EPI>::SW;
+  constexpr int BN_OUT = Fp8Tile<EPI>::BN_OUT;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -213,7 +238,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
           tma_load_2d(sA + stage * A_BYTES, &tmA, kb * BK, row0, &full[stage]);
-          if (SWIGLU) {
+          if (B_MN) {
+            // [128 K rows][128 N cols] x 2 tiles of columns nt*256 .. in one 3D box
+            tma_load_3d(sB + stage * B_BYTES, &tmB, 0, g * p.K + kb * BK, nt * (BN / 128),
+                        &full[stage]);
+          } else if (SWIGLU) {
             tma_load_2d(sB + stage * B_BYTES, &tmB, kb * BK, brow, &full[stage]);
             tma_load_2d(sB + stage * B_BYTES + B_BYTES / 2, &tmB, kb * BK, brow + p.half_b,
                         &full[stage]);
@@ -228,7 +257,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_e4m3_f32(BM, BN);
+      constexpr uint32_t idesc = idesc_e4m3_f32(BM, BN) | (B_MN ? (1u << 16) : 0u);
       int stage = 0, pb = 0;
       uint32_t phase = 0, pphase = 0;
       bool ok = true;
@@ -246,7 +275,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t d_tmem = tmem_base + pb * BN;
 #pragma unroll
           for (int k = 0; k < BK / 32; ++k)
-            mma_f8_ss(d_tmem, smem_desc_k_sw128(a0 + k * 32), smem_desc_k_sw128(b0 + k * 32),
+            mma_f8_ss(d_tmem, smem_desc_k_sw128(a0 + k * 32),
+                      B_MN ? smem_desc_mn_sw128(b0 + k * 4096, B_BYTES / 2)
+                           : smem_desc_k_sw128(b0 + k * 32),
                       idesc, k != 0);
           mma_commit(&empty[stage]);
           mma_commit(&pfull[pb]);
@@ -277,7 +308,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool valid = rit < mv;
       const int arow = valid ? row0 + rit : row0;   // clamp scale reads for padding rows
       const float* sa_row = p.a_scale + (size_t)arow * nkb_a;
-      const int nbw = p.b_rows_per_group / 128;     // weight row blocks per group
+      // weight N blocks per group; block scales [nbw][K/128], or [K/128][nbw] for B_MN
+      const int nbw = B_MN ? p.N / 128 : p.b_rows_per_group / 128;
       const float* sw_g = p.b_scale + (size_t)g * nbw * nkb_a;
       // weight row blocks of this thread's two 32-column chunks
       int blk0, blk1;
@@ -298,8 +330,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       float sa = sa_row[0];
       for (int kb = 0; kb < nk; ++kb) {
         const float sa_next = (kb + 1 < nk) ? sa_row[kb + 1] : 0.f;
-        const float s0 = sa * sw_g[(size_t)blk0 * nkb_a + kb];
-        const float s1 = sa * sw_g[(size_t)blk1 * nkb_a + kb];
+        const float s0 = sa * (B_MN ? sw_g[(size_t)kb * nbw + blk0] : sw_g[(size_t)blk0 * nkb_a + kb]);
+        const float s1 = sa * (B_MN ? sw_g[(size_t)kb * nbw + blk1] : sw_g[(size_t)blk1 * nkb_a + kb]);
         const bool got = mbar_wait_bounded(&pfull[pb], pphase, abort_flag, kWaitNs);
         if (!__all_sync(0xffffffffu, got)) {
           raise_abort(abort_flag, p.err);
@@ -329,7 +361,108 @@ __global__ void __launch_bounds__(kThreads, 1)
       float acc[CW];
 #pragma unroll
       for (int i = 0; i < CW / 2; ++i) f2_unpack(acc2[i], acc[2 * i], acc[2 * i + 1]);
-      if (SWIGLU) {
+      if (EPI == F8_SWIGLU_SAVE && valid) {
+        // gate / up pre-activations (float32 values rounded to bf16) for the backward
+        __nv_bfloat16* sg = p.S + (size_t)(row0 + rit) * p.lds + nt * 128 + wg * 32;
+        __nv_bfloat16* su = sg + p.half_b;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint32_t wg4[4], wu4[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            __nv_bfloat162 a2 = __floats2bfloat162_rn(acc[q4 * 8 + 2 * i], acc[q4 * 8 + 2 * i + 1]);
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[32 + q4 * 8 + 2 * i], acc[32 + q4 * 8 + 2 * i + 1]);
+            wg4[i] = *reinterpret_cast<uint32_t*>(&a2);
+            wu4[i] = *reinterpret_cast<uint32_t*>(&b2);
+          }
+          reinterpret_cast<uint4*>(sg)[q4] = make_uint4(wg4[0], wg4[1], wg4[2], wg4[3]);
+          reinterpret_cast<uint4*>(su)[q4] = make_uint4(wu4[0], wu4[1], wu4[2], wu4[3]);
+        }
+      }
+      if (EPI == F8_DSWIGLU) {
+        // acc = dh for columns c0 .. c0+63 of this row; a, b from the saved pre-activations
+        const int I = p.N;
+        const int c0 = nt * BN + wg * CW;
+        const size_t row = (size_t)(valid ? row0 + rit : row0);
+        const __nv_bfloat16* sa_p = p.S + row * p.lds + c0;
+        const __nv_bfloat16* sb_p = sa_p + I;
+        float ma = 0.f, mb = 0.f;
+        // pass 1: dA in bf16, and the amax of this thread's 64 da and 64 db values
+#pragma unroll
+        for (int j8 = 0; j8 < CW / 8; ++j8) {
+          float fa[8], fb[8], da[8], db[8];
+          if (valid) {
+            const uint4 av = reinterpret_cast<const uint4*>(sa_p)[j8];
+            const uint4 bv = reinterpret_cast<const uint4*>(sb_p)[j8];
+            Vec<__nv_bfloat16>::load(av, fa);
+            Vec<__nv_bfloat16>::load(bv, fb);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float dhv = acc[j8 * 8 + i];
+              const float sg = __fdividef(1.0f, 1.0f + __expf(-fa[i]));
+              da[i] = dhv * fb[i] * (sg * (1.0f + fa[i] * (1.0f - sg)));
+              db[i] = dhv * fa[i] * sg;
+              ma = fmaxf(ma, fabsf(da[i]));
+              mb = fmaxf(mb, fabsf(db[i]));
+            }
+            reinterpret_cast<uint4*>(p.C2 + row * (2 * I) + c0)[j8] = Vec<__nv_bfloat16>::store(da);
+            reinterpret_cast<uint4*>(p.C2 + row * (2 * I) + I + c0)[j8] = Vec<__nv_bfloat16>::store(db);
+          }
+        }
+        // a 128-column tile of da (and of db) spans warpgroups wg and wg ^ 1
+        const int sl = it & 1;
+        float* slot = amax_x + sl * 2 * kEpiWG * BM;
+        slot[wg * BM + rit] = ma;
+        slot[(kEpiWG + wg) * BM + rit] = mb;
+        mbar_arrive(&xbar[sl]);
+        const bool xok = mbar_wait_bounded(&xbar[sl], (it >> 1) & 1, abort_flag, kWaitNs);
+        if (!xok) {
+          raise_abort(abort_flag, p.err);
+          break;
+        }
+        ma = fmaxf(ma, slot[(wg ^ 1) * BM + rit]);
+        mb = fmaxf(mb, slot[(kEpiWG + (wg ^ 1)) * BM + rit]);
+        const float sca = ma == 0.f ? 1.f : __fdiv_rn(ma, 448.f);
+        const float scb = mb == 0.f ? 1.f : __fdiv_rn(mb, 448.f);
+        if (valid) {
+          // pass 2: the same float32 da, db again, quantised with the tile scales
+          uint8_t* qa_p = static_cast<uint8_t*>(p.C) + row * (2 * I) + c0;
+          uint8_t* qb_p = qa_p + I;
+#pragma unroll
+          for (int j16 = 0; j16 < CW / 16; ++j16) {
+            uint32_t wa[4], wb[4];
+#pragma unroll
+            for (int h8 = 0; h8 < 2; ++h8) {
+              float fa[8], fb[8];
+              Vec<__nv_bfloat16>::load(reinterpret_cast<const uint4*>(sa_p)[j16 * 2 + h8], fa);
+              Vec<__nv_bfloat16>::load(reinterpret_cast<const uint4*>(sb_p)[j16 * 2 + h8], fb);
+              float da[8], db[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float dhv = acc[j16 * 16 + h8 * 8 + i];
+                const float sg = __fdividef(1.0f, 1.0f + __expf(-fa[i]));
+                da[i] = dhv * fb[i] * (sg * (1.0f + fa[i] * (1.0f - sg)));
+                db[i] = dhv * fa[i] * sg;
+              }
+              wa[h8 * 2] = e4m3x4(__fdiv_rn(da[0], sca), __fdiv_rn(da[1], sca),
+                                  __fdiv_rn(da[2], sca), __fdiv_rn(da[3], sca));
+              wa[h8 * 2 + 1] = e4m3x4(__fdiv_rn(da[4], sca), __fdiv_rn(da[5], sca),
+                                      __fdiv_rn(da[6], sca), __fdiv_rn(da[7], sca));
+              wb[h8 * 2] = e4m3x4(__fdiv_rn(db[0], scb), __fdiv_rn(db[1], scb),
+                                  __fdiv_rn(db[2], scb), __fdiv_rn(db[3], scb));
+              wb[h8 * 2 + 1] = e4m3x4(__fdiv_rn(db[4], scb), __fdiv_rn(db[5], scb),
+                                      __fdiv_rn(db[6], scb), __fdiv_rn(db[7], scb));
+            }
+            reinterpret_cast<uint4*>(qa_p)[j16] = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+            reinterpret_cast<uint4*>(qb_p)[j16] = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+          }
+          if ((wg & 1) == 0) {
+            const int tile = c0 / 128;
+            p.c_scale[row * (2 * I / 128) + tile] = sca;
+            p.c_scale[row * (2 * I / 128) + I / 128 + tile] = scb;
+          }
+        }
+      } else if (SWIGLU) {
         float amax = 0.f;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
@@ -339,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // The row's 128 h columns are spread over the warpgroups: exchange amax.
         const int sl = it & 1;
-        float* slot = amax_x + sl * kEpiWG * BM;
+        float* slot = amax_x + sl * 2 * kEpiWG * BM;
         slot[wg * BM + rit] = amax;
         mbar_arrive(&xbar[sl]);
         const bool xok = mbar_wait_bounded(&xbar[sl], (it >> 1) & 1, abort_flag, kWaitNs);
@@ -392,19 +525,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <bool SWIGLU>
+template <int EPI, bool B_MN>
 moe_status fp8_launch(const void* A, const float* a_scale, const void* B, const float* b_scale,
                       int b_rows_per_group, const int32_t* offsets, int n_groups, int rows, int N,
-                      int K, void* C, float* c_scale, cudaStream_t s) {
-  constexpr int BN_OUT = SWIGLU ? BN / 2 : BN;
+                      int K, void* C, float* c_scale, void* S, int lds, void* C2,
+                      cudaStream_t s) {
+  constexpr int BN_OUT = Fp8Tile<EPI>::BN_OUT;
   CUtensorMap tmA, tmB;
   moe_status st = make_tmap_2d(&tmA, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, rows, BK, BM);
   if (st != MOE_OK) return st;
   const int G = offsets ? n_groups : 1;
-  st = make_tmap_2d(&tmB, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, (uint64_t)G * b_rows_per_group,
-                    BK, SWIGLU ? 128 : BN);
+  if (B_MN)
+    st = make_tmap_col_blocks(&tmB, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, (uint64_t)G * K, 128,
+                              BK, BN / 128);
+  else
+    st = make_tmap_2d(&tmB, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, (uint64_t)G * b_rows_per_group,
+                      BK, Fp8Tile<EPI>::SW ? 128 : BN);
   if (st != MOE_OK) return st;
-  auto kern = fp8_gemm_kernel<SWIGLU>;
+  auto kern = fp8_gemm_kernel<EPI, B_MN>;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e =
@@ -419,11 +557,14 @@ moe_status fp8_launch(const void* A, const float* a_scale, const void* B, const 
   p.N = N;
   p.K = K;
   p.b_rows_per_group = b_rows_per_group;
-  p.half_b = SWIGLU ? b_rows_per_group / 2 : 0;
+  p.half_b = Fp8Tile<EPI>::SW ? b_rows_per_group / 2 : 0;
   p.a_scale = a_scale;
   p.b_scale = b_scale;
   p.C = C;
   p.c_scale = c_scale;
+  p.S = static_cast<__nv_bfloat16*>(S);
+  p.lds = lds;
+  p.C2 = static_cast<__nv_bfloat16*>(C2);
   p.err = device_error_word();
   if (!p.err) return fail(MOE_ERR_CUDA, "device error word unavailable");
   const long long max_tiles = ((long long)(rows + BM - 1) / BM + (offsets ? G : 0)) * (N / BN_OUT);
@@ -439,18 +580,42 @@ moe_status launch_fp8_gemm(const void* A, const float* a_scale, const void* B,
                            const float* b_scale, int b_rows_per_group, const int32_t* offsets,
                            int n_groups, int rows, int N, int K, bool swiglu, void* C,
                            float* c_scale, cudaStream_t s) {
+  return launch_fp8_gemm_ex(A, a_scale, B, b_scale, b_rows_per_group, offsets, n_groups, rows, N,
+                            K, swiglu ? F8_SWIGLU : F8_STORE, false, C, c_scale, nullptr, 0,
+                            nullptr, s);
+}
+
+moe_status launch_fp8_gemm_ex(const void* A, const float* a_scale, const void* B,
+                              const float* b_scale, int b_rows_per_group, const int32_t* offsets,
+                              int n_groups, int rows, int N, int K, Fp8Epi epi, bool b_mn,
+                              void* C, float* c_scale, void* S, int lds, void* C2,
+                              cudaStream_t s) {
   if (rows <= 0) return MOE_OK;
   if (K % BK) return fail(MOE_ERR_UNSUPPORTED, "fp8 gemm: K=%d not a multiple of 128", K);
   if (offsets && n_groups > kMaxGroups)
     return fail(MOE_ERR_UNSUPPORTED, "fp8 gemm: at most %d groups", kMaxGroups);
-  if (swiglu) {
-    if (N % 128) return fail(MOE_ERR_UNSUPPORTED, "fp8 gemm swiglu: N=%d %% 128", N);
-    return fp8_launch<true>(A, a_scale, B, b_scale, b_rows_per_group, offsets, n_groups, rows, N,
-                            K, C, c_scale, s);
+  const bool sw = epi == F8_SWIGLU || epi == F8_SWIGLU_SAVE;
+  if (sw && N % 128) return fail(MOE_ERR_UNSUPPORTED, "fp8 gemm swiglu: N=%d %% 128", N);
+  if (!sw && N % 256) return fail(MOE_ERR_UNSUPPORTED, "fp8 gemm: N=%d must be a multiple of 256", N);
+  if (sw && b_mn) return fail(MOE_ERR_UNSUPPORTED, "fp8 gemm: MN-major weights with swiglu");
+  if (epi == F8_DSWIGLU && !b_mn) return fail(MOE_ERR_UNSUPPORTED, "fp8 dswiglu needs MN-major W");
+  switch (epi) {
+    case F8_SWIGLU:
+      return fp8_launch<F8_SWIGLU, false>(A, a_scale, B, b_scale, b_rows_per_group, offsets,
+                                          n_groups, rows, N, K, C, c_scale, S, lds, C2, s);
+    case F8_SWIGLU_SAVE:
+      return fp8_launch<F8_SWIGLU_SAVE, false>(A, a_scale, B, b_scale, b_rows_per_group, offsets,
+                                               n_groups, rows, N, K, C, c_scale, S, lds, C2, s);
+    case F8_STORE:
+      return b_mn ? fp8_launch<F8_STORE, true>(A, a_scale, B, b_scale, b_rows_per_group, offsets,
+                                               n_groups, rows, N, K, C, c_scale, S, lds, C2, s)
+                  : fp8_launch<F8_STORE, false>(A, a_scale, B, b_scale, b_rows_per_group, offsets,
+                                                n_groups, rows, N, K, C, c_scale, S, lds, C2, s);
+    case F8_DSWIGLU:
+      return fp8_launch<F8_DSWIGLU, true>(A, a_scale, B, b_scale, b_rows_per_group, offsets,
+                                          n_groups, rows, N, K, C, c_scale, S, lds, C2, s);
   }
-  if (N % 256) return fail(MOE_ERR_UNSUPPORTED, "fp8 gemm down: d=%d must be a multiple of 256", N);
-  return fp8_launch<false>(A, a_scale, B, b_scale, b_rows_per_group, offsets, n_groups, rows, N, K,
-                           C, c_scale, s);
+  return fail(MOE_ERR_INVALID_ARG, "fp8 gemm: unknown epilogue %d", (int)epi);
 }
 
 }  // namespace moe

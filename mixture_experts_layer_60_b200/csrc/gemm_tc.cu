@@ -345,10 +345,20 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
 
 }  // namespace
 
-// Shared with gemm_fp8.cu.
+// Shared with the other tcgen05 kernels: 128-byte swizzle.
+moe_status make_tmap_2d_swz(CUtensorMap* tm, const void* base, CUtensorMapDataType dtype,
+                            int elem_bytes, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                            uint32_t box_outer, CUtensorMapSwizzle swz);
 moe_status make_tmap_2d(CUtensorMap* tm, const void* base, CUtensorMapDataType dtype,
                         int elem_bytes, uint64_t inner, uint64_t outer, uint32_t box_inner,
                         uint32_t box_outer) {
+  return make_tmap_2d_swz(tm, base, dtype, elem_bytes, inner, outer, box_inner, box_outer,
+                          CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+moe_status make_tmap_2d_swz(CUtensorMap* tm, const void* base, CUtensorMapDataType dtype,
+                            int elem_bytes, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                            uint32_t box_outer, CUtensorMapSwizzle swz) {
   static EncodeTiledFn encode = nullptr;
   if (!encode) {
     void* fn = nullptr;
@@ -368,9 +378,42 @@ moe_status make_tmap_2d(CUtensorMap* tm, const void* base, CUtensorMapDataType d
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = encode(tm, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
-                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return MOE_OK;
+}
+
+// A row-major [rows, cols] matrix seen as blocks of `bc` columns: dimensions
+// (bc columns, rows, cols/bc blocks) with strides (row pitch, bc * elem bytes),
+// so that one box of (bc, box_rows, box_blocks) lands in shared memory as
+// box_blocks consecutive [box_rows][bc] tiles (128-byte swizzle, bc * elem = 128).
+moe_status make_tmap_col_blocks(CUtensorMap* tm, const void* base, CUtensorMapDataType dtype,
+                                int elem_bytes, uint64_t cols, uint64_t rows, uint32_t bc,
+                                uint32_t box_rows, uint32_t box_blocks) {
+  static EncodeTiledFn encode = nullptr;
+  if (!encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
+      return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled not available");
+    encode = reinterpret_cast<EncodeTiledFn>(fn);
+  }
+  if (reinterpret_cast<uintptr_t>(base) % 16 != 0)
+    return fail(MOE_ERR_INVALID_ARG, "TMA operand base %p is not 16-byte aligned", base);
+  if ((cols * elem_bytes) % 16 != 0 || cols % bc != 0)
+    return fail(MOE_ERR_UNSUPPORTED, "TMA column blocks: %llu columns",
+                (unsigned long long)cols);
+  cuuint64_t dims[3] = {bc, rows, cols / bc};
+  cuuint64_t strides[2] = {cols * elem_bytes, (cuuint64_t)bc * elem_bytes};
+  cuuint32_t box[3] = {bc, box_rows, box_blocks};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = encode(tm, dtype, 3, const_cast<void*>(base), dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled (column blocks) failed (%d)", (int)r);
   return MOE_OK;
 }
 

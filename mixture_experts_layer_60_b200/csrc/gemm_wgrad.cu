@@ -16,8 +16,11 @@
 // tokens gets C_g = 0 from the epilogue without touching TMEM.
 //
 // Roles: warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer (the whole
-// warp zeroes ragged rows, one lane issues), warps 2-9 epilogue (warp w
-// reads TMEM lanes 32*(w%4).. = C rows and one 128-column half).  Every wait
+// warp zeroes ragged rows, one lane issues), warps 2-17 epilogue (warp w
+// reads TMEM lanes 32*(w%4).. = C rows and one 64-column quarter of the
+// tile; each 32x32 block is converted to bf16 into a 2 KB shared-memory
+// patch laid out as a 64-byte-swizzled [32 rows][32 cols] TMA box and written
+// to global memory by one TMA store).  Every wait
 // is bounded (1 s) and reported through the device error word.
 #include "launch.h"
 #include "sm100.cuh"
@@ -32,7 +35,7 @@ constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 64;              // token rows per stage
 constexpr int STAGES = 4;
-constexpr int kEpiWarps = 8;
+constexpr int kEpiWarps = 16;       // 4 per TMEM lane quarter, 64 columns each
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint64_t kWaitNs = 1000000000ull;
 constexpr uint32_t TMEM_COLS = 512;
@@ -41,7 +44,8 @@ constexpr int BOX_BYTES = 64 * BK * 2;         // one [64 tok][64 mn] bf16 box: 
 constexpr int A_BYTES = 2 * BOX_BYTES;         // 16 KB
 constexpr int B_BYTES = 4 * BOX_BYTES;         // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int OFF_BAR = STAGES * STAGE_BYTES;
+constexpr int OFF_PATCH = STAGES * STAGE_BYTES;        // one 2 KB transpose patch per epilogue warp
+constexpr int OFF_BAR = OFF_PATCH + kEpiWarps * 2048;
 constexpr int N_BARS = 2 * STAGES + 5;
 constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16;
@@ -73,7 +77,8 @@ __device__ __forceinline__ void raise_abort(volatile int* abort, int* err) {
 
 __global__ void __launch_bounds__(kThreads, 1)
     wgrad_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
-                      const __grid_constant__ CUtensorMap tmB, const WgParams p) {
+                      const __grid_constant__ CUtensorMap tmB,
+                      const __grid_constant__ CUtensorMap tmC, const WgParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -131,12 +136,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* a_dst = smem + stage * STAGE_BYTES;
           uint8_t* b_dst = a_dst + A_BYTES;
           const int row = r0 + kb * BK;
-#pragma unroll
-          for (int j = 0; j < 2; ++j)
-            tma_load_2d(a_dst + j * BOX_BYTES, &tmA, mt * BM + 64 * j, row, &full[stage]);
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            tma_load_2d(b_dst + j * BOX_BYTES, &tmB, nt * BN + 64 * j, row, &full[stage]);
+          // one TMA per operand: 2 (A) / 4 (B) consecutive [64 tok][64 col] tiles
+          tma_load_3d(a_dst, &tmA, 0, row, mt * (BM / 64), &full[stage]);
+          tma_load_3d(b_dst, &tmB, 0, row, nt * (BN / 64), &full[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
@@ -209,7 +211,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ---------------------------------------------------------------- epilogue
     const int q = warp & 3;                       // TMEM lane quarter = C rows q*32..
-    const int half = (warp - 2) >> 2;             // 128-column half of the tile
+    const int cq = (warp - 2) >> 2;               // 64-column quarter of the tile
+    uint4* patch = reinterpret_cast<uint4*>(smem + OFF_PATCH + (warp - 2) * 2048);   // [32][4]
     int used = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
       const int g = t / per_group, loc = t - g * per_group;
@@ -217,10 +220,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       int r0, cnt;
       group_rows(p, g, r0, cnt);
       const int m = mt * BM + q * 32 + lane;
-      __nv_bfloat16* dst_row = p.C + ((size_t)g * p.M + m) * p.N + nt * BN + half * 128;
+      __nv_bfloat16* dst_row = p.C + ((size_t)g * p.M + m) * p.N + nt * BN + cq * 64;
       if (cnt <= 0) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
+        for (int i = 0; i < 8; ++i)
           reinterpret_cast<uint4*>(dst_row)[i] = make_uint4(0u, 0u, 0u, 0u);
         continue;
       }
@@ -233,28 +236,42 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const uint32_t tl = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ab * BN + half * 128;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tl + c * 32, r);
-        tmem_wait_ld();
-        uint32_t w[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          __nv_bfloat162 pr = __floats2bfloat162_rn(__uint_as_float(r[2 * i]),
-                                                    __uint_as_float(r[2 * i + 1]));
-          w[i] = *reinterpret_cast<uint32_t*>(&pr);
-        }
-        uint4* d4 = reinterpret_cast<uint4*>(dst_row + c * 32);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-      }
+      const uint32_t tl = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ab * BN + cq * 64;
+      uint32_t r[2][32];
+      tmem_ld_32x32b_x32(tl, r[0]);
+      tmem_ld_32x32b_x32(tl + 32, r[1]);
+      tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(&tempty[ab]);
+      mbar_arrive(&tempty[ab]);      // accumulator read: the next tile's MMAs may start
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        // the previous TMA store must have read the patch before it is rewritten
+        if (lane == 0) tma_store_wait_read_all();
+        __syncwarp();
+        // row `lane` (64 bytes) into the patch, 64-byte swizzle: 16-byte slot i
+        // of row r sits at i ^ ((r >> 1) & 3) (also spreads 8 lanes over 8 bank groups)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          uint32_t w4[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            __nv_bfloat162 pr = __floats2bfloat162_rn(__uint_as_float(r[c][8 * i + 2 * k]),
+                                                      __uint_as_float(r[c][8 * i + 2 * k + 1]));
+            w4[k] = *reinterpret_cast<uint32_t*>(&pr);
+          }
+          patch[lane * 4 + (i ^ ((lane >> 1) & 3))] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tmC, patch, nt * BN + cq * 64 + c * 32, g * p.M + mt * BM + q * 32);
+          tma_store_commit();
+        }
+      }
     }
   }
 
+  if (warp >= 2 && lane == 0) tma_store_wait_all();   // stores done before the CTA exits
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -268,6 +285,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 moe_status make_tmap_2d(CUtensorMap* tm, const void* base, CUtensorMapDataType dtype,
                         int elem_bytes, uint64_t inner, uint64_t outer, uint32_t box_inner,
                         uint32_t box_outer);
+moe_status make_tmap_2d_swz(CUtensorMap* tm, const void* base, CUtensorMapDataType dtype,
+                            int elem_bytes, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                            uint32_t box_outer, CUtensorMapSwizzle swz);
+moe_status make_tmap_col_blocks(CUtensorMap* tm, const void* base, CUtensorMapDataType dtype,
+                                int elem_bytes, uint64_t cols, uint64_t rows, uint32_t bc,
+                                uint32_t box_rows, uint32_t box_blocks);
 
 moe_status launch_wgrad_gemm(const void* A, int M, const void* B, int N, const int32_t* offsets,
                              int n_groups, int rows, void* C, cudaStream_t s) {
@@ -280,10 +303,15 @@ moe_status launch_wgrad_gemm(const void* A, int M, const void* B, int N, const i
     // every group is empty: C = 0
     return cuda_check(cudaMemsetAsync(C, 0, (size_t)G * M * N * 2, s), "wgrad zero fill");
   }
-  CUtensorMap tmA, tmB;
-  moe_status st = make_tmap_2d(&tmA, A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, rows, 64, BK);
+  CUtensorMap tmA, tmB, tmC;
+  moe_status st = make_tmap_col_blocks(&tmA, A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, rows, 64,
+                                       BK, BM / 64);
   if (st != MOE_OK) return st;
-  st = make_tmap_2d(&tmB, B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, rows, 64, BK);
+  st = make_tmap_col_blocks(&tmB, B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, rows, 64, BK, BN / 64);
+  if (st != MOE_OK) return st;
+  // output: [G*M rows][N cols], stored in [32 rows][32 cols] boxes with 64-byte swizzle
+  st = make_tmap_2d_swz(&tmC, C, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, (uint64_t)G * M, 32, 32,
+                        CU_TENSOR_MAP_SWIZZLE_64B);
   if (st != MOE_OK) return st;
   static bool attr_set = false;
   if (!attr_set) {
@@ -304,7 +332,7 @@ moe_status launch_wgrad_gemm(const void* A, int M, const void* B, int N, const i
   const long long tiles = (long long)G * (M / BM) * (N / BN);
   int grid = sm_count();
   if (tiles < grid) grid = (int)tiles;
-  wgrad_gemm_kernel<<<grid, kThreads, SMEM_ALLOC, s>>>(tmA, tmB, p);
+  wgrad_gemm_kernel<<<grid, kThreads, SMEM_ALLOC, s>>>(tmA, tmB, tmC, p);
   return cuda_check(cudaGetLastError(), "wgrad gemm launch");
 }
 

@@ -1,0 +1,367 @@
+// FP8 weight-gradient GEMM (the Wgrad pass under the FP8 recipe of
+// "DeepSeek-V3 技術報告", section 核心概念: E4M3 operands, 1x128 activation
+// tiles, FP32 promotion every N_c = 128).  The contraction runs over an
+// expert's tokens, so an activation tile is 128 consecutive rows of one
+// expert (blocks start at the expert's first row) x 1 column:
+//   C_g[m, n] = sum over g's blocks b of
+//               (sum_{r in b} qa[r, m] qb[r, n]) * sa[b, m] * sb[b, n]
+// qa [rows, M], qb [rows, N] e4m3 row-major (both MMA operands MN-major);
+// sa [blocks, M], sb [blocks, N] float32; C [G, M, N] bf16.
+//
+// Tile 128 x 256 outputs; each shared-memory stage is one 128-row block
+// (A: one [128 tok][128 m] box, B: two [128 tok][128 n] boxes, 128-byte
+// swizzle, 48 KB), 4 stages.  The MMA warp writes each block's partial
+// product into one of two TMEM buffers (tcgen05.mma kind::f8f6f4, K = 32 per
+// instruction; the rows of a ragged last block past the expert's end are
+// zeroed in shared memory first and only ceil(valid/32) MMAs are issued); 16
+// epilogue warps read it back (warp w: TMEM lanes 32*(w%4).. = C rows, 64
+// columns), add P * sa[b, m] * sb[b, n] into float32 registers with paired
+// FMAs, and after the expert's last block write bf16 through a 64-byte-
+// swizzled shared-memory patch and TMA stores.  Waits are bounded (1 s).
+#include "launch.h"
+#include "sm100.cuh"
+
+namespace moe {
+
+moe_status make_tmap_2d(CUtensorMap* tm, const void* base, CUtensorMapDataType dtype,
+                        int elem_bytes, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                        uint32_t box_outer);
+moe_status make_tmap_2d_swz(CUtensorMap* tm, const void* base, CUtensorMapDataType dtype,
+                            int elem_bytes, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                            uint32_t box_outer, CUtensorMapSwizzle swz);
+moe_status make_tmap_col_blocks(CUtensorMap* tm, const void* base, CUtensorMapDataType dtype,
+                                int elem_bytes, uint64_t cols, uint64_t rows, uint32_t bc,
+                                uint32_t box_rows, uint32_t box_blocks);
+
+namespace {
+
+using namespace sm100;
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 128;             // token rows per stage = one promotion block
+constexpr int STAGES = 4;
+constexpr int kEpiWarps = 16;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr uint64_t kWaitNs = 1000000000ull;
+constexpr uint32_t TMEM_COLS = 512;
+
+constexpr int BOX_BYTES = 128 * BK;            // [128 tok][128 e4m3]: 16 KB
+constexpr int A_BYTES = BOX_BYTES;
+constexpr int B_BYTES = 2 * BOX_BYTES;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int OFF_PATCH = STAGES * STAGE_BYTES;
+constexpr int OFF_BAR = OFF_PATCH + kEpiWarps * 2048;
+constexpr int N_BARS = 2 * STAGES + 5;
+constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
+constexpr int SMEM_BYTES = OFF_MISC + 16;
+constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
+
+struct Wg8Params {
+  const int32_t* offsets;
+  int n_groups;
+  int rows;
+  int M, N;
+  const float* sa;            // [blocks, M]
+  const float* sb;            // [blocks, N]
+  const int32_t* block_start; // [G+1]
+  __nv_bfloat16* Cp;          // [G, M, N]
+  int* err;
+  __device__ __nv_bfloat16* C(int g, int m, int n) const {
+    return Cp + ((size_t)g * M + m) * N + n;
+  }
+};
+
+__device__ __forceinline__ void group_rows(const Wg8Params& p, int g, int& r0, int& cnt) {
+  if (p.offsets) {
+    r0 = p.offsets[g];
+    cnt = p.offsets[g + 1] - r0;
+  } else {
+    r0 = 0;
+    cnt = p.rows;
+  }
+}
+
+__device__ __forceinline__ void raise_abort(volatile int* abort, int* err) {
+  *abort = 1;
+  atomicOr(err, ERR_GEMM_FP8_TIMEOUT);
+}
+
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+// c += (x0, x1) * s2 with x0, x1 the raw bits of two float32 TMEM words
+__device__ __forceinline__ uint64_t fma2_bits(uint32_t x0, uint32_t x1, uint64_t s2, uint64_t c) {
+  asm("{\n\t.reg .b64 t;\n\tmov.b64 t, {%1, %2};\n\tfma.rn.f32x2 %0, t, %3, %0;\n\t}"
+      : "+l"(c)
+      : "r"(x0), "r"(x1), "l"(s2));
+  return c;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    wgrad_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
+                     const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmC, const Wg8Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* empty = full + STAGES;
+  uint64_t* pfull = empty + STAGES;      // [2] partial product ready
+  uint64_t* pempty = pfull + 2;          // [2] partial product read by the epilogue
+  uint64_t* mma_done = pempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = p.offsets ? p.n_groups : 1;
+  const int n_m = p.M / BM, n_n = p.N / BN;
+  const int per_group = n_m * n_n;
+  const int total = G * per_group;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&pfull[b], 1); mbar_init(&pempty[b], 32 * kEpiWarps); }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const int g = t / per_group, loc = t - g * per_group;
+        const int mt = loc / n_n, nt = loc - mt * n_n;
+        int r0, cnt;
+        group_rows(p, g, r0, cnt);
+        const int nkb = (cnt + BK - 1) / BK;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, kWaitNs)) {
+            raise_abort(abort_flag, p.err);
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+          uint8_t* a_dst = smem + stage * STAGE_BYTES;
+          const int row = r0 + kb * BK;
+          tma_load_2d(a_dst, &tmA, mt * BM, row, &full[stage]);
+          tma_load_3d(a_dst + A_BYTES, &tmB, 0, row, nt * (BN / 128), &full[stage]);   // 2 tiles
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+      for (int s = 0; s < STAGES; ++s)
+        mbar_wait_bounded(&full[s], ((s < stage) ? phase : phase ^ 1), nullptr, kWaitNs);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    int stage = 0, pb = 0;
+    uint32_t phase = 0, pphase = 0;
+    bool ok = true;
+    const uint32_t idesc = idesc_e4m3_f32(BM, BN) | (1u << 15) | (1u << 16);   // A, B MN-major
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      const int g = t / per_group;
+      int r0, cnt;
+      group_rows(p, g, r0, cnt);
+      const int nkb = (cnt + BK - 1) / BK;
+      for (int kb = 0; kb < nkb; ++kb) {
+        const bool w1 = mbar_wait_bounded(&pempty[pb], pphase ^ 1, abort_flag, kWaitNs);
+        const bool w2 = w1 && mbar_wait_bounded(&full[stage], phase, abort_flag, kWaitNs);
+        if (!__all_sync(0xffffffffu, w2)) {
+          if (lane == 0) raise_abort(abort_flag, p.err);
+          ok = false;
+          break;
+        }
+        uint8_t* a_st = smem + stage * STAGE_BYTES;
+        const int valid = min(BK, cnt - kb * BK);
+        const int nks = (valid + 31) / 32;
+        if (valid < nks * 32) {
+          // rows [valid, nks*32) of the A box belong to the next expert: zero them
+          const int chunks = (nks * 32 - valid) * 8;     // 16-byte chunks
+          for (int i = lane; i < chunks; i += 32) {
+            uint8_t* dst = a_st + (valid + (i >> 3)) * 128 + (i & 7) * 16;
+            *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+          }
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t a0 = smem_u32(a_st), b0 = a0 + A_BYTES;
+          const uint32_t d_tmem = tmem_base + pb * BN;
+          for (int k = 0; k < nks; ++k)
+            mma_f8_ss(d_tmem, smem_desc_mn_sw128(a0 + k * 4096, BOX_BYTES),
+                      smem_desc_mn_sw128(b0 + k * 4096, BOX_BYTES), idesc, k != 0);
+          mma_commit(&empty[stage]);
+          mma_commit(&pfull[pb]);
+        }
+        __syncwarp();
+        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        if (++pb == 2) { pb = 0; pphase ^= 1; }
+      }
+    }
+    if (lane == 0) {
+      mma_commit(mma_done);
+      mbar_wait_bounded(mma_done, 0, nullptr, kWaitNs);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int q = warp & 3;                       // TMEM lane quarter = C rows q*32..
+    const int cq = (warp - 2) >> 2;               // 64-column quarter of the tile
+    uint4* patch = reinterpret_cast<uint4*>(smem + OFF_PATCH + (warp - 2) * 2048);   // [32][4]
+    int pb = 0;
+    uint32_t pphase = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      const int g = t / per_group, loc = t - g * per_group;
+      const int mt = loc / n_n, nt = loc - mt * n_n;
+      int r0, cnt;
+      group_rows(p, g, r0, cnt);
+      const int m = mt * BM + q * 32 + lane;
+      const int n0 = nt * BN + cq * 64;
+      if (cnt <= 0) {
+        uint4* d4 = reinterpret_cast<uint4*>(p.C(g, m, n0));
+#pragma unroll
+        for (int i = 0; i < 8; ++i) d4[i] = make_uint4(0u, 0u, 0u, 0u);
+        continue;
+      }
+      uint64_t acc2[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) acc2[i] = 0ull;
+      const int nkb = (cnt + BK - 1) / BK;
+      const int blk0 = p.block_start[g];
+      for (int kb = 0; kb < nkb; ++kb) {
+        const float sa = p.sa[(size_t)(blk0 + kb) * p.M + m];
+        const float* sbr = p.sb + (size_t)(blk0 + kb) * p.N + n0;
+        const bool got = mbar_wait_bounded(&pfull[pb], pphase, abort_flag, kWaitNs);
+        if (!__all_sync(0xffffffffu, got)) {
+          if (lane == 0) raise_abort(abort_flag, p.err);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + pb * BN + cq * 64;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[16];
+          tmem_ld_32x32b_x16(tb + c * 16, r);
+          tmem_wait_ld();
+          if (c == 3) {
+            tc_fence_before();
+            mbar_arrive(&pempty[pb]);   // partial read: the MMA may overwrite it
+          }
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const float4 s4 = *reinterpret_cast<const float4*>(sbr + c * 16 + v * 4);
+            acc2[c * 8 + 2 * v] = fma2_bits(r[4 * v], r[4 * v + 1], f2_pack(sa * s4.x, sa * s4.y),
+                                             acc2[c * 8 + 2 * v]);
+            acc2[c * 8 + 2 * v + 1] = fma2_bits(r[4 * v + 2], r[4 * v + 3],
+                                                f2_pack(sa * s4.z, sa * s4.w),
+                                                acc2[c * 8 + 2 * v + 1]);
+          }
+        }
+        if (++pb == 2) { pb = 0; pphase ^= 1; }
+      }
+      if (!ok) break;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        if (lane == 0) tma_store_wait_read_all();
+        __syncwarp();
+        // row `lane` (64 bytes) into the 64-byte-swizzled patch: slot i at i ^ ((lane >> 1) & 3)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          uint32_t w4[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            float x0, x1;
+            f2_unpack(acc2[c * 16 + 4 * i + k], x0, x1);
+            __nv_bfloat162 pr = __floats2bfloat162_rn(x0, x1);
+            w4[k] = *reinterpret_cast<uint32_t*>(&pr);
+          }
+          patch[lane * 4 + (i ^ ((lane >> 1) & 3))] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tmC, patch, n0 + c * 32, g * p.M + mt * BM + q * 32);
+          tma_store_commit();
+        }
+      }
+    }
+  }
+
+  if (warp >= 2 && lane == 0) tma_store_wait_all();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace
+
+moe_status launch_wgrad_fp8(const void* qa, const float* sa, int M, const void* qb,
+                            const float* sb, int N, const int32_t* offsets, int n_groups,
+                            int rows, const int32_t* block_start, void* C, cudaStream_t s) {
+  const int G = offsets ? n_groups : 1;
+  if (G <= 0) return MOE_OK;
+  if (M % BM || N % BN)
+    return fail(MOE_ERR_UNSUPPORTED, "fp8 wgrad: M=%d must be a multiple of %d, N=%d of %d", M,
+                BM, N, BN);
+  if (rows <= 0)
+    return cuda_check(cudaMemsetAsync(C, 0, (size_t)G * M * N * 2, s), "fp8 wgrad zero fill");
+  CUtensorMap tmA, tmB, tmC;
+  moe_status st = make_tmap_2d(&tmA, qa, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, rows, 128, BK);
+  if (st != MOE_OK) return st;
+  st = make_tmap_col_blocks(&tmB, qb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, rows, 128, BK, BN / 128);
+  if (st != MOE_OK) return st;
+  st = make_tmap_2d_swz(&tmC, C, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, (uint64_t)G * M, 32, 32,
+                        CU_TENSOR_MAP_SWIZZLE_64B);
+  if (st != MOE_OK) return st;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(wgrad_fp8_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
+    if (e != cudaSuccess) return cuda_check(e, "fp8 wgrad smem attribute");
+    attr_set = true;
+  }
+  Wg8Params p;
+  p.offsets = offsets;
+  p.n_groups = G;
+  p.rows = rows;
+  p.M = M;
+  p.N = N;
+  p.sa = sa;
+  p.sb = sb;
+  p.block_start = block_start;
+  p.Cp = static_cast<__nv_bfloat16*>(C);
+  p.err = device_error_word();
+  if (!p.err) return fail(MOE_ERR_CUDA, "device error word unavailable");
+  const long long tiles = (long long)G * (M / BM) * (N / BN);
+  int grid = sm_count();
+  if (tiles < grid) grid = (int)tiles;
+  wgrad_fp8_kernel<<<grid, kThreads, SMEM_ALLOC, s>>>(tmA, tmB, tmC, p);
+  return cuda_check(cudaGetLastError(), "fp8 wgrad launch");
+}
+
+}  // namespace moe

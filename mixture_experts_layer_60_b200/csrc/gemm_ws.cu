@@ -305,7 +305,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (EPI == WS_DSWIGLU) {
         // dh[tok, col] from TMEM; a = S[tok, col], b = S[tok, I + col]:
         //   dA[tok, col] = dh * b * SiLU'(a),  dA[tok, I + col] = dh * SiLU(a).
-        // Lane = feature column, so each access of the warp covers 64 contiguous bytes.
+        // dh goes through a float32 [16 tok][32 col] patch so that every
+        // global access is a 16-byte vector along a token row.
+        float* pf = reinterpret_cast<float*>(patch);
         for (int c = ch; c < nch; c += 2) {
           uint32_t r0[32], r1[32];
           tmem_ld_32x32b_x32(tl + c * 32, r0);
@@ -313,19 +315,53 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_ld();
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
-            const int col = nt * 256 + hh * 128 + q * 32 + lane;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int tok = c * 32 + j;
-              if (tok < count) {
-                const size_t row = (size_t)(tok0 + tok);
-                const float dhv = __uint_as_float(hh == 0 ? r0[j] : r1[j]);
-                const float a = __bfloat162float(p.S[row * p.lds + col]);
-                const float b = __bfloat162float(p.S[row * p.lds + p.N + col]);
-                const float sg = __fdividef(1.0f, 1.0f + __expf(-a));
-                p.C[row * p.ldc + col] = __float2bfloat16_rn(dhv * b * (sg * (1.0f + a * (1.0f - sg))));
-                p.C[row * p.ldc + p.N + col] = __float2bfloat16_rn(dhv * a * sg);
+            for (int sub = 0; sub < 2; ++sub) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j)
+                pf[j * 32 + lane] = __uint_as_float(hh == 0 ? r0[sub * 16 + j] : r1[sub * 16 + j]);
+              __syncwarp();
+              // both 16-byte pieces of this lane first, then the arithmetic
+              uint4 av[2], bv[2];
+              size_t grow[2];
+              int col[2], c8[2], row[2];
+              bool ok[2];
+#pragma unroll
+              for (int it = 0; it < 2; ++it) {
+                const int idx = it * 32 + lane;
+                row[it] = idx >> 2;
+                c8[it] = (idx & 3) * 8;
+                const int tok = c * 32 + sub * 16 + row[it];
+                ok[it] = tok < count;
+                grow[it] = (size_t)(tok0 + (ok[it] ? tok : 0));
+                col[it] = nt * 256 + hh * 128 + q * 32 + c8[it];
+                if (ok[it]) {
+                  av[it] = *reinterpret_cast<const uint4*>(p.S + grow[it] * p.lds + col[it]);
+                  bv[it] = *reinterpret_cast<const uint4*>(p.S + grow[it] * p.lds + p.N + col[it]);
+                }
               }
+#pragma unroll
+              for (int it = 0; it < 2; ++it) {
+                if (ok[it]) {
+                  const float4 d0 = *reinterpret_cast<const float4*>(pf + row[it] * 32 + c8[it]);
+                  const float4 d1 = *reinterpret_cast<const float4*>(pf + row[it] * 32 + c8[it] + 4);
+                  const float dv[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+                  float fa[8], fb[8], oa[8], ob[8];
+                  Vec<__nv_bfloat16>::load(av[it], fa);
+                  Vec<__nv_bfloat16>::load(bv[it], fb);
+#pragma unroll
+                  for (int i = 0; i < 8; ++i) {
+                    const float sg = __fdividef(1.0f, 1.0f + __expf(-fa[i]));
+                    oa[i] = dv[i] * fb[i] * (sg * (1.0f + fa[i] * (1.0f - sg)));
+                    ob[i] = dv[i] * fa[i] * sg;
+                  }
+                  *reinterpret_cast<uint4*>(p.C + grow[it] * p.ldc + col[it]) =
+                      Vec<__nv_bfloat16>::store(oa);
+                  *reinterpret_cast<uint4*>(p.C + grow[it] * p.ldc + p.N + col[it]) =
+                      Vec<__nv_bfloat16>::store(ob);
+                }
+              }
+              __syncwarp();
             }
           }
         }

@@ -70,15 +70,39 @@ moe_status launch_ws_gemm_ex(const void* X, const void* W, int b_rows_per_group,
 moe_status launch_wgrad_gemm(const void* A, int M, const void* B, int N, const int32_t* offsets,
                              int n_groups, int rows, void* C, cudaStream_t s);
 
+// gemm_wgrad_fp8.cu ----------------------------------------------------------
+// C[g] [M, N] = sum over g's 128-row blocks b of (qa_b^T qb_b) * sa[b, m] * sb[b, n].
+moe_status launch_wgrad_fp8(const void* qa, const float* sa, int M, const void* qb,
+                            const float* sb, int N, const int32_t* offsets, int n_groups,
+                            int rows, const int32_t* block_start, void* C, cudaStream_t s);
+
 // gemm_fp8.cu ----------------------------------------------------------------
 moe_status launch_fp8_gemm(const void* A, const float* a_scale, const void* B,
                            const float* b_scale, int b_rows_per_group,
                            const int32_t* offsets, int n_groups, int rows, int N, int K,
                            bool swiglu, void* C, float* c_scale, cudaStream_t s);
+// Epilogues as in gemm_fp8.cu's header; b_mn: B stored [G*K rows][N cols].
+enum Fp8Epi { F8_SWIGLU = 0, F8_STORE = 1, F8_SWIGLU_SAVE = 2, F8_DSWIGLU = 3 };
+moe_status launch_fp8_gemm_ex(const void* A, const float* a_scale, const void* B,
+                              const float* b_scale, int b_rows_per_group, const int32_t* offsets,
+                              int n_groups, int rows, int N, int K, Fp8Epi epi, bool b_mn,
+                              void* C, float* c_scale, void* S, int lds, void* C2,
+                              cudaStream_t s);
 moe_status launch_quant_1x128(const void* x, int rows, int cols, uint8_t* q, float* scale,
                               cudaStream_t s);
 moe_status launch_quant_128x128(const void* w, int groups, int rows, int cols, uint8_t* q,
                                 float* scale, cudaStream_t s);
+// Wgrad operands: group-aligned 128-row blocks, one scale per (block, column).
+// block_start[g] = first block of group g (computed by launch_block_table).
+moe_status launch_block_table(const int32_t* offsets, int n_groups, int rows,
+                              int32_t* block_start, cudaStream_t s);
+// x [*, ldx] bf16; row r of the operand is x[src_rows ? src_rows[r] : r];
+// swiglu_in: the operand is SiLU(x[:, 0:cols]) * x[:, cols:2cols].
+// q [rows, cols] e4m3, scale [blocks, cols] float32.
+moe_status launch_quant_128x1(const void* x, int ldx, const int32_t* src_rows, bool swiglu_in,
+                              int rows, int cols, const int32_t* offsets, int n_groups,
+                              const int32_t* block_start, uint8_t* q, float* scale,
+                              cudaStream_t s);
 
 // combine.cu -----------------------------------------------------------------
 moe_status launch_combine(const void* u, const void* y_shared, int N_s, const void* y_perm,
@@ -98,8 +122,8 @@ moe_status launch_unpermute_backward(const void* dh, const void* dx_shared, int 
                                      const int32_t* idx, const float* d_logit, const void* E,
                                      moe_dtype dt, int T, int d, int K, void* du,
                                      cudaStream_t s);
-moe_status launch_router_weight_grad(const void* x_perm, const float* d_logit_perm,
-                                     const int32_t* offsets, moe_dtype dt, int N_r, int d,
-                                     float* dE, cudaStream_t s);
+moe_status launch_router_weight_grad(const void* x, const int32_t* x_rows,
+                                     const float* d_logit_perm, const int32_t* offsets,
+                                     moe_dtype dt, int N_r, int d, float* dE, cudaStream_t s);
 
 }  // namespace moe

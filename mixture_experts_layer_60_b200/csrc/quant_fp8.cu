@@ -118,4 +118,130 @@ moe_status launch_quant_128x128(const void* w, int groups, int rows, int cols, u
   return cuda_check(cudaGetLastError(), "quant_128x128 launch");
 }
 
+namespace {
+
+// ---------------------------------------------------------------- Wgrad operands
+// 128x1 tiles along the rows of each group (the contraction of a weight
+// gradient runs over an expert's tokens): blocks of 128 consecutive rows start
+// at every group's first row, the last block of a group may be shorter, and
+// every column of a block gets its own scale.
+
+// block_start[g] = sum over g' < g of ceil(rows of g' / 128); block_start[G] = total.
+__global__ void __launch_bounds__(1024) block_table_kernel(const int32_t* __restrict__ offsets,
+                                                           int G, int rows,
+                                                           int32_t* __restrict__ block_start) {
+  __shared__ int warp_sum[32];
+  const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+  int run = 0;
+  for (int base = 0; base < G; base += 1024) {
+    const int g = base + t;
+    int c = 0;
+    if (g < G) {
+      const int n = offsets ? offsets[g + 1] - offsets[g] : rows;
+      c = (n + 127) / 128;
+    }
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) warp_sum[w] = incl;
+    __syncthreads();
+    if (w == 0) {
+      int ws = warp_sum[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, ws, o);
+        if (lane >= o) ws += v;
+      }
+      warp_sum[lane] = ws;
+    }
+    __syncthreads();
+    const int before = (w > 0 ? warp_sum[w - 1] : 0) + incl - c;
+    if (g < G) block_start[g] = run + before;
+    const int chunk_total = warp_sum[31];
+    __syncthreads();
+    run += chunk_total;
+  }
+  if (t == 0) block_start[G] = run;
+}
+
+__device__ __forceinline__ float silu_fast(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
+
+// Two columns per thread, 256 columns per block; blockIdx.x = 128-row block.
+// SWIGLU_IN: the value of (row, c) is SiLU(x[row, c]) * x[row, cols + c].
+template <bool SWIGLU_IN>
+__global__ void __launch_bounds__(128) quant_128x1_kernel(
+    const __nv_bfloat16* __restrict__ x, int ldx, const int32_t* __restrict__ src_rows, int rows,
+    int cols, const int32_t* __restrict__ offsets, int G, const int32_t* __restrict__ block_start,
+    uint8_t* __restrict__ q, float* __restrict__ scale) {
+  const int blk = blockIdx.x;
+  if (blk >= block_start[G]) return;
+  int lo = 0, hi = G - 1;                  // last group whose first block is <= blk
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (block_start[mid] <= blk) lo = mid; else hi = mid - 1;
+  }
+  const int g0 = offsets ? offsets[lo] : 0;
+  const int g1 = offsets ? offsets[lo + 1] : rows;
+  const int r0 = g0 + (blk - block_start[lo]) * 128;
+  const int r1 = min(r0 + 128, g1);
+  const int c = (blockIdx.y * 128 + threadIdx.x) * 2;
+  if (c >= cols) return;
+  auto load = [&](int r, float& v0, float& v1) {
+    const size_t row = (size_t)(src_rows ? src_rows[r] : r);
+    const uint32_t a = *reinterpret_cast<const uint32_t*>(x + row * ldx + c);
+    v0 = __uint_as_float(a << 16);
+    v1 = __uint_as_float(a & 0xffff0000u);
+    if (SWIGLU_IN) {
+      const uint32_t b = *reinterpret_cast<const uint32_t*>(x + row * ldx + cols + c);
+      v0 = silu_fast(v0) * __uint_as_float(b << 16);
+      v1 = silu_fast(v1) * __uint_as_float(b & 0xffff0000u);
+    }
+  };
+  float m0 = 0.f, m1 = 0.f;
+#pragma unroll 4
+  for (int r = r0; r < r1; ++r) {
+    float v0, v1;
+    load(r, v0, v1);
+    m0 = fmaxf(m0, fabsf(v0));
+    m1 = fmaxf(m1, fabsf(v1));
+  }
+  const float s0 = tile_scale(m0), s1 = tile_scale(m1);
+#pragma unroll 4
+  for (int r = r0; r < r1; ++r) {
+    float v0, v1;
+    load(r, v0, v1);
+    const uint16_t pk = (uint16_t)to_e4m3(__fdiv_rn(v0, s0)) | ((uint16_t)to_e4m3(__fdiv_rn(v1, s1)) << 8);
+    *reinterpret_cast<uint16_t*>(q + (size_t)r * cols + c) = pk;
+  }
+  *reinterpret_cast<float2*>(scale + (size_t)blk * cols + c) = make_float2(s0, s1);
+}
+
+}  // namespace
+
+moe_status launch_block_table(const int32_t* offsets, int n_groups, int rows,
+                              int32_t* block_start, cudaStream_t s) {
+  block_table_kernel<<<1, 1024, 0, s>>>(offsets, n_groups, rows, block_start);
+  return cuda_check(cudaGetLastError(), "block_table launch");
+}
+
+moe_status launch_quant_128x1(const void* x, int ldx, const int32_t* src_rows, bool swiglu_in,
+                              int rows, int cols, const int32_t* offsets, int n_groups,
+                              const int32_t* block_start, uint8_t* q, float* scale,
+                              cudaStream_t s) {
+  if (rows <= 0) return MOE_OK;
+  const int G = offsets ? n_groups : 1;
+  dim3 grid((rows + 127) / 128 + G, (cols + 255) / 256), block(128);
+  auto X = static_cast<const __nv_bfloat16*>(x);
+  if (swiglu_in)
+    quant_128x1_kernel<true><<<grid, block, 0, s>>>(X, ldx, src_rows, rows, cols, offsets, G,
+                                                    block_start, q, scale);
+  else
+    quant_128x1_kernel<false><<<grid, block, 0, s>>>(X, ldx, src_rows, rows, cols, offsets, G,
+                                                     block_start, q, scale);
+  return cuda_check(cudaGetLastError(), "quant_128x1 launch");
+}
+
 }  // namespace moe

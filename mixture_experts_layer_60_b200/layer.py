@@ -4,9 +4,9 @@ MoELayer owns the layer's device state (centroids, bias, expert weights,
 FP8 copies of them) and the per-step buffers, and runs one step as
     moe_route -> [moe_quantize_1x128] -> moe_permute -> moe_expert_ffn (routed)
     -> moe_expert_ffn (each shared expert) -> moe_combine [-> moe_bias_update]
-on one CUDA stream.  For training (bf16), forward_train keeps the activations
-the backward needs and backward(dh) returns du and fills self.grad with the
-gradients of E and of every expert weight.  Every step of the layer runs in libmoe's kernels; this
+on one CUDA stream.  For training (bf16 or FP8), forward_train keeps the
+activations the backward needs and backward(dh) returns du and fills
+self.grad with the gradients of E and of every expert weight.  Every step of the layer runs in libmoe's kernels; this
 module only allocates buffers and sequences calls.
 """
 from __future__ import annotations
@@ -133,12 +133,15 @@ class MoELayer:
                     self.topk_gate, h, stream)
         return h
 
-    # -- training (bf16): forward that keeps activations, then the backward ---
+    # -- training (bf16 / FP8): forward that keeps activations, then the backward
     def _alloc_train(self, T):
         c, dev = self.cfg, self.device
         R, bf = T * c.K, torch.bfloat16
         self.a_gu = torch.empty(R, 2 * c.I, dtype=bf, device=dev)
-        self.h_s = torch.empty(c.N_s, T, c.I, dtype=bf, device=dev)
+        hdt = torch.uint8 if self.fp8 else bf
+        self.h_s = torch.empty(c.N_s, T, c.I, dtype=hdt, device=dev)
+        self.h_s_scale = torch.empty(c.N_s, T, c.I // 128, dtype=torch.float32, device=dev) \
+            if self.fp8 else None
         self.a_s = torch.empty(c.N_s, T, 2 * c.I, dtype=bf, device=dev)
         self.dy_perm = torch.empty(R, c.d, dtype=bf, device=dev)
         self.d_gate = torch.empty(T, c.K, dtype=torch.float32, device=dev)
@@ -147,19 +150,21 @@ class MoELayer:
         self.dx_perm = torch.empty(R, c.d, dtype=bf, device=dev)
         self.dx_s = torch.empty(c.N_s, T, c.d, dtype=bf, device=dev)
         self.du = torch.empty(T, c.d, dtype=bf, device=dev)
-        self.bwd_ws = _ws(moe_expert_ffn_backward_workspace_size(MOE_BF16, max(R, T), c.I), dev)
+        dt = MOE_E4M3 if self.fp8 else MOE_BF16
+        self.bwd_ws = _ws(max(moe_expert_ffn_backward_workspace_size(dt, R, c.d, c.I, c.N_r),
+                              moe_expert_ffn_backward_workspace_size(dt, T, c.d, c.I, 1)), dev)
         if not hasattr(self, "grad"):
-            self.grad = {k: torch.empty_like(self.W[k][0]) for k in
+            self.grad = {k: torch.empty(self.W[k][0].shape, dtype=bf, device=dev) for k in
                          ("W_gate_up", "W_down", "Ws_gate_up", "Ws_down")}
             self.grad["E"] = torch.empty(c.N_r, c.d, dtype=torch.float32, device=dev)
         self.T_train = T
 
     def forward_train(self, u: torch.Tensor, stream=None) -> torch.Tensor:
         """forward() that also keeps the gate/up pre-activations and h of the
-        routed and shared experts for backward().  bf16 layers only."""
+        routed and shared experts for backward().  bf16 and FP8 layers."""
         c = self.cfg
-        if c.dtype != "bf16":
-            raise ValueError("the backward is implemented for bf16 layers")
+        if c.dtype not in ("bf16", "e4m3"):
+            raise ValueError("the backward is implemented for bf16 and FP8 layers")
         T = u.shape[0]
         if T != self.T_alloc:
             self._alloc(T)
@@ -171,43 +176,79 @@ class MoELayer:
         else:
             moe_route(u, self.E, self.b, c.K, self.topk_idx, self.topk_gate, self.counts,
                       self.route_ws, stream)
-        moe_permute(u, self.topk_idx, c.N_r, self.x_perm, self.offsets, self.perm_src,
-                    self.inv_row, self.perm_ws, stream=stream)
-        wgu, wdn = self.W["W_gate_up"][0], self.W["W_down"][0]
-        moe_expert_gate_up_save(self.x_perm, self.offsets, wgu, self.h_mid, self.a_gu, stream)
-        moe_expert_down(self.h_mid, self.offsets, wdn, self.y_perm, stream=stream)
-        wsgu, wsdn = self.W["Ws_gate_up"][0], self.W["Ws_down"][0]
+        (wgu, sgu), (wdn, sdn) = self.W["W_gate_up"], self.W["W_down"]
+        (wsgu, ssgu), (wsdn, ssdn) = self.W["Ws_gate_up"], self.W["Ws_down"]
+        sl = lambda t, j: None if t is None else t[j:j + 1]
+        if self.fp8:
+            moe_quantize_1x128(u, self.u_q, self.u_s, stream)
+            moe_permute(self.u_q, self.topk_idx, c.N_r, self.x_perm, self.offsets, self.perm_src,
+                        self.inv_row, self.perm_ws, u_scale=self.u_s, x_scale=self.x_scale,
+                        stream=stream)
+            x_sh, xs_sh = self.u_q, self.u_s
+        else:
+            moe_permute(u, self.topk_idx, c.N_r, self.x_perm, self.offsets, self.perm_src,
+                        self.inv_row, self.perm_ws, stream=stream)
+            x_sh, xs_sh = u, None
+        moe_expert_gate_up_save(self.x_perm, self.offsets, wgu, self.h_mid, self.a_gu,
+                                x_scale=self.x_scale if self.fp8 else None, w_scale_gate_up=sgu,
+                                h_scale=self.h_scale, stream=stream)
+        moe_expert_down(self.h_mid, self.offsets, wdn, self.y_perm, h_scale=self.h_scale,
+                        w_scale_down=sdn, stream=stream)
         for j in range(c.N_s):
-            moe_expert_gate_up_save(u, self.shared_offsets, wsgu[j:j + 1], self.h_s[j],
-                                    self.a_s[j], stream)
+            hs_scale = None if self.h_s_scale is None else self.h_s_scale[j]
+            moe_expert_gate_up_save(x_sh, self.shared_offsets, wsgu[j:j + 1], self.h_s[j],
+                                    self.a_s[j], x_scale=xs_sh, w_scale_gate_up=sl(ssgu, j),
+                                    h_scale=hs_scale, stream=stream)
             moe_expert_down(self.h_s[j], self.shared_offsets, wsdn[j:j + 1], self.y_shared[j],
-                            stream=stream)
+                            h_scale=hs_scale, w_scale_down=sl(ssdn, j), stream=stream)
         moe_combine(u, self.y_shared if c.N_s else None, self.y_perm, self.inv_row,
                     self.topk_gate, self.h_out, stream)
         self._u = u
         return self.h_out
 
-    def backward(self, dh: torch.Tensor, stream=None) -> torch.Tensor:
+    def backward(self, dh: torch.Tensor, stream=None, ffn_events=None) -> torch.Tensor:
         """Gradients for upstream dh = dL/dh' of the last forward_train:
         returns du (overwritten by the next call) and fills self.grad
-        (E: float32; W_gate_up, W_down, Ws_gate_up, Ws_down: bf16)."""
+        (E: float32; W_gate_up, W_down, Ws_gate_up, Ws_down: bf16).
+        ffn_events=(start, end) records CUDA events around the routed expert
+        FFN backward on the same stream."""
         c, g = self.cfg, self.grad
         u = self._u
+        st = torch.cuda.current_stream() if stream is None else stream
         moe_combine_backward(dh, u, self.E, self.y_perm, self.inv_row, self.topk_idx,
                              self.topk_gate, self.dy_perm, self.d_gate, self.d_logit,
                              self.d_logit_perm, stream)
-        moe_expert_ffn_backward(self.x_perm, self.offsets, self.W["W_gate_up"][0],
-                                self.W["W_down"][0], self.a_gu, self.h_mid, self.dy_perm,
-                                self.dx_perm, g["W_gate_up"], g["W_down"], self.bwd_ws, stream)
-        wsgu, wsdn = self.W["Ws_gate_up"][0], self.W["Ws_down"][0]
+        if ffn_events:
+            ffn_events[0].record(st)
+        (wgu, sgu), (wdn, sdn) = self.W["W_gate_up"], self.W["W_down"]
+        (wsgu, ssgu), (wsdn, ssdn) = self.W["Ws_gate_up"], self.W["Ws_down"]
+        sl = lambda t, j: None if t is None else t[j:j + 1]
+        if self.fp8:
+            # the FP8 Wgrad re-quantises the layer input: rows of u through perm_src
+            x_r, x_rows, h_r = u, self.perm_src, None
+        else:
+            x_r, x_rows, h_r = self.x_perm, None, self.h_mid
+        moe_expert_ffn_backward(x_r, self.offsets, wgu, wdn, self.a_gu, h_r, self.dy_perm,
+                                self.dx_perm, g["W_gate_up"], g["W_down"], self.bwd_ws,
+                                x_rows=x_rows, w_scale_gate_up=sgu, w_scale_down=sdn,
+                                stream=stream)
+        if ffn_events:
+            ffn_events[1].record(st)
         for j in range(c.N_s):
             moe_expert_ffn_backward(u, self.shared_offsets, wsgu[j:j + 1], wsdn[j:j + 1],
-                                    self.a_s[j], self.h_s[j], dh, self.dx_s[j],
-                                    g["Ws_gate_up"][j:j + 1], g["Ws_down"][j:j + 1], self.bwd_ws,
-                                    stream)
+                                    self.a_s[j], None if self.fp8 else self.h_s[j], dh,
+                                    self.dx_s[j], g["Ws_gate_up"][j:j + 1],
+                                    g["Ws_down"][j:j + 1], self.bwd_ws,
+                                    w_scale_gate_up=sl(ssgu, j), w_scale_down=sl(ssdn, j),
+                                    stream=stream)
         moe_unpermute_backward(dh, self.dx_s if c.N_s else None, self.dx_perm, self.inv_row,
                                self.topk_idx, self.d_logit, self.E, self.du, stream)
-        moe_router_weight_grad(self.x_perm, self.d_logit_perm, self.offsets, g["E"], stream)
+        if self.fp8:
+            moe_router_weight_grad(u, self.d_logit_perm, self.offsets, g["E"],
+                                   x_rows=self.perm_src, stream=stream)
+        else:
+            moe_router_weight_grad(self.x_perm, self.d_logit_perm, self.offsets, g["E"],
+                                   stream=stream)
         return self.du
 
     def bias_update(self, counts=None, T_total=None, stream=None):

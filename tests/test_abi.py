@@ -129,20 +129,30 @@ def test_product_path_fails_loudly_without_library(monkeypatch, tmp_path):
 
 def test_backward_argument_errors(L):
     d = ctypes.c_void_p(256)
-    # gate/up with saved pre-activations: bf16 only
-    assert L.moe_expert_gate_up_save(d, d, 4, 100, 256, 256, 0, d, d, d, None) == 2
-    assert L.moe_expert_gate_up_save(d, d, 4, 100, 256, 256, 1, d, None, d, None) == 1
-    # FFN backward: bf16, d and I multiples of 256, workspace size
-    assert L.moe_expert_ffn_backward_workspace_size(1, 1000, 256) >= 1000 * 512 * 2
-    assert L.moe_expert_ffn_backward_workspace_size(0, 1000, 256) == 0
-    args = lambda dt, dd, I, ws: (d, d, 4, 100, dd, I, dt, d, d, d, d, d, d, d, d, d, ws, None)
+    # gate/up with saved pre-activations: bf16 or e4m3 (with scales)
+    assert L.moe_expert_gate_up_save(d, None, d, 4, 100, 256, 256, 0, d, None, d, None, d,
+                                     None) == 2
+    assert L.moe_expert_gate_up_save(d, None, d, 4, 100, 256, 256, 1, d, None, None, None, d,
+                                     None) == 1
+    assert L.moe_expert_gate_up_save(d, None, d, 4, 100, 256, 256, 2, d, None, d, d, d,
+                                     None) == 1
+    # FFN backward: bf16 or e4m3, d and I multiples of 256, workspace size
+    assert L.moe_expert_ffn_backward_workspace_size(1, 1000, 256, 256, 4) >= 1000 * 512 * 2
+    assert L.moe_expert_ffn_backward_workspace_size(0, 1000, 256, 256, 4) == 0
+    f8 = L.moe_expert_ffn_backward_workspace_size(2, 1000, 256, 256, 4)
+    assert f8 >= 1000 * (256 + 512 + 1024 + 256 + 256 + 512 + 256)
+    args = lambda dt, dd, I, ws: (d, None, d, 4, 100, dd, I, dt, d, None, d, None, d, d, d, d, d,
+                                  d, d, ws, None)
     assert L.moe_expert_ffn_backward(*args(0, 256, 256, 1 << 30)) == 2
     assert L.moe_expert_ffn_backward(*args(1, 256, 128, 1 << 30)) == 2
     assert L.moe_expert_ffn_backward(*args(1, 384, 256, 1 << 30)) == 2
     assert L.moe_expert_ffn_backward(*args(1, 256, 256, 64)) == 3
     assert "workspace" in _last(L)
-    assert L.moe_expert_ffn_backward(d, d, 4, 100, 256, 256, 1, d, None, d, d, d, d, d, d, d,
-                                     1 << 30, None) == 1
+    assert L.moe_expert_ffn_backward(*args(2, 256, 256, 1 << 30)) == 1   # e4m3 needs scales
+    assert L.moe_expert_ffn_backward(d, d, d, 4, 100, 256, 256, 1, d, None, d, None, d, d, d, d,
+                                     d, d, d, 1 << 30, None) == 1          # x_rows only for e4m3
+    assert L.moe_expert_ffn_backward(d, None, d, 4, 100, 256, 256, 1, d, None, None, None, d, d,
+                                     d, d, d, d, d, 1 << 30, None) == 1
     # per-token backward kernels
     assert L.moe_combine_backward(d, d, d, d, d, d, d, 2, 8, 64, 4, d, d, d, d, None) == 2
     assert L.moe_combine_backward(d, d, d, d, d, d, d, 1, 8, 64, 17, d, d, d, d, None) == 2
@@ -150,5 +160,8 @@ def test_backward_argument_errors(L):
     assert L.moe_combine_backward(d, d, None, d, d, d, d, 1, 8, 64, 4, d, d, d, d, None) == 1
     assert L.moe_unpermute_backward(d, None, 1, d, d, d, d, d, 1, 8, 64, 4, d, None) == 1
     assert L.moe_unpermute_backward(d, d, 1, d, d, d, d, d, 2, 8, 64, 4, d, None) == 2
-    assert L.moe_router_weight_grad(d, d, d, 2, 16, 64, d, None) == 2
-    assert L.moe_router_weight_grad(d, d, None, 1, 16, 64, d, None) == 1
+    assert L.moe_router_weight_grad(d, None, d, d, 2, 16, 64, d, None) == 2
+    assert L.moe_router_weight_grad(d, None, d, None, 1, 16, 64, d, None) == 1
+    # FP8 Wgrad quantiser
+    assert L.moe_quantize_128x1_grouped(d, 100, 100, d, 4, d, d, d, None) == 2
+    assert L.moe_quantize_128x1_grouped(d, 100, 128, d, 4, d, d, None, None) == 1

@@ -53,8 +53,8 @@ def test_expert_ffn_backward_ragged_groups(sizes):
     dx = torch.full((rows, d), float("nan"), dtype=torch.bfloat16, device="cuda")
     dWgu = torch.full_like(Wgu, float("nan"))
     dWdn = torch.full_like(Wdn, float("nan"))
-    ws = torch.empty(moe_expert_ffn_backward_workspace_size(MOE_BF16, rows, I), dtype=torch.uint8,
-                     device="cuda")
+    ws = torch.empty(moe_expert_ffn_backward_workspace_size(MOE_BF16, rows, d, I, G),
+                     dtype=torch.uint8, device="cuda")
     moe_expert_ffn_backward(x, off, Wgu, Wdn, a_gu, h, dy, dx, dWgu, dWdn, ws)
     torch.cuda.synchronize()
     # the saving gate/up gives the same h as the plain one, bit for bit
