@@ -386,7 +386,7 @@ inline bool al16(const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 == 
 // the two Dgrads and two Wgrads and their scales (see fp8_bwd_layout).
 struct Fp8BwdLayout {
   size_t dy_q, dy_s, dA_q, dA_s, dA_bf, blk, dyT_q, dyT_s, hT_q, hT_s, dAT_q, dAT_s, xT_q, xT_s,
-      total;
+      tail, total;
 };
 Fp8BwdLayout fp8_bwd_layout(int rows, int d, int I, int G) {
   Fp8BwdLayout L;
@@ -407,13 +407,16 @@ Fp8BwdLayout fp8_bwd_layout(int rows, int d, int I, int G) {
   L.dAT_s = take(nb * 2 * I * 4);
   L.xT_q = take(R * d);
   L.xT_s = take(nb * d * 4);
+  L.tail = take(wgrad_tail_bytes((size_t)(d > 2 * I ? d : 2 * I), 128, G));   // Wgrad A tails
   L.total = o;
   return L;
 }
 
 size_t ffn_bwd_ws(moe_dtype dt, int rows, int d, int I, int G) {
   if (rows <= 0 || I <= 0 || d <= 0 || G <= 0) return 0;
-  if (dt == MOE_BF16) return align_up((size_t)rows * 2 * I * 2, 256);
+  if (dt == MOE_BF16)   // dA, then the Wgrad A operand's tail blocks
+    return align_up((size_t)rows * 2 * I * 2, 256) +
+           wgrad_tail_bytes((size_t)(d > 2 * I ? d : 2 * I) * 2, 64, G);
   if (dt == MOE_E4M3) return fp8_bwd_layout(rows, d, I, G).total;
   return 0;
 }
@@ -539,8 +542,9 @@ moe_status moe_expert_ffn_backward(const void* x, const int32_t* x_rows, const i
   MOE_TRY(check_device());
   if (dt == MOE_BF16) {
     void* dA = workspace;
+    void* tail = static_cast<uint8_t*>(workspace) + align_up((size_t)rows * 2 * I * 2, 256);
     // Wgrad of the down projection needs only dy and h
-    MOE_TRY(launch_wgrad_gemm(dy, d, h, I, offsets, n_groups, rows, dW_down, s));
+    MOE_TRY(launch_wgrad_gemm(dy, d, h, I, offsets, n_groups, rows, tail, dW_down, s));
     // Dgrad of the down projection fused with the SwiGLU backward -> dA
     MOE_TRY(launch_ws_gemm_ex(dy, W_down, 0, offsets, n_groups, rows, I, d, WS_DSWIGLU, true, dA,
                               2 * I, const_cast<void*>(a_gu), 2 * I, s));
@@ -548,7 +552,7 @@ moe_status moe_expert_ffn_backward(const void* x, const int32_t* x_rows, const i
     MOE_TRY(launch_ws_gemm_ex(dA, W_gate_up, 0, offsets, n_groups, rows, d, 2 * I, WS_STORE, true,
                               dx, d, nullptr, 0, s));
     // Wgrad of the gate/up projection
-    return launch_wgrad_gemm(dA, 2 * I, x, d, offsets, n_groups, rows, dW_gate_up, s);
+    return launch_wgrad_gemm(dA, 2 * I, x, d, offsets, n_groups, rows, tail, dW_gate_up, s);
   }
   // ---- FP8 (E4M3) backward
   const Fp8BwdLayout L = fp8_bwd_layout(rows, d, I, n_groups);
@@ -573,13 +577,13 @@ moe_status moe_expert_ffn_backward(const void* x, const int32_t* x_rows, const i
   MOE_TRY(launch_quant_128x1(a_gu, 2 * I, nullptr, true, rows, I, offsets, n_groups, blk,
                              w + L.hT_q, f32(L.hT_s), s));
   MOE_TRY(launch_wgrad_fp8(w + L.dyT_q, f32(L.dyT_s), d, w + L.hT_q, f32(L.hT_s), I, offsets,
-                           n_groups, rows, blk, dW_down, s));
+                           n_groups, rows, blk, w + L.tail, dW_down, s));
   MOE_TRY(launch_quant_128x1(w + L.dA_bf, 2 * I, nullptr, false, rows, 2 * I, offsets, n_groups,
                              blk, w + L.dAT_q, f32(L.dAT_s), s));
   MOE_TRY(launch_quant_128x1(x, d, x_rows, false, rows, d, offsets, n_groups, blk, w + L.xT_q,
                              f32(L.xT_s), s));
   return launch_wgrad_fp8(w + L.dAT_q, f32(L.dAT_s), 2 * I, w + L.xT_q, f32(L.xT_s), d, offsets,
-                          n_groups, rows, blk, dW_gate_up, s);
+                          n_groups, rows, blk, w + L.tail, dW_gate_up, s);
 }
 
 moe_status moe_unpermute_backward(const void* dh_out, const void* dx_shared, int N_s,

@@ -10,13 +10,14 @@
 // K step, 4 shared-memory stages of 48 KB (A: two [64 tok][64 m] TMA boxes,
 // B: four [64 tok][64 n] boxes, 128-byte swizzle), two TMEM accumulators of
 // 256 columns so the epilogue of one tile overlaps the MMAs of the next.
-// The last K step of a group is ragged: its A rows past the group's end are
-// zeroed in shared memory (they hold the next expert's tokens) before the
-// MMAs read them, and only ceil(valid/16) MMAs are issued.  A group with no
-// tokens gets C_g = 0 from the epilogue without touching TMEM.
+// The last K step of a group is ragged: its A rows come from a side buffer
+// of per-group tail blocks written beforehand by launch_wgrad_tails (rows
+// past the group's end are zero there, so the next expert's tokens never
+// enter), and only ceil(valid/16) MMAs are issued.  A group with no tokens
+// gets C_g = 0 from the epilogue without touching TMEM.
 //
-// Roles: warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer (the whole
-// warp zeroes ragged rows, one lane issues), warps 2-17 epilogue (warp w
+// Roles: warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer, warps 2-17
+// epilogue (warp w
 // reads TMEM lanes 32*(w%4).. = C rows and one 64-column quarter of the
 // tile; each 32x32 block is converted to bf16 into a 2 KB shared-memory
 // patch laid out as a 64-byte-swizzled [32 rows][32 cols] TMA box and written
@@ -62,8 +63,8 @@ struct WgParams {
 
 __device__ __forceinline__ void group_rows(const WgParams& p, int g, int& r0, int& cnt) {
   if (p.offsets) {
-    r0 = p.offsets[g];
-    cnt = p.offsets[g + 1] - r0;
+    r0 = __ldg(p.offsets + g);
+    cnt = __ldg(p.offsets + g + 1) - r0;
   } else {
     r0 = 0;
     cnt = p.rows;
@@ -78,7 +79,8 @@ __device__ __forceinline__ void raise_abort(volatile int* abort, int* err) {
 __global__ void __launch_bounds__(kThreads, 1)
     wgrad_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                       const __grid_constant__ CUtensorMap tmB,
-                      const __grid_constant__ CUtensorMap tmC, const WgParams p) {
+                      const __grid_constant__ CUtensorMap tmC,
+                      const __grid_constant__ CUtensorMap tmAt, const WgParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -136,8 +138,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* a_dst = smem + stage * STAGE_BYTES;
           uint8_t* b_dst = a_dst + A_BYTES;
           const int row = r0 + kb * BK;
-          // one TMA per operand: 2 (A) / 4 (B) consecutive [64 tok][64 col] tiles
-          tma_load_3d(a_dst, &tmA, 0, row, mt * (BM / 64), &full[stage]);
+          // one TMA per operand: 2 (A) / 4 (B) consecutive [64 tok][64 col] tiles;
+          // a group's last block of A comes from its zero-padded tail block
+          if (kb == nkb - 1)
+            tma_load_3d(a_dst, &tmAt, 0, g * BK, mt * (BM / 64), &full[stage]);
+          else
+            tma_load_3d(a_dst, &tmA, 0, row, mt * (BM / 64), &full[stage]);
           tma_load_3d(b_dst, &tmB, 0, row, nt * (BN / 64), &full[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
@@ -177,17 +183,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* a_st = smem + stage * STAGE_BYTES;
         const int valid = min(BK, cnt - kb * BK);
         const int nks = (valid + 15) / 16;
-        if (valid < nks * 16) {
-          // rows [valid, nks*16) of both A boxes belong to the next group: zero them
-          const int zrows = nks * 16 - valid;
-          const int chunks = zrows * 8;                   // 16-byte chunks per box
-          for (int i = lane; i < 2 * chunks; i += 32) {
-            const int box = i / chunks, rem = i - box * chunks;
-            uint8_t* dst = a_st + box * BOX_BYTES + (valid + (rem >> 3)) * 128 + (rem & 7) * 16;
-            *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
-          }
-          fence_proxy_async_smem();
-        }
         __syncwarp();
         tc_fence_after();
         if (lane == 0) {
@@ -292,8 +287,47 @@ moe_status make_tmap_col_blocks(CUtensorMap* tm, const void* base, CUtensorMapDa
                                 int elem_bytes, uint64_t cols, uint64_t rows, uint32_t bc,
                                 uint32_t box_rows, uint32_t box_blocks);
 
+namespace {
+
+// T[g][i] = row (start of g's last block) + i of A if it lies inside group g, else 0.
+__global__ void __launch_bounds__(256) wgrad_tails_kernel(const uint4* __restrict__ A,
+                                                          int row_vec, int block_rows,
+                                                          const int32_t* __restrict__ offsets,
+                                                          int rows, uint4* __restrict__ T) {
+  const int g = blockIdx.x, i = blockIdx.y;
+  const int r0 = offsets ? offsets[g] : 0;
+  const int r1 = offsets ? offsets[g + 1] : rows;
+  const int cnt = r1 - r0;
+  if (cnt <= 0) return;
+  const int row = r0 + ((cnt - 1) / block_rows) * block_rows + i;
+  uint4* dst = T + ((size_t)g * block_rows + i) * row_vec;
+  if (row < r1) {
+    const uint4* src = A + (size_t)row * row_vec;
+    for (int c = threadIdx.x; c < row_vec; c += blockDim.x) dst[c] = src[c];
+  } else {
+    for (int c = threadIdx.x; c < row_vec; c += blockDim.x) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+}  // namespace
+
+moe_status launch_wgrad_tails(const void* A, size_t row_bytes, int block_rows,
+                              const int32_t* offsets, int n_groups, int rows, void* T,
+                              cudaStream_t s) {
+  const int G = offsets ? n_groups : 1;
+  if (G <= 0 || rows <= 0) return MOE_OK;
+  dim3 grid(G, block_rows);
+  wgrad_tails_kernel<<<grid, 256, 0, s>>>(static_cast<const uint4*>(A), (int)(row_bytes / 16),
+                                          block_rows, offsets, rows, static_cast<uint4*>(T));
+  return cuda_check(cudaGetLastError(), "wgrad tails launch");
+}
+
+size_t wgrad_tail_bytes(size_t row_bytes, int block_rows, int n_groups) {
+  return align_up((size_t)n_groups * block_rows * row_bytes, 256);
+}
+
 moe_status launch_wgrad_gemm(const void* A, int M, const void* B, int N, const int32_t* offsets,
-                             int n_groups, int rows, void* C, cudaStream_t s) {
+                             int n_groups, int rows, void* A_tail, void* C, cudaStream_t s) {
   const int G = offsets ? n_groups : 1;
   if (G <= 0) return MOE_OK;
   if (M % BM || N % BN)
@@ -303,9 +337,14 @@ moe_status launch_wgrad_gemm(const void* A, int M, const void* B, int N, const i
     // every group is empty: C = 0
     return cuda_check(cudaMemsetAsync(C, 0, (size_t)G * M * N * 2, s), "wgrad zero fill");
   }
-  CUtensorMap tmA, tmB, tmC;
-  moe_status st = make_tmap_col_blocks(&tmA, A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, rows, 64,
-                                       BK, BM / 64);
+  // the A operand's tail blocks: [G * BK rows][M] (launch_wgrad_tails)
+  moe_status st = launch_wgrad_tails(A, (size_t)M * 2, BK, offsets, G, rows, A_tail, s);
+  if (st != MOE_OK) return st;
+  CUtensorMap tmA, tmB, tmC, tmAt;
+  st = make_tmap_col_blocks(&tmA, A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, rows, 64, BK, BM / 64);
+  if (st != MOE_OK) return st;
+  st = make_tmap_col_blocks(&tmAt, A_tail, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M,
+                            (uint64_t)G * BK, 64, BK, BM / 64);
   if (st != MOE_OK) return st;
   st = make_tmap_col_blocks(&tmB, B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, rows, 64, BK, BN / 64);
   if (st != MOE_OK) return st;
@@ -332,7 +371,7 @@ moe_status launch_wgrad_gemm(const void* A, int M, const void* B, int N, const i
   const long long tiles = (long long)G * (M / BM) * (N / BN);
   int grid = sm_count();
   if (tiles < grid) grid = (int)tiles;
-  wgrad_gemm_kernel<<<grid, kThreads, SMEM_ALLOC, s>>>(tmA, tmB, tmC, p);
+  wgrad_gemm_kernel<<<grid, kThreads, SMEM_ALLOC, s>>>(tmA, tmB, tmC, tmAt, p);
   return cuda_check(cudaGetLastError(), "wgrad gemm launch");
 }
 

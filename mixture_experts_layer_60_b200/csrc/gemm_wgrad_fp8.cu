@@ -10,14 +10,16 @@
 //
 // Tile 128 x 256 outputs; each shared-memory stage is one 128-row block
 // (A: one [128 tok][128 m] box, B: two [128 tok][128 n] boxes, 128-byte
-// swizzle, 48 KB), 4 stages.  The MMA warp writes each block's partial
-// product into one of two TMEM buffers (tcgen05.mma kind::f8f6f4, K = 32 per
-// instruction; the rows of a ragged last block past the expert's end are
-// zeroed in shared memory first and only ceil(valid/32) MMAs are issued); 16
-// epilogue warps read it back (warp w: TMEM lanes 32*(w%4).. = C rows, 64
-// columns), add P * sa[b, m] * sb[b, n] into float32 registers with paired
-// FMAs, and after the expert's last block write bf16 through a 64-byte-
-// swizzled shared-memory patch and TMA stores.  Waits are bounded (1 s).
+// swizzle, 48 KB), 4 stages; with every stage the producer also copies the
+// block's scales sa[b, m0:m0+128] and sb[b, n0:n0+256] into a ring of 6
+// scale slots (bulk copies on their own barriers).  The MMA warp writes each
+// block's partial product into one of two TMEM buffers (tcgen05.mma
+// kind::f8f6f4, K = 32 per instruction; the A rows of an expert's ragged last
+// block come from its zero-padded tail block, and only ceil(valid/32) MMAs are
+// issued); 16 epilogue warps read it back (warp w: TMEM lanes
+// 32*(w%4).. = C rows, 64 columns), add P * (sa * sb) into float32 registers
+// with paired multiplies and FMAs, and after the expert's last block write
+// bf16 rows to global memory.  Waits are bounded (1 s).
 #include "launch.h"
 #include "sm100.cuh"
 
@@ -50,9 +52,11 @@ constexpr int BOX_BYTES = 128 * BK;            // [128 tok][128 e4m3]: 16 KB
 constexpr int A_BYTES = BOX_BYTES;
 constexpr int B_BYTES = 2 * BOX_BYTES;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int OFF_PATCH = STAGES * STAGE_BYTES;
-constexpr int OFF_BAR = OFF_PATCH + kEpiWarps * 2048;
-constexpr int N_BARS = 2 * STAGES + 5;
+constexpr int SSLOTS = 6;                       // scale ring: sa [128] + sb [256] float32 per block
+constexpr int SLOT_BYTES = (BM + BN) * 4;
+constexpr int OFF_SCALE = STAGES * STAGE_BYTES;
+constexpr int OFF_BAR = OFF_SCALE + SSLOTS * SLOT_BYTES;
+constexpr int N_BARS = 2 * STAGES + 5 + 2 * SSLOTS;
 constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16;
 constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
@@ -74,8 +78,8 @@ struct Wg8Params {
 
 __device__ __forceinline__ void group_rows(const Wg8Params& p, int g, int& r0, int& cnt) {
   if (p.offsets) {
-    r0 = p.offsets[g];
-    cnt = p.offsets[g + 1] - r0;
+    r0 = __ldg(p.offsets + g);
+    cnt = __ldg(p.offsets + g + 1) - r0;
   } else {
     r0 = 0;
     cnt = p.rows;
@@ -95,6 +99,12 @@ __device__ __forceinline__ uint64_t f2_pack(float a, float b) {
 __device__ __forceinline__ void f2_unpack(uint64_t v, float& a, float& b) {
   asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
 }
+// (a0, a1) * (b0, b1), elementwise, rounded like two fmul
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
 // c += (x0, x1) * s2 with x0, x1 the raw bits of two float32 TMEM words
 __device__ __forceinline__ uint64_t fma2_bits(uint32_t x0, uint32_t x1, uint64_t s2, uint64_t c) {
   asm("{\n\t.reg .b64 t;\n\tmov.b64 t, {%1, %2};\n\tfma.rn.f32x2 %0, t, %3, %0;\n\t}"
@@ -103,10 +113,12 @@ __device__ __forceinline__ uint64_t fma2_bits(uint32_t x0, uint32_t x1, uint64_t
   return c;
 }
 
+// 18 warps put 5 on two of the SM's four sub-partitions, whose 16K-register
+// files then cap a thread at 96 registers (__launch_bounds__ below).
 __global__ void __launch_bounds__(kThreads, 1)
     wgrad_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
                      const __grid_constant__ CUtensorMap tmB,
-                     const __grid_constant__ CUtensorMap tmC, const Wg8Params p) {
+                     const __grid_constant__ CUtensorMap tmAt, const Wg8Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -115,6 +127,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* pfull = empty + STAGES;      // [2] partial product ready
   uint64_t* pempty = pfull + 2;          // [2] partial product read by the epilogue
   uint64_t* mma_done = pempty + 2;
+  uint64_t* sfull = mma_done + 1;        // [SSLOTS] scales landed
+  uint64_t* sempty = sfull + SSLOTS;     // [SSLOTS] scales read by the epilogue
+  float* scales = reinterpret_cast<float*>(smem + OFF_SCALE);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
 
@@ -128,6 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     for (int b = 0; b < 2; ++b) { mbar_init(&pfull[b], 1); mbar_init(&pempty[b], 32 * kEpiWarps); }
     mbar_init(mma_done, 1);
+    for (int i = 0; i < SSLOTS; ++i) { mbar_init(&sfull[i], 1); mbar_init(&sempty[i], 32 * kEpiWarps); }
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
@@ -145,8 +161,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
+      int stage = 0, ss = 0;
+      uint32_t phase = 0, sphase = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
         const int g = t / per_group, loc = t - g * per_group;
@@ -154,7 +170,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         int r0, cnt;
         group_rows(p, g, r0, cnt);
         const int nkb = (cnt + BK - 1) / BK;
+        const int blk0 = nkb > 0 ? p.block_start[g] : 0;
         for (int kb = 0; kb < nkb; ++kb) {
+          // this block's scales into the next slot of the ring
+          if (!mbar_wait_bounded(&sempty[ss], sphase ^ 1, abort_flag, kWaitNs)) {
+            raise_abort(abort_flag, p.err);
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&sfull[ss], SLOT_BYTES);
+          float* sl = scales + ss * (BM + BN);
+          bulk_load(sl, p.sa + (size_t)(blk0 + kb) * p.M + mt * BM, BM * 4, &sfull[ss]);
+          bulk_load(sl + BM, p.sb + (size_t)(blk0 + kb) * p.N + nt * BN, BN * 4, &sfull[ss]);
+          if (++ss == SSLOTS) { ss = 0; sphase ^= 1; }
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, kWaitNs)) {
             raise_abort(abort_flag, p.err);
             ok = false;
@@ -163,13 +191,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
           uint8_t* a_dst = smem + stage * STAGE_BYTES;
           const int row = r0 + kb * BK;
-          tma_load_2d(a_dst, &tmA, mt * BM, row, &full[stage]);
+          if (kb == nkb - 1)   // the expert's last block of A: its zero-padded tail block
+            tma_load_2d(a_dst, &tmAt, mt * BM, g * BK, &full[stage]);
+          else
+            tma_load_2d(a_dst, &tmA, mt * BM, row, &full[stage]);
           tma_load_3d(a_dst + A_BYTES, &tmB, 0, row, nt * (BN / 128), &full[stage]);   // 2 tiles
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
       for (int s = 0; s < STAGES; ++s)
         mbar_wait_bounded(&full[s], ((s < stage) ? phase : phase ^ 1), nullptr, kWaitNs);
+      for (int i = 0; i < SSLOTS; ++i)
+        mbar_wait_bounded(&sfull[i], ((i < ss) ? sphase : sphase ^ 1), nullptr, kWaitNs);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
@@ -193,15 +226,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* a_st = smem + stage * STAGE_BYTES;
         const int valid = min(BK, cnt - kb * BK);
         const int nks = (valid + 31) / 32;
-        if (valid < nks * 32) {
-          // rows [valid, nks*32) of the A box belong to the next expert: zero them
-          const int chunks = (nks * 32 - valid) * 8;     // 16-byte chunks
-          for (int i = lane; i < chunks; i += 32) {
-            uint8_t* dst = a_st + (valid + (i >> 3)) * 128 + (i & 7) * 16;
-            *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
-          }
-          fence_proxy_async_smem();
-        }
         __syncwarp();
         tc_fence_after();
         if (lane == 0) {
@@ -227,9 +251,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------------- epilogue
     const int q = warp & 3;                       // TMEM lane quarter = C rows q*32..
     const int cq = (warp - 2) >> 2;               // 64-column quarter of the tile
-    uint4* patch = reinterpret_cast<uint4*>(smem + OFF_PATCH + (warp - 2) * 2048);   // [32][4]
-    int pb = 0;
-    uint32_t pphase = 0;
+    int pb = 0, ss = 0;
+    uint32_t pphase = 0, sphase = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
       const int g = t / per_group, loc = t - g * per_group;
@@ -238,78 +261,72 @@ __global__ void __launch_bounds__(kThreads, 1)
       group_rows(p, g, r0, cnt);
       const int m = mt * BM + q * 32 + lane;
       const int n0 = nt * BN + cq * 64;
+      uint4* dst = reinterpret_cast<uint4*>(p.C(g, m, n0));
       if (cnt <= 0) {
-        uint4* d4 = reinterpret_cast<uint4*>(p.C(g, m, n0));
 #pragma unroll
-        for (int i = 0; i < 8; ++i) d4[i] = make_uint4(0u, 0u, 0u, 0u);
+        for (int i = 0; i < 8; ++i) dst[i] = make_uint4(0u, 0u, 0u, 0u);
         continue;
       }
       uint64_t acc2[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) acc2[i] = 0ull;
       const int nkb = (cnt + BK - 1) / BK;
-      const int blk0 = p.block_start[g];
       for (int kb = 0; kb < nkb; ++kb) {
-        const float sa = p.sa[(size_t)(blk0 + kb) * p.M + m];
-        const float* sbr = p.sb + (size_t)(blk0 + kb) * p.N + n0;
-        const bool got = mbar_wait_bounded(&pfull[pb], pphase, abort_flag, kWaitNs);
+        const bool gs = mbar_wait_bounded(&sfull[ss], sphase, abort_flag, kWaitNs);
+        const bool got = gs && mbar_wait_bounded(&pfull[pb], pphase, abort_flag, kWaitNs);
         if (!__all_sync(0xffffffffu, got)) {
           if (lane == 0) raise_abort(abort_flag, p.err);
           ok = false;
           break;
         }
         tc_fence_after();
+        const float* sl = scales + ss * (BM + BN);
+        const float sa = sl[q * 32 + lane];
+        const uint64_t sa2 = f2_pack(sa, sa);
+        const uint2* sb2 = reinterpret_cast<const uint2*>(sl + BM + cq * 64);   // column pairs
         const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + pb * BN + cq * 64;
+        // eight 8-column pieces: two TMEM loads in flight per wait, few live registers
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[16];
-          tmem_ld_32x32b_x16(tb + c * 16, r);
+        for (int c = 0; c < 8; c += 2) {
+          uint32_t r[2][8];
+          tmem_ld_32x32b_x8(tb + c * 8, r[0]);
+          tmem_ld_32x32b_x8(tb + c * 8 + 8, r[1]);
           tmem_wait_ld();
-          if (c == 3) {
+          if (c == 6) {
             tc_fence_before();
             mbar_arrive(&pempty[pb]);   // partial read: the MMA may overwrite it
           }
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const float4 s4 = *reinterpret_cast<const float4*>(sbr + c * 16 + v * 4);
-            acc2[c * 8 + 2 * v] = fma2_bits(r[4 * v], r[4 * v + 1], f2_pack(sa * s4.x, sa * s4.y),
-                                             acc2[c * 8 + 2 * v]);
-            acc2[c * 8 + 2 * v + 1] = fma2_bits(r[4 * v + 2], r[4 * v + 3],
-                                                f2_pack(sa * s4.z, sa * s4.w),
-                                                acc2[c * 8 + 2 * v + 1]);
+          for (int h = 0; h < 2; ++h) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const uint2 sbv = sb2[(c + h) * 4 + v];               // broadcast read
+              const uint64_t s2 = mul2(sa2, (uint64_t)sbv.x | ((uint64_t)sbv.y << 32));
+              acc2[(c + h) * 4 + v] =
+                  fma2_bits(r[h][2 * v], r[h][2 * v + 1], s2, acc2[(c + h) * 4 + v]);
+            }
           }
         }
+        mbar_arrive(&sempty[ss]);       // this block's scales are no longer read
         if (++pb == 2) { pb = 0; pphase ^= 1; }
+        if (++ss == SSLOTS) { ss = 0; sphase ^= 1; }
       }
       if (!ok) break;
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        if (lane == 0) tma_store_wait_read_all();
-        __syncwarp();
-        // row `lane` (64 bytes) into the 64-byte-swizzled patch: slot i at i ^ ((lane >> 1) & 3)
+      for (int i = 0; i < 8; ++i) {
+        uint32_t w4[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          uint32_t w4[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            float x0, x1;
-            f2_unpack(acc2[c * 16 + 4 * i + k], x0, x1);
-            __nv_bfloat162 pr = __floats2bfloat162_rn(x0, x1);
-            w4[k] = *reinterpret_cast<uint32_t*>(&pr);
-          }
-          patch[lane * 4 + (i ^ ((lane >> 1) & 3))] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        for (int k = 0; k < 4; ++k) {
+          float x0, x1;
+          f2_unpack(acc2[4 * i + k], x0, x1);
+          __nv_bfloat162 pr = __floats2bfloat162_rn(x0, x1);
+          w4[k] = *reinterpret_cast<uint32_t*>(&pr);
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_2d(&tmC, patch, n0 + c * 32, g * p.M + mt * BM + q * 32);
-          tma_store_commit();
-        }
+        dst[i] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
       }
     }
   }
 
-  if (warp >= 2 && lane == 0) tma_store_wait_all();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -320,9 +337,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
+moe_status launch_wgrad_tails(const void* A, size_t row_bytes, int block_rows,
+                              const int32_t* offsets, int n_groups, int rows, void* T,
+                              cudaStream_t s);
+
 moe_status launch_wgrad_fp8(const void* qa, const float* sa, int M, const void* qb,
                             const float* sb, int N, const int32_t* offsets, int n_groups,
-                            int rows, const int32_t* block_start, void* C, cudaStream_t s) {
+                            int rows, const int32_t* block_start, void* qa_tail, void* C,
+                            cudaStream_t s) {
   const int G = offsets ? n_groups : 1;
   if (G <= 0) return MOE_OK;
   if (M % BM || N % BN)
@@ -330,13 +352,14 @@ moe_status launch_wgrad_fp8(const void* qa, const float* sa, int M, const void* 
                 BM, N, BN);
   if (rows <= 0)
     return cuda_check(cudaMemsetAsync(C, 0, (size_t)G * M * N * 2, s), "fp8 wgrad zero fill");
-  CUtensorMap tmA, tmB, tmC;
-  moe_status st = make_tmap_2d(&tmA, qa, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, rows, 128, BK);
+  moe_status st = launch_wgrad_tails(qa, (size_t)M, BK, offsets, G, rows, qa_tail, s);
+  if (st != MOE_OK) return st;
+  CUtensorMap tmA, tmB, tmAt;
+  st = make_tmap_2d(&tmA, qa, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, rows, 128, BK);
+  if (st != MOE_OK) return st;
+  st = make_tmap_2d(&tmAt, qa_tail, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, (uint64_t)G * BK, 128, BK);
   if (st != MOE_OK) return st;
   st = make_tmap_col_blocks(&tmB, qb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, rows, 128, BK, BN / 128);
-  if (st != MOE_OK) return st;
-  st = make_tmap_2d_swz(&tmC, C, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, (uint64_t)G * M, 32, 32,
-                        CU_TENSOR_MAP_SWIZZLE_64B);
   if (st != MOE_OK) return st;
   static bool attr_set = false;
   if (!attr_set) {
@@ -360,7 +383,7 @@ moe_status launch_wgrad_fp8(const void* qa, const float* sa, int M, const void* 
   const long long tiles = (long long)G * (M / BM) * (N / BN);
   int grid = sm_count();
   if (tiles < grid) grid = (int)tiles;
-  wgrad_fp8_kernel<<<grid, kThreads, SMEM_ALLOC, s>>>(tmA, tmB, tmC, p);
+  wgrad_fp8_kernel<<<grid, kThreads, SMEM_ALLOC, s>>>(tmA, tmB, tmAt, p);
   return cuda_check(cudaGetLastError(), "fp8 wgrad launch");
 }
 

@@ -67,14 +67,23 @@ moe_status launch_ws_gemm_ex(const void* X, const void* W, int b_rows_per_group,
 
 // gemm_wgrad.cu --------------------------------------------------------------
 // C[g] [M, N] = sum over the rows r of group g of A[r, :]^T B[r, :] (bf16 in and out).
+// A_tail: scratch of wgrad_tail_bytes(M * 2, 64, groups) bytes for the groups'
+// zero-padded last 64-row blocks of A.
 moe_status launch_wgrad_gemm(const void* A, int M, const void* B, int N, const int32_t* offsets,
-                             int n_groups, int rows, void* C, cudaStream_t s);
+                             int n_groups, int rows, void* A_tail, void* C, cudaStream_t s);
+// T[g] = the last block_rows-row block of group g of A (rows past the group zeroed).
+moe_status launch_wgrad_tails(const void* A, size_t row_bytes, int block_rows,
+                              const int32_t* offsets, int n_groups, int rows, void* T,
+                              cudaStream_t s);
+size_t wgrad_tail_bytes(size_t row_bytes, int block_rows, int n_groups);
 
 // gemm_wgrad_fp8.cu ----------------------------------------------------------
 // C[g] [M, N] = sum over g's 128-row blocks b of (qa_b^T qb_b) * sa[b, m] * sb[b, n].
+// qa_tail: scratch of wgrad_tail_bytes(M, 128, groups) bytes.
 moe_status launch_wgrad_fp8(const void* qa, const float* sa, int M, const void* qb,
                             const float* sb, int N, const int32_t* offsets, int n_groups,
-                            int rows, const int32_t* block_start, void* C, cudaStream_t s);
+                            int rows, const int32_t* block_start, void* qa_tail, void* C,
+                            cudaStream_t s);
 
 // gemm_fp8.cu ----------------------------------------------------------------
 moe_status launch_fp8_gemm(const void* A, const float* a_scale, const void* B,
