@@ -379,6 +379,53 @@ moe_status moe_router_weight_grad(const void* x, const int32_t* x_rows,
                                   const float* d_logit_perm, const int32_t* offsets,
                                   moe_dtype dt, int N_r, int d, float* dE, void* stream);
 
+/* ========================================================================
+ * Expert parallelism ("DeepSeek V3 & R1 論文研究", sections DeepSeekMoE and
+ * Cross-Node All-to-All: routed experts spread over devices, tokens sent to
+ * the devices of their experts and the outputs returned).  W ranks (W <= 8,
+ * N_r % W == 0), E_loc = N_r / W experts per rank, expert e on rank e/E_loc.
+ * counts_all [W, N_r] int32: every rank's per-expert load (moe_route counts,
+ * all-gathered).  Rank d receives its rows grouped by local expert j,
+ * inside by source rank, inside by the source's token order:
+ *   recv_offsets[j] = sum_{j'<j} sum_s counts_all[s][d*E_loc + j']
+ * so the local grouped FFN runs on (recv_rows, recv_offsets, E_loc groups).
+ * A step on rank s: moe_route, moe_permute (for offsets / inv_row),
+ * moe_ep_plan, moe_ep_dispatch, [every rank's rows have arrived],
+ * moe_expert_ffn on the received rows, moe_ep_return, [every rank's outputs
+ * have arrived], moe_combine with y_perm = the return buffer.  The result
+ * equals the single-device layer's bit for bit.  Destination pointers may
+ * be another GPU's memory (peer access, e.g. symmetric memory); the calls
+ * only store to them.  Row positions outside a buffer's capacity are never
+ * written: the row is skipped and moe_device_status reports it.
+ * ======================================================================== */
+
+/* moe_ep_plan - this rank's receive offsets recv_offsets [E_loc+1] and, for
+ * every expert e, send_base [N_r]: where this rank's first row of expert e
+ * lands in the receive buffer of rank e/E_loc.  counts_all device int32. */
+moe_status moe_ep_plan(const int32_t* counts_all, int W, int rank, int N_r,
+                       int32_t* recv_offsets, int32_t* send_base, void* stream);
+
+/* moe_ep_dispatch - sends row (t, k) of u (this rank's tokens [T, d], dt
+ * MOE_F32 or MOE_BF16) to rank d = topk_idx[t,k]/E_loc, at position
+ * send_base[e] + inv_row[t,k] - offsets[e] of recv_rows[d] ([recv_cap, d]
+ * rows of dt), and writes the tag (rank, inv_row[t,k]) at the same position
+ * of recv_tags[d] ([recv_cap] x int32 pairs).  recv_rows / recv_tags: host
+ * arrays of W device pointers.  topk_idx, inv_row, offsets: this rank's
+ * moe_route / moe_permute outputs. */
+moe_status moe_ep_dispatch(const void* u, moe_dtype dt, int T, int d, int K,
+                           const int32_t* topk_idx, const int32_t* inv_row,
+                           const int32_t* offsets, const int32_t* send_base, int N_r, int W,
+                           int rank, void* const* recv_rows, void* const* recv_tags,
+                           long long recv_cap, void* stream);
+
+/* moe_ep_return - writes row p of y ([recv_cap, d] dt, the expert outputs of
+ * the received rows; p < recv_offsets[E_loc]) to row tag.y of ret_rows[tag.x]
+ * ([ret_cap, d] dt on every rank: its grouped positions), tag = recv_tags[p].
+ * n_rows: device pointer to the received row count (recv_offsets + E_loc). */
+moe_status moe_ep_return(const void* y, moe_dtype dt, const void* recv_tags,
+                         const int32_t* n_rows, long long recv_cap, int d, int W,
+                         void* const* ret_rows, long long ret_cap, void* stream);
+
 /* ------------------------------------------------------------------------
  * moe_device_status - synchronises the current device, then returns (and
  * clears) the library's device-side error word: 0 if no kernel gave up a

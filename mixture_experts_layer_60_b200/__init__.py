@@ -20,7 +20,7 @@ __all__ = [
     "moe_route_workspace_size", "moe_permute_workspace_size", "moe_expert_ffn_workspace_size",
     "moe_expert_gate_up_save", "moe_combine_backward", "moe_expert_ffn_backward",
     "moe_expert_ffn_backward_workspace_size", "moe_unpermute_backward", "moe_router_weight_grad",
-    "moe_quantize_128x1_grouped",
+    "moe_quantize_128x1_grouped", "moe_ep_plan", "moe_ep_dispatch", "moe_ep_return",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
@@ -64,6 +64,11 @@ SYMBOLS = {
                                     _vp]),
     "moe_router_weight_grad": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp]),
     "moe_quantize_128x1_grouped": (_i, [_vp, _i, _i, _vp, _i, _vp, _vp, _vp, _vp]),
+    "moe_ep_plan": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp]),
+    "moe_ep_dispatch": (_i, [_vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _i, _i, _i,
+                             ctypes.POINTER(_vp), ctypes.POINTER(_vp), ctypes.c_longlong, _vp]),
+    "moe_ep_return": (_i, [_vp, _i, _vp, _vp, ctypes.c_longlong, _i, _i, ctypes.POINTER(_vp),
+                           ctypes.c_longlong, _vp]),
 }
 
 
@@ -294,3 +299,36 @@ def moe_quantize_128x1_grouped(x, offsets, q, scale, block_start, stream=None):
     n_groups = 1 if offsets is None else offsets.shape[0] - 1
     _check(lib().moe_quantize_128x1_grouped(_p(x), rows, cols, _p(offsets), n_groups, _p(q),
                                             _p(scale), _p(block_start), _s(stream)))
+
+
+# ------------------------------------------------------------------ expert parallelism
+
+def _ptrs(tensors):
+    arr = (ctypes.c_void_p * len(tensors))(*[_p(t) for t in tensors])
+    return ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p)), arr
+
+
+def moe_ep_plan(counts_all, rank, recv_offsets, send_base, stream=None):
+    W, N_r = counts_all.shape
+    _check(lib().moe_ep_plan(_p(counts_all), W, rank, N_r, _p(recv_offsets), _p(send_base),
+                             _s(stream)))
+
+
+def moe_ep_dispatch(u, topk_idx, inv_row, offsets, send_base, rank, recv_rows, recv_tags,
+                    stream=None):
+    """recv_rows / recv_tags: one tensor per rank (this GPU's or a peer's)."""
+    T, d = u.shape
+    W = len(recv_rows)
+    rp, _k1 = _ptrs(recv_rows)
+    tp, _k2 = _ptrs(recv_tags)
+    _check(lib().moe_ep_dispatch(_p(u), _dt(u), T, d, topk_idx.shape[1], _p(topk_idx),
+                                 _p(inv_row), _p(offsets), _p(send_base), send_base.shape[0], W,
+                                 rank, rp, tp, recv_rows[0].shape[0], _s(stream)))
+
+
+def moe_ep_return(y, recv_tags, n_rows, ret_rows, stream=None):
+    cap, d = y.shape
+    W = len(ret_rows)
+    rp, _k = _ptrs(ret_rows)
+    _check(lib().moe_ep_return(_p(y), _dt(y), _p(recv_tags), _p(n_rows), cap, d, W, rp,
+                               ret_rows[0].shape[0], _s(stream)))

@@ -622,6 +622,64 @@ moe_status moe_router_weight_grad(const void* x_perm, const int32_t* x_rows,
                                    as_stream(stream));
 }
 
+// ---------------------------------------------------------------- expert parallelism
+
+moe_status moe_ep_plan(const int32_t* counts_all, int W, int rank, int N_r,
+                       int32_t* recv_offsets, int32_t* send_base, void* stream) {
+  clear_last_error();
+  MOE_REQUIRE(W >= 1 && W <= 8 && rank >= 0 && rank < W, MOE_ERR_INVALID_ARG,
+              "moe_ep_plan: W=%d (1..8) rank=%d", W, rank);
+  MOE_REQUIRE(N_r > 0 && N_r % W == 0, MOE_ERR_INVALID_ARG,
+              "moe_ep_plan: N_r=%d must be a positive multiple of W=%d", N_r, W);
+  MOE_REQUIRE(counts_all && recv_offsets && send_base, MOE_ERR_INVALID_ARG,
+              "moe_ep_plan: null pointer");
+  MOE_TRY(check_device());
+  return launch_ep_plan(counts_all, W, rank, N_r, recv_offsets, send_base, as_stream(stream));
+}
+
+moe_status moe_ep_dispatch(const void* u, moe_dtype dt, int T, int d, int K,
+                           const int32_t* topk_idx, const int32_t* inv_row,
+                           const int32_t* offsets, const int32_t* send_base, int N_r, int W,
+                           int rank, void* const* recv_rows, void* const* recv_tags,
+                           long long recv_cap, void* stream) {
+  clear_last_error();
+  MOE_TRY(check_rowwise("moe_ep_dispatch", dt, T, d, K));
+  MOE_REQUIRE(W >= 1 && W <= 8 && rank >= 0 && rank < W && N_r > 0 && N_r % W == 0,
+              MOE_ERR_INVALID_ARG, "moe_ep_dispatch: W=%d rank=%d N_r=%d", W, rank, N_r);
+  if (T == 0) return MOE_OK;
+  MOE_REQUIRE(u && topk_idx && inv_row && offsets && send_base && recv_rows && recv_tags,
+              MOE_ERR_INVALID_ARG, "moe_ep_dispatch: null pointer");
+  for (int i = 0; i < W; ++i)
+    MOE_REQUIRE(recv_rows[i] && recv_tags[i] && al16(recv_rows[i]) &&
+                    reinterpret_cast<uintptr_t>(recv_tags[i]) % 8 == 0,
+                MOE_ERR_INVALID_ARG, "moe_ep_dispatch: rank %d buffers null or misaligned", i);
+  MOE_REQUIRE(al16(u), MOE_ERR_INVALID_ARG, "moe_ep_dispatch: u must be 16-byte aligned");
+  MOE_REQUIRE(recv_cap >= 0, MOE_ERR_INVALID_ARG, "moe_ep_dispatch: recv_cap");
+  MOE_TRY(check_device());
+  return launch_ep_dispatch(u, dtype_bytes(dt), T, d, K, topk_idx, inv_row, offsets, send_base,
+                            N_r, W, rank, recv_rows, recv_tags, recv_cap, as_stream(stream));
+}
+
+moe_status moe_ep_return(const void* y, moe_dtype dt, const void* recv_tags,
+                         const int32_t* n_rows, long long recv_cap, int d, int W,
+                         void* const* ret_rows, long long ret_cap, void* stream) {
+  clear_last_error();
+  MOE_TRY(check_rowwise("moe_ep_return", dt, 0, d, 1));
+  MOE_REQUIRE(W >= 1 && W <= 8, MOE_ERR_INVALID_ARG, "moe_ep_return: W=%d", W);
+  MOE_REQUIRE(recv_cap >= 0 && recv_cap < (1LL << 31) && ret_cap >= 0, MOE_ERR_INVALID_ARG,
+              "moe_ep_return: capacities");
+  if (recv_cap == 0) return MOE_OK;
+  MOE_REQUIRE(y && recv_tags && n_rows && ret_rows, MOE_ERR_INVALID_ARG,
+              "moe_ep_return: null pointer");
+  for (int i = 0; i < W; ++i)
+    MOE_REQUIRE(ret_rows[i] && al16(ret_rows[i]), MOE_ERR_INVALID_ARG,
+                "moe_ep_return: rank %d buffer null or misaligned", i);
+  MOE_REQUIRE(al16(y), MOE_ERR_INVALID_ARG, "moe_ep_return: y must be 16-byte aligned");
+  MOE_TRY(check_device());
+  return launch_ep_return(y, dtype_bytes(dt), recv_tags, n_rows, (int)recv_cap, d, W, ret_rows,
+                          ret_cap, as_stream(stream));
+}
+
 moe_status moe_device_status(int* flags) {
   clear_last_error();
   MOE_REQUIRE(flags, MOE_ERR_INVALID_ARG, "moe_device_status: null pointer");

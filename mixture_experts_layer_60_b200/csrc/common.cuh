@@ -35,6 +35,7 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 enum : int {
   ERR_GEMM_TIMEOUT = 1,       // tcgen05 GEMM: an mbarrier wait ran out
   ERR_GEMM_FP8_TIMEOUT = 2,   // FP8 tcgen05 GEMM: an mbarrier wait ran out
+  ERR_EP_BOUNDS = 4,          // expert-parallel copy: a row position past its buffer (skipped)
 };
 
 // ---------------------------------------------------------------- device side

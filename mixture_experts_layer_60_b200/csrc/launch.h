@@ -135,4 +135,17 @@ moe_status launch_router_weight_grad(const void* x, const int32_t* x_rows,
                                      const float* d_logit_perm, const int32_t* offsets,
                                      moe_dtype dt, int N_r, int d, float* dE, cudaStream_t s);
 
+// ep.cu ----------------------------------------------------------------------
+// Expert-parallel receive layout, dispatch and return (see ep.cu's header).
+moe_status launch_ep_plan(const int32_t* counts_all, int W, int rank, int N_r,
+                          int32_t* recv_offsets, int32_t* send_base, cudaStream_t s);
+moe_status launch_ep_dispatch(const void* u, int elem_bytes, int T, int d, int K,
+                              const int32_t* idx, const int32_t* inv_row, const int32_t* offsets,
+                              const int32_t* send_base, int N_r, int W, int rank,
+                              void* const* recv_rows, void* const* recv_src, long long recv_cap,
+                              cudaStream_t s);
+moe_status launch_ep_return(const void* y, int elem_bytes, const void* recv_src,
+                            const int32_t* n_rows, int rows_cap, int d, int W,
+                            void* const* ret_rows, long long ret_cap, cudaStream_t s);
+
 }  // namespace moe
