@@ -161,3 +161,34 @@ def test_layer_backward_v3_sampled():
     hs = O.silu(u @ Wg.T) * (u @ Wu.T)
     want = f64(dh)[:, rows].T @ hs
     assert_close(f64(lay.grad["Ws_down"][0])[rows], want, BF, "shared dW_down rows")
+
+
+@pytest.mark.parametrize("N_s,K", [(0, 1), (2, 6)])
+def test_layer_backward_edge_shapes(N_s, K):
+    """No shared expert with K = 1, and two shared experts with K = 6; expert
+    0 gets no token (bias -1), so its weight gradients must be exactly zero."""
+    cfg = LayerConfig(f"bwd_edge_{N_s}_{K}", T=200, d=256, N_r=16, K=K, N_s=N_s, I=256,
+                      dtype="bf16", seed=22)
+    w = make_layer_inputs(cfg, "cuda")
+    w["b"][0] = -1.0
+    lay = MoELayer(cfg, w)
+    lay.forward_train(w["u"])
+    dh = upstream_grad(cfg, "cuda")
+    lay.backward(dh)
+    torch.cuda.synchronize()
+    idx = lay.topk_idx.cpu().numpy()
+    assert not (idx == 0).any()
+    assert not lay.grad["W_gate_up"][0].any() and not lay.grad["W_down"][0].any()
+    ref = B.layer_backward(f64(w["u"]), f64(w["E"]), idx,
+                           LazyExperts(w["W_gate_up"], w["W_down"]),
+                           LazyExperts(w["Ws_gate_up"], w["Ws_down"]) if N_s else [], f64(dh))
+    assert_close(f64(lay.du), ref["du"], BF, "du")
+    assert_close(lay.grad["E"].double().cpu().numpy(), ref["dE"], BF, "dE")
+    I = cfg.I
+    for e, (dWg, dWu, dWd) in ref["routed"].items():
+        assert_close(f64(lay.grad["W_gate_up"][e][:I]), dWg, BF, f"dW_gate {e}")
+        assert_close(f64(lay.grad["W_down"][e]), dWd, BF, f"dW_down {e}")
+    for j in range(N_s):
+        dWg, dWu, dWd = ref["shared"][j]
+        assert_close(f64(lay.grad["Ws_gate_up"][j][I:]), dWu, BF, f"shared {j} dW_up")
+        assert_close(f64(lay.grad["Ws_down"][j]), dWd, BF, f"shared {j} dW_down")
