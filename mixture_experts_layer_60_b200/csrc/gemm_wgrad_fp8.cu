@@ -99,6 +99,16 @@ __device__ __forceinline__ uint64_t f2_pack(float a, float b) {
 __device__ __forceinline__ void f2_unpack(uint64_t v, float& a, float& b) {
   asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
 }
+__device__ __forceinline__ float lds_f32(uint32_t a) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint64_t lds_b64(uint32_t a) {
+  uint64_t v;
+  asm volatile("ld.shared.b64 %0, [%1];" : "=l"(v) : "r"(a));
+  return v;
+}
 // (a0, a1) * (b0, b1), elementwise, rounded like two fmul
 __device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
   uint64_t r;
@@ -259,10 +269,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int mt = loc / n_n, nt = loc - mt * n_n;
       int r0, cnt;
       group_rows(p, g, r0, cnt);
-      const int m = mt * BM + q * 32 + lane;
-      const int n0 = nt * BN + cq * 64;
-      uint4* dst = reinterpret_cast<uint4*>(p.C(g, m, n0));
       if (cnt <= 0) {
+        uint4* dst = reinterpret_cast<uint4*>(p.C(g, mt * BM + q * 32 + lane, nt * BN + cq * 64));
 #pragma unroll
         for (int i = 0; i < 8; ++i) dst[i] = make_uint4(0u, 0u, 0u, 0u);
         continue;
@@ -280,31 +288,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        const float* sl = scales + ss * (BM + BN);
-        const float sa = sl[q * 32 + lane];
+        // 32-bit shared addresses keep the hot loop's register count down
+        const uint32_t sl = smem_u32(scales) + ss * (BM + BN) * 4;
+        const float sa = lds_f32(sl + (q * 32 + lane) * 4);
         const uint64_t sa2 = f2_pack(sa, sa);
-        const uint2* sb2 = reinterpret_cast<const uint2*>(sl + BM + cq * 64);   // column pairs
+        const uint32_t sb = sl + (BM + cq * 64) * 4;                           // column pairs
         const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + pb * BN + cq * 64;
-        // eight 8-column pieces: two TMEM loads in flight per wait, few live registers
+        // eight 8-column pieces
 #pragma unroll
-        for (int c = 0; c < 8; c += 2) {
-          uint32_t r[2][8];
-          tmem_ld_32x32b_x8(tb + c * 8, r[0]);
-          tmem_ld_32x32b_x8(tb + c * 8 + 8, r[1]);
+        for (int c = 0; c < 8; ++c) {
+          uint32_t r[8];
+          tmem_ld_32x32b_x8(tb + c * 8, r);
           tmem_wait_ld();
-          if (c == 6) {
+          if (c == 7) {
             tc_fence_before();
             mbar_arrive(&pempty[pb]);   // partial read: the MMA may overwrite it
           }
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              const uint2 sbv = sb2[(c + h) * 4 + v];               // broadcast read
-              const uint64_t s2 = mul2(sa2, (uint64_t)sbv.x | ((uint64_t)sbv.y << 32));
-              acc2[(c + h) * 4 + v] =
-                  fma2_bits(r[h][2 * v], r[h][2 * v + 1], s2, acc2[(c + h) * 4 + v]);
-            }
+          for (int v = 0; v < 4; ++v) {
+            const uint64_t s2 = mul2(sa2, lds_b64(sb + (c * 8 + 2 * v) * 4));   // broadcast read
+            acc2[c * 4 + v] = fma2_bits(r[2 * v], r[2 * v + 1], s2, acc2[c * 4 + v]);
           }
         }
         mbar_arrive(&sempty[ss]);       // this block's scales are no longer read
@@ -312,6 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (++ss == SSLOTS) { ss = 0; sphase ^= 1; }
       }
       if (!ok) break;
+      uint4* dst = reinterpret_cast<uint4*>(p.C(g, mt * BM + q * 32 + lane, nt * BN + cq * 64));
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         uint32_t w4[4];
