@@ -153,52 +153,44 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    int stage = 0, used = 0;
-    uint32_t phase = 0;
-    bool ok = true;
-    const uint32_t idesc = idesc_bf16_f32_major(BM, BN, true, true);
-    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-      const int g = t / per_group;
-      int r0, cnt;
-      group_rows(p, g, r0, cnt);
-      if (cnt <= 0) continue;
-      const int ab = used & 1;
-      const uint32_t tpar = ((used >> 1) & 1) ^ 1;
-      ++used;
-      const bool got = mbar_wait_bounded(&tempty[ab], tpar, abort_flag, kWaitNs);
-      if (!__all_sync(0xffffffffu, got)) {
-        if (lane == 0) raise_abort(abort_flag, p.err);
-        break;
-      }
-      tc_fence_after();
-      const uint32_t d_tmem = tmem_base + ab * BN;
-      const int nkb = (cnt + BK - 1) / BK;
-      for (int kb = 0; kb < nkb; ++kb) {
-        const bool f = mbar_wait_bounded(&full[stage], phase, abort_flag, kWaitNs);
-        if (!__all_sync(0xffffffffu, f)) {
-          if (lane == 0) raise_abort(abort_flag, p.err);
-          ok = false;
+    if (lane == 0) {
+      int stage = 0, used = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      const uint32_t idesc = idesc_bf16_f32_major(BM, BN, true, true);
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const int g = t / per_group;
+        int r0, cnt;
+        group_rows(p, g, r0, cnt);
+        if (cnt <= 0) continue;
+        const int ab = used & 1;
+        const uint32_t tpar = ((used >> 1) & 1) ^ 1;
+        ++used;
+        if (!mbar_wait_bounded(&tempty[ab], tpar, abort_flag, kWaitNs)) {
+          raise_abort(abort_flag, p.err);
           break;
         }
-        uint8_t* a_st = smem + stage * STAGE_BYTES;
-        const int valid = min(BK, cnt - kb * BK);
-        const int nks = (valid + 15) / 16;
-        __syncwarp();
         tc_fence_after();
-        if (lane == 0) {
-          const uint32_t a0 = smem_u32(a_st), b0 = a0 + A_BYTES;
+        const uint32_t d_tmem = tmem_base + ab * BN;
+        const int nkb = (cnt + BK - 1) / BK;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait_bounded(&full[stage], phase, abort_flag, kWaitNs)) {
+            raise_abort(abort_flag, p.err);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int valid = min(BK, cnt - kb * BK);
+          const int nks = (valid + 15) / 16;
+          const uint32_t a0 = smem_u32(smem + stage * STAGE_BYTES), b0 = a0 + A_BYTES;
           for (int k = 0; k < nks; ++k)
             mma_f16_ss(d_tmem, smem_desc_mn_sw128(a0 + k * 2048, BOX_BYTES),
                        smem_desc_mn_sw128(b0 + k * 2048, BOX_BYTES), idesc, (kb | k) != 0);
           mma_commit(&empty[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
-        __syncwarp();
-        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        mma_commit(&tfull[ab]);
       }
-      if (lane == 0) mma_commit(&tfull[ab]);
-      __syncwarp();
-    }
-    if (lane == 0) {
       mma_commit(mma_done);
       mbar_wait_bounded(mma_done, 0, nullptr, kWaitNs);
     }

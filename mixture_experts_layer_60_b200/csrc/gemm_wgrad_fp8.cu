@@ -216,43 +216,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    int stage = 0, pb = 0;
-    uint32_t phase = 0, pphase = 0;
-    bool ok = true;
-    const uint32_t idesc = idesc_e4m3_f32(BM, BN) | (1u << 15) | (1u << 16);   // A, B MN-major
-    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-      const int g = t / per_group;
-      int r0, cnt;
-      group_rows(p, g, r0, cnt);
-      const int nkb = (cnt + BK - 1) / BK;
-      for (int kb = 0; kb < nkb; ++kb) {
-        const bool w1 = mbar_wait_bounded(&pempty[pb], pphase ^ 1, abort_flag, kWaitNs);
-        const bool w2 = w1 && mbar_wait_bounded(&full[stage], phase, abort_flag, kWaitNs);
-        if (!__all_sync(0xffffffffu, w2)) {
-          if (lane == 0) raise_abort(abort_flag, p.err);
-          ok = false;
-          break;
-        }
-        uint8_t* a_st = smem + stage * STAGE_BYTES;
-        const int valid = min(BK, cnt - kb * BK);
-        const int nks = (valid + 31) / 32;
-        __syncwarp();
-        tc_fence_after();
-        if (lane == 0) {
-          const uint32_t a0 = smem_u32(a_st), b0 = a0 + A_BYTES;
+    if (lane == 0) {
+      int stage = 0, pb = 0;
+      uint32_t phase = 0, pphase = 0;
+      bool ok = true;
+      const uint32_t idesc = idesc_e4m3_f32(BM, BN) | (1u << 15) | (1u << 16);   // A, B MN-major
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const int g = t / per_group;
+        int r0, cnt;
+        group_rows(p, g, r0, cnt);
+        const int nkb = (cnt + BK - 1) / BK;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait_bounded(&pempty[pb], pphase ^ 1, abort_flag, kWaitNs) ||
+              !mbar_wait_bounded(&full[stage], phase, abort_flag, kWaitNs)) {
+            raise_abort(abort_flag, p.err);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int valid = min(BK, cnt - kb * BK);
+          const int nks = (valid + 31) / 32;
+          const uint32_t a0 = smem_u32(smem + stage * STAGE_BYTES), b0 = a0 + A_BYTES;
           const uint32_t d_tmem = tmem_base + pb * BN;
           for (int k = 0; k < nks; ++k)
             mma_f8_ss(d_tmem, smem_desc_mn_sw128(a0 + k * 4096, BOX_BYTES),
                       smem_desc_mn_sw128(b0 + k * 4096, BOX_BYTES), idesc, k != 0);
           mma_commit(&empty[stage]);
           mma_commit(&pfull[pb]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          if (++pb == 2) { pb = 0; pphase ^= 1; }
         }
-        __syncwarp();
-        if (++stage == STAGES) { stage = 0; phase ^= 1; }
-        if (++pb == 2) { pb = 0; pphase ^= 1; }
       }
-    }
-    if (lane == 0) {
       mma_commit(mma_done);
       mbar_wait_bounded(mma_done, 0, nullptr, kWaitNs);
     }
