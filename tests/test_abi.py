@@ -165,3 +165,20 @@ def test_backward_argument_errors(L):
     # FP8 Wgrad quantiser
     assert L.moe_quantize_128x1_grouped(d, 100, 100, d, 4, d, d, d, None) == 2
     assert L.moe_quantize_128x1_grouped(d, 100, 128, d, 4, d, d, None, None) == 1
+
+
+def test_expert_parallel_argument_errors(L):
+    d = ctypes.c_void_p(256)
+    assert L.moe_ep_plan(d, 9, 0, 16, d, d, None) == 1           # at most 8 ranks
+    assert L.moe_ep_plan(d, 3, 0, 16, d, d, None) == 1           # N_r % W
+    assert L.moe_ep_plan(d, 2, 2, 16, d, d, None) == 1           # rank < W
+    assert L.moe_ep_plan(None, 2, 0, 16, d, d, None) == 1
+    two = (ctypes.c_void_p * 2)(256, 256)
+    pp = ctypes.cast(two, ctypes.POINTER(ctypes.c_void_p))
+    nul = (ctypes.c_void_p * 2)(256, None)
+    pn = ctypes.cast(nul, ctypes.POINTER(ctypes.c_void_p))
+    assert L.moe_ep_dispatch(d, 2, 8, 64, 4, d, d, d, d, 16, 2, 0, pp, pp, 64, None) == 2  # dtype
+    assert L.moe_ep_dispatch(d, 1, 8, 64, 4, d, d, d, d, 16, 2, 0, pn, pp, 64, None) == 1  # null rank buffer
+    assert L.moe_ep_dispatch(d, 1, 8, 64, 4, d, d, d, d, 15, 2, 0, pp, pp, 64, None) == 1  # N_r % W
+    assert L.moe_ep_return(d, 1, d, d, 64, 64, 9, pp, 64, None) == 1                       # W
+    assert L.moe_ep_return(d, 1, d, d, 64, 64, 2, pn, 64, None) == 1
