@@ -102,6 +102,26 @@ def _check(status: int):
         raise MoeError(status, lib().moe_last_error().decode(errors="replace"))
 
 
+# Tracing: with MOE_NVTX=1 in the environment every call below is wrapped in
+# an NVTX range named after the C entry point (visible in ncu / nsys timelines).
+_NVTX = os.environ.get("MOE_NVTX", "0") not in ("", "0")
+
+
+def _traced(fn):
+    if not _NVTX:
+        return fn
+    import functools
+
+    @functools.wraps(fn)
+    def wrap(*a, **k):
+        torch.cuda.nvtx.range_push(fn.__name__)
+        try:
+            return fn(*a, **k)
+        finally:
+            torch.cuda.nvtx.range_pop()
+    return wrap
+
+
 def _p(t):
     if t is None:
         return None
@@ -332,3 +352,9 @@ def moe_ep_return(y, recv_tags, n_rows, ret_rows, stream=None):
     rp, _k = _ptrs(ret_rows)
     _check(lib().moe_ep_return(_p(y), _dt(y), _p(recv_tags), _p(n_rows), cap, d, W, rp,
                                ret_rows[0].shape[0], _s(stream)))
+
+
+# wrap the public calls for tracing (no-op unless MOE_NVTX is set)
+for _name in [n for n in __all__ if n.startswith("moe_") and n in globals()
+              and not n.endswith("workspace_size")]:
+    globals()[_name] = _traced(globals()[_name])

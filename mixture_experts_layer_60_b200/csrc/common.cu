@@ -47,6 +47,16 @@ int* device_error_word() {
   return g_err_word_addr[dev];
 }
 
+moe_status ensure_max_smem(const void* kernel, int bytes, bool* done, const char* what) {
+  const int dev = current_device();
+  if (dev < 0) return fail(MOE_ERR_CUDA, "%s: no current device", what);
+  if (done[dev]) return MOE_OK;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return cuda_check(e, what);
+  done[dev] = true;
+  return MOE_OK;
+}
+
 int sm_count() {
   const int dev = current_device();
   if (dev < 0) return 148;

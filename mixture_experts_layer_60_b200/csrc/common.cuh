@@ -23,6 +23,11 @@ moe_status cuda_check(cudaError_t e, const char* what);
 // (one int per device, set by kernels that give up a bounded wait).
 int* device_error_word();
 
+// Raises a kernel's dynamic shared-memory limit to `bytes` once per device
+// (done: a per-call-site array of kMaxSmemDevices flags).
+constexpr int kMaxSmemDevices = 64;
+moe_status ensure_max_smem(const void* kernel, int bytes, bool* done, const char* what);
+
 // Number of SMs of the current device (cached per device).
 int sm_count();
 

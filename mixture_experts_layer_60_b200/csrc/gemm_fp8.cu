@@ -543,12 +543,11 @@ moe_status fp8_launch(const void* A, const float* a_scale, const void* B, const 
                       BK, Fp8Tile<EPI>::SW ? 128 : BN);
   if (st != MOE_OK) return st;
   auto kern = fp8_gemm_kernel<EPI, B_MN>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
-    if (e != cudaSuccess) return cuda_check(e, "fp8_gemm smem attribute");
-    attr_set = true;
+  static bool attr_done[kMaxSmemDevices] = {};   // per instantiation and device
+  {
+    const moe_status sst = ensure_max_smem(reinterpret_cast<const void*>(kern), SMEM_ALLOC,
+                                           attr_done, "fp8_gemm smem attribute");
+    if (sst != MOE_OK) return sst;
   }
   Fp8Params p;
   p.offsets = offsets;

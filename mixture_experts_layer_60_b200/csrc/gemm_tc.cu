@@ -432,11 +432,11 @@ moe_status tc_launch(const void* A, const void* B, int b_rows_per_group, const i
                     (uint64_t)G * b_rows_per_group, BK, BN_OUT);
   if (st != MOE_OK) return st;
   auto kern = tc_gemm_kernel<BN, EPI, STAGES>;
-  static bool attr_set = false;  // per instantiation
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
-    if (e != cudaSuccess) return cuda_check(e, "tc_gemm smem attribute");
-    attr_set = true;
+  static bool attr_done[kMaxSmemDevices] = {};   // per instantiation and device
+  {
+    const moe_status sst = ensure_max_smem(reinterpret_cast<const void*>(kern), L::ALLOC,
+                                           attr_done, "tc_gemm smem attribute");
+    if (sst != MOE_OK) return sst;
   }
   TcParams p;
   p.offsets = offsets;

@@ -344,12 +344,11 @@ moe_status launch_wgrad_gemm(const void* A, int M, const void* B, int N, const i
   st = make_tmap_2d_swz(&tmC, C, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, (uint64_t)G * M, 32, 32,
                         CU_TENSOR_MAP_SWIZZLE_64B);
   if (st != MOE_OK) return st;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(wgrad_gemm_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
-    if (e != cudaSuccess) return cuda_check(e, "wgrad smem attribute");
-    attr_set = true;
+  static bool attr_done[kMaxSmemDevices] = {};   // per instantiation and device
+  {
+    const moe_status sst = ensure_max_smem(reinterpret_cast<const void*>(wgrad_gemm_kernel), SMEM_ALLOC,
+                                           attr_done, "wgrad smem attribute");
+    if (sst != MOE_OK) return sst;
   }
   WgParams p;
   p.offsets = offsets;

@@ -359,12 +359,11 @@ moe_status launch_wgrad_fp8(const void* qa, const float* sa, int M, const void* 
   if (st != MOE_OK) return st;
   st = make_tmap_col_blocks(&tmB, qb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, rows, 128, BK, BN / 128);
   if (st != MOE_OK) return st;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(wgrad_fp8_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
-    if (e != cudaSuccess) return cuda_check(e, "fp8 wgrad smem attribute");
-    attr_set = true;
+  static bool attr_done[kMaxSmemDevices] = {};   // per instantiation and device
+  {
+    const moe_status sst = ensure_max_smem(reinterpret_cast<const void*>(wgrad_fp8_kernel), SMEM_ALLOC,
+                                           attr_done, "fp8 wgrad smem attribute");
+    if (sst != MOE_OK) return sst;
   }
   Wg8Params p;
   p.offsets = offsets;

@@ -441,12 +441,11 @@ moe_status ws_launch(const void* X, const void* W, int b_rows_per_group, const i
   st = make_tmap_2d(&tmX, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, rows, BK, XBOX);
   if (st != MOE_OK) return st;
   auto kern = ws_gemm_kernel<EPI, WMN>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
-    if (e != cudaSuccess) return cuda_check(e, "ws_gemm smem attribute");
-    attr_set = true;
+  static bool attr_done[kMaxSmemDevices] = {};   // per instantiation and device
+  {
+    const moe_status sst = ensure_max_smem(reinterpret_cast<const void*>(kern), SMEM_ALLOC,
+                                           attr_done, "ws_gemm smem attribute");
+    if (sst != MOE_OK) return sst;
   }
   WsParams p;
   p.offsets = offsets;
