@@ -12,7 +12,7 @@ gradient), and keeps the MoE gating module in its original precision.  The
 pages print no backward formulas; what follows is the chain rule applied to
 the forward definitions, step by step in reverse order.
 
-Readings (listed again in the design doc):
+Readings taken where the pages are silent:
 
   B1  The selection S_t (top-K of s+b) is piecewise constant in u, E and b:
       it is held fixed and has no gradient; b receives none.  Gradient flows

@@ -17,7 +17,7 @@ arXiv 2412.19437), section 方法 / 2. "具備無輔助損失平衡機制的 Dee
                    1x128 activation tiles, 128x128 weight blocks, FP32 promotion every
                    N_c = 128 accumulation steps.
 
-Readings taken where the page is silent (each listed again in the design doc):
+Readings taken where the page is silent:
 
   R1  g = g' / sum_j g'_j over the selected experts (no extra scale, no epsilon; s > 0).
   R2  top-K ties go to the lower expert index; the K outputs are ordered by
