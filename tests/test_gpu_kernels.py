@@ -206,6 +206,9 @@ def _ffn_case(sizes, d, I, dtype, seed, extra_rows=0):
     ([5000], 768, 256),                             # one large group (the shared-expert shape)
     ([64, 200, 333], 384, 256),                     # d not a multiple of 256 (128-column down tiles)
     ([255, 256, 257, 511, 513, 17, 16, 15], 256, 128),  # token tiling around 256-row boundaries
+    # tiny, empty and 256-row boundary groups with 256-column weight tiles on both GEMMs
+    ([255, 256, 257, 511, 513, 17, 16, 15, 1, 8, 9, 0, 24], 512, 256),
+    ([3] * 40 + [700, 0, 129], 1024, 768),            # many small groups, 3 gate/up pair tiles
 ])
 def test_expert_ffn_bf16(sizes, d, I):
     got, ref, n = _ffn_case(sizes, d, I, torch.bfloat16, sum(sizes) + d, extra_rows=3)
