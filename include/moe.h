@@ -113,7 +113,8 @@ moe_status moe_route_grouped(const void* u, const void* E, moe_dtype dt, const f
  *
  *   u        [T, d]      device, dt (MOE_F32, MOE_BF16 or MOE_E4M3)
  *   u_scale  [T, d/128]  device, float32: only for MOE_E4M3 (tile scales of u), else NULL
- *   topk_idx [T, K]      device, int32: from moe_route
+ *   topk_idx [T, K]      device, int32: from moe_route (an id outside [0, N_r)
+ *                        is left out: its inv_row is -1 and no row is copied)
  *   x_perm   [T*K, d]    device, dt out: x_perm[p] = u[perm_src[p]]
  *   x_scale  [T*K, d/128] device, float32 out (MOE_E4M3 only, else NULL)
  *   offsets  [N_r+1]     device, int32 out: group g is rows [offsets[g], offsets[g+1])

@@ -41,10 +41,27 @@ moe_status check_device() {
     if (_st != MOE_OK) return _st;    \
   } while (0)
 
-// Router workspace: float32 logits [T, N_r], then the tie-break list [1 + T] int32.
+// Router workspace: float32 logits [T, N_r], then the tie-break lists: a
+// 2-word header and tok/start/num [T] int32, candidate pairs [T*N_r] int32
+// and their float64 affinities [T*N_r] float32.
 size_t route_ws(int T, int N_r) {
   if (T <= 0 || N_r <= 0) return 0;
-  return align_up((size_t)T * N_r * sizeof(float), 256) + align_up((size_t)(T + 1) * 4, 256);
+  const size_t tn = align_up((size_t)T * N_r * sizeof(float), 256);
+  return tn + align_up((size_t)(2 + 3 * (size_t)T) * 4, 256) + 2 * tn;
+}
+
+RefineLists refine_lists(void* workspace, int T, int N_r) {
+  const size_t tn = align_up((size_t)T * N_r * sizeof(float), 256);
+  uint8_t* p = static_cast<uint8_t*>(workspace) + tn;
+  RefineLists rl;
+  rl.hdr = reinterpret_cast<int32_t*>(p);
+  rl.tok = rl.hdr + 2;
+  rl.start = rl.tok + T;
+  rl.num = rl.start + T;
+  p += align_up((size_t)(2 + 3 * (size_t)T) * 4, 256);
+  rl.pair = reinterpret_cast<int32_t*>(p);
+  rl.s64 = reinterpret_cast<float*>(p + tn);
+  return rl;
 }
 
 // Routing decided by a key gap below this is redone from float64 logits: the
@@ -106,6 +123,8 @@ moe_status route_impl(const char* who, const void* u, const void* E, moe_dtype d
   MOE_REQUIRE((long long)topk_groups * (N_r / n_groups) >= K, MOE_ERR_INVALID_ARG,
               "%s: the kept groups hold fewer than K experts", who);
   MOE_REQUIRE(d % 64 == 0, MOE_ERR_UNSUPPORTED, "%s: d=%d must be a multiple of 64", who, d);
+  MOE_REQUIRE((long long)T * N_r <= 0x7fffffffLL, MOE_ERR_UNSUPPORTED,
+              "%s: T * N_r must fit in 31 bits (T=%d N_r=%d)", who, T, N_r);
   MOE_REQUIRE(E && b && counts, MOE_ERR_INVALID_ARG, "%s: null pointer", who);
   MOE_REQUIRE(T == 0 || (u && topk_idx && topk_gate && workspace), MOE_ERR_INVALID_ARG,
               "%s: null pointer", who);
@@ -123,12 +142,11 @@ moe_status route_impl(const char* who, const void* u, const void* E, moe_dtype d
   } else {
     MOE_TRY(launch_logits_simt(u, E, dt, T, d, N_r, logits, s));
   }
-  int32_t* refine = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) +
-                                               align_up((size_t)T * N_r * sizeof(float), 256));
-  MOE_TRY(cuda_check(cudaMemsetAsync(refine, 0, sizeof(int32_t), s), "zero tie-break list"));
+  const RefineLists rl = refine_lists(workspace, T, N_r);
+  MOE_TRY(cuda_check(cudaMemsetAsync(rl.hdr, 0, 2 * sizeof(int32_t), s), "zero tie-break lists"));
   MOE_TRY(launch_topk(logits, b, T, N_r, K, n_groups, topk_groups, topk_idx, topk_gate, counts,
-                      refine, kRefineGap, s));
-  return launch_refine(u, E, dt, logits, b, d, N_r, K, n_groups, topk_groups, refine, T, topk_idx,
+                      rl, kRefineGap, s));
+  return launch_refine(u, E, dt, logits, b, d, N_r, K, n_groups, topk_groups, rl, T, topk_idx,
                        topk_gate, counts, s);
 }
 
@@ -169,8 +187,6 @@ moe_status moe_permute(const void* u, const float* u_scale, moe_dtype dt, const 
               "moe_permute: need 1 <= K <= N_r <= 1024");
   MOE_REQUIRE(((size_t)d * eb) % 16 == 0, MOE_ERR_UNSUPPORTED,
               "moe_permute: a row (%d x %d bytes) must be a multiple of 16 bytes", d, eb);
-  MOE_REQUIRE((8LL * N_r + 256LL * K) * 4 <= 200 * 1024, MOE_ERR_UNSUPPORTED,
-              "moe_permute: K=%d with N_r=%d exceeds the rank kernel's shared memory", K, N_r);
   MOE_REQUIRE(offsets, MOE_ERR_INVALID_ARG, "moe_permute: null offsets");
   MOE_REQUIRE(T == 0 || (u && topk_idx && x_perm && perm_src && inv_row && workspace),
               MOE_ERR_INVALID_ARG, "moe_permute: null pointer");

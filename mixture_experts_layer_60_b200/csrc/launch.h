@@ -10,18 +10,32 @@ namespace moe {
 // logits[t, i] = sum_k u[t,k] E[i,k] on CUDA cores (float32 accumulation).
 moe_status launch_logits_simt(const void* u, const void* E, moe_dtype dt, int T, int d,
                               int N_r, float* logits, cudaStream_t s);
+// Float64 tie-break lists (device, inside the router workspace):
+//   hdr[0]  tokens listed, hdr[1] candidate pairs (both zeroed before top-K)
+//   tok, start, num [T]   per listed token: its id, first pair, number of pairs
+//   pair [T*N_r]          candidate (token, expert) as t*N_r + e, grouped per token
+//   s64  [T*N_r]          float32: the pair's float64 affinity, rounded once
+struct RefineLists {
+  int32_t* hdr;
+  int32_t* tok;
+  int32_t* start;
+  int32_t* num;
+  int32_t* pair;
+  float* s64;
+};
 // sigmoid, biased top-K, gates, histogram (counts must be zeroed beforehand).
 // n_groups > 1 && topk_groups < n_groups restricts each token to its best groups.
-// Tokens whose routing was decided by a key gap < refine_gap are appended to
-// refine ([0] = count, zeroed beforehand; [1..T] = token ids).
+// A token whose routing was decided by a key gap < refine_gap is listed with
+// the experts whose float32 key lies near one of its decision boundaries.
 moe_status launch_topk(const float* logits, const float* b, int T, int N_r, int K, int n_groups,
                        int topk_groups, int32_t* idx, float* gate, int32_t* counts,
-                       int32_t* refine, float refine_gap, cudaStream_t s);
-// Redoes the routing of the listed tokens from float64 logits.
+                       RefineLists rl, float refine_gap, cudaStream_t s);
+// Float64 affinities of the listed pairs, then the listed tokens' routing
+// redone from them.
 moe_status launch_refine(const void* u, const void* E, moe_dtype dt, const float* logits,
-                         const float* b, int d,
-                         int N_r, int K, int n_groups, int topk_groups, const int32_t* refine,
-                         int T, int32_t* idx, float* gate, int32_t* counts, cudaStream_t s);
+                         const float* b, int d, int N_r, int K, int n_groups, int topk_groups,
+                         RefineLists rl, int T, int32_t* idx, float* gate, int32_t* counts,
+                         cudaStream_t s);
 
 // permute.cu -----------------------------------------------------------------
 size_t permute_ws_bytes(int T, int N_r);

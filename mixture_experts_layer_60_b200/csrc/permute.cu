@@ -32,7 +32,10 @@ __global__ void __launch_bounds__(kChunk) chunk_hist_kernel(const int32_t* __res
   const int c = blockIdx.x;
   const int t = c * kChunk + threadIdx.x;
   if (t < T)
-    for (int k = 0; k < K; ++k) atomicAdd(&h[idx[(size_t)t * K + k]], 1);
+    for (int k = 0; k < K; ++k) {
+      const int e = idx[(size_t)t * K + k];
+      if ((unsigned)e < (unsigned)N_r) atomicAdd(&h[e], 1);
+    }
   __syncthreads();
   for (int i = threadIdx.x; i < N_r; i += blockDim.x) chunk_hist[(size_t)c * N_r + i] = h[i];
 }
@@ -81,34 +84,40 @@ __global__ void __launch_bounds__(1024) chunk_scan_kernel(const int32_t* __restr
 }
 
 // Stable rank: pair (t, k) with expert e lands on
-//   chunk_base[c][e] + #(earlier warps of the chunk routed to e)
+//   chunk_base[c][e] + #(tokens of earlier warps of the chunk routed to e)
 //                    + #(earlier lanes of this warp routed to e).
-// A token never holds the same expert twice, so ordering by token is total.
+// A token never holds the same expert twice, so ordering by token is total,
+// and a warp's tokens routed to e form one 32-bit lane mask: the counts are
+// population counts of those masks.
 __global__ void __launch_bounds__(kChunk) chunk_rank_kernel(const int32_t* __restrict__ idx, int T,
                                                             int N_r, int K,
                                                             const int32_t* __restrict__ chunk_base,
                                                             int32_t* __restrict__ perm_src,
                                                             int32_t* __restrict__ inv_row) {
-  extern __shared__ int sm[];
-  int* whist = sm;                          // [kChunk/32][N_r]
-  int* ids = sm + (kChunk / 32) * N_r;      // [kChunk][K]
+  extern __shared__ unsigned lanes_of[];    // [kChunk/32][N_r]: lanes of warp w routed to e
   const int c = blockIdx.x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int t = c * kChunk + threadIdx.x;
-  for (int i = threadIdx.x; i < (kChunk / 32) * N_r; i += blockDim.x) whist[i] = 0;
-  for (int k = 0; k < K; ++k) ids[threadIdx.x * K + k] = t < T ? idx[(size_t)t * K + k] : -1;
+  for (int i = threadIdx.x; i < (kChunk / 32) * N_r; i += blockDim.x) lanes_of[i] = 0;
   __syncthreads();
+  const int32_t* it = idx + (size_t)t * K;
   if (t < T)
-    for (int k = 0; k < K; ++k) atomicAdd(&whist[warp * N_r + ids[threadIdx.x * K + k]], 1);
+    for (int k = 0; k < K; ++k) {
+      const int e = it[k];
+      if ((unsigned)e < (unsigned)N_r) atomicOr(&lanes_of[warp * N_r + e], 1u << lane);
+    }
   __syncthreads();
   if (t < T) {
+    const unsigned below = (1u << lane) - 1u;
     for (int k = 0; k < K; ++k) {
-      const int e = ids[threadIdx.x * K + k];
+      const int e = it[k];
+      if ((unsigned)e >= (unsigned)N_r) {     // not an expert id: the pair is left out
+        inv_row[(size_t)t * K + k] = -1;
+        continue;
+      }
       int r = chunk_base[(size_t)c * N_r + e];
-      for (int w = 0; w < warp; ++w) r += whist[w * N_r + e];
-      const int* base = ids + (warp * 32) * K;
-      for (int l = 0; l < lane; ++l)
-        for (int kk = 0; kk < K; ++kk) r += (base[l * K + kk] == e);
+      for (int w = 0; w < warp; ++w) r += __popc(lanes_of[w * N_r + e]);
+      r += __popc(lanes_of[warp * N_r + e] & below);
       perm_src[r] = t;
       inv_row[(size_t)t * K + k] = r;
     }
@@ -137,7 +146,7 @@ __global__ void __launch_bounds__(256) scatter_rows_kernel(const uint4* __restri
     const uint4 v0 = src[c], v1 = src[c + 32], v2 = src[c + 64], v3 = src[c + 96];
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
-      if (k < Kc) {
+      if (k < Kc && rows[k] >= 0) {
         uint4* dst = x_perm + (size_t)rows[k] * nvec;
         dst[c] = v0; dst[c + 32] = v1; dst[c + 64] = v2; dst[c + 96] = v3;
       }
@@ -147,15 +156,17 @@ __global__ void __launch_bounds__(256) scatter_rows_kernel(const uint4* __restri
     const uint4 v = src[c];
 #pragma unroll
     for (int k = 0; k < 16; ++k)
-      if (k < Kc) x_perm[(size_t)rows[k] * nvec + c] = v;
+      if (k < Kc && rows[k] >= 0) x_perm[(size_t)rows[k] * nvec + c] = v;
   }
   for (int k = 16; k < K; ++k) {
     const int r = inv_row[(size_t)t * K + k];
+    if (r < 0) continue;
     for (int cc = lane; cc < nvec; cc += 32) x_perm[(size_t)r * nvec + cc] = src[cc];
   }
   if (u_scale) {
     for (int k = 0; k < K; ++k) {
       const int r = inv_row[(size_t)t * K + k];
+      if (r < 0) continue;
       for (int j = lane; j < nscale; j += 32)
         x_scale[(size_t)r * nscale + j] = u_scale[(size_t)t * nscale + j];
     }
@@ -173,7 +184,7 @@ moe_status launch_permute(const void* u, const float* u_scale, int elem_bytes, c
   chunk_hist_kernel<<<nch, kChunk, N_r * sizeof(int), s>>>(idx, T, N_r, K, chunk_hist);
   const int scan_threads = (N_r + 31) / 32 * 32;
   chunk_scan_kernel<<<1, scan_threads, 0, s>>>(chunk_hist, nch, N_r, chunk_base, offsets);
-  const size_t rank_smem = ((size_t)(kChunk / 32) * N_r + (size_t)kChunk * K) * sizeof(int);
+  const size_t rank_smem = (size_t)(kChunk / 32) * N_r * sizeof(unsigned);
   if (rank_smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(chunk_rank_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -251,10 +262,6 @@ extern "C" moe_status moe_permute_noalloc(const void* u, const float* u_scale, m
                 d, N_r, K);
   if (N_r > 1024 || K > N_r)
     return fail(MOE_ERR_UNSUPPORTED, "moe_permute_noalloc: need 1 <= K <= N_r <= 1024");
-  if ((8LL * N_r + 256LL * K) * 4 > 200 * 1024)
-    return fail(MOE_ERR_UNSUPPORTED,
-                "moe_permute_noalloc: K=%d with N_r=%d exceeds the rank kernel's shared memory", K,
-                N_r);
   if (((size_t)d * eb) % 16 != 0)
     return fail(MOE_ERR_UNSUPPORTED, "moe_permute_noalloc: a row must be a multiple of 16 bytes");
   if (!offsets) return fail(MOE_ERR_INVALID_ARG, "moe_permute_noalloc: null offsets");

@@ -16,10 +16,32 @@ moe_status launch_logits_simt(const void* u, const void* E, moe_dtype dt, int T,
   return launch_simt_gemm(u, E, 0, nullptr, 1, T, N_r, d, false, dt, logits, MOE_F32, s);
 }
 
+// Precise tie-break.  The tensor-core logits are float32 sums of d products,
+// which can move s by a few 1e-6 at V3 width.  A token whose routing was
+// decided by a key gap below the refine gap is listed together with the
+// experts whose float32 key lies within kNearBoundary of one of its decision
+// boundaries; those experts get float64 logits (s = Sigmoid in float64,
+// rounded once to float32: the affinity line's exact value) and the token is
+// routed again.  The other experts keep their float32 keys, which are too far
+// below every boundary for the float32 error to matter.  If the group choice
+// changes, every expert of the token is recomputed.
+constexpr float kNearBoundary = 6e-5f;   // > 2 x the largest float32 key error
+
+// Order-preserving map of a float key to an unsigned integer (every real key
+// maps above 0; -0 is taken as +0, so equal keys map to equal integers).
+__device__ __forceinline__ uint32_t ord_key(float f) {
+  const uint32_t b = __float_as_uint(f + 0.0f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float ord_float(uint32_t o) {
+  return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
+}
+
 // One warp per token.  Lane l holds experts e = j*32 + l (j < V), so a
 // token's logits are read with coalesced loads.  K rounds of a warp-wide
 // arg-max with the order (key descending, index ascending) give the
-// selection in the documented output order.
+// selection in the documented output order; lane k keeps the k-th winner
+// (k < 32) so that the gates are normalised and written from registers.
 //
 // Group limit (n_groups > 1, topk_groups < n_groups): experts form n_groups
 // groups of N_r/n_groups consecutive indices; a group's score is its largest
@@ -33,8 +55,8 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
                                                    int N_r, int K, int n_groups, int topk_groups,
                                                    int32_t* __restrict__ idx,
                                                    float* __restrict__ gate,
-                                                   int32_t* __restrict__ counts,
-                                                   int32_t* __restrict__ refine, float refine_gap) {
+                                                   int32_t* __restrict__ counts, RefineLists rl,
+                                                   float refine_gap) {
   extern __shared__ int hist[];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -45,7 +67,7 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
   __syncthreads();
 
   for (int t = blockIdx.x * warps_per_block + warp; t < T; t += gridDim.x * warps_per_block) {
-    float key[V], sv[V];
+    float key[V], sv[V], kb[V];
 #pragma unroll
     for (int j = 0; j < V; ++j) {
       const int e = j * 32 + lane;
@@ -58,8 +80,10 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
         sv[j] = 0.f;
         key[j] = -INFINITY;
       }
+      kb[j] = key[j];
     }
-    float margin = INFINITY;   // smallest key gap that decided this token's routing
+    float margin = INFINITY;     // smallest key gap that decided this token's routing
+    float next_group = INFINITY; // score of the best group left out (group limit only)
     if (grouped) {
       const int gs = N_r / n_groups;
 #pragma unroll
@@ -88,6 +112,7 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
           last_kept = bk;
         } else {
           margin = fminf(margin, last_kept - bk);   // kept vs excluded group scores
+          next_group = bk;
         }
       }
 #pragma unroll
@@ -96,84 +121,119 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
         if (e < N_r && !((kept >> (e / gs)) & 1u)) key[j] = -INFINITY;
       }
     }
-    float sum = 0.f, prev = INFINITY;
+    // K+1 rounds of a warp arg-max on order-preserving integer keys: each
+    // lane keeps the best of its own keys (ties to the lower index), the warp
+    // takes the largest with one reduction and the lowest expert id holding it
+    // with another; the winner's lane then drops it and rescans its keys.
+    uint32_t ko[V];
+#pragma unroll
+    for (int j = 0; j < V; ++j) ko[j] = j * 32 + lane < N_r ? ord_key(key[j]) : 0u;
+    uint32_t lb = 0u;
+    int lj = 0;
+#pragma unroll
+    for (int j = 0; j < V; ++j)
+      if (ko[j] > lb) { lb = ko[j]; lj = j; }
+    float sum = 0.f, prev = INFINITY, next_key = -INFINITY;
+    int my_e = 0;
+    float my_s = 0.f;
     for (int k = 0; k <= K; ++k) {             // round K only measures the next key
-      // lane-local best
-      float bk = -INFINITY;
-      int be = 0x7fffffff;
-#pragma unroll
-      for (int j = 0; j < V; ++j) {
-        const int e = j * 32 + lane;
-        if (key[j] > bk || (key[j] == bk && e < be)) {
-          if (e < N_r) { bk = key[j]; be = e; }
-        }
-      }
-      // warp arg-max
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-        if (ok > bk || (ok == bk && oe < be)) { bk = ok; be = oe; }
-      }
+      const uint32_t m = __reduce_max_sync(0xffffffffu, lb);
+      if (m == 0u) break;                       // no key left (only after the K-th round)
+      const int be = __reduce_min_sync(0xffffffffu, lb == m ? lj * 32 + lane : 0x7fffffff);
+      const float bk = ord_float(m);
       margin = fminf(margin, prev - bk);        // adjacent selected keys, and K-th vs next
       prev = bk;
-      if (k == K) break;
-      // the owner removes the winner and broadcasts its unbiased s
+      if (k == K) { next_key = bk; break; }
+      // the owner drops the winner (compared by expert id so that the arrays
+      // stay in registers) and rescans; its unbiased s is broadcast
       float s_win = 0.f;
-      if ((be & 31) == lane) {
+      uint32_t nb = 0u;
+      int nj = 0;
 #pragma unroll
-        for (int j = 0; j < V; ++j)
-          if (j == (be >> 5)) { s_win = sv[j]; key[j] = -INFINITY; }
+      for (int j = 0; j < V; ++j) {
+        if (j * 32 + lane == be) { s_win = sv[j]; ko[j] = 0u; }
+        if (ko[j] > nb) { nb = ko[j]; nj = j; }
       }
+      lb = nb;
+      lj = nj;
       s_win = __shfl_sync(0xffffffffu, s_win, be & 31);
       sum += s_win;
-      if (lane == 0) {
+      if (k < 32) {
+        if (lane == k) { my_e = be; my_s = s_win; }
+      } else if (lane == 0) {
         idx[(size_t)t * K + k] = be;
         gate[(size_t)t * K + k] = s_win;
         atomicAdd(&hist[be], 1);
       }
     }
-    __syncwarp();
-    for (int k = lane; k < K; k += 32) {
-      const size_t p = (size_t)t * K + k;
-      gate[p] = gate[p] / sum;
+    if (lane < K) {
+      idx[(size_t)t * K + lane] = my_e;
+      gate[(size_t)t * K + lane] = my_s / sum;
+      atomicAdd(&hist[my_e], 1);
     }
-    if (lane == 0 && margin < refine_gap) refine[1 + atomicAdd(&refine[0], 1)] = t;
+    if (K > 32) {
+      __syncwarp();
+      for (int k = 32 + lane; k < K; k += 32) {
+        const size_t p = (size_t)t * K + k;
+        gate[p] = gate[p] / sum;
+      }
+    }
+    if (margin < refine_gap) {
+      // list the token with every expert whose float32 key is near the lowest
+      // key a decision hinged on (the (K+1)-th key inside the kept groups and,
+      // with the group limit, the best excluded group's score)
+      const float thr = fminf(next_key, next_group) - kNearBoundary;
+      int c = 0;
+#pragma unroll
+      for (int j = 0; j < V; ++j)
+        if (j * 32 + lane < N_r && kb[j] >= thr) ++c;
+      int incl = c;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+      }
+      const int total = __shfl_sync(0xffffffffu, incl, 31);
+      int base = 0, slot = 0;
+      if (lane == 0) {
+        base = atomicAdd(&rl.hdr[1], total);
+        slot = atomicAdd(&rl.hdr[0], 1);
+        rl.tok[slot] = t;
+        rl.start[slot] = base;
+        rl.num[slot] = total;
+      }
+      int w = __shfl_sync(0xffffffffu, base, 0) + incl - c;
+#pragma unroll
+      for (int j = 0; j < V; ++j) {
+        const int e = j * 32 + lane;
+        if (e < N_r && kb[j] >= thr) rl.pair[w++] = t * N_r + e;
+      }
+    }
   }
   __syncthreads();
   for (int i = threadIdx.x; i < N_r; i += blockDim.x)
     if (hist[i]) atomicAdd(&counts[i], hist[i]);
 }
 
-// Precise tie-break.  The tensor-core logits are float32 sums of d products,
-// which can move s by a few 1e-6 at V3 width.  For every token whose routing
-// was decided by a key gap below the refine gap, the experts whose float32
-// key lies within kNearBoundary of a decision boundary get float64 logits
-// (s = Sigmoid in float64, rounded once to float32: the affinity line's exact
-// value); the others keep their float32 keys, which are too far below every
-// boundary for the float32 error to matter.  Selection (with the group limit),
-// gates and load are then redone.  If the group choice changes, every expert
-// is recomputed.  One block per listed token; its warps share the float64
-// dot products.
-constexpr float kNearBoundary = 6e-5f;   // > 2 x the largest float32 key error
-
+// Float64 dot product of one token row and one centroid row: each lane
+// accumulates its share in two float64 accumulators; returns the lane's part.
 template <typename Tin>
-__device__ __forceinline__ float exact_affinity(const Tin* __restrict__ ut,
-                                                const Tin* __restrict__ er, int d, int lane) {
+__device__ __forceinline__ double dot64_part(const Tin* __restrict__ ut,
+                                             const Tin* __restrict__ er, int nv, int v0,
+                                             int stride) {
   double a0 = 0.0, a1 = 0.0;
-  const int nv = d / (16 / (int)sizeof(Tin));
   const uint4* u4 = reinterpret_cast<const uint4*>(ut);
   const uint4* e4 = reinterpret_cast<const uint4*>(er);
-  for (int v0 = lane; v0 < nv; v0 += 128) {
-    uint4 x[4], w[4];
+  for (int vb = v0; vb < nv; vb += 8 * stride) {
+    uint4 x[8], w[8];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {         // four independent 16-byte loads in flight
-      const int v = v0 + q * 32;
+    for (int q = 0; q < 8; ++q) {         // eight independent 16-byte loads per operand in flight
+      const int v = vb + q * stride;
       x[q] = v < nv ? u4[v] : make_uint4(0, 0, 0, 0);
       w[q] = v < nv ? e4[v] : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < 8; ++q) {
       const uint32_t xs[4] = {x[q].x, x[q].y, x[q].z, x[q].w};
       const uint32_t ws[4] = {w[q].x, w[q].y, w[q].z, w[q].w};
       if (sizeof(Tin) == 2) {
@@ -190,10 +250,49 @@ __device__ __forceinline__ float exact_affinity(const Tin* __restrict__ ut,
       }
     }
   }
-  double acc = a0 + a1;
+  return a0 + a1;
+}
+
+__device__ __forceinline__ float affinity64(double logit) {
+  return (float)(1.0 / (1.0 + exp(-logit)));
+}
+
+// s of one expert from a float64 logit, the whole warp on one dot product.
+template <typename Tin>
+__device__ __forceinline__ float exact_affinity_warp(const Tin* __restrict__ ut,
+                                                     const Tin* __restrict__ er, int d, int lane) {
+  double acc = dot64_part(ut, er, d / (16 / (int)sizeof(Tin)), lane, 32);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  return (float)(1.0 / (1.0 + exp(-acc)));
+  return affinity64(acc);
+}
+
+// One block of kDotThreads per listed pair: s64[p] = float64 affinity.
+constexpr int kDotThreads = 128;
+template <typename Tin>
+__global__ void __launch_bounds__(kDotThreads) refine_dot_kernel(const Tin* __restrict__ u,
+                                                                 const Tin* __restrict__ E, int d,
+                                                                 int N_r, RefineLists rl) {
+  __shared__ double part[kDotThreads / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int n = rl.hdr[1];
+  const int nv = d / (16 / (int)sizeof(Tin));
+  for (int p = blockIdx.x; p < n; p += gridDim.x) {
+    const int code = rl.pair[p];
+    const int t = code / N_r, e = code - t * N_r;
+    double acc = dot64_part(u + (size_t)t * d, E + (size_t)e * d, nv, threadIdx.x, kDotThreads);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) part[warp] = acc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      double a = 0.0;
+#pragma unroll
+      for (int w = 0; w < kDotThreads / 32; ++w) a += part[w];
+      rl.s64[p] = affinity64(a);
+    }
+    __syncthreads();
+  }
 }
 
 // Warp-wide arg-max of (key desc, index asc) over keys held lane-strided in kv[].
@@ -213,13 +312,13 @@ __device__ __forceinline__ void warp_best(const float* kv, int N_r, int lane, fl
 // Group limit on keys kv[]: returns the kept-group mask (topk_groups best
 // group maxima, ties to the lower group index).
 __device__ __forceinline__ unsigned keep_groups(const float* kv, int N_r, int n_groups,
-                                                int topk_groups, int lane, float* next_score) {
+                                                int topk_groups, int lane) {
   const int gs = N_r / n_groups;
   float gscore = -INFINITY;
   if (lane < n_groups)
     for (int j = 0; j < gs; ++j) gscore = fmaxf(gscore, kv[lane * gs + j]);
   unsigned kept = 0;
-  for (int r = 0; r <= topk_groups && r < n_groups; ++r) {
+  for (int r = 0; r < topk_groups; ++r) {
     float bk = (lane < n_groups && !((kept >> lane) & 1u)) ? gscore : -INFINITY;
     int bg = (lane < n_groups && !((kept >> lane) & 1u)) ? lane : 0x7fffffff;
 #pragma unroll
@@ -228,91 +327,55 @@ __device__ __forceinline__ unsigned keep_groups(const float* kv, int N_r, int n_
       const int og = __shfl_xor_sync(0xffffffffu, bg, off);
       if (ok > bk || (ok == bk && og < bg)) { bk = ok; bg = og; }
     }
-    if (r < topk_groups) kept |= 1u << bg;
-    else *next_score = bk;
+    kept |= 1u << bg;
   }
   return kept;
 }
 
+// One block per listed token: float32 keys for every expert, the float64
+// affinities of its listed experts on top, then selection, gates and load
+// redone (a changed group choice recomputes every expert in float64).
 template <typename Tin>
-__global__ void __launch_bounds__(256) refine_kernel(const Tin* __restrict__ u,
-                                                     const Tin* __restrict__ E,
-                                                     const float* __restrict__ logits,
-                                                     const float* __restrict__ bias, int d, int N_r,
-                                                     int K, int n_groups, int topk_groups,
-                                                     const int32_t* __restrict__ refine,
-                                                     int32_t* __restrict__ idx,
-                                                     float* __restrict__ gate,
-                                                     int32_t* __restrict__ counts) {
+__global__ void __launch_bounds__(256) refine_select_kernel(
+    const Tin* __restrict__ u, const Tin* __restrict__ E, const float* __restrict__ logits,
+    const float* __restrict__ bias, int d, int N_r, int K, int n_groups, int topk_groups,
+    RefineLists rl, int32_t* __restrict__ idx, float* __restrict__ gate,
+    int32_t* __restrict__ counts) {
   extern __shared__ float sm_r[];
   float* sv = sm_r;            // s [N_r]
   float* kv = sv + N_r;        // key [N_r]
   float* kw = kv + N_r;        // scratch keys [N_r]
-  int* cand = reinterpret_cast<int*>(kw + N_r);   // [N_r] experts to recompute, [N_r] = count
   __shared__ int s_full;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   const bool grouped = n_groups > 1 && topk_groups < n_groups;
   const int gs = grouped ? N_r / n_groups : N_r;
-  const int n = refine[0];
+  const int n = rl.hdr[0];
   for (int i = blockIdx.x; i < n; i += gridDim.x) {
-    const int t = refine[1 + i];
-    const Tin* ut = u + (size_t)t * d;
+    const int t = rl.tok[i], p0 = rl.start[i], np = rl.num[i];
     for (int e = threadIdx.x; e < N_r; e += blockDim.x) {
       const float sf = 1.0f / (1.0f + expf(-logits[(size_t)t * N_r + e]));   // as the top-K kernel
       sv[e] = sf;
-      kv[e] = sf + bias[e];
-      kw[e] = kv[e];
+      kw[e] = sf + bias[e];
     }
     __syncthreads();
     unsigned kept32 = 0xffffffffu;
-    if (warp == 0) {
-      // lowest key any decision can hinge on: the (K+1)-th key inside the kept
-      // groups and, with the group limit, the best excluded group's score
-      float floor_key = INFINITY;
-      if (grouped) {
-        float next_g = -INFINITY;
-        kept32 = keep_groups(kw, N_r, n_groups, topk_groups, lane, &next_g);
-        floor_key = next_g;
-        for (int e = lane; e < N_r; e += 32)
-          if (!((kept32 >> (e / gs)) & 1u)) kw[e] = -INFINITY;
-        __syncwarp();
-      }
-      for (int k = 0; k <= K; ++k) {
-        float bk;
-        int be;
-        warp_best(kw, N_r, lane, bk, be);
-        if (k == K || be >= N_r) { floor_key = fminf(floor_key, bk); break; }
-        __syncwarp();
-        if (lane == 0) kw[be] = -INFINITY;
-        __syncwarp();
-      }
-      if (lane == 0) {
-        int c = 0;
-        for (int e = 0; e < N_r; ++e)
-          if (kv[e] >= floor_key - kNearBoundary) cand[c++] = e;
-        cand[N_r] = c;
-      }
+    if (grouped && warp == 0) kept32 = keep_groups(kw, N_r, n_groups, topk_groups, lane);
+    for (int c = threadIdx.x; c < np; c += blockDim.x) {
+      const int e = rl.pair[p0 + c] - t * N_r;
+      sv[e] = rl.s64[p0 + c];
     }
     __syncthreads();
-    // float64 affinity of the candidates, one warp per candidate
-    for (int c = warp; c < cand[N_r]; c += nw) {
-      const int e = cand[c];
-      const float sf = exact_affinity(ut, E + (size_t)e * d, d, lane);
-      if (lane == 0) { sv[e] = sf; kv[e] = sf + bias[e]; }
-    }
+    for (int e = threadIdx.x; e < N_r; e += blockDim.x) kv[e] = sv[e] + bias[e];
     __syncthreads();
     if (grouped) {
       if (warp == 0) {
-        for (int e = lane; e < N_r; e += 32) kw[e] = kv[e];
-        __syncwarp();
-        float next_g = -INFINITY;
-        const unsigned kept = keep_groups(kw, N_r, n_groups, topk_groups, lane, &next_g);
+        const unsigned kept = keep_groups(kv, N_r, n_groups, topk_groups, lane);
         if (lane == 0) s_full = kept != kept32;   // group choice moved: refine every expert
       }
       __syncthreads();
       if (s_full) {
         for (int e = warp; e < N_r; e += nw) {
-          const float sf = exact_affinity(ut, E + (size_t)e * d, d, lane);
+          const float sf = exact_affinity_warp(u + (size_t)t * d, E + (size_t)e * d, d, lane);
           if (lane == 0) { sv[e] = sf; kv[e] = sf + bias[e]; }
         }
       }
@@ -322,8 +385,7 @@ __global__ void __launch_bounds__(256) refine_kernel(const Tin* __restrict__ u,
       for (int e = lane; e < N_r; e += 32) kw[e] = kv[e];
       __syncwarp();
       if (grouped) {
-        float next_g = -INFINITY;
-        const unsigned kept = keep_groups(kw, N_r, n_groups, topk_groups, lane, &next_g);
+        const unsigned kept = keep_groups(kw, N_r, n_groups, topk_groups, lane);
         for (int e = lane; e < N_r; e += 32)
           if (!((kept >> (e / gs)) & 1u)) kw[e] = -INFINITY;
         __syncwarp();
@@ -357,34 +419,46 @@ __global__ void __launch_bounds__(256) refine_kernel(const Tin* __restrict__ u,
 
 moe_status launch_refine(const void* u, const void* E, moe_dtype dt, const float* logits,
                          const float* b, int d, int N_r, int K, int n_groups, int topk_groups,
-                         const int32_t* refine, int T, int32_t* idx, float* gate, int32_t* counts,
+                         RefineLists rl, int T, int32_t* idx, float* gate, int32_t* counts,
                          cudaStream_t s) {
+  // pairs: a fixed grid striding over the device-side count
+  const int dot_blocks = 16 * sm_count();
+  if (dt == MOE_F32)
+    refine_dot_kernel<float><<<dot_blocks, kDotThreads, 0, s>>>(
+        static_cast<const float*>(u), static_cast<const float*>(E), d, N_r, rl);
+  else
+    refine_dot_kernel<__nv_bfloat16><<<dot_blocks, kDotThreads, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(u), static_cast<const __nv_bfloat16*>(E), d, N_r, rl);
+  {
+    const moe_status st = cuda_check(cudaGetLastError(), "refine_dot_kernel launch");
+    if (st != MOE_OK) return st;
+  }
   const int threads = 256;
   int blocks = 2 * sm_count();
   if (blocks > T) blocks = T > 0 ? T : 1;
-  const size_t smem = (size_t)4 * N_r * sizeof(float) + sizeof(int);
+  const size_t smem = (size_t)3 * N_r * sizeof(float);
   if (smem > 48 * 1024) {
     cudaError_t e = dt == MOE_F32
-        ? cudaFuncSetAttribute(refine_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)smem)
-        : cudaFuncSetAttribute(refine_kernel<__nv_bfloat16>,
+        ? cudaFuncSetAttribute(refine_select_kernel<float>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
+        : cudaFuncSetAttribute(refine_select_kernel<__nv_bfloat16>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return cuda_check(e, "refine_kernel smem attribute");
+    if (e != cudaSuccess) return cuda_check(e, "refine_select_kernel smem attribute");
   }
   if (dt == MOE_F32)
-    refine_kernel<float><<<blocks, threads, smem, s>>>(
+    refine_select_kernel<float><<<blocks, threads, smem, s>>>(
         static_cast<const float*>(u), static_cast<const float*>(E), logits, b, d, N_r, K,
-        n_groups, topk_groups, refine, idx, gate, counts);
+        n_groups, topk_groups, rl, idx, gate, counts);
   else
-    refine_kernel<__nv_bfloat16><<<blocks, threads, smem, s>>>(
+    refine_select_kernel<__nv_bfloat16><<<blocks, threads, smem, s>>>(
         static_cast<const __nv_bfloat16*>(u), static_cast<const __nv_bfloat16*>(E), logits, b, d,
-        N_r, K, n_groups, topk_groups, refine, idx, gate, counts);
-  return cuda_check(cudaGetLastError(), "refine_kernel launch");
+        N_r, K, n_groups, topk_groups, rl, idx, gate, counts);
+  return cuda_check(cudaGetLastError(), "refine_select_kernel launch");
 }
 
 moe_status launch_topk(const float* logits, const float* b, int T, int N_r, int K, int n_groups,
                        int topk_groups, int32_t* idx, float* gate, int32_t* counts,
-                       int32_t* refine, float refine_gap, cudaStream_t s) {
+                       RefineLists rl, float refine_gap, cudaStream_t s) {
   const int threads = 256;
   const int wpb = threads / 32;
   int blocks = (T + wpb - 1) / wpb;
@@ -395,7 +469,7 @@ moe_status launch_topk(const float* logits, const float* b, int T, int N_r, int 
   const int V = (N_r + 31) / 32;
 #define MOE_TOPK_CASE(v)                                                                    \
   topk_kernel<v><<<blocks, threads, smem, s>>>(logits, b, T, N_r, K, n_groups, topk_groups, idx, \
-                                               gate, counts, refine, refine_gap);             \
+                                               gate, counts, rl, refine_gap);                 \
   break;
   switch (V <= 1 ? 1 : V <= 2 ? 2 : V <= 4 ? 4 : V <= 8 ? 8 : V <= 16 ? 16 : 32) {
     case 1: MOE_TOPK_CASE(1)

@@ -86,6 +86,66 @@ def test_route_grouped_matches_oracle(T, d, N_r, K, G, M):
     assert max(len(set((r // gsz).tolist())) for r in idx.cpu().numpy()) <= M
 
 
+def _listed_tokens(ws, T, N_r):
+    """Tokens the router sent to its float64 tie-break (white-box: the count
+    is the first word after the float32 logits in the router workspace)."""
+    off = (T * N_r * 4 + 255) // 256 * 256
+    return int(ws[off:off + 4].view(torch.int32)[0])
+
+
+def test_route_v3_width_float64_tie_break():
+    """d = 7168 (V3): float32 tensor-core logits are off by a few 1e-6, so
+    some tokens are decided within the refine gap; routing must still match
+    the float64 oracle."""
+    T, d, N_r, K = 2048, 7168, 256, 8
+    g = _gen(7168)
+    u = _randn((T, d), g, 1.0)
+    E = _randn((N_r, d), g, d ** -0.5)
+    b = ((torch.rand(N_r, generator=g, device=DEV) * 2 - 1) * 0.01).float()
+    idx = torch.empty(T, K, dtype=torch.int32, device=DEV)
+    gate = torch.empty(T, K, dtype=torch.float32, device=DEV)
+    counts = torch.empty(N_r, dtype=torch.int32, device=DEV)
+    ws = _ws(moe.moe_route_workspace_size(T, N_r))
+    moe.moe_route(u, E, b, K, idx, gate, counts, ws)
+    torch.cuda.synchronize()
+    assert _listed_tokens(ws, T, N_r) > 0, "no token reached the float64 tie-break"
+    ref = O.route(f64(u), f64(E), b.cpu().numpy(), K)
+    check_routing(idx.cpu().numpy(), gate.cpu().numpy(), counts.cpu().numpy(), ref, K,
+                  gate_tol=GATE_TOL["bf16"])
+
+
+@pytest.mark.parametrize("grouped", [False, True])
+def test_route_duplicate_centroids_exact_ties(grouped):
+    """Experts 2j and 2j+1 share a centroid and b = 0: every key is tied, every
+    token goes through the float64 tie-break, and ties go to the lower index."""
+    T, d, N_r, K = 600, 512, 64, 6
+    g = _gen(99)
+    u = _randn((T, d), g)
+    E = _randn((N_r // 2, d), g, d ** -0.5).repeat_interleave(2, dim=0).contiguous()
+    b = torch.zeros(N_r, device=DEV)
+    idx = torch.empty(T, K, dtype=torch.int32, device=DEV)
+    gate = torch.empty(T, K, dtype=torch.float32, device=DEV)
+    counts = torch.empty(N_r, dtype=torch.int32, device=DEV)
+    ws = _ws(moe.moe_route_workspace_size(T, N_r))
+    if grouped:
+        moe.moe_route_grouped(u, E, b, K, 8, 3, idx, gate, counts, ws)
+    else:
+        moe.moe_route(u, E, b, K, idx, gate, counts, ws)
+    torch.cuda.synchronize()
+    assert _listed_tokens(ws, T, N_r) == T
+    got = idx.cpu().numpy()
+    if grouped:
+        ref = O.route_grouped(f64(u), f64(E), b.cpu().numpy(), K, 8, 3)
+        check_routing(got, gate.cpu().numpy(), counts.cpu().numpy(),
+                      grouped_reference(ref, K, 8, 3), K, gate_tol=GATE_TOL["bf16"])
+    else:
+        ref = O.route(f64(u), f64(E), b.cpu().numpy(), K)
+        check_routing(got, gate.cpu().numpy(), counts.cpu().numpy(), ref, K,
+                      gate_tol=GATE_TOL["bf16"])
+    # K even: both members of each chosen pair are selected, lower index first
+    assert (got[:, 0::2] % 2 == 0).all() and (got[:, 1::2] == got[:, 0::2] + 1).all()
+
+
 def test_route_zero_centroids_gates_are_uniform():
     """E = 0: s = 1/2 everywhere, selection follows b, gates are exactly 1/K."""
     T, d, N_r, K = 100, 256, 64, 4
@@ -153,6 +213,39 @@ def test_permute_bit_exact(T, d, N_r, K, dtype):
     assert torch.equal(x_perm, u[src])
     if x_scale is not None:
         assert torch.equal(x_scale, u_scale[src])
+
+
+def test_permute_skips_ids_out_of_range():
+    """Pairs whose expert id is outside [0, N_r) are left out: inv_row = -1, no
+    row copied, and the other pairs keep their stable grouped order."""
+    T, d, N_r, K = 300, 128, 32, 4
+    idx_np = _rand_idx(T, N_r, K, 5)
+    rng = np.random.default_rng(6)
+    bad = rng.random((T, K)) < 0.05
+    idx_np[bad] = np.where(rng.random(int(bad.sum())) < 0.5, -1, N_r + 3)
+    u = _randn((T, d), _gen(3))
+    idx = torch.from_numpy(idx_np).to(DEV)
+    x_perm = torch.full((T * K, d), float("nan"), dtype=torch.bfloat16, device=DEV)
+    offsets = torch.empty(N_r + 1, dtype=torch.int32, device=DEV)
+    perm_src = torch.full((T * K,), -5, dtype=torch.int32, device=DEV)
+    inv_row = torch.empty(T, K, dtype=torch.int32, device=DEV)
+    moe.moe_permute(u, idx, N_r, x_perm, offsets, perm_src, inv_row,
+                    _ws(moe.moe_permute_workspace_size(T, N_r)))
+    torch.cuda.synchronize()
+    # brute force over the valid pairs: grouped by expert, tokens ascending
+    pairs = sorted((int(e), t, k) for t in range(T) for k, e in enumerate(idx_np[t])
+                   if 0 <= e < N_r)
+    want_inv = np.full((T, K), -1, np.int64)
+    for r, (e, t, k) in enumerate(pairs):
+        want_inv[t, k] = r
+    want_off = np.searchsorted([p[0] for p in pairs], np.arange(N_r + 1), side="left")
+    np.testing.assert_array_equal(offsets.cpu().numpy(), want_off)
+    np.testing.assert_array_equal(inv_row.cpu().numpy(), want_inv)
+    n = len(pairs)
+    np.testing.assert_array_equal(perm_src.cpu().numpy()[:n], [t for _, t, _ in pairs])
+    src = torch.tensor([t for _, t, _ in pairs], device=DEV)
+    assert torch.equal(x_perm[:n], u[src])
+    assert torch.isnan(x_perm[n:].float()).all()
 
 
 def test_permute_empty_batch():
