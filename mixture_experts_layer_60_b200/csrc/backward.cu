@@ -202,6 +202,11 @@ moe_status launch_combine_backward(const void* dh, const void* u, const void* E,
                                    const int32_t* idx, const float* gate, moe_dtype dt, int T,
                                    int d, int K, void* dy_perm, float* d_gate, float* d_logit,
                                    float* d_logit_perm, cudaStream_t s) {
+  const long long rb = (long long)d * (dt == MOE_F32 ? 4 : 2);
+  if (gather_pipe_supported(GATHER_COMBINE_BWD, 0, K, rb))
+    return launch_gather_pipe(GATHER_COMBINE_BWD, dt, dh, u, nullptr, 0, y_perm,
+                              (long long)T * K, E, inv_row, idx, gate, T, K, rb, dy_perm, d_gate,
+                              d_logit, d_logit_perm, s);
   if (dt == MOE_F32)
     return combine_bwd_dispatch<float>(dh, u, E, y_perm, inv_row, idx, gate, T, d, K, dy_perm,
                                        d_gate, d_logit, d_logit_perm, s);
@@ -234,6 +239,11 @@ moe_status launch_unpermute_backward(const void* dh, const void* dx_shared, int 
                                      const int32_t* idx, const float* d_logit, const void* E,
                                      moe_dtype dt, int T, int d, int K, void* du,
                                      cudaStream_t s) {
+  const long long rb = (long long)d * (dt == MOE_F32 ? 4 : 2);
+  if (gather_pipe_supported(GATHER_UNPERM_BWD, N_s, K, rb))
+    return launch_gather_pipe(GATHER_UNPERM_BWD, dt, dh, nullptr, dx_shared, N_s, dx_perm,
+                              (long long)T * K, E, inv_row, idx, d_logit, T, K, rb, du, nullptr,
+                              nullptr, nullptr, s);
   if (dt == MOE_F32)
     return unpermute_bwd_dispatch<float>(dh, dx_shared, N_s, dx_perm, inv_row, idx, d_logit, E,
                                          T, d, K, du, s);

@@ -41,6 +41,7 @@ enum : int {
   ERR_GEMM_TIMEOUT = 1,       // tcgen05 GEMM: an mbarrier wait ran out
   ERR_GEMM_FP8_TIMEOUT = 2,   // FP8 tcgen05 GEMM: an mbarrier wait ran out
   ERR_EP_BOUNDS = 4,          // expert-parallel copy: a row position past its buffer (skipped)
+  ERR_GATHER_TIMEOUT = 8,     // row-gather pipeline (combine and its backward): a wait ran out
 };
 
 // ---------------------------------------------------------------- device side

@@ -1,0 +1,404 @@
+// Row-gather pipeline for the per-token kernels that read K routed rows from
+// random places in the grouped buffers (the combine of the h'-equation of
+// "DeepSeek-V3 技術報告", section 方法 / 2, and its backward).  These kernels
+// move whole 16-byte-aligned rows and do a few FMAs per element, so they are
+// bound by how many bytes each SM keeps in flight: here one producer warp
+// stages every row a step needs into shared memory with bulk asynchronous
+// copies (a ring of stages, ~180 KB per SM), and four consumer warps do the
+// arithmetic from shared memory.
+//
+// A job is (token t, column chunk q of 2 KB, or 1 KB / 512 B when a stage of
+// many rows would leave fewer than four stages).  Tokens go in groups of four, one
+// per consumer warp, and a group's jobs are ordered chunk-major, so the four
+// warps work side by side and every per-token reduction stays inside one warp
+// (no block-wide barrier after the start).  Every wait is bounded (1 s) and
+// reported through the device error word.
+//
+// Row slots of a job, by mode:
+//   COMBINE      u_t, ys_j[t] (N_s), y_perm[r_k] (K)            -> h'_t
+//   COMBINE_BWD  dh_t, u_t, y_perm[r_k] (K), e_idx(t,k) (K)      -> dy_perm[r_k], d_gate, d_logit
+//   UNPERM_BWD   dh_t, dxs_j[t] (N_s), dx_perm[r_k] (K), e_k (K) -> du_t
+// Sums are float32 in the same order as the per-warp kernels (residual or
+// upstream row, shared rows j ascending, routed rows k ascending, centroid
+// terms k ascending).  A slot whose grouped row lies outside [0, n_perm) is
+// left out.
+#include "launch.h"
+#include "sm100.cuh"
+
+namespace moe {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kMaxChunk = 2048;              // bytes of a row per job (2048, 1024 or 512)
+constexpr int kConsumerWarps = 4;            // one token of a group each
+constexpr int kThreads = 32 * (kConsumerWarps + 1);
+constexpr int kSmemBudget = 200 * 1024;
+constexpr int kMaxStages = 8;
+constexpr int kMaxSlots = 48;
+constexpr uint64_t kWaitNs = 1000000000ull;
+
+struct GatherParams {
+  const uint8_t* a;          // u (COMBINE) or dh (backward): row t
+  const uint8_t* b;          // u (COMBINE_BWD): row t
+  const uint8_t* sh;         // shared-expert rows [N_s][T] (ys or dxs)
+  int N_s;
+  const uint8_t* perm;       // grouped rows (y_perm or dx_perm)
+  long long n_perm;          // rows of perm
+  const uint8_t* cent;       // centroids E [N_r][d] (backward)
+  const int32_t* inv_row;    // [T, K]
+  const int32_t* idx;        // [T, K]
+  const float* w;            // gate (COMBINE, COMBINE_BWD) or d_logit (UNPERM_BWD) [T, K]
+  int T, K;
+  long long row_bytes;
+  uint8_t* out;              // h' / dy_perm / du
+  float* d_gate;             // COMBINE_BWD outputs
+  float* d_logit;
+  float* d_logit_perm;
+  int chunk;                 // bytes of a row per job
+  int stages;                // >= kConsumerWarps (see the ring below)
+  int* err;
+};
+
+__host__ __device__ inline int slots_of(int mode, int N_s, int K) {
+  return mode == GATHER_COMBINE ? 1 + N_s + K : mode == GATHER_COMBINE_BWD ? 2 + 2 * K
+                                                                           : 1 + N_s + 2 * K;
+}
+
+// Source row of slot `s` of token t, or nullptr (slot unused or row left out).
+template <int MODE>
+__device__ __forceinline__ const uint8_t* slot_row(const GatherParams& p, int t, int s) {
+  const int K = p.K, N_s = p.N_s;
+  const size_t rb = (size_t)p.row_bytes;
+  if (s == 0) return p.a + (size_t)t * rb;
+  if (MODE == GATHER_COMBINE_BWD) {
+    if (s == 1) return p.b + (size_t)t * rb;
+    s -= 2;
+  } else {
+    if (s <= N_s) return p.sh + ((size_t)(s - 1) * p.T + t) * rb;
+    s -= 1 + N_s;
+  }
+  if (s < K) {
+    const int r = p.inv_row[(size_t)t * K + s];
+    return (r >= 0 && r < p.n_perm) ? p.perm + (size_t)r * rb : nullptr;
+  }
+  s -= K;
+  if (MODE != GATHER_COMBINE && s < K) return p.cent + (size_t)p.idx[(size_t)t * K + s] * rb;
+  return nullptr;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+template <int MODE, typename E, int KMAX>
+__global__ void __launch_bounds__(kThreads, 1) gather_pipe_kernel(const GatherParams p) {
+  constexpr int N = Vec<E>::N;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* buf = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~static_cast<uintptr_t>(127));
+  const int K = p.K, N_s = p.N_s, S = p.stages, CH = p.chunk;
+  const int R = slots_of(MODE, N_s, K);
+  const int stage_bytes = R * CH;
+  uint64_t* full = reinterpret_cast<uint64_t*>(buf + (size_t)S * stage_bytes);
+  uint64_t* empty = full + S;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + S);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const int Q = (int)((p.row_bytes + CH - 1) / CH);
+  const int n_groups = (p.T + kConsumerWarps - 1) / kConsumerWarps;
+
+  if (warp == kConsumerWarps) {
+    // ---------------------------------------------------------------- producer
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int g = blockIdx.x; g < n_groups && ok; g += gridDim.x) {
+      // this lane's slots (lane, lane + 32) of the group's four tokens
+      const uint8_t* src[kConsumerWarps][2];
+      int nvalid[kConsumerWarps];
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) {
+        const int t = g * kConsumerWarps + w;
+        const bool tv = t < p.T;
+        src[w][0] = tv && lane < R ? slot_row<MODE>(p, t, lane) : nullptr;
+        src[w][1] = tv && lane + 32 < R ? slot_row<MODE>(p, t, lane + 32) : nullptr;
+        nvalid[w] = __popc(__ballot_sync(0xffffffffu, src[w][0] != nullptr)) +
+                    __popc(__ballot_sync(0xffffffffu, src[w][1] != nullptr));
+      }
+      for (int q = 0; q < Q && ok; ++q) {
+        const uint32_t cb = (uint32_t)min((long long)CH, p.row_bytes - (long long)q * CH);
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) {
+          bool got = true;
+          if (lane == 0) got = mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, kWaitNs);
+          got = __shfl_sync(0xffffffffu, got, 0);
+          if (!got) {
+            if (lane == 0) { *abort_flag = 1; atomicOr(p.err, ERR_GATHER_TIMEOUT); }
+            ok = false;
+            break;
+          }
+          if (lane == 0) mbar_arrive_expect_tx(&full[stage], (uint32_t)nvalid[w] * cb);
+          __syncwarp();
+          uint8_t* dst = buf + (size_t)stage * stage_bytes;
+          const size_t off = (size_t)q * CH;
+          if (src[w][0]) bulk_load(dst + lane * CH, src[w][0] + off, cb, &full[stage]);
+          if (src[w][1]) bulk_load(dst + (lane + 32) * CH, src[w][1] + off, cb, &full[stage]);
+          if (++stage == S) { stage = 0; phase ^= 1; }
+        }
+      }
+    }
+    // drain: every stage filled has been released by its consumer, so no
+    // copy is still writing shared memory
+    if (lane == 0)
+      for (int s = 0; s < S; ++s) {
+        mbar_wait_bounded(&empty[stage], phase ^ 1, nullptr, kWaitNs);
+        if (++stage == S) { stage = 0; phase ^= 1; }
+      }
+  } else {
+    // ---------------------------------------------------------------- consumers
+    // warp w takes token w of every group; in a group its job of chunk q is
+    // number 4q + w, so it skips the other warps' jobs in the ring.  When it
+    // waits for job m, its previous job m - 4 was filled, hence so was every
+    // job up to m - 4 >= m - S: the stage's barrier is at most one phase
+    // behind, and the parity wait cannot pass on an older phase.
+    long long n = warp;                 // ring position of this warp's next job
+    for (int g = blockIdx.x; g < n_groups; g += gridDim.x) {
+      const int t = g * kConsumerWarps + warp;
+      const bool tv = t < p.T;
+      int rows[KMAX];
+      float wk[KMAX], dg[KMAX], lg[KMAX];
+#pragma unroll
+      for (int k = 0; k < KMAX; ++k) {
+        rows[k] = -1;
+        wk[k] = 0.f;
+        dg[k] = 0.f;
+        lg[k] = 0.f;
+        if (tv && k < K) {
+          const int r = p.inv_row[(size_t)t * K + k];
+          rows[k] = (r >= 0 && r < p.n_perm) ? r : -1;
+          wk[k] = p.w[(size_t)t * K + k];
+        }
+      }
+      bool ok = true;
+      for (int q = 0; q < Q; ++q, n += kConsumerWarps) {
+        const int stage = (int)(n % S);
+        const uint32_t phase = (uint32_t)((n / S) & 1);
+        const bool got = mbar_wait_bounded(&full[stage], phase, abort_flag, kWaitNs);
+        if (!__all_sync(0xffffffffu, got)) {
+          if (lane == 0) { *abort_flag = 1; atomicOr(p.err, ERR_GATHER_TIMEOUT); }
+          ok = false;
+          break;
+        }
+        if (tv) {
+          const uint8_t* st = buf + (size_t)stage * stage_bytes;
+          const long long cb = min((long long)CH, p.row_bytes - (long long)q * CH);
+#pragma unroll
+          for (int m = 0; m < kMaxChunk / 512; ++m) {
+            const int cbyte = m * 512 + lane * 16;
+            if (cbyte >= cb) break;
+            const size_t gcol = (size_t)q * CH + cbyte;   // byte offset inside a row
+            auto row = [&](int slot) {
+              return *reinterpret_cast<const uint4*>(st + slot * CH + cbyte);
+            };
+            float acc[N], tmp[N];
+            if (MODE == GATHER_COMBINE) {
+              Vec<E>::load(row(0), acc);
+              for (int j = 0; j < N_s; ++j) {
+                Vec<E>::load(row(1 + j), tmp);
+#pragma unroll
+                for (int i = 0; i < N; ++i) acc[i] += tmp[i];
+              }
+#pragma unroll
+              for (int k = 0; k < KMAX; ++k) {
+                if (k < K && rows[k] >= 0) {
+                  Vec<E>::load(row(1 + N_s + k), tmp);
+#pragma unroll
+                  for (int i = 0; i < N; ++i) acc[i] = fmaf(wk[k], tmp[i], acc[i]);
+                }
+              }
+              *reinterpret_cast<uint4*>(p.out + (size_t)t * p.row_bytes + gcol) =
+                  Vec<E>::store(acc);
+            } else if (MODE == GATHER_COMBINE_BWD) {
+              float fd[N], fu[N];
+              Vec<E>::load(row(0), fd);
+              Vec<E>::load(row(1), fu);
+#pragma unroll
+              for (int k = 0; k < KMAX; ++k) {
+                if (k < K) {
+                  if (rows[k] >= 0) {
+                    Vec<E>::load(row(2 + k), tmp);
+#pragma unroll
+                    for (int i = 0; i < N; ++i) dg[k] = fmaf(fd[i], tmp[i], dg[k]);
+#pragma unroll
+                    for (int i = 0; i < N; ++i) tmp[i] = wk[k] * fd[i];
+                    *reinterpret_cast<uint4*>(p.out + (size_t)rows[k] * p.row_bytes + gcol) =
+                        Vec<E>::store(tmp);
+                  }
+                  Vec<E>::load(row(2 + K + k), tmp);
+#pragma unroll
+                  for (int i = 0; i < N; ++i) lg[k] = fmaf(fu[i], tmp[i], lg[k]);
+                }
+              }
+            } else {
+              Vec<E>::load(row(0), acc);
+              for (int j = 0; j < N_s; ++j) {
+                Vec<E>::load(row(1 + j), tmp);
+#pragma unroll
+                for (int i = 0; i < N; ++i) acc[i] += tmp[i];
+              }
+#pragma unroll
+              for (int k = 0; k < KMAX; ++k) {
+                if (k < K && rows[k] >= 0) {
+                  Vec<E>::load(row(1 + N_s + k), tmp);
+#pragma unroll
+                  for (int i = 0; i < N; ++i) acc[i] += tmp[i];
+                }
+              }
+#pragma unroll
+              for (int k = 0; k < KMAX; ++k) {
+                if (k < K) {
+                  Vec<E>::load(row(1 + N_s + K + k), tmp);
+#pragma unroll
+                  for (int i = 0; i < N; ++i) acc[i] = fmaf(wk[k], tmp[i], acc[i]);
+                }
+              }
+              *reinterpret_cast<uint4*>(p.out + (size_t)t * p.row_bytes + gcol) =
+                  Vec<E>::store(acc);
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[stage]);
+      }
+      if (!ok) break;
+      if (MODE == GATHER_COMBINE_BWD && tv) {
+        // the token's gate and affinity gradients (selection held fixed):
+        //   ds_k = (dg_k - sum_j g_j dg_j) / sum_j s_j,  dlogit_k = ds_k s_k (1 - s_k)
+#pragma unroll
+        for (int k = 0; k < KMAX; ++k) {
+          if (k < K) {
+            dg[k] = warp_sum(dg[k]);
+            lg[k] = warp_sum(lg[k]);
+          }
+        }
+        if (lane == 0) {
+          float S_sum = 0.f, gdg = 0.f, sk[KMAX];
+#pragma unroll
+          for (int k = 0; k < KMAX; ++k) {
+            if (k < K) {
+              sk[k] = 1.0f / (1.0f + expf(-lg[k]));
+              S_sum += sk[k];
+              gdg = fmaf(wk[k], dg[k], gdg);
+            }
+          }
+#pragma unroll
+          for (int k = 0; k < KMAX; ++k) {
+            if (k < K) {
+              const float ds = (dg[k] - gdg) / S_sum;
+              const float dl = ds * sk[k] * (1.0f - sk[k]);
+              p.d_gate[(size_t)t * K + k] = dg[k];
+              p.d_logit[(size_t)t * K + k] = dl;
+              if (rows[k] >= 0) p.d_logit_perm[rows[k]] = dl;
+            }
+          }
+        }
+      }
+    }
+  }
+}
+
+template <int MODE, typename E, int KMAX>
+moe_status pipe_launch(const GatherParams& p, size_t smem, int grid, cudaStream_t s) {
+  auto kern = gather_pipe_kernel<MODE, E, KMAX>;
+  static bool attr_done[kMaxSmemDevices] = {};
+  // the attribute is set once per device: always the whole budget
+  const moe_status st = ensure_max_smem(reinterpret_cast<const void*>(kern), kSmemBudget,
+                                        attr_done, "gather pipeline smem attribute");
+  if (st != MOE_OK) return st;
+  kern<<<grid, kThreads, smem, s>>>(p);
+  return cuda_check(cudaGetLastError(), "gather pipeline launch");
+}
+
+template <int MODE, typename E>
+moe_status pipe_dispatch(const GatherParams& p, size_t smem, int grid, cudaStream_t s) {
+  if (p.K <= 8) return pipe_launch<MODE, E, 8>(p, smem, grid, s);
+  return pipe_launch<MODE, E, 16>(p, smem, grid, s);
+}
+
+}  // namespace
+
+bool gather_pipe_supported(int mode, int N_s, int K, long long row_bytes) {
+  return K >= 1 && K <= 16 && N_s >= 0 && row_bytes > 0 && row_bytes % 16 == 0 &&
+         slots_of(mode, N_s, K) <= kMaxSlots;
+}
+
+moe_status launch_gather_pipe(int mode, moe_dtype dt, const void* a, const void* b,
+                              const void* sh, int N_s, const void* perm, long long n_perm,
+                              const void* cent, const int32_t* inv_row, const int32_t* idx,
+                              const float* w, int T, int K, long long row_bytes, void* out,
+                              float* d_gate, float* d_logit, float* d_logit_perm,
+                              cudaStream_t s) {
+  if (T <= 0) return MOE_OK;
+  GatherParams p;
+  p.a = static_cast<const uint8_t*>(a);
+  p.b = static_cast<const uint8_t*>(b);
+  p.sh = static_cast<const uint8_t*>(sh);
+  p.N_s = N_s;
+  p.perm = static_cast<const uint8_t*>(perm);
+  p.n_perm = n_perm;
+  p.cent = static_cast<const uint8_t*>(cent);
+  p.inv_row = inv_row;
+  p.idx = idx;
+  p.w = w;
+  p.T = T;
+  p.K = K;
+  p.row_bytes = row_bytes;
+  p.out = static_cast<uint8_t*>(out);
+  p.d_gate = d_gate;
+  p.d_logit = d_logit;
+  p.d_logit_perm = d_logit_perm;
+  p.err = device_error_word();
+  if (!p.err) return fail(MOE_ERR_CUDA, "device error word unavailable");
+  // the largest chunk that leaves room for kConsumerWarps stages
+  const int R = slots_of(mode, N_s, K);
+  int chunk = kMaxChunk, stages = 0;
+  for (; chunk >= 512; chunk /= 2) {
+    stages = (kSmemBudget - 1024) / (R * chunk);
+    if (stages >= kConsumerWarps) break;
+  }
+  if (stages < kConsumerWarps)
+    return fail(MOE_ERR_UNSUPPORTED, "gather pipeline: %d row slots", R);
+  if (stages > kMaxStages) stages = kMaxStages;
+  const int stage_bytes = R * chunk;
+  p.chunk = chunk;
+  p.stages = stages;
+  const size_t smem = 128 + (size_t)stages * stage_bytes + (size_t)stages * 16 + 16;
+  if (smem > (size_t)kSmemBudget) return fail(MOE_ERR_UNSUPPORTED, "gather pipeline: smem");
+  const int n_groups = (T + kConsumerWarps - 1) / kConsumerWarps;
+  int grid = sm_count();
+  if (grid > n_groups) grid = n_groups;
+  const bool f32 = dt == MOE_F32;
+  switch (mode) {
+    case GATHER_COMBINE:
+      return f32 ? pipe_dispatch<GATHER_COMBINE, float>(p, smem, grid, s)
+                 : pipe_dispatch<GATHER_COMBINE, __nv_bfloat16>(p, smem, grid, s);
+    case GATHER_COMBINE_BWD:
+      return f32 ? pipe_dispatch<GATHER_COMBINE_BWD, float>(p, smem, grid, s)
+                 : pipe_dispatch<GATHER_COMBINE_BWD, __nv_bfloat16>(p, smem, grid, s);
+    case GATHER_UNPERM_BWD:
+      return f32 ? pipe_dispatch<GATHER_UNPERM_BWD, float>(p, smem, grid, s)
+                 : pipe_dispatch<GATHER_UNPERM_BWD, __nv_bfloat16>(p, smem, grid, s);
+  }
+  return fail(MOE_ERR_INVALID_ARG, "gather pipeline: mode %d", mode);
+}
+
+}  // namespace moe

@@ -79,6 +79,20 @@ moe_status launch_ws_gemm_ex(const void* X, const void* W, int b_rows_per_group,
                              WsEpi epi, bool w_mn, void* C, int ldc, void* S, int lds,
                              cudaStream_t s);
 
+// gather.cu ------------------------------------------------------------------
+// Row-gather pipeline (bulk copies into a shared-memory ring, one producer
+// warp, four consumer warps) for the per-token combine kernels.
+enum GatherMode { GATHER_COMBINE = 0, GATHER_COMBINE_BWD = 1, GATHER_UNPERM_BWD = 2 };
+bool gather_pipe_supported(int mode, int N_s, int K, long long row_bytes);
+// a: u (COMBINE) or dh; b: u (COMBINE_BWD); sh: shared-expert rows [N_s][T];
+// perm: grouped rows (n_perm of them); cent: centroids; w: gate or d_logit.
+moe_status launch_gather_pipe(int mode, moe_dtype dt, const void* a, const void* b,
+                              const void* sh, int N_s, const void* perm, long long n_perm,
+                              const void* cent, const int32_t* inv_row, const int32_t* idx,
+                              const float* w, int T, int K, long long row_bytes, void* out,
+                              float* d_gate, float* d_logit, float* d_logit_perm,
+                              cudaStream_t s);
+
 // gemm_wgrad.cu --------------------------------------------------------------
 // C[g] [M, N] = sum over the rows r of group g of A[r, :]^T B[r, :] (bf16 in and out).
 // A_tail: scratch of wgrad_tail_bytes(M * 2, 64, groups) bytes for the groups'

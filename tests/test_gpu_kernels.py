@@ -7,6 +7,7 @@ import pytest
 import torch
 
 import mixture_experts_layer_60_b200 as moe
+from oracle import moe_backward as B
 from oracle import moe_oracle as O
 from tests.harness import (GATE_TOL, TOL, LazyExperts, assert_close, check_routing, f64,
                            grouped_reference)
@@ -321,6 +322,9 @@ def test_expert_ffn_f32(sizes, d, I):
 @pytest.mark.parametrize("T,d,K,N_s,dtype", [
     (1000, 512, 6, 2, torch.bfloat16), (333, 256, 8, 1, torch.bfloat16),
     (200, 128, 4, 0, torch.float32), (64, 256, 17, 1, torch.bfloat16),
+    (77, 7168, 8, 1, torch.bfloat16),     # V3 row: seven 2 KB chunks, a partial token group
+    (130, 1536, 16, 3, torch.bfloat16),   # K = 16, ragged last chunk (3072 B rows)
+    (50, 2560, 16, 2, torch.float32),     # float32 rows of five chunks
 ])
 def test_combine(T, d, K, N_s, dtype):
     g = _gen(T + K)
@@ -338,6 +342,83 @@ def test_combine(T, d, K, N_s, dtype):
     ref = ref + np.einsum("tk,tkd->td", f64(gate), f64(yp)[inv.long().cpu().numpy()])
     tol = TOL["f32"] if dtype == torch.float32 else 2 ** -8
     assert_close(f64(out), ref, tol, "h'")
+
+
+def test_combine_skips_rows_left_out():
+    """A slot whose grouped row is -1 (an expert id the permute left out)
+    contributes nothing."""
+    T, d, K = 90, 1024, 8
+    g = _gen(5)
+    u = _randn((T, d), g)
+    yp = _randn((T * K, d), g, 0.5)
+    inv = torch.randperm(T * K, generator=torch.Generator().manual_seed(1)).view(T, K)
+    inv[::7, 3] = -1
+    inv = inv.to(torch.int32).to(DEV)
+    gate = torch.rand(T, K, generator=g, device=DEV)
+    out = torch.empty(T, d, dtype=torch.bfloat16, device=DEV)
+    moe.moe_combine(u, None, yp, inv, gate, out)
+    torch.cuda.synchronize()
+    iv = inv.long().cpu().numpy()
+    w = np.where(iv >= 0, f64(gate), 0.0)
+    ref = f64(u) + np.einsum("tk,tkd->td", w, f64(yp)[np.maximum(iv, 0)])
+    assert_close(f64(out), ref, 2 ** -8, "h'")
+
+
+def _bwd_case(T, d, K, N_s, dtype, seed):
+    g = _gen(seed)
+    N_r = 3 * K
+    u = _randn((T, d), g, 1.0, dtype)
+    E = _randn((N_r, d), g, d ** -0.5, dtype)
+    dh = _randn((T, d), g, 0.1, dtype)
+    yp = _randn((T * K, d), g, 0.5, dtype)
+    dxp = _randn((T * K, d), g, 0.1, dtype)
+    dxs = _randn((N_s, T, d), g, 0.1, dtype) if N_s else None
+    rng = np.random.default_rng(seed)
+    idx = np.stack([rng.choice(N_r, K, replace=False) for _ in range(T)]).astype(np.int32)
+    inv = rng.permutation(T * K).reshape(T, K).astype(np.int32)
+    # gates as the router makes them: g = s / sum(s) over the selected experts
+    s_sel = B.sigmoid(np.einsum("td,tkd->tk", f64(u), f64(E)[idx]))
+    gate = torch.from_numpy(s_sel / s_sel.sum(1, keepdims=True)).float().to(DEV)
+    return u, E, dh, yp, dxp, dxs, idx, inv, gate
+
+
+@pytest.mark.parametrize("T,d,K,N_s,dtype", [
+    (77, 7168, 8, 1, torch.bfloat16),     # V3 rows, a partial token group
+    (130, 1536, 16, 2, torch.bfloat16),   # K = 16, ragged last chunk
+    (45, 2560, 16, 0, torch.float32),
+    (333, 256, 6, 3, torch.float32),      # rows shorter than one chunk
+    (64, 256, 3, 1, torch.bfloat16),      # small K
+])
+def test_combine_and_unpermute_backward(T, d, K, N_s, dtype):
+    """moe_combine_backward and moe_unpermute_backward against the chain rule
+    written out with the oracle's gate backward (selection held fixed)."""
+    u, E, dh, yp, dxp, dxs, idx, inv, gate = _bwd_case(T, d, K, N_s, dtype, T + d + K)
+    idx_d = torch.from_numpy(idx).to(DEV)
+    inv_d = torch.from_numpy(inv).to(DEV)
+    dyp = torch.full((T * K, d), float("nan"), dtype=dtype, device=DEV)
+    d_gate = torch.empty(T, K, device=DEV)
+    d_logit = torch.empty(T, K, device=DEV)
+    d_logit_perm = torch.empty(T * K, device=DEV)
+    moe.moe_combine_backward(dh, u, E, yp, inv_d, idx_d, gate, dyp, d_gate, d_logit, d_logit_perm)
+    du = torch.empty(T, d, dtype=dtype, device=DEV)
+    moe.moe_unpermute_backward(dh, dxs, dxp, inv_d, idx_d, d_logit, E, du)
+    torch.cuda.synchronize()
+    tol = TOL["f32"] if dtype == torch.float32 else TOL["bf16"]
+    g64, dh64, ys = f64(gate), f64(dh), f64(yp)
+    want_dyp = np.zeros((T * K, d))
+    want_dyp[inv] = g64[:, :, None] * dh64[:, None, :]
+    assert_close(f64(dyp), want_dyp, tol, "dy_perm")
+    want_dg = np.einsum("td,tkd->tk", dh64, ys[inv])
+    assert_close(d_gate.double().cpu().numpy(), want_dg, tol, "d_gate")
+    s_sel = B.sigmoid(np.einsum("td,tkd->tk", f64(u), f64(E)[idx]))
+    want_dl = B.gate_backward(s_sel, want_dg) * s_sel * (1 - s_sel)
+    assert_close(d_logit.double().cpu().numpy(), want_dl, tol, "d_logit")
+    assert_close(d_logit_perm.double().cpu().numpy()[inv], want_dl, tol, "d_logit_perm")
+    dl = d_logit.double().cpu().numpy()
+    want_du = dh64 + (f64(dxs).sum(0) if N_s else 0) + f64(dxp)[inv].sum(1) + \
+        np.einsum("tk,tkd->td", dl, f64(E)[idx])
+    assert_close(f64(du), want_du, tol, "du")
+    assert moe.moe_device_status() == 0
 
 
 def test_bias_update_bit_exact():
