@@ -116,10 +116,11 @@ MEASURED_GATE_UP_TRAFFIC = {
 
 
 def gpu_launches_per_step(cfg):
-    # route: logits GEMM + top-K + float64 tie-break pass; permute: histogram,
-    # scan, rank, scatter; routed FFN: gate/up + down; shared FFN: 2 each;
-    # combine: 1; bias update: 1; FP8: + activation quantiser
-    n = 3 + 4 + 2 + 2 * cfg.N_s + 1 + 1
+    # route: logits GEMM + top-K + float64 tie-break (pair dot products, then
+    # re-selection); permute: histogram, scan, rank, scatter; routed FFN:
+    # gate/up + down; shared FFN: 2 each; combine: 1; bias update: 1;
+    # FP8: + activation quantiser
+    n = 4 + 4 + 2 + 2 * cfg.N_s + 1 + 1
     if cfg.dtype == "e4m3":
         n += 1
     return n

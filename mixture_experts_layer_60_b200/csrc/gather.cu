@@ -8,7 +8,7 @@
 // arithmetic from shared memory.
 //
 // A job is (token t, column chunk q of 2 KB, or 1 KB / 512 B when a stage of
-// many rows would leave fewer than four stages).  Tokens go in groups of four, one
+// many rows would leave fewer than eight stages).  Tokens go in groups of four, one
 // per consumer warp, and a group's jobs are ordered chunk-major, so the four
 // warps work side by side and every per-token reduction stays inside one warp
 // (no block-wide barrier after the start).  Every wait is bounded (1 s) and
@@ -57,7 +57,7 @@ struct GatherParams {
   float* d_logit;
   float* d_logit_perm;
   int chunk;                 // bytes of a row per job
-  int stages;                // >= kConsumerWarps (see the ring below)
+  int stages;                // a multiple of kConsumerWarps (see the ring below)
   int* err;
 };
 
@@ -166,10 +166,11 @@ __global__ void __launch_bounds__(kThreads, 1) gather_pipe_kernel(const GatherPa
   } else {
     // ---------------------------------------------------------------- consumers
     // warp w takes token w of every group; in a group its job of chunk q is
-    // number 4q + w, so it skips the other warps' jobs in the ring.  When it
-    // waits for job m, its previous job m - 4 was filled, hence so was every
-    // job up to m - 4 >= m - S: the stage's barrier is at most one phase
-    // behind, and the parity wait cannot pass on an older phase.
+    // number 4q + w, so it skips the other warps' jobs in the ring.  S is a
+    // multiple of kConsumerWarps, so job n's stage n % S is only ever used by
+    // warp n % 4: each stage has one consumer, which takes its jobs in ring
+    // order (the one-producer, one-consumer ring: a stage's barrier is never
+    // more than one phase away from the job its consumer waits for).
     long long n = warp;                 // ring position of this warp's next job
     for (int g = blockIdx.x; g < n_groups; g += gridDim.x) {
       const int t = g * kConsumerWarps + warp;
@@ -368,16 +369,18 @@ moe_status launch_gather_pipe(int mode, moe_dtype dt, const void* a, const void*
   p.d_logit_perm = d_logit_perm;
   p.err = device_error_word();
   if (!p.err) return fail(MOE_ERR_CUDA, "device error word unavailable");
-  // the largest chunk that leaves room for kConsumerWarps stages
+  // a multiple of kConsumerWarps stages (one consumer warp per stage): the
+  // largest chunk that fits kMaxStages of them, else the largest with four
   const int R = slots_of(mode, N_s, K);
-  int chunk = kMaxChunk, stages = 0;
-  for (; chunk >= 512; chunk /= 2) {
-    stages = (kSmemBudget - 1024) / (R * chunk);
-    if (stages >= kConsumerWarps) break;
+  int chunk = 0, stages = 0;
+  for (int c = kMaxChunk; c >= 512; c /= 2) {
+    int st = (kSmemBudget - 1024) / (R * c) / kConsumerWarps * kConsumerWarps;
+    if (st > kMaxStages) st = kMaxStages;
+    if (st > stages) { stages = st; chunk = c; }
+    if (stages == kMaxStages) break;
   }
   if (stages < kConsumerWarps)
     return fail(MOE_ERR_UNSUPPORTED, "gather pipeline: %d row slots", R);
-  if (stages > kMaxStages) stages = kMaxStages;
   const int stage_bytes = R * chunk;
   p.chunk = chunk;
   p.stages = stages;
