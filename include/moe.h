@@ -185,7 +185,8 @@ moe_status moe_expert_down(const void* h, const float* h_scale, const int32_t* o
  *   u         [T, d]       device, dt (MOE_F32 or MOE_BF16)
  *   y_shared  [N_s, T, d]  device, dt (may be NULL when N_s == 0)
  *   y_perm    [T*K, d]     device, dt: routed expert outputs in grouped order
- *   inv_row   [T, K]       device, int32: from moe_permute
+ *   inv_row   [T, K]       device, int32: from moe_permute (a slot outside
+ *                          [0, T*K), e.g. -1, adds nothing)
  *   topk_gate [T, K]       device, float32: from moe_route
  *   h_out     [T, d]       device, dt out (must not alias the inputs)
  * Requires d * sizeof(dt) % 16 == 0.
@@ -288,6 +289,8 @@ moe_status moe_expert_gate_up_save(const void* x, const float* x_scale, const in
  *   MOE_BF16); inv_row, topk_idx [T, K] int32 and topk_gate [T, K] float32
  *   from the forward; dy_perm [T*K, d] dt out; d_gate, d_logit [T, K] and
  *   d_logit_perm [T*K] float32 out.  K <= 16, d * sizeof(dt) % 16 == 0.
+ *   A slot whose inv_row lies outside [0, T*K) is left out (no dy_perm row
+ *   written, no d_logit_perm entry, no d_gate contribution).
  * The shared experts' upstream gradient is dh_out itself (weight 1).
  * ------------------------------------------------------------------------ */
 moe_status moe_combine_backward(const void* dh_out, const void* u, const void* E,
@@ -359,7 +362,9 @@ moe_status moe_expert_ffn_backward(const void* x, const int32_t* x_rows, const i
  *           + sum_k d_logit[t,k] E[topk_idx[t,k]]
  * summed in float32 in that order, rounded once to dt.  dh_out, du [T, d];
  * dx_shared [N_s, T, d] (NULL when N_s == 0); dx_perm [T*K, d]; E [N_r, d]:
- * device, dt (MOE_F32 or MOE_BF16).  K <= 16, d * sizeof(dt) % 16 == 0.
+ * device, dt (MOE_F32 or MOE_BF16).  K <= 16, N_s + 2K <= 63,
+ * d * sizeof(dt) % 16 == 0.  A slot whose inv_row lies outside [0, T*K) is
+ * left out of the sum.
  * ------------------------------------------------------------------------ */
 moe_status moe_unpermute_backward(const void* dh_out, const void* dx_shared, int N_s,
                                   const void* dx_perm, const int32_t* inv_row,
@@ -430,7 +435,11 @@ moe_status moe_ep_return(const void* y, moe_dtype dt, const void* recv_tags,
 /* ------------------------------------------------------------------------
  * moe_device_status - synchronises the current device, then returns (and
  * clears) the library's device-side error word: 0 if no kernel gave up a
- * bounded wait since the last call, else a bit set naming the kernel.
+ * bounded wait since the last call, else a bit set naming the kernel:
+ *   1  a tcgen05 bf16 GEMM (expert FFN, router logits, Wgrad)
+ *   2  an FP8 tcgen05 GEMM
+ *   4  an expert-parallel copy skipped a row position past its buffer
+ *   8  the row-gather pipeline (combine, combine and unpermute backward)
  * ------------------------------------------------------------------------ */
 moe_status moe_device_status(int* flags);
 

@@ -609,6 +609,8 @@ moe_status moe_unpermute_backward(const void* dh_out, const void* dx_shared, int
   clear_last_error();
   MOE_TRY(check_rowwise("moe_unpermute_backward", dt, T, d, K));
   MOE_REQUIRE(N_s >= 0, MOE_ERR_INVALID_ARG, "moe_unpermute_backward: N_s=%d", N_s);
+  MOE_REQUIRE(N_s + 2 * K <= 63, MOE_ERR_UNSUPPORTED,
+              "moe_unpermute_backward: N_s + 2K = %d exceeds 63", N_s + 2 * K);
   if (T == 0) return MOE_OK;
   MOE_REQUIRE(dh_out && dx_perm && inv_row && topk_idx && d_logit && E && du &&
                   (N_s == 0 || dx_shared),

@@ -36,7 +36,7 @@ constexpr int kConsumerWarps = 4;            // one token of a group each
 constexpr int kThreads = 32 * (kConsumerWarps + 1);
 constexpr int kSmemBudget = 200 * 1024;
 constexpr int kMaxStages = 8;
-constexpr int kMaxSlots = 48;
+constexpr int kMaxSlots = 64;              // two per producer lane
 constexpr uint64_t kWaitNs = 1000000000ull;
 
 struct GatherParams {

@@ -160,6 +160,9 @@ def test_backward_argument_errors(L):
     assert L.moe_combine_backward(d, d, None, d, d, d, d, 1, 8, 64, 4, d, d, d, d, None) == 1
     assert L.moe_unpermute_backward(d, None, 1, d, d, d, d, d, 1, 8, 64, 4, d, None) == 1
     assert L.moe_unpermute_backward(d, d, 1, d, d, d, d, d, 2, 8, 64, 4, d, None) == 2
+    # row slots of the gather pipeline: N_s + 2K at most 63
+    assert L.moe_unpermute_backward(d, d, 32, d, d, d, d, d, 1, 8, 64, 16, d, None) == 2
+    assert L.moe_unpermute_backward(d, d, 31, d, d, d, d, d, 1, 0, 64, 16, d, None) == 0
     assert L.moe_router_weight_grad(d, None, d, d, 2, 16, 64, d, None) == 2
     assert L.moe_router_weight_grad(d, None, d, None, 1, 16, 64, d, None) == 1
     # FP8 Wgrad quantiser

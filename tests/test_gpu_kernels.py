@@ -325,6 +325,7 @@ def test_expert_ffn_f32(sizes, d, I):
     (77, 7168, 8, 1, torch.bfloat16),     # V3 row: seven 2 KB chunks, a partial token group
     (130, 1536, 16, 3, torch.bfloat16),   # K = 16, ragged last chunk (3072 B rows)
     (50, 2560, 16, 2, torch.float32),     # float32 rows of five chunks
+    (41, 1024, 16, 40, torch.bfloat16),   # 57 row slots: 512-byte chunks, four stages
 ])
 def test_combine(T, d, K, N_s, dtype):
     g = _gen(T + K)
@@ -388,6 +389,7 @@ def _bwd_case(T, d, K, N_s, dtype, seed):
     (45, 2560, 16, 0, torch.float32),
     (333, 256, 6, 3, torch.float32),      # rows shorter than one chunk
     (64, 256, 3, 1, torch.bfloat16),      # small K
+    (37, 1536, 16, 20, torch.bfloat16),   # 53 row slots: 512-byte chunks, four stages
 ])
 def test_combine_and_unpermute_backward(T, d, K, N_s, dtype):
     """moe_combine_backward and moe_unpermute_backward against the chain rule
