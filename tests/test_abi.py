@@ -185,3 +185,41 @@ def test_expert_parallel_argument_errors(L):
     assert L.moe_ep_dispatch(d, 1, 8, 64, 4, d, d, d, d, 15, 2, 0, pp, pp, 64, None) == 1  # N_r % W
     assert L.moe_ep_return(d, 1, d, d, 64, 64, 9, pp, 64, None) == 1                       # W
     assert L.moe_ep_return(d, 1, d, d, 64, 64, 2, pn, 64, None) == 1
+
+
+def test_plain_c_program_links_and_calls(L, tmp_path):
+    """include/moe.h is a C header: a strict C99 program compiles against it,
+    links libmoe.so and calls the host-side entry points (no GPU needed)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_moe.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include <string.h>
+#include "moe.h"
+int main(void) {
+  if (moe_abi_version() <= 0) return 1;
+  if (strcmp(moe_status_string(MOE_ERR_WORKSPACE), "MOE_ERR_WORKSPACE") != 0) return 2;
+  if (moe_route_workspace_size(0, 256) != 0) return 3;
+  if (moe_route_workspace_size(8192, 256) == 0) return 4;
+  /* a bad argument answers with a status before any device work */
+  if (moe_combine(NULL, NULL, 0, NULL, NULL, NULL, MOE_BF16, 8, 64, 4, NULL, NULL) !=
+      MOE_ERR_INVALID_ARG)
+    return 5;
+  if (moe_last_error()[0] == 0) return 6;
+  printf("ok %d\n", moe_abi_version());
+  return 0;
+}
+''')
+    exe = tmp_path / "use_moe"
+    lib_dir = os.path.dirname(moe.LIB_PATH)
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                        "-I" + os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                        "-L" + lib_dir, "-lmoe", "-Wl,-rpath," + lib_dir],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0 and r.stdout.startswith("ok"), (r.returncode, r.stdout, r.stderr)
