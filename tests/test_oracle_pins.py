@@ -465,3 +465,176 @@ def test_grouped_topk_special_cases():
         np.testing.assert_array_equal(O.grouped_topk(s, b, 6, G, G)[0], plain)
     idx, key = O.grouped_topk(s, b, 6, 8, 2)
     assert np.all(idx[:, 0] == np.argmax(key, axis=1))   # the best expert's group always survives
+
+
+# --------------------------------------------------------------------------
+# near-tie margins used by the routing comparison
+# --------------------------------------------------------------------------
+
+def test_topk_margins_hand_worked():
+    """Worked by hand: row 0 sorts to 0.80, 0.80, 0.79 | 0.50 ...: the K-th
+    (3rd) key 0.79 minus the next key 0.50, and a zero gap between the two
+    equal selected keys; row 1 sorts to 0.9, 0.7, 0.65 | 0.6: gaps 0.05 and
+    min(0.2, 0.05).  K = N_r has no next key (infinite gap), K = 1 has no
+    adjacent selected pair (infinite gap)."""
+    f = np.float32
+    key = np.array([[0.50, 0.80, 0.30, 0.80, 0.79, 0.10],
+                    [0.90, 0.60, 0.70, 0.65, 0.20, 0.10]], np.float32)
+    idx, _ = O.biased_topk(key, np.zeros(6, np.float32), 3)
+    assert idx.tolist() == [[1, 3, 4], [0, 2, 3]]
+    sel, inner = O.topk_margins(key, idx)
+    assert sel[0] == float(f(0.79)) - float(f(0.50))
+    assert sel[1] == float(f(0.65)) - float(f(0.60))
+    assert inner[0] == 0.0
+    assert inner[1] == float(f(0.70)) - float(f(0.65))
+    full, _ = O.biased_topk(key, np.zeros(6, np.float32), 6)
+    sel6, inner6 = O.topk_margins(key, full)
+    assert np.all(np.isinf(sel6)) and inner6[0] == 0.0
+    one, _ = O.biased_topk(key, np.zeros(6, np.float32), 1)
+    sel1, inner1 = O.topk_margins(key, one)
+    assert sel1[0] == 0.0 and sel1[1] == float(f(0.90)) - float(f(0.70))
+    assert np.all(np.isinf(inner1))
+
+
+# --------------------------------------------------------------------------
+# the layer under the FP8 recipe
+# --------------------------------------------------------------------------
+
+def _fp8_layer_case(seed, T=12, d=256, N_r=5, I=128, N_s=1):
+    rng = np.random.default_rng(seed)
+    u = rng.standard_normal((T, d)).astype(np.float32).astype(np.float64)
+    E = rng.standard_normal((N_r, d)) / math.sqrt(d)
+
+    def q():
+        return O.quantise_expert((rng.standard_normal((I, d)) / math.sqrt(d)).astype(np.float32),
+                                 (rng.standard_normal((I, d)) / math.sqrt(d)).astype(np.float32),
+                                 (rng.standard_normal((d, I)) / math.sqrt(I)).astype(np.float32))
+    return u, E, [q() for _ in range(N_r)], [q() for _ in range(N_s)]
+
+
+def test_fp8_layer_identical_experts():
+    """All routed experts equal: the gates sum to 1, so the routed term is one
+    FP8 FFN whatever the routing; the shared term enters with weight 1."""
+    u, E, routed, shared = _fp8_layer_case(21)
+    r = O.route(u, E, np.zeros(len(routed), np.float32), 3)
+    got = O.layer_forward_fp8(u, r["idx"], r["gate"], [routed[0]] * len(routed), shared)
+    want = u + O.fp8_swiglu_ffn(u, shared[0]) + O.fp8_swiglu_ffn(u, routed[0])
+    np.testing.assert_allclose(got, want, rtol=1e-6, atol=1e-6)
+
+
+def test_fp8_layer_zero_down_and_zero_input():
+    """W_down = 0 quantises to zero codes with unit scales: h' = u exactly;
+    u = 0 quantises to zero codes: every FFN is 0 and h' = 0 exactly."""
+    u, E, routed, shared = _fp8_layer_case(22)
+    zero = lambda Wq: {**Wq, "down": (np.zeros_like(Wq["down"][0]),
+                                      O.tile_scale(np.zeros_like(Wq["down"][1])))}
+    r = O.route(u, E, np.zeros(len(routed), np.float32), 2)
+    got = O.layer_forward_fp8(u, r["idx"], r["gate"], [zero(w) for w in routed],
+                              [zero(w) for w in shared])
+    np.testing.assert_array_equal(got, u)
+    z = np.zeros_like(u)
+    rz = O.route(z, E, np.zeros(len(routed), np.float32), 2)
+    np.testing.assert_array_equal(O.layer_forward_fp8(z, rz["idx"], rz["gate"], routed, shared), z)
+
+
+def test_fp8_layer_dense_mixture():
+    """K = N_r, b = 0: the FP8 layer is u + sum_s FFN8_s(u) + sum_i (s_i / sum_j
+    s_j) FFN8_i(u), written here as a plain loop over every expert on every
+    token (activation scales are per row, so each row quantises alike in any
+    batch).  Catches a gate applied to the wrong slot or a dropped term."""
+    u, E, routed, shared = _fp8_layer_case(23, N_s=2)
+    N_r = len(routed)
+    r = O.route(u, E, np.zeros(N_r, np.float32), N_r)
+    got = O.layer_forward_fp8(u, r["idx"], r["gate"], routed, shared)
+    s = (1.0 / (1.0 + np.exp(-(u @ E.T)))).astype(np.float32).astype(np.float64)
+    w = s / s.sum(axis=1, keepdims=True)
+    want = u.copy()
+    for Wq in shared:
+        want += O.fp8_swiglu_ffn(u, Wq)
+    for i in range(N_r):
+        want += w[:, i:i + 1] * O.fp8_swiglu_ffn(u, routed[i])
+    np.testing.assert_allclose(got, want, rtol=2e-6, atol=2e-6)
+
+
+def _e4m3_nearest(x):
+    """Brute force: the nearest of the 253 finite E4M3 values (saturating),
+    ties to the code with the even mantissa, found by search over the table."""
+    vals, even = [], []
+    for e in range(16):
+        for m in range(8):
+            if e == 15 and m == 7:
+                continue
+            v = (m / 8.0) * 2.0 ** -6 if e == 0 else (1 + m / 8.0) * 2.0 ** (e - 7)
+            for sgn in (1.0, -1.0):
+                vals.append(sgn * v)
+                even.append(m % 2 == 0)
+    vals, even = np.array(vals), np.array(even)
+    x = np.asarray(x, np.float64)
+    dist = np.abs(x.reshape(-1, 1) - vals[None, :])
+    best = dist.min(axis=1, keepdims=True)
+    cand = dist == best
+    pick = np.where(cand & even[None, :], 1, 0) + np.where(cand, 1, 0)
+    return vals[np.argmax(pick, axis=1)].reshape(x.shape)
+
+
+def _fp8_ffn_brute(x, Wg, Wu, Wd, h_round):
+    """The FP8 SwiGLU FFN of reading R6 with scalar loops on a tiny case:
+    1x128 activation tiles and 128x128 weight blocks with float32 scales
+    amax/448, each 128-deep partial sum times its two scales, h formed by
+    h_round (float32 per R6) and re-quantised 1x128."""
+    f32 = np.float32
+
+    def quant(M, rb, cb):
+        M = np.asarray(M, np.float32)
+        q = np.zeros(M.shape)
+        sc = np.zeros((M.shape[0] // rb, M.shape[1] // cb), np.float32)
+        for i in range(sc.shape[0]):
+            for j in range(sc.shape[1]):
+                blk = M[i * rb:(i + 1) * rb, j * cb:(j + 1) * cb]
+                amax = f32(np.abs(blk).max())
+                s = f32(1.0) if amax == 0 else f32(amax / f32(448.0))
+                sc[i, j] = s
+                q[i * rb:(i + 1) * rb, j * cb:(j + 1) * cb] = _e4m3_nearest(blk / s)
+        return q, sc
+
+    def gemm(qa, sa, qw, sw):
+        R, Kd = qa.shape
+        out = np.zeros((R, qw.shape[0]))
+        for r in range(R):
+            for n in range(qw.shape[0]):
+                acc = 0.0
+                for kb in range(Kd // 128):
+                    part = 0.0
+                    for k in range(kb * 128, kb * 128 + 128):
+                        part += qa[r, k] * qw[n, k]
+                    acc += part * float(sa[r, kb]) * float(sw[n // 128, kb])
+                out[r, n] = acc
+        return out
+
+    qx, sx = quant(x, 1, 128)
+    g = gemm(qx, sx, *quant(Wg, 128, 128))
+    v = gemm(qx, sx, *quant(Wu, 128, 128))
+    h = np.array([[h_round(gg / (1.0 + math.exp(-gg)) * vv) for gg, vv in zip(gr, vr)]
+                  for gr, vr in zip(g, v)])
+    qh, sh = quant(h, 1, 128)
+    return gemm(qh, sh, *quant(Wd, 128, 128))
+
+
+def test_fp8_ffn_bruteforce_tiny():
+    """fp8_swiglu_ffn equals the brute-force evaluation of reading R6 (own
+    E4M3 table search, scalar loops) on a 3-row case with two 128-deep K
+    blocks, and the case is sensitive to the precision of h: rounding h to
+    bf16 instead of float32 before its re-quantisation changes the result."""
+    rng = np.random.default_rng(31)
+    d, I = 256, 128
+    x = rng.standard_normal((3, d)).astype(np.float32)
+    x[1, 7] = 40.0                                        # an outlier in one tile
+    Wg = (rng.standard_normal((I, d)) / 16).astype(np.float32)
+    Wu = (rng.standard_normal((I, d)) / 16).astype(np.float32)
+    Wd = (rng.standard_normal((d, I)) / math.sqrt(I)).astype(np.float32)
+    got = O.fp8_swiglu_ffn(x, O.quantise_expert(Wg, Wu, Wd))
+    want = _fp8_ffn_brute(x, Wg, Wu, Wd, lambda z: float(np.float32(z)))
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+    bf16 = lambda z: float(torch.tensor(z, dtype=torch.float32).to(torch.bfloat16).float())
+    other = _fp8_ffn_brute(x, Wg, Wu, Wd, bf16)
+    assert np.abs(other - want).max() > 1e-6 * np.abs(want).max()
