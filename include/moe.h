@@ -139,7 +139,13 @@ moe_status moe_permute(const void* u, const float* u_scale, moe_dtype dt,
  *   x          [rows, d]        device, dt
  *   x_scale    [rows, d/128]    device, float32 (MOE_E4M3 only, else NULL)
  *   offsets    [n_groups+1]     device, int32, non-decreasing, offsets[0] = 0,
- *                               offsets[n_groups] <= rows
+ *                               offsets[n_groups] <= rows.  Values outside
+ *                               [0, rows], or below an earlier value, are
+ *                               clamped on the device (bf16 / FP8: each raised
+ *                               to the largest earlier value and cut to rows;
+ *                               f32: each group's range cut into [0, rows));
+ *                               rows outside every group are not written and
+ *                               moe_device_status() reports bit 16
  *   W_gate_up  [n_groups, 2I, d] device, dt: rows [0,I) are W_gate, [I,2I) W_up
  *   w_scale_gate_up [n_groups, 2I/128, d/128] float32 (MOE_E4M3 only, else NULL)
  *   W_down     [n_groups, d, I] device, dt
@@ -176,6 +182,32 @@ moe_status moe_expert_gate_up(const void* x, const float* x_scale, const int32_t
 moe_status moe_expert_down(const void* h, const float* h_scale, const int32_t* offsets,
                            int n_groups, int rows, int d, int I, moe_dtype dt,
                            const void* W_down, const float* w_scale_down, void* y, void* stream);
+
+/* ------------------------------------------------------------------------
+ * moe_expert_gate_up_shared / moe_expert_down_shared - the two halves of the
+ * routed grouped FFN with the N_s shared experts of the h'-equation (every
+ * token, weight 1) run as extra groups of the same launch, so that their
+ * tiles fill the routed launch's tail.  MOE_BF16 only; same arithmetic as
+ * moe_expert_gate_up / moe_expert_down.
+ *   x          [rows, d]        device bf16: routed rows (moe_permute's x_perm)
+ *   offsets    [n_groups+1]     device int32: routed groups, as moe_expert_ffn
+ *   u          [T, d]           device bf16: the layer input (shared experts' rows)
+ *   W_gate_up  [n_groups, 2I, d], Ws_gate_up [N_s, 2I, d]   device bf16
+ *   W_down     [n_groups, d, I],  Ws_down    [N_s, d, I]    device bf16
+ *   h          [rows + N_s*T, I] device bf16: routed rows first, then shared
+ *              expert j's rows at rows + j*T + t (SiLU(gate) * up of u[t])
+ *   y          [rows + N_s*T, d] device bf16: y[r] = W_down[g] h[r] for the
+ *              routed rows, y[rows + j*T + t] = Ws_down[j] h[rows + j*T + t];
+ *              so y + rows*d is the y_shared [N_s, T, d] of moe_combine.
+ * Requires d % 256 == 0 and I % 128 == 0 (down: d a multiple of 256).
+ * ------------------------------------------------------------------------ */
+moe_status moe_expert_gate_up_shared(const void* x, const int32_t* offsets, int n_groups,
+                                     int rows, const void* u, int T, int N_s, int d, int I,
+                                     const void* W_gate_up, const void* Ws_gate_up, void* h,
+                                     void* stream);
+moe_status moe_expert_down_shared(const void* h, const int32_t* offsets, int n_groups, int rows,
+                                  int T, int N_s, int d, int I, const void* W_down,
+                                  const void* Ws_down, void* y, void* stream);
 
 /* ------------------------------------------------------------------------
  * moe_combine - the h'-equation with the residual:
@@ -235,8 +267,10 @@ moe_status moe_quantize_128x128(const void* w, int groups, int rows, int cols,
  * only 2 * ceil(T/256) * N_r * 4 bytes <= 1 MiB (T <= 131072 at N_r = 256);
  * larger problems get MOE_ERR_UNSUPPORTED and launch nothing.  The first
  * call on a device looks up the array's device address (make it before any
- * stream capture).  Every call uses the same array: calls whose work
- * overlaps on the GPU (other streams or host threads) race on it.
+ * stream capture) and keeps it for the life of the process: a
+ * cudaDeviceReset unloads the array, so do not use the library across one.
+ * Every call uses the same array: calls whose work overlaps on the GPU
+ * (other streams or host threads) race on it.
  * ------------------------------------------------------------------------ */
 moe_status moe_permute_noalloc(const void* u, const float* u_scale, moe_dtype dt,
                                const int32_t* topk_idx, int T, int d, int N_r, int K,
@@ -288,15 +322,19 @@ moe_status moe_expert_gate_up_save(const void* x, const float* x_scale, const in
  *   dh_out, u [T, d]; E [N_r, d]; y_perm [T*K, d]: device, dt (MOE_F32 or
  *   MOE_BF16); inv_row, topk_idx [T, K] int32 and topk_gate [T, K] float32
  *   from the forward; dy_perm [T*K, d] dt out; d_gate, d_logit [T, K] and
- *   d_logit_perm [T*K] float32 out.  K <= 16, d * sizeof(dt) % 16 == 0.
- *   A slot whose inv_row lies outside [0, T*K) is left out (no dy_perm row
- *   written, no d_logit_perm entry, no d_gate contribution).
+ *   d_logit_perm [T*K] float32 out.  N_r: rows of E.  K <= 16,
+ *   d * sizeof(dt) % 16 == 0.
+ *   A slot whose inv_row lies outside [0, T*K) or whose expert id lies
+ *   outside [0, N_r) (moe_permute gives such ids inv_row -1) is left out of
+ *   the selection: no dy_perm row is written, no d_logit_perm entry, its
+ *   d_gate and d_logit are 0, its s is not part of S, and neither its row
+ *   nor its centroid is read.
  * The shared experts' upstream gradient is dh_out itself (weight 1).
  * ------------------------------------------------------------------------ */
 moe_status moe_combine_backward(const void* dh_out, const void* u, const void* E,
                                 const void* y_perm, const int32_t* inv_row,
                                 const int32_t* topk_idx, const float* topk_gate, moe_dtype dt,
-                                int T, int d, int K, void* dy_perm, float* d_gate,
+                                int T, int d, int K, int N_r, void* dy_perm, float* d_gate,
                                 float* d_logit, float* d_logit_perm, void* stream);
 
 /* ------------------------------------------------------------------------
@@ -362,14 +400,16 @@ moe_status moe_expert_ffn_backward(const void* x, const int32_t* x_rows, const i
  *           + sum_k d_logit[t,k] E[topk_idx[t,k]]
  * summed in float32 in that order, rounded once to dt.  dh_out, du [T, d];
  * dx_shared [N_s, T, d] (NULL when N_s == 0); dx_perm [T*K, d]; E [N_r, d]:
- * device, dt (MOE_F32 or MOE_BF16).  K <= 16, N_s + 2K <= 63,
- * d * sizeof(dt) % 16 == 0.  A slot whose inv_row lies outside [0, T*K) is
- * left out of the sum.
+ * device, dt (MOE_F32 or MOE_BF16); N_r rows of E.  K <= 16, N_s + 2K <= 63,
+ * d * sizeof(dt) % 16 == 0.  A slot whose inv_row lies outside [0, T*K) or
+ * whose expert id lies outside [0, N_r) is left out of both sums (neither
+ * its dx_perm row nor its centroid is read).
  * ------------------------------------------------------------------------ */
 moe_status moe_unpermute_backward(const void* dh_out, const void* dx_shared, int N_s,
                                   const void* dx_perm, const int32_t* inv_row,
                                   const int32_t* topk_idx, const float* d_logit, const void* E,
-                                  moe_dtype dt, int T, int d, int K, void* du, void* stream);
+                                  moe_dtype dt, int T, int d, int K, int N_r, void* du,
+                                  void* stream);
 
 /* ------------------------------------------------------------------------
  * moe_router_weight_grad - gradient of the expert centroids E:
@@ -435,13 +475,28 @@ moe_status moe_ep_return(const void* y, moe_dtype dt, const void* recv_tags,
 /* ------------------------------------------------------------------------
  * moe_device_status - synchronises the current device, then returns (and
  * clears) the library's device-side error word: 0 if no kernel gave up a
- * bounded wait since the last call, else a bit set naming the kernel:
+ * bounded wait or clamped bad input since the last call, else a bit set
+ * naming the kernel:
  *   1  a tcgen05 bf16 GEMM (expert FFN, router logits, Wgrad)
  *   2  an FP8 tcgen05 GEMM
  *   4  an expert-parallel copy skipped a row position past its buffer
  *   8  the row-gather pipeline (combine, combine and unpermute backward)
+ *  16  a grouped GEMM met group offsets outside [0, rows] or decreasing and
+ *      clamped them (no row outside [0, rows) was read or written)
  * ------------------------------------------------------------------------ */
 moe_status moe_device_status(int* flags);
+
+/* ------------------------------------------------------------------------
+ * moe_set_pipeline_wait_limit - the bound, in nanoseconds, of every wait of
+ * the row-gather pipeline (moe_combine, moe_combine_backward,
+ * moe_unpermute_backward) on a shared-memory stage; 0 restores the default
+ * of 1 s.  After a wait runs out the kernel stops taking rows, lets the
+ * copies it issued land (within 1 s), returns, and moe_device_status()
+ * reports bit 8; rows it did not reach are not written.  Process-wide; it
+ * takes effect at the next launch.  The pages have no counterpart: the
+ * knob exists so that the timeout path can be exercised.
+ * ------------------------------------------------------------------------ */
+moe_status moe_set_pipeline_wait_limit(unsigned long long ns);
 
 #ifdef __cplusplus
 }

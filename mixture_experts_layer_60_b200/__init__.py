@@ -17,6 +17,7 @@ __all__ = [
     "MoeError", "lib", "LIB_PATH", "SYMBOLS",
     "moe_route", "moe_route_grouped", "moe_permute", "moe_permute_noalloc", "moe_expert_ffn", "moe_expert_gate_up", "moe_expert_down", "moe_combine", "moe_bias_update",
     "moe_quantize_1x128", "moe_quantize_128x128", "moe_device_status",
+    "moe_set_pipeline_wait_limit", "moe_expert_gate_up_shared", "moe_expert_down_shared",
     "moe_route_workspace_size", "moe_permute_workspace_size", "moe_expert_ffn_workspace_size",
     "moe_expert_gate_up_save", "moe_combine_backward", "moe_expert_ffn_backward",
     "moe_expert_ffn_backward_workspace_size", "moe_unpermute_backward", "moe_router_weight_grad",
@@ -52,15 +53,18 @@ SYMBOLS = {
     "moe_quantize_1x128": (_i, [_vp, _i, _i, _vp, _vp, _vp]),
     "moe_quantize_128x128": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp]),
     "moe_device_status": (_i, [ctypes.POINTER(_i)]),
+    "moe_set_pipeline_wait_limit": (_i, [ctypes.c_ulonglong]),
+    "moe_expert_gate_up_shared": (_i, [_vp, _vp, _i, _i, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
+    "moe_expert_down_shared": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
     "moe_permute_noalloc": (_i, [_vp, _vp, _i, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
     "moe_expert_gate_up_save": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp,
                                      _vp]),
-    "moe_combine_backward": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp,
-                                  _vp, _vp]),
+    "moe_combine_backward": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp,
+                                  _vp, _vp, _vp]),
     "moe_expert_ffn_backward_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
     "moe_expert_ffn_backward": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp,
                                      _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
-    "moe_unpermute_backward": (_i, [_vp, _vp, _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp,
+    "moe_unpermute_backward": (_i, [_vp, _vp, _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp,
                                     _vp]),
     "moe_router_weight_grad": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp]),
     "moe_quantize_128x1_grouped": (_i, [_vp, _i, _i, _vp, _i, _vp, _vp, _vp, _vp]),
@@ -230,6 +234,26 @@ def moe_expert_down(h, offsets, W_down, y, h_scale=None, w_scale_down=None, stre
                                  _p(W_down), _p(w_scale_down), _p(y), _s(stream)))
 
 
+def moe_expert_gate_up_shared(x, offsets, W_gate_up, u, Ws_gate_up, h, stream=None):
+    """Routed gate/up (x [rows, d]) with the shared experts' gate/up of u
+    [T, d] as extra groups of one launch: h [rows + N_s*T, I]."""
+    rows, d = x.shape
+    n_groups, two_i, _ = W_gate_up.shape
+    T, N_s = u.shape[0], Ws_gate_up.shape[0]
+    _check(lib().moe_expert_gate_up_shared(_p(x), _p(offsets), n_groups, rows, _p(u), T, N_s, d,
+                                           two_i // 2, _p(W_gate_up), _p(Ws_gate_up), _p(h),
+                                           _s(stream)))
+
+
+def moe_expert_down_shared(h, offsets, W_down, Ws_down, rows, T, y, stream=None):
+    """Routed down projection of h[:rows] and the shared experts' of
+    h[rows + j*T + t] in one launch: y [rows + N_s*T, d]."""
+    n_groups, d, I = W_down.shape
+    N_s = Ws_down.shape[0]
+    _check(lib().moe_expert_down_shared(_p(h), _p(offsets), n_groups, rows, T, N_s, d, I,
+                                        _p(W_down), _p(Ws_down), _p(y), _s(stream)))
+
+
 def moe_combine(u, y_shared, y_perm, inv_row, topk_gate, h_out, stream=None):
     T, d = u.shape
     N_s = 0 if y_shared is None else y_shared.shape[0]
@@ -249,6 +273,11 @@ def moe_quantize_1x128(x, q, scale, stream=None):
 def moe_quantize_128x128(w, q, scale, stream=None):
     groups, rows, cols = w.shape
     _check(lib().moe_quantize_128x128(_p(w), groups, rows, cols, _p(q), _p(scale), _s(stream)))
+
+
+def moe_set_pipeline_wait_limit(ns: int = 0):
+    """Bound (ns) of the row-gather pipeline's waits; 0 restores the default 1 s."""
+    _check(lib().moe_set_pipeline_wait_limit(int(ns)))
 
 
 def moe_device_status() -> int:
@@ -280,8 +309,8 @@ def moe_combine_backward(dh_out, u, E, y_perm, inv_row, topk_idx, topk_gate, dy_
     T, d = u.shape
     _check(lib().moe_combine_backward(_p(dh_out), _p(u), _p(E), _p(y_perm), _p(inv_row),
                                       _p(topk_idx), _p(topk_gate), _dt(u), T, d,
-                                      inv_row.shape[1], _p(dy_perm), _p(d_gate), _p(d_logit),
-                                      _p(d_logit_perm), _s(stream)))
+                                      inv_row.shape[1], E.shape[0], _p(dy_perm), _p(d_gate),
+                                      _p(d_logit), _p(d_logit_perm), _s(stream)))
 
 
 def moe_expert_ffn_backward(x, offsets, W_gate_up, W_down, a_gu, h, dy, dx, dW_gate_up, dW_down,
@@ -305,7 +334,7 @@ def moe_unpermute_backward(dh_out, dx_shared, dx_perm, inv_row, topk_idx, d_logi
     N_s = 0 if dx_shared is None else dx_shared.shape[0]
     _check(lib().moe_unpermute_backward(_p(dh_out), _p(dx_shared), N_s, _p(dx_perm), _p(inv_row),
                                         _p(topk_idx), _p(d_logit), _p(E), _dt(dh_out), T, d,
-                                        inv_row.shape[1], _p(du), _s(stream)))
+                                        inv_row.shape[1], E.shape[0], _p(du), _s(stream)))
 
 
 def moe_router_weight_grad(x, d_logit_perm, offsets, dE, x_rows=None, stream=None):

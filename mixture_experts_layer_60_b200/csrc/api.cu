@@ -2,18 +2,15 @@
 // validates its arguments on the host, then enqueues kernels on `stream`.
 #include "launch.h"
 
-namespace moe {
-const char* last_error_text();
-void clear_last_error();
-}  // namespace moe
-
 using namespace moe;
 
 namespace {
 
-constexpr int kAbiVersion = 1;
+constexpr int kAbiVersion = 2;
 
 inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+inline bool al16(const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0; }
 
 int dtype_bytes(moe_dtype dt) {
   switch (dt) {
@@ -24,11 +21,7 @@ int dtype_bytes(moe_dtype dt) {
   return 0;
 }
 
-moe_status check_device() {
-  if (!device_is_sm100())
-    return fail(MOE_ERR_UNSUPPORTED, "libmoe kernels need an sm_100 (B200) device");
-  return MOE_OK;
-}
+moe_status check_device() { return check_sm100(); }
 
 #define MOE_REQUIRE(cond, status, ...) \
   do {                                 \
@@ -41,13 +34,13 @@ moe_status check_device() {
     if (_st != MOE_OK) return _st;    \
   } while (0)
 
-// Router workspace: float32 logits [T, N_r], then the tie-break lists: a
-// 2-word header and tok/start/num [T] int32, candidate pairs [T*N_r] int32
-// and their float64 affinities [T*N_r] float32.
+// Router workspace: float32 logits [T, N_r] (the fused router writes only
+// the rows of listed tokens), then the tie-break lists: a 2-word header,
+// tok/start/num [T] int32 and candidate pairs [T*N_r] int32.
 size_t route_ws(int T, int N_r) {
   if (T <= 0 || N_r <= 0) return 0;
   const size_t tn = align_up((size_t)T * N_r * sizeof(float), 256);
-  return tn + align_up((size_t)(2 + 3 * (size_t)T) * 4, 256) + 2 * tn;
+  return tn + align_up((size_t)(2 + 3 * (size_t)T) * 4, 256) + tn;
 }
 
 RefineLists refine_lists(void* workspace, int T, int N_r) {
@@ -60,13 +53,8 @@ RefineLists refine_lists(void* workspace, int T, int N_r) {
   rl.num = rl.start + T;
   p += align_up((size_t)(2 + 3 * (size_t)T) * 4, 256);
   rl.pair = reinterpret_cast<int32_t*>(p);
-  rl.s64 = reinterpret_cast<float*>(p + tn);
   return rl;
 }
-
-// Routing decided by a key gap below this is redone from float64 logits: the
-// float32 tensor-core logits over d <= 16384 products stay well within it.
-constexpr float kRefineGap = 2e-5f;
 
 size_t ffn_ws(moe_dtype dt, int rows, int I) {
   if (rows <= 0 || I <= 0) return 0;
@@ -137,15 +125,19 @@ moe_status route_impl(const char* who, const void* u, const void* E, moe_dtype d
   MOE_TRY(cuda_check(cudaMemsetAsync(counts, 0, (size_t)N_r * sizeof(int32_t), s), "zero counts"));
   if (T == 0) return MOE_OK;
   float* logits = static_cast<float*>(workspace);
-  if (dt == MOE_BF16 && N_r % 64 == 0) {
-    MOE_TRY(launch_tc_gemm(u, E, N_r, nullptr, 1, T, N_r, d, TC_EPI_STORE_F32, logits, s));
-  } else {
-    MOE_TRY(launch_logits_simt(u, E, dt, T, d, N_r, logits, s));
-  }
   const RefineLists rl = refine_lists(workspace, T, N_r);
   MOE_TRY(cuda_check(cudaMemsetAsync(rl.hdr, 0, 2 * sizeof(int32_t), s), "zero tie-break lists"));
-  MOE_TRY(launch_topk(logits, b, T, N_r, K, n_groups, topk_groups, topk_idx, topk_gate, counts,
-                      rl, kRefineGap, s));
+  if (router_tc_supported(dt, d, N_r, K, n_groups, topk_groups)) {
+    MOE_TRY(launch_router_tc(u, E, b, T, d, N_r, K, n_groups, topk_groups, topk_idx, topk_gate,
+                             counts, logits, rl, kRouterRefineGap, kRouterNearBoundary, s));
+  } else {
+    if (dt == MOE_BF16 && N_r % 64 == 0)
+      MOE_TRY(launch_tc_gemm(u, E, N_r, nullptr, 1, T, N_r, d, TC_EPI_STORE_F32, logits, s));
+    else
+      MOE_TRY(launch_logits_simt(u, E, dt, T, d, N_r, logits, s));
+    MOE_TRY(launch_topk(logits, b, T, N_r, K, n_groups, topk_groups, topk_idx, topk_gate, counts,
+                        rl, kRouterRefineGap, s));
+  }
   return launch_refine(u, E, dt, logits, b, d, N_r, K, n_groups, topk_groups, rl, T, topk_idx,
                        topk_gate, counts, s);
 }
@@ -174,36 +166,57 @@ size_t moe_permute_workspace_size(int T, int N_r) {
   return permute_ws_bytes(T, N_r);
 }
 
+}  // extern "C"
+
+namespace moe {
+
+moe_status validate_permute_args(const char* who, const void* u, const float* u_scale,
+                                 moe_dtype dt, const int32_t* topk_idx, int T, int d, int N_r,
+                                 int K, const void* x_perm, const float* x_scale,
+                                 const int32_t* offsets, const int32_t* perm_src,
+                                 const int32_t* inv_row, int* elem_bytes) {
+  const int eb = dtype_bytes(dt);
+  MOE_REQUIRE(eb > 0, MOE_ERR_UNSUPPORTED, "%s: unknown dtype %d", who, (int)dt);
+  MOE_REQUIRE(T >= 0 && d > 0 && N_r > 0 && K > 0, MOE_ERR_INVALID_ARG,
+              "%s: bad sizes T=%d d=%d N_r=%d K=%d", who, T, d, N_r, K);
+  MOE_REQUIRE(N_r <= 1024 && K <= N_r, MOE_ERR_UNSUPPORTED, "%s: need 1 <= K <= N_r <= 1024",
+              who);
+  MOE_REQUIRE(((size_t)d * eb) % 16 == 0, MOE_ERR_UNSUPPORTED,
+              "%s: a row (%d x %d bytes) must be a multiple of 16 bytes", who, d, eb);
+  MOE_REQUIRE(offsets, MOE_ERR_INVALID_ARG, "%s: null offsets", who);
+  MOE_REQUIRE(T == 0 || (u && topk_idx && x_perm && perm_src && inv_row), MOE_ERR_INVALID_ARG,
+              "%s: null pointer", who);
+  if (dt == MOE_E4M3) {
+    MOE_REQUIRE(d % 128 == 0, MOE_ERR_UNSUPPORTED, "%s: e4m3 needs d %% 128 == 0", who);
+    MOE_REQUIRE(T == 0 || (u_scale && x_scale), MOE_ERR_INVALID_ARG,
+                "%s: e4m3 needs u_scale and x_scale", who);
+  } else {
+    MOE_REQUIRE(!u_scale && !x_scale, MOE_ERR_INVALID_ARG, "%s: scales are only for MOE_E4M3",
+                who);
+  }
+  MOE_REQUIRE(reinterpret_cast<uintptr_t>(u) % 16 == 0 &&
+                  reinterpret_cast<uintptr_t>(x_perm) % 16 == 0,
+              MOE_ERR_INVALID_ARG, "%s: u and x_perm must be 16-byte aligned", who);
+  *elem_bytes = eb;
+  return MOE_OK;
+}
+
+}  // namespace moe
+
+extern "C" {
+
 moe_status moe_permute(const void* u, const float* u_scale, moe_dtype dt, const int32_t* topk_idx,
                        int T, int d, int N_r, int K, void* x_perm, float* x_scale,
                        int32_t* offsets, int32_t* perm_src, int32_t* inv_row, void* workspace,
                        size_t workspace_bytes, void* stream) {
   clear_last_error();
-  const int eb = dtype_bytes(dt);
-  MOE_REQUIRE(eb > 0, MOE_ERR_UNSUPPORTED, "moe_permute: unknown dtype %d", (int)dt);
-  MOE_REQUIRE(T >= 0 && d > 0 && N_r > 0 && K > 0, MOE_ERR_INVALID_ARG,
-              "moe_permute: bad sizes T=%d d=%d N_r=%d K=%d", T, d, N_r, K);
-  MOE_REQUIRE(N_r <= 1024 && K <= N_r, MOE_ERR_UNSUPPORTED,
-              "moe_permute: need 1 <= K <= N_r <= 1024");
-  MOE_REQUIRE(((size_t)d * eb) % 16 == 0, MOE_ERR_UNSUPPORTED,
-              "moe_permute: a row (%d x %d bytes) must be a multiple of 16 bytes", d, eb);
-  MOE_REQUIRE(offsets, MOE_ERR_INVALID_ARG, "moe_permute: null offsets");
-  MOE_REQUIRE(T == 0 || (u && topk_idx && x_perm && perm_src && inv_row && workspace),
-              MOE_ERR_INVALID_ARG, "moe_permute: null pointer");
-  if (dt == MOE_E4M3) {
-    MOE_REQUIRE(d % 128 == 0, MOE_ERR_UNSUPPORTED, "moe_permute: e4m3 needs d %% 128 == 0");
-    MOE_REQUIRE(T == 0 || (u_scale && x_scale), MOE_ERR_INVALID_ARG,
-                "moe_permute: e4m3 needs u_scale and x_scale");
-  } else {
-    MOE_REQUIRE(!u_scale && !x_scale, MOE_ERR_INVALID_ARG,
-                "moe_permute: scales are only for MOE_E4M3");
-  }
+  int eb = 0;
+  MOE_TRY(validate_permute_args("moe_permute", u, u_scale, dt, topk_idx, T, d, N_r, K, x_perm,
+                                x_scale, offsets, perm_src, inv_row, &eb));
+  MOE_REQUIRE(T == 0 || workspace, MOE_ERR_INVALID_ARG, "moe_permute: null workspace");
   MOE_REQUIRE(workspace_bytes >= moe_permute_workspace_size(T, N_r), MOE_ERR_WORKSPACE,
               "moe_permute: workspace %zu < %zu bytes", workspace_bytes,
               moe_permute_workspace_size(T, N_r));
-  MOE_REQUIRE(reinterpret_cast<uintptr_t>(u) % 16 == 0 &&
-                  reinterpret_cast<uintptr_t>(x_perm) % 16 == 0,
-              MOE_ERR_INVALID_ARG, "moe_permute: u and x_perm must be 16-byte aligned");
   MOE_TRY(check_device());
   cudaStream_t s = as_stream(stream);
   if (T == 0)
@@ -332,6 +345,70 @@ moe_status moe_expert_down(const void* h, const float* h_scale, const int32_t* o
                   as_stream(stream));
 }
 
+namespace {
+
+moe_status check_shared_common(const char* who, const int32_t* offsets, int n_groups, int rows,
+                               int T, int N_s, int d, int I, const void* W, const void* Ws,
+                               const void* out) {
+  MOE_REQUIRE(rows >= 0 && T >= 0 && N_s >= 0 && d > 0 && I > 0 && n_groups > 0,
+              MOE_ERR_INVALID_ARG, "%s: bad sizes rows=%d T=%d N_s=%d d=%d I=%d n_groups=%d", who,
+              rows, T, N_s, d, I, n_groups);
+  MOE_REQUIRE(n_groups <= 1024, MOE_ERR_UNSUPPORTED, "%s: at most 1024 groups", who);
+  MOE_REQUIRE(d % 256 == 0 && I % 128 == 0, MOE_ERR_UNSUPPORTED,
+              "%s: d=%d must be a multiple of 256 and I=%d of 128", who, d, I);
+  MOE_REQUIRE((long long)rows + (long long)N_s * T < (1LL << 31), MOE_ERR_UNSUPPORTED,
+              "%s: rows + N_s*T must fit in 31 bits", who);
+  MOE_REQUIRE(offsets && W && out && (N_s == 0 || Ws), MOE_ERR_INVALID_ARG, "%s: null pointer",
+              who);
+  MOE_REQUIRE(al16(out), MOE_ERR_INVALID_ARG, "%s: outputs must be 16-byte aligned", who);
+  return MOE_OK;
+}
+
+}  // namespace
+
+moe_status moe_expert_gate_up_shared(const void* x, const int32_t* offsets, int n_groups,
+                                     int rows, const void* u, int T, int N_s, int d, int I,
+                                     const void* W_gate_up, const void* Ws_gate_up, void* h,
+                                     void* stream) {
+  clear_last_error();
+  const char* who = "moe_expert_gate_up_shared";
+  MOE_TRY(check_shared_common(who, offsets, n_groups, rows, T, N_s, d, I, W_gate_up, Ws_gate_up,
+                              h));
+  MOE_REQUIRE(rows == 0 || x, MOE_ERR_INVALID_ARG, "%s: null x", who);
+  MOE_REQUIRE(N_s == 0 || T == 0 || u, MOE_ERR_INVALID_ARG, "%s: null u", who);
+  MOE_REQUIRE(al16(x) && al16(u), MOE_ERR_INVALID_ARG, "%s: x and u must be 16-byte aligned", who);
+  if (rows == 0 && (N_s == 0 || T == 0)) return MOE_OK;
+  MOE_TRY(check_device());
+  WsExtraGroups ex;
+  ex.X = u;
+  ex.W = Ws_gate_up;
+  ex.n_extra = T > 0 ? N_s : 0;
+  ex.T = T;
+  ex.x_local = true;
+  // a routed buffer of no rows still needs a valid tensor map: use u's
+  return launch_ws_gemm(rows ? x : u, W_gate_up, 2 * I, offsets, n_groups, rows, I, d, true, h,
+                        as_stream(stream), &ex);
+}
+
+moe_status moe_expert_down_shared(const void* h, const int32_t* offsets, int n_groups, int rows,
+                                  int T, int N_s, int d, int I, const void* W_down,
+                                  const void* Ws_down, void* y, void* stream) {
+  clear_last_error();
+  const char* who = "moe_expert_down_shared";
+  MOE_TRY(check_shared_common(who, offsets, n_groups, rows, T, N_s, d, I, W_down, Ws_down, y));
+  MOE_REQUIRE(h && al16(h), MOE_ERR_INVALID_ARG, "%s: h null or misaligned", who);
+  if (rows == 0 && (N_s == 0 || T == 0)) return MOE_OK;
+  MOE_TRY(check_device());
+  WsExtraGroups ex;
+  ex.X = h;
+  ex.W = Ws_down;
+  ex.n_extra = T > 0 ? N_s : 0;
+  ex.T = T;
+  ex.x_local = false;
+  return launch_ws_gemm(h, W_down, d, offsets, n_groups, rows, d, I, false, y, as_stream(stream),
+                        &ex);
+}
+
 moe_status moe_combine(const void* u, const void* y_shared, int N_s, const void* y_perm,
                        const int32_t* inv_row, const float* topk_gate, moe_dtype dt, int T, int d,
                        int K, void* h_out, void* stream) {
@@ -396,7 +473,6 @@ moe_status moe_quantize_128x128(const void* w, int groups, int rows, int cols, u
 
 namespace {
 
-inline bool al16(const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0; }
 
 // Backward workspace.  bf16: dA [rows, 2I] bf16.  e4m3: the FP8 operands of
 // the two Dgrads and two Wgrads and their scales (see fp8_bwd_layout).
@@ -478,10 +554,11 @@ moe_status moe_expert_gate_up_save(const void* x, const float* x_scale, const in
 moe_status moe_combine_backward(const void* dh_out, const void* u, const void* E,
                                 const void* y_perm, const int32_t* inv_row,
                                 const int32_t* topk_idx, const float* topk_gate, moe_dtype dt,
-                                int T, int d, int K, void* dy_perm, float* d_gate,
+                                int T, int d, int K, int N_r, void* dy_perm, float* d_gate,
                                 float* d_logit, float* d_logit_perm, void* stream) {
   clear_last_error();
   MOE_TRY(check_rowwise("moe_combine_backward", dt, T, d, K));
+  MOE_REQUIRE(N_r > 0, MOE_ERR_INVALID_ARG, "moe_combine_backward: N_r=%d", N_r);
   if (T == 0) return MOE_OK;
   MOE_REQUIRE(dh_out && u && E && y_perm && inv_row && topk_idx && topk_gate && dy_perm &&
                   d_gate && d_logit && d_logit_perm,
@@ -490,7 +567,7 @@ moe_status moe_combine_backward(const void* dh_out, const void* u, const void* E
               MOE_ERR_INVALID_ARG, "moe_combine_backward: rows must be 16-byte aligned");
   MOE_TRY(check_device());
   return launch_combine_backward(dh_out, u, E, y_perm, inv_row, topk_idx, topk_gate, dt, T, d, K,
-                                 dy_perm, d_gate, d_logit, d_logit_perm, as_stream(stream));
+                                 N_r, dy_perm, d_gate, d_logit, d_logit_perm, as_stream(stream));
 }
 
 moe_status moe_quantize_128x1_grouped(const void* x, int rows, int cols, const int32_t* offsets,
@@ -605,10 +682,12 @@ moe_status moe_expert_ffn_backward(const void* x, const int32_t* x_rows, const i
 moe_status moe_unpermute_backward(const void* dh_out, const void* dx_shared, int N_s,
                                   const void* dx_perm, const int32_t* inv_row,
                                   const int32_t* topk_idx, const float* d_logit, const void* E,
-                                  moe_dtype dt, int T, int d, int K, void* du, void* stream) {
+                                  moe_dtype dt, int T, int d, int K, int N_r, void* du,
+                                  void* stream) {
   clear_last_error();
   MOE_TRY(check_rowwise("moe_unpermute_backward", dt, T, d, K));
-  MOE_REQUIRE(N_s >= 0, MOE_ERR_INVALID_ARG, "moe_unpermute_backward: N_s=%d", N_s);
+  MOE_REQUIRE(N_s >= 0 && N_r > 0, MOE_ERR_INVALID_ARG, "moe_unpermute_backward: N_s=%d N_r=%d",
+              N_s, N_r);
   MOE_REQUIRE(N_s + 2 * K <= 63, MOE_ERR_UNSUPPORTED,
               "moe_unpermute_backward: N_s + 2K = %d exceeds 63", N_s + 2 * K);
   if (T == 0) return MOE_OK;
@@ -619,7 +698,7 @@ moe_status moe_unpermute_backward(const void* dh_out, const void* dx_shared, int
               MOE_ERR_INVALID_ARG, "moe_unpermute_backward: rows must be 16-byte aligned");
   MOE_TRY(check_device());
   return launch_unpermute_backward(dh_out, dx_shared, N_s, dx_perm, inv_row, topk_idx, d_logit, E,
-                                   dt, T, d, K, du, as_stream(stream));
+                                   dt, T, d, K, N_r, du, as_stream(stream));
 }
 
 moe_status moe_router_weight_grad(const void* x_perm, const int32_t* x_rows,

@@ -50,23 +50,23 @@ __global__ void __launch_bounds__(128) router_weight_grad_kernel(
 moe_status launch_combine_backward(const void* dh, const void* u, const void* E,
                                    const void* y_perm, const int32_t* inv_row,
                                    const int32_t* idx, const float* gate, moe_dtype dt, int T,
-                                   int d, int K, void* dy_perm, float* d_gate, float* d_logit,
-                                   float* d_logit_perm, cudaStream_t s) {
+                                   int d, int K, int N_r, void* dy_perm, float* d_gate,
+                                   float* d_logit, float* d_logit_perm, cudaStream_t s) {
   const long long rb = (long long)d * (dt == MOE_F32 ? 4 : 2);
   return launch_gather_pipe(GATHER_COMBINE_BWD, dt, dh, u, nullptr, 0, y_perm, (long long)T * K,
-                            E, inv_row, idx, gate, T, K, rb, dy_perm, d_gate, d_logit,
+                            E, N_r, inv_row, idx, gate, T, K, rb, dy_perm, d_gate, d_logit,
                             d_logit_perm, s);
 }
 
 moe_status launch_unpermute_backward(const void* dh, const void* dx_shared, int N_s,
                                      const void* dx_perm, const int32_t* inv_row,
                                      const int32_t* idx, const float* d_logit, const void* E,
-                                     moe_dtype dt, int T, int d, int K, void* du,
+                                     moe_dtype dt, int T, int d, int K, int N_r, void* du,
                                      cudaStream_t s) {
   const long long rb = (long long)d * (dt == MOE_F32 ? 4 : 2);
   return launch_gather_pipe(GATHER_UNPERM_BWD, dt, dh, nullptr, dx_shared, N_s, dx_perm,
-                            (long long)T * K, E, inv_row, idx, d_logit, T, K, rb, du, nullptr,
-                            nullptr, nullptr, s);
+                            (long long)T * K, E, N_r, inv_row, idx, d_logit, T, K, rb, du,
+                            nullptr, nullptr, nullptr, s);
 }
 
 moe_status launch_router_weight_grad(const void* x_perm, const int32_t* x_rows,

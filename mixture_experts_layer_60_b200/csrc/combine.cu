@@ -107,8 +107,8 @@ moe_status launch_combine(const void* u, const void* y_shared, int N_s, const vo
   const long long rb = (long long)d * (dt == MOE_F32 ? 4 : 2);
   if (gather_pipe_supported(GATHER_COMBINE, N_s, K, rb))
     return launch_gather_pipe(GATHER_COMBINE, dt, u, nullptr, y_shared, N_s, y_perm,
-                              (long long)T * K, nullptr, inv_row, nullptr, gate, T, K, rb, h_out,
-                              nullptr, nullptr, nullptr, s);
+                              (long long)T * K, nullptr, 0, inv_row, nullptr, gate, T, K, rb,
+                              h_out, nullptr, nullptr, nullptr, s);
   if (dt == MOE_F32)
     combine_dispatch<float>(u, y_shared, N_s, y_perm, inv_row, gate, T, d, K, h_out, s);
   else

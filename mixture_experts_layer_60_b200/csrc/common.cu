@@ -81,6 +81,12 @@ bool device_is_sm100() {
   return g_is_sm100[dev] == 1;
 }
 
+moe_status check_sm100() {
+  if (!device_is_sm100())
+    return fail(MOE_ERR_UNSUPPORTED, "libmoe kernels need an sm_100 (B200) device");
+  return MOE_OK;
+}
+
 const char* last_error_text() { return g_last_error; }
 void clear_last_error() { g_last_error[0] = 0; }
 

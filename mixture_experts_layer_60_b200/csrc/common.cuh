@@ -33,6 +33,13 @@ int sm_count();
 
 // True when the current device is compute capability 10.0 (sm_100a kernels).
 bool device_is_sm100();
+// MOE_OK on an sm_100 device, else MOE_ERR_UNSUPPORTED with a message.
+moe_status check_sm100();
+
+// The calling thread's last-error text, and its reset at the start of every
+// entry point.
+const char* last_error_text();
+void clear_last_error();
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -42,11 +49,73 @@ enum : int {
   ERR_GEMM_FP8_TIMEOUT = 2,   // FP8 tcgen05 GEMM: an mbarrier wait ran out
   ERR_EP_BOUNDS = 4,          // expert-parallel copy: a row position past its buffer (skipped)
   ERR_GATHER_TIMEOUT = 8,     // row-gather pipeline (combine and its backward): a wait ran out
+  ERR_BAD_OFFSETS = 16,       // group offsets outside [0, rows] or decreasing (clamped)
 };
 
 // ---------------------------------------------------------------- device side
 
 __device__ __forceinline__ float bf2f(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// Row range [r0, r1) of group g from the caller's offsets, clamped so that
+// 0 <= r0 <= r1 <= rows (offsets == nullptr: one group of all rows); a clamp
+// that changes a value sets ERR_BAD_OFFSETS in *err (err may be null).
+__device__ __forceinline__ void clamp_group_rows(const int32_t* offsets, int g, int rows, int* err,
+                                                 int& r0, int& r1) {
+  if (!offsets) {
+    r0 = 0;
+    r1 = rows;
+    return;
+  }
+  const int a = __ldg(offsets + g), b = __ldg(offsets + g + 1);
+  r0 = min(max(a, 0), rows);
+  r1 = min(max(b, r0), rows);
+  if (err && (r0 != a || r1 != b)) atomicOr(err, ERR_BAD_OFFSETS);
+}
+
+// roff[0..G] = the caller's group offsets made safe, by one whole warp: each
+// value clamped to [0, rows] and raised to the largest earlier one, so the
+// groups are disjoint row ranges inside [0, rows).  A change sets
+// ERR_BAD_OFFSETS in *err.  offsets == nullptr: one group [0, rows).
+__device__ __forceinline__ void load_offsets_warp(const int32_t* offsets, int G, int rows,
+                                                  int* roff, int* err) {
+  const int lane = threadIdx.x & 31;
+  if (!offsets) {
+    if (lane == 0) {
+      roff[0] = 0;
+      roff[1] = rows;
+    }
+    __syncwarp();
+    return;
+  }
+  const int n = G + 1, per = (n + 31) / 32, j0 = lane * per;
+  int run = 0;
+  for (int i = 0; i < per; ++i) {
+    const int j = j0 + i;
+    if (j < n) {
+      run = max(run, min(max(offsets[j], 0), rows));
+      roff[j] = run;
+    }
+  }
+  int incl = run;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl = max(incl, v);
+  }
+  int before = __shfl_up_sync(0xffffffffu, incl, 1);
+  if (lane == 0) before = 0;
+  bool bad = false;
+  for (int i = 0; i < per; ++i) {
+    const int j = j0 + i;
+    if (j < n) {
+      const int v = max(roff[j], before);
+      bad |= v != offsets[j];
+      roff[j] = v;
+    }
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0 && err) atomicOr(err, ERR_BAD_OFFSETS);
+  __syncwarp();
+}
 
 template <typename T> struct IO;
 template <> struct IO<float> {

@@ -34,7 +34,9 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(const Tin* __restrict__ 
     } else {
       int acc = 0;
       for (int i = 0; i < n_groups; ++i) {
-        const int m = offsets[i + 1] - offsets[i];
+        int r0, r1;
+        clamp_group_rows(offsets, i, rows, nullptr, r0, r1);
+        const int m = r1 - r0;
         const int tiles = (m + BM - 1) / BM;
         if ((int)blockIdx.y < acc + tiles) { g = i; mt = blockIdx.y - acc; break; }
         acc += tiles;
@@ -46,8 +48,8 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(const Tin* __restrict__ 
   __syncthreads();
   const int g = s_group;
   if (g < 0) return;
-  const int row0 = (offsets ? offsets[g] : 0);
-  const int row_end = (offsets ? offsets[g + 1] : rows);
+  int row0, row_end;
+  clamp_group_rows(offsets, g, rows, nullptr, row0, row_end);
   const int m0 = row0 + s_mtile * BM;
   const int n0 = blockIdx.x * BN;
   const Tin* Bg = B + (long long)g * b_group_stride;

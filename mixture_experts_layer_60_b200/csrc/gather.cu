@@ -20,14 +20,21 @@
 //   UNPERM_BWD   dh_t, dxs_j[t] (N_s), dx_perm[r_k] (K), e_k (K) -> du_t
 // Sums are float32 in the same order as the per-warp kernels (residual or
 // upstream row, shared rows j ascending, routed rows k ascending, centroid
-// terms k ascending).  A slot whose grouped row lies outside [0, n_perm) is
-// left out.
+// terms k ascending).  A slot whose grouped row lies outside [0, n_perm), or
+// (backward) whose expert id lies outside [0, N_r), is left out: nothing is
+// read for it and it takes no part in any sum.
+#include <atomic>
+
 #include "launch.h"
 #include "sm100.cuh"
 
 namespace moe {
 
 namespace {
+
+// Bound of the pipeline's stage waits (moe_set_pipeline_wait_limit).
+constexpr uint64_t kDefaultWaitNs = 1000000000ull;
+std::atomic<uint64_t> g_pipeline_wait_ns{kDefaultWaitNs};
 
 using namespace sm100;
 
@@ -47,8 +54,9 @@ struct GatherParams {
   const uint8_t* perm;       // grouped rows (y_perm or dx_perm)
   long long n_perm;          // rows of perm
   const uint8_t* cent;       // centroids E [N_r][d] (backward)
+  int N_r;                   // rows of cent (backward)
   const int32_t* inv_row;    // [T, K]
-  const int32_t* idx;        // [T, K]
+  const int32_t* idx;        // [T, K] (backward), else nullptr
   const float* w;            // gate (COMBINE, COMBINE_BWD) or d_logit (UNPERM_BWD) [T, K]
   int T, K;
   long long row_bytes;
@@ -58,6 +66,7 @@ struct GatherParams {
   float* d_logit_perm;
   int chunk;                 // bytes of a row per job
   int stages;                // a multiple of kConsumerWarps (see the ring below)
+  uint64_t wait_ns;          // bound of every wait on a stage (the drain keeps kWaitNs)
   int* err;
 };
 
@@ -66,7 +75,20 @@ __host__ __device__ inline int slots_of(int mode, int N_s, int K) {
                                                                            : 1 + N_s + 2 * K;
 }
 
-// Source row of slot `s` of token t, or nullptr (slot unused or row left out).
+// Grouped row of slot k of token t, or -1 when the slot is left out: its row
+// lies outside [0, n_perm) or, where expert ids are read (backward), its id
+// lies outside [0, N_r).
+__device__ __forceinline__ int slot_grouped_row(const GatherParams& p, int t, int k) {
+  const int r = p.inv_row[(size_t)t * p.K + k];
+  if (r < 0 || r >= p.n_perm) return -1;
+  if (p.idx) {
+    const int e = p.idx[(size_t)t * p.K + k];
+    if (e < 0 || e >= p.N_r) return -1;
+  }
+  return r;
+}
+
+// Source row of slot `s` of token t, or nullptr (slot unused or left out).
 template <int MODE>
 __device__ __forceinline__ const uint8_t* slot_row(const GatherParams& p, int t, int s) {
   const int K = p.K, N_s = p.N_s;
@@ -80,11 +102,14 @@ __device__ __forceinline__ const uint8_t* slot_row(const GatherParams& p, int t,
     s -= 1 + N_s;
   }
   if (s < K) {
-    const int r = p.inv_row[(size_t)t * K + s];
-    return (r >= 0 && r < p.n_perm) ? p.perm + (size_t)r * rb : nullptr;
+    const int r = slot_grouped_row(p, t, s);
+    return r >= 0 ? p.perm + (size_t)r * rb : nullptr;
   }
   s -= K;
-  if (MODE != GATHER_COMBINE && s < K) return p.cent + (size_t)p.idx[(size_t)t * K + s] * rb;
+  if (MODE != GATHER_COMBINE && s < K) {
+    if (slot_grouped_row(p, t, s) < 0) return nullptr;
+    return p.cent + (size_t)p.idx[(size_t)t * K + s] * rb;
+  }
   return nullptr;
 }
 
@@ -121,6 +146,7 @@ __global__ void __launch_bounds__(kThreads, 1) gather_pipe_kernel(const GatherPa
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
+    long long armed = 0;                // jobs whose copies were issued
     for (int g = blockIdx.x; g < n_groups && ok; g += gridDim.x) {
       // this lane's slots (lane, lane + 32) of the group's four tokens
       const uint8_t* src[kConsumerWarps][2];
@@ -139,7 +165,7 @@ __global__ void __launch_bounds__(kThreads, 1) gather_pipe_kernel(const GatherPa
 #pragma unroll
         for (int w = 0; w < kConsumerWarps; ++w) {
           bool got = true;
-          if (lane == 0) got = mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, kWaitNs);
+          if (lane == 0) got = mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.wait_ns);
           got = __shfl_sync(0xffffffffu, got, 0);
           if (!got) {
             if (lane == 0) { *abort_flag = 1; atomicOr(p.err, ERR_GATHER_TIMEOUT); }
@@ -152,17 +178,25 @@ __global__ void __launch_bounds__(kThreads, 1) gather_pipe_kernel(const GatherPa
           const size_t off = (size_t)q * CH;
           if (src[w][0]) bulk_load(dst + lane * CH, src[w][0] + off, cb, &full[stage]);
           if (src[w][1]) bulk_load(dst + (lane + 32) * CH, src[w][1] + off, cb, &full[stage]);
+          ++armed;
           if (++stage == S) { stage = 0; phase ^= 1; }
         }
       }
     }
-    // drain: every stage filled has been released by its consumer, so no
-    // copy is still writing shared memory
-    if (lane == 0)
-      for (int s = 0; s < S; ++s) {
-        mbar_wait_bounded(&empty[stage], phase ^ 1, nullptr, kWaitNs);
-        if (++stage == S) { stage = 0; phase ^= 1; }
+    // drain: no copy may still be writing shared memory when the block
+    // exits.  Only the last S jobs can have copies in flight, and no later
+    // job reused their stages, so each one's full barrier completes with the
+    // job's own phase whether or not a consumer took it (after an abort the
+    // consumers stop taking jobs).  One deadline bounds the whole drain.
+    if (lane == 0) {
+      const uint64_t t0 = globaltimer_ns();
+      for (long long j = armed > S ? armed - S : 0; j < armed; ++j) {
+        uint64_t* bar = &full[(int)(j % S)];
+        const uint32_t par = (uint32_t)((j / S) & 1);
+        while (!mbar_try_wait(bar, par) && globaltimer_ns() - t0 <= kWaitNs) {
+        }
       }
+    }
   } else {
     // ---------------------------------------------------------------- consumers
     // warp w takes token w of every group; in a group its job of chunk q is
@@ -184,8 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1) gather_pipe_kernel(const GatherPa
         dg[k] = 0.f;
         lg[k] = 0.f;
         if (tv && k < K) {
-          const int r = p.inv_row[(size_t)t * K + k];
-          rows[k] = (r >= 0 && r < p.n_perm) ? r : -1;
+          rows[k] = slot_grouped_row(p, t, k);
           wk[k] = p.w[(size_t)t * K + k];
         }
       }
@@ -193,7 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1) gather_pipe_kernel(const GatherPa
       for (int q = 0; q < Q; ++q, n += kConsumerWarps) {
         const int stage = (int)(n % S);
         const uint32_t phase = (uint32_t)((n / S) & 1);
-        const bool got = mbar_wait_bounded(&full[stage], phase, abort_flag, kWaitNs);
+        const bool got = mbar_wait_bounded(&full[stage], phase, abort_flag, p.wait_ns);
         if (!__all_sync(0xffffffffu, got)) {
           if (lane == 0) { *abort_flag = 1; atomicOr(p.err, ERR_GATHER_TIMEOUT); }
           ok = false;
@@ -234,16 +267,14 @@ __global__ void __launch_bounds__(kThreads, 1) gather_pipe_kernel(const GatherPa
               Vec<E>::load(row(1), fu);
 #pragma unroll
               for (int k = 0; k < KMAX; ++k) {
-                if (k < K) {
-                  if (rows[k] >= 0) {
-                    Vec<E>::load(row(2 + k), tmp);
+                if (k < K && rows[k] >= 0) {
+                  Vec<E>::load(row(2 + k), tmp);
 #pragma unroll
-                    for (int i = 0; i < N; ++i) dg[k] = fmaf(fd[i], tmp[i], dg[k]);
+                  for (int i = 0; i < N; ++i) dg[k] = fmaf(fd[i], tmp[i], dg[k]);
 #pragma unroll
-                    for (int i = 0; i < N; ++i) tmp[i] = wk[k] * fd[i];
-                    *reinterpret_cast<uint4*>(p.out + (size_t)rows[k] * p.row_bytes + gcol) =
-                        Vec<E>::store(tmp);
-                  }
+                  for (int i = 0; i < N; ++i) tmp[i] = wk[k] * fd[i];
+                  *reinterpret_cast<uint4*>(p.out + (size_t)rows[k] * p.row_bytes + gcol) =
+                      Vec<E>::store(tmp);
                   Vec<E>::load(row(2 + K + k), tmp);
 #pragma unroll
                   for (int i = 0; i < N; ++i) lg[k] = fmaf(fu[i], tmp[i], lg[k]);
@@ -266,7 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1) gather_pipe_kernel(const GatherPa
               }
 #pragma unroll
               for (int k = 0; k < KMAX; ++k) {
-                if (k < K) {
+                if (k < K && rows[k] >= 0) {
                   Vec<E>::load(row(1 + N_s + K + k), tmp);
 #pragma unroll
                   for (int i = 0; i < N; ++i) acc[i] = fmaf(wk[k], tmp[i], acc[i]);
@@ -292,10 +323,13 @@ __global__ void __launch_bounds__(kThreads, 1) gather_pipe_kernel(const GatherPa
           }
         }
         if (lane == 0) {
+          // a left-out slot is not part of the selection: no s in the sum,
+          // zero gradients
           float S_sum = 0.f, gdg = 0.f, sk[KMAX];
 #pragma unroll
           for (int k = 0; k < KMAX; ++k) {
-            if (k < K) {
+            sk[k] = 0.f;
+            if (k < K && rows[k] >= 0) {
               sk[k] = 1.0f / (1.0f + expf(-lg[k]));
               S_sum += sk[k];
               gdg = fmaf(wk[k], dg[k], gdg);
@@ -304,11 +338,12 @@ __global__ void __launch_bounds__(kThreads, 1) gather_pipe_kernel(const GatherPa
 #pragma unroll
           for (int k = 0; k < KMAX; ++k) {
             if (k < K) {
+              const bool in = rows[k] >= 0;
               const float ds = (dg[k] - gdg) / S_sum;
-              const float dl = ds * sk[k] * (1.0f - sk[k]);
-              p.d_gate[(size_t)t * K + k] = dg[k];
+              const float dl = in ? ds * sk[k] * (1.0f - sk[k]) : 0.f;
+              p.d_gate[(size_t)t * K + k] = in ? dg[k] : 0.f;
               p.d_logit[(size_t)t * K + k] = dl;
-              if (rows[k] >= 0) p.d_logit_perm[rows[k]] = dl;
+              if (in) p.d_logit_perm[rows[k]] = dl;
             }
           }
         }
@@ -344,10 +379,10 @@ bool gather_pipe_supported(int mode, int N_s, int K, long long row_bytes) {
 
 moe_status launch_gather_pipe(int mode, moe_dtype dt, const void* a, const void* b,
                               const void* sh, int N_s, const void* perm, long long n_perm,
-                              const void* cent, const int32_t* inv_row, const int32_t* idx,
-                              const float* w, int T, int K, long long row_bytes, void* out,
-                              float* d_gate, float* d_logit, float* d_logit_perm,
-                              cudaStream_t s) {
+                              const void* cent, int N_r, const int32_t* inv_row,
+                              const int32_t* idx, const float* w, int T, int K,
+                              long long row_bytes, void* out, float* d_gate, float* d_logit,
+                              float* d_logit_perm, cudaStream_t s) {
   if (T <= 0) return MOE_OK;
   GatherParams p;
   p.a = static_cast<const uint8_t*>(a);
@@ -357,8 +392,9 @@ moe_status launch_gather_pipe(int mode, moe_dtype dt, const void* a, const void*
   p.perm = static_cast<const uint8_t*>(perm);
   p.n_perm = n_perm;
   p.cent = static_cast<const uint8_t*>(cent);
+  p.N_r = N_r;
   p.inv_row = inv_row;
-  p.idx = idx;
+  p.idx = mode == GATHER_COMBINE ? nullptr : idx;
   p.w = w;
   p.T = T;
   p.K = K;
@@ -369,6 +405,7 @@ moe_status launch_gather_pipe(int mode, moe_dtype dt, const void* a, const void*
   p.d_logit_perm = d_logit_perm;
   p.err = device_error_word();
   if (!p.err) return fail(MOE_ERR_CUDA, "device error word unavailable");
+  p.wait_ns = g_pipeline_wait_ns.load(std::memory_order_relaxed);
   // a multiple of kConsumerWarps stages (one consumer warp per stage): the
   // largest chunk that fits kMaxStages of them, else the largest with four
   const int R = slots_of(mode, N_s, K);
@@ -405,3 +442,9 @@ moe_status launch_gather_pipe(int mode, moe_dtype dt, const void* a, const void*
 }
 
 }  // namespace moe
+
+extern "C" moe_status moe_set_pipeline_wait_limit(unsigned long long ns) {
+  moe::clear_last_error();
+  moe::g_pipeline_wait_ns.store(ns ? (uint64_t)ns : moe::kDefaultWaitNs, std::memory_order_relaxed);
+  return MOE_OK;
+}

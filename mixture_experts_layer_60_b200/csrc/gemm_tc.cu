@@ -139,19 +139,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   if (warp == 2) {
-    // Tile table: prefix[g] = first tile of group g (tiles ordered n-major, m fastest).
+    // Tile table: prefix[g] = first tile of group g (tiles ordered n-major, m
+    // fastest), from offsets clamped into disjoint ranges of [0, rows).
+    load_offsets_warp(p.offsets, G, p.rows, roff, p.err);
     const int per = (G + 31) / 32;
     const int g0 = lane * per;
     int local = 0;
     for (int i = 0; i < per; ++i) {
       const int g = g0 + i;
-      if (g < G) {
-        const int a = p.offsets ? p.offsets[g] : 0;
-        const int b = p.offsets ? p.offsets[g + 1] : p.rows;
-        roff[g] = a;
-        if (g == G - 1) roff[G] = b;
-        local += ((b - a + BM - 1) / BM) * n_tiles_n;
-      }
+      if (g < G) local += ((roff[g + 1] - roff[g] + BM - 1) / BM) * n_tiles_n;
     }
     int incl = local;
 #pragma unroll

@@ -61,14 +61,11 @@ struct WgParams {
   int* err;
 };
 
+// Rows [r0, r0 + cnt) of group g, clamped into [0, rows) (ERR_BAD_OFFSETS on a clamp).
 __device__ __forceinline__ void group_rows(const WgParams& p, int g, int& r0, int& cnt) {
-  if (p.offsets) {
-    r0 = __ldg(p.offsets + g);
-    cnt = __ldg(p.offsets + g + 1) - r0;
-  } else {
-    r0 = 0;
-    cnt = p.rows;
-  }
+  int r1;
+  clamp_group_rows(p.offsets, g, p.rows, p.err, r0, r1);
+  cnt = r1 - r0;
 }
 
 __device__ __forceinline__ void raise_abort(volatile int* abort, int* err) {
@@ -287,8 +284,8 @@ __global__ void __launch_bounds__(256) wgrad_tails_kernel(const uint4* __restric
                                                           const int32_t* __restrict__ offsets,
                                                           int rows, uint4* __restrict__ T) {
   const int g = blockIdx.x, i = blockIdx.y;
-  const int r0 = offsets ? offsets[g] : 0;
-  const int r1 = offsets ? offsets[g + 1] : rows;
+  int r0, r1;
+  clamp_group_rows(offsets, g, rows, nullptr, r0, r1);   // the GEMM reports a clamp
   const int cnt = r1 - r0;
   if (cnt <= 0) return;
   const int row = r0 + ((cnt - 1) / block_rows) * block_rows + i;

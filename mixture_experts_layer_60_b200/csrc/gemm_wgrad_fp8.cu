@@ -76,14 +76,11 @@ struct Wg8Params {
   }
 };
 
+// Rows [r0, r0 + cnt) of group g, clamped into [0, rows) (ERR_BAD_OFFSETS on a clamp).
 __device__ __forceinline__ void group_rows(const Wg8Params& p, int g, int& r0, int& cnt) {
-  if (p.offsets) {
-    r0 = __ldg(p.offsets + g);
-    cnt = __ldg(p.offsets + g + 1) - r0;
-  } else {
-    r0 = 0;
-    cnt = p.rows;
-  }
+  int r1;
+  clamp_group_rows(p.offsets, g, p.rows, p.err, r0, r1);
+  cnt = r1 - r0;
 }
 
 __device__ __forceinline__ void raise_abort(volatile int* abort, int* err) {

@@ -22,6 +22,13 @@
 // epilogue.  3 shared-memory stages of 64 KB; one TMEM accumulator pair
 // (512 columns).  Every wait is bounded (1 s) and reported through the
 // device error word.
+//
+// Extra groups (the shared experts of the h'-equation, weight 1): n_extra
+// groups of T_extra rows each run in the same launch after the routed
+// groups, with their own weight map (group j = row block j of W_extra) and
+// token map (gate/up: the layer input u, rows [0, T_extra); down: the same
+// h buffer as the routed rows).  Extra group j's output rows are
+// rows + j*T_extra + [0, T_extra) of C.
 #include <math.h>
 
 #include "launch.h"
@@ -69,6 +76,9 @@ struct WsParams {
   int ldc;                  // row stride of C in elements
   __nv_bfloat16* S;         // SWIGLU_SAVE: pre-activations written; DSWIGLU: read
   int lds;                  // row stride of S (2I)
+  int n_extra;              // extra groups after the routed ones (0: none)
+  int T_extra;              // rows of each extra group
+  int x_extra_local;        // 1: extra groups read X rows [0, T_extra); 0: their C rows
   int* err;
 };
 
@@ -88,23 +98,40 @@ __device__ __forceinline__ void token_tiling(int m, int& n_t, int& step) {
   n_t = (m + step - 1) / step;
 }
 
-__device__ __forceinline__ void decode_tile(int t, const int* prefix, const int* roff,
-                                            int G, int& g, int& nt,
-                                            int& tok0, int& count) {
-  int lo = 0, hi = G - 1;
+// Rows of group g: routed groups from roff, extra group j = g - G at
+// C rows base = rows + j * T_extra.
+__device__ __forceinline__ void group_span(int g, int G, const int* roff, const WsParams& p,
+                                           int& base, int& m) {
+  if (g < G) {
+    base = roff[g];
+    m = roff[g + 1] - roff[g];
+  } else {
+    base = p.rows + (g - G) * p.T_extra;
+    m = p.T_extra;
+  }
+}
+
+// Tile t -> group g, weight tile nt, first C row tok0, rows count, and the
+// first row xrow0 of X that the tile reads.
+__device__ __forceinline__ void decode_tile(int t, const int* prefix, const int* roff, int G,
+                                            int Gtot, const WsParams& p, int& g, int& nt,
+                                            int& tok0, int& count, int& xrow0) {
+  int lo = 0, hi = Gtot - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
     if (prefix[mid] <= t) lo = mid; else hi = mid - 1;
   }
   g = lo;
-  const int m = roff[g + 1] - roff[g];
+  int base, m;
+  group_span(g, G, roff, p, base, m);
   int n_t, step;
   token_tiling(m, n_t, step);
   const int local = t - prefix[g];
   nt = local / n_t;
   const int ti = local - nt * n_t;
-  tok0 = roff[g] + ti * step;
+  tok0 = base + ti * step;
   count = min(step, m - ti * step);
+  xrow0 = (g >= G && p.x_extra_local) ? ti * step : tok0;
 }
 
 __device__ __forceinline__ void raise_abort(volatile int* abort, int* err) {
@@ -118,7 +145,8 @@ __device__ __forceinline__ float silu_f(float x) { return __fdividef(x, 1.0f + _
 template <int EPI, bool WMN>
 __global__ void __launch_bounds__(kThreads, 1)
     ws_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
-                   const WsParams p) {
+                   const __grid_constant__ CUtensorMap tmW2,
+                   const __grid_constant__ CUtensorMap tmX2, const WsParams p) {
   constexpr int OUT_COLS = TileMath<EPI>::OUT_COLS;
   constexpr bool SWIGLU = TileMath<EPI>::SW;
   extern __shared__ uint8_t smem_raw[];
@@ -139,6 +167,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.offsets ? p.n_groups : 1;
+  const int Gtot = G + p.n_extra;
   const int n_wt = p.N / OUT_COLS;   // weight tiles per group
 
   if (warp == 0 && lane == 0) {
@@ -150,6 +179,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tmW);
     tma_prefetch_desc(&tmX);
+    if (p.n_extra) {
+      tma_prefetch_desc(&tmW2);
+      tma_prefetch_desc(&tmX2);
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, TMEM_COLS);
@@ -157,19 +190,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp == 2) {
     // Tile table: prefix[g] = first tile of group g; tiles of a group are
-    // ordered weight-tile major, token-tile fastest.
-    const int per = (G + 31) / 32;
+    // ordered weight-tile major, token-tile fastest.  Offsets are clamped
+    // into disjoint ranges of [0, rows) first.
+    load_offsets_warp(p.offsets, G, p.rows, roff, p.err);
+    const int per = (Gtot + 31) / 32;
     const int g0 = lane * per;
     int local = 0;
     for (int i = 0; i < per; ++i) {
       const int g = g0 + i;
-      if (g < G) {
-        const int a = p.offsets ? p.offsets[g] : 0;
-        const int b = p.offsets ? p.offsets[g + 1] : p.rows;
-        int n_t, step;
-        token_tiling(b - a, n_t, step);
-        roff[g] = a;
-        if (g == G - 1) roff[G] = b;
+      if (g < Gtot) {
+        int base, m, n_t, step;
+        group_span(g, G, roff, p, base, m);
+        token_tiling(m, n_t, step);
         local += n_t * n_wt;
       }
     }
@@ -183,20 +215,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     int run = incl - local;
     for (int i = 0; i < per; ++i) {
       const int g = g0 + i;
-      if (g < G) {
+      if (g < Gtot) {
         prefix[g] = run;
-        int n_t, step;
-        token_tiling(roff[g + 1] - roff[g], n_t, step);
+        int base, m, n_t, step;
+        group_span(g, G, roff, p, base, m);
+        token_tiling(m, n_t, step);
         run += n_t * n_wt;
       }
     }
-    if (lane == 31) prefix[G] = incl;
+    if (lane == 31) prefix[Gtot] = incl;
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int total = prefix[G];
+  const int total = prefix[Gtot];
   const int nk = p.K / BK;
 
   if (warp == 0) {
@@ -206,11 +239,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        int g, nt, tok0, count;
-        decode_tile(t, prefix, roff, G, g, nt, tok0, count);
+        int g, nt, tok0, count, xrow0;
+        decode_tile(t, prefix, roff, G, Gtot, p, g, nt, tok0, count, xrow0);
+        const bool extra = g >= G;
+        const CUtensorMap* tw = extra ? &tmW2 : &tmW;
+        const CUtensorMap* tx = extra ? &tmX2 : &tmX;
         const int nbox = (count + XBOX - 1) / XBOX;
         const uint32_t bytes = W_BYTES + nbox * XBOX_BYTES;
-        const int wrow = g * p.b_rows_per_group + nt * (SWIGLU ? 128 : 256);
+        const int wrow = (extra ? g - G : g) * p.b_rows_per_group + nt * (SWIGLU ? 128 : 256);
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, kWaitNs)) {
             raise_abort(abort_flag, p.err);
@@ -226,13 +262,13 @@ __global__ void __launch_bounds__(kThreads, 1)
               tma_load_2d(w_dst + j * WBOX_MN_BYTES, &tmW, nt * 256 + 64 * j,
                           g * p.K + kb * BK, &full[stage]);
           } else {
-            tma_load_2d(w_dst, &tmW, kb * BK, wrow, &full[stage]);
-            tma_load_2d(w_dst + W_BYTES / 2, &tmW, kb * BK, wrow + (SWIGLU ? p.half_b : 128),
+            tma_load_2d(w_dst, tw, kb * BK, wrow, &full[stage]);
+            tma_load_2d(w_dst + W_BYTES / 2, tw, kb * BK, wrow + (SWIGLU ? p.half_b : 128),
                         &full[stage]);
           }
           uint8_t* x_dst = sX + stage * X_BYTES;
           for (int b = 0; b < nbox; ++b)
-            tma_load_2d(x_dst + b * XBOX_BYTES, &tmX, kb * BK, tok0 + b * XBOX, &full[stage]);
+            tma_load_2d(x_dst + b * XBOX_BYTES, tx, kb * BK, xrow0 + b * XBOX, &full[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
@@ -246,8 +282,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0, tphase = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        int g, nt, tok0, count;
-        decode_tile(t, prefix, roff, G, g, nt, tok0, count);
+        int g, nt, tok0, count, xrow0;
+        decode_tile(t, prefix, roff, G, Gtot, p, g, nt, tok0, count, xrow0);
         const int n_mma = (count + 15) / 16 * 16;
         const uint32_t idesc = idesc_bf16_f32_major(128, n_mma, WMN, false);
         if (!mbar_wait_bounded(tempty, tphase ^ 1, abort_flag, kWaitNs)) {
@@ -292,8 +328,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint16_t* patch = reinterpret_cast<uint16_t*>(sOut + (warp - 2) * 2048);   // [32 tok][32 col]
     uint32_t tphase = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
-      int g, nt, tok0, count;
-      decode_tile(t, prefix, roff, G, g, nt, tok0, count);
+      int g, nt, tok0, count, xrow0;
+      decode_tile(t, prefix, roff, G, Gtot, p, g, nt, tok0, count, xrow0);
       const bool got = mbar_wait_bounded(tfull, tphase, abort_flag, kWaitNs);
       if (!__all_sync(0xffffffffu, got)) {
         raise_abort(abort_flag, p.err);
@@ -429,17 +465,31 @@ namespace {
 template <int EPI, bool WMN>
 moe_status ws_launch(const void* X, const void* W, int b_rows_per_group, const int32_t* offsets,
                      int n_groups, int rows, int N, int K, void* C, int ldc, void* S, int lds,
-                     cudaStream_t s) {
+                     const WsExtraGroups& ex, cudaStream_t s) {
   constexpr int OUT_COLS = TileMath<EPI>::OUT_COLS;
-  CUtensorMap tmW, tmX;
+  CUtensorMap tmW, tmX, tmW2, tmX2;
   const int G = offsets ? n_groups : 1;
+  long long x_rows = ex.n_extra && !ex.x_local ? rows + (long long)ex.n_extra * ex.T : rows;
+  if (x_rows == 0) x_rows = ex.T;   // no routed rows: a map over the extra X, never read
   moe_status st = WMN ? make_tmap_2d(&tmW, W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N,
                                      (uint64_t)G * K, 64, BK)
                       : make_tmap_2d(&tmW, W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K,
                                      (uint64_t)G * b_rows_per_group, BK, 128);
   if (st != MOE_OK) return st;
-  st = make_tmap_2d(&tmX, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, rows, BK, XBOX);
+  st = make_tmap_2d(&tmX, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, (uint64_t)x_rows, BK, XBOX);
   if (st != MOE_OK) return st;
+  tmW2 = tmW;
+  tmX2 = tmX;
+  if (ex.n_extra) {
+    st = make_tmap_2d(&tmW2, ex.W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K,
+                      (uint64_t)ex.n_extra * b_rows_per_group, BK, 128);
+    if (st != MOE_OK) return st;
+    if (ex.x_local) {
+      st = make_tmap_2d(&tmX2, ex.X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, (uint64_t)ex.T, BK,
+                        XBOX);
+      if (st != MOE_OK) return st;
+    }
+  }
   auto kern = ws_gemm_kernel<EPI, WMN>;
   static bool attr_done[kMaxSmemDevices] = {};   // per instantiation and device
   {
@@ -459,12 +509,17 @@ moe_status ws_launch(const void* X, const void* W, int b_rows_per_group, const i
   p.ldc = ldc;
   p.S = static_cast<__nv_bfloat16*>(S);
   p.lds = lds;
+  p.n_extra = ex.n_extra;
+  p.T_extra = ex.T;
+  p.x_extra_local = ex.x_local ? 1 : 0;
   p.err = device_error_word();
   if (!p.err) return fail(MOE_ERR_CUDA, "device error word unavailable");
-  const long long max_tiles = ((long long)(rows + TMAX - 1) / TMAX + (offsets ? G : 0)) * (N / OUT_COLS);
+  const long long max_tiles =
+      ((long long)(rows + TMAX - 1) / TMAX + (offsets ? G : 0) +
+       (long long)ex.n_extra * ((ex.T + TMAX - 1) / TMAX)) * (N / OUT_COLS);
   int grid = sm_count();
   if (max_tiles < grid) grid = (int)(max_tiles > 0 ? max_tiles : 1);
-  kern<<<grid, kThreads, SMEM_ALLOC, s>>>(tmW, tmX, p);
+  kern<<<grid, kThreads, SMEM_ALLOC, s>>>(tmW, tmX, tmW2, tmX2, p);
   return cuda_check(cudaGetLastError(), "ws_gemm launch");
 }
 
@@ -472,16 +527,20 @@ moe_status ws_launch(const void* X, const void* W, int b_rows_per_group, const i
 
 moe_status launch_ws_gemm(const void* X, const void* W, int b_rows_per_group,
                           const int32_t* offsets, int n_groups, int rows, int N, int K,
-                          bool swiglu, void* C, cudaStream_t s) {
+                          bool swiglu, void* C, cudaStream_t s, const WsExtraGroups* extra) {
   return launch_ws_gemm_ex(X, W, b_rows_per_group, offsets, n_groups, rows, N, K,
-                           swiglu ? WS_SWIGLU : WS_STORE, false, C, N, nullptr, 0, s);
+                           swiglu ? WS_SWIGLU : WS_STORE, false, C, N, nullptr, 0, s, extra);
 }
 
 moe_status launch_ws_gemm_ex(const void* X, const void* W, int b_rows_per_group,
                              const int32_t* offsets, int n_groups, int rows, int N, int K,
                              WsEpi epi, bool w_mn, void* C, int ldc, void* S, int lds,
-                             cudaStream_t s) {
-  if (rows <= 0) return MOE_OK;
+                             cudaStream_t s, const WsExtraGroups* extra) {
+  const WsExtraGroups none{};
+  const WsExtraGroups& ex = extra ? *extra : none;
+  if (ex.n_extra && (epi == WS_SWIGLU_SAVE || epi == WS_DSWIGLU || w_mn))
+    return fail(MOE_ERR_UNSUPPORTED, "ws gemm: extra groups only with the forward epilogues");
+  if (rows <= 0 && (ex.n_extra == 0 || ex.T <= 0)) return MOE_OK;
   if (K % BK) return fail(MOE_ERR_UNSUPPORTED, "ws gemm: K=%d not a multiple of %d", K, BK);
   if (offsets && n_groups > kMaxGroups)
     return fail(MOE_ERR_UNSUPPORTED, "ws gemm: at most %d groups", kMaxGroups);
@@ -492,19 +551,19 @@ moe_status launch_ws_gemm_ex(const void* X, const void* W, int b_rows_per_group,
   switch (epi) {
     case WS_SWIGLU:
       return ws_launch<WS_SWIGLU, false>(X, W, b_rows_per_group, offsets, n_groups, rows, N, K,
-                                         C, ldc, S, lds, s);
+                                         C, ldc, S, lds, ex, s);
     case WS_SWIGLU_SAVE:
       return ws_launch<WS_SWIGLU_SAVE, false>(X, W, b_rows_per_group, offsets, n_groups, rows,
-                                              N, K, C, ldc, S, lds, s);
+                                              N, K, C, ldc, S, lds, ex, s);
     case WS_STORE:
       return w_mn ? ws_launch<WS_STORE, true>(X, W, b_rows_per_group, offsets, n_groups, rows, N,
-                                              K, C, ldc, S, lds, s)
+                                              K, C, ldc, S, lds, ex, s)
                   : ws_launch<WS_STORE, false>(X, W, b_rows_per_group, offsets, n_groups, rows,
-                                               N, K, C, ldc, S, lds, s);
+                                               N, K, C, ldc, S, lds, ex, s);
     case WS_DSWIGLU:
       if (!w_mn) return fail(MOE_ERR_UNSUPPORTED, "ws gemm dswiglu: needs MN-major weights");
       return ws_launch<WS_DSWIGLU, true>(X, W, b_rows_per_group, offsets, n_groups, rows, N, K,
-                                         C, ldc, S, lds, s);
+                                         C, ldc, S, lds, ex, s);
   }
   return fail(MOE_ERR_INVALID_ARG, "ws gemm: unknown epilogue %d", (int)epi);
 }

@@ -14,15 +14,20 @@ moe_status launch_logits_simt(const void* u, const void* E, moe_dtype dt, int T,
 //   hdr[0]  tokens listed, hdr[1] candidate pairs (both zeroed before top-K)
 //   tok, start, num [T]   per listed token: its id, first pair, number of pairs
 //   pair [T*N_r]          candidate (token, expert) as t*N_r + e, grouped per token
-//   s64  [T*N_r]          float32: the pair's float64 affinity, rounded once
 struct RefineLists {
   int32_t* hdr;
   int32_t* tok;
   int32_t* start;
   int32_t* num;
   int32_t* pair;
-  float* s64;
 };
+// A token whose selection or output order was decided by a key gap below
+// kRouterRefineGap is listed with every expert whose float32 key lies within
+// kRouterNearBoundary of the lowest key a decision hinged on; the tie-break
+// recomputes those experts' affinities in float64.  Both are set from the
+// bound on the float32 key error of the tensor-core logits.
+constexpr float kRouterRefineGap = 2e-5f;
+constexpr float kRouterNearBoundary = 6e-5f;
 // sigmoid, biased top-K, gates, histogram (counts must be zeroed beforehand).
 // n_groups > 1 && topk_groups < n_groups restricts each token to its best groups.
 // A token whose routing was decided by a key gap < refine_gap is listed with
@@ -30,8 +35,20 @@ struct RefineLists {
 moe_status launch_topk(const float* logits, const float* b, int T, int N_r, int K, int n_groups,
                        int topk_groups, int32_t* idx, float* gate, int32_t* counts,
                        RefineLists rl, float refine_gap, cudaStream_t s);
-// Float64 affinities of the listed pairs, then the listed tokens' routing
-// redone from them.
+
+// router_tc.cu ----------------------------------------------------------------
+// The fused router (logits on tcgen05 CTA pairs, sigmoid, biased top-K, gates,
+// load, near-tie listing) for bf16 u and E with 32 <= N_r <= 256, N_r % 32 == 0,
+// K <= 16 and, under a group limit, groups of a power-of-two size.  Writes the
+// float32 logits rows of listed tokens only; counts must be zeroed and the
+// tie-break header cleared beforehand.
+bool router_tc_supported(moe_dtype dt, int d, int N_r, int K, int n_groups, int topk_groups);
+moe_status launch_router_tc(const void* u, const void* E, const float* b, int T, int d, int N_r,
+                            int K, int n_groups, int topk_groups, int32_t* idx, float* gate,
+                            int32_t* counts, float* logits, RefineLists rl, float refine_gap,
+                            float near, cudaStream_t s);
+// Per listed token: float64 affinities of its listed experts, then its
+// routing redone from them.
 moe_status launch_refine(const void* u, const void* E, moe_dtype dt, const float* logits,
                          const float* b, int d, int N_r, int K, int n_groups, int topk_groups,
                          RefineLists rl, int T, int32_t* idx, float* gate, int32_t* counts,
@@ -39,6 +56,13 @@ moe_status launch_refine(const void* u, const void* E, moe_dtype dt, const float
 
 // permute.cu -----------------------------------------------------------------
 size_t permute_ws_bytes(int T, int N_r);
+// Argument checks shared by moe_permute and moe_permute_noalloc (api.cu);
+// on success *elem_bytes is the size of one element of a row.
+moe_status validate_permute_args(const char* who, const void* u, const float* u_scale,
+                                 moe_dtype dt, const int32_t* topk_idx, int T, int d, int N_r,
+                                 int K, const void* x_perm, const float* x_scale,
+                                 const int32_t* offsets, const int32_t* perm_src,
+                                 const int32_t* inv_row, int* elem_bytes);
 moe_status launch_permute(const void* u, const float* u_scale, int elem_bytes, const int32_t* idx,
                           int T, int d, int N_r, int K, void* x_perm, float* x_scale,
                           int32_t* offsets, int32_t* perm_src, int32_t* inv_row,
@@ -64,9 +88,20 @@ moe_status launch_tc_gemm(const void* A, const void* B, int b_rows_per_group,
 // Weights-stationary grouped bf16 GEMM (expert FFNs): weights on the MMA's M
 // side, each expert's tokens on N (tiles of <= 256 tokens, 16-row granularity).
 // swiglu: B holds W_gate rows [0, I) and W_up rows [I, 2I) of a group.
+// Extra groups (shared experts) run in the same launch: n_extra groups of T
+// rows, weights W (row block j for group j), output rows rows + j*T of C;
+// x_local: they read rows [0, T) of X (else their own C rows of the main X).
+struct WsExtraGroups {
+  const void* X = nullptr;
+  const void* W = nullptr;
+  int n_extra = 0;
+  int T = 0;
+  bool x_local = false;
+};
 moe_status launch_ws_gemm(const void* X, const void* W, int b_rows_per_group,
                           const int32_t* offsets, int n_groups, int rows, int N, int K,
-                          bool swiglu, void* C, cudaStream_t s);
+                          bool swiglu, void* C, cudaStream_t s,
+                          const WsExtraGroups* extra = nullptr);
 // Epilogues: SWIGLU  C = SiLU(gate) * up (N = I columns);
 //            SWIGLU_SAVE  the same, plus S[:, 0:I] = gate, S[:, I:2I] = up;
 //            STORE   C = the product (N columns);
@@ -77,7 +112,7 @@ enum WsEpi { WS_SWIGLU = 0, WS_STORE = 1, WS_SWIGLU_SAVE = 2, WS_DSWIGLU = 3 };
 moe_status launch_ws_gemm_ex(const void* X, const void* W, int b_rows_per_group,
                              const int32_t* offsets, int n_groups, int rows, int N, int K,
                              WsEpi epi, bool w_mn, void* C, int ldc, void* S, int lds,
-                             cudaStream_t s);
+                             cudaStream_t s, const WsExtraGroups* extra = nullptr);
 
 // gather.cu ------------------------------------------------------------------
 // Row-gather pipeline (bulk copies into a shared-memory ring, one producer
@@ -87,13 +122,15 @@ enum GatherMode { GATHER_COMBINE = 0, GATHER_COMBINE_BWD = 1, GATHER_UNPERM_BWD 
 // COMBINE_BWD 2 + 2K, UNPERM_BWD 1 + N_s + 2K) are at most 64.
 bool gather_pipe_supported(int mode, int N_s, int K, long long row_bytes);
 // a: u (COMBINE) or dh; b: u (COMBINE_BWD); sh: shared-expert rows [N_s][T];
-// perm: grouped rows (n_perm of them); cent: centroids; w: gate or d_logit.
+// perm: grouped rows (n_perm of them); cent: centroids [N_r] (backward);
+// w: gate or d_logit.  Slots with a grouped row outside [0, n_perm) or
+// (backward) an expert id outside [0, N_r) are left out.
 moe_status launch_gather_pipe(int mode, moe_dtype dt, const void* a, const void* b,
                               const void* sh, int N_s, const void* perm, long long n_perm,
-                              const void* cent, const int32_t* inv_row, const int32_t* idx,
-                              const float* w, int T, int K, long long row_bytes, void* out,
-                              float* d_gate, float* d_logit, float* d_logit_perm,
-                              cudaStream_t s);
+                              const void* cent, int N_r, const int32_t* inv_row,
+                              const int32_t* idx, const float* w, int T, int K,
+                              long long row_bytes, void* out, float* d_gate, float* d_logit,
+                              float* d_logit_perm, cudaStream_t s);
 
 // gemm_wgrad.cu --------------------------------------------------------------
 // C[g] [M, N] = sum over the rows r of group g of A[r, :]^T B[r, :] (bf16 in and out).
@@ -154,12 +191,12 @@ moe_status launch_bias_update(float* b, const int32_t* counts, int N_r, int T, i
 moe_status launch_combine_backward(const void* dh, const void* u, const void* E,
                                    const void* y_perm, const int32_t* inv_row,
                                    const int32_t* idx, const float* gate, moe_dtype dt, int T,
-                                   int d, int K, void* dy_perm, float* d_gate, float* d_logit,
-                                   float* d_logit_perm, cudaStream_t s);
+                                   int d, int K, int N_r, void* dy_perm, float* d_gate,
+                                   float* d_logit, float* d_logit_perm, cudaStream_t s);
 moe_status launch_unpermute_backward(const void* dh, const void* dx_shared, int N_s,
                                      const void* dx_perm, const int32_t* inv_row,
                                      const int32_t* idx, const float* d_logit, const void* E,
-                                     moe_dtype dt, int T, int d, int K, void* du,
+                                     moe_dtype dt, int T, int d, int K, int N_r, void* du,
                                      cudaStream_t s);
 moe_status launch_router_weight_grad(const void* x, const int32_t* x_rows,
                                      const float* d_logit_perm, const int32_t* offsets,

@@ -216,10 +216,15 @@ moe_status launch_permute(const void* u, const float* u_scale, int elem_bytes, c
 // In host code the array's name is only a host-side handle, so its device
 // address is looked up once per device (cudaGetSymbolAddress, with that
 // device current) on the first call there; make that first call before any
-// stream capture.  All calls share the array: two calls whose work overlaps
-// on the GPU (different streams, or different host threads) race on it.
-// Every word a call reads is first written by the same call, so nothing has
-// to be cleared between calls.
+// stream capture.  The per-device cache is atomic, so host threads may race
+// on the first lookup (they store the same address).  A cudaDeviceReset
+// unloads the library's device arrays; the cached address is then stale, so
+// the library must not be used across a reset.  All calls share the array:
+// two calls whose work overlaps on the GPU (different streams, or different
+// host threads) race on it.  Every word a call reads is first written by the
+// same call, so nothing has to be cleared between calls.
+#include <atomic>
+
 namespace moe {
 namespace {
 
@@ -227,7 +232,7 @@ constexpr size_t kNoAllocScratchBytes = 1u << 20;   // 1 MiB: T up to 131072 at 
 constexpr int kNoAllocMaxDevices = 64;
 
 __device__ __align__(256) unsigned char g_permute_scratch[kNoAllocScratchBytes];
-void* g_permute_scratch_addr[kNoAllocMaxDevices] = {nullptr};
+std::atomic<void*> g_permute_scratch_addr[kNoAllocMaxDevices];
 
 moe_status permute_scratch_address(void** out) {
   int dev = -1;
@@ -235,15 +240,15 @@ moe_status permute_scratch_address(void** out) {
   if (e != cudaSuccess) return cuda_check(e, "moe_permute_noalloc: cudaGetDevice");
   if (dev < 0 || dev >= kNoAllocMaxDevices)
     return fail(MOE_ERR_UNSUPPORTED, "moe_permute_noalloc: device %d out of range", dev);
-  if (!g_permute_scratch_addr[dev]) {
-    void* p = nullptr;
+  void* p = g_permute_scratch_addr[dev].load(std::memory_order_acquire);
+  if (!p) {
     e = cudaGetSymbolAddress(&p, g_permute_scratch);
     if (e != cudaSuccess || !p)
       return cuda_check(e != cudaSuccess ? e : cudaErrorInvalidSymbol,
                         "moe_permute_noalloc: cudaGetSymbolAddress of the static scratch");
-    g_permute_scratch_addr[dev] = p;
+    g_permute_scratch_addr[dev].store(p, std::memory_order_release);
   }
-  *out = g_permute_scratch_addr[dev];
+  *out = p;
   return MOE_OK;
 }
 
@@ -255,41 +260,25 @@ extern "C" moe_status moe_permute_noalloc(const void* u, const float* u_scale, m
                                           void* x_perm, float* x_scale, int32_t* offsets,
                                           int32_t* perm_src, int32_t* inv_row, void* stream) {
   using namespace moe;
-  const int eb = dt == MOE_F32 ? 4 : dt == MOE_BF16 ? 2 : dt == MOE_E4M3 ? 1 : 0;
-  if (eb == 0) return fail(MOE_ERR_UNSUPPORTED, "moe_permute_noalloc: unknown dtype %d", (int)dt);
-  if (T < 0 || d <= 0 || N_r <= 0 || K <= 0)
-    return fail(MOE_ERR_INVALID_ARG, "moe_permute_noalloc: bad sizes T=%d d=%d N_r=%d K=%d", T,
-                d, N_r, K);
-  if (N_r > 1024 || K > N_r)
-    return fail(MOE_ERR_UNSUPPORTED, "moe_permute_noalloc: need 1 <= K <= N_r <= 1024");
-  if (((size_t)d * eb) % 16 != 0)
-    return fail(MOE_ERR_UNSUPPORTED, "moe_permute_noalloc: a row must be a multiple of 16 bytes");
-  if (!offsets) return fail(MOE_ERR_INVALID_ARG, "moe_permute_noalloc: null offsets");
-  if (T > 0 && !(u && topk_idx && x_perm && perm_src && inv_row))
-    return fail(MOE_ERR_INVALID_ARG, "moe_permute_noalloc: null pointer");
-  if (dt == MOE_E4M3) {
-    if (d % 128) return fail(MOE_ERR_UNSUPPORTED, "moe_permute_noalloc: e4m3 needs d %% 128 == 0");
-    if (T > 0 && !(u_scale && x_scale))
-      return fail(MOE_ERR_INVALID_ARG, "moe_permute_noalloc: e4m3 needs u_scale and x_scale");
-  } else if (u_scale || x_scale) {
-    return fail(MOE_ERR_INVALID_ARG, "moe_permute_noalloc: scales are only for MOE_E4M3");
-  }
-  if (reinterpret_cast<uintptr_t>(u) % 16 || reinterpret_cast<uintptr_t>(x_perm) % 16)
-    return fail(MOE_ERR_INVALID_ARG, "moe_permute_noalloc: u and x_perm must be 16-byte aligned");
+  clear_last_error();
+  int eb = 0;
+  moe_status st = validate_permute_args("moe_permute_noalloc", u, u_scale, dt, topk_idx, T, d,
+                                        N_r, K, x_perm, x_scale, offsets, perm_src, inv_row, &eb);
+  if (st != MOE_OK) return st;
   const size_t need = T > 0 ? permute_ws_bytes(T, N_r) : 0;
   if (need > kNoAllocScratchBytes)
     return fail(MOE_ERR_UNSUPPORTED,
                 "moe_permute_noalloc: T=%d, N_r=%d needs %zu bytes of scratch, more than the "
                 "%zu-byte static array; use moe_permute with a workspace",
                 T, N_r, need, kNoAllocScratchBytes);
-  if (!device_is_sm100())
-    return fail(MOE_ERR_UNSUPPORTED, "libmoe kernels need an sm_100 (B200) device");
+  st = check_sm100();
+  if (st != MOE_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (T == 0)
     return cuda_check(cudaMemsetAsync(offsets, 0, (size_t)(N_r + 1) * sizeof(int32_t), s),
                       "zero offsets");
   void* scratch = nullptr;
-  moe_status st = permute_scratch_address(&scratch);
+  st = permute_scratch_address(&scratch);
   if (st != MOE_OK) return st;
   return launch_permute(u, dt == MOE_E4M3 ? u_scale : nullptr, eb, topk_idx, T, d, N_r, K, x_perm,
                         dt == MOE_E4M3 ? x_scale : nullptr, offsets, perm_src, inv_row, scratch, s);

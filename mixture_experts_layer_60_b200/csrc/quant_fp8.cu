@@ -127,6 +127,8 @@ namespace {
 // every column of a block gets its own scale.
 
 // block_start[g] = sum over g' < g of ceil(rows of g' / 128); block_start[G] = total.
+// A group's rows are clamped into [0, rows) (its size is never negative), so
+// the total never exceeds ceil(rows / 128) + G.
 __global__ void __launch_bounds__(1024) block_table_kernel(const int32_t* __restrict__ offsets,
                                                            int G, int rows,
                                                            int32_t* __restrict__ block_start) {
@@ -137,8 +139,9 @@ __global__ void __launch_bounds__(1024) block_table_kernel(const int32_t* __rest
     const int g = base + t;
     int c = 0;
     if (g < G) {
-      const int n = offsets ? offsets[g + 1] - offsets[g] : rows;
-      c = (n + 127) / 128;
+      int r0, r1;
+      clamp_group_rows(offsets, g, rows, nullptr, r0, r1);
+      c = (r1 - r0 + 127) / 128;
     }
     int incl = c;
 #pragma unroll
@@ -183,8 +186,8 @@ __global__ void __launch_bounds__(128) quant_128x1_kernel(
     const int mid = (lo + hi + 1) >> 1;
     if (block_start[mid] <= blk) lo = mid; else hi = mid - 1;
   }
-  const int g0 = offsets ? offsets[lo] : 0;
-  const int g1 = offsets ? offsets[lo + 1] : rows;
+  int g0, g1;
+  clamp_group_rows(offsets, lo, rows, nullptr, g0, g1);
   const int r0 = g0 + (blk - block_start[lo]) * 128;
   const int r1 = min(r0 + 128, g1);
   const int c = (blockIdx.y * 128 + threadIdx.x) * 2;

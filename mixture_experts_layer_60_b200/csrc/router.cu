@@ -19,13 +19,12 @@ moe_status launch_logits_simt(const void* u, const void* E, moe_dtype dt, int T,
 // Precise tie-break.  The tensor-core logits are float32 sums of d products,
 // which can move s by a few 1e-6 at V3 width.  A token whose routing was
 // decided by a key gap below the refine gap is listed together with the
-// experts whose float32 key lies within kNearBoundary of one of its decision
+// experts whose float32 key lies within kRouterNearBoundary of one of its decision
 // boundaries; those experts get float64 logits (s = Sigmoid in float64,
 // rounded once to float32: the affinity line's exact value) and the token is
 // routed again.  The other experts keep their float32 keys, which are too far
 // below every boundary for the float32 error to matter.  If the group choice
 // changes, every expert of the token is recomputed.
-constexpr float kNearBoundary = 6e-5f;   // > 2 x the largest float32 key error
 
 // Order-preserving map of a float key to an unsigned integer (every real key
 // maps above 0; -0 is taken as +0, so equal keys map to equal integers).
@@ -182,7 +181,7 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
       // list the token with every expert whose float32 key is near the lowest
       // key a decision hinged on (the (K+1)-th key inside the kept groups and,
       // with the group limit, the best excluded group's score)
-      const float thr = fminf(next_key, next_group) - kNearBoundary;
+      const float thr = fminf(next_key, next_group) - kRouterNearBoundary;
       int c = 0;
 #pragma unroll
       for (int j = 0; j < V; ++j)
@@ -267,34 +266,6 @@ __device__ __forceinline__ float exact_affinity_warp(const Tin* __restrict__ ut,
   return affinity64(acc);
 }
 
-// One block of kDotThreads per listed pair: s64[p] = float64 affinity.
-constexpr int kDotThreads = 128;
-template <typename Tin>
-__global__ void __launch_bounds__(kDotThreads) refine_dot_kernel(const Tin* __restrict__ u,
-                                                                 const Tin* __restrict__ E, int d,
-                                                                 int N_r, RefineLists rl) {
-  __shared__ double part[kDotThreads / 32];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int n = rl.hdr[1];
-  const int nv = d / (16 / (int)sizeof(Tin));
-  for (int p = blockIdx.x; p < n; p += gridDim.x) {
-    const int code = rl.pair[p];
-    const int t = code / N_r, e = code - t * N_r;
-    double acc = dot64_part(u + (size_t)t * d, E + (size_t)e * d, nv, threadIdx.x, kDotThreads);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) part[warp] = acc;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      double a = 0.0;
-#pragma unroll
-      for (int w = 0; w < kDotThreads / 32; ++w) a += part[w];
-      rl.s64[p] = affinity64(a);
-    }
-    __syncthreads();
-  }
-}
-
 // Warp-wide arg-max of (key desc, index asc) over keys held lane-strided in kv[].
 __device__ __forceinline__ void warp_best(const float* kv, int N_r, int lane, float& bk, int& be) {
   bk = -INFINITY;
@@ -332,11 +303,14 @@ __device__ __forceinline__ unsigned keep_groups(const float* kv, int N_r, int n_
   return kept;
 }
 
-// One block per listed token: float32 keys for every expert, the float64
-// affinities of its listed experts on top, then selection, gates and load
-// redone (a changed group choice recomputes every expert in float64).
+// One block per listed token: the float64 affinities of its listed experts
+// (one warp per expert), float32 keys for every other expert (from the
+// float32 logits, as the selection computed them), then selection, gates and
+// load redone; a changed group choice recomputes every expert in float64.
+// A token's listed experts are pair[start, start + num) (t*N_r + e codes).
+constexpr int kRefineThreads = 256;
 template <typename Tin>
-__global__ void __launch_bounds__(256) refine_select_kernel(
+__global__ void __launch_bounds__(kRefineThreads) refine_token_kernel(
     const Tin* __restrict__ u, const Tin* __restrict__ E, const float* __restrict__ logits,
     const float* __restrict__ bias, int d, int N_r, int K, int n_groups, int topk_groups,
     RefineLists rl, int32_t* __restrict__ idx, float* __restrict__ gate,
@@ -345,6 +319,7 @@ __global__ void __launch_bounds__(256) refine_select_kernel(
   float* sv = sm_r;            // s [N_r]
   float* kv = sv + N_r;        // key [N_r]
   float* kw = kv + N_r;        // scratch keys [N_r]
+  float* s64 = kw + N_r;       // float64 affinity of listed expert c, rounded once [N_r]
   __shared__ int s_full;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   const bool grouped = n_groups > 1 && topk_groups < n_groups;
@@ -352,18 +327,20 @@ __global__ void __launch_bounds__(256) refine_select_kernel(
   const int n = rl.hdr[0];
   for (int i = blockIdx.x; i < n; i += gridDim.x) {
     const int t = rl.tok[i], p0 = rl.start[i], np = rl.num[i];
+    for (int c = warp; c < np; c += nw) {
+      const int e = rl.pair[p0 + c] - t * N_r;
+      const float sf = exact_affinity_warp(u + (size_t)t * d, E + (size_t)e * d, d, lane);
+      if (lane == 0) s64[c] = sf;
+    }
     for (int e = threadIdx.x; e < N_r; e += blockDim.x) {
-      const float sf = 1.0f / (1.0f + expf(-logits[(size_t)t * N_r + e]));   // as the top-K kernel
+      const float sf = 1.0f / (1.0f + expf(-logits[(size_t)t * N_r + e]));   // as the selection
       sv[e] = sf;
       kw[e] = sf + bias[e];
     }
     __syncthreads();
     unsigned kept32 = 0xffffffffu;
     if (grouped && warp == 0) kept32 = keep_groups(kw, N_r, n_groups, topk_groups, lane);
-    for (int c = threadIdx.x; c < np; c += blockDim.x) {
-      const int e = rl.pair[p0 + c] - t * N_r;
-      sv[e] = rl.s64[p0 + c];
-    }
+    for (int c = threadIdx.x; c < np; c += blockDim.x) sv[rl.pair[p0 + c] - t * N_r] = s64[c];
     __syncthreads();
     for (int e = threadIdx.x; e < N_r; e += blockDim.x) kv[e] = sv[e] + bias[e];
     __syncthreads();
@@ -421,39 +398,26 @@ moe_status launch_refine(const void* u, const void* E, moe_dtype dt, const float
                          const float* b, int d, int N_r, int K, int n_groups, int topk_groups,
                          RefineLists rl, int T, int32_t* idx, float* gate, int32_t* counts,
                          cudaStream_t s) {
-  // pairs: a fixed grid striding over the device-side count
-  const int dot_blocks = 16 * sm_count();
-  if (dt == MOE_F32)
-    refine_dot_kernel<float><<<dot_blocks, kDotThreads, 0, s>>>(
-        static_cast<const float*>(u), static_cast<const float*>(E), d, N_r, rl);
-  else
-    refine_dot_kernel<__nv_bfloat16><<<dot_blocks, kDotThreads, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(u), static_cast<const __nv_bfloat16*>(E), d, N_r, rl);
-  {
-    const moe_status st = cuda_check(cudaGetLastError(), "refine_dot_kernel launch");
-    if (st != MOE_OK) return st;
-  }
-  const int threads = 256;
   int blocks = 2 * sm_count();
   if (blocks > T) blocks = T > 0 ? T : 1;
-  const size_t smem = (size_t)3 * N_r * sizeof(float);
+  const size_t smem = (size_t)4 * N_r * sizeof(float);
   if (smem > 48 * 1024) {
     cudaError_t e = dt == MOE_F32
-        ? cudaFuncSetAttribute(refine_select_kernel<float>,
+        ? cudaFuncSetAttribute(refine_token_kernel<float>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
-        : cudaFuncSetAttribute(refine_select_kernel<__nv_bfloat16>,
+        : cudaFuncSetAttribute(refine_token_kernel<__nv_bfloat16>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return cuda_check(e, "refine_select_kernel smem attribute");
+    if (e != cudaSuccess) return cuda_check(e, "refine_token_kernel smem attribute");
   }
   if (dt == MOE_F32)
-    refine_select_kernel<float><<<blocks, threads, smem, s>>>(
+    refine_token_kernel<float><<<blocks, kRefineThreads, smem, s>>>(
         static_cast<const float*>(u), static_cast<const float*>(E), logits, b, d, N_r, K,
         n_groups, topk_groups, rl, idx, gate, counts);
   else
-    refine_select_kernel<__nv_bfloat16><<<blocks, threads, smem, s>>>(
+    refine_token_kernel<__nv_bfloat16><<<blocks, kRefineThreads, smem, s>>>(
         static_cast<const __nv_bfloat16*>(u), static_cast<const __nv_bfloat16*>(E), logits, b, d,
         N_r, K, n_groups, topk_groups, rl, idx, gate, counts);
-  return cuda_check(cudaGetLastError(), "refine_select_kernel launch");
+  return cuda_check(cudaGetLastError(), "refine_token_kernel launch");
 }
 
 moe_status launch_topk(const float* logits, const float* b, int T, int N_r, int K, int n_groups,

@@ -2,8 +2,10 @@
 
 MoELayer owns the layer's device state (centroids, bias, expert weights,
 FP8 copies of them) and the per-step buffers, and runs one step as
-    moe_route -> [moe_quantize_1x128] -> moe_permute -> moe_expert_ffn (routed)
-    -> moe_expert_ffn (each shared expert) -> moe_combine [-> moe_bias_update]
+    moe_route -> [moe_quantize_1x128] -> moe_permute
+    -> gate/up and down of the routed experts (bf16: with the shared experts
+       as extra groups of the same two launches; FP8 / f32: the shared
+       experts' moe_expert_ffn after them) -> moe_combine [-> moe_bias_update]
 on one CUDA stream.  For training (bf16 or FP8), forward_train keeps the
 activations the backward needs and backward(dh) returns du and fills
 self.grad with the gradients of E and of every expert weight.  Every step of the layer runs in libmoe's kernels; this
@@ -14,9 +16,9 @@ from __future__ import annotations
 import torch
 
 from . import (MOE_BF16, MOE_E4M3, MOE_F32, moe_bias_update, moe_combine, moe_combine_backward,
-               moe_expert_down, moe_expert_ffn, moe_expert_ffn_backward,
+               moe_expert_down, moe_expert_down_shared, moe_expert_ffn, moe_expert_ffn_backward,
                moe_expert_ffn_backward_workspace_size, moe_expert_ffn_workspace_size,
-               moe_expert_gate_up, moe_expert_gate_up_save, moe_permute,
+               moe_expert_gate_up, moe_expert_gate_up_save, moe_expert_gate_up_shared, moe_permute,
                moe_permute_workspace_size, moe_quantize_128x128, moe_quantize_1x128, moe_route,
                moe_route_grouped, moe_route_workspace_size, moe_router_weight_grad,
                moe_unpermute_backward)
@@ -68,11 +70,18 @@ class MoELayer:
         self.offsets = torch.zeros(N_r + 1, dtype=torch.int32, device=dev)
         self.perm_src = torch.empty(R, dtype=torch.int32, device=dev)
         self.inv_row = torch.empty(T, K, dtype=torch.int32, device=dev)
-        self.y_perm = torch.empty(R, d, dtype=act, device=dev)
-        self.y_shared = torch.empty(N_s, T, d, dtype=act, device=dev)
+        # bf16: the shared experts run as extra groups of the routed launches,
+        # their rows after the routed ones in the same h and y buffers
+        self.merged_shared = (c.dtype == "bf16" and N_s > 0 and d % 256 == 0
+                              and c.I % 128 == 0)
+        self.y_all = torch.empty(R + N_s * T, d, dtype=act, device=dev)
+        self.y_perm = self.y_all[:R]
+        self.y_shared = self.y_all[R:].view(N_s, T, d)
         self.ffn_ws = _ws(moe_expert_ffn_workspace_size(ffn_dt, T, c.I), dev)
         hdt = torch.uint8 if self.fp8 else act
-        self.h_mid = torch.empty(R, c.I, dtype=hdt, device=dev)
+        self.h_all = torch.empty(R + (N_s * T if self.merged_shared else 0), c.I, dtype=hdt,
+                                 device=dev)
+        self.h_mid = self.h_all[:R]
         self.h_scale = torch.empty(R, c.I // 128, dtype=torch.float32, device=dev) if self.fp8 \
             else None
         self.h_out = torch.empty(T, d, dtype=act, device=dev)
@@ -85,21 +94,34 @@ class MoELayer:
 
     # -- one step ------------------------------------------------------------
     def forward(self, u: torch.Tensor, stream=None, gate_up_events=None,
-                out: torch.Tensor | None = None) -> torch.Tensor:
+                out: torch.Tensor | None = None, phase_events=None) -> torch.Tensor:
         """h' for the T tokens of u, written to `out` (default: the layer's own
         h_out buffer, overwritten by the next call).  gate_up_events=(start,
         end) records CUDA events around the routed gate/up GEMM launch on the
-        same stream."""
+        same stream; phase_events, a dict name -> (start, end) for any of
+        "route", "permute", "gate_up", "down", "shared", "combine", records
+        events around those phases."""
         c = self.cfg
         T = u.shape[0]
         if T != self.T_alloc:
             self._alloc(T)
+        st = torch.cuda.current_stream() if stream is None else stream
+        pe = phase_events or {}
+        if gate_up_events:
+            pe = dict(pe, gate_up=gate_up_events)
+
+        def mark(name, i):
+            if name in pe:
+                pe[name][i].record(st)
+        mark("route", 0)
         if c.n_groups > 1:
             moe_route_grouped(u, self.E, self.b, c.K, c.n_groups, c.topk_groups, self.topk_idx,
                               self.topk_gate, self.counts, self.route_ws, stream)
         else:
             moe_route(u, self.E, self.b, c.K, self.topk_idx, self.topk_gate, self.counts,
                       self.route_ws, stream)
+        mark("route", 1)
+        mark("permute", 0)
         if self.fp8:
             moe_quantize_1x128(u, self.u_q, self.u_s, stream)
             moe_permute(self.u_q, self.topk_idx, c.N_r, self.x_perm, self.offsets, self.perm_src,
@@ -110,27 +132,43 @@ class MoELayer:
             moe_permute(u, self.topk_idx, c.N_r, self.x_perm, self.offsets, self.perm_src,
                         self.inv_row, self.perm_ws, stream=stream)
             x_sh, xs_sh = u, None
+        mark("permute", 1)
         (wgu, sgu), (wdn, sdn) = self.W["W_gate_up"], self.W["W_down"]
-        st = torch.cuda.current_stream() if stream is None else stream
-        if gate_up_events:
-            gate_up_events[0].record(st)
-        moe_expert_gate_up(self.x_perm, self.offsets, wgu, self.h_mid,
-                           x_scale=self.x_scale if self.fp8 else None, w_scale_gate_up=sgu,
-                           h_scale=self.h_scale, stream=stream)
-        if gate_up_events:
-            gate_up_events[1].record(st)
-        moe_expert_down(self.h_mid, self.offsets, wdn, self.y_perm, h_scale=self.h_scale,
-                        w_scale_down=sdn, stream=stream)
         (wsgu, ssgu), (wsdn, ssdn) = self.W["Ws_gate_up"], self.W["Ws_down"]
-        for j in range(c.N_s):
-            moe_expert_ffn(x_sh, self.shared_offsets, wsgu[j:j + 1], wsdn[j:j + 1],
-                           self.y_shared[j], self.ffn_ws, x_scale=xs_sh,
-                           w_scale_gate_up=None if ssgu is None else ssgu[j:j + 1],
-                           w_scale_down=None if ssdn is None else ssdn[j:j + 1], stream=stream)
+        if self.merged_shared:
+            # routed + shared experts: one gate/up launch, one down launch
+            mark("gate_up", 0)
+            moe_expert_gate_up_shared(self.x_perm, self.offsets, wgu, u, wsgu, self.h_all,
+                                      stream=stream)
+            mark("gate_up", 1)
+            mark("down", 0)
+            moe_expert_down_shared(self.h_all, self.offsets, wdn, wsdn, T * c.K, T, self.y_all,
+                                   stream=stream)
+            mark("down", 1)
+        else:
+            mark("gate_up", 0)
+            moe_expert_gate_up(self.x_perm, self.offsets, wgu, self.h_mid,
+                               x_scale=self.x_scale if self.fp8 else None, w_scale_gate_up=sgu,
+                               h_scale=self.h_scale, stream=stream)
+            mark("gate_up", 1)
+            mark("down", 0)
+            moe_expert_down(self.h_mid, self.offsets, wdn, self.y_perm, h_scale=self.h_scale,
+                            w_scale_down=sdn, stream=stream)
+            mark("down", 1)
+            mark("shared", 0)
+            for j in range(c.N_s):
+                moe_expert_ffn(x_sh, self.shared_offsets, wsgu[j:j + 1], wsdn[j:j + 1],
+                               self.y_shared[j], self.ffn_ws, x_scale=xs_sh,
+                               w_scale_gate_up=None if ssgu is None else ssgu[j:j + 1],
+                               w_scale_down=None if ssdn is None else ssdn[j:j + 1],
+                               stream=stream)
+            mark("shared", 1)
         u_res = u
         h = self.h_out if out is None else out
+        mark("combine", 0)
         moe_combine(u_res, self.y_shared if c.N_s else None, self.y_perm, self.inv_row,
                     self.topk_gate, h, stream)
+        mark("combine", 1)
         return h
 
     # -- training (bf16 / FP8): forward that keeps activations, then the backward

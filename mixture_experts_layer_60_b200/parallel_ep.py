@@ -103,6 +103,8 @@ class _EPRank:
                     self.perm_src[:T * c.K], self.inv_row[:T], self.perm_ws, stream=stream)
 
     def plan(self, counts_all, stream=None):
+        if stream is not None:
+            stream.wait_stream(torch.cuda.current_stream())   # counts_all gathered there
         moe_ep_plan(counts_all, self.rank, self.recv_offsets, self.send_base, stream)
 
     def dispatch(self, recv_rows, recv_tags, stream=None):
@@ -140,6 +142,8 @@ class EPGroupEmulated:
         R = self.ranks
         for r, u in zip(R, u_list):
             r.route_permute(u, stream)
+        if stream is not None:
+            torch.cuda.current_stream().wait_stream(stream)   # the stack reads the loads
         counts_all = torch.stack([r.counts for r in R])
         for r in R:
             r.plan(counts_all, stream)
@@ -182,14 +186,31 @@ class EPRankDistributed:
         ret, self.peer_ret, _ = shared((R, cfg.d), act)
         self.r = _EPRank(cfg, weights, W, rank, T_max, dev, recv, tags, ret)
 
-    def forward(self, u, stream=None):
+    def _arrived(self, stream):
+        """Cross-rank wait between two phases, in stream order: this rank's
+        work queued so far on `stream` is ordered before a barrier collective
+        (NCCL: an all-reduce queued on the current stream, which completes
+        only after every rank's copy of it ran, i.e. after every rank's
+        earlier work), and the work queued next on `stream` after it."""
         import torch.distributed as dist
+        cur = torch.cuda.current_stream()
+        other = stream is not None and stream != cur
+        if other:
+            cur.wait_stream(stream)
+        dist.barrier(group=self.group)
+        if other:
+            stream.wait_stream(cur)
+
+    def forward(self, u, stream=None):
         r = self.r
         r.route_permute(u, stream)
-        r.plan(gather_counts(r.counts, self.group), stream)
+        counts = r.counts
+        if stream is not None:
+            torch.cuda.current_stream().wait_stream(stream)   # the gather reads the load
+        r.plan(gather_counts(counts, self.group), stream)
         r.dispatch(self.peer_recv, self.peer_tags, stream)
-        dist.barrier(group=self.group)           # every rank's rows have arrived
+        self._arrived(stream)                    # every rank's rows have arrived
         r.experts(stream)
         r.give_back(self.peer_ret, stream)
-        dist.barrier(group=self.group)           # every rank's outputs have arrived
+        self._arrived(stream)                    # every rank's outputs have arrived
         return r.combine(stream)

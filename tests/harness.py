@@ -112,3 +112,42 @@ def grouped_reference(ref, K, n_groups, topk_groups):
     out = dict(ref)
     out["key"] = masked
     return out
+
+
+def oracle_layer_rows(w, rows, idx, gate, fp8=False):
+    """h' of the tokens `rows` of w["u"] (routing idx, gate for those rows) by
+    the C++ oracle, one expert at a time: each selected or shared expert's
+    stored weights are copied to the host only while it is evaluated.
+    float64 [len(rows), d]."""
+    from oracle import moe_ref as R
+    dev = w["u"].device
+    u = w["u"][torch.as_tensor(np.asarray(rows), device=dev)].cpu()
+    out = f64(u)
+    for j in range(w["Ws_gate_up"].shape[0]):
+        out += R.expert_ffn(u, w["Ws_gate_up"][j].cpu(), w["Ws_down"][j].cpu(), fp8=fp8)
+    idx = np.asarray(idx)
+    gate = np.asarray(gate, np.float64)
+    for e in np.unique(idx):
+        t, k = np.nonzero(idx == e)
+        y = R.expert_ffn(u[torch.from_numpy(t)], w["W_gate_up"][int(e)].cpu(),
+                         w["W_down"][int(e)].cpu(), fp8=fp8)
+        out[t] += gate[t, k][:, None] * y
+    return out
+
+
+def check_whole_experts(layer, w, experts, tol, fp8=False):
+    """Every grouped row of each expert in `experts` (the routed FFN output
+    y_perm of the last forward) against the C++ oracle's FFN of the same
+    token rows, within tol of max|ref| per expert."""
+    from oracle import moe_ref as R
+    off = layer.offsets.cpu().numpy()
+    src = layer.perm_src.cpu().numpy()
+    errs = {}
+    for e in experts:
+        a, b = int(off[e]), int(off[e + 1])
+        if b == a:
+            continue
+        u = w["u"][torch.from_numpy(src[a:b]).to(w["u"].device)].cpu()
+        want = R.expert_ffn(u, w["W_gate_up"][e].cpu(), w["W_down"][e].cpu(), fp8=fp8)
+        errs[int(e)] = assert_close(f64(layer.y_perm[a:b]), want, tol, f"expert {e} rows")
+    return errs

@@ -40,7 +40,7 @@ def test_binding_names_match_header():
 
 
 def test_abi_version_and_status_strings(L):
-    assert L.moe_abi_version() == 1
+    assert L.moe_abi_version() == 2
     assert L.moe_status_string(0) == b"MOE_OK"
     assert L.moe_status_string(3) == b"MOE_ERR_WORKSPACE"
 
@@ -154,15 +154,17 @@ def test_backward_argument_errors(L):
     assert L.moe_expert_ffn_backward(d, None, d, 4, 100, 256, 256, 1, d, None, None, None, d, d,
                                      d, d, d, d, d, 1 << 30, None) == 1
     # per-token backward kernels
-    assert L.moe_combine_backward(d, d, d, d, d, d, d, 2, 8, 64, 4, d, d, d, d, None) == 2
-    assert L.moe_combine_backward(d, d, d, d, d, d, d, 1, 8, 64, 17, d, d, d, d, None) == 2
-    assert L.moe_combine_backward(d, d, d, d, d, d, d, 1, 8, 4, 4, d, d, d, d, None) == 2
-    assert L.moe_combine_backward(d, d, None, d, d, d, d, 1, 8, 64, 4, d, d, d, d, None) == 1
-    assert L.moe_unpermute_backward(d, None, 1, d, d, d, d, d, 1, 8, 64, 4, d, None) == 1
-    assert L.moe_unpermute_backward(d, d, 1, d, d, d, d, d, 2, 8, 64, 4, d, None) == 2
+    assert L.moe_combine_backward(d, d, d, d, d, d, d, 2, 8, 64, 4, 16, d, d, d, d, None) == 2
+    assert L.moe_combine_backward(d, d, d, d, d, d, d, 1, 8, 64, 17, 32, d, d, d, d, None) == 2
+    assert L.moe_combine_backward(d, d, d, d, d, d, d, 1, 8, 4, 4, 16, d, d, d, d, None) == 2
+    assert L.moe_combine_backward(d, d, None, d, d, d, d, 1, 8, 64, 4, 16, d, d, d, d, None) == 1
+    assert L.moe_combine_backward(d, d, d, d, d, d, d, 1, 8, 64, 4, 0, d, d, d, d, None) == 1
+    assert L.moe_unpermute_backward(d, None, 1, d, d, d, d, d, 1, 8, 64, 4, 16, d, None) == 1
+    assert L.moe_unpermute_backward(d, d, 1, d, d, d, d, d, 2, 8, 64, 4, 16, d, None) == 2
+    assert L.moe_unpermute_backward(d, d, 1, d, d, d, d, d, 1, 8, 64, 4, 0, d, None) == 1
     # row slots of the gather pipeline: N_s + 2K at most 63
-    assert L.moe_unpermute_backward(d, d, 32, d, d, d, d, d, 1, 8, 64, 16, d, None) == 2
-    assert L.moe_unpermute_backward(d, d, 31, d, d, d, d, d, 1, 0, 64, 16, d, None) == 0
+    assert L.moe_unpermute_backward(d, d, 32, d, d, d, d, d, 1, 8, 64, 16, 32, d, None) == 2
+    assert L.moe_unpermute_backward(d, d, 31, d, d, d, d, d, 1, 0, 64, 16, 32, d, None) == 0
     assert L.moe_router_weight_grad(d, None, d, d, 2, 16, 64, d, None) == 2
     assert L.moe_router_weight_grad(d, None, d, None, 1, 16, 64, d, None) == 1
     # FP8 Wgrad quantiser

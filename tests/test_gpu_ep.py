@@ -11,6 +11,8 @@ from mixture_experts_layer_60_b200.configs import LayerConfig
 from mixture_experts_layer_60_b200.layer import MoELayer
 from mixture_experts_layer_60_b200.parallel_ep import EPGroupEmulated
 from mixture_experts_layer_60_b200.synth import make_layer_inputs, step_u
+from oracle import moe_oracle as O
+from tests.harness import GATE_TOL, TOL, LazyExperts, assert_close, check_routing, f64
 
 pytestmark = pytest.mark.gpu
 
@@ -34,3 +36,14 @@ def test_ep_emulated_equals_single_device(W, dtype, N_r, T):
         ref = MoELayer(cfg, w, T_max=u.shape[0]).forward(u)
         torch.cuda.synchronize()
         assert torch.equal(hs[s], ref), f"rank {s}"
+    # and against the oracle directly: each rank's routing and h'
+    routed = LazyExperts(w["W_gate_up"], w["W_down"])
+    shared = LazyExperts(w["Ws_gate_up"], w["Ws_down"])
+    for s, u in enumerate(us):
+        rk, T_s = grp.ranks[s], u.shape[0]
+        ref = O.route(f64(u), f64(w["E"]), w["b"].cpu().numpy(), cfg.K)
+        _, idx, gate = check_routing(rk.topk_idx[:T_s].cpu().numpy(),
+                                     rk.topk_gate[:T_s].cpu().numpy(), rk.counts.cpu().numpy(),
+                                     ref, cfg.K, gate_tol=GATE_TOL[dtype])
+        want = O.layer_forward(f64(u), idx, gate, routed, shared)
+        assert_close(f64(hs[s]), want, TOL[dtype], f"rank {s} h' against the oracle")

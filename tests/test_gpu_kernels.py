@@ -52,6 +52,8 @@ def _route(u, E, b, K):
     (64, 128, 64, 1, torch.bfloat16),       # K = 1
     (50, 128, 64, 64, torch.bfloat16),      # K = N_r
     (1, 128, 64, 6, torch.bfloat16),        # one token
+    (20000, 256, 256, 8, torch.bfloat16),   # more 256-token tiles than CTA pairs: tile loop
+    (700, 256, 96, 16, torch.bfloat16),     # N_r = 96, K = 16
 ])
 def test_route_matches_oracle(T, d, N_r, K, dt):
     g = _gen(T * 31 + d)
@@ -63,11 +65,13 @@ def test_route_matches_oracle(T, d, N_r, K, dt):
     check_routing(idx.cpu().numpy(), gate.cpu().numpy(), counts.cpu().numpy(), ref, K,
                   gate_tol=GATE_TOL["f32" if dt == torch.float32 else "bf16"])
     np.testing.assert_allclose(gate.double().sum(1).cpu().numpy(), 1.0, atol=4e-7)
+    assert moe.moe_device_status() == 0
 
 
 @pytest.mark.parametrize("T,d,N_r,K,G,M", [
     (1000, 512, 256, 8, 8, 4), (333, 256, 64, 6, 4, 2), (200, 128, 64, 4, 16, 1),
     (300, 256, 128, 8, 8, 8),    # keeping every group: same as no limit
+    (20000, 256, 256, 8, 8, 4),  # tile loop of the fused router
 ])
 def test_route_grouped_matches_oracle(T, d, N_r, K, G, M):
     g = _gen(T + G * 7)
@@ -311,6 +315,32 @@ def test_expert_ffn_bf16(sizes, d, I):
     assert moe.moe_device_status() == 0
 
 
+def test_expert_ffn_clamps_bad_offsets():
+    """Offsets that decrease or run past `rows` are clamped on the device: the
+    groups become [0, 100), [100, 100), [100, 250), [250, 250) of 250 rows,
+    nothing past row 250 of y is written, moe_device_status reports bit 16,
+    and the next call with good offsets is clean."""
+    d, I, rows = 256, 128, 250
+    g = _gen(4242)
+    x = _randn((rows, d), g)
+    wgu = _randn((4, 2 * I, d), g, d ** -0.5)
+    wdn = _randn((4, d, I), g, I ** -0.5)
+    y = torch.full((rows + 40, d), float("nan"), dtype=torch.bfloat16, device=DEV)
+    ws = _ws(moe.moe_expert_ffn_workspace_size(moe.MOE_BF16, rows, I))
+    bad = torch.tensor([0, 100, 50, 300, 260], dtype=torch.int32, device=DEV)
+    moe.moe_expert_ffn(x, bad, wgu, wdn, y[:rows], ws)
+    assert moe.moe_device_status() == 16
+    got = f64(y)
+    assert np.isnan(got[rows:]).all(), "rows past the end were written"
+    ex = LazyExperts(wgu, wdn)
+    xs = f64(x)
+    assert_close(got[:100], O.swiglu_ffn(xs[:100], *ex[0]), TOL["bf16"], "group 0")
+    assert_close(got[100:rows], O.swiglu_ffn(xs[100:rows], *ex[2]), TOL["bf16"], "group 2")
+    good = torch.tensor([0, 100, 100, 250, 250], dtype=torch.int32, device=DEV)
+    moe.moe_expert_ffn(x, good, wgu, wdn, y[:rows], ws)
+    assert moe.moe_device_status() == 0
+
+
 @pytest.mark.parametrize("sizes,d,I", [([3, 0, 64, 65, 130], 256, 128), ([200], 128, 256)])
 def test_expert_ffn_f32(sizes, d, I):
     got, ref, n = _ffn_case(sizes, d, I, torch.float32, 7 + d)
@@ -421,6 +451,99 @@ def test_combine_and_unpermute_backward(T, d, K, N_s, dtype):
         np.einsum("tk,tkd->td", dl, f64(E)[idx])
     assert_close(f64(du), want_du, tol, "du")
     assert moe.moe_device_status() == 0
+
+
+def test_combine_wait_that_runs_out_is_reported_and_next_call_is_clean():
+    """With the pipeline's wait bound cut to 1 ns, a wait on a stage whose
+    copies are still in flight runs out: the kernel stops, returns, and
+    moe_device_status reports bit 8 (no fault, no hang).  With the default
+    bound restored the same call is clean and correct."""
+    T, d, K, N_s = 4096, 7168, 8, 1
+    g = _gen(808)
+    u = _randn((T, d), g)
+    ys = _randn((N_s, T, d), g, 0.5)
+    yp = _randn((T * K, d), g, 0.5)
+    inv = torch.randperm(T * K, generator=torch.Generator().manual_seed(3)).view(T, K)
+    inv = inv.to(torch.int32).to(DEV)
+    gate = torch.rand(T, K, generator=g, device=DEV)
+    out = torch.empty(T, d, dtype=torch.bfloat16, device=DEV)
+    assert moe.moe_device_status() == 0
+    try:
+        moe.moe_set_pipeline_wait_limit(1)
+        moe.moe_combine(u, ys, yp, inv, gate, out)
+        assert moe.moe_device_status() == 8
+    finally:
+        moe.moe_set_pipeline_wait_limit(0)
+    moe.moe_combine(u, ys, yp, inv, gate, out)
+    assert moe.moe_device_status() == 0
+    rows = np.arange(0, T, 97)
+    iv = inv.long().cpu().numpy()[rows]
+    ref = f64(u)[rows] + f64(ys)[0][rows] + np.einsum("tk,tkd->td", f64(gate)[rows],
+                                                      f64(yp)[iv])
+    assert_close(f64(out)[rows], ref, 2 ** -8, "h' after the timeout")
+
+
+def test_backward_leaves_out_slots_with_bad_expert_ids():
+    """Slots whose expert id is -1 or N_r (moe_permute gives them inv_row -1)
+    are left out of the backward: the selection is the remaining slots, so
+    d_gate and d_logit of the left-out slot are 0, no dy_perm row or
+    d_logit_perm entry is written, and the gate backward of the oracle runs
+    over the valid slots only; no centroid row outside E is read."""
+    T, d, K, N_s = 93, 1024, 8, 1
+    u, E, dh, yp, dxp, dxs, idx, inv, gate = _bwd_case(T, d, K, N_s, torch.bfloat16, 77)
+    N_r = E.shape[0]
+    rng = np.random.default_rng(5)
+    bad = rng.random((T, K)) < 0.12
+    bad[0, :] = False
+    bad[1, 2] = True
+    idx = idx.copy()
+    idx[bad] = np.where(rng.random(int(bad.sum())) < 0.5, -1, N_r)
+    inv = inv.copy()
+    inv[bad] = -1
+    s_all = B.sigmoid(np.einsum("td,tkd->tk", f64(u), f64(E)[np.clip(idx, 0, N_r - 1)]))
+    s_all[bad] = 0.0
+    g64 = s_all / s_all.sum(1, keepdims=True)
+    gate = torch.from_numpy(g64).float().to(DEV)
+    idx_d = torch.from_numpy(idx).to(DEV)
+    inv_d = torch.from_numpy(inv).to(DEV)
+    dyp = torch.full((T * K, d), 3.0, dtype=torch.bfloat16, device=DEV)
+    d_gate = torch.full((T, K), 9.0, device=DEV)
+    d_logit = torch.full((T, K), 9.0, device=DEV)
+    d_logit_perm = torch.full((T * K,), 9.0, device=DEV)
+    moe.moe_combine_backward(dh, u, E, yp, inv_d, idx_d, gate, dyp, d_gate, d_logit, d_logit_perm)
+    du = torch.empty(T, d, dtype=torch.bfloat16, device=DEV)
+    moe.moe_unpermute_backward(dh, dxs, dxp, inv_d, idx_d, d_logit, E, du)
+    torch.cuda.synchronize()
+    assert moe.moe_device_status() == 0
+    tol = TOL["bf16"]
+    dh64, ys = f64(dh), f64(yp)
+    ok = ~bad
+    want_dg = np.where(ok, np.einsum("td,tkd->tk", dh64, ys[np.maximum(inv, 0)]), 0.0)
+    want_dl = np.zeros((T, K))
+    for t in range(T):
+        v = ok[t]
+        ds = B.gate_backward(s_all[t:t + 1, v], want_dg[t:t + 1, v])[0]
+        want_dl[t, v] = ds * s_all[t, v] * (1 - s_all[t, v])
+    got_dg = d_gate.double().cpu().numpy()
+    got_dl = d_logit.double().cpu().numpy()
+    assert np.all(got_dg[bad] == 0) and np.all(got_dl[bad] == 0)
+    assert_close(got_dg, want_dg, tol, "d_gate")
+    assert_close(got_dl, want_dl, tol, "d_logit")
+    written = np.zeros(T * K, bool)
+    written[inv[ok]] = True
+    dlp = d_logit_perm.double().cpu().numpy()
+    assert np.all(dlp[~written] == 9.0)                     # left-out rows untouched
+    assert_close(dlp[inv[ok]], want_dl[ok], tol, "d_logit_perm")
+    got_dyp = f64(dyp)
+    assert np.all(got_dyp[~written] == 3.0)
+    want_dyp = g64[:, :, None] * dh64[:, None, :]
+    assert_close(got_dyp[inv[ok]], want_dyp[ok], tol, "dy_perm")
+    want_du = dh64 + f64(dxs).sum(0)
+    for t in range(T):
+        for k in range(K):
+            if ok[t, k]:
+                want_du[t] += f64(dxp)[inv[t, k]] + got_dl[t, k] * f64(E)[idx[t, k]]
+    assert_close(f64(du), want_du, tol, "du")
 
 
 def test_bias_update_bit_exact():
@@ -552,3 +675,47 @@ def test_expert_gate_up_fp8_codes_close():
     np.testing.assert_allclose(hs.cpu().numpy(), rs, rtol=1e-5)
     codes_equal = (_e4m3_values(h) == rq).mean()
     assert codes_equal > 0.999, codes_equal
+
+
+@pytest.mark.parametrize("sizes,T,N_s,d,I", [
+    ([0, 1, 127, 300, 5, 256], 700, 1, 512, 256),   # ragged routed groups + one shared expert
+    ([64, 200, 333], 1000, 2, 256, 384),            # two shared experts, I not a multiple of 256
+    ([0, 0, 0], 257, 1, 256, 128),                  # no routed rows: the shared experts alone
+])
+def test_expert_ffn_with_shared_groups(sizes, T, N_s, d, I):
+    """The shared experts as extra groups of the routed launches: routed rows
+    as moe_expert_ffn, shared expert j's rows at rows + j*T, equal to the
+    oracle's FFN of u; nothing past the last row is written."""
+    g = _gen(T + d + N_s)
+    G = len(sizes)
+    off = _groups(sizes)
+    rows = int(off[-1])
+    x = _randn((max(rows, 1), d), g)[:rows] if rows else torch.empty(0, d, dtype=torch.bfloat16,
+                                                                          device=DEV)
+    u = _randn((T, d), g)
+    wgu = _randn((G, 2 * I, d), g, d ** -0.5)
+    wdn = _randn((G, d, I), g, I ** -0.5)
+    wsgu = _randn((N_s, 2 * I, d), g, d ** -0.5)
+    wsdn = _randn((N_s, d, I), g, I ** -0.5)
+    h = torch.empty(rows + N_s * T, I, dtype=torch.bfloat16, device=DEV)
+    y = torch.full((rows + N_s * T + 5, d), float("nan"), dtype=torch.bfloat16, device=DEV)
+    offsets = torch.from_numpy(off).to(DEV)
+    moe.moe_expert_gate_up_shared(x if rows else u[:0], offsets, wgu, u, wsgu, h)
+    moe.moe_expert_down_shared(h, offsets, wdn, wsdn, rows, T, y[:rows + N_s * T])
+    torch.cuda.synchronize()
+    assert moe.moe_device_status() == 0
+    got = f64(y)
+    assert np.isnan(got[rows + N_s * T:]).all()
+    ex, exs = LazyExperts(wgu, wdn), LazyExperts(wsgu, wsdn)
+    if rows:
+        xs = f64(x)
+        ref = np.zeros((rows, d))
+        for e in range(G):
+            a, b_ = int(off[e]), int(off[e + 1])
+            if b_ > a:
+                ref[a:b_] = O.swiglu_ffn(xs[a:b_], *ex[e])
+        assert_close(got[:rows], ref, TOL["bf16"], "routed rows")
+    us = f64(u)
+    for j in range(N_s):
+        assert_close(got[rows + j * T: rows + (j + 1) * T], O.swiglu_ffn(us, *exs[j]),
+                     TOL["bf16"], f"shared expert {j}")

@@ -11,8 +11,8 @@ from mixture_experts_layer_60_b200.configs import CONFIGS
 from mixture_experts_layer_60_b200.layer import MoELayer
 from mixture_experts_layer_60_b200.synth import make_layer_inputs, step_u
 from oracle import moe_oracle as O
-from tests.harness import (GATE_TOL, TOL, LazyExperts, assert_close, check_routing, f64,
-                           grouped_reference)
+from tests.harness import (GATE_TOL, TOL, LazyExperts, assert_close, check_routing,
+                           check_whole_experts, f64, grouped_reference, oracle_layer_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -61,10 +61,21 @@ def _run(cfg, T=None, sample=None, seed_sample=0):
     Tn = u.shape[0]
     rows = np.arange(Tn) if sample is None else \
         np.sort(np.random.default_rng(seed_sample).choice(Tn, sample, replace=False))
-    want = _oracle_layer(cfg, w, f64(u)[rows], idx[rows], gate[rows])
+    if sample is None:
+        want = _oracle_layer(cfg, w, f64(u)[rows], idx[rows], gate[rows])
+    else:
+        want = oracle_layer_rows(w, rows, idx[rows], gate[rows], fp8=cfg.dtype == "e4m3")
     got = f64(h)[rows]
     err = assert_close(got, want, TOL[cfg.dtype], f"h' {cfg.name}")
     return layer, w, err, exempt
+
+
+def _three_experts(layer):
+    """The most-loaded expert, the least-loaded non-empty one and a median one."""
+    c = layer.counts.cpu().numpy()
+    nz = np.nonzero(c)[0]
+    order = nz[np.argsort(c[nz], kind="stable")]
+    return [int(order[-1]), int(order[0]), int(order[len(order) // 2])]
 
 
 def test_layer_tiny_f32():
@@ -76,7 +87,10 @@ def test_layer_small_bf16():
 
 
 def test_layer_v3_bf16_sampled():
-    _run(CONFIGS["v3_bf16"], sample=48)
+    """V3 shape (T = 8192): h' on 256 sampled tokens and every routed row of
+    three whole experts (the most loaded spans several 16-row token tiles)."""
+    layer, w, _, _ = _run(CONFIGS["v3_bf16"], sample=256)
+    check_whole_experts(layer, w, _three_experts(layer), TOL["bf16"])
 
 
 def test_layer_v3_bf16_ragged_T():
@@ -85,8 +99,11 @@ def test_layer_v3_bf16_ragged_T():
 
 
 def test_layer_v3_fp8_sampled():
-    """FP8 V3 shape (T = 16384, 0.1 % outliers x50) against the FP8-emulating oracle."""
-    _run(CONFIGS["v3_fp8"], sample=6, seed_sample=2)
+    """FP8 V3 shape (T = 16384, 0.1 % outliers x50) against the FP8-emulating
+    oracle: h' on 256 sampled tokens and every routed row of three whole
+    experts (the most loaded spans several 128-token tiles)."""
+    layer, w, _, _ = _run(CONFIGS["v3_fp8"], sample=256, seed_sample=2)
+    check_whole_experts(layer, w, _three_experts(layer), TOL["e4m3"], fp8=True)
 
 
 def test_layer_fp8_small_full():
@@ -225,3 +242,30 @@ def test_host_stepper_overlapped_equals_device_steps():
     for s in range(n):
         assert torch.equal(h_h[s], want[s]), s
     assert torch.equal(lay.b, ref.b)
+
+
+def test_skewed_load_full_shape_routing_and_bias():
+    """The skewed-popularity V3 configuration at its full shape (T = 8192,
+    Zipf(1.2) centroid norms): for 3 steps of forward + bias update with fresh
+    tokens, every token's routing equals the oracle's (with the bias the GPU
+    carries) bit for bit except genuine near-ties (key gap < 1e-6), the load
+    matches, b follows the oracle's rule bit for bit, and every routed row of
+    the most-loaded expert (thousands of rows, many token tiles) and two more
+    matches the oracle's FFN."""
+    cfg = CONFIGS["v3_zipf_bf16"]
+    w = make_layer_inputs(cfg, "cuda")
+    a = MoELayer(cfg, w)
+    E = f64(w["E"])
+    for s in range(3):
+        u = step_u(cfg, s, "cuda")
+        b_before = a.b.cpu().numpy().copy()
+        a.step(u)
+        torch.cuda.synchronize()
+        ref = O.route(f64(u), E, b_before, cfg.K)
+        check_routing(a.topk_idx.cpu().numpy(), a.topk_gate.cpu().numpy(),
+                      a.counts.cpu().numpy(), ref, cfg.K, gate_tol=GATE_TOL["bf16"])
+        np.testing.assert_array_equal(a.b.cpu().numpy(),
+                                      O.bias_update(b_before, a.counts.cpu().numpy(), cfg.T, cfg.K))
+    assert a.counts.max().item() > 4 * cfg.T * cfg.K / cfg.N_r       # the load is skewed
+    w_step = dict(w, u=u)
+    check_whole_experts(a, w_step, _three_experts(a), TOL["bf16"])
