@@ -410,6 +410,69 @@ def measure_train(args, cfg, layer, u, dev, group, p, steps):
     }
 
 
+def run_hbm_kernels(args, cfg, local):
+    """The HBM-bound steps alone (route, permute, combine) on T synthetic
+    tokens of the configuration's width, with random stand-ins for the
+    expert outputs and no expert weights on the device: a right-sized case
+    for profiling those kernels.  Prints one JSON line of per-step times."""
+    import mixture_experts_layer_60_b200 as moe
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    T, d, N_r, K, N_s = cfg.T, cfg.d, cfg.N_r, cfg.K, cfg.N_s
+    g = torch.Generator(device=dev)
+    g.manual_seed(cfg.seed)
+    u = torch.randn(T, d, generator=g, device=dev).to(torch.bfloat16)
+    E = (torch.randn(N_r, d, generator=g, device=dev) * d ** -0.5).to(torch.bfloat16)
+    b = torch.zeros(N_r, device=dev)
+    idx = torch.empty(T, K, dtype=torch.int32, device=dev)
+    gate = torch.empty(T, K, device=dev)
+    counts = torch.empty(N_r, dtype=torch.int32, device=dev)
+    rws = torch.empty(moe.moe_route_workspace_size(T, N_r), dtype=torch.uint8, device=dev)
+    pws = torch.empty(max(moe.moe_permute_workspace_size(T, N_r), 256), dtype=torch.uint8,
+                      device=dev)
+    x_perm = torch.empty(T * K, d, dtype=torch.bfloat16, device=dev)
+    offsets = torch.empty(N_r + 1, dtype=torch.int32, device=dev)
+    perm_src = torch.empty(T * K, dtype=torch.int32, device=dev)
+    inv_row = torch.empty(T, K, dtype=torch.int32, device=dev)
+    y_perm = torch.randn(T * K, d, generator=g, device=dev).to(torch.bfloat16)
+    y_sh = torch.randn(N_s, T, d, generator=g, device=dev).to(torch.bfloat16)
+    h = torch.empty(T, d, dtype=torch.bfloat16, device=dev)
+    names = ("route", "permute", "combine")
+    ev = {n: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)] for n in names}
+
+    def step(i=None):
+        def mark(n, j):
+            if i is not None:
+                ev[n][i][j].record()
+        mark("route", 0)
+        moe.moe_route(u, E, b, K, idx, gate, counts, rws)
+        mark("route", 1)
+        mark("permute", 0)
+        moe.moe_permute(u, idx, N_r, x_perm, offsets, perm_src, inv_row, pws)
+        mark("permute", 1)
+        mark("combine", 0)
+        moe.moe_combine(u, y_sh if N_s else None, y_perm, inv_row, gate, h)
+        mark("combine", 1)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        step(i)
+    torch.cuda.synchronize()
+    if moe.moe_device_status() != 0:
+        raise RuntimeError("a kernel reported a bounded-wait timeout")
+    ms = {n: sum(a.elapsed_time(c) for a, c in ev[n]) / args.steps for n in names}
+    nbytes = {"route": T * d * 2 + N_r * d * 2 + T * K * 8,
+              "permute": T * d * 2 * (1 + K) + T * K * 12,
+              "combine": T * d * 2 * (2 + N_s + K) + T * K * 8}
+    print(json.dumps({"mode": "hbm_kernels", "config": {"workload": cfg.name, "T": T, "d": d,
+                                                        "N_r": N_r, "K": K, "N_s": N_s},
+                      "ms": ms, "bytes": nbytes,
+                      "gbs": {n: nbytes[n] / (ms[n] / 1e3) / 1e9 for n in names}}), flush=True)
+
+
 def run_ours(args, cfg, ws, rank, local):
     from mixture_experts_layer_60_b200 import moe_device_status
     from mixture_experts_layer_60_b200.layer import MoELayer
@@ -598,8 +661,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-train", action="store_true",
                     help="skip the training-step (forward + backward) measurement")
-    ap.add_argument("--mode", default="forward", choices=["forward", "train"],
-                    help="train: time only training steps and print their line")
+    ap.add_argument("--mode", default="forward", choices=["forward", "train", "hbm_kernels"],
+                    help="train: time only training steps and print their line; hbm_kernels: "
+                         "route, permute and combine alone (no expert weights), for profiling")
     ap.add_argument("--tokens", type=int, default=None,
                     help="scaled-down variant: tokens per rank (default: the config's T)")
     ap.add_argument("--experts", type=int, default=None,
@@ -617,6 +681,8 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, cfg, ws, rank)
+        elif args.mode == "hbm_kernels":
+            run_hbm_kernels(args, cfg, local)
         else:
             run_ours(args, cfg, ws, rank, local)
     finally:

@@ -79,11 +79,27 @@ const char* moe_status_string(moe_status status);
  *   workspace          device, >= moe_route_workspace_size(T, N_r) bytes
  * Logits are accumulated in float32 from the stored values; sigmoid, keys and
  * gates are float32.  Tokens whose selection (or output order) was decided by
- * a key gap below 2e-5 are re-routed from float64 logits (sigmoid in float64,
- * s rounded once to float32), so the float32 accumulation error cannot flip
- * them.  Requires 1 <= K <= N_r <= 1024 and d % 64 == 0.
+ * a key gap below the refine gap (default 4e-5) are re-routed from float64
+ * logits for every expert within the near distance (default 6e-5) of the
+ * boundary (sigmoid in float64, s rounded once to float32), so the float32
+ * accumulation error cannot flip them; the defaults are 2B and 3B for the
+ * key-error bound B = 2e-5 of the tensor-core logits (see
+ * moe_set_router_tie_break).  Requires 1 <= K <= N_r <= 1024, d % 64 == 0 and
+ * rows of at most 32 KB (d <= 16384 bf16, 8192 float32).
  * ------------------------------------------------------------------------ */
 size_t moe_route_workspace_size(int T, int N_r);
+
+/* moe_set_router_tie_break - the thresholds of the float64 tie-break of
+ * moe_route / moe_route_grouped: a token is re-routed when a key gap that
+ * decided its selection or output order is below refine_gap, from float64
+ * affinities of every expert whose float32 key lies within `near` of the
+ * lowest key a decision hinged on.  Both >= 0; (0, 0) restores the defaults
+ * (4e-5, 6e-5).  Values below the defaults give up the exactness guarantee;
+ * larger values re-route more tokens (a refine gap of, say, 1e30 re-routes
+ * every token and leaves every token's float32 logit row in the first
+ * T*N_r floats of the workspace).  Process-wide, from the next call on. */
+moe_status moe_set_router_tie_break(float refine_gap, float near);
+
 moe_status moe_route(const void* u, const void* E, moe_dtype dt, const float* b,
                      int T, int d, int N_r, int K,
                      int32_t* topk_idx, float* topk_gate, int32_t* counts,

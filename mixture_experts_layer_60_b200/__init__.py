@@ -18,6 +18,7 @@ __all__ = [
     "moe_route", "moe_route_grouped", "moe_permute", "moe_permute_noalloc", "moe_expert_ffn", "moe_expert_gate_up", "moe_expert_down", "moe_combine", "moe_bias_update",
     "moe_quantize_1x128", "moe_quantize_128x128", "moe_device_status",
     "moe_set_pipeline_wait_limit", "moe_expert_gate_up_shared", "moe_expert_down_shared",
+    "moe_set_router_tie_break",
     "moe_route_workspace_size", "moe_permute_workspace_size", "moe_expert_ffn_workspace_size",
     "moe_expert_gate_up_save", "moe_combine_backward", "moe_expert_ffn_backward",
     "moe_expert_ffn_backward_workspace_size", "moe_unpermute_backward", "moe_router_weight_grad",
@@ -54,6 +55,7 @@ SYMBOLS = {
     "moe_quantize_128x128": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp]),
     "moe_device_status": (_i, [ctypes.POINTER(_i)]),
     "moe_set_pipeline_wait_limit": (_i, [ctypes.c_ulonglong]),
+    "moe_set_router_tie_break": (_i, [_f, _f]),
     "moe_expert_gate_up_shared": (_i, [_vp, _vp, _i, _i, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
     "moe_expert_down_shared": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
     "moe_permute_noalloc": (_i, [_vp, _vp, _i, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
@@ -273,6 +275,11 @@ def moe_quantize_1x128(x, q, scale, stream=None):
 def moe_quantize_128x128(w, q, scale, stream=None):
     groups, rows, cols = w.shape
     _check(lib().moe_quantize_128x128(_p(w), groups, rows, cols, _p(q), _p(scale), _s(stream)))
+
+
+def moe_set_router_tie_break(refine_gap: float = 0.0, near: float = 0.0):
+    """Thresholds of the router's float64 tie-break; (0, 0) restores the defaults."""
+    _check(lib().moe_set_router_tie_break(float(refine_gap), float(near)))
 
 
 def moe_set_pipeline_wait_limit(ns: int = 0):

@@ -2,6 +2,8 @@
 // validates its arguments on the host, then enqueues kernels on `stream`.
 #include "launch.h"
 
+#include <atomic>
+
 using namespace moe;
 
 namespace {
@@ -11,6 +13,9 @@ constexpr int kAbiVersion = 2;
 inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
 inline bool al16(const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0; }
+
+std::atomic<float> g_refine_gap{kRouterRefineGap};
+std::atomic<float> g_near{kRouterNearBoundary};
 
 int dtype_bytes(moe_dtype dt) {
   switch (dt) {
@@ -89,7 +94,24 @@ const char* moe_status_string(moe_status s) {
 
 size_t moe_route_workspace_size(int T, int N_r) { return route_ws(T, N_r); }
 
+moe_status moe_set_router_tie_break(float refine_gap, float near) {
+  clear_last_error();
+  MOE_REQUIRE(refine_gap >= 0.f && near >= 0.f, MOE_ERR_INVALID_ARG,
+              "moe_set_router_tie_break: gap %g and near %g must be >= 0", refine_gap, near);
+  const bool deflt = refine_gap == 0.f && near == 0.f;
+  g_refine_gap.store(deflt ? kRouterRefineGap : refine_gap);
+  g_near.store(deflt ? kRouterNearBoundary : near);
+  return MOE_OK;
+}
+
 }  // extern "C"
+
+namespace moe {
+void router_tie_break(float* refine_gap, float* near) {
+  *refine_gap = g_refine_gap.load();
+  *near = g_near.load();
+}
+}  // namespace moe
 
 namespace {
 
@@ -111,6 +133,8 @@ moe_status route_impl(const char* who, const void* u, const void* E, moe_dtype d
   MOE_REQUIRE((long long)topk_groups * (N_r / n_groups) >= K, MOE_ERR_INVALID_ARG,
               "%s: the kept groups hold fewer than K experts", who);
   MOE_REQUIRE(d % 64 == 0, MOE_ERR_UNSUPPORTED, "%s: d=%d must be a multiple of 64", who, d);
+  MOE_REQUIRE((long long)d * dtype_bytes(dt) <= 32768, MOE_ERR_UNSUPPORTED,
+              "%s: a row of u is at most 32 KB (d=%d)", who, d);
   MOE_REQUIRE((long long)T * N_r <= 0x7fffffffLL, MOE_ERR_UNSUPPORTED,
               "%s: T * N_r must fit in 31 bits (T=%d N_r=%d)", who, T, N_r);
   MOE_REQUIRE(E && b && counts, MOE_ERR_INVALID_ARG, "%s: null pointer", who);
@@ -127,19 +151,21 @@ moe_status route_impl(const char* who, const void* u, const void* E, moe_dtype d
   float* logits = static_cast<float*>(workspace);
   const RefineLists rl = refine_lists(workspace, T, N_r);
   MOE_TRY(cuda_check(cudaMemsetAsync(rl.hdr, 0, 2 * sizeof(int32_t), s), "zero tie-break lists"));
+  float gap, near;
+  router_tie_break(&gap, &near);
   if (router_tc_supported(dt, d, N_r, K, n_groups, topk_groups)) {
     MOE_TRY(launch_router_tc(u, E, b, T, d, N_r, K, n_groups, topk_groups, topk_idx, topk_gate,
-                             counts, logits, rl, kRouterRefineGap, kRouterNearBoundary, s));
+                             counts, logits, rl, gap, near, s));
   } else {
     if (dt == MOE_BF16 && N_r % 64 == 0)
       MOE_TRY(launch_tc_gemm(u, E, N_r, nullptr, 1, T, N_r, d, TC_EPI_STORE_F32, logits, s));
     else
       MOE_TRY(launch_logits_simt(u, E, dt, T, d, N_r, logits, s));
     MOE_TRY(launch_topk(logits, b, T, N_r, K, n_groups, topk_groups, topk_idx, topk_gate, counts,
-                        rl, kRouterRefineGap, s));
+                        rl, gap, near, s));
   }
-  return launch_refine(u, E, dt, logits, b, d, N_r, K, n_groups, topk_groups, rl, T, topk_idx,
-                       topk_gate, counts, s);
+  return launch_refine(u, E, dt, logits, b, d, N_r, K, n_groups, topk_groups, rl, near, T,
+                       topk_idx, topk_gate, counts, s);
 }
 
 }  // namespace

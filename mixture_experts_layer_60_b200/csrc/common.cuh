@@ -56,6 +56,15 @@ enum : int {
 
 __device__ __forceinline__ float bf2f(__nv_bfloat16 v) { return __bfloat162float(v); }
 
+// The router's float32 affinity Sigmoid(x) = 1 / (1 + e^-x), with the fast
+// exponential and division (a few 1e-7 from the exact value, well inside the
+// tie-break's key-error bound).  Every kernel that forms a float32 key (the
+// fused router, the top-K kernel, the tie-break's keys of unlisted experts)
+// uses this one expression, so equal logits give equal keys everywhere.
+__device__ __forceinline__ float router_affinity(float x) {
+  return __fdividef(1.0f, 1.0f + __expf(-x));
+}
+
 // Row range [r0, r1) of group g from the caller's offsets, clamped so that
 // 0 <= r0 <= r1 <= rows (offsets == nullptr: one group of all rows); a clamp
 // that changes a value sets ERR_BAD_OFFSETS in *err (err may be null).

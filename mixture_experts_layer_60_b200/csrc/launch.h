@@ -21,20 +21,26 @@ struct RefineLists {
   int32_t* num;
   int32_t* pair;
 };
-// A token whose selection or output order was decided by a key gap below
-// kRouterRefineGap is listed with every expert whose float32 key lies within
-// kRouterNearBoundary of the lowest key a decision hinged on; the tie-break
-// recomputes those experts' affinities in float64.  Both are set from the
-// bound on the float32 key error of the tensor-core logits.
-constexpr float kRouterRefineGap = 2e-5f;
-constexpr float kRouterNearBoundary = 6e-5f;
+// A token whose selection or output order was decided by a key gap below the
+// refine gap is listed with every expert whose float32 key lies within the
+// near distance of the lowest key a decision hinged on; the tie-break
+// recomputes those experts' affinities in float64.  With B a bound on the
+// float32 key error |s32 + b - (s64 + b)| of the tensor-core logits, a gap of
+// 2B lists every token whose float32 selection or order can differ from the
+// exact one, and a near distance of 2B or more recomputes every expert that
+// can take part in it; the defaults are 2B and 3B.
+constexpr float kRouterKeyErrorBound = 2e-5f;
+constexpr float kRouterRefineGap = 2.0f * kRouterKeyErrorBound;
+constexpr float kRouterNearBoundary = 3.0f * kRouterKeyErrorBound;
+// The thresholds in force (moe_set_router_tie_break; defaults above).
+void router_tie_break(float* refine_gap, float* near);
 // sigmoid, biased top-K, gates, histogram (counts must be zeroed beforehand).
 // n_groups > 1 && topk_groups < n_groups restricts each token to its best groups.
 // A token whose routing was decided by a key gap < refine_gap is listed with
 // the experts whose float32 key lies near one of its decision boundaries.
 moe_status launch_topk(const float* logits, const float* b, int T, int N_r, int K, int n_groups,
                        int topk_groups, int32_t* idx, float* gate, int32_t* counts,
-                       RefineLists rl, float refine_gap, cudaStream_t s);
+                       RefineLists rl, float refine_gap, float near, cudaStream_t s);
 
 // router_tc.cu ----------------------------------------------------------------
 // The fused router (logits on tcgen05 CTA pairs, sigmoid, biased top-K, gates,
@@ -51,8 +57,8 @@ moe_status launch_router_tc(const void* u, const void* E, const float* b, int T,
 // routing redone from them.
 moe_status launch_refine(const void* u, const void* E, moe_dtype dt, const float* logits,
                          const float* b, int d, int N_r, int K, int n_groups, int topk_groups,
-                         RefineLists rl, int T, int32_t* idx, float* gate, int32_t* counts,
-                         cudaStream_t s);
+                         RefineLists rl, float near, int T, int32_t* idx, float* gate,
+                         int32_t* counts, cudaStream_t s);
 
 // permute.cu -----------------------------------------------------------------
 size_t permute_ws_bytes(int T, int N_r);

@@ -30,6 +30,7 @@
 #include <math.h>
 
 #include "launch.h"
+#include "router_warp.cuh"
 #include "sm100.cuh"
 
 namespace moe {
@@ -44,31 +45,42 @@ using namespace sm100;
 
 constexpr int BK = 64;                 // bf16 K elements per 128-byte swizzle row
 constexpr int TM = 128;                // token rows per CTA (TMEM lanes)
-constexpr int STAGES = 6;
 constexpr int kMaxN = 256;             // N_r limit of the pair MMA
-constexpr int kThreads = 192;
-constexpr int kEpiWarps = 4;
+constexpr int kParts = 4;              // epilogue warps per TMEM lane quarter (column parts)
+constexpr int kEpiWarps = 4 * kParts;
+constexpr int kEpiThreads = 32 * kEpiWarps;
+constexpr int kThreads = 64 + kEpiThreads;
 constexpr uint64_t kWaitNs = 1000000000ull;
+constexpr int kEpiBarrier = 1;         // named barrier of the epilogue warps
+constexpr int STAGES = 4;
+constexpr int HALF_ROWS = TM / 2;      // token rows staged in shared memory at a time
 
 constexpr int A_BYTES = TM * BK * 2;                  // 16 KB
 constexpr int B_MAX_BYTES = (kMaxN / 2) * BK * 2;     // 16 KB
+constexpr int XLD = kMaxN + 4;                        // float stride of a staged logit row
 constexpr int OFF_B = STAGES * A_BYTES;
-constexpr int OFF_BAR = OFF_B + STAGES * B_MAX_BYTES;
-constexpr int N_BARS = 2 * STAGES + 4;                // full, empty, tfull, tempty, peer_ready, mma_done
+constexpr int RING_BYTES = OFF_B + STAGES * B_MAX_BYTES;
+// S > 1: each CTA stages its partial logits of the rows other slices own in
+// [TM][XLD] floats from offset 0 (over the ring, free once the tile's MMAs
+// are done), then the logits of its own rows go to sX
+constexpr int STAGE_BYTES = TM * XLD * 4;
+constexpr int OFF_X = RING_BYTES > STAGE_BYTES ? RING_BYTES : STAGE_BYTES;   // [HALF_ROWS][XLD]
+constexpr int OFF_WK = OFF_X + HALF_ROWS * XLD * 4;   // float [kEpiWarps][kMaxN] group keys
+constexpr int OFF_BAR = OFF_WK + kEpiWarps * kMaxN * 4;
+constexpr int N_BARS = 2 * STAGES + 4;     // full, empty, tfull, tempty, peer_ready, mma_done
 constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;        // tmem slot, abort flag
 constexpr int OFF_BIAS = OFF_MISC + 16;               // float [kMaxN]
 constexpr int OFF_HIST = OFF_BIAS + kMaxN * 4;        // int [kMaxN]
-constexpr int OFF_GS = OFF_HIST + kMaxN * 4;          // float [32 groups][128 rows]
-constexpr int SMEM_BYTES = OFF_GS + 32 * TM * 4;
+constexpr int SMEM_BYTES = OFF_HIST + kMaxN * 4;
 constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
-constexpr int STAGE_LD = kMaxN + 4;                   // float stride of a staged partial row
 
 struct RouterParams {
   const float* bias;     // [N_r]
   int T, N_r, K;
   int nk;                // d / BK
   int n_tiles;           // ceil(T / 256)
-  int n_groups, topk_groups, gshift;   // grouped: group of expert e is e >> gshift
+  int parts;             // column parts actually used (<= kParts), N_r / parts % 16 == 0
+  int n_groups, topk_groups;
   int32_t* idx;
   float* gate;
   int32_t* counts;
@@ -83,68 +95,60 @@ __device__ __forceinline__ void raise_abort(volatile int* abort, int* err) {
   atomicOr(err, ERR_GEMM_TIMEOUT);
 }
 
-__device__ __forceinline__ float affinity32(float x) { return 1.0f / (1.0f + expf(-x)); }
-
-// Logits of this thread's token for columns [c*32, c*32+32): its own TMEM
-// partial plus, in slice order, the partials the other S-1 pairs staged.
-template <int S>
-__device__ __forceinline__ void load_logits32(uint32_t tmem_row, int c, const uint32_t* peer_row,
-                                              float* x) {
-  uint32_t r[32];
-  tmem_ld_32x32b_x32(tmem_row + c * 32, r);
-  tmem_wait_ld();
-#pragma unroll
-  for (int j = 0; j < 32; ++j) x[j] = __uint_as_float(r[j]);
-#pragma unroll
-  for (int q = 1; q < S; ++q) {
-#pragma unroll
-    for (int v = 0; v < 8; ++v) {
-      const float4 f = ld_shared_cluster_v4(peer_row[q] + (uint32_t)(c * 32 + 4 * v) * 4u);
-      x[4 * v] += f.x;
-      x[4 * v + 1] += f.y;
-      x[4 * v + 2] += f.z;
-      x[4 * v + 3] += f.w;
-    }
-  }
+__device__ __forceinline__ void epi_sync() {
+  asm volatile("bar.sync %0, %1;" ::"n"(kEpiBarrier), "n"(kEpiThreads) : "memory");
+}
+// True on every epilogue thread when `v` is true on any of them (a barrier).
+__device__ __forceinline__ bool epi_any(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(r)
+      : "r"((uint32_t)v), "n"(kEpiBarrier), "n"(kEpiThreads)
+      : "memory");
+  return r != 0;
 }
 
-// Inserts (key, e, s) into the list sorted by (key desc, index asc): slots
-// [0, K] hold the K+1 best so far; a new key equal to a listed one goes
-// after it (experts arrive in ascending order).
-template <int KMAX>
-__device__ __forceinline__ void insert_top(float key, int e, float s, int K, float* tk, int* te,
-                                           float* ts) {
+// Logits of this thread's token for columns [c, c + CH): the partial sums
+// of the S slices of the contraction added in slice order, this CTA's own
+// (slice `slice`) from TMEM, the others from their staged copies.
+constexpr int CH = 16;                 // columns per TMEM load in the epilogue
+template <int S>
+__device__ __forceinline__ void load_logits(uint32_t tmem_row, int c, int slice, uint32_t half,
+                                            uint32_t stage_addr, float* x) {
+  uint32_t r[CH];
+  tmem_ld_32x32b_x16(tmem_row + c, r);
+  tmem_wait_ld();
+  if constexpr (S == 1) {
 #pragma unroll
-  for (int j = KMAX; j >= 1; --j) {
-    if (j <= K) {
-      if (key > tk[j - 1]) {
-        tk[j] = tk[j - 1];
-        te[j] = te[j - 1];
-        ts[j] = ts[j - 1];
-      } else if (key > tk[j]) {
-        tk[j] = key;
-        te[j] = e;
-        ts[j] = s;
+    for (int j = 0; j < CH; ++j) x[j] = __uint_as_float(r[j]);
+  } else {
+#pragma unroll
+    for (int j = 0; j < CH; ++j) x[j] = 0.f;
+#pragma unroll
+    for (int q = 0; q < S; ++q) {
+      if (q == slice) {
+#pragma unroll
+        for (int j = 0; j < CH; ++j) x[j] += __uint_as_float(r[j]);
+      } else {
+        const uint32_t peer = map_shared_to(stage_addr, half + 2u * (uint32_t)q);
+#pragma unroll
+        for (int v = 0; v < CH / 4; ++v) {
+          const float4 f = ld_shared_cluster_v4(peer + (uint32_t)(c + 4 * v) * 4u);
+          x[4 * v] += f.x;
+          x[4 * v + 1] += f.y;
+          x[4 * v + 2] += f.z;
+          x[4 * v + 3] += f.w;
+        }
       }
     }
   }
-  if (key > tk[0]) {
-    tk[0] = key;
-    te[0] = e;
-    ts[0] = s;
-  }
 }
 
-template <int KMAX>
-__device__ __forceinline__ float slot_value(const float* a, int k) {
-  float v = a[0];
-#pragma unroll
-  for (int j = 1; j <= KMAX; ++j)
-    if (j == k) v = a[j];
-  return v;
-}
-
-template <int S, int KMAX, bool GROUPED>
+template <int S, int V>
 __global__ void __launch_bounds__(kThreads, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmU,
                      const __grid_constant__ CUtensorMap tmE, const RouterParams p) {
@@ -153,6 +157,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + OFF_B;
+  float* sX = reinterpret_cast<float*>(smem + OFF_X);
+  float* s_wkeys = reinterpret_cast<float*>(smem + OFF_WK);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
@@ -163,7 +169,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
   float* s_bias = reinterpret_cast<float*>(smem + OFF_BIAS);
   int* s_hist = reinterpret_cast<int*>(smem + OFF_HIST);
-  float* s_gscore = reinterpret_cast<float*>(smem + OFF_GS);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -271,160 +276,86 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue (every CTA)
-    const int q = warp & 3;                       // TMEM lane quarter
+    // Warp w: TMEM lane quarter q = w % 4 (its 32 token rows) and column part
+    // `part` (columns [part*cols, +cols) of those rows) when reading TMEM; one
+    // token per warp when routing.
+    const int ew = warp - 2;                      // epilogue warp 0 .. kEpiWarps-1
+    const int q = warp & 3;
+    const int part = ew >> 2;
     const int row = q * 32 + lane;                // token row of this CTA
+    const int P = p.parts;
+    const int cols = N / P;
+    const int c0 = part * cols;
+    const bool active = part < P;
     const uint32_t tmem_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-    float* stage_row = reinterpret_cast<float*>(smem) + (size_t)row * STAGE_LD;
+    float* stage_row = reinterpret_cast<float*>(smem) + (size_t)row * XLD;
+    float* wkeys = s_wkeys + ew * kMaxN;
+    // rows of the tile this CTA routes: all of them (S == 1) or slice
+    // `slice`'s share of TM / S rows (S > 1; the other slices' CTAs route the rest)
+    const int own0 = S == 1 ? 0 : slice * (TM / S);
+    const int own1 = S == 1 ? TM : own0 + TM / S;
     uint32_t tphase = 0;
     for (int tile = first_tile; tile < p.n_tiles; tile += tile_step) {
       const bool got = mbar_wait_bounded(tfull, tphase, abort_flag, kWaitNs);
-      if (!__all_sync(0xffffffffu, got)) {
-        raise_abort(abort_flag, p.err);
+      if (epi_any(!got)) {
+        if (lane == 0) raise_abort(abort_flag, p.err);
         break;
       }
       tc_fence_after();
-      if (slice > 0) {
-        // stage this slice's partial logits for the first pair, then signal it
-        for (int c = 0; c < N / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(tmem_row + c * 32, r);
-          tmem_wait_ld();
+      if (S > 1) {
+        // stage this slice's partial logits of the rows the other slices own,
+        // signal their CTAs, wait for theirs of this CTA's rows
+        if (active && (row < own0 || row >= own1)) {
+          for (int c = c0; c < c0 + cols; c += CH) {
+            uint32_t r[CH];
+            tmem_ld_32x32b_x16(tmem_row + c, r);
+            tmem_wait_ld();
 #pragma unroll
-          for (int v = 0; v < 8; ++v)
-            *reinterpret_cast<uint4*>(stage_row + c * 32 + 4 * v) =
-                make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+            for (int v = 0; v < CH / 4; ++v)
+              *reinterpret_cast<uint4*>(stage_row + c + 4 * v) =
+                  make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+          }
         }
         __syncwarp();
         if (lane == 0)
-          mbar_arrive_remote(map_shared_to(smem_u32(peer_ready), rank - 2u * (uint32_t)slice));
-        tc_fence_before();
-        break;                                  // S > 1: one tile per cluster
-      }
-      uint32_t peer_row[S > 1 ? S : 1];
-      if (S > 1) {
+          for (int s2 = 0; s2 < S; ++s2)
+            if (s2 != slice)
+              mbar_arrive_remote(map_shared_to(smem_u32(peer_ready), half + 2u * (uint32_t)s2));
         const bool ready = mbar_wait_cluster_bounded(peer_ready, 0, abort_flag, kWaitNs);
-        if (!__all_sync(0xffffffffu, ready)) {
-          raise_abort(abort_flag, p.err);
+        if (epi_any(!ready)) {
+          if (lane == 0) raise_abort(abort_flag, p.err);
           break;
         }
-#pragma unroll
-        for (int s2 = 1; s2 < S; ++s2)
-          peer_row[s2] = map_shared_to(smem_u32(stage_row), rank + 2u * (uint32_t)s2);
       }
-      const int t = tile * 2 * TM + (int)half * TM + row;
-      const bool tv = t < p.T;
-      const int K = p.K;
-      // ---- group limit: group scores, kept groups, the kept-vs-excluded gap
-      float margin = INFINITY, next_group = INFINITY;
-      unsigned kept = 0xffffffffu;
-      if (GROUPED) {
-        const int G = p.n_groups;
-        for (int g = 0; g < G; ++g) s_gscore[g * TM + row] = -INFINITY;
-        for (int c = 0; c < N / 32; ++c) {
-          float x[32];
-          load_logits32<S>(tmem_row, c, peer_row, x);
+      const int tok0 = tile * 2 * TM + (int)half * TM;
+      // own rows in blocks of HALF_ROWS (lane quarters 2h, 2h+1)
+      for (int h0 = own0; h0 < own1; h0 += HALF_ROWS) {
+        const int h1 = min(own1, h0 + HALF_ROWS);
+        if (active && row >= h0 && row < h1) {
+          float* xr = sX + (size_t)(row - h0) * XLD;
+          for (int c = c0; c < c0 + cols; c += CH) {
+            float x[CH];
+            load_logits<S>(tmem_row, c, slice, half, smem_u32(stage_row), x);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int e = c * 32 + j;
-            const float key = affinity32(x[j]) + s_bias[e];
-            float* gs = &s_gscore[(e >> p.gshift) * TM + row];
-            *gs = fmaxf(*gs, key);
+            for (int v = 0; v < CH / 4; ++v)
+              *reinterpret_cast<float4*>(xr + c + 4 * v) =
+                  make_float4(x[4 * v], x[4 * v + 1], x[4 * v + 2], x[4 * v + 3]);
           }
         }
-        // topk_groups rounds of (score desc, group asc), plus one round that
-        // finds the best excluded group
-        kept = 0u;
-        float last_kept = INFINITY;
-        for (int r = 0; r <= p.topk_groups; ++r) {
-          float bk = -INFINITY;
-          int bg = -1;
-          for (int g = 0; g < G; ++g) {
-            const float v = s_gscore[g * TM + row];
-            if (!((kept >> g) & 1u) && (bg < 0 || v > bk)) { bk = v; bg = g; }
-          }
-          if (r < p.topk_groups) {
-            kept |= 1u << bg;
-            last_kept = bk;
-          } else {
-            margin = last_kept - bk;
-            next_group = bk;
-          }
+        tc_fence_before();
+        epi_sync();
+        if (h1 == own1 && lane == 0)
+          mbar_arrive_remote(tempty_leader);    // TMEM read: the next tile's MMA may go
+        // one token per warp
+        for (int r = ew; r < h1 - h0; r += kEpiWarps) {
+          const int t = tok0 + h0 + r;
+          if (t < p.T)
+            route_token_warp<V>(sX + (size_t)r * XLD, s_bias, t, N, p.K, p.n_groups,
+                                p.topk_groups, wkeys, p.idx, p.gate, s_hist, p.rl, p.refine_gap,
+                                p.near, p.logits);
         }
+        epi_sync();                             // sX is rewritten next
       }
-      // ---- top-(K+1) of the eligible keys, sorted by (key desc, index asc)
-      float tk[KMAX + 1], ts[KMAX + 1];
-      int te[KMAX + 1];
-#pragma unroll
-      for (int j = 0; j <= KMAX; ++j) {
-        tk[j] = -INFINITY;
-        ts[j] = 0.f;
-        te[j] = 0x7fffffff;
-      }
-      float thr = -INFINITY;                        // the (K+1)-th key so far
-      for (int c = 0; c < N / 32; ++c) {
-        float x[32];
-        load_logits32<S>(tmem_row, c, peer_row, x);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int e = c * 32 + j;
-          const float s = affinity32(x[j]);
-          const float key = s + s_bias[e];
-          const bool elig = !GROUPED || ((kept >> (e >> p.gshift)) & 1u);
-          if (elig && key > thr) {
-            insert_top<KMAX>(key, e, s, K, tk, te, ts);
-            thr = slot_value<KMAX>(tk, K);
-          }
-        }
-      }
-      // ---- gates, outputs, load
-      float sum = 0.f;
-#pragma unroll
-      for (int j = 0; j < KMAX; ++j)
-        if (j < K) sum += ts[j];
-      if (tv) {
-#pragma unroll
-        for (int j = 0; j < KMAX; ++j) {
-          if (j < K) {
-            p.idx[(size_t)t * K + j] = te[j];
-            p.gate[(size_t)t * K + j] = ts[j] / sum;
-            atomicAdd(&s_hist[te[j]], 1);
-          }
-        }
-#pragma unroll
-        for (int j = 0; j < KMAX; ++j)
-          if (j < K) margin = fminf(margin, tk[j] - tk[j + 1]);   // tk[K] = -inf when K = N_r
-      }
-      // ---- near-tie listing: the token, every expert whose key lies within
-      // `near` of the lowest key a decision hinged on, and its logit row
-      const bool listed = tv && margin < p.refine_gap;
-      if (__any_sync(0xffffffffu, listed)) {
-        const float lim = fminf(thr, next_group) - p.near;
-        int cnt = 0;
-        int32_t* pr = p.rl.pair + (size_t)t * N;
-        float* lg = p.logits + (size_t)t * N;
-        for (int c = 0; c < N / 32; ++c) {
-          float x[32];
-          load_logits32<S>(tmem_row, c, peer_row, x);
-          if (listed) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int e = c * 32 + j;
-              lg[e] = x[j];
-              const float key = affinity32(x[j]) + s_bias[e];
-              if (key >= lim) pr[cnt++] = t * N + e;
-            }
-          }
-        }
-        if (listed) {
-          const int slot = atomicAdd(&p.rl.hdr[0], 1);
-          p.rl.tok[slot] = t;
-          p.rl.start[slot] = t * N;
-          p.rl.num[slot] = cnt;
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_remote(tempty_leader);
       tphase ^= 1;
     }
   }
@@ -440,10 +371,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int S, int KMAX, bool GROUPED>
+template <int S, int V>
 moe_status router_launch(const CUtensorMap& tmU, const CUtensorMap& tmE, const RouterParams& p,
                          int n_clusters, cudaStream_t s) {
-  auto kern = router_tc_kernel<S, KMAX, GROUPED>;
+  auto kern = router_tc_kernel<S, V>;
   static bool attr_done[kMaxSmemDevices] = {};
   const moe_status st = ensure_max_smem(reinterpret_cast<const void*>(kern), SMEM_ALLOC,
                                         attr_done, "router_tc smem attribute");
@@ -464,13 +395,13 @@ moe_status router_launch(const CUtensorMap& tmU, const CUtensorMap& tmE, const R
 }
 
 // Clusters of 2S CTAs of this kernel that fit on the device at once.
-template <int S, int KMAX, bool GROUPED>
+template <int S, int V>
 int resident_clusters() {
   static int cached[kMaxSmemDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxSmemDevices) return 0;
   if (cached[dev]) return cached[dev];
-  auto kern = router_tc_kernel<S, KMAX, GROUPED>;
+  auto kern = router_tc_kernel<S, V>;
   static bool attr_done[kMaxSmemDevices] = {};
   if (ensure_max_smem(reinterpret_cast<const void*>(kern), SMEM_ALLOC, attr_done,
                       "router_tc smem attribute") != MOE_OK)
@@ -497,30 +428,27 @@ int resident_clusters() {
   return n;
 }
 
-template <int KMAX, bool GROUPED>
+template <int V>
 moe_status router_dispatch_s(const CUtensorMap& tmU, const CUtensorMap& tmE,
                              const RouterParams& p, cudaStream_t s) {
   // the largest slice count whose clusters all run in one wave and whose
   // slices each get at least one 64-wide block of the contraction
-  if (p.nk >= 4 && resident_clusters<4, KMAX, GROUPED>() >= p.n_tiles)
-    return router_launch<4, KMAX, GROUPED>(tmU, tmE, p, p.n_tiles, s);
-  if (p.nk >= 2 && resident_clusters<2, KMAX, GROUPED>() >= p.n_tiles)
-    return router_launch<2, KMAX, GROUPED>(tmU, tmE, p, p.n_tiles, s);
-  const int pairs = resident_clusters<1, KMAX, GROUPED>();
+  if (p.nk >= 4 && resident_clusters<4, V>() >= p.n_tiles)
+    return router_launch<4, V>(tmU, tmE, p, p.n_tiles, s);
+  if (p.nk >= 2 && resident_clusters<2, V>() >= p.n_tiles)
+    return router_launch<2, V>(tmU, tmE, p, p.n_tiles, s);
+  const int pairs = resident_clusters<1, V>();
   if (pairs <= 0) return fail(MOE_ERR_CUDA, "router_tc: no resident CTA pair");
-  return router_launch<1, KMAX, GROUPED>(tmU, tmE, p, pairs < p.n_tiles ? pairs : p.n_tiles, s);
+  return router_launch<1, V>(tmU, tmE, p, pairs < p.n_tiles ? pairs : p.n_tiles, s);
 }
 
 }  // namespace
 
 bool router_tc_supported(moe_dtype dt, int d, int N_r, int K, int n_groups, int topk_groups) {
+  (void)topk_groups;
   if (dt != MOE_BF16 || d % BK != 0 || N_r % 32 != 0 || N_r < 32 || N_r > kMaxN) return false;
-  if (K < 1 || K > 16) return false;
-  if (n_groups > 1 && topk_groups < n_groups) {
-    const int gs = N_r / n_groups;
-    if (n_groups > 32 || (gs & (gs - 1)) != 0) return false;
-  }
-  return true;
+  if (K < 1 || K > N_r) return false;
+  return n_groups >= 1 && n_groups <= 32;
 }
 
 moe_status launch_router_tc(const void* u, const void* E, const float* b, int T, int d, int N_r,
@@ -540,12 +468,13 @@ moe_status launch_router_tc(const void* u, const void* E, const float* b, int T,
   p.K = K;
   p.nk = d / BK;
   p.n_tiles = (T + 2 * TM - 1) / (2 * TM);
-  const bool grouped = n_groups > 1 && topk_groups < n_groups;
-  p.n_groups = grouped ? n_groups : 1;
-  p.topk_groups = grouped ? topk_groups : 1;
-  p.gshift = 0;
-  if (grouped)
-    while ((1 << p.gshift) < N_r / n_groups) ++p.gshift;
+  // column parts per token row when reading TMEM: the most (<= 4) that
+  // split N_r into 16-column pieces
+  p.parts = 1;
+  for (int parts = kParts; parts > 1; --parts)
+    if ((N_r / CH) % parts == 0) { p.parts = parts; break; }
+  p.n_groups = n_groups;
+  p.topk_groups = topk_groups;
   p.idx = idx;
   p.gate = gate;
   p.counts = counts;
@@ -555,11 +484,11 @@ moe_status launch_router_tc(const void* u, const void* E, const float* b, int T,
   p.near = near;
   p.err = device_error_word();
   if (!p.err) return fail(MOE_ERR_CUDA, "device error word unavailable");
-  if (K <= 8)
-    return grouped ? router_dispatch_s<8, true>(tmU, tmE, p, s)
-                   : router_dispatch_s<8, false>(tmU, tmE, p, s);
-  return grouped ? router_dispatch_s<16, true>(tmU, tmE, p, s)
-                 : router_dispatch_s<16, false>(tmU, tmE, p, s);
+  const int V = N_r / 32;
+  if (V <= 1) return router_dispatch_s<1>(tmU, tmE, p, s);
+  if (V <= 2) return router_dispatch_s<2>(tmU, tmE, p, s);
+  if (V <= 4) return router_dispatch_s<4>(tmU, tmE, p, s);
+  return router_dispatch_s<8>(tmU, tmE, p, s);
 }
 
 }  // namespace moe

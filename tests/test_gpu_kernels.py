@@ -10,7 +10,7 @@ import mixture_experts_layer_60_b200 as moe
 from oracle import moe_backward as B
 from oracle import moe_oracle as O
 from tests.harness import (GATE_TOL, TOL, LazyExperts, assert_close, check_routing, f64,
-                           grouped_reference)
+                           TIE_GAP, grouped_reference)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -117,6 +117,59 @@ def test_route_v3_width_float64_tie_break():
     ref = O.route(f64(u), f64(E), b.cpu().numpy(), K)
     check_routing(idx.cpu().numpy(), gate.cpu().numpy(), counts.cpu().numpy(), ref, K,
                   gate_tol=GATE_TOL["bf16"])
+
+
+def test_route_grouped_group_choice_moved_by_tie_break():
+    """Experts 24 (group 3) and 32 (group 4) differ in one centroid entry and
+    carry the same bias, so the 4th and 5th group scores are closer than the
+    float32 logit error for many tokens: where the float32 logits order the
+    two the wrong way, the float64 tie-break moves the group choice and the
+    new group's experts near the (K+1)-th key get float64 keys too.  Every
+    token whose float64 keys are clear of other near-ties must match the
+    oracle exactly."""
+    T, d, N_r, K, G, M = 2048, 7168, 64, 8, 8, 4
+    g = _gen(4242)
+    u = _randn((T, d), g, 1.0)
+    E = _randn((N_r, d), g, d ** -0.5)
+    E[32] = E[24]
+    E[24, 5] = 0.0
+    E[32, 5] = 2.0 ** -19
+    b = torch.zeros(N_r, device=DEV)
+    b[[0, 8, 16]] = 2.0            # groups 0-2 always kept
+    b[[24, 32]] = 1.0              # groups 3 and 4 contend for the last place
+    idx = torch.empty(T, K, dtype=torch.int32, device=DEV)
+    gate = torch.empty(T, K, dtype=torch.float32, device=DEV)
+    counts = torch.empty(N_r, dtype=torch.int32, device=DEV)
+    ws = _ws(moe.moe_route_workspace_size(T, N_r))
+    ws.fill_(0xFF)                 # float32 logits of unlisted tokens stay NaN
+    moe.moe_route_grouped(u, E, b, K, G, M, idx, gate, counts, ws)
+    torch.cuda.synchronize()
+    assert moe.moe_device_status() == 0
+    ref = O.route_grouped(f64(u), f64(E), b.cpu().numpy(), K, G, M)
+    got = idx.cpu().numpy()
+    check_routing(got, gate.cpu().numpy(), counts.cpu().numpy(),
+                  grouped_reference(ref, K, G, M), K, gate_tol=GATE_TOL["bf16"])
+    # the float32 logits of the listed tokens (white-box: copied to the
+    # workspace for the tie-break) put the wrong group first for some tokens
+    x32 = ws[:T * N_r * 4].view(torch.float32).view(T, N_r).cpu().numpy()
+    listed = ~np.isnan(x32).any(1)
+    key = ref["key"]
+    f64_g4 = key[:, 32] > key[:, 24]
+    moved = listed & ((x32[:, 32] > x32[:, 24]) != f64_g4) & (key[:, 32] != key[:, 24])
+    assert moved.sum() > 0, "no token had its group choice moved"
+    # exact where the oracle's group choice is not a float32 tie and its
+    # selection inside the kept groups has no near-tie
+    gs = N_r // G
+    gsc = key.reshape(T, G, gs).max(2)
+    kept = np.zeros((T, G), bool)
+    np.put_along_axis(kept, np.argsort(-gsc, axis=1, kind="stable")[:, :M], True, axis=1)
+    masked = np.where(np.repeat(kept, gs, axis=1), key, -np.inf)
+    sel_gap, ord_gap = O.topk_margins(masked, ref["idx"])
+    strict = (key[:, 32] != key[:, 24]) & (sel_gap >= TIE_GAP) & (ord_gap >= TIE_GAP)
+    assert strict[moved].sum() > 0
+    bad = strict & np.any(got != ref["idx"], axis=1)
+    assert not bad.any(), f"{int(bad.sum())} of {int(strict.sum())} tokens differ " \
+        f"({int((bad & moved).sum())} with a moved group choice)"
 
 
 @pytest.mark.parametrize("grouped", [False, True])
@@ -719,3 +772,47 @@ def test_expert_ffn_with_shared_groups(sizes, T, N_s, d, I):
     for j in range(N_s):
         assert_close(got[rows + j * T: rows + (j + 1) * T], O.swiglu_ffn(us, *exs[j]),
                      TOL["bf16"], f"shared expert {j}")
+
+
+# B, the bound on the float32 key error behind the router's tie-break (refine
+# gap 2B, near distance 3B; include/moe.h, moe_route).
+KEY_ERROR_BOUND = 2e-5
+
+
+@pytest.mark.parametrize("config,step", [("v3_bf16", None), ("v3_zipf_bf16", 0),
+                                         ("v3_zipf_bf16", 1)])
+def test_router_float32_key_error_within_bound(config, step):
+    """With every token re-routed (refine gap 1e30, near 0) the workspace holds
+    the fused router's float32 logits for every token.  At the V3 width
+    (d 7168, 256 experts, 8192 tokens) on the V3 recipe and on the skewed
+    recipe (centroid norms up to 5, logits up to ~22) every key's float32
+    error against the float64 affinity stays below B; the routing of the
+    fully re-routed batch equals the oracle's."""
+    from mixture_experts_layer_60_b200.configs import CONFIGS
+    from mixture_experts_layer_60_b200.synth import make_layer_inputs, step_u
+    cfg = CONFIGS[config]
+    w = make_layer_inputs(cfg, DEV)
+    u = w["u"] if step is None else step_u(cfg, step, DEV)
+    E, b = w["E"], w["b"]
+    T, N_r, K = u.shape[0], E.shape[0], cfg.K
+    idx = torch.empty(T, K, dtype=torch.int32, device=DEV)
+    gate = torch.empty(T, K, dtype=torch.float32, device=DEV)
+    counts = torch.empty(N_r, dtype=torch.int32, device=DEV)
+    ws = _ws(moe.moe_route_workspace_size(T, N_r))
+    moe.moe_set_router_tie_break(1e30, 0.0)
+    try:
+        moe.moe_route(u, E, b, K, idx, gate, counts, ws)
+        torch.cuda.synchronize()
+    finally:
+        moe.moe_set_router_tie_break()
+    assert moe.moe_device_status() == 0
+    assert _listed_tokens(ws, T, N_r) == T
+    x32 = ws[:T * N_r * 4].view(torch.float32).view(T, N_r)
+    x64 = u.double() @ E.double().T
+    s32 = 1.0 / (1.0 + torch.exp(-x32))
+    s64 = 1.0 / (1.0 + torch.exp(-x64))
+    err = (s32.double() - s64).abs().max().item()
+    assert err < KEY_ERROR_BOUND, f"float32 key error {err:.3e} over the bound"
+    ref = O.route(f64(u), f64(E), b.cpu().numpy(), K)
+    check_routing(idx.cpu().numpy(), gate.cpu().numpy(), counts.cpu().numpy(), ref, K,
+                  gate_tol=GATE_TOL["bf16"])
