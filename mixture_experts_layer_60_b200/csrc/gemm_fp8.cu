@@ -139,8 +139,6 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
          ((uint32_t)__nv_cvt_float_to_fp8(d, __NV_SATFINITE, __NV_E4M3) << 24);
 }
 
-__device__ __forceinline__ float silu_fast(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
-
 template <int EPI, bool B_MN>
 __global__ void __launch_bounds__(kThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA,

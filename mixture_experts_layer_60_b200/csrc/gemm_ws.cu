@@ -528,6 +528,9 @@ moe_status ws_launch(const void* X, const void* W, int b_rows_per_group, const i
 moe_status launch_ws_gemm(const void* X, const void* W, int b_rows_per_group,
                           const int32_t* offsets, int n_groups, int rows, int N, int K,
                           bool swiglu, void* C, cudaStream_t s, const WsExtraGroups* extra) {
+  // the down projection (STORE) runs on CTA pairs where the shape allows
+  if (!swiglu && ws2_gemm_supported(N, K, n_groups, offsets != nullptr))
+    return launch_ws2_gemm(X, W, b_rows_per_group, offsets, n_groups, rows, N, K, C, s, extra);
   return launch_ws_gemm_ex(X, W, b_rows_per_group, offsets, n_groups, rows, N, K,
                            swiglu ? WS_SWIGLU : WS_STORE, false, C, N, nullptr, 0, s, extra);
 }

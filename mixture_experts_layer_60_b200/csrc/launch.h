@@ -108,6 +108,14 @@ moe_status launch_ws_gemm(const void* X, const void* W, int b_rows_per_group,
                           const int32_t* offsets, int n_groups, int rows, int N, int K,
                           bool swiglu, void* C, cudaStream_t s,
                           const WsExtraGroups* extra = nullptr);
+// The STORE epilogue on CTA pairs (256 weight rows per pair, token tiles in
+// multiples of 16, two TMEM accumulators per CTA, 128-wide K stages);
+// launch_ws_gemm takes this path for the down projection whenever
+// ws2_gemm_supported holds (N % 256 == 0, K % 128 == 0).
+bool ws2_gemm_supported(int N, int K, int n_groups, bool grouped);
+moe_status launch_ws2_gemm(const void* X, const void* W, int b_rows_per_group,
+                           const int32_t* offsets, int n_groups, int rows, int N, int K, void* C,
+                           cudaStream_t s, const WsExtraGroups* extra = nullptr);
 // Epilogues: SWIGLU  C = SiLU(gate) * up (N = I columns);
 //            SWIGLU_SAVE  the same, plus S[:, 0:I] = gate, S[:, I:2I] = up;
 //            STORE   C = the product (N columns);
