@@ -139,7 +139,12 @@ KERNEL_SOURCES = {"bf16": ["mixture_experts_layer_60_b200/csrc/gemm_ws.cu",
                            "mixture_experts_layer_60_b200/csrc/sm100.cuh"],
                   "e4m3": ["mixture_experts_layer_60_b200/csrc/gemm_fp8.cu",
                            "mixture_experts_layer_60_b200/csrc/sm100.cuh"]}
-MEASURED_GATE_UP_TRAFFIC = {}   # workload -> {"bytes": B, "sha": hex prefix}
+# v3_bf16: 2,179,612,160 B read + written by the gate/up launch of 32 experts x
+# 256 tokens + the shared expert over 1024 tokens (2,107,637,760 algorithmic
+# bytes), scaled by the algorithmic bytes of the 256-expert launch.
+MEASURED_GATE_UP_TRAFFIC = {   # workload -> {"bytes": B, "sha": hex prefix}
+    "v3_bf16": {"bytes": 17011818690, "sha": "0b70cf9029e61dd4"},
+}
 
 
 def sources_sha(dtype):

@@ -43,7 +43,6 @@ using namespace sm100;
 constexpr int WROWS = 256;          // weight rows per tile (two M=128 MMAs)
 constexpr int TMAX = 256;           // max token rows per tile (MMA N)
 constexpr int BK = 64;              // bf16 elements per 128-byte swizzle row
-constexpr int XBOX = 64;            // token rows per TMA box (fewer, larger TMA operations)
 constexpr int STAGES = 3;
 constexpr int kEpiWarps = 8;        // two warps per TMEM lane quarter, alternating token chunks
 constexpr int kThreads = 64 + 32 * kEpiWarps;
@@ -53,7 +52,6 @@ constexpr uint32_t TMEM_COLS = 512;
 
 constexpr int W_BYTES = WROWS * BK * 2;       // 32 KB
 constexpr int X_BYTES = TMAX * BK * 2;        // 32 KB
-constexpr int XBOX_BYTES = XBOX * BK * 2;     // 8 KB
 constexpr int WBOX_MN_BYTES = 64 * BK * 2;    // MN-major weights: one [64 K][64 N] box, 8 KB
 constexpr int OFF_X = STAGES * W_BYTES;
 constexpr int OFF_STAGE_OUT = OFF_X + STAGES * X_BYTES;   // one 2 KB transpose patch per epilogue warp
@@ -145,8 +143,12 @@ __device__ __forceinline__ float silu_f(float x) { return __fdividef(x, 1.0f + _
 template <int EPI, bool WMN>
 __global__ void __launch_bounds__(kThreads, 1)
     ws_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                   const __grid_constant__ CUtensorMap tmX128,
+                   const __grid_constant__ CUtensorMap tmX256,
                    const __grid_constant__ CUtensorMap tmW2,
-                   const __grid_constant__ CUtensorMap tmX2, const WsParams p) {
+                   const __grid_constant__ CUtensorMap tmX2,
+                   const __grid_constant__ CUtensorMap tmX2_128,
+                   const __grid_constant__ CUtensorMap tmX2_256, const WsParams p) {
   constexpr int OUT_COLS = TileMath<EPI>::OUT_COLS;
   constexpr bool SWIGLU = TileMath<EPI>::SW;
   extern __shared__ uint8_t smem_raw[];
@@ -179,9 +181,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tmW);
     tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmX128);
+    tma_prefetch_desc(&tmX256);
     if (p.n_extra) {
       tma_prefetch_desc(&tmW2);
       tma_prefetch_desc(&tmX2);
+      tma_prefetch_desc(&tmX2_128);
+      tma_prefetch_desc(&tmX2_256);
     }
   }
   if (warp == 1) {
@@ -243,9 +249,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         decode_tile(t, prefix, roff, G, Gtot, p, g, nt, tok0, count, xrow0);
         const bool extra = g >= G;
         const CUtensorMap* tw = extra ? &tmW2 : &tmW;
-        const CUtensorMap* tx = extra ? &tmX2 : &tmX;
-        const int nbox = (count + XBOX - 1) / XBOX;
-        const uint32_t bytes = W_BYTES + nbox * XBOX_BYTES;
+        // one token box per stage: 64, 128 or 256 rows (it may read past the
+        // tile's rows, which the MMA's N or the epilogue leaves unused)
+        const int xb = count <= 64 ? 64 : count <= 128 ? 128 : 256;
+        const CUtensorMap* tx = xb == 64 ? (extra ? &tmX2 : &tmX)
+                                : xb == 128 ? (extra ? &tmX2_128 : &tmX128)
+                                            : (extra ? &tmX2_256 : &tmX256);
+        const uint32_t bytes = W_BYTES + (uint32_t)xb * BK * 2;
         const int wrow = (extra ? g - G : g) * p.b_rows_per_group + nt * (SWIGLU ? 128 : 256);
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, kWaitNs)) {
@@ -266,9 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_2d(w_dst + W_BYTES / 2, tw, kb * BK, wrow + (SWIGLU ? p.half_b : 128),
                         &full[stage]);
           }
-          uint8_t* x_dst = sX + stage * X_BYTES;
-          for (int b = 0; b < nbox; ++b)
-            tma_load_2d(x_dst + b * XBOX_BYTES, tx, kb * BK, xrow0 + b * XBOX, &full[stage]);
+          tma_load_2d(sX + stage * X_BYTES, tx, kb * BK, xrow0, &full[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
@@ -467,7 +475,7 @@ moe_status ws_launch(const void* X, const void* W, int b_rows_per_group, const i
                      int n_groups, int rows, int N, int K, void* C, int ldc, void* S, int lds,
                      const WsExtraGroups& ex, cudaStream_t s) {
   constexpr int OUT_COLS = TileMath<EPI>::OUT_COLS;
-  CUtensorMap tmW, tmX, tmW2, tmX2;
+  CUtensorMap tmW, tmX, tmX128, tmX256, tmW2, tmX2, tmX2_128, tmX2_256;
   const int G = offsets ? n_groups : 1;
   long long x_rows = ex.n_extra && !ex.x_local ? rows + (long long)ex.n_extra * ex.T : rows;
   if (x_rows == 0) x_rows = ex.T;   // no routed rows: a map over the extra X, never read
@@ -476,17 +484,25 @@ moe_status ws_launch(const void* X, const void* W, int b_rows_per_group, const i
                       : make_tmap_2d(&tmW, W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K,
                                      (uint64_t)G * b_rows_per_group, BK, 128);
   if (st != MOE_OK) return st;
-  st = make_tmap_2d(&tmX, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, (uint64_t)x_rows, BK, XBOX);
+  auto xmaps = [&](const void* base, uint64_t n, CUtensorMap* m64, CUtensorMap* m128,
+                   CUtensorMap* m256) -> moe_status {
+    moe_status r = make_tmap_2d(m64, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, n, BK, 64);
+    if (r == MOE_OK) r = make_tmap_2d(m128, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, n, BK, 128);
+    if (r == MOE_OK) r = make_tmap_2d(m256, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, n, BK, 256);
+    return r;
+  };
+  st = xmaps(X, (uint64_t)x_rows, &tmX, &tmX128, &tmX256);
   if (st != MOE_OK) return st;
   tmW2 = tmW;
   tmX2 = tmX;
+  tmX2_128 = tmX128;
+  tmX2_256 = tmX256;
   if (ex.n_extra) {
     st = make_tmap_2d(&tmW2, ex.W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K,
                       (uint64_t)ex.n_extra * b_rows_per_group, BK, 128);
     if (st != MOE_OK) return st;
     if (ex.x_local) {
-      st = make_tmap_2d(&tmX2, ex.X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, (uint64_t)ex.T, BK,
-                        XBOX);
+      st = xmaps(ex.X, (uint64_t)ex.T, &tmX2, &tmX2_128, &tmX2_256);
       if (st != MOE_OK) return st;
     }
   }
@@ -519,7 +535,7 @@ moe_status ws_launch(const void* X, const void* W, int b_rows_per_group, const i
        (long long)ex.n_extra * ((ex.T + TMAX - 1) / TMAX)) * (N / OUT_COLS);
   int grid = sm_count();
   if (max_tiles < grid) grid = (int)(max_tiles > 0 ? max_tiles : 1);
-  kern<<<grid, kThreads, SMEM_ALLOC, s>>>(tmW, tmX, tmW2, tmX2, p);
+  kern<<<grid, kThreads, SMEM_ALLOC, s>>>(tmW, tmX, tmX128, tmX256, tmW2, tmX2, tmX2_128, tmX2_256, p);
   return cuda_check(cudaGetLastError(), "ws_gemm launch");
 }
 
