@@ -168,7 +168,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int a = 0; a < 2; ++a) { mbar_init(&pfull[a], 1); mbar_init(&pempty[a], 128 * kEpiWG); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&pfull[a], 1); mbar_init(&pempty[a], 4 * kEpiWG); }   // one arrival per epilogue warp
     mbar_init(mma_done, 1);
     mbar_init(&xbar[0], 128 * kEpiWG);
     mbar_init(&xbar[1], 128 * kEpiWG);
@@ -342,7 +342,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_ld();
           if (c == 3) {
             tc_fence_before();
-            mbar_arrive(&pempty[pb]);   // partial read: the MMA may overwrite it
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&pempty[pb]);   // partial read: the MMA may overwrite it
           }
           const uint64_t sc2 = c < 2 ? f2_pack(s0, s0) : f2_pack(s1, s1);
 #pragma unroll

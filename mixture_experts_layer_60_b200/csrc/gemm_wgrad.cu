@@ -97,7 +97,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], 32 * kEpiWarps); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], kEpiWarps); }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -226,7 +226,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld_32x32b_x32(tl + 32, r[1]);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(&tempty[ab]);      // accumulator read: the next tile's MMAs may start
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[ab]);   // accumulator read: the next tile's MMAs may start
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         // the previous TMA store must have read the patch before it is rewritten

@@ -148,9 +148,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(&pfull[b], 1); mbar_init(&pempty[b], 32 * kEpiWarps); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&pfull[b], 1); mbar_init(&pempty[b], kEpiWarps); }
     mbar_init(mma_done, 1);
-    for (int i = 0; i < SSLOTS; ++i) { mbar_init(&sfull[i], 1); mbar_init(&sempty[i], 32 * kEpiWarps); }
+    for (int i = 0; i < SSLOTS; ++i) { mbar_init(&sfull[i], 1); mbar_init(&sempty[i], kEpiWarps); }
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
@@ -293,7 +293,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_ld();
           if (c == 7) {
             tc_fence_before();
-            mbar_arrive(&pempty[pb]);   // partial read: the MMA may overwrite it
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&pempty[pb]);   // partial read: the MMA may overwrite it
           }
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
@@ -301,7 +302,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             acc2[c * 4 + v] = fma2_bits(r[2 * v], r[2 * v + 1], s2, acc2[c * 4 + v]);
           }
         }
-        mbar_arrive(&sempty[ss]);       // this block's scales are no longer read
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sempty[ss]);   // this block's scales are no longer read
         if (++pb == 2) { pb = 0; pphase ^= 1; }
         if (++ss == SSLOTS) { ss = 0; sphase ^= 1; }
       }

@@ -175,7 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     mbar_init(tfull, 1);
-    mbar_init(tempty, 32 * kEpiWarps);
+    mbar_init(tempty, kEpiWarps);      // one arrival per epilogue warp
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -449,7 +449,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(tempty);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty);
       tphase ^= 1;
     }
   }
