@@ -64,8 +64,12 @@ constexpr int OFF_BAR = OFF_B + STAGES * B_BYTES;
 constexpr int N_BARS = 2 * STAGES + 7;
 constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
 constexpr int OFF_AMAX = OFF_MISC + 16;                 // [2 slots][2][kEpiWG][BM] float
-constexpr int OFF_TAB = OFF_AMAX + 2 * 2 * kEpiWG * BM * 4;
+// STORE: [32 rows][16 cols] bf16 per warp, read and written as 16-byte vectors
+constexpr int OFF_PATCH = (OFF_AMAX + 2 * 2 * kEpiWG * BM * 4 + 127) / 128 * 128;
+static_assert(OFF_PATCH % 16 == 0, "16-byte vectors");
+constexpr int OFF_TAB = OFF_PATCH + 4 * kEpiWG * 1024;
 constexpr int SMEM_BYTES = OFF_TAB + 2 * (kMaxGroups + 1) * 4;
+static_assert(SMEM_BYTES + 1024 <= 227 * 1024, "shared memory");
 constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
 
 struct Fp8Params {
@@ -494,19 +498,36 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (wg == 0) p.c_scale[(size_t)(row0 + rit) * (p.N / 128) + nt] = sc;
         }
-      } else if (valid) {
-        __nv_bfloat16* dst =
-            static_cast<__nv_bfloat16*>(p.C) + (size_t)(row0 + rit) * p.N + nt * BN + wg * CW;
-        uint4* d4 = reinterpret_cast<uint4*>(dst);
+      } else {
+        // STORE: 16 columns at a time through a 1 KB patch per warp, so that
+        // each store instruction writes 16 rows x 32 bytes (whole sectors)
+        // instead of 32 rows x 16 bytes
+        uint4* patch = reinterpret_cast<uint4*>(smem + OFF_PATCH + (warp - 2) * 1024);   // [32][2]
+        __nv_bfloat16* cbase = static_cast<__nv_bfloat16*>(p.C) + nt * BN + wg * CW;
 #pragma unroll
-        for (int q = 0; q < CW / 8; ++q) {
-          uint32_t w[4];
+        for (int q16 = 0; q16 < CW / 16; ++q16) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            __nv_bfloat162 pr = __floats2bfloat162_rn(acc[q * 8 + 2 * i], acc[q * 8 + 2 * i + 1]);
-            w[i] = *reinterpret_cast<uint32_t*>(&pr);
+          for (int h = 0; h < 2; ++h) {
+            uint32_t w[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int j = q16 * 16 + h * 8 + 2 * i;
+              __nv_bfloat162 pr = __floats2bfloat162_rn(acc[j], acc[j + 1]);
+              w[i] = *reinterpret_cast<uint32_t*>(&pr);
+            }
+            patch[lane * 2 + h] = make_uint4(w[0], w[1], w[2], w[3]);
           }
-          d4[q] = make_uint4(w[0], w[1], w[2], w[3]);
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const int piece = i * 32 + lane;
+            const int r = piece >> 1;                    // row of this warp's 32
+            const int rr = sub * 32 + r;                 // row inside the tile
+            if (rr < mv)
+              *reinterpret_cast<uint4*>(cbase + (size_t)(row0 + rr) * p.N + q16 * 16 +
+                                        (piece & 1) * 8) = patch[piece];
+          }
+          __syncwarp();
         }
       }
     }
