@@ -159,7 +159,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* pfull = empty + STAGES;   // [2] partial ready
   uint64_t* pempty = pfull + 2;       // [2] partial consumed (256 arrivals)
   uint64_t* mma_done = pempty + 2;
-  uint64_t* xbar = mma_done + 1;      // [2] amax exchange between the warpgroups (256 arrivals)
+  uint64_t* xbar = mma_done + 1;      // [2] amax exchange between the warpgroups (one arrival per warp)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
   float* amax_x = reinterpret_cast<float*>(smem + OFF_AMAX);
@@ -174,8 +174,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     for (int a = 0; a < 2; ++a) { mbar_init(&pfull[a], 1); mbar_init(&pempty[a], 4 * kEpiWG); }   // one arrival per epilogue warp
     mbar_init(mma_done, 1);
-    mbar_init(&xbar[0], 128 * kEpiWG);
-    mbar_init(&xbar[1], 128 * kEpiWG);
+    mbar_init(&xbar[0], 4 * kEpiWG);                 // one arrival per epilogue warp
+    mbar_init(&xbar[1], 4 * kEpiWG);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
@@ -413,7 +413,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         float* slot = amax_x + sl * 2 * kEpiWG * BM;
         slot[wg * BM + rit] = ma;
         slot[(kEpiWG + wg) * BM + rit] = mb;
-        mbar_arrive(&xbar[sl]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&xbar[sl]);   // this warp's amax values are in place
         const bool xok = mbar_wait_bounded(&xbar[sl], (it >> 1) & 1, abort_flag, kWaitNs);
         if (!xok) {
           raise_abort(abort_flag, p.err);
@@ -473,7 +474,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int sl = it & 1;
         float* slot = amax_x + sl * 2 * kEpiWG * BM;
         slot[wg * BM + rit] = amax;
-        mbar_arrive(&xbar[sl]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&xbar[sl]);   // this warp's amax values are in place
         const bool xok = mbar_wait_bounded(&xbar[sl], (it >> 1) & 1, abort_flag, kWaitNs);
         if (!xok) {
           raise_abort(abort_flag, p.err);
