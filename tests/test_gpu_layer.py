@@ -87,9 +87,9 @@ def test_layer_small_bf16():
 
 
 def test_layer_v3_bf16_sampled():
-    """V3 shape (T = 8192): h' on 256 sampled tokens and every routed row of
+    """V3 shape (T = 8192): h' on 1024 sampled tokens and every routed row of
     three whole experts (the most loaded spans several 16-row token tiles)."""
-    layer, w, _, _ = _run(CONFIGS["v3_bf16"], sample=256)
+    layer, w, _, _ = _run(CONFIGS["v3_bf16"], sample=1024)
     check_whole_experts(layer, w, _three_experts(layer), TOL["bf16"])
 
 
@@ -100,9 +100,9 @@ def test_layer_v3_bf16_ragged_T():
 
 def test_layer_v3_fp8_sampled():
     """FP8 V3 shape (T = 16384, 0.1 % outliers x50) against the FP8-emulating
-    oracle: h' on 256 sampled tokens and every routed row of three whole
+    oracle: h' on 1024 sampled tokens and every routed row of three whole
     experts (the most loaded spans several 128-token tiles)."""
-    layer, w, _, _ = _run(CONFIGS["v3_fp8"], sample=256, seed_sample=2)
+    layer, w, _, _ = _run(CONFIGS["v3_fp8"], sample=1024, seed_sample=2)
     check_whole_experts(layer, w, _three_experts(layer), TOL["e4m3"], fp8=True)
 
 
@@ -114,13 +114,15 @@ def test_layer_fp8_small_full():
 
 
 def test_layer_v3_decode_sampled():
-    """Decode-shaped batch (T = 256, ~8 tokens per expert): 16-row token tiles."""
-    _run(CONFIGS["v3_decode_bf16"], sample=16, seed_sample=3)
+    """Decode-shaped batch (T = 256, ~8 tokens per expert; 16-row token
+    tiles): every token's h' against the oracle."""
+    _run(CONFIGS["v3_decode_bf16"], sample=256, seed_sample=3)
 
 
 def test_layer_v3_grouped_sampled():
-    """Node-limited routing at V3 shape: 8 groups of 32 experts, at most 4 per token."""
-    _run(CONFIGS["v3_grouped_bf16"], sample=16, seed_sample=4)
+    """Node-limited routing at V3 shape (8 groups of 32 experts, at most 4 per
+    token): routing of every token, h' on 256 sampled tokens."""
+    _run(CONFIGS["v3_grouped_bf16"], sample=256, seed_sample=4)
 
 
 def test_layer_all_tokens_one_expert():
