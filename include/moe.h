@@ -499,6 +499,9 @@ moe_status moe_ep_return(const void* y, moe_dtype dt, const void* recv_tags,
  *   8  the row-gather pipeline (combine, combine and unpermute backward)
  *  16  a grouped GEMM met group offsets outside [0, rows] or decreasing and
  *      clamped them (no row outside [0, rows) was read or written)
+ *  32  (bounds-checked build libmoe_checked.so only, compiled with
+ *      -DMOE_CHECK_BOUNDS) an internal index lay outside the buffer it
+ *      addresses; the access was skipped
  * ------------------------------------------------------------------------ */
 moe_status moe_device_status(int* flags);
 

@@ -25,7 +25,10 @@ __all__ = [
     "moe_quantize_128x1_grouped", "moe_ep_plan", "moe_ep_dispatch", "moe_ep_return",
 ]
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
+# MOE_LIBRARY (environment) selects another build of the library, e.g. the
+# bounds-checked libmoe_checked.so; default: the in-tree libmoe.so.
+LIB_PATH = os.environ.get("MOE_LIBRARY") or os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                                                         "libmoe.so")
 
 MOE_F32, MOE_BF16, MOE_E4M3 = 0, 1, 2
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",

@@ -50,9 +50,23 @@ enum : int {
   ERR_EP_BOUNDS = 4,          // expert-parallel copy: a row position past its buffer (skipped)
   ERR_GATHER_TIMEOUT = 8,     // row-gather pipeline (combine and its backward): a wait ran out
   ERR_BAD_OFFSETS = 16,       // group offsets outside [0, rows] or decreasing (clamped)
+  ERR_BOUNDS = 32,            // checked build: an index outside its buffer (access skipped)
 };
 
 // ---------------------------------------------------------------- device side
+
+// Checked build (-DMOE_CHECK_BOUNDS): internal indices are tested against the
+// buffer they address before the access; a failed test records ERR_BOUNDS in
+// the device error word and the access is skipped (no trap).  The release
+// build compiles the tests away.
+#ifdef MOE_CHECK_BOUNDS
+__device__ __forceinline__ bool in_bounds(bool ok, int* err) {
+  if (!ok) atomicOr(err, ERR_BOUNDS);
+  return ok;
+}
+#else
+__device__ __forceinline__ bool in_bounds(bool, int*) { return true; }
+#endif
 
 __device__ __forceinline__ float bf2f(__nv_bfloat16 v) { return __bfloat162float(v); }
 

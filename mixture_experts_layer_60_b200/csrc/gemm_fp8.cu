@@ -303,7 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
       int g, nt, row0, mv;
       decode_tile(t, prefix, roff, G, g, nt, row0, mv);
-      const bool valid = rit < mv;
+      const bool valid = rit < mv && in_bounds(row0 + rit < p.rows, p.err);
       const int arow = valid ? row0 + rit : row0;   // clamp scale reads for padding rows
       const float* sa_row = p.a_scale + (size_t)arow * nkb_a;
       // weight N blocks per group; block scales [nbw][K/128], or [K/128][nbw] for B_MN
@@ -525,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int piece = i * 32 + lane;
             const int r = piece >> 1;                    // row of this warp's 32
             const int rr = sub * 32 + r;                 // row inside the tile
-            if (rr < mv)
+            if (rr < mv && in_bounds(row0 + rr < p.rows, p.err))
               *reinterpret_cast<uint4*>(cbase + (size_t)(row0 + rr) * p.N + q16 * 16 +
                                         (piece & 1) * 8) = patch[piece];
           }

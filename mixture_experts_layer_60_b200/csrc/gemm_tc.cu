@@ -260,8 +260,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(sub * 32) << 16) + acc * BN;
-      const bool valid = rit < mv;
       const size_t orow = static_cast<size_t>(row0 + rit);
+      const bool valid = rit < mv && in_bounds(orow < (size_t)p.rows, p.err);
       if (EPI == TC_EPI_SWIGLU_BF16) {
         __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.C) + orow * p.N + nt * BN_OUT;
 #pragma unroll 1

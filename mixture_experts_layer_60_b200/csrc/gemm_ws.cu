@@ -376,7 +376,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 row[it] = idx >> 2;
                 c8[it] = (idx & 3) * 8;
                 const int tok = c * 32 + sub * 16 + row[it];
-                ok[it] = tok < count;
+                ok[it] = tok < count &&
+                         in_bounds(tok0 + tok < p.rows + p.n_extra * p.T_extra, p.err);
                 grow[it] = (size_t)(tok0 + (ok[it] ? tok : 0));
                 col[it] = nt * 256 + hh * 128 + q * 32 + c8[it];
                 if (ok[it]) {
@@ -440,7 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int j = it * 8 + (lane >> 2);
             const int tok = c * 32 + j;
             const uint4 v = *reinterpret_cast<const uint4*>(patch + j * 32 + (lane & 3) * 8);
-            if (tok < count) {
+            if (tok < count && in_bounds(tok0 + tok < p.rows + p.n_extra * p.T_extra, p.err)) {
               __nv_bfloat16* dst = base + (size_t)(tok0 + tok) * ld + col0 + (lane & 3) * 8;
               *reinterpret_cast<uint4*>(dst) = v;
             }

@@ -336,7 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int j = i * 8 + (lane >> 2);
           const int tok = c * 32 + j;
           const uint4 v = *reinterpret_cast<const uint4*>(patch + j * 32 + (lane & 3) * 8);
-          if (tok < count)
+          if (tok < count && in_bounds(tok0 + tok < p.rows + p.n_extra * p.T_extra, p.err))
             *reinterpret_cast<uint4*>(p.C + (size_t)(tok0 + tok) * p.ldc + col) = v;
         }
         __syncwarp();                             // the patch is rewritten next

@@ -131,15 +131,20 @@ __global__ void __launch_bounds__(256) scatter_rows_kernel(const uint4* __restri
                                                            const int32_t* __restrict__ inv_row,
                                                            int T, int nvec, int nscale, int K,
                                                            uint4* __restrict__ x_perm,
-                                                           float* __restrict__ x_scale) {
+                                                           float* __restrict__ x_scale,
+                                                           int* err) {
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;
   int rows[16];  // K <= 16 on this path; larger K takes the generic loop below
   const int Kc = K < 16 ? K : 16;
+  const long long R = (long long)T * K;   // rows of x_perm
 #pragma unroll
   for (int k = 0; k < 16; ++k)
-    if (k < Kc) rows[k] = inv_row[(size_t)t * K + k];
+    if (k < Kc) {
+      rows[k] = inv_row[(size_t)t * K + k];
+      if (rows[k] >= 0 && !in_bounds(rows[k] < R, err)) rows[k] = -1;
+    }
   const uint4* src = u + (size_t)t * nvec;
   int c = lane;
   for (; c + 96 < nvec; c += 128) {
@@ -160,13 +165,13 @@ __global__ void __launch_bounds__(256) scatter_rows_kernel(const uint4* __restri
   }
   for (int k = 16; k < K; ++k) {
     const int r = inv_row[(size_t)t * K + k];
-    if (r < 0) continue;
+    if (r < 0 || !in_bounds(r < R, err)) continue;
     for (int cc = lane; cc < nvec; cc += 32) x_perm[(size_t)r * nvec + cc] = src[cc];
   }
   if (u_scale) {
     for (int k = 0; k < K; ++k) {
       const int r = inv_row[(size_t)t * K + k];
-      if (r < 0) continue;
+      if (r < 0 || !in_bounds(r < R, err)) continue;
       for (int j = lane; j < nscale; j += 32)
         x_scale[(size_t)r * nscale + j] = u_scale[(size_t)t * nscale + j];
     }
@@ -196,7 +201,7 @@ moe_status launch_permute(const void* u, const float* u_scale, int elem_bytes, c
   const int wpb = 8;
   scatter_rows_kernel<<<(T + wpb - 1) / wpb, wpb * 32, 0, s>>>(
       static_cast<const uint4*>(u), u_scale, inv_row, T, nvec, u_scale ? d / 128 : 0, K,
-      static_cast<uint4*>(x_perm), x_scale);
+      static_cast<uint4*>(x_perm), x_scale, device_error_word());
   return cuda_check(cudaGetLastError(), "permute launches");
 }
 

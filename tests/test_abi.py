@@ -35,6 +35,16 @@ def test_header_symbols_exported(L):
         assert n in moe.SYMBOLS, f"{n} has no binding"
 
 
+def test_checked_build_exports_the_same_symbols():
+    """The bounds-checked variant (-DMOE_CHECK_BOUNDS) builds from the same
+    sources and exports every entry point of the header."""
+    path = moe_build.build(check_bounds=True)
+    assert path.endswith("libmoe_checked.so")
+    raw = ctypes.CDLL(path)
+    for n in header_functions():
+        assert hasattr(raw, n), f"{n} missing from the checked build"
+
+
 def test_binding_names_match_header():
     assert set(moe.SYMBOLS) == set(header_functions())
 
