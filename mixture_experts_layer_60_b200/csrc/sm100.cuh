@@ -330,8 +330,8 @@ __device__ __forceinline__ float4 ld_shared_cluster_v4(uint32_t cluster_addr) {
   return v;
 }
 // 2D TMA tile load into this CTA's shared memory whose completion is
-// signalled on the pair leader's mbarrier (a shared::cluster address).  No
-// multicast: every CTA loads its own tile.
+// signalled on the pair leader's mbarrier (a shared::cluster address).  Every
+// CTA loads its own tile; only the completion count is shared.
 __device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorMap* tm, int c0,
                                                  int c1, uint32_t leader_bar) {
   asm volatile(
