@@ -2,10 +2,12 @@
 // random places in the grouped buffers (the combine of the h'-equation of
 // "DeepSeek-V3 技術報告", section 方法 / 2, and its backward).  These kernels
 // move whole 16-byte-aligned rows and do a few FMAs per element, so they are
-// bound by how many bytes each SM keeps in flight: here one producer warp
-// stages every row a step needs into shared memory with bulk asynchronous
-// copies (a ring of stages, ~180 KB per SM), and four consumer warps do the
-// arithmetic from shared memory.
+// bound by how many bytes each SM keeps in flight: here two producer warps
+// stage every row a step needs into shared memory with bulk asynchronous
+// copies (a ring of stages, ~180 KB per SM; producer warp p fills the stages
+// of the jobs j with j % 2 == p, which halves the per-copy issue cost that one
+// warp alone is bound by), and four consumer warps do the arithmetic from
+// shared memory.
 //
 // A job is (token t, column chunk q of 2 KB, or 1 KB / 512 B when a stage of
 // many rows would leave fewer than eight stages).  Tokens go in groups of four, one
@@ -40,10 +42,11 @@ using namespace sm100;
 
 constexpr int kMaxChunk = 2048;              // bytes of a row per job (2048, 1024 or 512)
 constexpr int kConsumerWarps = 4;            // one token of a group each
-constexpr int kThreads = 32 * (kConsumerWarps + 1);
+constexpr int kProducers = 2;
+constexpr int kThreads = 32 * (kConsumerWarps + kProducers);
 constexpr int kSmemBudget = 200 * 1024;
 constexpr int kMaxStages = 8;
-constexpr int kMaxSlots = 64;              // two per producer lane
+constexpr int kMaxSlots = 64;              // two per lane of a producer warp
 constexpr uint64_t kWaitNs = 1000000000ull;
 
 struct GatherParams {
@@ -141,12 +144,16 @@ __global__ void __launch_bounds__(kThreads, 1) gather_pipe_kernel(const GatherPa
   const int Q = (int)((p.row_bytes + CH - 1) / CH);
   const int n_groups = (p.T + kConsumerWarps - 1) / kConsumerWarps;
 
-  if (warp == kConsumerWarps) {
-    // ---------------------------------------------------------------- producer
+  if (warp >= kConsumerWarps) {
+    // ---------------------------------------------------------------- producers
+    // Every producer walks the whole ring (stage and phase advance for every
+    // job) and arms only its own jobs, so each stage (S is even) has a
+    // single producer as well as a single consumer.
+    const int pw = warp - kConsumerWarps;
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    long long armed = 0;                // jobs whose copies were issued
+    long long armed = 0;                // ring positions passed (every producer's jobs)
     for (int g = blockIdx.x; g < n_groups && ok; g += gridDim.x) {
       // this lane's slots (lane, lane + 32) of the group's four tokens
       const uint8_t* src[kConsumerWarps][2];
@@ -164,6 +171,11 @@ __global__ void __launch_bounds__(kThreads, 1) gather_pipe_kernel(const GatherPa
         const uint32_t cb = (uint32_t)min((long long)CH, p.row_bytes - (long long)q * CH);
 #pragma unroll
         for (int w = 0; w < kConsumerWarps; ++w) {
+          if ((int)(armed % kProducers) != pw) {
+            ++armed;
+            if (++stage == S) { stage = 0; phase ^= 1; }
+            continue;
+          }
           bool got = true;
           if (lane == 0) got = mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.wait_ns);
           got = __shfl_sync(0xffffffffu, got, 0);
@@ -191,6 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1) gather_pipe_kernel(const GatherPa
     if (lane == 0) {
       const uint64_t t0 = globaltimer_ns();
       for (long long j = armed > S ? armed - S : 0; j < armed; ++j) {
+        if ((int)(j % kProducers) != pw) continue;
         uint64_t* bar = &full[(int)(j % S)];
         const uint32_t par = (uint32_t)((j / S) & 1);
         while (!mbar_try_wait(bar, par) && globaltimer_ns() - t0 <= kWaitNs) {

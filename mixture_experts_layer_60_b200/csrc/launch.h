@@ -129,8 +129,8 @@ moe_status launch_ws_gemm_ex(const void* X, const void* W, int b_rows_per_group,
                              cudaStream_t s, const WsExtraGroups* extra = nullptr);
 
 // gather.cu ------------------------------------------------------------------
-// Row-gather pipeline (bulk copies into a shared-memory ring, one producer
-// warp, four consumer warps) for the per-token combine kernels.
+// Row-gather pipeline (bulk copies into a shared-memory ring, two producer
+// warps, four consumer warps) for the per-token combine kernels.
 enum GatherMode { GATHER_COMBINE = 0, GATHER_COMBINE_BWD = 1, GATHER_UNPERM_BWD = 2 };
 // Supported when K <= 16 and the row slots of a job (COMBINE 1 + N_s + K,
 // COMBINE_BWD 2 + 2K, UNPERM_BWD 1 + N_s + 2K) are at most 64.
