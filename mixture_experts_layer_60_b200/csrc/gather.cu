@@ -2,10 +2,10 @@
 // random places in the grouped buffers (the combine of the h'-equation of
 // "DeepSeek-V3 技術報告", section 方法 / 2, and its backward).  These kernels
 // move whole 16-byte-aligned rows and do a few FMAs per element, so they are
-// bound by how many bytes each SM keeps in flight: here two producer warps
+// bound by how many bytes each SM keeps in flight: here four producer warps
 // stage every row a step needs into shared memory with bulk asynchronous
 // copies (a ring of stages, ~180 KB per SM; producer warp p fills the stages
-// of the jobs j with j % 2 == p, which halves the per-copy issue cost that one
+// of the jobs j with j % 4 == p, spreading the per-copy issue cost that one
 // warp alone is bound by), and four consumer warps do the arithmetic from
 // shared memory.
 //
@@ -42,8 +42,10 @@ using namespace sm100;
 
 constexpr int kMaxChunk = 2048;              // bytes of a row per job (2048, 1024 or 512)
 constexpr int kConsumerWarps = 4;            // one token of a group each
-constexpr int kProducers = 2;
+constexpr int kProducers = 4;               // 256 threads: at most 255 registers each
 constexpr int kThreads = 32 * (kConsumerWarps + kProducers);
+// the stage count is a multiple of kConsumerWarps, hence of kProducers
+static_assert(kConsumerWarps % kProducers == 0, "one producer per stage");
 constexpr int kSmemBudget = 200 * 1024;
 constexpr int kMaxStages = 8;
 constexpr int kMaxSlots = 64;              // two per lane of a producer warp
@@ -147,8 +149,8 @@ __global__ void __launch_bounds__(kThreads, 1) gather_pipe_kernel(const GatherPa
   if (warp >= kConsumerWarps) {
     // ---------------------------------------------------------------- producers
     // Every producer walks the whole ring (stage and phase advance for every
-    // job) and arms only its own jobs, so each stage (S is even) has a
-    // single producer as well as a single consumer.
+    // job) and arms only its own jobs, so each stage (S is a multiple of
+    // kProducers) has a single producer as well as a single consumer.
     const int pw = warp - kConsumerWarps;
     int stage = 0;
     uint32_t phase = 0;

@@ -129,7 +129,7 @@ moe_status launch_ws_gemm_ex(const void* X, const void* W, int b_rows_per_group,
                              cudaStream_t s, const WsExtraGroups* extra = nullptr);
 
 // gather.cu ------------------------------------------------------------------
-// Row-gather pipeline (bulk copies into a shared-memory ring, two producer
+// Row-gather pipeline (bulk copies into a shared-memory ring, four producer
 // warps, four consumer warps) for the per-token combine kernels.
 enum GatherMode { GATHER_COMBINE = 0, GATHER_COMBINE_BWD = 1, GATHER_UNPERM_BWD = 2 };
 // Supported when K <= 16 and the row slots of a job (COMBINE 1 + N_s + K,

@@ -80,11 +80,12 @@ def test_stage_count_multiple_of_consumer_warps_never_passes_early():
             assert run(S, 64, seed) == "ok", (S, seed)
 
 
-def test_two_producers_never_pass_early():
-    """The kernel's two producer warps (job n armed by warp n % 2)."""
-    for S in (4, 8):
-        for seed in range(300):
-            assert run(S, 64, seed, P=2) == "ok", (S, seed)
+def test_several_producers_never_pass_early():
+    """Two or four producer warps (job n armed by warp n % P); the kernel uses four."""
+    for P in (2, 4):
+        for S in (4, 8):
+            for seed in range(300):
+                assert run(S, 64, seed, P=P) == "ok", (P, S, seed)
 
 
 def test_five_stages_go_wrong():
@@ -93,6 +94,6 @@ def test_five_stages_go_wrong():
 
 def test_two_producers_need_a_stage_count_multiple_of_four():
     """S odd (a stage with two producers) or S = 6 (two consumers): schedules
-    pass early."""
-    for S in (9, 6):
-        assert any(run(S, 64, seed, P=2) == "early" for seed in range(300)), S
+    pass early; likewise four producers on 6 stages."""
+    for S, P in ((9, 2), (6, 2), (6, 4)):
+        assert any(run(S, 64, seed, P=P) == "early" for seed in range(300)), (S, P)
