@@ -307,13 +307,21 @@ def cpu_oracle_sample(cfg, w, n_tokens, seed=0, host=None):
 def cpu_cores():
     """OpenMP threads the C++ oracle runs with (its default: one per core the
     process may use, unless OMP_NUM_THREADS says otherwise)."""
-    n = os.environ.get("OMP_NUM_THREADS")
-    if n and n.isdigit():
-        return int(n)
+    from oracle import moe_ref as R
+    return R.set_threads(0)
+
+
+def cpu_model():
+    """The host CPU's model name (/proc/cpuinfo), or the platform string."""
     try:
-        return len(os.sched_getaffinity(0))
-    except Exception:
-        return os.cpu_count() or 1
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or platform.machine()
 
 
 # ---------------------------------------------------------------- arms
@@ -324,7 +332,7 @@ def run_reference(args, cfg, ws, rank):
     from mixture_experts_layer_60_b200.synth import make_layer_inputs
     torch.cuda.set_device(0)
     w = make_layer_inputs(cfg, "cuda")
-    n_tok = args.ref_tokens
+    n_tok = min(args.ref_tokens, cfg.T)
     host = {}
     for _ in range(args.warmup):
         cpu_oracle_sample(cfg, w, n_tok, seed=1, host=host)
@@ -342,7 +350,7 @@ def run_reference(args, cfg, ws, rank):
             "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "N_r": cfg.N_r, "K": cfg.K,
                        "N_s": cfg.N_s, "I": cfg.I, "tokens_per_step": n_tok},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
-                             "kind": "oracle", "sample": sample},
+                             "cpu_model": cpu_model(), "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -606,12 +614,23 @@ def run_ours(args, cfg, ws, rank, local):
     # ---- CPU oracle baseline (rank 0, N = 1 only)
     cpu = None
     if ws == 1 and not args.no_cpu_baseline:
-        n_tok = args.cpu_tokens
+        from oracle import moe_ref as R
+        n_tok = min(args.cpu_tokens, cfg.T)
         secs = cpu_oracle_sample(cfg, w, n_tok)
-        cpu = {"value": n_tok / secs, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
+        cpu = {"value": n_tok / secs, "unit": "tokens/s", "cores": cpu_cores(),
+               "cpu_model": cpu_model(), "kind": "oracle",
                "sample": f"{n_tok} tokens of the {cfg.T}-token batch, full route + whole layer "
                          f"in float64 by the C++ oracle, weights staged in host memory before "
                          f"the timer ({secs:.1f} s)"}
+        if cfg.T <= 4096:
+            # the small configurations also on one thread (the same sample)
+            n_all = R.set_threads(0)
+            R.set_threads(1)
+            try:
+                secs1 = cpu_oracle_sample(cfg, w, n_tok)
+            finally:
+                R.set_threads(n_all)
+            cpu["one_thread"] = {"value": n_tok / secs1, "unit": "tokens/s", "cores": 1}
 
     if rank != 0:
         return

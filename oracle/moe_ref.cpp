@@ -32,6 +32,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <omp.h>
+
 #include <algorithm>
 #include <vector>
 
@@ -211,6 +213,13 @@ void ffn_accumulate_fp8(const void* u, int dt, int d, int I, const std::vector<i
 extern "C" {
 
 int moe_ref_version(void) { return 1; }
+
+// OpenMP threads of the following calls (n > 0); returns the count in force.
+// Only the timing of the CPU baseline uses it: results do not depend on it.
+int ref_set_threads(int n) {
+  if (n > 0) omp_set_num_threads(n);
+  return omp_get_max_threads();
+}
 
 // Router (affinity line, g'-equation, R1-R3, R11).  u [T, d], E [N_r, d]
 // stored as dt; b [N_r] float32.  Writes idx [T, K], gate [T, K], counts

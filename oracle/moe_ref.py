@@ -12,6 +12,7 @@ raw 16-bit words).
     bias_update(b, counts, T, K, gamma=0.001) -> b'
     layer_forward(u, idx, gate, routed, shared, fp8=False) -> h' [T, d] float64
     expert_ffn(x, W_gate_up, W_down, fp8=False) -> y [n, d] float64
+    set_threads(n) -> OpenMP threads in force (timing only)
 """
 from __future__ import annotations
 
@@ -55,6 +56,8 @@ def lib():
         L.ref_layer_forward.restype = _I
         L.ref_layer_forward.argtypes = [_P, _I, _I, _I, _I, _P, _P, _I, _P, _P, _I, _P, _P, _I, _I,
                                         _P]
+        L.ref_set_threads.restype = _I
+        L.ref_set_threads.argtypes = [_I]
         L.ref_expert_ffn.restype = None
         L.ref_expert_ffn.argtypes = [_P, _I, _I, _I, _I, _P, _P, _I, _P]
         _lib = L
@@ -85,6 +88,12 @@ def _stored(a):
 
 def _ptr(a):
     return None if a is None else a.ctypes.data_as(_P)
+
+
+def set_threads(n: int) -> int:
+    """OpenMP threads of the following oracle calls (n > 0); returns the count
+    in force (n <= 0 only queries it).  Results do not depend on it."""
+    return int(lib().ref_set_threads(int(n)))
 
 
 def route(u, E, b, K, n_groups=1, topk_groups=1):

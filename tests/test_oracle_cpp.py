@@ -158,3 +158,26 @@ def test_fp8_layer_matches_numpy_oracle():
     y = R.expert_ffn(u[:9], routed[0][0], routed[0][1], fp8=True)
     np.testing.assert_allclose(y, O.fp8_swiglu_ffn(_f64(u[:9]), q(routed[0])), rtol=0,
                                atol=1e-12 * np.abs(y).max())
+
+
+def test_thread_count_leaves_results_unchanged():
+    """The oracle's OpenMP thread count (set for the benchmark's one-thread
+    baseline) changes no result: route and layer are bit-identical on one
+    thread and on all."""
+    rng = np.random.default_rng(13)
+    T, d, N_r, K, N_s, I = 50, 256, 8, 2, 1, 128
+    u = _bf16(rng.standard_normal((T, d)))
+    E = _bf16(rng.standard_normal((N_r, d)) / math.sqrt(d))
+    routed, shared = _experts(rng, N_r, d, I, _bf16), _experts(rng, N_s, d, I, _bf16)
+    n_all = R.set_threads(0)
+    try:
+        outs = []
+        for n in (1, max(n_all, 2)):
+            assert R.set_threads(n) == n
+            r = R.route(u, E, np.zeros(N_r, np.float32), K)
+            outs.append((r["idx"], r["key"], R.layer_forward(u, r["idx"], r["gate"], routed,
+                                                             shared)))
+    finally:
+        R.set_threads(n_all)
+    for a, b in zip(outs[0], outs[1]):
+        np.testing.assert_array_equal(a, b)
