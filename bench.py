@@ -608,7 +608,11 @@ def run_ours(args, cfg, ws, rank, local):
     # ---- training step (bf16 layers): forward keeping activations + backward
     train = None
     if cfg.dtype in ("bf16", "e4m3") and not args.no_train:
-        train = measure_train(args, cfg, layer, u, dev, group, p, max(3, args.steps // 4))
+        if cfg.d % 256 == 0 and cfg.I % 256 == 0:
+            train = measure_train(args, cfg, layer, u, dev, group, p, max(3, args.steps // 4))
+        else:
+            train = {"skipped": f"the backward needs d and I multiples of 256 (d={cfg.d}, "
+                                f"I={cfg.I})"}
     status = moe_device_status()
 
     # ---- CPU oracle baseline (rank 0, N = 1 only)
