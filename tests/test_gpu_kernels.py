@@ -54,6 +54,7 @@ def _route(u, E, b, K):
     (1, 128, 64, 6, torch.bfloat16),        # one token
     (20000, 256, 256, 8, torch.bfloat16),   # more 256-token tiles than CTA pairs: tile loop
     (700, 256, 96, 16, torch.bfloat16),     # N_r = 96, K = 16
+    (300, 256, 1024, 8, torch.bfloat16),    # N_r = 1024, the most the library takes
 ])
 def test_route_matches_oracle(T, d, N_r, K, dt):
     g = _gen(T * 31 + d)
@@ -243,6 +244,7 @@ def _rand_idx(T, N_r, K, seed, skew=False):
     (300, 128, 16, 4, torch.float32),
     (513, 256, 32, 2, torch.uint8),           # FP8 rows + tile scales
     (40, 128, 64, 17, torch.bfloat16),        # K > 16 path
+    (2000, 128, 1024, 8, torch.bfloat16),     # N_r = 1024, the most the library takes
 ])
 def test_permute_bit_exact(T, d, N_r, K, dtype):
     idx_np = _rand_idx(T, N_r, K, T + K, skew=True)
@@ -366,6 +368,40 @@ def test_expert_ffn_bf16(sizes, d, I):
     assert_close(got[:n], ref, TOL["bf16"], "y")
     assert np.isnan(got[n:]).all(), "rows outside every group were written"
     assert moe.moe_device_status() == 0
+
+
+def _max_group_sizes(seed):
+    """1024 ragged groups (the most a grouped launch takes): ~40 % empty, the
+    rest 1-40 rows, one of 300 rows (two 256-row token tiles)."""
+    rng = np.random.default_rng(seed)
+    sizes = np.where(rng.random(1024) < 0.4, 0, rng.integers(1, 41, 1024))
+    sizes[517] = 300
+    return sizes.tolist()
+
+
+def test_expert_ffn_bf16_max_groups():
+    got, ref, n = _ffn_case(_max_group_sizes(1), 256, 128, torch.bfloat16, 1024, extra_rows=3)
+    assert_close(got[:n], ref, TOL["bf16"], "y")
+    assert np.isnan(got[n:]).all(), "rows outside every group were written"
+    assert moe.moe_device_status() == 0
+
+
+def test_expert_ffn_fp8_max_groups():
+    got, ref = _fp8_ffn_case(_max_group_sizes(2), 256, 128, 1025)
+    assert_close(got, ref, TOL["e4m3"], "y fp8")
+
+
+def test_expert_ffn_refuses_more_than_1024_groups():
+    """1025 groups: MOE_ERR_UNSUPPORTED from the host checks, nothing launched."""
+    d, I, G = 256, 128, 1025
+    x = torch.zeros(8, d, dtype=torch.bfloat16, device=DEV)
+    wgu = torch.zeros(G, 2 * I, d, dtype=torch.bfloat16, device=DEV)
+    wdn = torch.zeros(G, d, I, dtype=torch.bfloat16, device=DEV)
+    offsets = torch.zeros(G + 1, dtype=torch.int32, device=DEV)
+    y = torch.empty(8, d, dtype=torch.bfloat16, device=DEV)
+    ws = _ws(moe.moe_expert_ffn_workspace_size(moe.MOE_BF16, 8, I))
+    with pytest.raises(moe.MoeError, match="MOE_ERR_UNSUPPORTED"):
+        moe.moe_expert_ffn(x, offsets, wgu, wdn, y, ws)
 
 
 def test_expert_ffn_clamps_bad_offsets():
