@@ -97,7 +97,7 @@ class ClockSampler:
         time.sleep(0.25)
         self.proc.terminate()
         self.proc.wait()
-        sm, mx, reasons = [], [], set()
+        sm, mx, pw, reasons = [], [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in open(self.path):
             parts = [x.strip() for x in line.split(",")]
@@ -108,13 +108,17 @@ class ClockSampler:
                 mx.append(float(parts[3].split()[0]))
             except ValueError:
                 continue
+            try:
+                pw.append(float(parts[4].split()[0]))
+            except ValueError:
+                pass
             for n, v in zip(names, parts[6:10]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
         os.unlink(self.path)
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "power_w": statistics.median(pw) if pw else None}
 
 
 # ---------------------------------------------------------------- helpers
@@ -664,6 +668,9 @@ def run_ours(args, cfg, ws, rank, local):
                            "peak_kind": "burst bf16" + (" (FP8: measured E4M3 peak)"
                                                         if cfg.dtype == "e4m3" else "")},
         "clocks": clk,
+        # tokens per joule of board energy (the median power.draw sampled
+        # during the timed region; this GPU's board only, so N = 1 alone)
+        "tokens_per_joule": (value / clk["power_w"]) if ws == 1 and clk.get("power_w") else None,
         "e2e": {"value": cfg.T * ws / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": u.numel() * u.element_size(),
                 "d2h_bytes_per_step": u.numel() * u.element_size(),
