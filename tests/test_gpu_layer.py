@@ -271,3 +271,32 @@ def test_skewed_load_full_shape_routing_and_bias():
     assert a.counts.max().item() > 4 * cfg.T * cfg.K / cfg.N_r       # the load is skewed
     w_step = dict(w, u=u)
     check_whole_experts(a, w_step, _three_experts(a), TOL["bf16"])
+
+
+def test_skewed_load_full_protocol_100_steps():
+    """The skewed-popularity configuration's whole protocol: T = 8192 fresh
+    tokens per step for 100 steps of forward + bias update.  At every step
+    each token's routing equals the oracle's with the bias the GPU carries
+    (bit for bit except genuine near-ties), the load matches, and b follows
+    the oracle's rule bit for bit; over the run the bias lowers the
+    max/mean expert load."""
+    cfg = CONFIGS["v3_zipf_bf16"]
+    w = make_layer_inputs(cfg, "cuda")
+    a = MoELayer(cfg, w)
+    E = f64(w["E"])
+    mean = cfg.T * cfg.K / cfg.N_r
+    ratios = []
+    for s in range(100):
+        u = step_u(cfg, s, "cuda")
+        b_before = a.b.cpu().numpy().copy()
+        a.step(u)
+        torch.cuda.synchronize()
+        counts = a.counts.cpu().numpy()
+        ref = O.route(f64(u), E, b_before, cfg.K)
+        check_routing(a.topk_idx.cpu().numpy(), a.topk_gate.cpu().numpy(), counts, ref, cfg.K,
+                      gate_tol=GATE_TOL["bf16"])
+        np.testing.assert_array_equal(a.b.cpu().numpy(),
+                                      O.bias_update(b_before, counts, cfg.T, cfg.K))
+        ratios.append(counts.max() / mean)
+    assert ratios[0] > 4.0, ratios[0]
+    assert np.mean(ratios[-10:]) < np.mean(ratios[:10]), (ratios[:10], ratios[-10:])
