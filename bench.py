@@ -517,6 +517,8 @@ def run_ours(args, cfg, ws, rank, local):
         return h
 
     if args.mode == "train":
+        if cfg.dtype == "e4m3":
+            p["fp8"] = measure_fp8_peak(dev)
         tr = measure_train(args, cfg, layer, u, dev, group, p, args.steps)
         if moe_device_status() != 0:
             raise RuntimeError("a kernel reported a bounded-wait timeout")
