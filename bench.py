@@ -78,7 +78,8 @@ class ClockSampler:
     """nvidia-smi samples every 200 ms while the timed region runs."""
     FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,"
+              "enforced.power.limit")
 
     def __init__(self, device_index):
         self.path = tempfile.mktemp(suffix=".csv")
@@ -97,7 +98,7 @@ class ClockSampler:
         time.sleep(0.25)
         self.proc.terminate()
         self.proc.wait()
-        sm, mx, pw, reasons = [], [], [], set()
+        sm, mx, pw, lim, reasons = [], [], [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in open(self.path):
             parts = [x.strip() for x in line.split(",")]
@@ -112,13 +113,18 @@ class ClockSampler:
                 pw.append(float(parts[4].split()[0]))
             except ValueError:
                 pass
+            try:
+                lim.append(float(parts[10].split()[0]))
+            except (ValueError, IndexError):
+                pass
             for n, v in zip(names, parts[6:10]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
         os.unlink(self.path)
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
-                "samples": len(sm), "power_w": statistics.median(pw) if pw else None}
+                "samples": len(sm), "power_w": statistics.median(pw) if pw else None,
+                "power_limit_w": max(lim) if lim else None}
 
 
 # ---------------------------------------------------------------- helpers
