@@ -676,9 +676,6 @@ def run_ours(args, cfg, ws, rank, local):
                            "peak_kind": "burst bf16" + (" (FP8: measured E4M3 peak)"
                                                         if cfg.dtype == "e4m3" else "")},
         "clocks": clk,
-        # tokens per joule of board energy (the median power.draw sampled
-        # during the timed region; this GPU's board only, so N = 1 alone)
-        "tokens_per_joule": (value / clk["power_w"]) if ws == 1 and clk.get("power_w") else None,
         "e2e": {"value": cfg.T * ws / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": u.numel() * u.element_size(),
                 "d2h_bytes_per_step": u.numel() * u.element_size(),
