@@ -106,6 +106,18 @@ def test_layer_v3_fp8_sampled():
     check_whole_experts(layer, w, _three_experts(layer), TOL["e4m3"], fp8=True)
 
 
+def test_layer_v3_fp8_ragged_T():
+    """FP8 at V3 width with T not a multiple of the 128-row tile (1000 tokens):
+    routing of every token, h' on 64 sampled tokens."""
+    _run(CONFIGS["v3_fp8"], T=1000, sample=64, seed_sample=5)
+
+
+def test_layer_v3_fp8_decode_batch():
+    """FP8 at V3 width with a decode-sized batch (256 tokens, ~8 per expert,
+    so every 128-row expert tile is mostly padding): every token's h'."""
+    _run(CONFIGS["v3_fp8"], T=256, sample=256, seed_sample=6)
+
+
 def test_layer_fp8_small_full():
     """FP8 layer on a small shape, every token compared."""
     from dataclasses import replace
