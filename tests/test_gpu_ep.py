@@ -47,3 +47,38 @@ def test_ep_emulated_equals_single_device(W, dtype, N_r, T):
                                      ref, cfg.K, gate_tol=GATE_TOL[dtype])
         want = O.layer_forward(f64(u), idx, gate, routed, shared)
         assert_close(f64(hs[s]), want, TOL[dtype], f"rank {s} h' against the oracle")
+
+
+def test_ep_emulated_v3_width_eight_ranks():
+    """Eight emulated ranks at the V3 shape (d 7168, 256 routed experts, 32 per
+    rank, K 8, I 2048), 512 tokens per rank (one rank 495): every rank's h'
+    equals the single-device layer bit for bit, every row arrives once, and
+    32 sampled tokens per rank match the oracle."""
+    import numpy as np
+    from mixture_experts_layer_60_b200.configs import CONFIGS
+    from tests.harness import oracle_layer_rows
+    W, T = 8, 512
+    cfg = CONFIGS["v3_bf16"].with_T(T)
+    w = make_layer_inputs(cfg, "cuda")
+    us = [step_u(cfg, s, "cuda") for s in range(W)]
+    us[1] = us[1][: T - 17].contiguous()
+    grp = EPGroupEmulated(cfg, w, W, T_max=T)
+    hs = grp.forward(us)
+    torch.cuda.synchronize()
+    assert moe_device_status() == 0
+    total = sum(int(r.recv_offsets[-1]) for r in grp.ranks)
+    assert total == sum(u.shape[0] for u in us) * cfg.K
+    single = MoELayer(cfg, w, T_max=T)
+    E = f64(w["E"])
+    for s, u in enumerate(us):
+        ref = single.forward(u)
+        torch.cuda.synchronize()
+        assert torch.equal(hs[s], ref), f"rank {s}"
+        rk, T_s = grp.ranks[s], u.shape[0]
+        r = O.route(f64(u), E, w["b"].cpu().numpy(), cfg.K)
+        _, idx, gate = check_routing(rk.topk_idx[:T_s].cpu().numpy(),
+                                     rk.topk_gate[:T_s].cpu().numpy(), rk.counts.cpu().numpy(),
+                                     r, cfg.K, gate_tol=GATE_TOL["bf16"])
+        rows = np.sort(np.random.default_rng(s).choice(T_s, 32, replace=False))
+        want = oracle_layer_rows(dict(w, u=u), rows, idx[rows], gate[rows])
+        assert_close(f64(hs[s])[rows], want, TOL["bf16"], f"rank {s} h' against the oracle")
