@@ -497,6 +497,89 @@ def run_hbm_kernels(args, cfg, local):
                       "gbs": {n: nbytes[n] / (ms[n] / 1e3) / 1e9 for n in names}}), flush=True)
 
 
+def run_ep_emulated(args, cfg, local):
+    """Expert parallelism with W ranks emulated on one GPU (each rank keeps
+    N_r/W experts and T/W of the tokens): per-phase times of the step and the
+    rate of the dispatch and return copy kernels.  On one GPU the rows move
+    through this GPU's HBM, not NVLink, so the copy rates are those of the
+    kernels, not of the links.  Prints one JSON line."""
+    from mixture_experts_layer_60_b200 import moe_device_status
+    from mixture_experts_layer_60_b200.parallel_ep import EPGroupEmulated
+    from mixture_experts_layer_60_b200.synth import make_layer_inputs, step_u
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    W = args.ep_ranks
+    T_r = cfg.T // W
+    sub = cfg.with_T(T_r)
+    w = make_layer_inputs(sub, dev)
+    us = [step_u(sub, s, dev) for s in range(W)]
+    grp = EPGroupEmulated(sub, w, W, T_max=T_r, device=dev)
+    R = grp.ranks
+    stream = torch.cuda.current_stream(dev)
+
+    def phases(ev):
+        def mark(name, i):
+            if ev is not None:
+                ev[name][i].record(stream)
+        mark("route_permute", 0)
+        for r, u in zip(R, us):
+            r.route_permute(u)
+        mark("route_permute", 1)
+        counts_all = torch.stack([r.counts for r in R])
+        mark("plan", 0)
+        for r in R:
+            r.plan(counts_all)
+        mark("plan", 1)
+        mark("dispatch", 0)
+        for r in R:
+            r.dispatch([x.recv_rows for x in R], [x.recv_tags for x in R])
+        mark("dispatch", 1)
+        mark("experts", 0)
+        for r in R:
+            r.experts()
+        mark("experts", 1)
+        mark("return", 0)
+        for r in R:
+            r.give_back([x.ret_rows for x in R])
+        mark("return", 1)
+        mark("combine", 0)
+        for r in R:
+            r.combine()
+        mark("combine", 1)
+
+    names = ("route_permute", "plan", "dispatch", "experts", "return", "combine")
+    for _ in range(args.warmup):
+        phases(None)
+    torch.cuda.synchronize()
+    evs = [{n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for n in names} for _ in range(args.steps)]
+    for i in range(args.steps):
+        phases(evs[i])
+    torch.cuda.synchronize()
+    if moe_device_status() != 0:
+        raise RuntimeError("a kernel reported a bounded-wait timeout")
+    ms = {n: sum(e[n][0].elapsed_time(e[n][1]) for e in evs) / args.steps for n in names}
+    row_bytes = sub.d * 2
+    moved = cfg.T * cfg.K * row_bytes           # every (token, slot) row once
+    print(json.dumps({"mode": "ep_emulated", "ranks": W,
+                      "config": {"workload": cfg.name, "T": cfg.T, "tokens_per_rank": T_r,
+                                 "d": cfg.d, "N_r": cfg.N_r, "experts_per_rank": cfg.N_r // W,
+                                 "K": cfg.K, "N_s": cfg.N_s, "I": cfg.I},
+                      "ms": ms, "ms_per_step": sum(ms.values()),
+                      "tokens_per_s": cfg.T / (sum(ms.values()) / 1e3),
+                      "copy_bytes": moved,
+                      # row bytes moved per second; the HBM traffic of a copy on one GPU
+                      # is twice that (read + write)
+                      "dispatch_gbs": moved / (ms["dispatch"] / 1e3) / 1e9,
+                      "return_gbs": moved / (ms["return"] / 1e3) / 1e9,
+                      "dispatch_hbm_frac": 2 * moved / (ms["dispatch"] / 1e3) / 1e9 /
+                                           peaks()["hbm_gbs"],
+                      "return_hbm_frac": 2 * moved / (ms["return"] / 1e3) / 1e9 /
+                                         peaks()["hbm_gbs"],
+                      "note": "ranks emulated on one GPU: dispatch and return copy through "
+                              "this GPU's HBM (read + write), not over NVLink"}), flush=True)
+
+
 def run_ours(args, cfg, ws, rank, local):
     from mixture_experts_layer_60_b200 import moe_device_status
     from mixture_experts_layer_60_b200.layer import MoELayer
@@ -702,9 +785,13 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-train", action="store_true",
                     help="skip the training-step (forward + backward) measurement")
-    ap.add_argument("--mode", default="forward", choices=["forward", "train", "hbm_kernels"],
+    ap.add_argument("--mode", default="forward",
+                    choices=["forward", "train", "hbm_kernels", "ep_emulated"],
                     help="train: time only training steps and print their line; hbm_kernels: "
-                         "route, permute and combine alone (no expert weights), for profiling")
+                         "route, permute and combine alone (no expert weights), for profiling; "
+                         "ep_emulated: expert-parallel phases with --ep-ranks ranks on one GPU")
+    ap.add_argument("--ep-ranks", type=int, default=8,
+                    help="ep_emulated: ranks emulated on the GPU (each keeps N_r/ranks experts)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="scaled-down variant: tokens per rank (default: the config's T)")
     ap.add_argument("--experts", type=int, default=None,
@@ -724,6 +811,8 @@ def main():
             run_reference(args, cfg, ws, rank)
         elif args.mode == "hbm_kernels":
             run_hbm_kernels(args, cfg, local)
+        elif args.mode == "ep_emulated":
+            run_ep_emulated(args, cfg, local)
         else:
             run_ours(args, cfg, ws, rank, local)
     finally:

@@ -147,6 +147,18 @@ moe_status moe_permute(const void* u, const float* u_scale, moe_dtype dt,
                        void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * moe_permute_index - the grouping of moe_permute without the row copies:
+ * offsets, perm_src and inv_row exactly as moe_permute writes them, for
+ * callers that move the token rows themselves (the expert-parallel dispatch,
+ * moe_ep_dispatch, reads them from u through inv_row).  Same requirements on
+ * topk_idx, T, N_r, K and the workspace (>= moe_permute_workspace_size(T,
+ * N_r) bytes).
+ * ------------------------------------------------------------------------ */
+moe_status moe_permute_index(const int32_t* topk_idx, int T, int N_r, int K, int32_t* offsets,
+                             int32_t* perm_src, int32_t* inv_row, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * moe_expert_ffn - grouped SwiGLU expert FFN: for every group g and every row
  * r in [offsets[g], offsets[g+1]):
  *     y[r] = W_down[g] (SiLU(W_gate[g] x[r]) * (W_up[g] x[r]))

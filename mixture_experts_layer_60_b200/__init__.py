@@ -23,6 +23,7 @@ __all__ = [
     "moe_expert_gate_up_save", "moe_combine_backward", "moe_expert_ffn_backward",
     "moe_expert_ffn_backward_workspace_size", "moe_unpermute_backward", "moe_router_weight_grad",
     "moe_quantize_128x1_grouped", "moe_ep_plan", "moe_ep_dispatch", "moe_ep_return",
+    "moe_permute_index",
 ]
 
 # MOE_LIBRARY (environment) selects another build of the library, e.g. the
@@ -62,6 +63,7 @@ SYMBOLS = {
     "moe_expert_gate_up_shared": (_i, [_vp, _vp, _i, _i, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
     "moe_expert_down_shared": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
     "moe_permute_noalloc": (_i, [_vp, _vp, _i, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "moe_permute_index": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_expert_gate_up_save": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp,
                                      _vp]),
     "moe_combine_backward": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp,
@@ -211,6 +213,13 @@ def moe_permute_noalloc(u, topk_idx, N_r, x_perm, offsets, perm_src, inv_row, u_
     _check(lib().moe_permute_noalloc(_p(u), _p(u_scale), _dt(u), _p(topk_idx), T, d, N_r, K,
                                      _p(x_perm), _p(x_scale), _p(offsets), _p(perm_src),
                                      _p(inv_row), _s(stream)))
+
+
+def moe_permute_index(topk_idx, N_r, offsets, perm_src, inv_row, workspace, stream=None):
+    """The grouping of moe_permute (offsets, perm_src, inv_row) without the row copies."""
+    T, K = topk_idx.shape
+    _check(lib().moe_permute_index(_p(topk_idx), T, N_r, K, _p(offsets), _p(perm_src),
+                                   _p(inv_row), _p(workspace), _nbytes(workspace), _s(stream)))
 
 
 def moe_expert_ffn(x, offsets, W_gate_up, W_down, y, workspace, x_scale=None,

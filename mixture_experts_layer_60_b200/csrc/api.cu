@@ -253,6 +253,30 @@ moe_status moe_permute(const void* u, const float* u_scale, moe_dtype dt, const 
                         s);
 }
 
+moe_status moe_permute_index(const int32_t* topk_idx, int T, int N_r, int K, int32_t* offsets,
+                             int32_t* perm_src, int32_t* inv_row, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  clear_last_error();
+  const char* who = "moe_permute_index";
+  MOE_REQUIRE(T >= 0 && N_r > 0 && K > 0, MOE_ERR_INVALID_ARG, "%s: bad sizes T=%d N_r=%d K=%d",
+              who, T, N_r, K);
+  MOE_REQUIRE(N_r <= 1024 && K <= N_r, MOE_ERR_UNSUPPORTED, "%s: need 1 <= K <= N_r <= 1024",
+              who);
+  MOE_REQUIRE(offsets, MOE_ERR_INVALID_ARG, "%s: null offsets", who);
+  MOE_REQUIRE(T == 0 || (topk_idx && perm_src && inv_row && workspace), MOE_ERR_INVALID_ARG,
+              "%s: null pointer", who);
+  MOE_REQUIRE(workspace_bytes >= moe_permute_workspace_size(T, N_r), MOE_ERR_WORKSPACE,
+              "%s: workspace %zu < %zu bytes", who, workspace_bytes,
+              moe_permute_workspace_size(T, N_r));
+  MOE_TRY(check_device());
+  cudaStream_t s = as_stream(stream);
+  if (T == 0)
+    return cuda_check(cudaMemsetAsync(offsets, 0, (size_t)(N_r + 1) * sizeof(int32_t), s),
+                      "zero offsets");
+  return launch_permute(nullptr, nullptr, 0, topk_idx, T, 0, N_r, K, nullptr, nullptr, offsets,
+                        perm_src, inv_row, workspace, s);
+}
+
 size_t moe_expert_ffn_workspace_size(moe_dtype dt, int rows, int I) { return ffn_ws(dt, rows, I); }
 
 namespace {

@@ -69,6 +69,7 @@ moe_status validate_permute_args(const char* who, const void* u, const float* u_
                                  int K, const void* x_perm, const float* x_scale,
                                  const int32_t* offsets, const int32_t* perm_src,
                                  const int32_t* inv_row, int* elem_bytes);
+// x_perm == nullptr: the grouping only (offsets, perm_src, inv_row), no rows copied.
 moe_status launch_permute(const void* u, const float* u_scale, int elem_bytes, const int32_t* idx,
                           int T, int d, int N_r, int K, void* x_perm, float* x_scale,
                           int32_t* offsets, int32_t* perm_src, int32_t* inv_row,

@@ -197,6 +197,7 @@ moe_status launch_permute(const void* u, const float* u_scale, int elem_bytes, c
     if (e != cudaSuccess) return cuda_check(e, "chunk_rank_kernel smem attribute");
   }
   chunk_rank_kernel<<<nch, kChunk, rank_smem, s>>>(idx, T, N_r, K, chunk_base, perm_src, inv_row);
+  if (!x_perm) return cuda_check(cudaGetLastError(), "permute index launches");
   const int nvec = (int)((size_t)d * elem_bytes / 16);
   const int wpb = 8;
   scatter_rows_kernel<<<(T + wpb - 1) / wpb, wpb * 32, 0, s>>>(

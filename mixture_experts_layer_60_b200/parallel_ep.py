@@ -4,7 +4,7 @@ Each rank keeps E_loc = N_r / W of the routed experts (expert e on rank
 e // E_loc), a copy of the router and of every shared expert, and routes its
 own tokens.  One step on rank s:
 
-    moe_route -> moe_permute (offsets, inv_row) -> all-gather of the loads
+    moe_route -> moe_permute_index (offsets, inv_row) -> all-gather of the loads
     -> moe_ep_plan -> moe_ep_dispatch (rows straight into each expert's rank)
     -> [all rows arrived] -> moe_expert_ffn on the received rows (E_loc groups)
     -> moe_ep_return (outputs straight back to their source rank and grouped
@@ -25,8 +25,8 @@ from __future__ import annotations
 import torch
 
 from . import (moe_combine, moe_ep_dispatch, moe_ep_plan, moe_ep_return, moe_expert_ffn,
-               moe_expert_ffn_workspace_size, moe_permute, moe_permute_workspace_size, moe_route,
-               moe_route_workspace_size, MOE_BF16, MOE_F32)
+               moe_expert_ffn_workspace_size, moe_permute_index, moe_permute_workspace_size,
+               moe_route, moe_route_workspace_size, MOE_BF16, MOE_F32)
 from .configs import LayerConfig
 
 
@@ -70,7 +70,6 @@ class _EPRank:
         self.counts = torch.zeros(c.N_r, dtype=torch.int32, device=dev)
         self.route_ws = _ws(moe_route_workspace_size(T_max, c.N_r), dev)
         self.perm_ws = _ws(moe_permute_workspace_size(T_max, c.N_r), dev)
-        self.x_perm = torch.empty(R, c.d, dtype=act, device=dev)
         self.offsets = torch.zeros(c.N_r + 1, dtype=torch.int32, device=dev)
         self.perm_src = torch.empty(R, dtype=torch.int32, device=dev)
         self.inv_row = torch.empty(T_max, c.K, dtype=torch.int32, device=dev)
@@ -99,8 +98,9 @@ class _EPRank:
         self.u = u
         moe_route(u, self.E, self.b, c.K, self.topk_idx[:T], self.topk_gate[:T], self.counts,
                   self.route_ws, stream)
-        moe_permute(u, self.topk_idx[:T], c.N_r, self.x_perm[:T * c.K], self.offsets,
-                    self.perm_src[:T * c.K], self.inv_row[:T], self.perm_ws, stream=stream)
+        # the grouping only: moe_ep_dispatch copies the rows from u itself
+        moe_permute_index(self.topk_idx[:T], c.N_r, self.offsets, self.perm_src[:T * c.K],
+                          self.inv_row[:T], self.perm_ws, stream=stream)
 
     def plan(self, counts_all, stream=None):
         if stream is not None:

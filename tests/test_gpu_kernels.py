@@ -275,6 +275,24 @@ def test_permute_bit_exact(T, d, N_r, K, dtype):
         assert torch.equal(x_scale, u_scale[src])
 
 
+@pytest.mark.parametrize("T,N_r,K", [(1000, 64, 6), (40, 64, 17), (1, 8, 3)])
+def test_permute_index_bit_exact(T, N_r, K):
+    """moe_permute_index writes the grouping of moe_permute (offsets,
+    perm_src, inv_row) equal to the oracle's, and copies no rows."""
+    idx_np = _rand_idx(T, N_r, K, T + 2 * K, skew=True)
+    idx = torch.from_numpy(idx_np).to(DEV)
+    offsets = torch.empty(N_r + 1, dtype=torch.int32, device=DEV)
+    perm_src = torch.empty(T * K, dtype=torch.int32, device=DEV)
+    inv_row = torch.empty(T, K, dtype=torch.int32, device=DEV)
+    moe.moe_permute_index(idx, N_r, offsets, perm_src, inv_row,
+                          _ws(moe.moe_permute_workspace_size(T, N_r)))
+    torch.cuda.synchronize()
+    r_off, r_src, r_inv = O.permute_indices(idx_np, N_r)
+    np.testing.assert_array_equal(offsets.cpu().numpy(), r_off)
+    np.testing.assert_array_equal(perm_src.cpu().numpy(), r_src)
+    np.testing.assert_array_equal(inv_row.cpu().numpy(), r_inv)
+
+
 def test_permute_skips_ids_out_of_range():
     """Pairs whose expert id is outside [0, N_r) are left out: inv_row = -1, no
     row copied, and the other pairs keep their stable grouped order."""
