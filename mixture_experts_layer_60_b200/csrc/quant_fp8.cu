@@ -19,33 +19,63 @@ __device__ __forceinline__ uint8_t to_e4m3(float v) {
   return static_cast<uint8_t>(__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3));
 }
 
-// One warp per (row, 128-column tile); lane j holds columns 4j..4j+3.
+// One half-warp per (row, 128-column tile): lane l of the half holds columns
+// 8l..8l+7 (one 16-byte load); each half-warp quantises kQU tiles, their
+// loads issued together so that enough bytes are in flight per SM.
+constexpr int kQU = 4;
+
 __global__ void __launch_bounds__(256) quant_1x128_kernel(const __nv_bfloat16* __restrict__ x,
                                                           int rows, int cols,
                                                           uint8_t* __restrict__ q,
                                                           float* __restrict__ scale) {
-  const int lane = threadIdx.x & 31;
+  const int l16 = threadIdx.x & 15;
   const int tiles_per_row = cols / 128;
-  const long long tile = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (tile >= (long long)rows * tiles_per_row) return;
-  const long long r = tile / tiles_per_row;
-  const int tb = (int)(tile % tiles_per_row);
-  const size_t base = (size_t)r * cols + tb * 128 + lane * 4;
-  const uint2 raw = *reinterpret_cast<const uint2*>(x + base);
-  float v[4];
-  v[0] = __uint_as_float(raw.x << 16);
-  v[1] = __uint_as_float(raw.x & 0xffff0000u);
-  v[2] = __uint_as_float(raw.y << 16);
-  v[3] = __uint_as_float(raw.y & 0xffff0000u);
-  float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+  const long long n_tiles = (long long)rows * tiles_per_row;
+  const long long n_half = (long long)gridDim.x * (blockDim.x >> 4);
+  const long long h = (long long)blockIdx.x * (blockDim.x >> 4) + (threadIdx.x >> 4);
+  uint4 raw[kQU];
+  size_t base[kQU];
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-  const float sc = tile_scale(amax);
-  uint32_t packed = 0;
+  for (int k = 0; k < kQU; ++k) {
+    const long long t = h + k * n_half;
+    base[k] = 0;
+    raw[k] = make_uint4(0u, 0u, 0u, 0u);
+    if (t < n_tiles) {
+      const long long r = t / tiles_per_row;
+      const int tb = (int)(t - r * tiles_per_row);
+      base[k] = (size_t)r * cols + (size_t)tb * 128 + l16 * 8;
+      raw[k] = *reinterpret_cast<const uint4*>(x + base[k]);
+    }
+  }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) packed |= (uint32_t)to_e4m3(__fdiv_rn(v[i], sc)) << (8 * i);
-  *reinterpret_cast<uint32_t*>(q + base) = packed;
-  if (lane == 0) scale[(size_t)r * tiles_per_row + tb] = sc;
+  for (int k = 0; k < kQU; ++k) {
+    const long long t = h + k * n_half;
+    const uint32_t w[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = __uint_as_float(w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    // the tile's 16 lanes (every lane shuffles: the offsets stay inside a half)
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1)
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    if (t < n_tiles) {
+      const float sc = tile_scale(amax);
+      uint32_t lo = 0, hi = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        lo |= (uint32_t)to_e4m3(__fdiv_rn(v[i], sc)) << (8 * i);
+        hi |= (uint32_t)to_e4m3(__fdiv_rn(v[4 + i], sc)) << (8 * i);
+      }
+      *reinterpret_cast<uint2*>(q + base[k]) = make_uint2(lo, hi);
+      if (l16 == 0) scale[(size_t)t] = sc;
+    }
+  }
 }
 
 // One 256-thread block per 128x128 block of one group.
@@ -100,10 +130,11 @@ __global__ void __launch_bounds__(256) quant_128x128_kernel(const __nv_bfloat16*
 moe_status launch_quant_1x128(const void* x, int rows, int cols, uint8_t* q, float* scale,
                               cudaStream_t s) {
   const long long tiles = (long long)rows * (cols / 128);
-  const int wpb = 8;
-  const long long blocks = (tiles + wpb - 1) / wpb;
+  const int per_block = (256 / 16) * kQU;        // 16 half-warps, kQU tiles each
+  const long long blocks = (tiles + per_block - 1) / per_block;
   if (blocks > 0x7fffffffLL) return fail(MOE_ERR_UNSUPPORTED, "quantize_1x128: too many tiles");
-  quant_1x128_kernel<<<(unsigned)blocks, wpb * 32, 0, s>>>(
+  if (blocks == 0) return MOE_OK;
+  quant_1x128_kernel<<<(unsigned)blocks, 256, 0, s>>>(
       static_cast<const __nv_bfloat16*>(x), rows, cols, q, scale);
   return cuda_check(cudaGetLastError(), "quant_1x128 launch");
 }

@@ -686,6 +686,33 @@ def test_quantize_1x128_bit_exact():
     np.testing.assert_array_equal(_e4m3_values(q), rq)
 
 
+def test_quantize_1x128_every_bf16_value_bit_exact():
+    """Every finite bf16 value x with |x| below the tile's amax, in tiles of 127
+    such values plus one amax (several amax values, so the quotients x/scale
+    land everywhere on the E4M3 grid, its rounding midpoints included): codes
+    and scales equal the oracle's IEEE-division quantisation bit for bit."""
+    bits = torch.arange(0, 1 << 16, dtype=torch.int32).to(torch.int16)
+    allv = bits.view(torch.bfloat16).float()
+    finite = allv[torch.isfinite(allv)]
+    rows = []
+    for amax in (1.0, 0.7, 3.140625, 0.0009765625, 250.0):
+        v = finite[finite.abs() < amax]
+        v = v[torch.randperm(v.numel(), generator=torch.Generator().manual_seed(7))]
+        pad = (-v.numel()) % 127
+        v = torch.cat([v, torch.zeros(pad)]).view(-1, 127)
+        rows.append(torch.cat([v, torch.full((v.shape[0], 1), amax)], dim=1))
+    x = torch.cat(rows).to(torch.bfloat16)                     # [tiles, 128]
+    n = x.shape[0] // 7 * 7
+    x = x[:n].reshape(n // 7, 7 * 128).contiguous().to(DEV)    # 7 tiles per row
+    q = torch.empty(x.shape, dtype=torch.uint8, device=DEV)
+    s = torch.empty(x.shape[0], 7, device=DEV)
+    moe.moe_quantize_1x128(x, q, s)
+    torch.cuda.synchronize()
+    rq, rs = O.quant_1x128(f64(x).astype(np.float32))
+    np.testing.assert_array_equal(s.cpu().numpy(), rs)
+    np.testing.assert_array_equal(_e4m3_values(q), rq)
+
+
 def test_quantize_128x128_bit_exact():
     g = _gen(6)
     w = _randn((3, 256, 384), g, 0.02)
