@@ -99,6 +99,19 @@ def test_permute_argument_errors(L):
     assert L.moe_permute(d, None, 1, d, 8, 4, 16, 4, d, None, d, d, d, d, 1 << 20, None) == 2
 
 
+def test_permute_index_argument_errors(L):
+    d = ctypes.c_void_p(256)
+    # moe_permute_index(topk_idx, T, N_r, K, offsets, perm_src, inv_row, ws, bytes, stream)
+    assert L.moe_permute_index(d, -1, 16, 4, d, d, d, d, 1 << 20, None) == 1     # T < 0
+    assert L.moe_permute_index(d, 8, 16, 0, d, d, d, d, 1 << 20, None) == 1      # K = 0
+    assert L.moe_permute_index(d, 8, 2048, 4, d, d, d, d, 1 << 20, None) == 2    # N_r > 1024
+    assert L.moe_permute_index(d, 8, 16, 17, d, d, d, d, 1 << 20, None) == 2     # K > N_r
+    assert L.moe_permute_index(d, 8, 16, 4, None, d, d, d, 1 << 20, None) == 1   # no offsets
+    assert L.moe_permute_index(d, 8, 16, 4, d, None, d, d, 1 << 20, None) == 1   # no perm_src
+    assert L.moe_permute_index(d, 8, 16, 4, d, d, d, d, 8, None) == 3            # workspace
+    assert b"moe_permute_index" in L.moe_last_error()
+
+
 def test_expert_ffn_argument_errors(L):
     d = ctypes.c_void_p(256)
     assert L.moe_expert_ffn(d, None, d, 4, 100, 192, 128, 1, d, None, d, None, d, d, 1 << 30,
